@@ -1,0 +1,185 @@
+"""Top-k selection and the three search pipelines (fp64 oracle).
+
+Order ("Latent Sparse Attention", section "What the kernels do about the
+top-p": a packed key with the score bits above the inverted id, so a higher
+score wins and, among equal scores, the lower id):
+
+    score descending, then position ascending.
+
+Readings where the pages are silent: -0.0 and +0.0 are equal scores; NaN ranks
+below every number including -inf; the selected list is returned in that
+canonical order (the pages leave it unsorted); a row with fewer than k
+eligible positions is padded with position -1 and value -inf.
+
+Pipelines:
+
+* decode / prefill selection: exact scores of every eligible position, then
+  top-k (k = 512; LeanSparse podcast transcript, 01:33-02:06).
+* two-stage decode search (LeanSparse podcast transcript, 07:12-08:00): scores
+  from compact keys, keep a shortlist, score the shortlist's original keys
+  exactly, keep the top k of those.
+* bucket search ("Latent Sparse Attention", "How LSA finds the keys" and "The
+  method, term by term", steps 5-6): score every bucket centroid with the
+  indexer score, keep the top-p buckets, read them best first appending their
+  members until the budget is held (the last bucket cut short), score those
+  keys exactly and keep the top k.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .formats import bf16_to_f64, dequant
+from .indexer import eligible_count, indexer_scores
+
+
+def select_topk(values: np.ndarray, positions: np.ndarray, k: int):
+    """Top-k of one candidate list by (value desc, position asc).
+
+    Returns (positions [k] int64, values [k]) padded with (-1, -inf)."""
+    values = np.asarray(values)
+    positions = np.asarray(positions, dtype=np.int64)
+    nan = np.isnan(values)
+    v = np.where(nan, 0.0, values).astype(np.float64)
+    # np.lexsort: the last key is the primary one.
+    order = np.lexsort((positions, -v, nan))
+    take = order[:k]
+    pos = np.full(k, -1, dtype=np.int64)
+    val = np.full(k, -np.inf, dtype=values.dtype if values.dtype.kind == "f" else np.float64)
+    pos[: take.size] = positions[take]
+    val[: take.size] = values[take]
+    return pos, val
+
+
+def topk_rows(scores: np.ndarray, n_valid, k: int):
+    """Row-wise top-k over the prefix [0, n_valid[r]) of each row.
+
+    Works in the dtype of ``scores`` (fp32 arrays are compared as fp32)."""
+    scores = np.atleast_2d(scores)
+    R, N = scores.shape
+    if n_valid is None:
+        n_valid = np.full(R, N)
+    idx = np.empty((R, k), dtype=np.int64)
+    val = np.empty((R, k), dtype=scores.dtype)
+    for r in range(R):
+        n = int(min(max(int(n_valid[r]), 0), N))
+        idx[r], val[r] = select_topk(scores[r, :n], np.arange(n), k)
+    return idx, val
+
+
+# --------------------------------------------------------------------------- #
+# pipelines
+# --------------------------------------------------------------------------- #
+def decode_select(q_bits, w, k_bits, n_valid, k: int = 512, return_scores: bool = False):
+    """One query per sequence over bf16 keys: exact scores then top-k."""
+    B = q_bits.shape[0]
+    idx = np.empty((B, k), dtype=np.int64)
+    val = np.empty((B, k), dtype=np.float64)
+    all_scores = []
+    for b in range(B):
+        n = int(n_valid[b]) if n_valid is not None else k_bits.shape[1]
+        s = indexer_scores(bf16_to_f64(q_bits[b])[None], np.asarray(w[b], np.float64)[None],
+                           bf16_to_f64(k_bits[b, :n]))[0]
+        idx[b], val[b] = select_topk(s, np.arange(n), k)
+        all_scores.append(s)
+    if return_scores:
+        return idx, val, all_scores
+    return idx, val
+
+
+def prefill_select(q_bits, w, q_pos, k_bits, stride: int = 4, k: int = 512, rows=None,
+                   return_scores: bool = False):
+    """Causal prefill selection for the queries in ``rows`` (default: all)."""
+    T = q_bits.shape[0]
+    N = k_bits.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    n_t = eligible_count(q_pos, stride, N)
+    keys = bf16_to_f64(k_bits)
+    idx = np.empty((rows.size, k), dtype=np.int64)
+    val = np.empty((rows.size, k), dtype=np.float64)
+    all_scores = []
+    for i, t in enumerate(rows):
+        n = int(n_t[t])
+        s = indexer_scores(bf16_to_f64(q_bits[t])[None], np.asarray(w[t], np.float64)[None], keys[:n])[0]
+        idx[i], val[i] = select_topk(s, np.arange(n), k)
+        all_scores.append(s)
+    if return_scores:
+        return idx, val, all_scores
+    return idx, val
+
+
+def two_stage_select(q_bits, w, ck, ck_scale, fk, fk_scale, n_valid, shortlist: int, k: int = 512,
+                     rows=None, return_detail: bool = False):
+    """Compact scan -> shortlist -> exact re-rank of the originals -> top-k."""
+    B = q_bits.shape[0]
+    rows = np.arange(B) if rows is None else np.asarray(rows)
+    idx = np.empty((rows.size, k), dtype=np.int64)
+    val = np.empty((rows.size, k), dtype=np.float64)
+    detail = []
+    for i, b in enumerate(rows):
+        n = int(n_valid[b]) if n_valid is not None else ck.shape[1]
+        qb = bf16_to_f64(q_bits[b])[None]
+        wb = np.asarray(w[b], np.float64)[None]
+        s_hat = indexer_scores(qb, wb, dequant(ck[b, :n], ck_scale[b, :n], "int8"))[0]
+        short, _ = select_topk(s_hat, np.arange(n), shortlist)
+        short = short[short >= 0]
+        exact = indexer_scores(qb, wb, dequant(fk[b, short], fk_scale[b, short], "e4m3"))[0]
+        idx[i], val[i] = select_topk(exact, short, k)
+        if return_detail:
+            detail.append({"s_hat": s_hat, "shortlist": short, "exact_short": exact})
+    if return_detail:
+        return idx, val, detail
+    return idx, val
+
+
+def expand_buckets(picked, bucket_off, bucket_mem, budget: int) -> np.ndarray:
+    """Best-first expansion: members of the picked buckets in pick order, in
+    stored order within a bucket, until ``budget`` keys are held."""
+    out = []
+    for p in picked:
+        if p < 0:
+            break
+        for m in bucket_mem[bucket_off[p]: bucket_off[p + 1]]:
+            if len(out) == budget:
+                return np.asarray(out, dtype=np.int64)
+            out.append(int(m))
+    return np.asarray(out, dtype=np.int64)
+
+
+def bucket_select(q_bits, w, centroids, bucket_off, bucket_mem, key_bits, top_p: int, budget: int,
+                  k: int = 512, rows=None, return_detail: bool = False):
+    """Centroid scores -> top-p buckets -> expansion -> exact rescore -> top-k."""
+    T = q_bits.shape[0]
+    P = centroids.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    cent = bf16_to_f64(centroids)
+    idx = np.empty((rows.size, k), dtype=np.int64)
+    val = np.empty((rows.size, k), dtype=np.float64)
+    detail = []
+    for i, t in enumerate(rows):
+        qt = bf16_to_f64(q_bits[t])[None]
+        wt = np.asarray(w[t], np.float64)[None]
+        cs = indexer_scores(qt, wt, cent)[0]
+        picked, _ = select_topk(cs, np.arange(P), top_p)
+        cand = expand_buckets(picked, bucket_off, bucket_mem, budget)
+        exact = indexer_scores(qt, wt, bf16_to_f64(key_bits[cand]))[0]
+        idx[i], val[i] = select_topk(exact, cand, k)
+        if return_detail:
+            detail.append({"centroid_scores": cs, "picked": picked, "cand": cand, "exact_cand": exact})
+    if return_detail:
+        return idx, val, detail
+    return idx, val
+
+
+def recall_at_k(sel: np.ndarray, ref: np.ndarray) -> float:
+    """|S intersect S*| / |S*| averaged over rows (padding ignored)."""
+    sel = np.atleast_2d(sel)
+    ref = np.atleast_2d(ref)
+    tot = 0.0
+    for a, b in zip(sel, ref):
+        bs = set(int(x) for x in b if x >= 0)
+        if not bs:
+            tot += 1.0
+            continue
+        tot += len(bs & set(int(x) for x in a if x >= 0)) / len(bs)
+    return tot / len(sel)

@@ -1,0 +1,368 @@
+"""Pins of the fp64 oracle against facts fixed outside it (no GPU).
+
+Each test checks the oracle against something it cannot simply repeat: the
+formats' library decoders, pure-Python brute force, closed forms, invariants,
+explicit block construction, the pages' printed figures.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import brute, sizes
+from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64
+from oracle.indexer import eligible_blocks, eligible_count, indexer_scores
+from oracle.select import (
+    bucket_select, decode_select, expand_buckets, prefill_select, recall_at_k, select_topk,
+    topk_rows, two_stage_select,
+)
+from workloads import make_workload
+from workloads.synth import make_bucket, make_decode, make_two_stage, to_bf16_bits
+
+
+# --------------------------------------------------------------------------- #
+# formats: every code against the library casts
+# --------------------------------------------------------------------------- #
+def test_bf16_decode_all_codes():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = bf16_to_f64(bits)
+    both_nan = np.isnan(ref) & np.isnan(got)
+    assert np.array_equal(got[~both_nan], ref[~both_nan])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+
+
+def test_e4m3_decode_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = e4m3_to_f64(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    # a few fixed points of the format: max finite, smallest subnormal, 1.0
+    assert e4m3_to_f64(np.array([0x7E]))[0] == 448.0
+    assert e4m3_to_f64(np.array([0x01]))[0] == 2.0 ** -9
+    assert e4m3_to_f64(np.array([0x38]))[0] == 1.0
+    assert e4m3_to_f64(np.array([0xB8]))[0] == -1.0
+
+
+def test_dequant_scales():
+    codes = np.array([[0x38, 0x40]], dtype=np.uint8)  # 1.0, 2.0
+    v = dequant(codes, np.array([0.5], np.float32), "e4m3")
+    assert np.array_equal(v, [[0.5, 1.0]])
+    v = dequant(np.array([[-127, 3]], np.int8), np.array([0.25], np.float32), "int8")
+    assert np.array_equal(v, [[-31.75, 0.75]])
+
+
+# --------------------------------------------------------------------------- #
+# scores
+# --------------------------------------------------------------------------- #
+def test_scores_closed_form():
+    # H=2, d=2.  Head 0 sees +k0 dims, head 1 sees -k0: exactly one ReLU is open.
+    q = np.array([[[1.0, 0.0], [-1.0, 0.0]]])
+    w = np.array([[2.0, -3.0]])
+    k = np.array([[5.0, 7.0], [-2.0, 11.0]])
+    s = indexer_scores(q, w, k)
+    # s0 = 2*max(0,5) - 3*max(0,-5) = 10 ; s1 = 2*max(0,-2) - 3*max(0,2) = -6
+    assert np.array_equal(s, [[10.0, -6.0]])
+
+
+def test_scores_brute_force_tiny():
+    rng = np.random.default_rng(1)
+    T, H, d, N = 3, 4, 5, 9
+    q = rng.standard_normal((T, H, d))
+    w = rng.standard_normal((T, H))
+    k = rng.standard_normal((N, d))
+    got = indexer_scores(q, w, k)
+    for t in range(T):
+        for s in range(N):
+            ref = brute.score(q[t].tolist(), w[t].tolist(), k[s].tolist())
+            assert abs(got[t, s] - ref) <= 1e-12 * (1 + abs(ref))
+
+
+def test_scores_gemv_special_case():
+    # one head, unit weight, every dot positive: the score is a plain GEMV
+    rng = np.random.default_rng(2)
+    q = np.abs(rng.standard_normal((1, 1, 16)))
+    k = np.abs(rng.standard_normal((33, 16)))
+    got = indexer_scores(q, np.ones((1, 1)), k)[0]
+    assert np.allclose(got, np.dot(k, q[0, 0]), rtol=1e-14, atol=0)
+
+
+def test_scores_invariants():
+    rng = np.random.default_rng(3)
+    T, H, d, N = 2, 6, 8, 20
+    q = rng.standard_normal((T, H, d))
+    w = rng.standard_normal((T, H))
+    k = rng.standard_normal((N, d))
+    s = indexer_scores(q, w, k)
+    # positive homogeneity of ReLU in q and linearity in w
+    assert np.allclose(indexer_scores(2.5 * q, w, k), 2.5 * s, rtol=1e-12, atol=1e-12)
+    assert np.allclose(indexer_scores(q, -w, k), -s, rtol=1e-12, atol=1e-12)
+    # heads are a set: permuting them together with w changes nothing
+    perm = rng.permutation(H)
+    assert np.allclose(indexer_scores(q[:, perm], w[:, perm], k), s, rtol=1e-12, atol=1e-12)
+    # keys are positions: permuting keys permutes the scores
+    kp = rng.permutation(N)
+    assert np.allclose(indexer_scores(q, w, k[kp]), s[:, kp], rtol=1e-12, atol=1e-12)
+    # a head whose dots are all negative contributes nothing
+    q2 = q.copy()
+    q2[:, 0] = 0.0
+    w2 = w.copy()
+    w2[:, 0] = 1e6
+    assert np.allclose(indexer_scores(q2, w2, k), indexer_scores(q2[:, 1:], w2[:, 1:], k))
+
+
+# --------------------------------------------------------------------------- #
+# eligibility
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("stride", [1, 2, 3, 4])
+def test_eligibility_matches_blocks(stride):
+    n_keys = 12
+    for t in range(0, 4 * n_keys + 3):
+        blocks = eligible_blocks(t, stride, n_keys)
+        n = int(eligible_count(np.array([t]), stride, n_keys)[0])
+        assert blocks == list(range(n)), (t, stride)
+
+
+def test_eligibility_edges_stride4():
+    # t = 0..7: the first block [0..3] completes at t = 3, the second at t = 7
+    got = eligible_count(np.arange(8), 4, 100).tolist()
+    assert got == [0, 0, 0, 1, 1, 1, 1, 2]
+
+
+def test_prefill_chunk_eligible_pairs():
+    t = np.arange(126976, 131072)
+    n = eligible_count(t, 4, 32768)
+    assert n.min() == 31744 and n.max() == 32768
+    assert int(n.sum()) == 132119552
+
+
+# --------------------------------------------------------------------------- #
+# top-k order
+# --------------------------------------------------------------------------- #
+def _check_topk_vs_brute(vals, k):
+    pos = list(range(len(vals)))
+    bp, bv = brute.topk([float(v) for v in vals], pos, k)
+    gp, gv = select_topk(np.asarray(vals), np.arange(len(vals)), k)
+    assert gp.tolist() == bp
+    for a, b in zip(gv.tolist(), bv):
+        assert (math.isnan(a) and math.isnan(b)) or a == b
+
+
+def test_topk_brute_force_with_ties():
+    rng = np.random.default_rng(4)
+    for trial in range(30):
+        n = int(rng.integers(1, 60))
+        vals = rng.integers(-3, 4, size=n).astype(np.float64)
+        if trial % 3 == 0:
+            vals[rng.integers(0, n, size=max(1, n // 5))] = np.nan
+        if trial % 4 == 0:
+            vals[rng.integers(0, n, size=max(1, n // 5))] = -np.inf
+        for k in (1, 5, n, n + 3):
+            _check_topk_vs_brute(vals, k)
+
+
+def test_topk_adversarial():
+    # all equal: the first k positions
+    p, _ = select_topk(np.zeros(100, np.float32), np.arange(100), 10)
+    assert p.tolist() == list(range(10))
+    # -0.0 ties +0.0: lower position first whatever the sign bit
+    v = np.array([0.0, -0.0, 0.0, -0.0], np.float32)
+    p, val = select_topk(v, np.arange(4), 4)
+    assert p.tolist() == [0, 1, 2, 3]
+    assert np.signbit(val).tolist() == [False, True, False, True]
+    # -inf above NaN, NaN above padding
+    v = np.array([np.nan, -np.inf, 1.0], np.float32)
+    p, val = select_topk(v, np.arange(3), 5)
+    assert p.tolist() == [2, 1, 0, -1, -1]
+    assert val[3] == -np.inf and math.isnan(val[2])
+    # duplicated maxima
+    v = np.array([1, 5, 5, 2, 5], np.float32)
+    p, _ = select_topk(v, np.arange(5), 2)
+    assert p.tolist() == [1, 2]
+    # positions are labels, not indexes: ties go to the lower label
+    p, _ = select_topk(np.array([1.0, 1.0]), np.array([9, 4]), 1)
+    assert p.tolist() == [4]
+
+
+def test_topk_rows_prefix_and_padding():
+    s = np.array([[3, 1, 2, 9], [5, 5, 5, 5]], np.float32)
+    idx, val = topk_rows(s, np.array([3, 0]), 2)
+    assert idx.tolist() == [[0, 2], [-1, -1]]
+    assert val.dtype == np.float32
+
+
+def test_topk_is_prefix_of_full_sort():
+    rng = np.random.default_rng(5)
+    v = rng.standard_normal(500).astype(np.float32)
+    v[::7] = v[3]
+    full_p, _ = brute.full_sort(v.tolist(), list(range(500)))
+    for k in (1, 17, 128, 499):
+        p, _ = select_topk(v, np.arange(500), k)
+        assert p.tolist() == full_p[:k]
+
+
+# --------------------------------------------------------------------------- #
+# pipelines
+# --------------------------------------------------------------------------- #
+def test_decode_select_brute_force_tiny():
+    data = make_decode(B=2, N=40, H=3, d=6, seed=7, n_valid=np.array([40, 23]))
+    idx, val = decode_select(data["q"], data["w"], data["k"], data["n_valid"], k=8)
+    for b in range(2):
+        n = int(data["n_valid"][b])
+        qb = bf16_to_f64(data["q"][b]).tolist()
+        kb = bf16_to_f64(data["k"][b, :n]).tolist()
+        sc = [brute.score(qb, data["w"][b].astype(np.float64).tolist(), kb[s]) for s in range(n)]
+        bp, bv = brute.topk(sc, list(range(n)), 8)
+        assert idx[b].tolist() == bp
+        assert np.allclose(val[b], bv, rtol=1e-12, atol=1e-15)
+
+
+def test_prefill_select_brute_force_tiny():
+    data = make_workload("prefill_s")
+    q, w, k, q_pos = data["q"][:4, :3, :], data["w"][:4, :3], data["k"][:80], data["q_pos"][:4] - 3800
+    idx, val = prefill_select(q, w, q_pos, k, stride=4, k=16)
+    kf = bf16_to_f64(k).tolist()
+    for t in range(4):
+        elig = eligible_blocks(int(q_pos[t]), 4, 80)
+        sc = [brute.score(bf16_to_f64(q[t]).tolist(), w[t].astype(np.float64).tolist(), kf[s]) for s in elig]
+        bp, bv = brute.topk(sc, elig, 16)
+        assert idx[t].tolist() == bp
+
+
+def test_two_stage_full_shortlist_equals_exact():
+    d = make_two_stage(B=2, N=700, H=4, d=16, seed=8, plant_frac=0.05, ragged=100)
+    n = d["n_valid"]
+    got_i, got_v = two_stage_select(d["q"], d["w"], d["ck"], d["ck_scale"], d["fk"], d["fk_scale"], n,
+                                    shortlist=700, k=32)
+    for b in range(2):
+        keys = dequant(d["fk"][b, : n[b]], d["fk_scale"][b, : n[b]], "e4m3")
+        s = indexer_scores(bf16_to_f64(d["q"][b])[None], d["w"][b].astype(np.float64)[None], keys)[0]
+        ei, ev = select_topk(s, np.arange(n[b]), 32)
+        assert np.array_equal(got_i[b], ei)
+        assert np.array_equal(got_v[b], ev)
+
+
+def test_two_stage_brute_force_tiny():
+    d = make_two_stage(B=1, N=60, H=2, d=8, seed=9, plant_frac=0.1)
+    gi, gv, det = two_stage_select(d["q"], d["w"], d["ck"], d["ck_scale"], d["fk"], d["fk_scale"],
+                                   d["n_valid"], shortlist=12, k=5, return_detail=True)
+    qb = bf16_to_f64(d["q"][0]).tolist()
+    wb = d["w"][0].astype(np.float64).tolist()
+    ck = [[float(x) * float(d["ck_scale"][0, s]) for x in d["ck"][0, s]] for s in range(60)]
+    fk = e4m3_to_f64(d["fk"][0]) * d["fk_scale"][0].astype(np.float64)[:, None]
+    shat = [brute.score(qb, wb, ck[s]) for s in range(60)]
+    short, _ = brute.topk(shat, list(range(60)), 12)
+    ex = [brute.score(qb, wb, fk[s].tolist()) for s in short]
+    bp, _ = brute.topk(ex, short, 5)
+    assert gi[0].tolist() == bp
+    assert det[0]["shortlist"].tolist() == short
+
+
+def test_bucket_full_budget_equals_exact():
+    d = make_bucket(T=3, clusters=50, cluster_size=8, H=4, d=16, seed=10, min_size=4, max_size=16)
+    P = 50
+    N = d["keys"].shape[0]
+    gi, gv = bucket_select(d["q"], d["w"], d["centroids"], d["bucket_off"], d["bucket_mem"], d["keys"],
+                           top_p=P, budget=N, k=64)
+    ri, rv = decode_select(d["q"], d["w"], np.broadcast_to(d["keys"], (3,) + d["keys"].shape),
+                           np.full(3, N), k=64)
+    assert np.array_equal(gi, ri)
+    assert np.array_equal(gv, rv)
+
+
+def test_bucket_expansion_cuts_last_bucket():
+    off = np.array([0, 3, 5, 9])
+    mem = np.array([10, 11, 12, 20, 21, 30, 31, 32, 33])
+    # picked order 2, 0, 1 with budget 6: all of bucket 2, then 2 of bucket 0
+    assert expand_buckets([2, 0, 1], off, mem, 6).tolist() == [30, 31, 32, 33, 10, 11]
+    assert expand_buckets([1, -1], off, mem, 6).tolist() == [20, 21]
+
+
+def test_bucket_brute_force_tiny():
+    d = make_bucket(T=2, clusters=12, cluster_size=8, H=2, d=8, seed=11, min_size=2, max_size=6)
+    gi, gv, det = bucket_select(d["q"], d["w"], d["centroids"], d["bucket_off"], d["bucket_mem"], d["keys"],
+                                top_p=4, budget=10, k=6, return_detail=True)
+    cf = bf16_to_f64(d["centroids"]).tolist()
+    kf = bf16_to_f64(d["keys"]).tolist()
+    for t in range(2):
+        qt = bf16_to_f64(d["q"][t]).tolist()
+        wt = d["w"][t].astype(np.float64).tolist()
+        cs = [brute.score(qt, wt, c) for c in cf]
+        picked, _ = brute.topk(cs, list(range(12)), 4)
+        cand = []
+        for p in picked:
+            for m in d["bucket_mem"][d["bucket_off"][p]: d["bucket_off"][p + 1]]:
+                if len(cand) < 10:
+                    cand.append(int(m))
+        ex = [brute.score(qt, wt, kf[m]) for m in cand]
+        bp, _ = brute.topk(ex, cand, 6)
+        assert gi[t].tolist() == bp
+        assert det[t]["cand"].tolist() == cand
+
+
+def test_recall():
+    assert recall_at_k(np.array([[1, 2, 3]]), np.array([[3, 2, 1]])) == 1.0
+    assert recall_at_k(np.array([[1, 2, 9]]), np.array([[3, 2, 1]])) == pytest.approx(2 / 3)
+
+
+def test_bucket_generator_centroid_is_member_mean():
+    d = make_bucket(T=1, clusters=20, cluster_size=8, H=2, d=16, seed=12)
+    kf = bf16_to_f64(d["keys"])
+    for p in range(20):
+        mem = d["bucket_mem"][d["bucket_off"][p]: d["bucket_off"][p + 1]]
+        assert list(mem) == sorted(mem)
+        mean = kf[mem].mean(axis=0)
+        assert np.array_equal(d["centroids"][p], to_bf16_bits(mean))
+
+
+# --------------------------------------------------------------------------- #
+# the pages' printed figures
+# --------------------------------------------------------------------------- #
+def _golden(golden_dir):
+    with open(os.path.join(golden_dir, "page_figures.json")) as f:
+        return json.load(f)
+
+
+def _close(got, fig):
+    if "abs_tol" in fig:
+        return abs(got - fig["value"]) <= fig["abs_tol"]
+    return abs(got - fig["value"]) <= fig["rel_tol"] * abs(fig["value"]) + 1e-12
+
+
+def test_page_figures(golden_dir):
+    g = _golden(golden_dir)
+    assert sizes.INDEXER_ENTRY_BYTES == g["indexer_entry_bytes"]["value"]
+    assert sizes.KV_ENTRY_BYTES == g["kv_latent_entry_bytes"]["value"]
+    f = g["indexer_mb_per_layer_128k"]
+    assert _close(sizes.indexer_bytes(f["tokens"]) / 1e6, f)
+    f = g["indexer_gb_61_layers_128k"]
+    assert _close(f["layers"] * sizes.indexer_bytes(f["tokens"]) / 1e9, f)
+    f = g["indexer_kflop_per_token_64_heads"]
+    assert _close(sizes.indexer_flops_per_pair(f["heads"]) / 1e3, f)
+    f = g["indexer_main_crossover_tokens"]
+    assert _close(f["k"] * sizes.KV_ENTRY_BYTES / sizes.INDEXER_ENTRY_BYTES, f)
+    f = g["prefill_history_load_ms"]
+    assert _close(sizes.prefill_history_load_ms(f["tokens"], f["gbps"]), f)
+    f = g["key_to_hot_buffer_ratio_512k"]
+    assert _close(sizes.key_to_hot_buffer_ratio(f["tokens"]), f)
+    h = sizes.lsa_holding(g["lsa_10m_buckets"]["tokens"])
+    assert h["buckets"] == g["lsa_10m_buckets"]["value"]
+    assert h["centroid_bytes"] == g["lsa_10m_centroid_mib"]["value"] * 2 ** 20
+    assert h["member_bytes"] == g["lsa_10m_member_mib"]["value"] * 2 ** 20
+    assert h["glm_keys"] == g["glm_10m_indexer_keys"]["value"]
+    assert h["glm_key_bytes"] == g["glm_10m_indexer_key_mib"]["value"] * 2 ** 20
+
+
+def test_ratio_readings():
+    # 512K read as 512,000 tokens gives 7.16 (the printed 7.2); the binary
+    # reading gives 7.33; without the 4 B scale the figures drop to 6.94 / 7.11.
+    assert sizes.key_to_hot_buffer_ratio(512000) == pytest.approx(7.1615, abs=1e-3)
+    assert sizes.key_to_hot_buffer_ratio(524288) == pytest.approx(7.3333, abs=1e-3)
+    assert sizes.key_to_hot_buffer_ratio(512000, with_scale=False) == pytest.approx(6.944, abs=1e-3)
+    assert abs(sizes.key_to_hot_buffer_ratio(512000) - 7.2) <= 0.05

@@ -1,0 +1,106 @@
+"""Shapes of the indexer workloads.
+
+Five full-size workloads follow the shapes the pages use:
+
+* ``decode_tiny``   -- 4 sequences x 8192 tokens (2048 stride-4 compressed
+  positions), one query each.
+* ``decode_batch``  -- 64 sequences x 131072 tokens (32768 positions each).
+* ``prefill_chunk`` -- one 4096-query chunk at token positions
+  126976..131071 against 131072 history tokens (32768 positions), history
+  streamed in 8192-key tiles through two device buffers (LeanSparse podcast
+  transcript, 05:36-06:44).
+* ``two_stage``     -- 32 sequences x 524288 tokens (131072 positions each):
+  compact int8 scan, 4096-entry shortlist, exact re-rank of fp8 originals
+  (LeanSparse podcast transcript, 07:12-08:00).
+* ``bucket``        -- one sequence of 1048576 tokens (262144 keys) built as
+  32768 clusters of 8 keys; 256 decode queries keep 64 buckets and expand them
+  to 512 keys ("Latent Sparse Attention", "How LSA finds the keys").
+
+Indexer geometry everywhere: H = 32 heads, d = 128, top-k = 512 (the
+GLM-shaped indexer of "Latent Sparse Attention", "Where the time goes"; k = 512
+as in the LeanSparse transcript, 01:33-02:06).
+
+Reduced variants (suffix ``_s``) keep every structural feature (several tiles,
+ragged tails, causal prefix, planted keys, clusters) at sizes the fp64 oracle
+finishes in seconds; they are parity cases.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field, replace
+from typing import Dict
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str  # "decode" | "prefill" | "two_stage" | "bucket"
+    H: int = 32
+    d: int = 128
+    k: int = 512
+    seed: int = 0
+    # decode / two_stage
+    B: int = 0
+    N: int = 0
+    # ragged decode: per-sequence valid lengths drawn in [N - ragged, N]
+    ragged: int = 0
+    # prefill
+    T: int = 0
+    q_pos0: int = 0
+    stride: int = 4
+    tile_keys: int = 8192
+    # two_stage
+    shortlist: int = 0
+    plant_frac: float = 0.0
+    plant_cos: float = 0.6
+    # bucket
+    clusters: int = 0
+    cluster_size: int = 0
+    noise_rel: float = 0.3
+    top_p: int = 0
+    budget: int = 0
+    extra: Dict[str, int] = field(default_factory=dict)
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+    # ---- sizes used by the benchmark and the tests -------------------------
+    @property
+    def n_keys(self) -> int:
+        if self.kind == "bucket":
+            return self.clusters * self.cluster_size
+        return self.N
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "decode_tiny": Workload("decode_tiny", "decode", B=4, N=2048),
+    "decode_batch": Workload("decode_batch", "decode", B=64, N=32768),
+    "prefill_chunk": Workload(
+        "prefill_chunk", "prefill", T=4096, q_pos0=126976, N=32768, stride=4, tile_keys=8192
+    ),
+    "two_stage": Workload(
+        "two_stage", "two_stage", B=32, N=131072, shortlist=4096, plant_frac=0.05, plant_cos=0.6
+    ),
+    "bucket": Workload(
+        "bucket", "bucket", T=256, clusters=32768, cluster_size=8, noise_rel=0.3, top_p=64, budget=512
+    ),
+    # ---- reduced parity cases: several tiles, ragged tails ------------------
+    "decode_s": Workload("decode_s", "decode", B=5, N=3000, ragged=700),
+    "prefill_s": Workload(
+        "prefill_s", "prefill", T=77, q_pos0=4000, N=1019, stride=4, tile_keys=256
+    ),
+    "two_stage_s": Workload(
+        "two_stage_s", "two_stage", B=3, N=9000, shortlist=1024, plant_frac=0.05, plant_cos=0.6, ragged=1500
+    ),
+    "bucket_s": Workload(
+        "bucket_s", "bucket", T=19, clusters=1500, cluster_size=8, noise_rel=0.3, top_p=64, budget=512,
+        extra={"min_size": 4, "max_size": 16},
+    ),
+}
+
+
+def get_workload(name: str) -> Workload:
+    try:
+        return WORKLOADS[name]
+    except KeyError:
+        raise KeyError(f"unknown workload {name!r}; known: {sorted(WORKLOADS)}") from None

@@ -1,0 +1,227 @@
+"""Seeded generators for the indexer workloads.
+
+Every generator draws from ``numpy.random.default_rng(seed)`` in a fixed order
+and returns host numpy arrays holding the exact bytes both the CUDA path and the
+oracle read:
+
+* bf16 tensors as ``uint16`` bit patterns (fp64 draws rounded to nearest even
+  through torch's bf16 cast),
+* fp8 e4m3 tensors as ``uint8`` codes (torch's ``float8_e4m3fn`` cast, input
+  clipped to +-448 first so nothing becomes NaN),
+* int8 tensors as ``int8``, scales and head weights as ``float32``,
+* positions as ``int64`` / ``int32``.
+
+Distributions (all workloads): q, k ~ N(0, 1)/sqrt(d), w ~ N(0, 1)/sqrt(H).
+
+Random numbers only: the scoring and selection arithmetic lives in the oracle
+and in the CUDA library, never here.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from .shapes import Workload, get_workload
+
+
+# --------------------------------------------------------------------------- #
+# storage-format encoders (library casts)
+# --------------------------------------------------------------------------- #
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp64/fp32 array -> bf16 bit patterns (uint16), round to nearest even."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def bf16_bits_to_f32(u: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(u).view(np.int16)).view(torch.bfloat16)
+    return t.to(torch.float32).numpy()
+
+
+def to_e4m3_codes(x: np.ndarray) -> np.ndarray:
+    """Values already divided by their scale -> e4m3 codes (uint8)."""
+    x = np.clip(np.asarray(x, dtype=np.float32), -448.0, 448.0)
+    t = torch.from_numpy(np.ascontiguousarray(x)).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy().copy()
+
+
+def e4m3_codes_to_f32(c: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(c, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float32).numpy()
+
+
+def _normal(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
+    return rng.standard_normal(shape) * scale
+
+
+# --------------------------------------------------------------------------- #
+# decode: B sequences, one query each, bf16 keys
+# --------------------------------------------------------------------------- #
+def make_decode(
+    B: int, N: int, H: int = 32, d: int = 128, seed: int = 0, ragged: int = 0,
+    n_valid: Optional[np.ndarray] = None,
+) -> Dict[str, np.ndarray]:
+    rng = np.random.default_rng(seed)
+    q = to_bf16_bits(_normal(rng, (B, H, d), 1.0 / math.sqrt(d)))
+    w = _normal(rng, (B, H), 1.0 / math.sqrt(H)).astype(np.float32)
+    k = np.empty((B, N, d), dtype=np.uint16)
+    for b in range(B):  # per sequence, to bound the fp64 working set
+        k[b] = to_bf16_bits(_normal(rng, (N, d), 1.0 / math.sqrt(d)))
+    if n_valid is None:
+        if ragged:
+            n_valid = rng.integers(max(N - ragged, 0), N + 1, size=B)
+        else:
+            n_valid = np.full(B, N)
+    return {"q": q, "w": w, "k": k, "n_valid": np.asarray(n_valid, dtype=np.int32)}
+
+
+# --------------------------------------------------------------------------- #
+# prefill: T queries at consecutive token positions, one history of N keys
+# --------------------------------------------------------------------------- #
+def make_prefill(
+    T: int, N: int, q_pos0: int, H: int = 32, d: int = 128, seed: int = 0
+) -> Dict[str, np.ndarray]:
+    rng = np.random.default_rng(seed)
+    q = to_bf16_bits(_normal(rng, (T, H, d), 1.0 / math.sqrt(d)))
+    w = _normal(rng, (T, H), 1.0 / math.sqrt(H)).astype(np.float32)
+    k = np.empty((N, d), dtype=np.uint16)
+    step = 8192
+    for s in range(0, N, step):
+        e = min(N, s + step)
+        k[s:e] = to_bf16_bits(_normal(rng, (e - s, d), 1.0 / math.sqrt(d)))
+    q_pos = (q_pos0 + np.arange(T)).astype(np.int64)
+    return {"q": q, "w": w, "k": k, "q_pos": q_pos}
+
+
+# --------------------------------------------------------------------------- #
+# two-stage decode: fp8 full keys with planted high scorers, int8 compact keys
+# --------------------------------------------------------------------------- #
+def make_two_stage(
+    B: int, N: int, H: int = 32, d: int = 128, seed: int = 0, plant_frac: float = 0.05,
+    plant_cos: float = 0.6, ragged: int = 0,
+) -> Dict[str, np.ndarray]:
+    """Full keys: fp8 e4m3 codes with a per-key fp32 scale amax/448.
+
+    A fraction ``plant_frac`` of positions per sequence (chosen uniformly
+    without replacement) is replaced by keys whose direction has cosine
+    ``plant_cos`` with a per-sequence query direction u = normalise(sum_h
+    max(w_h, 0) q_h); the key keeps the norm of the Gaussian draw it replaces.
+
+    Compact keys: int8 codes of the dequantised full key with a per-key fp32
+    scale amax/127, rounded half to even, clamped to +-127.
+    """
+    rng = np.random.default_rng(seed)
+    q = to_bf16_bits(_normal(rng, (B, H, d), 1.0 / math.sqrt(d)))
+    w = _normal(rng, (B, H), 1.0 / math.sqrt(H)).astype(np.float32)
+    qf = bf16_bits_to_f32(q).astype(np.float64)
+    fk = np.empty((B, N, d), dtype=np.uint8)
+    fk_scale = np.empty((B, N), dtype=np.float32)
+    ck = np.empty((B, N, d), dtype=np.int8)
+    ck_scale = np.empty((B, N), dtype=np.float32)
+    planted = []
+    sin = math.sqrt(max(0.0, 1.0 - plant_cos * plant_cos))
+    for b in range(B):
+        g = _normal(rng, (N, d), 1.0 / math.sqrt(d))
+        n_plant = int(round(plant_frac * N))
+        pos = np.sort(rng.choice(N, size=n_plant, replace=False))
+        u = (np.maximum(w[b].astype(np.float64), 0.0)[:, None] * qf[b]).sum(0)
+        u /= np.linalg.norm(u)
+        z = rng.standard_normal((n_plant, d))
+        z -= (z @ u)[:, None] * u[None, :]
+        z /= np.linalg.norm(z, axis=1, keepdims=True)
+        norms = np.linalg.norm(g[pos], axis=1, keepdims=True)
+        g[pos] = norms * (plant_cos * u[None, :] + sin * z)
+        planted.append(pos.astype(np.int32))
+        amax = np.abs(g).max(axis=1)
+        sc = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32)
+        codes = to_e4m3_codes(g / sc.astype(np.float64)[:, None])
+        fk[b] = codes
+        fk_scale[b] = sc
+        deq = e4m3_codes_to_f32(codes).astype(np.float64) * sc.astype(np.float64)[:, None]
+        camax = np.abs(deq).max(axis=1)
+        cs = np.where(camax > 0, camax / 127.0, 1.0).astype(np.float32)
+        ck[b] = np.clip(np.rint(deq / cs.astype(np.float64)[:, None]), -127, 127).astype(np.int8)
+        ck_scale[b] = cs
+    if ragged:
+        n_valid = rng.integers(max(N - ragged, 0), N + 1, size=B)
+    else:
+        n_valid = np.full(B, N)
+    return {
+        "q": q, "w": w, "fk": fk, "fk_scale": fk_scale, "ck": ck, "ck_scale": ck_scale,
+        "n_valid": n_valid.astype(np.int32), "planted": planted,
+    }
+
+
+# --------------------------------------------------------------------------- #
+# bucket search: clusters of keys scattered over positions, centroid = mean
+# --------------------------------------------------------------------------- #
+def make_bucket(
+    T: int, clusters: int, cluster_size: int, H: int = 32, d: int = 128, seed: int = 0,
+    noise_rel: float = 0.3, min_size: int = 0, max_size: int = 0,
+) -> Dict[str, np.ndarray]:
+    """Clustered keys for the bucket search.
+
+    Cluster centres ~ N(0, 1)/sqrt(d); each member = centre + noise whose
+    expected norm is ``noise_rel`` times the centre's norm (per-coordinate std
+    noise_rel*|c|/sqrt(d)).  Members sit at positions given by a seeded
+    permutation, stored in ascending order per bucket (CSR ``bucket_off`` /
+    ``bucket_mem``).  The stored centroid is the fp64 mean of the bucket's
+    stored bf16 keys, rounded to bf16.  With ``min_size``/``max_size`` set,
+    bucket sizes are drawn uniformly from that range instead of being
+    ``cluster_size``.
+    """
+    rng = np.random.default_rng(seed)
+    P = clusters
+    if min_size and max_size:
+        sizes = rng.integers(min_size, max_size + 1, size=P)
+    else:
+        sizes = np.full(P, cluster_size)
+    off = np.zeros(P + 1, dtype=np.int64)
+    np.cumsum(sizes, out=off[1:])
+    N = int(off[-1])
+    centres = _normal(rng, (P, d), 1.0 / math.sqrt(d))
+    sigma = noise_rel * np.linalg.norm(centres, axis=1) / math.sqrt(d)
+    member_keys = np.repeat(centres, sizes, axis=0) + rng.standard_normal((N, d)) * np.repeat(sigma, sizes)[:, None]
+    perm = rng.permutation(N)
+    members = np.empty(N, dtype=np.int32)
+    keys = np.empty((N, d), dtype=np.uint16)
+    kb = to_bf16_bits(member_keys)
+    for p in range(P):
+        s, e = off[p], off[p + 1]
+        order = np.argsort(perm[s:e], kind="stable")
+        pos = perm[s:e][order]
+        members[s:e] = pos
+        keys[pos] = kb[s:e][order]
+    kf = bf16_bits_to_f32(keys).astype(np.float64)
+    sums = np.add.reduceat(kf[members], off[:-1], axis=0)
+    centroids = to_bf16_bits(sums / sizes[:, None])
+    q = to_bf16_bits(_normal(rng, (T, H, d), 1.0 / math.sqrt(d)))
+    w = _normal(rng, (T, H), 1.0 / math.sqrt(H)).astype(np.float32)
+    return {
+        "q": q, "w": w, "centroids": centroids, "bucket_off": off.astype(np.int32),
+        "bucket_mem": members, "keys": keys,
+    }
+
+
+def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Inputs for a named workload (or a ``Workload``)."""
+    if isinstance(wl, str):
+        wl = get_workload(wl)
+    assert isinstance(wl, Workload)
+    s = wl.seed if seed is None else seed
+    if wl.kind == "decode":
+        return make_decode(wl.B, wl.N, wl.H, wl.d, s, ragged=wl.ragged)
+    if wl.kind == "prefill":
+        return make_prefill(wl.T, wl.N, wl.q_pos0, wl.H, wl.d, s)
+    if wl.kind == "two_stage":
+        return make_two_stage(wl.B, wl.N, wl.H, wl.d, s, wl.plant_frac, wl.plant_cos, ragged=wl.ragged)
+    if wl.kind == "bucket":
+        return make_bucket(
+            wl.T, wl.clusters, wl.cluster_size, wl.H, wl.d, s, wl.noise_rel,
+            wl.extra.get("min_size", 0), wl.extra.get("max_size", 0),
+        )
+    raise ValueError(wl.kind)
