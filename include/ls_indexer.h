@@ -1,0 +1,210 @@
+/*
+ * ls_indexer.h -- C ABI of the B200 (sm_100a) lightning-indexer selection
+ * library, libls_indexer.so.
+ *
+ * The library computes the lightning-indexer pass of a compressed-sparse-
+ * attention layer: every eligible compressed history position s of a query t
+ * is scored as
+ *
+ *     score(t, s) = sum_h w[t, h] * max(0, q[t, h] . k[s])
+ *
+ * (the weighted-ReLU dot product of the DSA lightning indexer, "03 long
+ * context" lecture, section "The Architectural Answer: Read Less of the Past",
+ * stage 1; the 32-head x 128-d GLM-shaped form with ReLU and head weights,
+ * "Latent Sparse Attention", section "Where the time goes"), and the top-k
+ * positions are selected (k = 512 in DeepSeek-V4-Flash, LeanSparse podcast
+ * transcript 01:33-02:06).
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Tensor arguments are DEVICE pointers owned by the caller, row-major and
+ *   contiguous, unless a call says otherwise.  bf16 tensors are passed as
+ *   16-bit patterns (uint16_t), fp8 e4m3 as uint8_t codes.
+ * - q, key and centroid tensors must be 16-byte aligned (they are read by TMA
+ *   or bulk copies); w, scales and outputs must be 16-byte aligned too.
+ * - Only H = 32 heads and d = 128 are built; other shapes return
+ *   LS_ERR_UNSUPPORTED.  k <= 4096 (no 2048 cap).
+ * - All work is enqueued asynchronously on the caller's stream(s); a stream
+ *   argument is a cudaStream_t passed as void* (NULL = legacy default stream).
+ * - Scratch memory comes from the caller: calls that need it take (ws,
+ *   ws_bytes) and have a *_workspace_size() query.  The library allocates no
+ *   device memory.  A short workspace returns LS_ERR_WORKSPACE.
+ * - Ordering of selections: score descending, then position ascending; -0.0
+ *   equals +0.0; NaN ranks below -inf.  Selected lists are written in that
+ *   order.  Rows with fewer than k eligible positions are padded with
+ *   idx = -1, val = -inf.  Values are bit copies of the scores.
+ * - Masked (ineligible) positions in score outputs hold -inf.
+ * - Errors: every call returns an ls_status; ls_last_error() gives a
+ *   thread-local message for the last failing call of the thread.  No C++
+ *   exception crosses the ABI.  Kernels never trap: a wait inside a kernel
+ *   that exceeds its time limit sets a device fault word that
+ *   ls_device_status() reads (LS_FAULT_* bits).
+ */
+#ifndef LS_INDEXER_H
+#define LS_INDEXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int ls_status;
+#define LS_OK 0
+#define LS_ERR_INVALID_ARG 1  /* null / misaligned pointer, bad size, bad enum */
+#define LS_ERR_WORKSPACE 2    /* ws_bytes smaller than the *_workspace_size() answer */
+#define LS_ERR_UNSUPPORTED 3  /* shape or dtype not built (H != 32, d != 128, ...) */
+#define LS_ERR_CUDA 4         /* a CUDA runtime call failed; see ls_last_error() */
+#define LS_ERR_TIMEOUT 5      /* a bounded device wait ran out (ls_device_status) */
+
+/* device fault bits reported by ls_device_status() */
+#define LS_FAULT_WAIT_TIMEOUT 1 /* an in-kernel wait exceeded its limit */
+#define LS_FAULT_BAD_INDEX 2    /* a gathered row id was outside the key array */
+
+/* key storage formats */
+#define LS_KEY_BF16 0     /* [.][d] bf16 */
+#define LS_KEY_FP8_E4M3 1 /* [.][d] e4m3 codes + per-key fp32 scale (128 B + 4 B) */
+#define LS_KEY_INT8 2     /* [.][d] int8 codes + per-key fp32 scale */
+
+/* Message describing the last failing call on this thread ("" if none). */
+const char* ls_last_error(void);
+
+/* ABI version of this header (major*100 + minor). */
+int ls_version(void);
+
+/*
+ * Read and clear the device fault word (LS_FAULT_* bits) after synchronising
+ * `stream`.  Returns LS_ERR_TIMEOUT if LS_FAULT_WAIT_TIMEOUT was set,
+ * LS_ERR_INVALID_ARG if only LS_FAULT_BAD_INDEX was set, LS_OK otherwise;
+ * *flags (may be NULL) receives the bits.  Blocks the host.
+ */
+ls_status ls_device_status(int* flags, void* stream);
+
+/*
+ * ls_indexer_score -- indexer scores of every key for every query.
+ * ("03 long context", "The Architectural Answer: Read Less of the Past".)
+ *
+ *   q        [B][T][H][d] bf16        queries (T per sequence)
+ *   w        [B][T][H]    fp32        head weights
+ *   keys     [B][N][d]    key_dtype   keys of each sequence
+ *   key_scale[B][N]       fp32        per-key scale (FP8/INT8 keys; NULL for BF16);
+ *                                     FP8/INT8 scores use max(0, scale*(q.code))
+ *   n_valid  [B] int32 or NULL        keys n >= n_valid[b] are masked
+ *   q_pos    [B][T] int64 or NULL     token position of each query; when given,
+ *                                     key n is masked unless stride*n+stride-1 <= q_pos
+ *                                     (a compressed entry is visible once its whole
+ *                                     block of `stride` tokens precedes the query;
+ *                                     LeanSparse transcript 02:36-02:56)
+ *   scores   [B][T][N]    fp32        output; masked entries are -inf
+ * BF16 keys take any T >= 1 (tensor-core tiles of 8 queries x 32 heads when
+ * T > 1, one query per tile when T == 1).  FP8/INT8 keys take T == 1 and no
+ * q_pos.  No workspace.
+ */
+ls_status ls_indexer_score(const uint16_t* q, const float* w, const void* keys, int key_dtype,
+                           const float* key_scale, const int32_t* n_valid, const int64_t* q_pos, int stride,
+                           int B, int T, int H, int d, int N, float* scores, void* stream);
+
+/*
+ * ls_topk_select -- exact row-wise top-k of given fp32 scores, bit-exact.
+ * (Packed score-above-inverted-id radix select, "Latent Sparse Attention",
+ * "What the kernels do about the top-p".)
+ *
+ *   scores  row r starts at scores + r*ld (ld >= N)
+ *   n_valid [R] int32 or NULL: columns >= n_valid[r] are not candidates
+ *   idx_out [R][k] int32 column ids (-1 padding);  val_out [R][k] fp32 or NULL
+ * 1 <= k <= 4096.  No workspace.
+ */
+ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int N, int k,
+                         int32_t* idx_out, float* val_out, void* stream);
+
+/*
+ * ls_decode_select -- decode selection: one query per sequence over bf16 keys,
+ * full scan then exact top-k (ls_indexer_score + ls_topk_select fused in one
+ * call).  Shapes as ls_indexer_score with T = 1; outputs [B][k].
+ * Workspace: ls_decode_select_workspace_size(B, N) bytes.
+ */
+size_t ls_decode_select_workspace_size(int B, int N);
+ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid, int B,
+                           int H, int d, int N, int k, int32_t* idx_out, float* val_out, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * ls_prefill_select_stream -- causal top-k for a chunk of prefill queries
+ * against a history that lives in host memory and is streamed through two
+ * alternating device buffers (LeanSparse podcast transcript, 05:36-06:44:
+ * one buffer is scored while the other receives the next part of history).
+ *
+ *   q       [T][H][d] bf16, w [T][H] fp32, q_pos [T] int64 (device)
+ *   hist_k  [N][d] bf16 history keys in PINNED host memory (device memory is
+ *           accepted too); tile j holds keys [j*tile_keys, min(N, (j+1)*tile_keys))
+ *   buf0, buf1 [tile_keys][d] bf16 device buffers, caller-owned, 16-B aligned
+ *   stride  compression stride (4 for CSA); query t sees keys n < (q_pos[t]+1)/stride
+ *   idx_out [T][k] int32, val_out [T][k] fp32 (or NULL)
+ * Copies run on copy_stream and are ordered against the scoring kernels on
+ * compute_stream with events; the outputs are complete when compute_stream
+ * reaches the end of the call.  The call never blocks the host.  The first
+ * copy waits for work already queued on compute_stream (buffers may be in use).
+ * Workspace: ls_prefill_select_workspace_size(T, N) bytes.
+ */
+size_t ls_prefill_select_workspace_size(int T, int N);
+ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int64_t* q_pos, int T, int H, int d,
+                                   const uint16_t* hist_k, int N, int stride, int tile_keys, uint16_t* buf0,
+                                   uint16_t* buf1, int k, int32_t* idx_out, float* val_out, void* ws,
+                                   size_t ws_bytes, void* compute_stream, void* copy_stream);
+
+/*
+ * ls_decode_two_stage_select -- LeanSparse two-stage decode search
+ * (podcast transcript, 07:12-08:00): scan compact keys, keep a shortlist,
+ * fetch the shortlist's original keys and re-rank exactly, keep the top k.
+ *
+ *   q [B][H][d] bf16, w [B][H] fp32
+ *   ck [B][N][d] int8, ck_scale [B][N] fp32      compact keys (coarse pass)
+ *   fk [B][N][d] fp8 e4m3, fk_scale [B][N] fp32  original keys (132 B per key)
+ *   n_valid [B] int32 or NULL
+ *   shortlist  shortlist length S (k <= S <= 4096)
+ *   idx_out [B][k] positions, val_out [B][k] exact scores (or NULL)
+ *   shortlist_out [B][S] int32 or NULL: the shortlist (positions in coarse-score
+ *   order, -1 padding)
+ * Workspace: ls_two_stage_workspace_size(B, N, S) bytes.
+ */
+size_t ls_two_stage_workspace_size(int B, int N, int shortlist);
+ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const int8_t* ck, const float* ck_scale,
+                                     const uint8_t* fk, const float* fk_scale, const int32_t* n_valid, int B,
+                                     int H, int d, int N, int shortlist, int k, int32_t* idx_out, float* val_out,
+                                     int32_t* shortlist_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ls_bucket_select -- LSA-style flat bucket search with indexer-form scoring
+ * ("Latent Sparse Attention", "How LSA finds the keys" and "The method, term
+ * by term", steps 5-6): score every bucket centroid, keep the top_p buckets,
+ * expand them best first into `budget` key positions (members in stored
+ * order, the last bucket cut short), score those keys exactly, keep the top k.
+ *
+ *   q [T][H][d] bf16, w [T][H] fp32
+ *   centroids [P][d] bf16
+ *   bucket_off [P+1] int32, bucket_mem [M] int32   CSR member lists (positions < N)
+ *   keys [N][d] bf16
+ *   top_p <= 4096, k <= budget, k <= 4096
+ *   idx_out [T][k], val_out [T][k] (or NULL), picked_out [T][top_p] or NULL
+ * Workspace: ls_bucket_workspace_size(T, P, top_p, budget) bytes.
+ */
+size_t ls_bucket_workspace_size(int T, int P, int top_p, int budget);
+ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* centroids, const int32_t* bucket_off,
+                           const int32_t* bucket_mem, const uint16_t* keys, int T, int H, int d, int P, int N,
+                           int top_p, int budget, int k, int32_t* idx_out, float* val_out, int32_t* picked_out,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ls_selftest_wait_probe -- failure-detection check: launches a kernel whose
+ * mbarrier is never completed; its bounded wait gives up after limit_ns
+ * nanoseconds, sets LS_FAULT_WAIT_TIMEOUT and returns.  *gave_up_dev (device
+ * int) receives 1 when the wait gave up.  The context stays usable.
+ */
+ls_status ls_selftest_wait_probe(uint64_t limit_ns, int* gave_up_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LS_INDEXER_H */

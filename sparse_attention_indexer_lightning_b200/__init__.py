@@ -1,0 +1,24 @@
+"""B200 (sm_100a) lightning-indexer selection: Python binding of libls_indexer.so.
+
+The binding only marshals arguments (torch tensors for device memory and the
+current CUDA stream) into the library's C ABI (include/ls_indexer.h); every
+step of the selection path runs in the library's CUDA kernels.  Importing the
+package loads the library and raises ImportError if it is missing.
+"""
+
+from ._lib import (  # noqa: F401
+    EXPORTED,
+    LIB_PATH,
+    LSError,
+    ls_bucket_select,
+    ls_decode_select,
+    ls_decode_two_stage_select,
+    ls_device_status,
+    ls_indexer_score,
+    ls_prefill_select_stream,
+    ls_selftest_wait_probe,
+    ls_topk_select,
+    lib,
+)
+
+lib()  # fail loudly at import when the CUDA library is absent

@@ -1,0 +1,285 @@
+"""ctypes binding of libls_indexer.so (the C ABI in include/ls_indexer.h).
+
+Argument marshalling only: the functions below check dtypes, devices and
+shapes of torch tensors, allocate outputs and workspace through torch, and
+call the library on the current CUDA stream.  Every step of the selection path
+runs in the library's kernels; there is no fallback.  Importing this module
+fails loudly when the shared library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libls_indexer.so")
+
+LS_OK = 0
+LS_ERR_INVALID_ARG = 1
+LS_ERR_WORKSPACE = 2
+LS_ERR_UNSUPPORTED = 3
+LS_ERR_CUDA = 4
+LS_ERR_TIMEOUT = 5
+LS_KEY_BF16 = 0
+LS_KEY_FP8_E4M3 = 1
+LS_KEY_INT8 = 2
+LS_FAULT_WAIT_TIMEOUT = 1
+LS_FAULT_BAD_INDEX = 2
+
+EXPORTED = (
+    "ls_last_error", "ls_version", "ls_device_status", "ls_indexer_score", "ls_topk_select",
+    "ls_decode_select_workspace_size", "ls_decode_select", "ls_prefill_select_workspace_size",
+    "ls_prefill_select_stream", "ls_two_stage_workspace_size", "ls_decode_two_stage_select",
+    "ls_bucket_workspace_size", "ls_bucket_select", "ls_selftest_wait_probe",
+)
+
+
+class LSError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"ls status {status}: {msg}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m sparse_attention_indexer_lightning_b200.build`"
+        )
+    lib = ctypes.CDLL(path)
+    P, I, I64, SZ, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
+    sig = {
+        "ls_last_error": (ctypes.c_char_p, []),
+        "ls_version": (I, []),
+        "ls_device_status": (I, [P, P]),
+        "ls_indexer_score": (I, [P, P, P, I, P, P, P, I, I, I, I, I, I, P, P]),
+        "ls_topk_select": (I, [P, I64, P, I, I, I, P, P, P]),
+        "ls_decode_select_workspace_size": (SZ, [I, I]),
+        "ls_decode_select": (I, [P, P, P, P, I, I, I, I, I, P, P, P, SZ, P]),
+        "ls_prefill_select_workspace_size": (SZ, [I, I]),
+        "ls_prefill_select_stream": (I, [P, P, P, I, I, I, P, I, I, I, P, P, I, P, P, P, SZ, P, P]),
+        "ls_two_stage_workspace_size": (SZ, [I, I, I]),
+        "ls_decode_two_stage_select": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P]),
+        "ls_bucket_workspace_size": (SZ, [I, I, I, I]),
+        "ls_bucket_select": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
+        "ls_selftest_wait_probe": (I, [U64, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = load_library()
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != LS_OK:
+        raise LSError(status, lib().ls_last_error().decode(errors="replace"))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None) -> torch.Tensor:
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _opt(t, dtype, name):
+    return None if t is None else _dev(t, dtype, name)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# --------------------------------------------------------------------------- #
+# the library's calls, one Python function per C entry point
+# --------------------------------------------------------------------------- #
+def ls_indexer_score(q, w, keys, key_scale=None, n_valid=None, q_pos=None, stride: int = 4, stream=None):
+    """q [B,T,H,d] bf16, w [B,T,H] f32, keys [B,N,d] (bf16 | float8_e4m3fn | int8) -> scores [B,T,N] f32."""
+    _dev(q, torch.bfloat16, "q", 4)
+    B, T, H, d = q.shape
+    _dev(w, torch.float32, "w", 3)
+    if keys.dtype == torch.bfloat16:
+        kd = LS_KEY_BF16
+    elif keys.dtype == torch.float8_e4m3fn:
+        kd = LS_KEY_FP8_E4M3
+    elif keys.dtype == torch.int8:
+        kd = LS_KEY_INT8
+    else:
+        raise TypeError(f"unsupported key dtype {keys.dtype}")
+    _dev(keys, keys.dtype, "keys", 3)
+    N = keys.shape[1]
+    _opt(key_scale, torch.float32, "key_scale")
+    _opt(n_valid, torch.int32, "n_valid")
+    _opt(q_pos, torch.int64, "q_pos")
+    out = torch.empty((B, T, N), dtype=torch.float32, device=q.device)
+    _check(lib().ls_indexer_score(_ptr(q), _ptr(w), _ptr(keys), kd, _ptr(key_scale), _ptr(n_valid), _ptr(q_pos),
+                                  stride, B, T, H, d, N, _ptr(out), _stream(stream)))
+    return out
+
+
+def ls_topk_select(scores, k: int, n_valid=None, with_values: bool = True, stream=None):
+    """scores [R,N] f32 (row-contiguous) -> (idx [R,k] int32, val [R,k] f32)."""
+    _dev(scores, torch.float32, "scores", 2)
+    R, N = scores.shape
+    _opt(n_valid, torch.int32, "n_valid")
+    idx = torch.empty((R, k), dtype=torch.int32, device=scores.device)
+    val = torch.empty((R, k), dtype=torch.float32, device=scores.device) if with_values else None
+    _check(lib().ls_topk_select(_ptr(scores), N, _ptr(n_valid), R, N, k, _ptr(idx), _ptr(val), _stream(stream)))
+    return idx, val
+
+
+def ls_decode_select(q, w, keys, k: int = 512, n_valid=None, ws=None, out=None, stream=None):
+    """q [B,H,d] bf16, w [B,H] f32, keys [B,N,d] bf16 -> (idx [B,k], val [B,k])."""
+    _dev(q, torch.bfloat16, "q", 3)
+    B, H, d = q.shape
+    _dev(w, torch.float32, "w", 2)
+    _dev(keys, torch.bfloat16, "keys", 3)
+    N = keys.shape[1]
+    _opt(n_valid, torch.int32, "n_valid")
+    need = lib().ls_decode_select_workspace_size(B, N)
+    if ws is None:
+        ws = _workspace(need, q.device)
+    if out is None:
+        out = (torch.empty((B, k), dtype=torch.int32, device=q.device),
+               torch.empty((B, k), dtype=torch.float32, device=q.device))
+    idx, val = out
+    _check(lib().ls_decode_select(_ptr(q), _ptr(w), _ptr(keys), _ptr(n_valid), B, H, d, N, k, _ptr(idx), _ptr(val),
+                                  _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, val
+
+
+def ls_prefill_select_stream(q, w, q_pos, hist_k, buf0, buf1, k: int = 512, stride: int = 4,
+                             tile_keys: Optional[int] = None, ws=None, out=None, copy_stream=None, stream=None):
+    """Causal prefill selection with the history streamed from (pinned) host memory.
+
+    q [T,H,d] bf16, w [T,H] f32, q_pos [T] int64 (device); hist_k [N,d] bf16 in
+    pinned host memory (or on the device); buf0/buf1 [tile_keys, d] bf16 device.
+    """
+    _dev(q, torch.bfloat16, "q", 3)
+    T, H, d = q.shape
+    _dev(w, torch.float32, "w", 2)
+    _dev(q_pos, torch.int64, "q_pos", 1)
+    if hist_k.dtype != torch.bfloat16 or hist_k.dim() != 2 or not hist_k.is_contiguous():
+        raise ValueError("hist_k must be a contiguous [N, d] bf16 tensor")
+    if hist_k.device.type == "cpu" and not hist_k.is_pinned():
+        raise ValueError("hist_k must be in pinned host memory")
+    N = hist_k.shape[0]
+    _dev(buf0, torch.bfloat16, "buf0", 2)
+    _dev(buf1, torch.bfloat16, "buf1", 2)
+    tk = buf0.shape[0] if tile_keys is None else tile_keys
+    if buf0.shape[0] < tk or buf1.shape[0] < tk:
+        raise ValueError("buffers are shorter than tile_keys")
+    need = lib().ls_prefill_select_workspace_size(T, N)
+    if ws is None:
+        ws = _workspace(need, q.device)
+    if out is None:
+        out = (torch.empty((T, k), dtype=torch.int32, device=q.device),
+               torch.empty((T, k), dtype=torch.float32, device=q.device))
+    idx, val = out
+    cs = _stream(stream)
+    xs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
+    _check(lib().ls_prefill_select_stream(_ptr(q), _ptr(w), _ptr(q_pos), T, H, d, _ptr(hist_k), N, stride, tk,
+                                          _ptr(buf0), _ptr(buf1), k, _ptr(idx), _ptr(val), _ptr(ws), ws.numel(),
+                                          cs, xs))
+    return idx, val
+
+
+def ls_decode_two_stage_select(q, w, ck, ck_scale, fk, fk_scale, n_valid=None, shortlist: int = 4096, k: int = 512,
+                               want_shortlist: bool = False, ws=None, out=None, stream=None):
+    """Two-stage decode search. ck int8 [B,N,d] + ck_scale [B,N]; fk e4m3 [B,N,d] + fk_scale [B,N]."""
+    _dev(q, torch.bfloat16, "q", 3)
+    B, H, d = q.shape
+    _dev(w, torch.float32, "w", 2)
+    _dev(ck, torch.int8, "ck", 3)
+    N = ck.shape[1]
+    _dev(ck_scale, torch.float32, "ck_scale", 2)
+    if fk.dtype == torch.uint8:
+        fk = fk.view(torch.float8_e4m3fn)
+    _dev(fk, torch.float8_e4m3fn, "fk", 3)
+    _dev(fk_scale, torch.float32, "fk_scale", 2)
+    _opt(n_valid, torch.int32, "n_valid")
+    need = lib().ls_two_stage_workspace_size(B, N, shortlist)
+    if ws is None:
+        ws = _workspace(need, q.device)
+    if out is None:
+        out = (torch.empty((B, k), dtype=torch.int32, device=q.device),
+               torch.empty((B, k), dtype=torch.float32, device=q.device))
+    idx, val = out
+    sl = torch.empty((B, shortlist), dtype=torch.int32, device=q.device) if want_shortlist else None
+    _check(lib().ls_decode_two_stage_select(_ptr(q), _ptr(w), _ptr(ck), _ptr(ck_scale), _ptr(fk), _ptr(fk_scale),
+                                            _ptr(n_valid), B, H, d, N, shortlist, k, _ptr(idx), _ptr(val), _ptr(sl),
+                                            _ptr(ws), ws.numel(), _stream(stream)))
+    if want_shortlist:
+        return idx, val, sl
+    return idx, val
+
+
+def ls_bucket_select(q, w, centroids, bucket_off, bucket_mem, keys, top_p: int = 64, budget: int = 512,
+                     k: int = 512, want_picked: bool = False, ws=None, out=None, stream=None):
+    """Bucket search. centroids [P,d] bf16, bucket_off [P+1] int32, bucket_mem [M] int32, keys [N,d] bf16."""
+    _dev(q, torch.bfloat16, "q", 3)
+    T, H, d = q.shape
+    _dev(w, torch.float32, "w", 2)
+    _dev(centroids, torch.bfloat16, "centroids", 2)
+    P = centroids.shape[0]
+    _dev(bucket_off, torch.int32, "bucket_off", 1)
+    _dev(bucket_mem, torch.int32, "bucket_mem", 1)
+    _dev(keys, torch.bfloat16, "keys", 2)
+    N = keys.shape[0]
+    need = lib().ls_bucket_workspace_size(T, P, top_p, budget)
+    if ws is None:
+        ws = _workspace(need, q.device)
+    if out is None:
+        out = (torch.empty((T, k), dtype=torch.int32, device=q.device),
+               torch.empty((T, k), dtype=torch.float32, device=q.device))
+    idx, val = out
+    picked = torch.empty((T, top_p), dtype=torch.int32, device=q.device) if want_picked else None
+    _check(lib().ls_bucket_select(_ptr(q), _ptr(w), _ptr(centroids), _ptr(bucket_off), _ptr(bucket_mem), _ptr(keys),
+                                  T, H, d, P, N, top_p, budget, k, _ptr(idx), _ptr(val), _ptr(picked), _ptr(ws),
+                                  ws.numel(), _stream(stream)))
+    if want_picked:
+        return idx, val, picked
+    return idx, val
+
+
+def ls_device_status(stream=None) -> int:
+    """Fault bits of the device fault word (read and cleared).  Raises on none."""
+    flags = ctypes.c_int(0)
+    st = lib().ls_device_status(ctypes.byref(flags), _stream(stream))
+    if st not in (LS_OK, LS_ERR_TIMEOUT, LS_ERR_INVALID_ARG):
+        _check(st)
+    return flags.value
+
+
+def ls_selftest_wait_probe(limit_ns: int, stream=None) -> torch.Tensor:
+    gave_up = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(lib().ls_selftest_wait_probe(limit_ns, _ptr(gave_up), _stream(stream)))
+    return gave_up

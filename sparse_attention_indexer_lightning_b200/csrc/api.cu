@@ -1,0 +1,441 @@
+// C ABI of the lightning-indexer selection library: argument checks,
+// workspace carving, TMA descriptor set-up and the launch sequence of each
+// search.  Every step of the path runs in the kernels of this library.
+//
+// The library is built as this single translation unit; the kernel headers
+// (score_tc.cuh, score_cvt.cuh, topk.cuh, misc.cuh) are included below.
+
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+#include "ls_indexer.h"
+#include "misc.cuh"
+#include "score_cvt.cuh"
+#include "score_tc.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using namespace lsi;
+
+thread_local char g_err[512] = "";
+
+ls_status fail(ls_status code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define LS_CHECK_ARG(cond, ...) \
+  do {                          \
+    if (!(cond)) return fail(LS_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define LS_CUDA(expr)                                                                               \
+  do {                                                                                              \
+    cudaError_t e_ = (expr);                                                                        \
+    if (e_ != cudaSuccess) return fail(LS_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_));      \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+int num_sms_current() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over [rows][128], box = 64 columns x box_rows, 128-byte swizzle.
+ls_status make_bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim * 2)};
+  cuuint32_t box[2] = {64u, box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LS_OK;
+}
+
+ls_status check_shape(int H, int d) {
+  if (H != kHeads || d != kDim)
+    return fail(LS_ERR_UNSUPPORTED, "only H=%d, d=%d are built (got H=%d, d=%d)", kHeads, kDim, H, d);
+  return LS_OK;
+}
+
+cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Scores of bf16 keys on the tensor cores (the TMA path).
+ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid,
+                     const int64_t* q_pos, int stride, int B, int T, int N, int key_base, int n_total, float* out,
+                     int64_t ld_out, cudaStream_t st) {
+  if (B == 0 || T == 0 || N == 0) return LS_OK;
+  const int qg = (T == 1) ? 1 : 8;
+  CUtensorMap kmap, qmap;
+  ls_status s = make_bf16_map(&kmap, keys, static_cast<uint64_t>(B) * N, kTileKeys);
+  if (s != LS_OK) return s;
+  s = make_bf16_map(&qmap, q, static_cast<uint64_t>(B) * T * kHeads, qg * kHeads);
+  if (s != LS_OK) return s;
+  ScoreParams p;
+  p.w = w;
+  p.n_valid = n_valid;
+  p.q_pos = q_pos;
+  p.out = out;
+  p.ld_out = ld_out;
+  p.stride = stride;
+  p.B = B;
+  p.T = T;
+  p.N = N;
+  p.key_base = key_base;
+  p.n_total = n_total;
+  LS_CUDA(launch_score_tc(qg, &kmap, &qmap, p, num_sms_current(), st));
+  return LS_OK;
+}
+
+ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_total, const float* w,
+                        const void* keys, const float* scale, const int32_t* rows, const int32_t* n_valid,
+                        int64_t key_rows, int64_t key_stride, int B, int N, int fmt, float* out, cudaStream_t st) {
+  if (B == 0 || N == 0) return LS_OK;
+  CUtensorMap qmap;
+  ls_status s = make_bf16_map(&qmap, q, static_cast<uint64_t>(q_rows_total), kHeads);
+  if (s != LS_OK) return s;
+  CvtParams p;
+  p.keys = keys;
+  p.scale = scale;
+  p.rows = rows;
+  p.n_valid = n_valid;
+  p.w = w;
+  p.out = out;
+  p.key_rows = key_rows;
+  p.key_stride = key_stride;
+  p.q_row_stride = q_row_stride;
+  p.B = B;
+  p.N = N;
+  p.fmt = fmt;
+  LS_CUDA(launch_score_cvt(&qmap, p, num_sms_current(), st));
+  return LS_OK;
+}
+
+ls_status topk(const float* scores, int64_t ld, const int32_t* n_valid, const int32_t* labels, int64_t ld_labels,
+               int R, int N, int k, int32_t* idx, float* val, int64_t ld_out, cudaStream_t st) {
+  TopkParams p;
+  p.scores = scores;
+  p.ld = ld;
+  p.n_valid = n_valid;
+  p.labels = labels;
+  p.ld_labels = ld_labels;
+  p.R = R;
+  p.N = N;
+  p.k = k;
+  p.idx_out = idx;
+  p.val_out = val;
+  p.ld_out = ld_out;
+  LS_CUDA(launch_topk(p, st));
+  return LS_OK;
+}
+
+struct Carver {
+  uint8_t* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    T* p = reinterpret_cast<T*>(base ? base + used : nullptr);
+    used += align_up(count * sizeof(T));
+    return p;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* ls_last_error(void) { return g_err; }
+
+int ls_version(void) { return 100; }
+
+ls_status ls_device_status(int* flags, void* stream) {
+  int h = 0;
+  const int e = read_and_clear_fault(S(stream), &h);
+  if (e != 0) return fail(LS_ERR_CUDA, "reading the fault word: %s", cudaGetErrorString(static_cast<cudaError_t>(e)));
+  if (flags) *flags = h;
+  if (h & FAULT_WAIT_TIMEOUT) return fail(LS_ERR_TIMEOUT, "a device wait exceeded its time limit");
+  if (h & FAULT_BAD_INDEX) return fail(LS_ERR_INVALID_ARG, "a gathered row id was outside the key array");
+  return LS_OK;
+}
+
+ls_status ls_indexer_score(const uint16_t* q, const float* w, const void* keys, int key_dtype,
+                           const float* key_scale, const int32_t* n_valid, const int64_t* q_pos, int stride,
+                           int B, int T, int H, int d, int N, float* scores, void* stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(B >= 0 && T >= 0 && N >= 0, "negative size (B=%d T=%d N=%d)", B, T, N);
+  if (B == 0 || T == 0 || N == 0) return LS_OK;
+  LS_CHECK_ARG(q && w && keys && scores, "null tensor pointer");
+  LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(keys), "q, w and keys must be 16-byte aligned");
+  LS_CHECK_ARG(q_pos == nullptr || stride >= 1, "stride must be >= 1 with q_pos");
+  if (key_dtype == LS_KEY_BF16) {
+    return score_bf16(q, w, static_cast<const uint16_t*>(keys), n_valid, q_pos, stride, B, T, N, 0, N, scores, N,
+                      S(stream));
+  }
+  LS_CHECK_ARG(key_dtype == LS_KEY_FP8_E4M3 || key_dtype == LS_KEY_INT8, "unknown key_dtype %d", key_dtype);
+  LS_CHECK_ARG(key_scale != nullptr, "FP8/INT8 keys need key_scale");
+  if (T != 1 || q_pos != nullptr)
+    return fail(LS_ERR_UNSUPPORTED, "FP8/INT8 keys are built for one query per sequence without q_pos");
+  return score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, keys, key_scale, nullptr, n_valid, N, N, B, N,
+                       key_dtype == LS_KEY_INT8 ? SRC_INT8 : SRC_E4M3, scores, S(stream));
+}
+
+ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int N, int k,
+                         int32_t* idx_out, float* val_out, void* stream) {
+  LS_CHECK_ARG(R >= 0 && N >= 0, "negative size");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  LS_CHECK_ARG(ld >= N, "ld (%lld) < N (%d)", static_cast<long long>(ld), N);
+  if (R == 0) return LS_OK;
+  LS_CHECK_ARG(idx_out && (scores || N == 0), "null tensor pointer");
+  return topk(scores, ld, n_valid, nullptr, 0, R, N, k, idx_out, val_out, k, S(stream));
+}
+
+size_t ls_decode_select_workspace_size(int B, int N) {
+  if (B <= 0 || N <= 0) return 0;
+  return align_up(static_cast<size_t>(B) * N * sizeof(float));
+}
+
+ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid, int B,
+                           int H, int d, int N, int k, int32_t* idx_out, float* val_out, void* ws,
+                           size_t ws_bytes, void* stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(B >= 0 && N >= 0, "negative size");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  if (B == 0) return LS_OK;
+  LS_CHECK_ARG(idx_out != nullptr, "null idx_out");
+  const size_t need = ls_decode_select_workspace_size(B, N);
+  if (ws_bytes < need || (need && !ws))
+    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  float* sc = static_cast<float*>(ws);
+  if (N > 0) {
+    LS_CHECK_ARG(q && w && keys, "null tensor pointer");
+    LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(keys), "q, w and keys must be 16-byte aligned");
+    s = score_bf16(q, w, keys, n_valid, nullptr, 1, B, 1, N, 0, N, sc, N, S(stream));
+    if (s != LS_OK) return s;
+  }
+  return topk(sc, N, n_valid, nullptr, 0, B, N, k, idx_out, val_out, k, S(stream));
+}
+
+size_t ls_prefill_select_workspace_size(int T, int N) {
+  if (T <= 0 || N <= 0) return 0;
+  return align_up(static_cast<size_t>(T) * N * sizeof(float)) + align_up(static_cast<size_t>(T) * sizeof(int32_t));
+}
+
+ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int64_t* q_pos, int T, int H, int d,
+                                   const uint16_t* hist_k, int N, int stride, int tile_keys, uint16_t* buf0,
+                                   uint16_t* buf1, int k, int32_t* idx_out, float* val_out, void* ws,
+                                   size_t ws_bytes, void* compute_stream, void* copy_stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(T >= 0 && N >= 0, "negative size");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  LS_CHECK_ARG(stride >= 1, "stride must be >= 1");
+  LS_CHECK_ARG(tile_keys >= 1, "tile_keys must be >= 1");
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(q && w && q_pos && idx_out, "null tensor pointer");
+  LS_CHECK_ARG(aligned16(q) && aligned16(w), "q and w must be 16-byte aligned");
+  const size_t need = ls_prefill_select_workspace_size(T, N);
+  if (ws_bytes < need || (need && !ws))
+    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  Carver cv(ws);
+  float* sc = cv.take<float>(static_cast<size_t>(T) * N);
+  int32_t* counts = cv.take<int32_t>(T);
+  cudaStream_t cs = S(compute_stream);
+  cudaStream_t xs = copy_stream ? S(copy_stream) : cs;
+  if (N > 0) {
+    LS_CHECK_ARG(hist_k && buf0 && buf1, "null history or buffer pointer");
+    LS_CHECK_ARG(aligned16(buf0) && aligned16(buf1) && aligned16(hist_k), "history and buffers must be 16-byte aligned");
+    cudaPointerAttributes attr;
+    LS_CUDA(cudaPointerGetAttributes(&attr, hist_k));
+    LS_CHECK_ARG(attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeDevice ||
+                     attr.type == cudaMemoryTypeManaged,
+                 "hist_k must be pinned host memory or device memory (pageable memory cannot be streamed)");
+    uint16_t* bufs[2] = {buf0, buf1};
+    cudaEvent_t start_ev, copied[2], freed[2];
+    LS_CUDA(cudaEventCreateWithFlags(&start_ev, cudaEventDisableTiming));
+    for (int i = 0; i < 2; ++i) {
+      LS_CUDA(cudaEventCreateWithFlags(&copied[i], cudaEventDisableTiming));
+      LS_CUDA(cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming));
+    }
+    ls_status st = LS_OK;
+    // Earlier work on the compute stream may still read the buffers.
+    cudaError_t e = cudaEventRecord(start_ev, cs);
+    if (e == cudaSuccess && xs != cs) e = cudaStreamWaitEvent(xs, start_ev, 0);
+    const int ntiles = (N + tile_keys - 1) / tile_keys;
+    for (int j = 0; j < ntiles && e == cudaSuccess && st == LS_OK; ++j) {
+      const int slot = j & 1;
+      const int k0 = j * tile_keys;
+      const int len = (N - k0 < tile_keys) ? (N - k0) : tile_keys;
+      if (j >= 2 && xs != cs) e = cudaStreamWaitEvent(xs, freed[slot], 0);
+      if (e != cudaSuccess) break;
+      e = cudaMemcpyAsync(bufs[slot], hist_k + static_cast<size_t>(k0) * kDim,
+                          static_cast<size_t>(len) * kDim * sizeof(uint16_t), cudaMemcpyDefault, xs);
+      if (e != cudaSuccess) break;
+      if (xs != cs) {
+        e = cudaEventRecord(copied[slot], xs);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, copied[slot], 0);
+        if (e != cudaSuccess) break;
+      }
+      st = score_bf16(q, w, bufs[slot], nullptr, q_pos, stride, 1, T, len, k0, N, sc, N, cs);
+      if (st != LS_OK) break;
+      if (xs != cs) e = cudaEventRecord(freed[slot], cs);
+    }
+    // The copy stream must not run ahead of this call's last kernels.
+    if (e == cudaSuccess && st == LS_OK && xs != cs) {
+      e = cudaEventRecord(start_ev, cs);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(xs, start_ev, 0);
+    }
+    cudaEventDestroy(start_ev);
+    for (int i = 0; i < 2; ++i) {
+      cudaEventDestroy(copied[i]);
+      cudaEventDestroy(freed[i]);
+    }
+    if (st != LS_OK) return st;
+    if (e != cudaSuccess) return fail(LS_ERR_CUDA, "history streaming: %s", cudaGetErrorString(e));
+  }
+  LS_CUDA(launch_causal_counts(q_pos, T, stride, N, counts, cs));
+  return topk(sc, N, counts, nullptr, 0, T, N, k, idx_out, val_out, k, cs);
+}
+
+size_t ls_two_stage_workspace_size(int B, int N, int shortlist) {
+  if (B <= 0 || N <= 0 || shortlist <= 0) return 0;
+  return align_up(static_cast<size_t>(B) * N * sizeof(float)) +
+         align_up(static_cast<size_t>(B) * shortlist * sizeof(int32_t)) +
+         align_up(static_cast<size_t>(B) * shortlist * sizeof(float));
+}
+
+ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const int8_t* ck, const float* ck_scale,
+                                     const uint8_t* fk, const float* fk_scale, const int32_t* n_valid, int B,
+                                     int H, int d, int N, int shortlist, int k, int32_t* idx_out, float* val_out,
+                                     int32_t* shortlist_out, void* ws, size_t ws_bytes, void* stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(B >= 0 && N >= 0, "negative size");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  LS_CHECK_ARG(shortlist >= k && shortlist <= kMaxTopK, "shortlist must be in [k, %d] (got %d)", kMaxTopK,
+               shortlist);
+  if (B == 0) return LS_OK;
+  LS_CHECK_ARG(idx_out != nullptr, "null idx_out");
+  const size_t need = ls_two_stage_workspace_size(B, N, shortlist);
+  if (ws_bytes < need || (need && !ws))
+    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  Carver cv(ws);
+  float* s_hat = cv.take<float>(static_cast<size_t>(B) * N);
+  int32_t* short_ws = cv.take<int32_t>(static_cast<size_t>(B) * shortlist);
+  float* exact = cv.take<float>(static_cast<size_t>(B) * shortlist);
+  int32_t* sl = shortlist_out ? shortlist_out : short_ws;
+  cudaStream_t st = S(stream);
+  if (N > 0) {
+    LS_CHECK_ARG(q && w && ck && ck_scale && fk && fk_scale, "null tensor pointer");
+    LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(ck) && aligned16(fk) && aligned16(ck_scale) &&
+                     aligned16(fk_scale),
+                 "tensors must be 16-byte aligned");
+    // coarse pass over compact keys
+    s = score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, ck, ck_scale, nullptr, n_valid, N, N, B, N,
+                      SRC_INT8, s_hat, st);
+    if (s != LS_OK) return s;
+  }
+  // shortlist: top-S positions by coarse score
+  s = topk(s_hat, N, n_valid, nullptr, 0, B, N, shortlist, sl, nullptr, shortlist, st);
+  if (s != LS_OK) return s;
+  if (N > 0) {
+    // exact re-rank: gather the shortlist's fp8 keys, score with the full query
+    s = score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, fk, fk_scale, sl, nullptr, N, N, B, shortlist,
+                      SRC_E4M3, exact, st);
+    if (s != LS_OK) return s;
+  }
+  return topk(exact, shortlist, nullptr, sl, shortlist, B, shortlist, k, idx_out, val_out, k, st);
+}
+
+size_t ls_bucket_workspace_size(int T, int P, int top_p, int budget) {
+  if (T <= 0 || P <= 0 || top_p <= 0 || budget <= 0) return 0;
+  return align_up(static_cast<size_t>(T) * P * sizeof(float)) +
+         align_up(static_cast<size_t>(T) * top_p * sizeof(int32_t)) +
+         align_up(static_cast<size_t>(T) * budget * sizeof(int32_t)) +
+         align_up(static_cast<size_t>(T) * budget * sizeof(float));
+}
+
+ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* centroids, const int32_t* bucket_off,
+                           const int32_t* bucket_mem, const uint16_t* keys, int T, int H, int d, int P, int N,
+                           int top_p, int budget, int k, int32_t* idx_out, float* val_out, int32_t* picked_out,
+                           void* ws, size_t ws_bytes, void* stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(T >= 0 && P >= 0 && N >= 0, "negative size");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  LS_CHECK_ARG(top_p >= 1 && top_p <= kMaxTopK, "top_p must be in [1, %d] (got %d)", kMaxTopK, top_p);
+  LS_CHECK_ARG(budget >= k, "budget (%d) must be >= k (%d)", budget, k);
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(idx_out != nullptr, "null idx_out");
+  const size_t need = ls_bucket_workspace_size(T, P, top_p, budget);
+  if (ws_bytes < need || (need && !ws))
+    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  Carver cv(ws);
+  float* cscore = cv.take<float>(static_cast<size_t>(T) * P);
+  int32_t* picked_ws = cv.take<int32_t>(static_cast<size_t>(T) * top_p);
+  int32_t* cand = cv.take<int32_t>(static_cast<size_t>(T) * budget);
+  float* exact = cv.take<float>(static_cast<size_t>(T) * budget);
+  int32_t* picked = picked_out ? picked_out : picked_ws;
+  cudaStream_t st = S(stream);
+  if (P > 0) {
+    LS_CHECK_ARG(q && w && centroids && bucket_off && bucket_mem, "null tensor pointer");
+    LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(centroids), "q, w and centroids must be 16-byte aligned");
+    s = score_bf16(q, w, centroids, nullptr, nullptr, 1, 1, T, P, 0, P, cscore, P, st);
+    if (s != LS_OK) return s;
+  }
+  s = topk(cscore, P, nullptr, nullptr, 0, T, P, top_p, picked, nullptr, top_p, st);
+  if (s != LS_OK) return s;
+  LS_CUDA(launch_expand(picked, T, top_p, bucket_off, bucket_mem, P, budget, cand, st));
+  if (N > 0) {
+    LS_CHECK_ARG(keys && aligned16(keys), "keys must be a 16-byte aligned device pointer");
+    s = score_convert(q, kHeads, static_cast<int64_t>(T) * kHeads, w, keys, nullptr, cand, nullptr, N, 0, T, budget,
+                      SRC_BF16, exact, st);
+    if (s != LS_OK) return s;
+  }
+  return topk(exact, budget, nullptr, cand, budget, T, budget, k, idx_out, val_out, k, st);
+}
+
+ls_status ls_selftest_wait_probe(uint64_t limit_ns, int* gave_up_dev, void* stream) {
+  LS_CHECK_ARG(gave_up_dev != nullptr, "null output");
+  LS_CUDA(launch_wait_probe(limit_ns, gave_up_dev, S(stream)));
+  return LS_OK;
+}
+
+}  // extern "C"

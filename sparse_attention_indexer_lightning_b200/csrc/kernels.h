@@ -1,0 +1,91 @@
+// Internal launchers shared between the kernel files and the C-ABI layer.
+// Nothing here is exported from the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lsi {
+
+constexpr int kHeads = 32;   // indexer heads built
+constexpr int kDim = 128;    // indexer key / query width
+constexpr int kTileKeys = 128;
+constexpr int kMaxTopK = 4096;
+
+// ---------------------------------------------------------------- scoring
+// Tensor-core scoring of bf16 keys read by TMA.  One launch covers B
+// sequences, T queries per sequence and N keys per sequence (keys of sequence
+// b are rows b*N .. b*N+N-1 of the key tensor map).
+//   out[(b*T + t)*ld_out + key_base + n] = sum_h w[b,t,h] * relu(q[b,t,h] . k[b,n])
+// or -inf where the key is masked: n >= n_valid[b] (when given) or, with
+// q_pos, key_base + n >= (q_pos[b,t] + 1) / stride (block-complete causal rule),
+// capped at n_total.
+struct ScoreParams {
+  const float* w;          // [B][T][H]
+  const int32_t* n_valid;  // [B] or nullptr
+  const int64_t* q_pos;    // [B][T] or nullptr
+  float* out;
+  int64_t ld_out;
+  int stride;
+  int B, T, N;
+  int key_base;
+  int n_total;             // causal cap: number of keys of the whole history
+};
+
+// qg = queries sharing one MMA B tile: 1 (one query per sequence) or 8.
+cudaError_t launch_score_tc(int qg, const CUtensorMap* kmap, const CUtensorMap* qmap,
+                            const ScoreParams& p, int num_sms, cudaStream_t st);
+
+// Source rows for the converting scorer.
+enum SrcFormat : int { SRC_INT8 = 0, SRC_E4M3 = 1, SRC_BF16 = 2 };
+
+// Scoring of keys that are either int8 / fp8 e4m3 codes with a per-key fp32
+// scale, or gathered bf16 rows.  Row j of problem b is key
+//   rows == nullptr : b*N + j                      (contiguous)
+//   rows != nullptr : b*key_stride + rows[b*N + j] (gathered; < 0 = padding)
+//   out[b*N + j] = sum_h w[b,h] * relu(scale * (q[b,h] . code))   (or -inf)
+struct CvtParams {
+  const void* keys;        // base of the key rows
+  const float* scale;      // per-key scale, indexed like the key rows (nullptr for bf16)
+  const int32_t* rows;     // [B][N] gathered row ids or nullptr
+  const int32_t* n_valid;  // [B] or nullptr (contiguous form only)
+  const float* w;          // [B][H]
+  float* out;              // [B][N]
+  int64_t key_rows;        // gathered form: valid row ids are [0, key_rows)
+  int64_t key_stride;      // gathered form: row offset of problem b is b*key_stride
+  int64_t q_row_stride;    // q rows per problem (H for one query per problem)
+  int B, N;
+  int fmt;
+};
+cudaError_t launch_score_cvt(const CUtensorMap* qmap, const CvtParams& p, int num_sms, cudaStream_t st);
+
+// ---------------------------------------------------------------- top-k
+// Row-wise top-k by (value desc, label asc); labels default to the column.
+struct TopkParams {
+  const float* scores;     // row r starts at scores + r*ld
+  int64_t ld;
+  const int32_t* n_valid;  // [R] or nullptr: columns >= n_valid[r] are absent
+  const int32_t* labels;   // [R][ld_labels] or nullptr; label < 0 = absent
+  int64_t ld_labels;
+  int R, N, k;
+  int32_t* idx_out;        // [R][k] labels, -1 padding
+  float* val_out;          // [R][k] values (bit copies), -inf padding; may be nullptr
+  int64_t ld_out;
+};
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t st);
+
+// ---------------------------------------------------------------- misc
+// n_valid[t] = clamp((q_pos[t] + 1) / stride, 0, n_total)
+cudaError_t launch_causal_counts(const int64_t* q_pos, int T, int stride, int n_total, int32_t* out,
+                                 cudaStream_t st);
+
+// Best-first bucket expansion: members of picked[t][0..top_p) in order until
+// budget positions are held; cand[t][budget] padded with -1.
+cudaError_t launch_expand(const int32_t* picked, int T, int top_p, const int32_t* off, const int32_t* mem,
+                          int P, int budget, int32_t* cand, cudaStream_t st);
+
+int read_and_clear_fault(cudaStream_t st, int* flags);
+cudaError_t launch_wait_probe(uint64_t limit_ns, int* waited, cudaStream_t st);
+
+}  // namespace lsi

@@ -1,0 +1,420 @@
+// Indexer scoring of keys that need converting before the tensor cores:
+//   * int8 compact keys with a per-key fp32 scale (the coarse pass of the
+//     two-stage decode search, LeanSparse podcast transcript 07:12-07:34),
+//   * fp8 e4m3 keys with a per-key fp32 scale, gathered by shortlist id (the
+//     exact re-rank, same transcript 07:34-08:00; the 128 B key + 4 B scale
+//     entry of "03 long context", "The Architectural Answer: Read Less of the
+//     Past"),
+//   * bf16 keys gathered by position (the exact rescore after bucket
+//     expansion, "Latent Sparse Attention", "The method, term by term").
+//
+//   score = sum_h w[h] * max(0, scale * (q[h] . code))
+//
+// Both 8-bit formats widen to bf16 exactly (int8 magnitudes <= 128 and e4m3
+// values fit bf16's 8-bit significand and exponent range), so the contraction
+// runs as a bf16 x bf16 -> fp32 tcgen05 MMA with one key per TMEM lane.
+//
+// Roles (320 threads, one persistent CTA per SM):
+//   warp 0      producer: 1-D bulk copies of raw rows (one copy per tile when
+//               contiguous, one per row when gathered) + TMA of the query tile
+//   warp 1      TMEM allocator + single-thread MMA issuer
+//   warps 2-5   converters: raw rows -> bf16 in the 128-byte-swizzled K-major
+//               layout the MMA descriptor expects
+//   warps 6-9   epilogue: scale, ReLU, head weights, head sum, store
+// All waits are bounded (see common.cuh).
+
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lsi {
+
+template <int FMT>
+struct CvtCfg {
+  static constexpr int BM = kTileKeys;
+  static constexpr int BN = kHeads;                       // one query per problem
+  static constexpr int ROW_BYTES = (FMT == SRC_BF16) ? 256 : 128;
+  static constexpr int RAW_BYTES = BM * ROW_BYTES;
+  static constexpr int A_BYTES = BM * kDim * 2;
+  static constexpr int A_HALF = BM * 64 * 2;
+  static constexpr int B_BYTES = BN * kDim * 2;
+  static constexpr int B_HALF = BN * 64 * 2;
+  static constexpr int RS = (FMT == SRC_BF16) ? 3 : 6;   // raw stages
+  static constexpr int AS = 3;                            // converted stages
+  static constexpr int ACC = 2;
+  static constexpr int TMEM_COLS = 64;
+  static constexpr int CVT_WARPS = 4;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int THREADS = (2 + CVT_WARPS + EPI_WARPS) * 32;
+  static constexpr size_t SMEM_RAW = size_t(RS) * RAW_BYTES;
+  static constexpr size_t SMEM_A = size_t(AS) * A_BYTES;
+  static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
+  static constexpr size_t SMEM_BAR = 512;
+  static constexpr size_t SMEM_TOTAL = 1024 + SMEM_RAW + SMEM_A + SMEM_B + SMEM_BAR;
+  static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
+};
+
+struct CvtBarriers {
+  uint64_t rfull[8];
+  uint64_t rempty[8];
+  uint64_t afull[4];
+  uint64_t aempty[4];
+  uint64_t bfull[2];
+  uint64_t bempty[2];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(CvtBarriers) <= 512, "barrier block");
+
+__device__ __forceinline__ void cvt_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > LSI_WAIT_LIMIT_NS) {
+      atomicOr(&g_fault, FAULT_WAIT_TIMEOUT);
+      return;
+    }
+  }
+}
+
+// 4 signed bytes -> 4 exact floats via the 2^23 magic number.
+__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  const uint32_t y = x ^ 0x80808080u;  // bias to unsigned: byte = v + 128
+  const float f0 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7540)) - 8388736.f;
+  const float f1 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7541)) - 8388736.f;
+  const float f2 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7542)) - 8388736.f;
+  const float f3 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7543)) - 8388736.f;
+  __nv_bfloat162 a = __floats2bfloat162_rn(f0, f1);
+  __nv_bfloat162 b = __floats2bfloat162_rn(f2, f3);
+  lo = *reinterpret_cast<uint32_t*>(&a);
+  hi = *reinterpret_cast<uint32_t*>(&b);
+}
+
+// 2 e4m3 codes (low 16 bits of x, element 0 in the low byte) -> bf16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t x) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(x));
+  __half2 h = *reinterpret_cast<__half2*>(&h2);
+  const float2 f = __half22float2(h);
+  __nv_bfloat162 r = __float22bfloat162_rn(f);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  lo = e4m3x2_to_bf16x2(x & 0xFFFFu);
+  hi = e4m3x2_to_bf16x2(x >> 16);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
+    score_cvt_kernel(const __grid_constant__ CUtensorMap qmap, const CvtParams p) {
+  using C = CvtCfg<FMT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sR = smem;
+  uint8_t* sA = smem + C::SMEM_RAW;
+  uint8_t* sB = sA + C::SMEM_A;
+  CvtBarriers* bars = reinterpret_cast<CvtBarriers*>(sB + C::SMEM_B);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int NT = (p.N + C::BM - 1) / C::BM;
+  const long long units = static_cast<long long>(p.B) * NT;
+  const long long u_begin = units * blockIdx.x / gridDim.x;
+  const long long u_end = units * (blockIdx.x + 1) / gridDim.x;
+  const uint8_t* keys = static_cast<const uint8_t*>(p.keys);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::RS; ++s) {
+      mbar_init(&bars->rfull[s], 1);
+      mbar_init(&bars->rempty[s], C::CVT_WARPS);
+    }
+    for (int s = 0; s < C::AS; ++s) {
+      mbar_init(&bars->afull[s], C::CVT_WARPS);
+      mbar_init(&bars->aempty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->bfull[s], 1);
+      mbar_init(&bars->bempty[s], 1);
+      mbar_init(&bars->tfull[s], 1);
+      mbar_init(&bars->tempty[s], C::EPI_WARPS);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&qmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int rs = 0;
+    uint32_t rphase = 0;
+    int prev_b = -1;
+    int bslot = 1;
+    uint32_t bphase[2] = {0, 0};
+    int issued[8];
+    uint32_t issued_par[8];
+    for (int s = 0; s < 8; ++s) issued[s] = 0, issued_par[s] = 0;
+    int b_issued[2] = {0, 0};
+    uint32_t b_par[2] = {0, 0};
+    bool ok = true;
+    for (long long u = u_begin; u < u_end; ++u) {
+      const int tile = static_cast<int>(u % NT);
+      const int b = static_cast<int>(u / NT);
+      if (b != prev_b) {
+        bslot ^= 1;
+        if (!mbar_wait(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
+        b_par[bslot] = bphase[bslot];
+        b_issued[bslot] = 1;
+        bphase[bslot] ^= 1;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars->bfull[bslot], C::B_BYTES);
+          const int qrow = static_cast<int>(static_cast<int64_t>(b) * p.q_row_stride);
+          uint8_t* dst = sB + bslot * C::B_BYTES;
+          tma_load_2d(dst, &qmap, &bars->bfull[bslot], 0, qrow);
+          tma_load_2d(dst + C::B_HALF, &qmap, &bars->bfull[bslot], 64, qrow);
+        }
+        prev_b = b;
+      }
+      if (!mbar_wait(&bars->rempty[rs], rphase ^ 1, abort_flag)) { ok = false; break; }
+      uint8_t* dst = sR + rs * C::RAW_BYTES;
+      const int j0 = tile * C::BM;
+      const int nrows = min(C::BM, p.N - j0);
+      if (p.rows == nullptr) {
+        if (lane == 0) {
+          const uint32_t bytes = static_cast<uint32_t>(nrows) * C::ROW_BYTES;
+          mbar_arrive_expect_tx(&bars->rfull[rs], bytes);
+          const uint8_t* src = keys + (static_cast<int64_t>(b) * p.N + j0) * C::ROW_BYTES;
+          bulk_load(dst, src, bytes, &bars->rfull[rs]);
+        }
+      } else {
+        // gathered: lane l copies rows l, l+32, l+64, l+96 of the tile
+        int32_t rid[4];
+        int cnt = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = j0 + lane + 32 * i;
+          int32_t r = -1;
+          if (j < p.N) r = p.rows[static_cast<int64_t>(b) * p.N + j];
+          if (r >= p.key_rows) {
+            atomicOr(&g_fault, FAULT_BAD_INDEX);
+            r = -1;
+          }
+          rid[i] = r;
+          cnt += (r >= 0);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0) mbar_arrive_expect_tx(&bars->rfull[rs], static_cast<uint32_t>(cnt) * C::ROW_BYTES);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (rid[i] >= 0) {
+            const uint8_t* src = keys + (static_cast<int64_t>(b) * p.key_stride + rid[i]) * C::ROW_BYTES;
+            bulk_load(dst + (lane + 32 * i) * C::ROW_BYTES, src, C::ROW_BYTES, &bars->rfull[rs]);
+          }
+        }
+      }
+      issued[rs] = 1;
+      issued_par[rs] = rphase;
+      if (++rs == C::RS) { rs = 0; rphase ^= 1; }
+    }
+    if (!ok && lane == 0) {
+      for (int s = 0; s < C::RS; ++s)
+        if (issued[s]) cvt_wait_drain(&bars->rfull[s], issued_par[s]);
+      for (int s = 0; s < 2; ++s)
+        if (b_issued[s]) cvt_wait_drain(&bars->bfull[s], b_par[s]);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::BN);
+      int as = 0;
+      uint32_t aphase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      int prev_b = -1;
+      int bslot = 1;
+      uint32_t bphase[2] = {0, 0};
+      const uint32_t a_base = smem_u32(sA);
+      const uint32_t b_base = smem_u32(sB);
+      for (long long u = u_begin; u < u_end; ++u) {
+        const int b = static_cast<int>(u / NT);
+        if (b != prev_b) {
+          if (prev_b >= 0) umma_commit(&bars->bempty[bslot]);
+          bslot ^= 1;
+          if (!mbar_wait(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
+          bphase[bslot] ^= 1;
+          prev_b = b;
+        }
+        if (!mbar_wait(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
+        tc_fence_after();
+        if (!mbar_wait(&bars->afull[as], aphase, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_addr = a_base + as * C::A_BYTES;
+        const uint32_t b_addr = b_base + bslot * C::B_BYTES;
+        const uint32_t d_tmem = tmem_base + acc * C::BN;
+#pragma unroll
+        for (int kk = 0; kk < kDim / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          const uint64_t adesc = sw128_kmajor_desc(a_addr + (kk >> 2) * C::A_HALF + koff);
+          const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + koff);
+          umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->aempty[as]);
+        umma_commit(&bars->tfull[acc]);
+        if (++as == C::AS) { as = 0; aphase ^= 1; }
+        if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
+      }
+      umma_commit(&bars->drain);
+      cvt_wait_drain(&bars->drain, 0);
+    }
+  } else if (warp < 2 + C::CVT_WARPS) {
+    // ------------------------------------------------------------ converters
+    const int ct = threadIdx.x - 64;  // 0..127
+    int rs = 0, as = 0;
+    uint32_t rphase = 0, aphase = 0;
+    for (long long u = u_begin; u < u_end; ++u) {
+      if (!mbar_wait(&bars->rfull[rs], rphase, abort_flag)) break;
+      if (!mbar_wait(&bars->aempty[as], aphase ^ 1, abort_flag)) break;
+      const uint8_t* raw = sR + rs * C::RAW_BYTES;
+      uint8_t* a = sA + as * C::A_BYTES;
+      if (FMT == SRC_BF16) {
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int id = i * 128 + ct;
+          const int row = id >> 4, cc = id & 15;
+          const uint4 v = *reinterpret_cast<const uint4*>(raw + row * 256 + cc * 16);
+          const int panel = cc >> 3, j = cc & 7;
+          *reinterpret_cast<uint4*>(a + panel * C::A_HALF + row * 128 + ((j ^ (row & 7)) << 4)) = v;
+        }
+      } else {
+#pragma unroll 2
+        for (int i = 0; i < 8; ++i) {
+          const int id = i * 128 + ct;
+          const int row = id >> 3, cc = id & 7;
+          const uint4 v = *reinterpret_cast<const uint4*>(raw + row * 128 + cc * 16);
+          uint4 o0, o1;
+          if (FMT == SRC_INT8) {
+            i8x4_to_bf16x4(v.x, o0.x, o0.y);
+            i8x4_to_bf16x4(v.y, o0.z, o0.w);
+            i8x4_to_bf16x4(v.z, o1.x, o1.y);
+            i8x4_to_bf16x4(v.w, o1.z, o1.w);
+          } else {
+            e4m3x4_to_bf16x4(v.x, o0.x, o0.y);
+            e4m3x4_to_bf16x4(v.y, o0.z, o0.w);
+            e4m3x4_to_bf16x4(v.z, o1.x, o1.y);
+            e4m3x4_to_bf16x4(v.w, o1.z, o1.w);
+          }
+          const int panel = cc >> 2;
+          const int j0 = (cc & 3) * 2;
+          uint8_t* rowp = a + panel * C::A_HALF + row * 128;
+          *reinterpret_cast<uint4*>(rowp + ((j0 ^ (row & 7)) << 4)) = o0;
+          *reinterpret_cast<uint4*>(rowp + (((j0 + 1) ^ (row & 7)) << 4)) = o1;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->rempty[rs]);
+        mbar_arrive(&bars->afull[as]);
+      }
+      if (++rs == C::RS) { rs = 0; rphase ^= 1; }
+      if (++as == C::AS) { as = 0; aphase ^= 1; }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (long long u = u_begin; u < u_end; ++u) {
+      const int tile = static_cast<int>(u % NT);
+      const int b = static_cast<int>(u / NT);
+      if (!mbar_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int j = tile * C::BM + quad * 32 + lane;
+      float v[32];
+      tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::BN), v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+      if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
+      if (j >= p.N) continue;
+      bool valid;
+      int64_t sidx;
+      if (p.rows) {
+        const int32_t r = p.rows[static_cast<int64_t>(b) * p.N + j];
+        valid = (r >= 0) && (r < p.key_rows);
+        sidx = static_cast<int64_t>(b) * p.key_stride + (valid ? r : 0);
+      } else {
+        valid = (p.n_valid == nullptr) || (j < p.n_valid[b]);
+        sidx = static_cast<int64_t>(b) * p.N + j;
+      }
+      float s = neg_inf();
+      if (valid) {
+        const float sc = (FMT == SRC_BF16) ? 1.f : __ldg(p.scale + sidx);
+        const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * kHeads);
+        float acc_s = 0.f;
+#pragma unroll
+        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+          const float4 wv = __ldg(w4 + h4);
+          acc_s = fmaf(wv.x, fmaxf(sc * v[4 * h4 + 0], 0.f), acc_s);
+          acc_s = fmaf(wv.y, fmaxf(sc * v[4 * h4 + 1], 0.f), acc_s);
+          acc_s = fmaf(wv.z, fmaxf(sc * v[4 * h4 + 2], 0.f), acc_s);
+          acc_s = fmaf(wv.w, fmaxf(sc * v[4 * h4 + 3], 0.f), acc_s);
+        }
+        s = acc_s;
+      }
+      p.out[static_cast<int64_t>(b) * p.N + j] = s;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+template <int FMT>
+static cudaError_t launch_cvt(const CUtensorMap* qmap, const CvtParams& p, int num_sms, cudaStream_t st) {
+  using C = CvtCfg<FMT>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(score_cvt_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::SMEM_TOTAL));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int NT = (p.N + C::BM - 1) / C::BM;
+  const long long units = static_cast<long long>(p.B) * NT;
+  if (units == 0) return cudaSuccess;
+  const int grid = static_cast<int>(units < num_sms ? units : num_sms);
+  score_cvt_kernel<FMT><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*qmap, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score_cvt(const CUtensorMap* qmap, const CvtParams& p, int num_sms, cudaStream_t st) {
+  switch (p.fmt) {
+    case SRC_INT8: return launch_cvt<SRC_INT8>(qmap, p, num_sms, st);
+    case SRC_E4M3: return launch_cvt<SRC_E4M3>(qmap, p, num_sms, st);
+    case SRC_BF16: return launch_cvt<SRC_BF16>(qmap, p, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lsi

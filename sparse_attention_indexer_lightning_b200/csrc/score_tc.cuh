@@ -1,0 +1,315 @@
+// Lightning-indexer scoring on the sm_100a tensor cores, bf16 keys.
+//
+// score(t, s) = sum_h w[t, h] * max(0, q[t, h] . k[s])   ("03 long context",
+// section "The Architectural Answer: Read Less of the Past", stage 1; the
+// GLM-shaped 32-head x 128-d form of "Latent Sparse Attention", "Where the
+// time goes").
+//
+// Layout of the contraction (swap-AB): the MMA's M side is a tile of 128 keys
+// (A, K-major, 128-byte swizzle, fed by TMA), the N side is QG queries x 32
+// heads (B, K-major, TMA), K = d = 128 as 8 MMAs of K = 16.  The fp32
+// accumulator lives in TMEM with one key per lane, so the epilogue thread that
+// owns a key reads its 32 head sums with one tcgen05.ld and reduces the heads
+// in registers: ReLU, multiply by w, add -- no shuffles.
+//
+// Roles (one persistent CTA per SM, contiguous runs of work units):
+//   warp 0      TMA producer (keys every unit, the query tile on group change)
+//   warp 1      TMEM allocator + single-thread MMA issuer
+//   warps 2..   epilogue (4 warps for QG = 1, 8 for QG = 8)
+// Pipelines: STAGES key buffers (full/empty mbarriers), 2 query-tile slots,
+// 2 TMEM accumulators so the epilogue of unit i overlaps the MMA of unit i+1.
+// Every wait is bounded; a wait that runs out raises the library fault word
+// and the CTA drains its copies and MMAs before it frees TMEM and exits.
+
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lsi {
+
+template <int QG>
+struct TcCfg {
+  static constexpr int BM = kTileKeys;             // keys per tile
+  static constexpr int BN = QG * kHeads;           // queries x heads per MMA
+  static constexpr int A_BYTES = BM * kDim * 2;    // 32 KB
+  static constexpr int A_HALF = BM * 64 * 2;       // one 64-wide swizzle panel
+  static constexpr int B_BYTES = BN * kDim * 2;
+  static constexpr int B_HALF = BN * 64 * 2;
+  static constexpr int STAGES = (QG == 1) ? 6 : 3;
+  static constexpr int ACC = 2;
+  static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
+  static constexpr int TMEM_COLS = (ACC * ACC_COLS <= 32) ? 32
+                                   : (ACC * ACC_COLS <= 64) ? 64
+                                   : (ACC * ACC_COLS <= 128) ? 128
+                                   : (ACC * ACC_COLS <= 256) ? 256 : 512;
+  static constexpr int EPI_WARPS = (QG == 1) ? 4 : 8;
+  static constexpr int THREADS = (2 + EPI_WARPS) * 32;
+  static constexpr int Q_PER_EPI_WARP = (QG == 1) ? 1 : QG / 2;
+  static constexpr size_t SMEM_A = size_t(STAGES) * A_BYTES;
+  static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
+  static constexpr size_t SMEM_BAR = 512;
+  static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR;
+  static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
+};
+
+struct TcBarriers {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t bfull[2];
+  uint64_t bempty[2];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(TcBarriers) <= 512, "barrier block");
+
+// Drain wait: bounded by time only (used after an abort).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > LSI_WAIT_LIMIT_NS) {
+      atomicOr(&g_fault, FAULT_WAIT_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <int QG>
+__global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                    const ScoreParams p) {
+  using C = TcCfg<QG>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::SMEM_A;
+  TcBarriers* bars = reinterpret_cast<TcBarriers*>(smem + C::SMEM_A + C::SMEM_B);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int G = (p.T + QG - 1) / QG;
+  const int NT = (p.N + C::BM - 1) / C::BM;
+  const long long units = static_cast<long long>(p.B) * G * NT;
+  const long long u_begin = units * blockIdx.x / gridDim.x;
+  const long long u_end = units * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->bfull[s], 1);
+      mbar_init(&bars->bempty[s], 1);
+      mbar_init(&bars->tfull[s], 1);
+      mbar_init(&bars->tempty[s], C::EPI_WARPS);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&qmap);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long prev_bg = -1;
+      int bslot = 1;
+      uint32_t bphase[2] = {0, 0};
+      int issued[8];
+      uint32_t issued_par[8];
+      for (int s = 0; s < 8; ++s) issued[s] = 0, issued_par[s] = 0;
+      int b_issued[2] = {0, 0};
+      uint32_t b_par[2] = {0, 0};
+      bool ok = true;
+      for (long long u = u_begin; u < u_end && ok; ++u) {
+        const int tile = static_cast<int>(u % NT);
+        const long long bg = u / NT;
+        const int g = static_cast<int>(bg % G);
+        const int b = static_cast<int>(bg / G);
+        if (bg != prev_bg) {
+          bslot ^= 1;
+          if (!mbar_wait(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
+          b_par[bslot] = bphase[bslot];
+          b_issued[bslot] = 1;
+          bphase[bslot] ^= 1;
+          mbar_arrive_expect_tx(&bars->bfull[bslot], C::B_BYTES);
+          const int qrow = (b * p.T + g * QG) * kHeads;
+          uint8_t* dst = sB + bslot * C::B_BYTES;
+          tma_load_2d(dst, &qmap, &bars->bfull[bslot], 0, qrow);
+          tma_load_2d(dst + C::B_HALF, &qmap, &bars->bfull[bslot], 64, qrow);
+          prev_bg = bg;
+        }
+        if (!mbar_wait(&bars->empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&bars->full[stage], C::A_BYTES);
+        const int krow = b * p.N + tile * C::BM;
+        uint8_t* dst = sA + stage * C::A_BYTES;
+        tma_load_2d(dst, &kmap, &bars->full[stage], 0, krow);
+        tma_load_2d(dst + C::A_HALF, &kmap, &bars->full[stage], 64, krow);
+        issued[stage] = 1;
+        issued_par[stage] = phase;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) {
+        // Let every copy this thread started land before the CTA goes away.
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued[s]) mbar_wait_drain(&bars->full[s], issued_par[s]);
+        for (int s = 0; s < 2; ++s)
+          if (b_issued[s]) mbar_wait_drain(&bars->bfull[s], b_par[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      long long prev_bg = -1;
+      int bslot = 1;
+      uint32_t bphase[2] = {0, 0};
+      const uint32_t a_base = smem_u32(sA);
+      const uint32_t b_base = smem_u32(sB);
+      for (long long u = u_begin; u < u_end; ++u) {
+        const long long bg = u / NT;
+        if (bg != prev_bg) {
+          if (prev_bg >= 0) umma_commit(&bars->bempty[bslot]);
+          bslot ^= 1;
+          if (!mbar_wait(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
+          bphase[bslot] ^= 1;
+          prev_bg = bg;
+        }
+        if (!mbar_wait(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
+        tc_fence_after();
+        if (!mbar_wait(&bars->full[stage], phase, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_addr = a_base + stage * C::A_BYTES;
+        const uint32_t b_addr = b_base + bslot * C::B_BYTES;
+        const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+#pragma unroll
+        for (int kk = 0; kk < kDim / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside a 128 B swizzle row
+          const uint64_t adesc = sw128_kmajor_desc(a_addr + (kk >> 2) * C::A_HALF + koff);
+          const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + koff);
+          umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->empty[stage]);
+        umma_commit(&bars->tfull[acc]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
+      }
+      // All MMAs this thread issued are complete once `drain` flips.
+      umma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;                  // 0 .. EPI_WARPS-1
+    const int quad = warp & 3;                // TMEM lane quadrant this warp may read
+    const int qset = (QG == 1) ? 0 : (ew >> 2);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (long long u = u_begin; u < u_end; ++u) {
+      const int tile = static_cast<int>(u % NT);
+      const long long bg = u / NT;
+      const int g = static_cast<int>(bg % G);
+      const int b = static_cast<int>(bg / G);
+      if (!mbar_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int n = tile * C::BM + quad * 32 + lane;       // key within this launch
+      int lim = p.N;
+      if (p.n_valid) lim = min(lim, p.n_valid[b]);
+#pragma unroll 1
+      for (int jq = 0; jq < C::Q_PER_EPI_WARP; ++jq) {
+        const int j = qset * C::Q_PER_EPI_WARP + jq;       // query inside the group
+        const int t = g * QG + j;
+        if (t >= p.T) break;                               // warp-uniform
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(acc * C::ACC_COLS + j * kHeads);
+        float v[32];
+        tmem_ld_32x32(taddr, v);
+        const float4* w4 = reinterpret_cast<const float4*>(p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads);
+        float s = 0.f;
+#pragma unroll
+        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+          const float4 wv = __ldg(w4 + h4);
+          s = fmaf(wv.x, fmaxf(v[4 * h4 + 0], 0.f), s);
+          s = fmaf(wv.y, fmaxf(v[4 * h4 + 1], 0.f), s);
+          s = fmaf(wv.z, fmaxf(v[4 * h4 + 2], 0.f), s);
+          s = fmaf(wv.w, fmaxf(v[4 * h4 + 3], 0.f), s);
+        }
+        int lim_t = lim;
+        if (p.q_pos) {
+          const int64_t qp = p.q_pos[static_cast<int64_t>(b) * p.T + t];
+          int64_t e = qp < 0 ? 0 : (qp + 1) / p.stride;
+          if (e > p.n_total) e = p.n_total;
+          const int64_t rel = e - p.key_base;
+          lim_t = static_cast<int>(rel < 0 ? 0 : (rel < lim_t ? rel : lim_t));
+        }
+        if (n < p.N) {
+          p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+      if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+template <int QG>
+static cudaError_t launch_tc(const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p, int num_sms,
+                             cudaStream_t st) {
+  using C = TcCfg<QG>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<QG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::SMEM_TOTAL));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int G = (p.T + QG - 1) / QG;
+  const int NT = (p.N + C::BM - 1) / C::BM;
+  const long long units = static_cast<long long>(p.B) * G * NT;
+  if (units == 0) return cudaSuccess;
+  const int grid = static_cast<int>(units < num_sms ? units : num_sms);
+  score_tc_kernel<QG><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*kmap, *qmap, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score_tc(int qg, const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p,
+                            int num_sms, cudaStream_t st) {
+  if (qg == 1) return launch_tc<1>(kmap, qmap, p, num_sms, st);
+  if (qg == 8) return launch_tc<8>(kmap, qmap, p, num_sms, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lsi

@@ -1,0 +1,80 @@
+"""The C ABI without a GPU: the shared library loads, exports every entry
+point the header declares, and rejects bad arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ls_indexer.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_indexer_lightning_b200 import build
+    build.build()
+    from sparse_attention_indexer_lightning_b200 import _lib
+    return _lib.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ls_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("ls_indexer_score", "ls_topk_select", "ls_prefill_select_stream", "ls_decode_two_stage_select",
+              "ls_bucket_select", "ls_decode_select", "ls_last_error", "ls_device_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    from sparse_attention_indexer_lightning_b200._lib import EXPORTED
+    assert set(EXPORTED) == set(declared_functions())
+
+
+def test_version_and_workspace_queries(lib):
+    assert lib.ls_version() == 100
+    assert lib.ls_decode_select_workspace_size(64, 32768) == 64 * 32768 * 4
+    assert lib.ls_prefill_select_workspace_size(4096, 32768) >= 4096 * 32768 * 4 + 4096 * 4
+    assert lib.ls_two_stage_workspace_size(32, 131072, 4096) >= 32 * 131072 * 4 + 2 * 32 * 4096 * 4
+    assert lib.ls_bucket_workspace_size(256, 32768, 64, 512) >= 256 * 32768 * 4
+    assert lib.ls_decode_select_workspace_size(0, 10) == 0
+
+
+def test_argument_checks_without_gpu(lib):
+    P = ctypes.c_void_p
+    dummy = P(16)
+    # H != 32 is not built
+    st = lib.ls_indexer_score(dummy, dummy, dummy, 0, None, None, None, 4, 1, 1, 16, 128, 64, dummy, None)
+    assert st == 3
+    assert b"H=32" in lib.ls_last_error()
+    # k out of range
+    assert lib.ls_topk_select(dummy, 10, None, 1, 10, 0, dummy, None, None) == 1
+    assert lib.ls_topk_select(dummy, 10, None, 1, 10, 5000, dummy, None, None) == 1
+    # ld < N
+    assert lib.ls_topk_select(dummy, 5, None, 1, 10, 3, dummy, None, None) == 1
+    # short workspace
+    st = lib.ls_decode_select(dummy, dummy, dummy, None, 2, 32, 128, 100, 8, dummy, None, dummy, 10, None)
+    assert st == 2
+    # unknown key dtype / misaligned pointers
+    st = lib.ls_indexer_score(dummy, dummy, dummy, 9, None, None, None, 4, 1, 1, 32, 128, 64, dummy, None)
+    assert st == 1
+    st = lib.ls_indexer_score(P(17), dummy, dummy, 0, None, None, None, 4, 1, 1, 32, 128, 64, dummy, None)
+    assert st == 1
+    # two-stage: shortlist shorter than k
+    st = lib.ls_decode_two_stage_select(dummy, dummy, dummy, dummy, dummy, dummy, None, 1, 32, 128, 100, 256, 512,
+                                        dummy, None, None, dummy, 1 << 30, None)
+    assert st == 1
+    # bucket: budget below k
+    st = lib.ls_bucket_select(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 128, 10, 80, 4, 100, 512, dummy,
+                              None, None, dummy, 1 << 30, None)
+    assert st == 1
+    # empty problems are a no-op
+    assert lib.ls_indexer_score(None, None, None, 0, None, None, None, 4, 0, 1, 32, 128, 64, None, None) == 0

@@ -1,0 +1,340 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Small workloads span several key tiles and ragged tails and are compared
+element by element; the full-size workloads are run in the benchmark's launch
+configuration and checked on sampled rows the oracle computes one by one.
+"""
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.formats import bf16_to_f64, dequant
+from oracle.indexer import eligible_count, indexer_scores
+from oracle.select import bucket_select, expand_buckets, recall_at_k, select_topk, topk_rows, two_stage_select
+from parity_util import (
+    RTOL_BF16, RTOL_FP8, check_scores, check_selection, check_set, dev, dev_bf16, dev_e4m3, f32_bits_equal,
+)
+from workloads import get_workload, make_workload
+from workloads.synth import make_decode
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_indexer_lightning_b200 import build as b
+    b.build()
+    import sparse_attention_indexer_lightning_b200 as lib
+    return lib
+
+
+@functools.lru_cache(maxsize=None)
+def data(name):
+    return make_workload(name)
+
+
+def _ref_decode_scores(d, b, n=None):
+    n = d["k"].shape[1] if n is None else n
+    return indexer_scores(bf16_to_f64(d["q"][b])[None], d["w"][b].astype(np.float64)[None],
+                          bf16_to_f64(d["k"][b, :n]))[0]
+
+
+# --------------------------------------------------------------------------- #
+# top-k given fp32 scores: bit-exact
+# --------------------------------------------------------------------------- #
+def _adversarial_rows(rng, R, N):
+    s = rng.standard_normal((R, N)).astype(np.float32)
+    if R > 1:
+        s[1] = np.round(s[1] * 4) / 4                 # heavy ties
+    if R > 2:
+        s[2] = 0.0
+        s[2, ::3] = -0.0                              # +-0 ties
+    if R > 3:
+        s[3, ::5] = np.nan
+        s[3, ::7] = -np.inf
+    if R > 4:
+        s[4] = 1.0                                    # all equal
+    if R > 5:
+        s[5, :] = -np.inf
+        s[5, ::11] = np.nan
+    return s
+
+
+@pytest.mark.parametrize("R,N,k", [(7, 3000, 512), (6, 517, 512), (6, 40000, 4096), (3, 131072, 4096),
+                                   (8, 1000, 1), (6, 129, 64)])
+def test_topk_bit_exact(L, R, N, k):
+    rng = np.random.default_rng(100 + N)
+    s = _adversarial_rows(rng, R, N)
+    n_valid = rng.integers(0, N + 1, size=R).astype(np.int32)
+    n_valid[0] = N
+    if R > 6:
+        n_valid[6] = 0
+    for nv in (None, n_valid):
+        idx, val = L.ls_topk_select(dev(s), k, None if nv is None else dev(nv))
+        ri, rv = topk_rows(s, nv, k)
+        assert np.array_equal(idx.cpu().numpy(), ri), (R, N, k)
+        assert f32_bits_equal(val.cpu().numpy(), rv), (R, N, k)
+
+
+# --------------------------------------------------------------------------- #
+# decode scoring and selection
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("name", ["decode_tiny", "decode_s"])
+def test_decode_scores_and_select(L, name):
+    d = data(name)
+    B, H, dd = d["q"].shape
+    q = dev_bf16(d["q"])
+    w = dev(d["w"])
+    k = dev_bf16(d["k"])
+    nv = dev(d["n_valid"])
+    sc = L.ls_indexer_score(q.view(B, 1, H, dd), w.view(B, 1, H), k, n_valid=nv)[:, 0].cpu().numpy()
+    idx, val = L.ls_decode_select(q, w, k, 512, n_valid=nv)
+    idx, val = idx.cpu().numpy(), val.cpu().numpy()
+    for b in range(B):
+        n = int(d["n_valid"][b])
+        ref = _ref_decode_scores(d, b, n)
+        check_scores(sc[b, :n], ref, RTOL_BF16, f"{name} row {b}")
+        assert np.all(np.isneginf(sc[b, n:]))
+        check_selection(idx[b], val[b], np.arange(n), ref, 512, RTOL_BF16, f"{name} row {b}")
+        # selection over the GPU's own scores is bit-exact with the oracle's top-k
+        ri, rv = select_topk(sc[b, :n], np.arange(n), 512)
+        assert np.array_equal(idx[b], ri) and f32_bits_equal(val[b], rv)
+
+
+def test_decode_edge_rows(L):
+    # rows with no eligible key, fewer than k, exactly k, a ragged final tile
+    d = make_decode(B=5, N=700, seed=21, n_valid=np.array([0, 1, 511, 512, 700]))
+    q, w, k, nv = dev_bf16(d["q"]), dev(d["w"]), dev_bf16(d["k"]), dev(d["n_valid"])
+    idx, val = L.ls_decode_select(q, w, k, 512, n_valid=nv)
+    idx, val = idx.cpu().numpy(), val.cpu().numpy()
+    for b in range(5):
+        n = int(d["n_valid"][b])
+        ref = _ref_decode_scores(d, b, n) if n else np.zeros(0)
+        check_selection(idx[b], val[b], np.arange(n), ref, 512, RTOL_BF16, f"edge row {b}")
+
+
+@pytest.mark.slow
+def test_decode_batch_full_size_sampled(L):
+    d = data("decode_batch")
+    B, H, dd = d["q"].shape
+    q, w, k = dev_bf16(d["q"]), dev(d["w"]), dev_bf16(d["k"])
+    idx, val = L.ls_decode_select(q, w, k, 512)
+    sc = L.ls_indexer_score(q.view(B, 1, H, dd), w.view(B, 1, H), k)[:, 0]
+    idx, val = idx.cpu().numpy(), val.cpu().numpy()
+    for b in (0, 31, 63):
+        ref = _ref_decode_scores(d, b)
+        check_scores(sc[b].cpu().numpy(), ref, RTOL_BF16, f"decode_batch row {b}")
+        check_selection(idx[b], val[b], np.arange(ref.size), ref, 512, RTOL_BF16, f"decode_batch row {b}")
+    # every row: the selection equals the bit-exact top-k of the kernel's own scores
+    ri, rv = topk_rows(sc.cpu().numpy(), None, 512)
+    assert np.array_equal(idx, ri) and f32_bits_equal(val, rv)
+
+
+# --------------------------------------------------------------------------- #
+# multi-query tiles and converted key formats
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("T", [2, 19, 64])
+def test_multiquery_scores_causal(L, T):
+    rng = np.random.default_rng(30 + T)
+    B, H, dd, N = 2, 32, 128, 900
+    from workloads.synth import to_bf16_bits
+    qb = to_bf16_bits(rng.standard_normal((B, T, H, dd)) / np.sqrt(dd))
+    kb = to_bf16_bits(rng.standard_normal((B, N, dd)) / np.sqrt(dd))
+    wv = (rng.standard_normal((B, T, H)) / np.sqrt(H)).astype(np.float32)
+    qpos = rng.integers(-2, 4 * N + 8, size=(B, T)).astype(np.int64)
+    nv = np.array([N, N - 77], np.int32)
+    sc = L.ls_indexer_score(dev_bf16(qb), dev(wv), dev_bf16(kb), n_valid=dev(nv), q_pos=dev(qpos), stride=4)
+    sc = sc.cpu().numpy()
+    for b in range(B):
+        ref = indexer_scores(bf16_to_f64(qb[b]), wv[b].astype(np.float64), bf16_to_f64(kb[b]))
+        lim = np.minimum(eligible_count(qpos[b], 4, N), nv[b])
+        for t in range(T):
+            check_scores(sc[b, t, : lim[t]], ref[t, : lim[t]], RTOL_BF16, f"T={T} b={b} t={t}")
+            assert np.all(np.isneginf(sc[b, t, lim[t]:]))
+
+
+@pytest.mark.parametrize("fmt", ["int8", "e4m3"])
+def test_converted_key_scores(L, fmt):
+    d = data("two_stage_s")
+    B, H, dd = d["q"].shape
+    q, w = dev_bf16(d["q"]), dev(d["w"])
+    if fmt == "int8":
+        keys, scale, rtol = dev(d["ck"]), dev(d["ck_scale"]), RTOL_BF16
+    else:
+        keys, scale, rtol = dev_e4m3(d["fk"]), dev(d["fk_scale"]), RTOL_BF16
+    nv = dev(d["n_valid"])
+    sc = L.ls_indexer_score(q.view(B, 1, H, dd), w.view(B, 1, H), keys, key_scale=scale, n_valid=nv)[:, 0]
+    sc = sc.cpu().numpy()
+    codes = d["ck"] if fmt == "int8" else d["fk"]
+    scales = d["ck_scale"] if fmt == "int8" else d["fk_scale"]
+    for b in range(B):
+        n = int(d["n_valid"][b])
+        kv = dequant(codes[b, :n], scales[b, :n], fmt)
+        ref = indexer_scores(bf16_to_f64(d["q"][b])[None], d["w"][b].astype(np.float64)[None], kv)[0]
+        check_scores(sc[b, :n], ref, rtol, f"{fmt} row {b}")
+        assert np.all(np.isneginf(sc[b, n:]))
+
+
+# --------------------------------------------------------------------------- #
+# prefill: streamed history, causal eligibility
+# --------------------------------------------------------------------------- #
+def _prefill_run(L, d, wl, use_copy_stream=True):
+    T = d["q"].shape[0]
+    q, w, qp = dev_bf16(d["q"]), dev(d["w"]), dev(d["q_pos"])
+    hist = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    buf0 = torch.empty((wl.tile_keys, 128), dtype=torch.bfloat16, device="cuda")
+    buf1 = torch.empty_like(buf0)
+    cs = torch.cuda.Stream() if use_copy_stream else None
+    idx, val = L.ls_prefill_select_stream(q, w, qp, hist, buf0, buf1, k=wl.k, stride=wl.stride,
+                                          tile_keys=wl.tile_keys, copy_stream=cs)
+    torch.cuda.synchronize()
+    return q, w, qp, idx.cpu().numpy(), val.cpu().numpy()
+
+
+def test_prefill_stream_small(L):
+    wl = get_workload("prefill_s")
+    d = data("prefill_s")
+    q, w, qp, idx, val = _prefill_run(L, d, wl)
+    T, H, dd = d["q"].shape
+    N = d["k"].shape[0]
+    n_t = eligible_count(d["q_pos"], wl.stride, N)
+    keys = bf16_to_f64(d["k"])
+    for t in range(T):
+        n = int(n_t[t])
+        ref = indexer_scores(bf16_to_f64(d["q"][t])[None], d["w"][t].astype(np.float64)[None], keys[:n])[0]
+        check_selection(idx[t], val[t], np.arange(n), ref, wl.k, RTOL_BF16, f"prefill_s t={t}")
+    # the streamed result equals scoring the resident history in one call
+    sc = L.ls_indexer_score(q.view(1, T, H, dd), w.view(1, T, H), dev_bf16(d["k"])[None], q_pos=qp.view(1, T),
+                            stride=wl.stride)[0]
+    ri, rv = L.ls_topk_select(sc, wl.k, n_valid=dev(n_t.astype(np.int32)))
+    assert np.array_equal(ri.cpu().numpy(), idx) and f32_bits_equal(rv.cpu().numpy(), val)
+    # same answer on a single stream
+    *_, idx2, val2 = _prefill_run(L, d, wl, use_copy_stream=False)
+    assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
+
+
+@pytest.mark.slow
+def test_prefill_chunk_full_size_sampled(L):
+    wl = get_workload("prefill_chunk")
+    d = data("prefill_chunk")
+    _, _, _, idx, val = _prefill_run(L, d, wl)
+    N = d["k"].shape[0]
+    n_t = eligible_count(d["q_pos"], wl.stride, N)
+    keys = bf16_to_f64(d["k"])
+    for t in (0, 1, 2, 3, 1023, 2048, 4093, 4094, 4095):
+        n = int(n_t[t])
+        ref = indexer_scores(bf16_to_f64(d["q"][t])[None], d["w"][t].astype(np.float64)[None], keys[:n])[0]
+        check_selection(idx[t], val[t], np.arange(n), ref, wl.k, RTOL_BF16, f"prefill t={t}")
+
+
+# --------------------------------------------------------------------------- #
+# two-stage decode search
+# --------------------------------------------------------------------------- #
+def _check_two_stage(L, name, rows):
+    wl = get_workload(name)
+    d = data(name)
+    q, w = dev_bf16(d["q"]), dev(d["w"])
+    idx, val, sl = L.ls_decode_two_stage_select(q, w, dev(d["ck"]), dev(d["ck_scale"]), dev_e4m3(d["fk"]),
+                                                dev(d["fk_scale"]), dev(d["n_valid"]), shortlist=wl.shortlist,
+                                                k=wl.k, want_shortlist=True)
+    idx, val, sl = idx.cpu().numpy(), val.cpu().numpy(), sl.cpu().numpy()
+    _, _, det = two_stage_select(d["q"], d["w"], d["ck"], d["ck_scale"], d["fk"], d["fk_scale"], d["n_valid"],
+                                 wl.shortlist, wl.k, rows=rows, return_detail=True)
+    recalls = []
+    for i, b in enumerate(rows):
+        n = int(d["n_valid"][b])
+        s_hat = det[i]["s_hat"]
+        # shortlist: the band rule on the compact scores (order of the shortlist
+        # is the coarse-score order, so its values are not checked here)
+        short = sl[b][sl[b] >= 0]
+        check_set(sl[b], np.arange(n), s_hat, wl.shortlist, RTOL_BF16, f"{name} shortlist row {b}")
+        # final: exact scores of the GPU's shortlist, band rule inside it
+        kv = dequant(d["fk"][b, short], d["fk_scale"][b, short], "e4m3")
+        exact = indexer_scores(bf16_to_f64(d["q"][b])[None], d["w"][b].astype(np.float64)[None], kv)[0]
+        check_selection(idx[b], val[b], short, exact, wl.k, RTOL_FP8, f"{name} final row {b}")
+        # recall against the exact full scan (reported, not pinned)
+        kfull = dequant(d["fk"][b, :n], d["fk_scale"][b, :n], "e4m3")
+        full = indexer_scores(bf16_to_f64(d["q"][b])[None], d["w"][b].astype(np.float64)[None], kfull)[0]
+        ei, _ = select_topk(full, np.arange(n), wl.k)
+        recalls.append(recall_at_k(idx[b][None], ei[None]))
+    return recalls
+
+
+def test_two_stage_small(L):
+    rec = _check_two_stage(L, "two_stage_s", [0, 1, 2])
+    assert min(rec) > 0.5
+
+
+@pytest.mark.slow
+def test_two_stage_full_size_sampled(L):
+    rec = _check_two_stage(L, "two_stage", [0, 17, 31])
+    assert min(rec) > 0.5
+
+
+# --------------------------------------------------------------------------- #
+# bucket search
+# --------------------------------------------------------------------------- #
+def _check_bucket(L, name, rows):
+    wl = get_workload(name)
+    d = data(name)
+    q, w = dev_bf16(d["q"]), dev(d["w"])
+    idx, val, picked = L.ls_bucket_select(q, w, dev_bf16(d["centroids"]), dev(d["bucket_off"]),
+                                          dev(d["bucket_mem"]), dev_bf16(d["keys"]), top_p=wl.top_p,
+                                          budget=wl.budget, k=wl.k, want_picked=True)
+    idx, val, picked = idx.cpu().numpy(), val.cpu().numpy(), picked.cpu().numpy()
+    P = d["centroids"].shape[0]
+    _, _, det = bucket_select(d["q"], d["w"], d["centroids"], d["bucket_off"], d["bucket_mem"], d["keys"],
+                              wl.top_p, wl.budget, wl.k, rows=rows, return_detail=True)
+    keys = bf16_to_f64(d["keys"])
+    recalls = []
+    for i, t in enumerate(rows):
+        cs = det[i]["centroid_scores"]
+        check_set(picked[t], np.arange(P), cs, wl.top_p, RTOL_BF16, f"{name} picked row {t}")
+        # expansion follows the GPU's pick order
+        cand = expand_buckets(picked[t], d["bucket_off"], d["bucket_mem"], wl.budget)
+        exact = indexer_scores(bf16_to_f64(d["q"][t])[None], d["w"][t].astype(np.float64)[None], keys[cand])[0]
+        check_selection(idx[t], val[t], cand, exact, wl.k, RTOL_BF16, f"{name} final row {t}")
+        full = indexer_scores(bf16_to_f64(d["q"][t])[None], d["w"][t].astype(np.float64)[None], keys)[0]
+        ei, _ = select_topk(full, np.arange(keys.shape[0]), wl.k)
+        recalls.append(recall_at_k(idx[t][None], ei[None]))
+    return recalls
+
+
+def test_bucket_small(L):
+    rec = _check_bucket(L, "bucket_s", list(range(19)))
+    assert min(rec) > 0.1
+
+
+@pytest.mark.slow
+def test_bucket_full_size_sampled(L):
+    rec = _check_bucket(L, "bucket", [0, 100, 255])
+    assert min(rec) > 0.3
+
+
+def test_bucket_bad_member_flagged(L):
+    d = data("bucket_s")
+    mem = d["bucket_mem"].copy()
+    mem[:] = np.where(np.arange(mem.size) % 5 == 0, d["keys"].shape[0] + 1000, mem)  # out of range ids
+    L.ls_device_status()
+    L.ls_bucket_select(dev_bf16(d["q"]), dev(d["w"]), dev_bf16(d["centroids"]), dev(d["bucket_off"]), dev(mem),
+                       dev_bf16(d["keys"]), top_p=64, budget=512, k=512)
+    flags = L.ls_device_status()
+    assert flags & 2  # LS_FAULT_BAD_INDEX: the bad rows were skipped, not read
+
+
+# --------------------------------------------------------------------------- #
+# failure detection: a bounded device wait ends with an error status
+# --------------------------------------------------------------------------- #
+def test_wait_probe_times_out_and_context_survives(L):
+    L.ls_device_status()
+    gave_up = L.ls_selftest_wait_probe(2_000_000)  # 2 ms
+    flags = L.ls_device_status()
+    assert int(gave_up.item()) == 1
+    assert flags & 1
+    # the context is still usable
+    test_decode_edge_rows(L)
