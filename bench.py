@@ -27,7 +27,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -55,59 +54,62 @@ def load_peaks():
 # clocks sampler (nvidia-smi during the timed region)
 # --------------------------------------------------------------------------- #
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and throttle reasons through NVML in a thread while the
+    timed region runs (the region is short, so the polling is tight)."""
+
+    REASONS = {  # NVML clocks-event-reason bits
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4,
+    }
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
-        self.thread = None
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nvml = nv
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.gpu]) if vis and vis.split(",")[0].isdigit() else self.gpu
+            self._h = nv.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            self._nvml = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
-        self.thread.start()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = fn(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                break
+            time.sleep(0.0005)
 
     def stop(self):
-        if self.proc is None:
+        if self._nvml is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        if self.thread:
-            self.thread.join(timeout=2)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=2)
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # --------------------------------------------------------------------------- #
@@ -197,40 +199,38 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
     q, w, k = to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev_bf16(d["k"])
     q4, w3 = q.view(B, 1, H, dd), w.view(B, 1, H)
     st = torch.cuda.current_stream()
-    sc = torch.empty((B, 1, N), dtype=torch.float32, device="cuda")
     idx = torch.empty((B, wl.k), dtype=torch.int32, device="cuda")
     val = torch.empty((B, wl.k), dtype=torch.float32, device="cuda")
     lib = L.lib()
     import ctypes
     P = ctypes.c_void_p
     stp = P(st.cuda_stream)
+    ws = torch.empty(lib.ls_decode_select_workspace_size(B, N), dtype=torch.uint8, device="cuda")
 
     def step(i, timed):
-        e0 = e1 = e2 = None
-        if timed:
-            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-            e0.record(st)
-        s1 = lib.ls_indexer_score(P(q4.data_ptr()), P(w3.data_ptr()), P(k.data_ptr()), 0, None, None, None, 4,
-                                  B, 1, H, dd, N, P(sc.data_ptr()), stp)
-        if timed:
-            e1.record(st)
-        s2 = lib.ls_topk_select(P(sc.data_ptr()), N, None, B, N, wl.k, P(idx.data_ptr()), P(val.data_ptr()), stp)
-        if s1 or s2:
+        s = lib.ls_decode_select(P(q.data_ptr()), P(w.data_ptr()), P(k.data_ptr()), None, B, H, dd, N, wl.k,
+                                 P(idx.data_ptr()), P(val.data_ptr()), P(ws.data_ptr()), ws.numel(), stp)
+        if s:
             raise RuntimeError(lib.ls_last_error().decode())
-        if timed:
-            e2.record(st)
-            return {"scan": (e0, e1), "topk": (e1, e2)}
         return None
 
     clocks = ClockSampler(torch.cuda.current_device())
+    for i in range(args.warmup):
+        step(i, None)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
-    total_ms, seg = time_loop(step, args.steps, args.warmup, st)
+    # the library brackets each of its kernel launches with CUDA events on the
+    # launch stream while profiling is on: per-kernel time over the timed region
+    L.ls_profile_begin()
+    total_ms, _ = time_loop(step, args.steps, 0, st)
+    prof = L.ls_profile_end()
     clk = clocks.stop()
     barrier(world)
     ms_per_step = max_over_ranks(total_ms / args.steps, world)
-    scan_ms = seg["scan"] / args.steps
+    scan_ms = prof["score_tc_kernel<1>"][0] / prof["score_tc_kernel<1>"][1]
+    topk_ms = prof["topk_kernel"][0] / prof["topk_kernel"][1]
+    launches = sum(c for _, c in prof.values())
     positions = B * N
     value = world * positions / (ms_per_step * 1e-3)
     key_bytes = B * N * dd * 2
@@ -243,10 +243,11 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
                    "heads": H, "d": dd, "k": wl.k, "parallelism": f"replicas x{world}",
                    "l2": "inputs (537 MB keys) larger than the 126 MB L2; no flush"},
         "selections_per_s": world * B / (ms_per_step * 1e-3),
-        "breakdown_ms": {"scan": scan_ms, "topk": seg["topk"] / args.steps},
+        "breakdown_ms": {"scan": scan_ms, "topk": topk_ms},
+        "kernels": {kname: {"total_ms": v[0], "launches": v[1]} for kname, v in prof.items()},
         "roofline": roofline("hbm", key_bytes / (scan_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                              traffic=args.scan_traffic, peak_kind=peak_kind),
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches,
         "clocks": clk,
     }
     out["roofline"]["kernel"] = "score_tc_kernel<1> (decode scan)"
@@ -258,8 +259,6 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
     hk = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
     oi = torch.empty((B, wl.k), dtype=torch.int32).pin_memory()
     ov = torch.empty((B, wl.k), dtype=torch.float32).pin_memory()
-    ws = torch.empty(lib.ls_decode_select_workspace_size(B, N), dtype=torch.uint8, device="cuda")
-
     def e2e_step(i, timed):
         q.copy_(hq, non_blocking=True)
         w.copy_(hw, non_blocking=True)
@@ -283,23 +282,42 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
     return out, d
 
 
-def bench_variants(L, args, peaks, peak_kind):
+def bench_variants(L, args, peaks, peak_kind, only=None):
     """Prefill chunk, two-stage and bucket searches: one timed loop each."""
+    res = {}
+    for name, fn in (("prefill_chunk", bench_prefill), ("bucket", bench_bucket), ("two_stage", bench_two_stage)):
+        if only in (None, name):
+            res[name] = fn(L, args, peaks, peak_kind)
+    return res
+
+
+def _profiled_loop(L, fn, steps, warm, st):
+    """Warm up, then time `steps` calls with the library's per-kernel events on."""
+    import torch
+    for i in range(warm):
+        fn(i, None)
+    torch.cuda.synchronize()
+    L.ls_profile_begin()
+    tot, _ = time_loop(fn, steps, 0, st)
+    prof = L.ls_profile_end()
+    kern = {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps} for k, v in prof.items()}
+    return tot / steps, kern
+
+
+def bench_prefill(L, args, peaks, peak_kind):
+    """Prefill chunk: history streamed from pinned host memory in 8192-key
+    tiles through two device buffers, causal top-512 of 4096 queries."""
     import torch
     from workloads import get_workload, make_workload
-    res = {}
     st = torch.cuda.current_stream()
     steps = max(3, args.steps)
     warm = max(3, args.warmup)
-
-    # ---- prefill chunk: streamed history, causal top-512 --------------------
     wl = get_workload("prefill_chunk")
     d = make_workload(wl)
     T, H, dd = d["q"].shape
     N = d["k"].shape[0]
     q, w, qp = to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev(d["q_pos"])
     hist = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
-    hist_dev = hist.cuda()
     buf0 = torch.empty((wl.tile_keys, dd), dtype=torch.bfloat16, device="cuda")
     buf1 = torch.empty_like(buf0)
     ws = torch.empty(L.lib().ls_prefill_select_workspace_size(T, N), dtype=torch.uint8, device="cuda")
@@ -309,51 +327,37 @@ def bench_variants(L, args, peaks, peak_kind):
     n_t = np.minimum((d["q_pos"] + 1) // wl.stride, N)
     pairs = int(n_t.sum())
 
-    def pf(i, timed, src):
-        L.ls_prefill_select_stream(q, w, qp, src, buf0, buf1, k=wl.k, stride=wl.stride, tile_keys=wl.tile_keys,
+    def pf(i, timed):
+        L.ls_prefill_select_stream(q, w, qp, hist, buf0, buf1, k=wl.k, stride=wl.stride, tile_keys=wl.tile_keys,
                                    ws=ws, out=out, copy_stream=cs)
         return None
 
-    tot, _ = time_loop(lambda i, t: pf(i, t, hist), steps, warm, st)
-    ms = tot / steps
-    # scoring kernels alone: the same 4 tile launches over device-resident history
-    sc = torch.empty((1, T, N), dtype=torch.float32, device="cuda")
-    lib = L.lib()
-    import ctypes
-    P = ctypes.c_void_p
-
-    def score_only(i, timed):
-        e0 = e1 = None
-        if timed:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(st)
-        s = lib.ls_indexer_score(P(q.data_ptr()), P(w.data_ptr()), P(hist_dev.data_ptr()), 0, None, None,
-                                 P(qp.data_ptr()), wl.stride, 1, T, H, dd, N, P(sc.data_ptr()), P(st.cuda_stream))
-        if s:
-            raise RuntimeError(lib.ls_last_error().decode())
-        if timed:
-            e1.record(st)
-            return {"score": (e0, e1)}
-        return None
-
-    _, seg = time_loop(score_only, steps, warm, st)
-    score_ms = seg["score"] / steps
+    ms, kern = _profiled_loop(L, pf, steps, warm, st)
+    score_ms = kern["score_tc_kernel<8>"]["ms_per_step"]
     flops_alg = pairs * 2 * H * dd
     peak_t = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
-    res["prefill_chunk"] = {
+    res = {
         "ms_per_step": ms, "positions_per_s": pairs / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
-        "score_kernel_ms": score_ms,
+        "kernels": kern,
         "roofline": roofline("tensor", flops_alg / (score_ms * 1e-3) / 1e12, peak_t, "TFLOP/s", peak_kind=peak_kind),
         "algorithmic_flops": flops_alg, "eligible_pairs": pairs,
         "note": "step = 4 streamed 8192-key tiles (H2D on a copy stream) + causal top-512 of 4096 queries; "
-                "score_kernel_ms = scoring of the whole history resident in HBM (one launch)",
+                "roofline over the 4 scoring launches of the step (score_tc_kernel<8>)",
     }
-    del sc, ws, hist_dev
+    del ws
+    return res
 
-    # ---- bucket search -------------------------------------------------------
+
+def bench_bucket(L, args, peaks, peak_kind):
+    """Bucket search over 32768 clusters of 8 keys, 256 queries."""
+    import torch
+    from workloads import get_workload, make_workload
+    st = torch.cuda.current_stream()
+    steps = max(3, args.steps)
+    warm = max(3, args.warmup)
     wl = get_workload("bucket")
     d = make_workload(wl)
-    T = d["q"].shape[0]
+    T, H, dd = d["q"].shape
     P_ = d["centroids"].shape[0]
     args_b = [to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev_bf16(d["centroids"]), to_dev(d["bucket_off"]),
               to_dev(d["bucket_mem"]), to_dev_bf16(d["keys"])]
@@ -366,14 +370,26 @@ def bench_variants(L, args, peaks, peak_kind):
         L.ls_bucket_select(*args_b, top_p=wl.top_p, budget=wl.budget, k=wl.k, ws=wsb, out=outb)
         return None
 
-    tot, _ = time_loop(bk, steps, warm, st)
-    ms = tot / steps
-    res["bucket"] = {"ms_per_step": ms, "positions_per_s": T * (P_ + wl.budget) / (ms * 1e-3),
-                     "selections_per_s": T / (ms * 1e-3),
-                     "note": "positions = centroids scored + keys rescored per query"}
+    ms, kern = _profiled_loop(L, bk, steps, warm, st)
+    cms = kern["score_tc_kernel<8>"]["ms_per_step"]
+    flops = T * P_ * 2 * H * dd
+    peak_t = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    res = {"ms_per_step": ms, "positions_per_s": T * (P_ + wl.budget) / (ms * 1e-3),
+           "selections_per_s": T / (ms * 1e-3), "kernels": kern,
+           "roofline": roofline("tensor", flops / (cms * 1e-3) / 1e12, peak_t, "TFLOP/s", peak_kind=peak_kind),
+           "algorithmic_flops_centroids": flops,
+           "note": "positions = centroids scored + keys rescored per query; roofline of the centroid scoring"}
     del args_b, wsb
+    return res
 
-    # ---- two-stage decode search ---------------------------------------------
+
+def bench_two_stage(L, args, peaks, peak_kind):
+    """Two-stage decode search: compact scan, shortlist, exact re-rank."""
+    import torch
+    from workloads import get_workload, make_workload
+    st = torch.cuda.current_stream()
+    steps = max(3, args.steps)
+    warm = max(3, args.warmup)
     wl = get_workload("two_stage")
     d = make_workload(wl)
     B, H, dd = d["q"].shape
@@ -388,34 +404,19 @@ def bench_variants(L, args, peaks, peak_kind):
         L.ls_decode_two_stage_select(*a2, shortlist=wl.shortlist, k=wl.k, ws=ws2, out=out2)
         return None
 
-    tot, _ = time_loop(ts, steps, warm, st)
-    ms = tot / steps
-    # the compact scan alone
-    s_hat = torch.empty((B, 1, N), dtype=torch.float32, device="cuda")
-
-    def scan_only(i, timed):
-        e0 = e1 = None
-        if timed:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(st)
-        L.ls_indexer_score(a2[0].view(B, 1, H, dd), a2[1].view(B, 1, H), a2[2], key_scale=a2[3])
-        if timed:
-            e1.record(st)
-            return {"scan": (e0, e1)}
-        return None
-
-    _, seg = time_loop(scan_only, steps, warm, st)
-    scan_ms = seg["scan"] / steps
+    ms, kern = _profiled_loop(L, ts, steps, warm, st)
+    scan_ms = kern["score_cvt_kernel<int8>"]["ms_per_step"]
     scan_bytes = B * N * (dd + 4)
-    res["two_stage"] = {
+    res = {
         "ms_per_step": ms, "positions_per_s": B * (N + wl.shortlist) / (ms * 1e-3),
-        "selections_per_s": B / (ms * 1e-3), "compact_scan_ms": scan_ms,
+        "selections_per_s": B / (ms * 1e-3), "kernels": kern,
         "roofline": roofline("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                              peak_kind=peak_kind),
         "algorithmic_bytes_scan": scan_bytes,
-        "note": "positions = compact keys scanned + shortlist re-ranked; scan roofline on int8 codes + scales",
+        "note": "positions = compact keys scanned + shortlist re-ranked; roofline of the compact scan "
+                "(int8 codes + fp32 scales)",
     }
-    del a2, ws2, s_hat
+    del a2, ws2
     torch.cuda.empty_cache()
     return res
 
@@ -436,13 +437,15 @@ def blas_threads():
 
 
 def oracle_decode_rate(d, budget_s: float, k: int):
-    """Oracle decode selection over whole sequences until budget_s elapses."""
+    """Oracle decode selection over whole sequences (cycling through the
+    batch) until budget_s of CPU time has elapsed."""
     from oracle.select import decode_select
     B, N = d["k"].shape[0], d["k"].shape[1]
     done = 0
     t0 = time.perf_counter()
-    while done < B and (time.perf_counter() - t0) < budget_s:
-        decode_select(d["q"][done:done + 1], d["w"][done:done + 1], d["k"][done:done + 1], None, k)
+    while (time.perf_counter() - t0) < budget_s:
+        b = done % B
+        decode_select(d["q"][b:b + 1], d["w"][b:b + 1], d["k"][b:b + 1], None, k)
         done += 1
     el = time.perf_counter() - t0
     return done * N / el, done, el
@@ -489,6 +492,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_batch")
     ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--only", default=None, choices=["prefill_chunk", "bucket", "two_stage"],
+                    help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scan-traffic", type=float, default=None,
                     help="dram bytes per scan launch from an ncu capture of the current kernel")
@@ -502,11 +507,14 @@ def main(argv=None):
     world, rank, local = dist_setup(args.gpus)
     import sparse_attention_indexer_lightning_b200 as L
     peaks, peak_kind = load_peaks()
+    if args.only:
+        print(json.dumps({"variant": args.only, **bench_variants(L, args, peaks, peak_kind, args.only)}))
+        return 0
     out, d = bench_decode(L, args, world, rank, peaks, peak_kind)
     if not args.no_variants and world == 1:
         out["variants"] = bench_variants(L, args, peaks, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, n_seq, el = oracle_decode_rate(d, 15.0, 512)
+        rate, n_seq, el = oracle_decode_rate(d, 12.0, 512)
         out["cpu_baseline"] = {"value": rate, "unit": "positions/s", "cores": blas_threads(), "kind": "oracle",
                                "sample": f"{n_seq} whole sequences x {d['k'].shape[1]} positions "
                                          f"({el:.1f} s of fp64 oracle work)"}

@@ -62,6 +62,15 @@ typedef int ls_status;
 #define LS_FAULT_WAIT_TIMEOUT 1 /* an in-kernel wait exceeded its limit */
 #define LS_FAULT_BAD_INDEX 2    /* a gathered row id was outside the key array */
 
+/*
+ * Selection histogram: LS_HIST_BINS counts per row of the top 11 bits of each
+ * score's order code, where the order code of an fp32 score with bit pattern
+ * b is: 0 for NaN; else with b = 0 for -0.0, (b & 0x80000000 ? ~b : b | 0x80000000).
+ * The scan produces it for free; the top-k uses it to skip its own counting
+ * pass.  A histogram that does not match the scores gives wrong selections.
+ */
+#define LS_HIST_BINS 2048
+
 /* key storage formats */
 #define LS_KEY_BF16 0     /* [.][d] bf16 */
 #define LS_KEY_FP8_E4M3 1 /* [.][d] e4m3 codes + per-key fp32 scale (128 B + 4 B) */
@@ -97,13 +106,16 @@ ls_status ls_device_status(int* flags, void* stream);
  *                                     block of `stride` tokens precedes the query;
  *                                     LeanSparse transcript 02:36-02:56)
  *   scores   [B][T][N]    fp32        output; masked entries are -inf
+ *   hist_out [B*T][2048] uint32 or NULL selection histogram of the unmasked scores
+ *                                     (see LS_HIST_BINS); counts are ADDED, so the
+ *                                     caller zeroes it first.  T == 1 only.
  * BF16 keys take any T >= 1 (tensor-core tiles of 8 queries x 32 heads when
  * T > 1, one query per tile when T == 1).  FP8/INT8 keys take T == 1 and no
  * q_pos.  No workspace.
  */
 ls_status ls_indexer_score(const uint16_t* q, const float* w, const void* keys, int key_dtype,
                            const float* key_scale, const int32_t* n_valid, const int64_t* q_pos, int stride,
-                           int B, int T, int H, int d, int N, float* scores, void* stream);
+                           int B, int T, int H, int d, int N, float* scores, uint32_t* hist_out, void* stream);
 
 /*
  * ls_topk_select -- exact row-wise top-k of given fp32 scores, bit-exact.
@@ -112,11 +124,13 @@ ls_status ls_indexer_score(const uint16_t* q, const float* w, const void* keys, 
  *
  *   scores  row r starts at scores + r*ld (ld >= N)
  *   n_valid [R] int32 or NULL: columns >= n_valid[r] are not candidates
+ *   hist    [R][LS_HIST_BINS] uint32 or NULL: the rows' selection histograms
+ *           (e.g. from ls_indexer_score); NULL = counted here in one extra pass
  *   idx_out [R][k] int32 column ids (-1 padding);  val_out [R][k] fp32 or NULL
  * 1 <= k <= 4096.  No workspace.
  */
-ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int N, int k,
-                         int32_t* idx_out, float* val_out, void* stream);
+ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, const uint32_t* hist, int R,
+                         int N, int k, int32_t* idx_out, float* val_out, void* stream);
 
 /*
  * ls_decode_select -- decode selection: one query per sequence over bf16 keys,
@@ -194,6 +208,18 @@ ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* ce
                            const int32_t* bucket_mem, const uint16_t* keys, int T, int H, int d, int P, int N,
                            int top_p, int budget, int k, int32_t* idx_out, float* val_out, int32_t* picked_out,
                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Profiling: between ls_profile_begin() and ls_profile_end(), every kernel the
+ * library launches is bracketed by two CUDA events on its launch stream.
+ * ls_profile_end() waits for those events and sums the durations per kernel
+ * name; ls_profile_kernel(i, ...) reads kernel i (0 <= i < *n_kernels).  The
+ * name pointer stays valid until the next ls_profile_begin().  Host thread
+ * safe; recording adds two event records per launch.
+ */
+ls_status ls_profile_begin(void);
+ls_status ls_profile_end(int* n_kernels);
+ls_status ls_profile_kernel(int i, const char** name, double* total_ms, long long* launches);
 
 /*
  * ls_selftest_wait_probe -- failure-detection check: launches a kernel whose

@@ -16,6 +16,8 @@ from ._lib import (  # noqa: F401
     ls_device_status,
     ls_indexer_score,
     ls_prefill_select_stream,
+    ls_profile_begin,
+    ls_profile_end,
     ls_selftest_wait_probe,
     ls_topk_select,
     lib,

@@ -34,8 +34,10 @@ EXPORTED = (
     "ls_last_error", "ls_version", "ls_device_status", "ls_indexer_score", "ls_topk_select",
     "ls_decode_select_workspace_size", "ls_decode_select", "ls_prefill_select_workspace_size",
     "ls_prefill_select_stream", "ls_two_stage_workspace_size", "ls_decode_two_stage_select",
-    "ls_bucket_workspace_size", "ls_bucket_select", "ls_selftest_wait_probe",
+    "ls_bucket_workspace_size", "ls_bucket_select", "ls_selftest_wait_probe", "ls_profile_begin",
+    "ls_profile_end", "ls_profile_kernel",
 )
+HIST_BINS = 2048
 
 
 class LSError(RuntimeError):
@@ -55,8 +57,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_last_error": (ctypes.c_char_p, []),
         "ls_version": (I, []),
         "ls_device_status": (I, [P, P]),
-        "ls_indexer_score": (I, [P, P, P, I, P, P, P, I, I, I, I, I, I, P, P]),
-        "ls_topk_select": (I, [P, I64, P, I, I, I, P, P, P]),
+        "ls_indexer_score": (I, [P, P, P, I, P, P, P, I, I, I, I, I, I, P, P, P]),
+        "ls_topk_select": (I, [P, I64, P, P, I, I, I, P, P, P]),
         "ls_decode_select_workspace_size": (SZ, [I, I]),
         "ls_decode_select": (I, [P, P, P, P, I, I, I, I, I, P, P, P, SZ, P]),
         "ls_prefill_select_workspace_size": (SZ, [I, I]),
@@ -66,6 +68,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_bucket_workspace_size": (SZ, [I, I, I, I]),
         "ls_bucket_select": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
         "ls_selftest_wait_probe": (I, [U64, P, P]),
+        "ls_profile_begin": (I, []),
+        "ls_profile_end": (I, [P]),
+        "ls_profile_kernel": (I, [I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -121,8 +126,11 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 # --------------------------------------------------------------------------- #
 # the library's calls, one Python function per C entry point
 # --------------------------------------------------------------------------- #
-def ls_indexer_score(q, w, keys, key_scale=None, n_valid=None, q_pos=None, stride: int = 4, stream=None):
-    """q [B,T,H,d] bf16, w [B,T,H] f32, keys [B,N,d] (bf16 | float8_e4m3fn | int8) -> scores [B,T,N] f32."""
+def ls_indexer_score(q, w, keys, key_scale=None, n_valid=None, q_pos=None, stride: int = 4, hist_out=None,
+                     stream=None):
+    """q [B,T,H,d] bf16, w [B,T,H] f32, keys [B,N,d] (bf16 | float8_e4m3fn | int8) -> scores [B,T,N] f32.
+
+    hist_out: optional zeroed int32 [B*T, 2048] tensor that receives the selection histogram (T == 1)."""
     _dev(q, torch.bfloat16, "q", 4)
     B, T, H, d = q.shape
     _dev(w, torch.float32, "w", 3)
@@ -139,20 +147,25 @@ def ls_indexer_score(q, w, keys, key_scale=None, n_valid=None, q_pos=None, strid
     _opt(key_scale, torch.float32, "key_scale")
     _opt(n_valid, torch.int32, "n_valid")
     _opt(q_pos, torch.int64, "q_pos")
+    _opt(hist_out, torch.int32, "hist_out")
     out = torch.empty((B, T, N), dtype=torch.float32, device=q.device)
     _check(lib().ls_indexer_score(_ptr(q), _ptr(w), _ptr(keys), kd, _ptr(key_scale), _ptr(n_valid), _ptr(q_pos),
-                                  stride, B, T, H, d, N, _ptr(out), _stream(stream)))
+                                  stride, B, T, H, d, N, _ptr(out), _ptr(hist_out), _stream(stream)))
     return out
 
 
-def ls_topk_select(scores, k: int, n_valid=None, with_values: bool = True, stream=None):
-    """scores [R,N] f32 (row-contiguous) -> (idx [R,k] int32, val [R,k] f32)."""
+def ls_topk_select(scores, k: int, n_valid=None, hist=None, with_values: bool = True, stream=None):
+    """scores [R,N] f32 (row-contiguous) -> (idx [R,k] int32, val [R,k] f32).
+
+    hist: optional int32 [R, 2048] selection histogram of the rows (from ls_indexer_score)."""
     _dev(scores, torch.float32, "scores", 2)
     R, N = scores.shape
     _opt(n_valid, torch.int32, "n_valid")
+    _opt(hist, torch.int32, "hist")
     idx = torch.empty((R, k), dtype=torch.int32, device=scores.device)
     val = torch.empty((R, k), dtype=torch.float32, device=scores.device) if with_values else None
-    _check(lib().ls_topk_select(_ptr(scores), N, _ptr(n_valid), R, N, k, _ptr(idx), _ptr(val), _stream(stream)))
+    _check(lib().ls_topk_select(_ptr(scores), N, _ptr(n_valid), _ptr(hist), R, N, k, _ptr(idx), _ptr(val),
+                                _stream(stream)))
     return idx, val
 
 
@@ -283,3 +296,21 @@ def ls_selftest_wait_probe(limit_ns: int, stream=None) -> torch.Tensor:
     gave_up = torch.zeros(1, dtype=torch.int32, device="cuda")
     _check(lib().ls_selftest_wait_probe(limit_ns, _ptr(gave_up), _stream(stream)))
     return gave_up
+
+
+def ls_profile_begin() -> None:
+    _check(lib().ls_profile_begin())
+
+
+def ls_profile_end() -> dict:
+    """Stop recording; {kernel name: (total ms, launches)} of the library's launches."""
+    n = ctypes.c_int(0)
+    _check(lib().ls_profile_end(ctypes.byref(n)))
+    out = {}
+    for i in range(n.value):
+        name = ctypes.c_char_p()
+        ms = ctypes.c_double()
+        cnt = ctypes.c_longlong()
+        _check(lib().ls_profile_kernel(i, ctypes.byref(name), ctypes.byref(ms), ctypes.byref(cnt)))
+        out[name.value.decode()] = (ms.value, cnt.value)
+    return out

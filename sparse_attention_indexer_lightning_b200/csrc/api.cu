@@ -11,6 +11,8 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "kernels.h"
 #include "ls_indexer.h"
@@ -45,6 +47,46 @@ ls_status fail(ls_status code, const char* fmt, ...) {
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- profiling
+// When recording is on, every kernel launch of the library is bracketed by
+// two CUDA events on its own stream; ls_profile_end() sums the durations per
+// kernel name.
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+struct ProfSum {
+  std::string name;
+  double ms;
+  long long launches;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<ProfSum> g_prof_sums;
+
+struct ProfScope {
+  ProfRec rec{};
+  bool on = false;
+  cudaStream_t st;
+  ProfScope(const char* name, cudaStream_t s) : st(s) {
+    if (!g_prof_on) return;
+    rec.name = name;
+    if (cudaEventCreate(&rec.a) != cudaSuccess) return;
+    if (cudaEventCreate(&rec.b) != cudaSuccess) {
+      cudaEventDestroy(rec.a);
+      return;
+    }
+    on = cudaEventRecord(rec.a, st) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(rec.b, st);
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof_recs.push_back(rec);
+  }
+};
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -98,7 +140,8 @@ cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 // Scores of bf16 keys on the tensor cores (the TMA path).
 ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid,
                      const int64_t* q_pos, int stride, int B, int T, int N, int key_base, int n_total, float* out,
-                     int64_t ld_out, cudaStream_t st) {
+                     int64_t ld_out, cudaStream_t st, uint32_t* hist = nullptr,
+                     const int32_t* lim_rows = nullptr) {
   if (B == 0 || T == 0 || N == 0) return LS_OK;
   const int qg = (T == 1) ? 1 : 8;
   CUtensorMap kmap, qmap;
@@ -118,13 +161,17 @@ ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, co
   p.N = N;
   p.key_base = key_base;
   p.n_total = n_total;
+  p.hist = hist;
+  p.lim_rows = lim_rows;
+  ProfScope prof(qg == 1 ? "score_tc_kernel<1>" : "score_tc_kernel<8>", st);
   LS_CUDA(launch_score_tc(qg, &kmap, &qmap, p, num_sms_current(), st));
   return LS_OK;
 }
 
 ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_total, const float* w,
                         const void* keys, const float* scale, const int32_t* rows, const int32_t* n_valid,
-                        int64_t key_rows, int64_t key_stride, int B, int N, int fmt, float* out, cudaStream_t st) {
+                        int64_t key_rows, int64_t key_stride, int B, int N, int fmt, float* out, cudaStream_t st,
+                        uint32_t* hist = nullptr) {
   if (B == 0 || N == 0) return LS_OK;
   CUtensorMap qmap;
   ls_status s = make_bf16_map(&qmap, q, static_cast<uint64_t>(q_rows_total), kHeads);
@@ -142,13 +189,19 @@ ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_
   p.B = B;
   p.N = N;
   p.fmt = fmt;
+  p.hist = hist;
+  ProfScope prof(fmt == SRC_INT8 ? "score_cvt_kernel<int8>" : fmt == SRC_E4M3 ? "score_cvt_kernel<e4m3>"
+                                                                               : "score_cvt_kernel<bf16>",
+                 st);
   LS_CUDA(launch_score_cvt(&qmap, p, num_sms_current(), st));
   return LS_OK;
 }
 
 ls_status topk(const float* scores, int64_t ld, const int32_t* n_valid, const int32_t* labels, int64_t ld_labels,
-               int R, int N, int k, int32_t* idx, float* val, int64_t ld_out, cudaStream_t st) {
+               int R, int N, int k, int32_t* idx, float* val, int64_t ld_out, cudaStream_t st,
+               const uint32_t* hist = nullptr) {
   TopkParams p;
+  p.hist = hist;
   p.scores = scores;
   p.ld = ld;
   p.n_valid = n_valid;
@@ -160,6 +213,7 @@ ls_status topk(const float* scores, int64_t ld, const int32_t* n_valid, const in
   p.idx_out = idx;
   p.val_out = val;
   p.ld_out = ld_out;
+  ProfScope prof("topk_kernel", st);
   LS_CUDA(launch_topk(p, st));
   return LS_OK;
 }
@@ -196,7 +250,7 @@ ls_status ls_device_status(int* flags, void* stream) {
 
 ls_status ls_indexer_score(const uint16_t* q, const float* w, const void* keys, int key_dtype,
                            const float* key_scale, const int32_t* n_valid, const int64_t* q_pos, int stride,
-                           int B, int T, int H, int d, int N, float* scores, void* stream) {
+                           int B, int T, int H, int d, int N, float* scores, uint32_t* hist_out, void* stream) {
   ls_status s = check_shape(H, d);
   if (s != LS_OK) return s;
   LS_CHECK_ARG(B >= 0 && T >= 0 && N >= 0, "negative size (B=%d T=%d N=%d)", B, T, N);
@@ -204,31 +258,34 @@ ls_status ls_indexer_score(const uint16_t* q, const float* w, const void* keys, 
   LS_CHECK_ARG(q && w && keys && scores, "null tensor pointer");
   LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(keys), "q, w and keys must be 16-byte aligned");
   LS_CHECK_ARG(q_pos == nullptr || stride >= 1, "stride must be >= 1 with q_pos");
+  if (hist_out && T != 1)
+    return fail(LS_ERR_UNSUPPORTED, "hist_out is built for one query per sequence (T == 1)");
   if (key_dtype == LS_KEY_BF16) {
     return score_bf16(q, w, static_cast<const uint16_t*>(keys), n_valid, q_pos, stride, B, T, N, 0, N, scores, N,
-                      S(stream));
+                      S(stream), hist_out);
   }
   LS_CHECK_ARG(key_dtype == LS_KEY_FP8_E4M3 || key_dtype == LS_KEY_INT8, "unknown key_dtype %d", key_dtype);
   LS_CHECK_ARG(key_scale != nullptr, "FP8/INT8 keys need key_scale");
   if (T != 1 || q_pos != nullptr)
     return fail(LS_ERR_UNSUPPORTED, "FP8/INT8 keys are built for one query per sequence without q_pos");
   return score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, keys, key_scale, nullptr, n_valid, N, N, B, N,
-                       key_dtype == LS_KEY_INT8 ? SRC_INT8 : SRC_E4M3, scores, S(stream));
+                       key_dtype == LS_KEY_INT8 ? SRC_INT8 : SRC_E4M3, scores, S(stream), hist_out);
 }
 
-ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, int R, int N, int k,
-                         int32_t* idx_out, float* val_out, void* stream) {
+ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid, const uint32_t* hist, int R,
+                         int N, int k, int32_t* idx_out, float* val_out, void* stream) {
   LS_CHECK_ARG(R >= 0 && N >= 0, "negative size");
   LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
   LS_CHECK_ARG(ld >= N, "ld (%lld) < N (%d)", static_cast<long long>(ld), N);
   if (R == 0) return LS_OK;
   LS_CHECK_ARG(idx_out && (scores || N == 0), "null tensor pointer");
-  return topk(scores, ld, n_valid, nullptr, 0, R, N, k, idx_out, val_out, k, S(stream));
+  return topk(scores, ld, n_valid, nullptr, 0, R, N, k, idx_out, val_out, k, S(stream), hist);
 }
 
 size_t ls_decode_select_workspace_size(int B, int N) {
   if (B <= 0 || N <= 0) return 0;
-  return align_up(static_cast<size_t>(B) * N * sizeof(float));
+  return align_up(static_cast<size_t>(B) * N * sizeof(float)) +
+         align_up(static_cast<size_t>(B) * kHistBins * sizeof(uint32_t));
 }
 
 ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid, int B,
@@ -243,14 +300,17 @@ ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* ke
   const size_t need = ls_decode_select_workspace_size(B, N);
   if (ws_bytes < need || (need && !ws))
     return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
-  float* sc = static_cast<float*>(ws);
+  Carver cv(ws);
+  float* sc = cv.take<float>(static_cast<size_t>(B) * N);
+  uint32_t* hist = cv.take<uint32_t>(static_cast<size_t>(B) * kHistBins);
   if (N > 0) {
     LS_CHECK_ARG(q && w && keys, "null tensor pointer");
     LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(keys), "q, w and keys must be 16-byte aligned");
-    s = score_bf16(q, w, keys, n_valid, nullptr, 1, B, 1, N, 0, N, sc, N, S(stream));
+    LS_CUDA(cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * kHistBins * sizeof(uint32_t), S(stream)));
+    s = score_bf16(q, w, keys, n_valid, nullptr, 1, B, 1, N, 0, N, sc, N, S(stream), hist);
     if (s != LS_OK) return s;
   }
-  return topk(sc, N, n_valid, nullptr, 0, B, N, k, idx_out, val_out, k, S(stream));
+  return topk(sc, N, n_valid, nullptr, 0, B, N, k, idx_out, val_out, k, S(stream), N > 0 ? hist : nullptr);
 }
 
 size_t ls_prefill_select_workspace_size(int T, int N) {
@@ -295,6 +355,10 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
       LS_CUDA(cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming));
     }
     ls_status st = LS_OK;
+    {
+      ProfScope prof("causal_counts_kernel", cs);
+      LS_CUDA(launch_causal_counts(q_pos, T, stride, N, counts, cs));
+    }
     // Earlier work on the compute stream may still read the buffers.
     cudaError_t e = cudaEventRecord(start_ev, cs);
     if (e == cudaSuccess && xs != cs) e = cudaStreamWaitEvent(xs, start_ev, 0);
@@ -313,7 +377,7 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
         if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, copied[slot], 0);
         if (e != cudaSuccess) break;
       }
-      st = score_bf16(q, w, bufs[slot], nullptr, q_pos, stride, 1, T, len, k0, N, sc, N, cs);
+      st = score_bf16(q, w, bufs[slot], nullptr, q_pos, stride, 1, T, len, k0, N, sc, N, cs, nullptr, counts);
       if (st != LS_OK) break;
       if (xs != cs) e = cudaEventRecord(freed[slot], cs);
     }
@@ -330,7 +394,10 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
     if (st != LS_OK) return st;
     if (e != cudaSuccess) return fail(LS_ERR_CUDA, "history streaming: %s", cudaGetErrorString(e));
   }
-  LS_CUDA(launch_causal_counts(q_pos, T, stride, N, counts, cs));
+  if (N == 0) {
+    ProfScope prof("causal_counts_kernel", cs);
+    LS_CUDA(launch_causal_counts(q_pos, T, stride, N, counts, cs));
+  }
   return topk(sc, N, counts, nullptr, 0, T, N, k, idx_out, val_out, k, cs);
 }
 
@@ -338,7 +405,8 @@ size_t ls_two_stage_workspace_size(int B, int N, int shortlist) {
   if (B <= 0 || N <= 0 || shortlist <= 0) return 0;
   return align_up(static_cast<size_t>(B) * N * sizeof(float)) +
          align_up(static_cast<size_t>(B) * shortlist * sizeof(int32_t)) +
-         align_up(static_cast<size_t>(B) * shortlist * sizeof(float));
+         align_up(static_cast<size_t>(B) * shortlist * sizeof(float)) +
+         align_up(static_cast<size_t>(B) * kHistBins * sizeof(uint32_t));
 }
 
 ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const int8_t* ck, const float* ck_scale,
@@ -360,6 +428,7 @@ ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const in
   float* s_hat = cv.take<float>(static_cast<size_t>(B) * N);
   int32_t* short_ws = cv.take<int32_t>(static_cast<size_t>(B) * shortlist);
   float* exact = cv.take<float>(static_cast<size_t>(B) * shortlist);
+  uint32_t* hist = cv.take<uint32_t>(static_cast<size_t>(B) * kHistBins);
   int32_t* sl = shortlist_out ? shortlist_out : short_ws;
   cudaStream_t st = S(stream);
   if (N > 0) {
@@ -367,13 +436,14 @@ ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const in
     LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(ck) && aligned16(fk) && aligned16(ck_scale) &&
                      aligned16(fk_scale),
                  "tensors must be 16-byte aligned");
-    // coarse pass over compact keys
+    // coarse pass over compact keys (also counts the selection histogram)
+    LS_CUDA(cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * kHistBins * sizeof(uint32_t), st));
     s = score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, ck, ck_scale, nullptr, n_valid, N, N, B, N,
-                      SRC_INT8, s_hat, st);
+                      SRC_INT8, s_hat, st, hist);
     if (s != LS_OK) return s;
   }
   // shortlist: top-S positions by coarse score
-  s = topk(s_hat, N, n_valid, nullptr, 0, B, N, shortlist, sl, nullptr, shortlist, st);
+  s = topk(s_hat, N, n_valid, nullptr, 0, B, N, shortlist, sl, nullptr, shortlist, st, N > 0 ? hist : nullptr);
   if (s != LS_OK) return s;
   if (N > 0) {
     // exact re-rank: gather the shortlist's fp8 keys, score with the full query
@@ -422,7 +492,10 @@ ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* ce
   }
   s = topk(cscore, P, nullptr, nullptr, 0, T, P, top_p, picked, nullptr, top_p, st);
   if (s != LS_OK) return s;
-  LS_CUDA(launch_expand(picked, T, top_p, bucket_off, bucket_mem, P, budget, cand, st));
+  {
+    ProfScope prof("expand_kernel", st);
+    LS_CUDA(launch_expand(picked, T, top_p, bucket_off, bucket_mem, P, budget, cand, st));
+  }
   if (N > 0) {
     LS_CHECK_ARG(keys && aligned16(keys), "keys must be a 16-byte aligned device pointer");
     s = score_convert(q, kHeads, static_cast<int64_t>(T) * kHeads, w, keys, nullptr, cand, nullptr, N, 0, T, budget,
@@ -430,6 +503,55 @@ ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* ce
     if (s != LS_OK) return s;
   }
   return topk(exact, budget, nullptr, cand, budget, T, budget, k, idx_out, val_out, k, st);
+}
+
+ls_status ls_profile_begin(void) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  for (auto& r : g_prof_recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof_recs.clear();
+  g_prof_sums.clear();
+  g_prof_on = true;
+  return LS_OK;
+}
+
+ls_status ls_profile_end(int* n_kernels) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = false;
+  g_prof_sums.clear();
+  cudaError_t err = cudaSuccess;
+  for (auto& r : g_prof_recs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess && err == cudaSuccess) err = e;
+    ProfSum* hit = nullptr;
+    for (auto& sum : g_prof_sums)
+      if (sum.name == r.name) hit = &sum;
+    if (!hit) {
+      g_prof_sums.push_back({r.name, 0.0, 0});
+      hit = &g_prof_sums.back();
+    }
+    hit->ms += ms;
+    hit->launches += 1;
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof_recs.clear();
+  if (n_kernels) *n_kernels = static_cast<int>(g_prof_sums.size());
+  if (err != cudaSuccess) return fail(LS_ERR_CUDA, "profiling events: %s", cudaGetErrorString(err));
+  return LS_OK;
+}
+
+ls_status ls_profile_kernel(int i, const char** name, double* total_ms, long long* launches) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  LS_CHECK_ARG(i >= 0 && i < static_cast<int>(g_prof_sums.size()), "kernel index %d out of range", i);
+  if (name) *name = g_prof_sums[i].name.c_str();
+  if (total_ms) *total_ms = g_prof_sums[i].ms;
+  if (launches) *launches = g_prof_sums[i].launches;
+  return LS_OK;
 }
 
 ls_status ls_selftest_wait_probe(uint64_t limit_ns, int* gave_up_dev, void* stream) {

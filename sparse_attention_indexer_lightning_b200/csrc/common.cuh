@@ -207,4 +207,62 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // --------------------------------------------------------------------------
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
+// Weighted-ReLU head reduction of one key's 32 head dot products:
+//   sum_h w[h] * max(0, scale * v[h])
+// with 8 independent partial sums (a single running sum would serialise 32
+// dependent FMAs).  w must be 16-byte aligned.
+template <bool SCALED>
+__device__ __forceinline__ float head_reduce(const float (&v)[32], const float* __restrict__ w, float scale) {
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+  float4 wv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) wv[i] = __ldg(w4 + i);
+  float part[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a0 = SCALED ? scale * v[4 * i + 0] : v[4 * i + 0];
+    const float a1 = SCALED ? scale * v[4 * i + 1] : v[4 * i + 1];
+    const float a2 = SCALED ? scale * v[4 * i + 2] : v[4 * i + 2];
+    const float a3 = SCALED ? scale * v[4 * i + 3] : v[4 * i + 3];
+    float t = wv[i].x * fmaxf(a0, 0.f);
+    t = fmaf(wv[i].y, fmaxf(a1, 0.f), t);
+    t = fmaf(wv[i].z, fmaxf(a2, 0.f), t);
+    t = fmaf(wv[i].w, fmaxf(a3, 0.f), t);
+    part[i] = t;
+  }
+  return ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+}
+
+// Order-preserving 32-bit code of a score: larger score -> larger code;
+// -0.0 and +0.0 share a code; every NaN maps to 0, below -inf.
+__device__ __forceinline__ uint32_t order_code(float f) {
+  uint32_t b = __float_as_uint(f);
+  if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Selection histograms count the top 11 bits of the order code (2048 bins).
+constexpr int kHistBits = 11;
+constexpr int kHistBins = 1 << kHistBits;
+__device__ __forceinline__ uint32_t hist_bin(uint32_t code) { return code >> (32 - kHistBits); }
+
+// Named barrier over the `count` threads of a role (id 0 is __syncthreads).
+__device__ __forceinline__ void role_barrier(int id, int count) {
+  __syncwarp();
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Shared-memory histogram of one row's scores, flushed into the row's global
+// histogram by the threads of a role when the row changes or the CTA ends.
+__device__ __forceinline__ void flush_hist(uint32_t* shist, uint32_t* ghist_row, int tid_in_role, int role_threads) {
+  for (int i = tid_in_role; i < kHistBins; i += role_threads) {
+    const uint32_t v = shist[i];
+    if (v) {
+      atomicAdd(ghist_row + i, v);
+      shist[i] = 0;
+    }
+  }
+}
+
 }  // namespace lsi

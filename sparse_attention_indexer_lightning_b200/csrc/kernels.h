@@ -31,6 +31,8 @@ struct ScoreParams {
   int B, T, N;
   int key_base;
   int n_total;             // causal cap: number of keys of the whole history
+  uint32_t* hist;          // [B*T][2048] selection histogram (counts added) or nullptr; qg == 1 only
+  const int32_t* lim_rows; // [B*T] eligible keys of the whole history per query (replaces q_pos) or nullptr
 };
 
 // qg = queries sharing one MMA B tile: 1 (one query per sequence) or 8.
@@ -57,6 +59,7 @@ struct CvtParams {
   int64_t q_row_stride;    // q rows per problem (H for one query per problem)
   int B, N;
   int fmt;
+  uint32_t* hist;          // [B][2048] selection histogram (counts added) or nullptr
 };
 cudaError_t launch_score_cvt(const CUtensorMap* qmap, const CvtParams& p, int num_sms, cudaStream_t st);
 
@@ -68,6 +71,8 @@ struct TopkParams {
   const int32_t* n_valid;  // [R] or nullptr: columns >= n_valid[r] are absent
   const int32_t* labels;   // [R][ld_labels] or nullptr; label < 0 = absent
   int64_t ld_labels;
+  const uint32_t* hist;    // [R][2048] counts of the top 11 order-code bits of the
+                           // present entries (from the scoring epilogue) or nullptr
   int R, N, k;
   int32_t* idx_out;        // [R][k] labels, -1 padding
   float* val_out;          // [R][k] values (bit copies), -inf padding; may be nullptr

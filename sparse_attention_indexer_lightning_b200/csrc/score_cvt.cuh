@@ -14,13 +14,14 @@
 // values fit bf16's 8-bit significand and exponent range), so the contraction
 // runs as a bf16 x bf16 -> fp32 tcgen05 MMA with one key per TMEM lane.
 //
-// Roles (320 threads, one persistent CTA per SM):
+// Roles (448 threads, one persistent CTA per SM):
 //   warp 0      producer: 1-D bulk copies of raw rows (one copy per tile when
 //               contiguous, one per row when gathered) + TMA of the query tile
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2-5   converters: raw rows -> bf16 in the 128-byte-swizzled K-major
+//   warps 2-9   converters: raw rows -> bf16 in the 128-byte-swizzled K-major
 //               layout the MMA descriptor expects
-//   warps 6-9   epilogue: scale, ReLU, head weights, head sum, store
+//   warps 10-13 epilogue: scale, ReLU, head weights, head sum, store (the next
+//               unit's row ids and scales are loaded one unit ahead)
 // All waits are bounded (see common.cuh).
 
 #pragma once
@@ -44,14 +45,15 @@ struct CvtCfg {
   static constexpr int AS = 3;                            // converted stages
   static constexpr int ACC = 2;
   static constexpr int TMEM_COLS = 64;
-  static constexpr int CVT_WARPS = 4;
+  static constexpr int CVT_WARPS = 8;
   static constexpr int EPI_WARPS = 4;
   static constexpr int THREADS = (2 + CVT_WARPS + EPI_WARPS) * 32;
   static constexpr size_t SMEM_RAW = size_t(RS) * RAW_BYTES;
   static constexpr size_t SMEM_A = size_t(AS) * A_BYTES;
   static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
   static constexpr size_t SMEM_BAR = 512;
-  static constexpr size_t SMEM_TOTAL = 1024 + SMEM_RAW + SMEM_A + SMEM_B + SMEM_BAR;
+  static constexpr size_t SMEM_HIST = kHistBins * 4;
+  static constexpr size_t SMEM_TOTAL = 1024 + SMEM_RAW + SMEM_A + SMEM_B + SMEM_BAR + SMEM_HIST;
   static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
 };
 
@@ -80,17 +82,21 @@ __device__ __forceinline__ void cvt_wait_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// 4 signed bytes -> 4 exact floats via the 2^23 magic number.
+// 4 signed bytes -> 4 bf16, exactly.  For a byte v = sign*128 + m (m < 128)
+// the bf16 pattern 0x4300 | m is 128 + m, and 0x4300 | (v & 0x80) is 128 or
+// 256; their bf16 difference m - sign*128 = v is representable, so the
+// packed subtraction is exact.
 __device__ __forceinline__ void i8x4_to_bf16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
-  const uint32_t y = x ^ 0x80808080u;  // bias to unsigned: byte = v + 128
-  const float f0 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7540)) - 8388736.f;
-  const float f1 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7541)) - 8388736.f;
-  const float f2 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7542)) - 8388736.f;
-  const float f3 = __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7543)) - 8388736.f;
-  __nv_bfloat162 a = __floats2bfloat162_rn(f0, f1);
-  __nv_bfloat162 b = __floats2bfloat162_rn(f2, f3);
-  lo = *reinterpret_cast<uint32_t*>(&a);
-  hi = *reinterpret_cast<uint32_t*>(&b);
+  const uint32_t t0 = __byte_perm(x, 0u, 0x4140);  // bytes 0,1 into the low byte of each half
+  const uint32_t t1 = __byte_perm(x, 0u, 0x4342);  // bytes 2,3
+  const uint32_t m0 = (t0 & 0x007F007Fu) | 0x43004300u, o0 = (t0 & 0x00800080u) | 0x43004300u;
+  const uint32_t m1 = (t1 & 0x007F007Fu) | 0x43004300u, o1 = (t1 & 0x00800080u) | 0x43004300u;
+  __nv_bfloat162 r0 = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&m0),
+                              *reinterpret_cast<const __nv_bfloat162*>(&o0));
+  __nv_bfloat162 r1 = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&m1),
+                              *reinterpret_cast<const __nv_bfloat162*>(&o1));
+  lo = *reinterpret_cast<uint32_t*>(&r0);
+  hi = *reinterpret_cast<uint32_t*>(&r1);
 }
 
 // 2 e4m3 codes (low 16 bits of x, element 0 in the low byte) -> bf16x2, exact.
@@ -118,7 +124,11 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
   uint8_t* sA = smem + C::SMEM_RAW;
   uint8_t* sB = sA + C::SMEM_A;
   CvtBarriers* bars = reinterpret_cast<CvtBarriers*>(sB + C::SMEM_B);
+  uint32_t* shist = reinterpret_cast<uint32_t*>(sB + C::SMEM_B + C::SMEM_BAR);
   volatile int* abort_flag = &bars->abort_flag;
+  const bool use_hist = p.hist != nullptr;
+  if (use_hist)
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) shist[i] = 0;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -283,7 +293,8 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     }
   } else if (warp < 2 + C::CVT_WARPS) {
     // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - 64;  // 0..127
+    constexpr int CT = C::CVT_WARPS * 32;
+    const int ct = threadIdx.x - 64;  // 0 .. CT-1
     int rs = 0, as = 0;
     uint32_t rphase = 0, aphase = 0;
     for (long long u = u_begin; u < u_end; ++u) {
@@ -292,31 +303,43 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
       const uint8_t* raw = sR + rs * C::RAW_BYTES;
       uint8_t* a = sA + as * C::A_BYTES;
       if (FMT == SRC_BF16) {
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int id = i * 128 + ct;
+        constexpr int PER = (C::BM * 16) / CT;  // 16-byte chunks per thread
+        uint4 v[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int id = i * CT + ct;
+          v[i] = *reinterpret_cast<const uint4*>(raw + (id >> 4) * 256 + (id & 15) * 16);
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int id = i * CT + ct;
           const int row = id >> 4, cc = id & 15;
-          const uint4 v = *reinterpret_cast<const uint4*>(raw + row * 256 + cc * 16);
           const int panel = cc >> 3, j = cc & 7;
-          *reinterpret_cast<uint4*>(a + panel * C::A_HALF + row * 128 + ((j ^ (row & 7)) << 4)) = v;
+          *reinterpret_cast<uint4*>(a + panel * C::A_HALF + row * 128 + ((j ^ (row & 7)) << 4)) = v[i];
         }
       } else {
-#pragma unroll 2
-        for (int i = 0; i < 8; ++i) {
-          const int id = i * 128 + ct;
+        constexpr int PER = (C::BM * 8) / CT;
+        uint4 v[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int id = i * CT + ct;
+          v[i] = *reinterpret_cast<const uint4*>(raw + (id >> 3) * 128 + (id & 7) * 16);
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int id = i * CT + ct;
           const int row = id >> 3, cc = id & 7;
-          const uint4 v = *reinterpret_cast<const uint4*>(raw + row * 128 + cc * 16);
           uint4 o0, o1;
           if (FMT == SRC_INT8) {
-            i8x4_to_bf16x4(v.x, o0.x, o0.y);
-            i8x4_to_bf16x4(v.y, o0.z, o0.w);
-            i8x4_to_bf16x4(v.z, o1.x, o1.y);
-            i8x4_to_bf16x4(v.w, o1.z, o1.w);
+            i8x4_to_bf16x4(v[i].x, o0.x, o0.y);
+            i8x4_to_bf16x4(v[i].y, o0.z, o0.w);
+            i8x4_to_bf16x4(v[i].z, o1.x, o1.y);
+            i8x4_to_bf16x4(v[i].w, o1.z, o1.w);
           } else {
-            e4m3x4_to_bf16x4(v.x, o0.x, o0.y);
-            e4m3x4_to_bf16x4(v.y, o0.z, o0.w);
-            e4m3x4_to_bf16x4(v.z, o1.x, o1.y);
-            e4m3x4_to_bf16x4(v.w, o1.z, o1.w);
+            e4m3x4_to_bf16x4(v[i].x, o0.x, o0.y);
+            e4m3x4_to_bf16x4(v[i].y, o0.z, o0.w);
+            e4m3x4_to_bf16x4(v[i].z, o1.x, o1.y);
+            e4m3x4_to_bf16x4(v[i].w, o1.z, o1.w);
           }
           const int panel = cc >> 2;
           const int j0 = (cc & 3) * 2;
@@ -336,12 +359,38 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    constexpr int EPI0 = (2 + C::CVT_WARPS) * 32;  // first epilogue thread
     const int quad = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
+    // what the epilogue needs from global memory besides TMEM, for one unit
+    auto fetch = [&](long long u, bool& valid, float& sc) {
+      const int tile = static_cast<int>(u % NT);
+      const int b = static_cast<int>(u / NT);
+      const int j = tile * C::BM + quad * 32 + lane;
+      valid = false;
+      sc = 1.f;
+      if (j >= p.N) return;
+      int64_t sidx;
+      if (p.rows) {
+        const int32_t r = __ldg(p.rows + static_cast<int64_t>(b) * p.N + j);
+        valid = (r >= 0) && (r < p.key_rows);
+        sidx = static_cast<int64_t>(b) * p.key_stride + (valid ? r : 0);
+      } else {
+        valid = (p.n_valid == nullptr) || (j < __ldg(p.n_valid + b));
+        sidx = static_cast<int64_t>(b) * p.N + j;
+      }
+      if (FMT != SRC_BF16 && valid) sc = __ldg(p.scale + sidx);
+    };
+    bool nvalid = false;
+    float nsc = 1.f;
+    if (u_begin < u_end) fetch(u_begin, nvalid, nsc);
     for (long long u = u_begin; u < u_end; ++u) {
       const int tile = static_cast<int>(u % NT);
       const int b = static_cast<int>(u / NT);
+      const bool valid = nvalid;
+      const float sc = nsc;
+      if (u + 1 < u_end) fetch(u + 1, nvalid, nsc);  // in flight while this unit waits and computes
       if (!mbar_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const int j = tile * C::BM + quad * 32 + lane;
@@ -351,33 +400,21 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->tempty[acc]);
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
-      if (j >= p.N) continue;
-      bool valid;
-      int64_t sidx;
-      if (p.rows) {
-        const int32_t r = p.rows[static_cast<int64_t>(b) * p.N + j];
-        valid = (r >= 0) && (r < p.key_rows);
-        sidx = static_cast<int64_t>(b) * p.key_stride + (valid ? r : 0);
-      } else {
-        valid = (p.n_valid == nullptr) || (j < p.n_valid[b]);
-        sidx = static_cast<int64_t>(b) * p.N + j;
-      }
-      float s = neg_inf();
-      if (valid) {
-        const float sc = (FMT == SRC_BF16) ? 1.f : __ldg(p.scale + sidx);
-        const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * kHeads);
-        float acc_s = 0.f;
-#pragma unroll
-        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
-          const float4 wv = __ldg(w4 + h4);
-          acc_s = fmaf(wv.x, fmaxf(sc * v[4 * h4 + 0], 0.f), acc_s);
-          acc_s = fmaf(wv.y, fmaxf(sc * v[4 * h4 + 1], 0.f), acc_s);
-          acc_s = fmaf(wv.z, fmaxf(sc * v[4 * h4 + 2], 0.f), acc_s);
-          acc_s = fmaf(wv.w, fmaxf(sc * v[4 * h4 + 3], 0.f), acc_s);
+      const bool last_of_row = (u + 1 == u_end) || ((u + 1) / NT != b);
+      if (j < p.N) {
+        float s = neg_inf();
+        if (valid) {
+          const float* wrow = p.w + static_cast<int64_t>(b) * kHeads;
+          s = (FMT == SRC_BF16) ? head_reduce<false>(v, wrow, 1.f) : head_reduce<true>(v, wrow, sc);
+          if (use_hist) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
         }
-        s = acc_s;
+        p.out[static_cast<int64_t>(b) * p.N + j] = s;
       }
-      p.out[static_cast<int64_t>(b) * p.N + j] = s;
+      if (use_hist && last_of_row) {  // warp-uniform: every epilogue warp sees the same unit
+        role_barrier(1, C::EPI_WARPS * 32);
+        flush_hist(shist, p.hist + static_cast<int64_t>(b) * kHistBins, threadIdx.x - EPI0, C::EPI_WARPS * 32);
+        role_barrier(1, C::EPI_WARPS * 32);
+      }
     }
   }
 

@@ -49,7 +49,8 @@ struct TcCfg {
   static constexpr size_t SMEM_A = size_t(STAGES) * A_BYTES;
   static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
   static constexpr size_t SMEM_BAR = 512;
-  static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR;
+  static constexpr size_t SMEM_HIST = (QG == 1) ? kHistBins * 4 : 0;  // per-row selection histogram
+  static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR + SMEM_HIST;
   static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
 };
 
@@ -87,7 +88,11 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::SMEM_A;
   TcBarriers* bars = reinterpret_cast<TcBarriers*>(smem + C::SMEM_A + C::SMEM_B);
+  uint32_t* shist = reinterpret_cast<uint32_t*>(smem + C::SMEM_A + C::SMEM_B + C::SMEM_BAR);
   volatile int* abort_flag = &bars->abort_flag;
+  const bool use_hist = (QG == 1) && (p.hist != nullptr);
+  if (use_hist)
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) shist[i] = 0;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -247,18 +252,12 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
                                static_cast<uint32_t>(acc * C::ACC_COLS + j * kHeads);
         float v[32];
         tmem_ld_32x32(taddr, v);
-        const float4* w4 = reinterpret_cast<const float4*>(p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads);
-        float s = 0.f;
-#pragma unroll
-        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
-          const float4 wv = __ldg(w4 + h4);
-          s = fmaf(wv.x, fmaxf(v[4 * h4 + 0], 0.f), s);
-          s = fmaf(wv.y, fmaxf(v[4 * h4 + 1], 0.f), s);
-          s = fmaf(wv.z, fmaxf(v[4 * h4 + 2], 0.f), s);
-          s = fmaf(wv.w, fmaxf(v[4 * h4 + 3], 0.f), s);
-        }
+        const float s = head_reduce<false>(v, p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads, 1.f);
         int lim_t = lim;
-        if (p.q_pos) {
+        if (p.lim_rows) {
+          const int rel = p.lim_rows[static_cast<int64_t>(b) * p.T + t] - p.key_base;
+          lim_t = rel < 0 ? 0 : (rel < lim_t ? rel : lim_t);
+        } else if (p.q_pos) {
           const int64_t qp = p.q_pos[static_cast<int64_t>(b) * p.T + t];
           int64_t e = qp < 0 ? 0 : (qp + 1) / p.stride;
           if (e > p.n_total) e = p.n_total;
@@ -267,12 +266,19 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
         }
         if (n < p.N) {
           p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
+          if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->tempty[acc]);
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
+      if (use_hist && (u + 1 == u_end || (u + 1) / NT != bg)) {
+        // the row (one query per sequence here) ends in this CTA: publish its counts
+        role_barrier(1, C::EPI_WARPS * 32);
+        flush_hist(shist, p.hist + static_cast<int64_t>(b) * p.T * kHistBins, ew * 32 + lane, C::EPI_WARPS * 32);
+        role_barrier(1, C::EPI_WARPS * 32);
+      }
     }
   }
 

@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_workspace_queries(lib):
     assert lib.ls_version() == 100
-    assert lib.ls_decode_select_workspace_size(64, 32768) == 64 * 32768 * 4
+    assert lib.ls_decode_select_workspace_size(64, 32768) == 64 * 32768 * 4 + 64 * 2048 * 4
     assert lib.ls_prefill_select_workspace_size(4096, 32768) >= 4096 * 32768 * 4 + 4096 * 4
     assert lib.ls_two_stage_workspace_size(32, 131072, 4096) >= 32 * 131072 * 4 + 2 * 32 * 4096 * 4
     assert lib.ls_bucket_workspace_size(256, 32768, 64, 512) >= 256 * 32768 * 4
@@ -52,22 +52,25 @@ def test_argument_checks_without_gpu(lib):
     P = ctypes.c_void_p
     dummy = P(16)
     # H != 32 is not built
-    st = lib.ls_indexer_score(dummy, dummy, dummy, 0, None, None, None, 4, 1, 1, 16, 128, 64, dummy, None)
+    st = lib.ls_indexer_score(dummy, dummy, dummy, 0, None, None, None, 4, 1, 1, 16, 128, 64, dummy, None, None)
     assert st == 3
     assert b"H=32" in lib.ls_last_error()
     # k out of range
-    assert lib.ls_topk_select(dummy, 10, None, 1, 10, 0, dummy, None, None) == 1
-    assert lib.ls_topk_select(dummy, 10, None, 1, 10, 5000, dummy, None, None) == 1
+    assert lib.ls_topk_select(dummy, 10, None, None, 1, 10, 0, dummy, None, None) == 1
+    assert lib.ls_topk_select(dummy, 10, None, None, 1, 10, 5000, dummy, None, None) == 1
     # ld < N
-    assert lib.ls_topk_select(dummy, 5, None, 1, 10, 3, dummy, None, None) == 1
+    assert lib.ls_topk_select(dummy, 5, None, None, 1, 10, 3, dummy, None, None) == 1
     # short workspace
     st = lib.ls_decode_select(dummy, dummy, dummy, None, 2, 32, 128, 100, 8, dummy, None, dummy, 10, None)
     assert st == 2
     # unknown key dtype / misaligned pointers
-    st = lib.ls_indexer_score(dummy, dummy, dummy, 9, None, None, None, 4, 1, 1, 32, 128, 64, dummy, None)
+    st = lib.ls_indexer_score(dummy, dummy, dummy, 9, None, None, None, 4, 1, 1, 32, 128, 64, dummy, None, None)
     assert st == 1
-    st = lib.ls_indexer_score(P(17), dummy, dummy, 0, None, None, None, 4, 1, 1, 32, 128, 64, dummy, None)
+    st = lib.ls_indexer_score(P(17), dummy, dummy, 0, None, None, None, 4, 1, 1, 32, 128, 64, dummy, None, None)
     assert st == 1
+    # the selection histogram is built for one query per sequence
+    st = lib.ls_indexer_score(dummy, dummy, dummy, 0, None, None, None, 4, 1, 2, 32, 128, 64, dummy, dummy, None)
+    assert st == 3
     # two-stage: shortlist shorter than k
     st = lib.ls_decode_two_stage_select(dummy, dummy, dummy, dummy, dummy, dummy, None, 1, 32, 128, 100, 256, 512,
                                         dummy, None, None, dummy, 1 << 30, None)
@@ -77,4 +80,9 @@ def test_argument_checks_without_gpu(lib):
                               None, None, dummy, 1 << 30, None)
     assert st == 1
     # empty problems are a no-op
-    assert lib.ls_indexer_score(None, None, None, 0, None, None, None, 4, 0, 1, 32, 128, 64, None, None) == 0
+    assert lib.ls_indexer_score(None, None, None, 0, None, None, None, 4, 0, 1, 32, 128, 64, None, None, None) == 0
+    # profiling with nothing recorded
+    n = ctypes.c_int(-1)
+    assert lib.ls_profile_begin() == 0
+    assert lib.ls_profile_end(ctypes.byref(n)) == 0 and n.value == 0
+    assert lib.ls_profile_kernel(0, None, None, None) == 1

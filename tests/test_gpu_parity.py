@@ -338,3 +338,56 @@ def test_wait_probe_times_out_and_context_survives(L):
     assert flags & 1
     # the context is still usable
     test_decode_edge_rows(L)
+
+
+# --------------------------------------------------------------------------- #
+# the selection histogram the scans count for the top-k
+# --------------------------------------------------------------------------- #
+def _order_codes(x):
+    """Order-preserving codes of fp32 scores, restated here for the check:
+    NaN -> 0, -0.0 -> code of +0.0, negatives bit-inverted, positives with the
+    sign bit set."""
+    x = np.asarray(x, np.float32)
+    b = x.view(np.uint32).copy()
+    b[b == 0x80000000] = 0
+    code = np.where(b & 0x80000000, ~b, b | 0x80000000).astype(np.uint32)
+    code[np.isnan(x)] = 0
+    return code
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "int8"])
+def test_scan_histogram_feeds_topk(L, fmt):
+    name = "decode_s" if fmt == "bf16" else "two_stage_s"
+    d = data(name)
+    B, H, dd = d["q"].shape
+    q, w, nv = dev_bf16(d["q"]), dev(d["w"]), dev(d["n_valid"])
+    hist = torch.zeros((B, 2048), dtype=torch.int32, device="cuda")
+    if fmt == "bf16":
+        sc = L.ls_indexer_score(q.view(B, 1, H, dd), w.view(B, 1, H), dev_bf16(d["k"]), n_valid=nv, hist_out=hist)
+    else:
+        sc = L.ls_indexer_score(q.view(B, 1, H, dd), w.view(B, 1, H), dev(d["ck"]), key_scale=dev(d["ck_scale"]),
+                                n_valid=nv, hist_out=hist)
+    sc = sc[:, 0].contiguous()
+    s_np = sc.cpu().numpy()
+    h_np = hist.cpu().numpy()
+    for b in range(B):
+        n = int(d["n_valid"][b])
+        ref = np.bincount(_order_codes(s_np[b, :n]) >> 21, minlength=2048)
+        assert np.array_equal(h_np[b], ref), f"histogram row {b}"
+    for k in (1, 512, 1024):
+        i1, v1 = L.ls_topk_select(sc, k, n_valid=nv, hist=hist)
+        i0, v0 = L.ls_topk_select(sc, k, n_valid=nv)
+        ri, rv = topk_rows(s_np, d["n_valid"], k)
+        assert np.array_equal(i1.cpu().numpy(), ri) and f32_bits_equal(v1.cpu().numpy(), rv)
+        assert np.array_equal(i0.cpu().numpy(), ri) and f32_bits_equal(v0.cpu().numpy(), rv)
+
+
+def test_profiling_counts_launches(L):
+    d = data("decode_tiny")
+    q, w, k = dev_bf16(d["q"]), dev(d["w"]), dev_bf16(d["k"])
+    L.ls_profile_begin()
+    for _ in range(3):
+        L.ls_decode_select(q, w, k, 512)
+    prof = L.ls_profile_end()
+    assert prof["score_tc_kernel<1>"][1] == 3 and prof["topk_kernel"][1] == 3
+    assert all(ms > 0 for ms, _ in prof.values())
