@@ -115,7 +115,9 @@ class ClockSampler:
 # --------------------------------------------------------------------------- #
 # distributed plumbing
 # --------------------------------------------------------------------------- #
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun env).  backend "gloo" drives the same
+    host logic on CPU (tests)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -123,10 +125,13 @@ def dist_setup(n_gpus: int):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -138,13 +143,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank time over all ranks (device tensor under NCCL)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, ms_per_step_max: float, world: int) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's step time."""
+    return world * units_per_rank / (ms_per_step_max * 1e-3)
 
 
 # --------------------------------------------------------------------------- #
@@ -232,7 +245,7 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
     topk_ms = prof["topk_kernel"][0] / prof["topk_kernel"][1]
     launches = sum(c for _, c in prof.values())
     positions = B * N
-    value = world * positions / (ms_per_step * 1e-3)
+    value = weak_scaling_value(positions, ms_per_step, world)
     key_bytes = B * N * dd * 2
     out = {
         "metric": "indexer query-positions scored/sec (decode selection, top-512)",

@@ -306,11 +306,13 @@ ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* ke
   if (N > 0) {
     LS_CHECK_ARG(q && w && keys, "null tensor pointer");
     LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(keys), "q, w and keys must be 16-byte aligned");
-    LS_CUDA(cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * kHistBins * sizeof(uint32_t), S(stream)));
-    s = score_bf16(q, w, keys, n_valid, nullptr, 1, B, 1, N, 0, N, sc, N, S(stream), hist);
+    // The top-k samples its own threshold; counting a histogram in the scan
+    // epilogue costs the scan more than it saves the selection.
+    (void)hist;
+    s = score_bf16(q, w, keys, n_valid, nullptr, 1, B, 1, N, 0, N, sc, N, S(stream));
     if (s != LS_OK) return s;
   }
-  return topk(sc, N, n_valid, nullptr, 0, B, N, k, idx_out, val_out, k, S(stream), N > 0 ? hist : nullptr);
+  return topk(sc, N, n_valid, nullptr, 0, B, N, k, idx_out, val_out, k, S(stream));
 }
 
 size_t ls_prefill_select_workspace_size(int T, int N) {
@@ -436,14 +438,14 @@ ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const in
     LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(ck) && aligned16(fk) && aligned16(ck_scale) &&
                      aligned16(fk_scale),
                  "tensors must be 16-byte aligned");
-    // coarse pass over compact keys (also counts the selection histogram)
-    LS_CUDA(cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * kHistBins * sizeof(uint32_t), st));
+    // coarse pass over compact keys
+    (void)hist;
     s = score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, ck, ck_scale, nullptr, n_valid, N, N, B, N,
-                      SRC_INT8, s_hat, st, hist);
+                      SRC_INT8, s_hat, st);
     if (s != LS_OK) return s;
   }
   // shortlist: top-S positions by coarse score
-  s = topk(s_hat, N, n_valid, nullptr, 0, B, N, shortlist, sl, nullptr, shortlist, st, N > 0 ? hist : nullptr);
+  s = topk(s_hat, N, n_valid, nullptr, 0, B, N, shortlist, sl, nullptr, shortlist, st);
   if (s != LS_OK) return s;
   if (N > 0) {
     // exact re-rank: gather the shortlist's fp8 keys, score with the full query
@@ -561,3 +563,4 @@ ls_status ls_selftest_wait_probe(uint64_t limit_ns, int* gave_up_dev, void* stre
 }
 
 }  // extern "C"
+

@@ -89,6 +89,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Warp-uniform bounded wait: lane 0 waits, every lane gets its verdict, so
+// warp-collective instructions after the wait never see a partial warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 // --------------------------------------------------------------------------
 // TMA
 // --------------------------------------------------------------------------
@@ -179,6 +187,33 @@ __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// The same load without the wait; tmem_wait_ld() must follow before any use of
+// r.  The wait names the registers as read-write operands, so the compiler
+// cannot move a consumer of r above it.
+__device__ __forceinline__ void tmem_ld_32x32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                 "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                 "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored with the
 // 128-byte swizzle: rows of 128 B (64 bf16), 8-row groups 1024 B apart.
 // Bits: start>>4 [0,14), LBO>>4 [16,30) (unused for this layout, 1),
@@ -205,32 +240,94 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // --------------------------------------------------------------------------
 // small helpers
 // --------------------------------------------------------------------------
+
+// Position of a persistent CTA in its contiguous run of work units, ordered
+// problem (b), then query group (g), then key tile; advanced without division.
+struct UnitPos {
+  int tile, g, b;
+  __device__ __forceinline__ void init(long long u0, int NT, int G) {
+    tile = static_cast<int>(u0 % NT);
+    const long long bg = u0 / NT;
+    g = static_cast<int>(bg % G);
+    b = static_cast<int>(bg / G);
+  }
+  __device__ __forceinline__ void next(int NT, int G) {
+    if (++tile == NT) {
+      tile = 0;
+      if (++g == G) {
+        g = 0;
+        ++b;
+      }
+    }
+  }
+};
+
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+// d += a * b on a pair of fp32 lanes (packed fp32x2 FMA of sm_100a).
+__device__ __forceinline__ void ffma2_acc(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 
 // Weighted-ReLU head reduction of one key's 32 head dot products:
 //   sum_h w[h] * max(0, scale * v[h])
-// with 8 independent partial sums (a single running sum would serialise 32
-// dependent FMAs).  w must be 16-byte aligned.
+// with 8 independent partial sums updated two at a time by packed FMAs (a
+// single running sum would serialise 32 dependent FMAs).  w must be 16-byte
+// aligned.
 template <bool SCALED>
 __device__ __forceinline__ float head_reduce(const float (&v)[32], const float* __restrict__ w, float scale) {
   const float4* w4 = reinterpret_cast<const float4*>(w);
   float4 wv[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) wv[i] = __ldg(w4 + i);
-  float part[8];
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float a0 = SCALED ? scale * v[4 * i + 0] : v[4 * i + 0];
-    const float a1 = SCALED ? scale * v[4 * i + 1] : v[4 * i + 1];
-    const float a2 = SCALED ? scale * v[4 * i + 2] : v[4 * i + 2];
-    const float a3 = SCALED ? scale * v[4 * i + 3] : v[4 * i + 3];
-    float t = wv[i].x * fmaxf(a0, 0.f);
-    t = fmaf(wv[i].y, fmaxf(a1, 0.f), t);
-    t = fmaf(wv[i].z, fmaxf(a2, 0.f), t);
-    t = fmaf(wv[i].w, fmaxf(a3, 0.f), t);
-    part[i] = t;
+    const float a0 = fmaxf(SCALED ? scale * v[4 * i + 0] : v[4 * i + 0], 0.f);
+    const float a1 = fmaxf(SCALED ? scale * v[4 * i + 1] : v[4 * i + 1], 0.f);
+    const float a2 = fmaxf(SCALED ? scale * v[4 * i + 2] : v[4 * i + 2], 0.f);
+    const float a3 = fmaxf(SCALED ? scale * v[4 * i + 3] : v[4 * i + 3], 0.f);
+    const int p = (2 * i) & 7;
+    ffma2_acc(acc[p], acc[p + 1], a0, a1, wv[i].x, wv[i].y);
+    const int q = (2 * i + 2) & 7;
+    ffma2_acc(acc[q], acc[q + 1], a2, a3, wv[i].z, wv[i].w);
   }
-  return ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+// head_reduce with the 32 head weights already in registers.
+__device__ __forceinline__ float head_reduce_w(const uint32_t (&r)[32], const float (&w)[32]) {
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int h = 0; h < 32; h += 2) {
+    const int p = h & 7;
+    ffma2_acc(acc[p], acc[p + 1], fmaxf(__uint_as_float(r[h]), 0.f), fmaxf(__uint_as_float(r[h + 1]), 0.f), w[h],
+              w[h + 1]);
+  }
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+// sum_h w[h] * max(0, sc * v[h]) for a per-key scale sc of either sign:
+// = |sc| * sum_h w[h] * max(0, sign(sc) * v[h]).  The sign is uniform across a
+// warp in practice (scales are magnitudes), so the branch does not diverge.
+__device__ __forceinline__ float head_reduce_scaled(const uint32_t (&r)[32], const float (&w)[32], float sc) {
+  float base;
+  if (sc >= 0.f) {
+    base = head_reduce_w(r, w);
+  } else {
+    uint32_t neg[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) neg[i] = r[i] ^ 0x80000000u;
+    base = head_reduce_w(neg, w);
+  }
+  return fabsf(sc) * base;
 }
 
 // Order-preserving 32-bit code of a score: larger score -> larger code;

@@ -180,12 +180,25 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     int b_issued[2] = {0, 0};
     uint32_t b_par[2] = {0, 0};
     bool ok = true;
-    for (long long u = u_begin; u < u_end; ++u) {
-      const int tile = static_cast<int>(u % NT);
-      const int b = static_cast<int>(u / NT);
+    // gathered form: row ids of a unit's tile (-1 past the end)
+    auto load_rids = [&](int tb, int ttile, int32_t (&out)[4]) {
+      const int jb = ttile * C::BM;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = jb + lane + 32 * i;
+        out[i] = (j < p.N) ? __ldg(p.rows + static_cast<int64_t>(tb) * p.N + j) : -1;
+      }
+    };
+    int32_t rid_next[4] = {-1, -1, -1, -1};
+    UnitPos up;
+    up.init(u_begin, NT, 1);
+    if (p.rows != nullptr && u_begin < u_end) load_rids(up.b, up.tile, rid_next);
+    for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
+      const int tile = up.tile;
+      const int b = up.b;
       if (b != prev_b) {
         bslot ^= 1;
-        if (!mbar_wait(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
+        if (!warp_wait(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
         b_par[bslot] = bphase[bslot];
         b_issued[bslot] = 1;
         bphase[bslot] ^= 1;
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
         }
         prev_b = b;
       }
-      if (!mbar_wait(&bars->rempty[rs], rphase ^ 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(&bars->rempty[rs], rphase ^ 1, abort_flag)) { ok = false; break; }
       uint8_t* dst = sR + rs * C::RAW_BYTES;
       const int j0 = tile * C::BM;
       const int nrows = min(C::BM, p.N - j0);
@@ -210,20 +223,24 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
           bulk_load(dst, src, bytes, &bars->rfull[rs]);
         }
       } else {
-        // gathered: lane l copies rows l, l+32, l+64, l+96 of the tile
+        // gathered: lane l copies rows l, l+32, l+64, l+96 of the tile; the
+        // row ids of the next unit are read now, so their latency overlaps
+        // this unit's copies
         int32_t rid[4];
         int cnt = 0;
 #pragma unroll
+        for (int i = 0; i < 4; ++i) rid[i] = rid_next[i];
+        if (u + 1 < u_end) {
+          if (tile + 1 == NT) load_rids(b + 1, 0, rid_next);
+          else load_rids(b, tile + 1, rid_next);
+        }
+#pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int j = j0 + lane + 32 * i;
-          int32_t r = -1;
-          if (j < p.N) r = p.rows[static_cast<int64_t>(b) * p.N + j];
-          if (r >= p.key_rows) {
+          if (rid[i] >= p.key_rows) {
             atomicOr(&g_fault, FAULT_BAD_INDEX);
-            r = -1;
+            rid[i] = -1;
           }
-          rid[i] = r;
-          cnt += (r >= 0);
+          cnt += (rid[i] >= 0);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
@@ -260,8 +277,10 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
       uint32_t bphase[2] = {0, 0};
       const uint32_t a_base = smem_u32(sA);
       const uint32_t b_base = smem_u32(sB);
-      for (long long u = u_begin; u < u_end; ++u) {
-        const int b = static_cast<int>(u / NT);
+      UnitPos up;
+      up.init(u_begin, NT, 1);
+      for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
+        const int b = up.b;
         if (b != prev_b) {
           if (prev_b >= 0) umma_commit(&bars->bempty[bslot]);
           bslot ^= 1;
@@ -298,8 +317,8 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     int rs = 0, as = 0;
     uint32_t rphase = 0, aphase = 0;
     for (long long u = u_begin; u < u_end; ++u) {
-      if (!mbar_wait(&bars->rfull[rs], rphase, abort_flag)) break;
-      if (!mbar_wait(&bars->aempty[as], aphase ^ 1, abort_flag)) break;
+      if (!warp_wait(&bars->rfull[rs], rphase, abort_flag)) break;
+      if (!warp_wait(&bars->aempty[as], aphase ^ 1, abort_flag)) break;
       const uint8_t* raw = sR + rs * C::RAW_BYTES;
       uint8_t* a = sA + as * C::A_BYTES;
       if (FMT == SRC_BF16) {
@@ -364,9 +383,7 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     // what the epilogue needs from global memory besides TMEM, for one unit
-    auto fetch = [&](long long u, bool& valid, float& sc) {
-      const int tile = static_cast<int>(u % NT);
-      const int b = static_cast<int>(u / NT);
+    auto fetch = [&](int b, int tile, bool& valid, float& sc) {
       const int j = tile * C::BM + quad * 32 + lane;
       valid = false;
       sc = 1.f;
@@ -384,28 +401,48 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     };
     bool nvalid = false;
     float nsc = 1.f;
-    if (u_begin < u_end) fetch(u_begin, nvalid, nsc);
-    for (long long u = u_begin; u < u_end; ++u) {
-      const int tile = static_cast<int>(u % NT);
-      const int b = static_cast<int>(u / NT);
+    UnitPos up;
+    up.init(u_begin, NT, 1);
+    if (u_begin < u_end) fetch(up.b, up.tile, nvalid, nsc);
+    int w_b = -1;
+    float wreg[32];
+    for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
+      const int tile = up.tile;
+      const int b = up.b;
       const bool valid = nvalid;
       const float sc = nsc;
-      if (u + 1 < u_end) fetch(u + 1, nvalid, nsc);  // in flight while this unit waits and computes
-      if (!mbar_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
+      if (u + 1 < u_end) {  // next unit's row id and scale are in flight while this unit waits and computes
+        if (tile + 1 == NT) fetch(b + 1, 0, nvalid, nsc);
+        else fetch(b, tile + 1, nvalid, nsc);
+      }
+      if (w_b != b) {                                // head weights of this problem, kept in registers
+        const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * kHeads);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 t4 = __ldg(w4 + i);
+          wreg[4 * i] = t4.x;
+          wreg[4 * i + 1] = t4.y;
+          wreg[4 * i + 2] = t4.z;
+          wreg[4 * i + 3] = t4.w;
+        }
+        w_b = b;
+      }
+      if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const int j = tile * C::BM + quad * 32 + lane;
-      float v[32];
-      tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::BN), v);
+      uint32_t v[32];
+      tmem_ld_32x32_nowait(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::BN),
+                           v);
+      tmem_wait_ld(v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->tempty[acc]);
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
-      const bool last_of_row = (u + 1 == u_end) || ((u + 1) / NT != b);
+      const bool last_of_row = (u + 1 == u_end) || (tile + 1 == NT);
       if (j < p.N) {
         float s = neg_inf();
         if (valid) {
-          const float* wrow = p.w + static_cast<int64_t>(b) * kHeads;
-          s = (FMT == SRC_BF16) ? head_reduce<false>(v, wrow, 1.f) : head_reduce<true>(v, wrow, sc);
+          s = (FMT == SRC_BF16) ? head_reduce_w(v, wreg) : head_reduce_scaled(v, wreg, sc);
           if (use_hist) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
         }
         p.out[static_cast<int64_t>(b) * p.N + j] = s;

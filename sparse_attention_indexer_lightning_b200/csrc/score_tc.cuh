@@ -145,11 +145,11 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
       int b_issued[2] = {0, 0};
       uint32_t b_par[2] = {0, 0};
       bool ok = true;
-      for (long long u = u_begin; u < u_end && ok; ++u) {
-        const int tile = static_cast<int>(u % NT);
-        const long long bg = u / NT;
-        const int g = static_cast<int>(bg % G);
-        const int b = static_cast<int>(bg / G);
+      UnitPos up;
+      up.init(u_begin, NT, G);
+      for (long long u = u_begin; u < u_end && ok; ++u, up.next(NT, G)) {
+        const int tile = up.tile, g = up.g, b = up.b;
+        const long long bg = static_cast<long long>(b) * G + g;
         if (bg != prev_bg) {
           bslot ^= 1;
           if (!mbar_wait(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
@@ -194,8 +194,10 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
       uint32_t bphase[2] = {0, 0};
       const uint32_t a_base = smem_u32(sA);
       const uint32_t b_base = smem_u32(sB);
-      for (long long u = u_begin; u < u_end; ++u) {
-        const long long bg = u / NT;
+      UnitPos up;
+      up.init(u_begin, NT, G);
+      for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
+        const long long bg = static_cast<long long>(up.b) * G + up.g;
         if (bg != prev_bg) {
           if (prev_bg >= 0) umma_commit(&bars->bempty[bslot]);
           bslot ^= 1;
@@ -228,34 +230,69 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each warp owns the 32 keys of its TMEM lane quadrant and Q_PER_EPI_WARP
+    // queries of the group.  The TMEM load of query j+1 is issued before the
+    // reduction of query j; the accumulator is handed back to the MMA warp as
+    // soon as the last load of the unit has landed in registers.
     const int ew = warp - 2;                  // 0 .. EPI_WARPS-1
     const int quad = warp & 3;                // TMEM lane quadrant this warp may read
     const int qset = (QG == 1) ? 0 : (ew >> 2);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (long long u = u_begin; u < u_end; ++u) {
-      const int tile = static_cast<int>(u % NT);
-      const long long bg = u / NT;
-      const int g = static_cast<int>(bg % G);
-      const int b = static_cast<int>(bg / G);
-      if (!mbar_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
-      tc_fence_after();
+    long long w_row = -1;                     // QG == 1: row whose weights sit in wreg
+    float wreg[32];
+    UnitPos up;
+    up.init(u_begin, NT, G);
+    for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
+      const int tile = up.tile, g = up.g, b = up.b;
+      const long long bg = static_cast<long long>(b) * G + g;
       const int n = tile * C::BM + quad * 32 + lane;       // key within this launch
       int lim = p.N;
-      if (p.n_valid) lim = min(lim, p.n_valid[b]);
+      if (p.n_valid) lim = min(lim, __ldg(p.n_valid + b));
+      int nq = p.T - g * QG - qset * C::Q_PER_EPI_WARP;   // queries of this warp in the group
+      nq = nq < 0 ? 0 : (nq > C::Q_PER_EPI_WARP ? C::Q_PER_EPI_WARP : nq);
+      if (QG == 1 && w_row != bg) {                        // one query per sequence: weights per row
+        const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * p.T * kHeads);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 t4 = __ldg(w4 + i);
+          wreg[4 * i] = t4.x;
+          wreg[4 * i + 1] = t4.y;
+          wreg[4 * i + 2] = t4.z;
+          wreg[4 * i + 3] = t4.w;
+        }
+        w_row = bg;
+      }
+      if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(acc * C::ACC_COLS + qset * C::Q_PER_EPI_WARP * kHeads);
+      uint32_t cur[32], nxt[32];
+      if (nq > 0) {
+        tmem_ld_32x32_nowait(tbase, cur);
+        tmem_wait_ld(cur);
+      }
+      if (nq <= 1) {                                       // nothing more to read: release now
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+      }
 #pragma unroll 1
-      for (int jq = 0; jq < C::Q_PER_EPI_WARP; ++jq) {
-        const int j = qset * C::Q_PER_EPI_WARP + jq;       // query inside the group
-        const int t = g * QG + j;
-        if (t >= p.T) break;                               // warp-uniform
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                               static_cast<uint32_t>(acc * C::ACC_COLS + j * kHeads);
-        float v[32];
-        tmem_ld_32x32(taddr, v);
-        const float s = head_reduce<false>(v, p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads, 1.f);
+      for (int jq = 0; jq < nq; ++jq) {
+        const int t = g * QG + qset * C::Q_PER_EPI_WARP + jq;
+        if (jq + 1 < nq) tmem_ld_32x32_nowait(tbase + static_cast<uint32_t>((jq + 1) * kHeads), nxt);
+        float s;
+        if (QG == 1) {
+          s = head_reduce_w(cur, wreg);
+        } else {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]);
+          s = head_reduce<false>(v, p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads, 1.f);
+        }
         int lim_t = lim;
         if (p.lim_rows) {
-          const int rel = p.lim_rows[static_cast<int64_t>(b) * p.T + t] - p.key_base;
+          const int rel = __ldg(p.lim_rows + static_cast<int64_t>(b) * p.T + t) - p.key_base;
           lim_t = rel < 0 ? 0 : (rel < lim_t ? rel : lim_t);
         } else if (p.q_pos) {
           const int64_t qp = p.q_pos[static_cast<int64_t>(b) * p.T + t];
@@ -268,12 +305,19 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
           p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
           if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
         }
+        if (jq + 1 < nq) {
+          tmem_wait_ld(nxt);
+          if (jq + 2 == nq) {                              // the unit's last load is in: release
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->tempty[acc]);
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
-      if (use_hist && (u + 1 == u_end || (u + 1) / NT != bg)) {
+      if (use_hist && (u + 1 == u_end || tile + 1 == NT)) {
         // the row (one query per sequence here) ends in this CTA: publish its counts
         role_barrier(1, C::EPI_WARPS * 32);
         flush_hist(shist, p.hist + static_cast<int64_t>(b) * p.T * kHistBins, ew * 32 + lane, C::EPI_WARPS * 32);

@@ -8,21 +8,28 @@
 // 0, below -inf), so the 64-bit keys of a row are distinct and the k-th
 // largest key is a unique threshold.
 //
-// One CTA of 1024 threads per row:
-//   1. A 2048-bin histogram of the top 11 code bits, either handed over by the
-//      scoring kernel (which counts its scores as it writes them) or built
-//      here in one pass over the row.
-//   2. The bin holding the k-th largest key splits the row: one pass copies
-//      every key above that bin to the selection and every key inside it to a
-//      shared-memory candidate buffer.
-//   3. An MSB-first 8-bit radix select over the candidates' remaining bits
-//      picks the rest; it stops as soon as every key sharing the current
-//      prefix is wanted.
-//   4. A bitonic sort of the k selected keys in shared memory gives the
-//      canonical order.
-// A row whose threshold bin holds more candidates than the buffer takes the
-// plain path instead: the same radix select run over the whole row in global
-// memory (one pass per 8-bit digit), then one collecting pass.
+// The same article's threshold idea (a sampled threshold decides how many
+// candidates are listed, never which are picked; a row whose estimate misses
+// falls back to exact work) shapes the kernel.  One CTA of 1024 threads per
+// row:
+//   1. A 2048-bin histogram of the top 11 code bits: handed over by the
+//      scoring kernel, counted exactly for rows of up to 8192 entries, or
+//      counted on a sample of about 4096-8192 entries (groups of 8
+//      consecutive entries, evenly spaced).
+//   2. A low bin is chosen so that the entries at or above it hold the top k
+//      (exactly, or with margin from the sample); one pass over the row lists
+//      them in a shared-memory candidate buffer.
+//   3. If the list is short of k or overflows the buffer, the row takes the
+//      exact plain path: an MSB-first radix select over the whole row in
+//      global memory, then one collecting pass.
+//   4. Otherwise an MSB-first radix select inside the buffer finds the k-th
+//      largest key and the k keys at or above it are compacted.
+//   5. Canonical order: the k keys are bucketed by their position in the
+//      [min, max] key range (2048 fine bins), and each key's output slot is
+//      its bucket's offset plus the number of larger keys in its bucket.
+//
+// Row passes keep many loads in flight (4 float4 per thread per chunk); writes
+// into shared buffers take one atomic per warp (a warp scan hands out slots).
 // Values are written as bit copies of the input.
 
 #pragma once
@@ -33,27 +40,138 @@
 namespace lsi {
 
 constexpr int kTopkThreads = 1024;
-constexpr int kCandCap = 4096;  // threshold-bin candidates kept in shared memory
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kCandCap = 8192;     // listed candidates kept in shared memory
+constexpr int kExactHistMax = 8192; // rows up to this length get an exact histogram
+constexpr int kVec = 4;            // float4 loads per thread per chunk
+constexpr int kChunk = kVec * 4;   // entries per thread per chunk
 
 struct TopkShared {
-  unsigned long long sel_key[kMaxTopK];
-  uint32_t sel_col[kMaxTopK];
   unsigned long long cand_key[kCandCap];
   uint32_t cand_col[kCandCap];
+  unsigned long long sel_key[kMaxTopK];
+  uint32_t sel_col[kMaxTopK];
   uint32_t hist[kHistBins];
-  uint32_t digit, need, done, total, cnt, ccnt, bstar, above, eq;
+  uint32_t fill[kHistBins];
+  uint32_t wsum[kTopkWarps];
+  unsigned long long wmin[kTopkWarps], wmax[kTopkWarps];
+  uint32_t digit, need, done, total, cnt, ccnt, eq;
 };
 
-// Warp 0: find the digit d of a descending histogram such that the keys in
-// bins above d number fewer than `want` and those in bins >= d at least
-// `want`.  Writes digit / need (= want - above) / done (bin d is taken whole).
-template <int BINS>
-__device__ __forceinline__ void find_digit(TopkShared& sh, const uint32_t* hist, uint32_t want) {
+__device__ __forceinline__ unsigned long long pack_key(float v, int32_t label) {
+  return (static_cast<unsigned long long>(order_code(v)) << 32) |
+         static_cast<uint32_t>(~static_cast<uint32_t>(label));
+}
+
+// Smallest float whose order code is `code` (codes >= 4 << 21 are finite).
+__device__ __forceinline__ float code_floor_value(uint32_t code) {
+  return __uint_as_float((code & 0x80000000u) ? (code & 0x7fffffffu) : ~code);
+}
+
+// One row of scores with optional labels.  `vec`: both row pointers are
+// 16-byte aligned, so chunks use float4 / int4 loads.
+struct RowRef {
+  const float* v;
+  const int32_t* lab;
+  int n;
+  bool vec;
+};
+
+struct Chunk {
+  float v[kChunk];
+  int32_t lab[kChunk];  // label (the column when the row has none); < 0 = absent
+};
+
+__device__ __forceinline__ int chunk_count(const RowRef& rr) {
+  if (rr.vec) {
+    const int n4 = rr.n >> 2;
+    return (n4 + kVec * kTopkThreads - 1) / (kVec * kTopkThreads) + ((rr.n & 3) ? 1 : 0);
+  }
+  return (rr.n + kChunk * kTopkThreads - 1) / (kChunk * kTopkThreads);
+}
+
+// Column of entry e of chunk `it` for this thread.
+__device__ __forceinline__ int chunk_col(const RowRef& rr, int it, int e) {
+  if (rr.vec) {
+    const int n4 = rr.n >> 2;
+    const int body = (n4 + kVec * kTopkThreads - 1) / (kVec * kTopkThreads);
+    if (it < body) return 4 * ((it * kVec + (e >> 2)) * kTopkThreads + static_cast<int>(threadIdx.x)) + (e & 3);
+    return 4 * n4 + static_cast<int>(threadIdx.x);  // tail chunk: entry 0 only
+  }
+  return (it * kChunk + e) * kTopkThreads + static_cast<int>(threadIdx.x);
+}
+
+// Loads chunk `it`; returns a bit per present entry.
+__device__ __forceinline__ uint32_t load_chunk(const RowRef& rr, int it, Chunk& c) {
+  uint32_t present = 0;
+  if (rr.vec) {
+    const int n4 = rr.n >> 2;
+    const int body = (n4 + kVec * kTopkThreads - 1) / (kVec * kTopkThreads);
+    if (it < body) {
+      float4 a[kVec];
+      int4 b[kVec];
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int j = (it * kVec + u) * kTopkThreads + static_cast<int>(threadIdx.x);
+        a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        b[u] = make_int4(-1, -1, -1, -1);
+        if (j < n4) {
+          a[u] = __ldg(reinterpret_cast<const float4*>(rr.v) + j);
+          b[u] = rr.lab ? __ldg(reinterpret_cast<const int4*>(rr.lab) + j) : make_int4(4 * j, 4 * j + 1, 4 * j + 2, 4 * j + 3);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        c.v[4 * u] = a[u].x;
+        c.v[4 * u + 1] = a[u].y;
+        c.v[4 * u + 2] = a[u].z;
+        c.v[4 * u + 3] = a[u].w;
+        c.lab[4 * u] = b[u].x;
+        c.lab[4 * u + 1] = b[u].y;
+        c.lab[4 * u + 2] = b[u].z;
+        c.lab[4 * u + 3] = b[u].w;
+      }
+    } else {
+      const int i = 4 * n4 + static_cast<int>(threadIdx.x);
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        c.v[e] = 0.f;
+        c.lab[e] = -1;
+      }
+      if (i < rr.n) {
+        c.v[0] = __ldg(rr.v + i);
+        c.lab[0] = rr.lab ? __ldg(rr.lab + i) : i;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kChunk; ++e) {
+      const int i = (it * kChunk + e) * kTopkThreads + static_cast<int>(threadIdx.x);
+      c.v[e] = 0.f;
+      c.lab[e] = -1;
+      if (i < rr.n) {
+        c.v[e] = __ldg(rr.v + i);
+        c.lab[e] = rr.lab ? __ldg(rr.lab + i) : i;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < kChunk; ++e)
+    if (c.lab[e] >= 0) present |= 1u << e;
+  return present;
+}
+
+// Warp 0: in a 256-bin histogram scanned from the top, find the digit d with
+// fewer than `want` keys above it and at least `want` at or above it.
+__device__ __forceinline__ void find_digit_256(TopkShared& sh, uint32_t want) {
   const int lane = threadIdx.x;
-  constexpr int PER = BINS / 32;
+  uint32_t c[8];
   uint32_t lsum = 0;
-#pragma unroll 8
-  for (int j = 0; j < PER; ++j) lsum += hist[BINS - 1 - PER * lane - j];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = sh.hist[255 - 8 * lane - j];
+    lsum += c[j];
+  }
   uint32_t incl = lsum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -62,47 +180,154 @@ __device__ __forceinline__ void find_digit(TopkShared& sh, const uint32_t* hist,
   }
   uint32_t cum = incl - lsum;
   if (cum < want && cum + lsum >= want) {
-    for (int j = 0; j < PER; ++j) {
-      const uint32_t c = hist[BINS - 1 - PER * lane - j];
-      if (cum + c >= want) {
-        sh.digit = BINS - 1 - PER * lane - j;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (cum < want && cum + c[j] >= want) {
+        sh.digit = 255 - 8 * lane - j;
         sh.need = want - cum;
-        sh.above = cum;
-        sh.eq = c;
-        sh.done = (c == want - cum) ? 1u : 0u;
-        break;
+        sh.eq = c[j];
+        sh.done = (c[j] == want - cum) ? 1u : 0u;
       }
-      cum += c;
+      cum += c[j];
     }
   }
 }
 
-// MSB-first radix select over `count` 64-bit keys produced by get(i).  Bits
-// at and above `hi` are equal across all keys; digits of 8 bits (the last one
-// narrower) are resolved from bit hi-1 down.  Returns the largest threshold T
-// such that exactly `want` keys are >= T (keys are distinct).
-template <class Get>
-__device__ unsigned long long radix_select(TopkShared& sh, Get get, int count, uint32_t want, int hi) {
+// All threads: exclusive prefix of a 2048-bin histogram taken from the top
+// (bin 2047 first) into `excl_out` (may alias nothing), the total into
+// sh.total, and for want = min(want_cap, total) > 0 the bin holding the
+// want-th entry (sh.digit / sh.need / sh.eq).
+__device__ __forceinline__ void scan_bins_2048(TopkShared& sh, const uint32_t* hist, uint32_t* excl_out,
+                                               uint32_t want_cap) {
+  const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5;
+  const int b0 = kHistBins - 1 - 2 * t, b1 = kHistBins - 2 - 2 * t;  // higher bin first
+  const uint32_t c0 = hist[b0], c1 = hist[b1];
+  const uint32_t c = c0 + c1;
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) sh.wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t wv = sh.wsum[lane];
+    uint32_t wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += v;
+    }
+    sh.wsum[lane] = wi - wv;
+    if (lane == 31) sh.total = wi;
+  }
+  __syncthreads();
+  const uint32_t excl = incl - c + sh.wsum[warp];
+  if (excl_out) {
+    excl_out[b0] = excl;
+    excl_out[b1] = excl + c0;
+  }
+  const uint32_t want = min(want_cap, sh.total);
+  if (want > 0 && excl < want && excl + c >= want) {
+    if (excl + c0 >= want) {
+      sh.digit = b0;
+      sh.need = want - excl;
+      sh.eq = c0;
+    } else {
+      sh.digit = b1;
+      sh.need = want - excl - c0;
+      sh.eq = c1;
+    }
+  }
+  __syncthreads();
+}
+
+// Append the keys flagged in `flags` (bit e of the chunk) at slots handed out
+// by one atomic on `counter` per warp; slots >= cap are counted, not stored.
+// Warp-collective.
+__device__ __forceinline__ void append_flagged(const RowRef& rr, int it, const Chunk& c, uint32_t flags,
+                                               unsigned long long* keys, uint32_t* cols, uint32_t* counter,
+                                               uint32_t cap) {
+  if (!__any_sync(0xffffffffu, flags != 0u)) return;  // the common case in a listing pass
+  const uint32_t mine = __popc(flags);
+  uint32_t incl = mine;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+  if (tot == 0) return;
+  uint32_t base = 0;
+  if (lane == 31) base = atomicAdd(counter, tot);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  if (!flags) return;
+  uint32_t slot = base + incl - mine;
+#pragma unroll
+  for (int e = 0; e < kChunk; ++e) {
+    if (flags & (1u << e)) {
+      if (slot < cap) {
+        keys[slot] = pack_key(c.v[e], c.lab[e]);
+        cols[slot] = static_cast<uint32_t>(chunk_col(rr, it, e));
+      }
+      ++slot;
+    }
+  }
+}
+
+// Plain path: MSB-first radix select over the whole row in global memory.
+// Returns the threshold T with exactly `want` present keys >= T.
+__device__ unsigned long long radix_select_row(TopkShared& sh, const RowRef& rr, uint32_t want) {
   unsigned long long prefix = 0ull;
-  while (hi > 0) {
-    const int width = hi < 8 ? hi : 8;
-    const int shift = hi - width;
+  const int chunks = chunk_count(rr);
+  for (int hi = 64; hi > 0; hi -= 8) {
+    const int shift = hi - 8;
     for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < count; i += kTopkThreads) {
-      unsigned long long key;
-      if (!get(i, key)) continue;
-      if (hi >= 64 || (key >> hi) == (prefix >> hi))
-        atomicAdd(&sh.hist[(key >> shift) & ((1u << width) - 1u)], 1u);
+    for (int it = 0; it < chunks; ++it) {
+      Chunk c;
+      const uint32_t present = load_chunk(rr, it, c);
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        if (present & (1u << e)) {
+          const unsigned long long key = pack_key(c.v[e], c.lab[e]);
+          if (hi >= 64 || (key >> hi) == (prefix >> hi)) atomicAdd(&sh.hist[(key >> shift) & 255u], 1u);
+        }
+      }
     }
     __syncthreads();
-    if (threadIdx.x < 32) find_digit<256>(sh, sh.hist, want);
+    if (threadIdx.x < 32) find_digit_256(sh, want);
     __syncthreads();
     prefix |= static_cast<unsigned long long>(sh.digit) << shift;
     want = sh.need;
     const uint32_t done = sh.done;
     __syncthreads();
-    hi = shift;
+    if (done) break;
+  }
+  return prefix;
+}
+
+// MSB-first radix select over the `nc` keys of the candidate buffer.
+__device__ unsigned long long radix_select_cand(TopkShared& sh, int nc, uint32_t want) {
+  unsigned long long prefix = 0ull;
+  for (int hi = 64; hi > 0; hi -= 8) {
+    const int shift = hi - 8;
+    for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += kTopkThreads) {
+      const unsigned long long key = sh.cand_key[i];
+      if (hi >= 64 || (key >> hi) == (prefix >> hi)) atomicAdd(&sh.hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) find_digit_256(sh, want);
+    __syncthreads();
+    prefix |= static_cast<unsigned long long>(sh.digit) << shift;
+    want = sh.need;
+    const uint32_t done = sh.done;
+    __syncthreads();
     if (done) break;
   }
   return prefix;
@@ -113,148 +338,224 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
   const int r = blockIdx.x;
   const int tid = threadIdx.x;
-  const float* row = p.scores + static_cast<int64_t>(r) * p.ld;
-  const int32_t* lab = p.labels ? p.labels + static_cast<int64_t>(r) * p.ld_labels : nullptr;
-  int n = p.N;
-  if (p.n_valid) n = max(0, min(n, p.n_valid[r]));
-
-  // key of element i (false when absent)
-  auto key_of = [&](int i, unsigned long long& key) -> bool {
-    uint32_t label = static_cast<uint32_t>(i);
-    if (lab) {
-      const int32_t l = lab[i];
-      if (l < 0) return false;
-      label = static_cast<uint32_t>(l);
-    }
-    key = (static_cast<unsigned long long>(order_code(row[i])) << 32) | static_cast<uint32_t>(~label);
-    return true;
-  };
+  const int lane = tid & 31, warp = tid >> 5;
+  RowRef rr;
+  rr.v = p.scores + static_cast<int64_t>(r) * p.ld;
+  rr.lab = p.labels ? p.labels + static_cast<int64_t>(r) * p.ld_labels : nullptr;
+  rr.n = p.N;
+  if (p.n_valid) rr.n = max(0, min(rr.n, p.n_valid[r]));
+  rr.vec = ((reinterpret_cast<uintptr_t>(rr.v) & 15u) == 0) &&
+           (rr.lab == nullptr || (reinterpret_cast<uintptr_t>(rr.lab) & 15u) == 0);
+  const int chunks = chunk_count(rr);
+  const uint32_t kcap = static_cast<uint32_t>(min(p.k, rr.n));  // k, or fewer entries
 
   // ---- 1. histogram of the top code bits ---------------------------------
+  if (tid == 0) {
+    sh.cnt = 0;
+    sh.ccnt = 0;
+  }
+  bool exact_hist = true;
+  int S = 1;  // sampling period in groups of 8 entries
   if (p.hist) {
     const uint32_t* gh = p.hist + static_cast<int64_t>(r) * kHistBins;
     for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = gh[i];
   } else {
     for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kTopkThreads) {
-      if (lab && lab[i] < 0) continue;
-      atomicAdd(&sh.hist[hist_bin(order_code(row[i]))], 1u);
-    }
-  }
-  __syncthreads();
-  if (tid < 32) {
-    uint32_t tot = 0;
-    for (int j = tid; j < kHistBins; j += 32) tot += sh.hist[j];
+    if (rr.n <= kExactHistMax) {
+      for (int i = tid; i < rr.n; i += kTopkThreads) {
+        const int32_t l = rr.lab ? __ldg(rr.lab + i) : i;
+        if (l >= 0) atomicAdd(&sh.hist[hist_bin(order_code(__ldg(rr.v + i)))], 1u);
+      }
+    } else {
+      exact_hist = false;
+      while ((rr.n / S) > kExactHistMax) S <<= 1;
+      const int groups = (rr.n + 7) >> 3;
+      for (int g = tid * S; g < groups; g += kTopkThreads * S) {
+        const int i0 = g << 3;
+        float v[8];
+        int32_t l[8];
+        if (rr.vec && i0 + 8 <= rr.n) {
+          const float4 a0 = __ldg(reinterpret_cast<const float4*>(rr.v + i0));
+          const float4 a1 = __ldg(reinterpret_cast<const float4*>(rr.v + i0) + 1);
+          v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
+          v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    const uint32_t want = min(static_cast<uint32_t>(p.k), tot);
-    if (tid == 0) {
-      sh.total = tot;
-      sh.cnt = 0;
-      sh.ccnt = 0;
-    }
-    if (want > 0) find_digit<kHistBins>(sh, sh.hist, want);
-  }
-  __syncthreads();
-  const int kk = static_cast<int>(min(static_cast<uint32_t>(p.k), sh.total));
-
-  if (kk > 0) {
-    const uint32_t bstar = sh.digit;
-    const uint32_t need = sh.need;
-    const uint32_t eq = sh.eq;
-    __syncthreads();
-    if (eq <= static_cast<uint32_t>(kCandCap)) {
-      // ---- 2. split the row at the threshold bin --------------------------
-      for (int i = tid; i < n; i += kTopkThreads) {
-        unsigned long long key;
-        if (!key_of(i, key)) continue;
-        const uint32_t bin = static_cast<uint32_t>(key >> (64 - kHistBits));
-        if (bin > bstar) {
-          const uint32_t s = atomicAdd(&sh.cnt, 1u);
-          if (s < static_cast<uint32_t>(kMaxTopK)) {
-            sh.sel_key[s] = key;
-            sh.sel_col[s] = static_cast<uint32_t>(i);
-          }
-        } else if (bin == bstar) {
-          const uint32_t c = atomicAdd(&sh.ccnt, 1u);
-          if (c < static_cast<uint32_t>(kCandCap)) {
-            sh.cand_key[c] = key;
-            sh.cand_col[c] = static_cast<uint32_t>(i);
+          for (int e = 0; e < 8; ++e) l[e] = rr.lab ? __ldg(rr.lab + i0 + e) : i0 + e;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const bool in = i0 + e < rr.n;
+            v[e] = in ? __ldg(rr.v + i0 + e) : 0.f;
+            l[e] = in ? (rr.lab ? __ldg(rr.lab + i0 + e) : i0 + e) : -1;
           }
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (l[e] >= 0) atomicAdd(&sh.hist[hist_bin(order_code(v[e]))], 1u);
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- 2. the low bin of the candidate list ---------------------------------
+  // exact histogram: the bin holding the k-th entry.  Sample: the bin where the
+  // sample holds k/S entries with a 25% + 16 margin.
+  uint32_t want_bins = kcap;
+  if (!exact_hist) want_bins = (kcap + kcap / 4) / static_cast<uint32_t>(S) + 16u;
+  scan_bins_2048(sh, sh.hist, nullptr, max(want_bins, 1u));
+  uint32_t blo = sh.digit;
+  const uint32_t hist_total = sh.total;
+  if (hist_total == 0) blo = 0;                          // nothing present (or nothing sampled)
+  if (!exact_hist && hist_total <= want_bins) blo = 0;   // the sample cannot place the bin: list everything
+  __syncthreads();
+
+  int kk = 0;
+  bool plain = false;
+  if (kcap > 0 && !(exact_hist && hist_total == 0)) {
+    {
+      // ---- listing pass: every present entry in a bin >= blo -------------
+      const bool by_value = blo >= 4;
+      const float tlo = by_value ? code_floor_value(blo << (32 - kHistBits)) : 0.f;
+      for (int it = 0; it < chunks; ++it) {
+        Chunk c;
+        const uint32_t present = load_chunk(rr, it, c);
+        uint32_t flags = 0;
+#pragma unroll
+        for (int e = 0; e < kChunk; ++e) {
+          const bool in = by_value ? (c.v[e] >= tlo) : (hist_bin(order_code(c.v[e])) >= blo);
+          if ((present & (1u << e)) && in) flags |= 1u << e;
+        }
+        append_flagged(rr, it, c, flags, sh.cand_key, sh.cand_col, &sh.ccnt, kCandCap);
       }
       __syncthreads();
-      // ---- 3. radix select inside the threshold bin -----------------------
-      const int nc = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(kCandCap)));
-      unsigned long long thr = 0ull;
-      if (need < static_cast<uint32_t>(nc)) {
-        thr = radix_select(
-            sh, [&](int i, unsigned long long& key) -> bool { key = sh.cand_key[i]; return true; }, nc, need,
-            64 - kHistBits);
-      }
-      for (int i = tid; i < nc; i += kTopkThreads) {
-        if (sh.cand_key[i] >= thr) {
-          const uint32_t s = atomicAdd(&sh.cnt, 1u);
-          if (s < static_cast<uint32_t>(kMaxTopK)) {
-            sh.sel_key[s] = sh.cand_key[i];
-            sh.sel_col[s] = sh.cand_col[i];
-          }
-        }
-      }
-    } else {
-      // ---- plain path: radix select over the whole row --------------------
-      const unsigned long long thr = radix_select(sh, key_of, n, static_cast<uint32_t>(kk), 64);
-      for (int i = tid; i < n; i += kTopkThreads) {
-        unsigned long long key;
-        if (!key_of(i, key)) continue;
-        if (key >= thr) {
-          const uint32_t s = atomicAdd(&sh.cnt, 1u);
-          if (s < static_cast<uint32_t>(kMaxTopK)) {
-            sh.sel_key[s] = key;
-            sh.sel_col[s] = static_cast<uint32_t>(i);
-          }
-        }
-      }
-    }
-    __syncthreads();
-    // ---- 4. canonical order ------------------------------------------------
-    int P2 = 1;
-    while (P2 < kk) P2 <<= 1;
-    for (int i = kk + tid; i < P2; i += kTopkThreads) {
-      sh.sel_key[i] = 0ull;
-      sh.sel_col[i] = 0u;
-    }
-    __syncthreads();
-    for (int size = 2; size <= P2; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < (P2 >> 1); i += kTopkThreads) {
-          const int lo = 2 * i - (i & (stride - 1));
-          const int hi = lo + stride;
-          const bool desc = (lo & size) == 0;
-          const unsigned long long a = sh.sel_key[lo], b = sh.sel_key[hi];
-          if (desc ? (a < b) : (a > b)) {
-            sh.sel_key[lo] = b;
-            sh.sel_key[hi] = a;
-            const uint32_t t = sh.sel_col[lo];
-            sh.sel_col[lo] = sh.sel_col[hi];
-            sh.sel_col[hi] = t;
-          }
-        }
-        __syncthreads();
-      }
+      const uint32_t listed = sh.ccnt;
+      // entries to select: exact when the histogram counted every present entry
+      kk = static_cast<int>(exact_hist ? min(kcap, hist_total) : kcap);
+      if (listed > static_cast<uint32_t>(kCandCap) || listed < static_cast<uint32_t>(kk)) plain = true;
     }
   }
+
+  if (kk > 0 && plain) {
+    // ---- 3. exact plain path ---------------------------------------------
+    // count the present entries first when the histogram was only sampled
+    if (!exact_hist) {
+      if (tid == 0) sh.cnt = 0;
+      __syncthreads();
+      for (int it = 0; it < chunks; ++it) {
+        Chunk c;
+        const uint32_t present = load_chunk(rr, it, c);
+        uint32_t cnt = __popc(present);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0 && cnt) atomicAdd(&sh.cnt, cnt);
+      }
+      __syncthreads();
+      kk = static_cast<int>(min(kcap, sh.cnt));
+      __syncthreads();
+    }
+    if (tid == 0) sh.cnt = 0;
+    __syncthreads();
+    if (kk > 0) {
+      const unsigned long long thr = radix_select_row(sh, rr, static_cast<uint32_t>(kk));
+      for (int it = 0; it < chunks; ++it) {
+        Chunk c;
+        const uint32_t present = load_chunk(rr, it, c);
+        uint32_t flags = 0;
+#pragma unroll
+        for (int e = 0; e < kChunk; ++e)
+          if ((present & (1u << e)) && pack_key(c.v[e], c.lab[e]) >= thr) flags |= 1u << e;
+        append_flagged(rr, it, c, flags, sh.sel_key, sh.sel_col, &sh.cnt, kMaxTopK);
+      }
+    }
+    __syncthreads();
+  } else if (kk > 0) {
+    // ---- 4. select inside the candidate list ------------------------------
+    const int nc = static_cast<int>(sh.ccnt);
+    unsigned long long thr = 0ull;
+    if (nc > kk) thr = radix_select_cand(sh, nc, static_cast<uint32_t>(kk));
+    if (tid == 0) sh.cnt = 0;
+    __syncthreads();
+    const int rounds = (nc + kTopkThreads - 1) / kTopkThreads;
+    for (int rd = 0; rd < rounds; ++rd) {
+      const int i = rd * kTopkThreads + tid;
+      const bool take = i < nc && sh.cand_key[i] >= thr;
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      uint32_t base = 0;
+      if (lane == 0 && bal) base = atomicAdd(&sh.cnt, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (take) {
+        const uint32_t s = base + __popc(bal & ((1u << lane) - 1u));
+        sh.sel_key[s] = sh.cand_key[i];
+        sh.sel_col[s] = sh.cand_col[i];
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- 5. canonical order: bucket by key range, rank inside the bucket ----
   int32_t* io = p.idx_out + static_cast<int64_t>(r) * p.ld_out;
   float* vo = p.val_out ? p.val_out + static_cast<int64_t>(r) * p.ld_out : nullptr;
-  for (int j = tid; j < p.k; j += kTopkThreads) {
-    if (j < kk) {
-      io[j] = static_cast<int32_t>(~static_cast<uint32_t>(sh.sel_key[j] & 0xffffffffull));
-      if (vo) vo[j] = row[sh.sel_col[j]];
-    } else {
-      io[j] = -1;
-      if (vo) vo[j] = neg_inf();
+  if (kk > 0) {
+    unsigned long long kmin = ~0ull, kmax = 0ull;
+    for (int i = tid; i < kk; i += kTopkThreads) {
+      const unsigned long long key = sh.sel_key[i];
+      kmin = key < kmin ? key : kmin;
+      kmax = key > kmax ? key : kmax;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+      const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
+      kmin = a < kmin ? a : kmin;
+      kmax = b > kmax ? b : kmax;
+    }
+    if (lane == 0) {
+      sh.wmin[warp] = kmin;
+      sh.wmax[warp] = kmax;
+    }
+    for (int i = tid; i < kHistBins; i += kTopkThreads) {
+      sh.hist[i] = 0;
+      sh.fill[i] = 0;
+    }
+    __syncthreads();
+    kmin = sh.wmin[0];
+    kmax = sh.wmax[0];
+    for (int wi = 1; wi < kTopkWarps; ++wi) {
+      kmin = sh.wmin[wi] < kmin ? sh.wmin[wi] : kmin;
+      kmax = sh.wmax[wi] > kmax ? sh.wmax[wi] : kmax;
+    }
+    const unsigned long long span = kmax - kmin;
+    const int shift = span ? max(0, 64 - __clzll(static_cast<long long>(span)) - kHistBits) : 0;
+    for (int i = tid; i < kk; i += kTopkThreads)
+      atomicAdd(&sh.hist[static_cast<uint32_t>((sh.sel_key[i] - kmin) >> shift)], 1u);
+    __syncthreads();
+    // bucket offsets from the top (largest keys first); fill holds the offsets
+    scan_bins_2048(sh, sh.hist, sh.fill, 0u);
+    // scatter into buckets (the candidate buffer is free now)
+    for (int i = tid; i < kk; i += kTopkThreads) {
+      const unsigned long long key = sh.sel_key[i];
+      const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
+      const uint32_t pos = atomicAdd(&sh.fill[bin], 1u);
+      sh.cand_key[pos] = key;
+      sh.cand_col[pos] = sh.sel_col[i];
+    }
+    __syncthreads();
+    // rank inside the bucket: after the scatter fill[bin] is the bucket's end
+    for (int i = tid; i < kk; i += kTopkThreads) {
+      const unsigned long long key = sh.cand_key[i];
+      const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
+      const uint32_t end = sh.fill[bin];
+      const uint32_t beg = end - sh.hist[bin];
+      uint32_t rank = beg;
+      for (uint32_t j = beg; j < end; ++j) rank += (sh.cand_key[j] > key) ? 1u : 0u;
+      io[rank] = static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull));
+      if (vo) vo[rank] = rr.v[sh.cand_col[i]];
+    }
+  }
+  for (int j = kk + tid; j < p.k; j += kTopkThreads) {
+    io[j] = -1;
+    if (vo) vo[j] = neg_inf();
   }
 }
 
