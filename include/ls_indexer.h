@@ -144,6 +144,28 @@ ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* ke
                            size_t ws_bytes, void* stream);
 
 /*
+ * ls_decode_select_noalloc -- ls_decode_select for callers that cannot
+ * allocate device memory (an engine that owns the whole device pool and gives
+ * its plugins no allocator; a latency-critical loop that cannot take the
+ * device-wide synchronisation of cudaMalloc).  The pages describe no such
+ * call; it is a deployment convenience of this library.
+ *
+ * Same arguments and results as ls_decode_select, without (ws, ws_bytes):
+ * the scratch is a fixed 10 MiB device array inside the library, held on
+ * every device that loads it until the process exits.  Sizes whose
+ * ls_decode_select_workspace_size(B, N) exceeds 10 MiB (B*N above about
+ * 2.5 million with B rows of histograms) return LS_ERR_WORKSPACE.  The first
+ * call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make it before any stream capture.  The call
+ * allocates nothing.  All calls share the array: calls that overlap on the
+ * GPU race and must be serialised by the caller; the part that must start at
+ * zero is cleared by every call.
+ */
+ls_status ls_decode_select_noalloc(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid,
+                                   int B, int H, int d, int N, int k, int32_t* idx_out, float* val_out,
+                                   void* stream);
+
+/*
  * ls_prefill_select_stream -- causal top-k for a chunk of prefill queries
  * against a history that lives in host memory and is streamed through two
  * alternating device buffers (LeanSparse podcast transcript, 05:36-06:44:

@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     LSError,
     ls_bucket_select,
     ls_decode_select,
+    ls_decode_select_noalloc,
     ls_decode_two_stage_select,
     ls_device_status,
     ls_indexer_score,

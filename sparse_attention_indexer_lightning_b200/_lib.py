@@ -35,7 +35,7 @@ EXPORTED = (
     "ls_decode_select_workspace_size", "ls_decode_select", "ls_prefill_select_workspace_size",
     "ls_prefill_select_stream", "ls_two_stage_workspace_size", "ls_decode_two_stage_select",
     "ls_bucket_workspace_size", "ls_bucket_select", "ls_selftest_wait_probe", "ls_profile_begin",
-    "ls_profile_end", "ls_profile_kernel",
+    "ls_profile_end", "ls_profile_kernel", "ls_decode_select_noalloc",
 )
 HIST_BINS = 2048
 
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_profile_begin": (I, []),
         "ls_profile_end": (I, [P]),
         "ls_profile_kernel": (I, [I, P, P, P]),
+        "ls_decode_select_noalloc": (I, [P, P, P, P, I, I, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -186,6 +187,27 @@ def ls_decode_select(q, w, keys, k: int = 512, n_valid=None, ws=None, out=None, 
     idx, val = out
     _check(lib().ls_decode_select(_ptr(q), _ptr(w), _ptr(keys), _ptr(n_valid), B, H, d, N, k, _ptr(idx), _ptr(val),
                                   _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, val
+
+
+def ls_decode_select_noalloc(q, w, keys, k: int = 512, n_valid=None, out=None, stream=None):
+    """ls_decode_select with the library's fixed device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory on this path; sizes above
+    the fixed scratch raise LSError (LS_ERR_WORKSPACE).  Calls share the
+    scratch, so calls that overlap on the GPU must be serialised."""
+    _dev(q, torch.bfloat16, "q", 3)
+    B, H, d = q.shape
+    _dev(w, torch.float32, "w", 2)
+    _dev(keys, torch.bfloat16, "keys", 3)
+    N = keys.shape[1]
+    _opt(n_valid, torch.int32, "n_valid")
+    if out is None:
+        out = (torch.empty((B, k), dtype=torch.int32, device=q.device),
+               torch.empty((B, k), dtype=torch.float32, device=q.device))
+    idx, val = out
+    _check(lib().ls_decode_select_noalloc(_ptr(q), _ptr(w), _ptr(keys), _ptr(n_valid), B, H, d, N, k, _ptr(idx),
+                                          _ptr(val), _stream(stream)))
     return idx, val
 
 

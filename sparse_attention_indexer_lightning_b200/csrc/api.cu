@@ -564,3 +564,66 @@ ls_status ls_selftest_wait_probe(uint64_t limit_ns, int* gave_up_dev, void* stre
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------
+// Decode selection for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand the library a workspace: an engine that
+// reserves the whole device pool at start-up and gives its plugins no
+// allocator, or a latency-critical loop where the implicit device-wide
+// synchronisation of cudaMalloc / cudaFree is not acceptable.  For them,
+// ls_decode_select_noalloc runs the same decode selection as
+// ls_decode_select with its scratch (the score rows and the selection
+// histograms) in the fixed device array below, which the library holds on
+// every device that loads it until the process exits.
+//
+// The array's host-side name is not a device address, so the first call on
+// each device (with that device current) asks the runtime for the address
+// with cudaGetSymbolAddress and caches it.  That first call should therefore
+// be made before any stream capture is started on that device.  Nothing else
+// is allocated: no cudaMalloc, cudaFree or allocating library call.
+//
+// All calls share the one array and it keeps the contents of the last call.
+// The histogram part, which must start at zero, is cleared on the stream by
+// every call; the score part is fully overwritten.  Calls whose work overlaps
+// on the GPU (on different streams, or from different host threads) race on
+// the array: order them on one stream or serialise them.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(10) << 20;  // 10 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+
+}  // namespace
+
+extern "C" ls_status ls_decode_select_noalloc(const uint16_t* q, const float* w, const uint16_t* keys,
+                                              const int32_t* n_valid, int B, int H, int d, int N, int k,
+                                              int32_t* idx_out, float* val_out, void* stream) {
+  LS_CHECK_ARG(B >= 0 && N >= 0, "negative size");
+  const size_t need = ls_decode_select_workspace_size(B, N);
+  if (need > kNoAllocScratchBytes)
+    return fail(LS_ERR_WORKSPACE,
+                "B=%d x N=%d needs %zu B of scratch; the fixed scratch of ls_decode_select_noalloc holds %zu B "
+                "(about 2.5M score entries in all); use ls_decode_select with a workspace",
+                B, N, need, kNoAllocScratchBytes);
+  int dev = 0;
+  LS_CUDA(cudaGetDevice(&dev));
+  LS_CHECK_ARG(dev >= 0 && dev < 64, "device ordinal %d beyond the 64 this call tracks", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess)
+        return fail(LS_ERR_CUDA, "cudaGetSymbolAddress of the fixed scratch on device %d: %s", dev,
+                    cudaGetErrorString(e));
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return ls_decode_select(q, w, keys, n_valid, B, H, d, N, k, idx_out, val_out, scratch, kNoAllocScratchBytes,
+                          stream);
+}
