@@ -2,8 +2,10 @@
 
 The binding only marshals arguments (torch tensors for device memory and the
 current CUDA stream) into the library's C ABI (include/ls_indexer.h); every
-step of the selection path runs in the library's CUDA kernels.  Importing the
-package loads the library and raises ImportError if it is missing.
+step of the selection path runs in the library's CUDA kernels.  The library
+is loaded on first use; a missing or stale libls_indexer.so raises
+ImportError there (build it with `python -m
+sparse_attention_indexer_lightning_b200.build`).  There is no fallback.
 """
 
 from ._lib import (  # noqa: F401
@@ -23,5 +25,3 @@ from ._lib import (  # noqa: F401
     ls_topk_select,
     lib,
 )
-
-lib()  # fail loudly at import when the CUDA library is absent

@@ -3,8 +3,8 @@
 Argument marshalling only: the functions below check dtypes, devices and
 shapes of torch tensors, allocate outputs and workspace through torch, and
 call the library on the current CUDA stream.  Every step of the selection path
-runs in the library's kernels; there is no fallback.  Importing this module
-fails loudly when the shared library is missing.
+runs in the library's kernels; there is no fallback.  The first call loads the
+shared library and raises ImportError when it is missing or stale.
 """
 
 from __future__ import annotations
@@ -74,7 +74,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_decode_select_noalloc": (I, [P, P, P, P, I, I, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError:
+            raise ImportError(f"{path} does not export {name}: it is stale, rebuild it") from None
         fn.restype = res
         fn.argtypes = args
     return lib

@@ -86,3 +86,9 @@ def test_argument_checks_without_gpu(lib):
     assert lib.ls_profile_begin() == 0
     assert lib.ls_profile_end(ctypes.byref(n)) == 0 and n.value == 0
     assert lib.ls_profile_kernel(0, None, None, None) == 1
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from sparse_attention_indexer_lightning_b200 import _lib
+    with pytest.raises(ImportError):
+        _lib.load_library(str(tmp_path / "libls_indexer.so"))
