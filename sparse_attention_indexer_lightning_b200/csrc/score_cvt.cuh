@@ -46,6 +46,8 @@ struct CvtCfg {
   static constexpr int ACC = 2;
   static constexpr int TMEM_COLS = 64;
   static constexpr int CVT_WARPS = 8;
+  static constexpr int CVT_GROUPS = 2;                       // tiles converted at once
+  static constexpr int CVT_GROUP_WARPS = CVT_WARPS / CVT_GROUPS;
   static constexpr int EPI_WARPS = 4;
   static constexpr int THREADS = (2 + CVT_WARPS + EPI_WARPS) * 32;
   static constexpr size_t SMEM_RAW = size_t(RS) * RAW_BYTES;
@@ -141,10 +143,10 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::RS; ++s) {
       mbar_init(&bars->rfull[s], 1);
-      mbar_init(&bars->rempty[s], C::CVT_WARPS);
+      mbar_init(&bars->rempty[s], C::CVT_GROUP_WARPS);
     }
     for (int s = 0; s < C::AS; ++s) {
-      mbar_init(&bars->afull[s], C::CVT_WARPS);
+      mbar_init(&bars->afull[s], C::CVT_GROUP_WARPS);
       mbar_init(&bars->aempty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -312,11 +314,15 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     }
   } else if (warp < 2 + C::CVT_WARPS) {
     // ------------------------------------------------------------ converters
-    constexpr int CT = C::CVT_WARPS * 32;
-    const int ct = threadIdx.x - 64;  // 0 .. CT-1
-    int rs = 0, as = 0;
-    uint32_t rphase = 0, aphase = 0;
-    for (long long u = u_begin; u < u_end; ++u) {
+    // CVT_GROUPS groups of warps take alternate units, so that many tiles are
+    // widened at once; each group's threads share one tile.
+    constexpr int CT = C::CVT_GROUP_WARPS * 32;
+    const int cg = (warp - 2) / C::CVT_GROUP_WARPS;
+    const int ct = threadIdx.x - 64 - cg * CT;  // 0 .. CT-1
+    const long long count = u_end - u_begin;
+    for (long long i = cg; i < count; i += C::CVT_GROUPS) {
+      const int rs = static_cast<int>(i % C::RS), as = static_cast<int>(i % C::AS);
+      const uint32_t rphase = static_cast<uint32_t>((i / C::RS) & 1), aphase = static_cast<uint32_t>((i / C::AS) & 1);
       if (!warp_wait(&bars->rfull[rs], rphase, abort_flag)) break;
       if (!warp_wait(&bars->aempty[as], aphase ^ 1, abort_flag)) break;
       const uint8_t* raw = sR + rs * C::RAW_BYTES;
@@ -373,8 +379,6 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
         mbar_arrive(&bars->rempty[rs]);
         mbar_arrive(&bars->afull[as]);
       }
-      if (++rs == C::RS) { rs = 0; rphase ^= 1; }
-      if (++as == C::AS) { as = 0; aphase ^= 1; }
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -267,53 +267,56 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * C::ACC_COLS + qset * C::Q_PER_EPI_WARP * kHeads);
-      uint32_t cur[32], nxt[32];
+      // two register buffers, alternated by the fully unrolled query loop
+      uint32_t ra[32], rb[32];
       if (nq > 0) {
-        tmem_ld_32x32_nowait(tbase, cur);
-        tmem_wait_ld(cur);
+        tmem_ld_32x32_nowait(tbase, ra);
+        tmem_wait_ld(ra);
       }
       if (nq <= 1) {                                       // nothing more to read: release now
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->tempty[acc]);
       }
-#pragma unroll 1
-      for (int jq = 0; jq < nq; ++jq) {
-        const int t = g * QG + qset * C::Q_PER_EPI_WARP + jq;
-        if (jq + 1 < nq) tmem_ld_32x32_nowait(tbase + static_cast<uint32_t>((jq + 1) * kHeads), nxt);
-        float s;
-        if (QG == 1) {
-          s = head_reduce_w(cur, wreg);
-        } else {
-          float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]);
-          s = head_reduce<false>(v, p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads, 1.f);
-        }
-        int lim_t = lim;
-        if (p.lim_rows) {
-          const int rel = __ldg(p.lim_rows + static_cast<int64_t>(b) * p.T + t) - p.key_base;
-          lim_t = rel < 0 ? 0 : (rel < lim_t ? rel : lim_t);
-        } else if (p.q_pos) {
-          const int64_t qp = p.q_pos[static_cast<int64_t>(b) * p.T + t];
-          int64_t e = qp < 0 ? 0 : (qp + 1) / p.stride;
-          if (e > p.n_total) e = p.n_total;
-          const int64_t rel = e - p.key_base;
-          lim_t = static_cast<int>(rel < 0 ? 0 : (rel < lim_t ? rel : lim_t));
-        }
-        if (n < p.N) {
-          p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
-          if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
-        }
-        if (jq + 1 < nq) {
-          tmem_wait_ld(nxt);
-          if (jq + 2 == nq) {                              // the unit's last load is in: release
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+      for (int jq = 0; jq < C::Q_PER_EPI_WARP; ++jq) {
+        if (jq < nq) {                                     // warp-uniform
+          uint32_t(&cur)[32] = (jq & 1) ? rb : ra;
+          uint32_t(&nxt)[32] = (jq & 1) ? ra : rb;
+          const int t = g * QG + qset * C::Q_PER_EPI_WARP + jq;
+          if (jq + 1 < nq) tmem_ld_32x32_nowait(tbase + static_cast<uint32_t>((jq + 1) * kHeads), nxt);
+          float s;
+          if (QG == 1) {
+            s = head_reduce_w(cur, wreg);
+          } else {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]);
+            s = head_reduce<false>(v, p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads, 1.f);
           }
-#pragma unroll
-          for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
+          int lim_t = lim;
+          if (p.lim_rows) {
+            const int rel = __ldg(p.lim_rows + static_cast<int64_t>(b) * p.T + t) - p.key_base;
+            lim_t = rel < 0 ? 0 : (rel < lim_t ? rel : lim_t);
+          } else if (p.q_pos) {
+            const int64_t qp = p.q_pos[static_cast<int64_t>(b) * p.T + t];
+            int64_t e = qp < 0 ? 0 : (qp + 1) / p.stride;
+            if (e > p.n_total) e = p.n_total;
+            const int64_t rel = e - p.key_base;
+            lim_t = static_cast<int>(rel < 0 ? 0 : (rel < lim_t ? rel : lim_t));
+          }
+          if (n < p.N) {
+            p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
+            if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
+          }
+          if (jq + 1 < nq) {
+            tmem_wait_ld(nxt);
+            if (jq + 2 == nq) {                            // the unit's last load is in: release
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+            }
+          }
         }
       }
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }

@@ -47,10 +47,12 @@ constexpr int kVec = 4;            // float4 loads per thread per chunk
 constexpr int kChunk = kVec * 4;   // entries per thread per chunk
 
 struct TopkShared {
-  unsigned long long cand_key[kCandCap];
-  uint32_t cand_col[kCandCap];
-  unsigned long long sel_key[kMaxTopK];
-  uint32_t sel_col[kMaxTopK];
+  float cand_val[kCandCap];            // listed entries: value and label
+  int32_t cand_lab[kCandCap];
+  unsigned long long sel_key[kMaxTopK];  // the k selected: packed key and value
+  float sel_val[kMaxTopK];
+  unsigned long long tmp_key[kMaxTopK];  // bucketed copy for the final order
+  float tmp_val[kMaxTopK];
   uint32_t hist[kHistBins];
   uint32_t fill[kHistBins];
   uint32_t wsum[kTopkWarps];
@@ -278,6 +280,139 @@ __device__ __forceinline__ void append_flagged(const RowRef& rr, int it, const C
   }
 }
 
+__device__ __forceinline__ float f4at(const float4& a, int q) {
+  return q == 0 ? a.x : q == 1 ? a.y : q == 2 ? a.z : a.w;
+}
+__device__ __forceinline__ int32_t i4at(const int4& a, int q) {
+  return q == 0 ? a.x : q == 1 ? a.y : q == 2 ? a.z : a.w;
+}
+
+// Warp-collective append of up to 16 flagged entries per thread: one atomic
+// per warp hands out the slots; slots >= cap are counted, not stored.
+__device__ __forceinline__ uint32_t warp_slots(uint32_t flags, uint32_t* counter) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t mine = __popc(flags);
+  uint32_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+  uint32_t base = 0;
+  if (lane == 31) base = atomicAdd(counter, tot);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  return base + incl - mine;
+}
+
+// Listing pass: every present entry whose key passes `keep(value, label)` is
+// appended to (vals, labs): its value and its label (the column when the row
+// has no labels).  Threads read 4 float4 (and int4
+// labels when the row has them) per step; all threads run the same number of
+// steps.  Rows without labels skip every label computation until an entry is
+// flagged.
+template <bool HAS_LAB, class Keep>
+__device__ __forceinline__ void list_row_t(const RowRef& rr, Keep keep, float* vals, int32_t* labs,
+                                           uint32_t* counter, uint32_t cap) {
+  const int tid = threadIdx.x;
+  if (rr.vec) {
+    const int n4 = rr.n >> 2;
+    const float4* v4 = reinterpret_cast<const float4*>(rr.v);
+    const int4* l4 = reinterpret_cast<const int4*>(rr.lab);
+    for (int base = 0; base < n4; base += kVec * kTopkThreads) {
+      float4 a[kVec];
+      int4 l[kVec];
+      uint32_t inb = 0;  // bit u: vector u exists
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int j = base + u * kTopkThreads + tid;
+        a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (HAS_LAB) l[u] = make_int4(-1, -1, -1, -1);
+        if (j < n4) {
+          a[u] = __ldg(v4 + j);
+          if (HAS_LAB) l[u] = __ldg(l4 + j);
+          inb |= 1u << u;
+        }
+      }
+      uint32_t flags = 0;
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        // label: the column when the row has none (dead code unless keep reads it)
+        const int32_t lb = HAS_LAB ? i4at(l[e >> 2], e & 3) : 4 * (base + (e >> 2) * kTopkThreads + tid) + (e & 3);
+        const bool ok = HAS_LAB ? (lb >= 0) : ((inb >> (e >> 2)) & 1u);
+        if (ok && keep(f4at(a[e >> 2], e & 3), lb)) flags |= 1u << e;
+      }
+      if (!__any_sync(0xffffffffu, flags != 0u)) continue;
+      uint32_t slot = warp_slots(flags, counter);
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        if (flags & (1u << e)) {
+          if (slot < cap) {
+            vals[slot] = f4at(a[e >> 2], e & 3);
+            labs[slot] = HAS_LAB ? i4at(l[e >> 2], e & 3) : 4 * (base + (e >> 2) * kTopkThreads + tid) + (e & 3);
+          }
+          ++slot;
+        }
+      }
+    }
+    // the n % 4 entries after the float4 body, one per thread
+    const int i = 4 * n4 + tid;
+    uint32_t flag = 0;
+    float v = 0.f;
+    int32_t lb = -1;
+    if (i < rr.n) {
+      v = __ldg(rr.v + i);
+      lb = HAS_LAB ? __ldg(rr.lab + i) : i;
+      if (lb >= 0 && keep(v, lb)) flag = 1u;
+    }
+    if (__any_sync(0xffffffffu, flag != 0u)) {
+      const uint32_t slot = warp_slots(flag, counter);
+      if (flag && slot < cap) {
+        vals[slot] = v;
+        labs[slot] = lb;
+      }
+    }
+  } else {
+    for (int base = 0; base < rr.n; base += kChunk * kTopkThreads) {
+      float a[kChunk];
+      int32_t l[kChunk];
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        const int i = base + e * kTopkThreads + tid;
+        a[e] = 0.f;
+        l[e] = -1;
+        if (i < rr.n) {
+          a[e] = __ldg(rr.v + i);
+          l[e] = HAS_LAB ? __ldg(rr.lab + i) : i;
+        }
+      }
+      uint32_t flags = 0;
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e)
+        if (l[e] >= 0 && keep(a[e], l[e])) flags |= 1u << e;
+      if (!__any_sync(0xffffffffu, flags != 0u)) continue;
+      uint32_t slot = warp_slots(flags, counter);
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        if (flags & (1u << e)) {
+          if (slot < cap) {
+            vals[slot] = a[e];
+            labs[slot] = l[e];
+          }
+          ++slot;
+        }
+      }
+    }
+  }
+}
+
+template <class Keep>
+__device__ __forceinline__ void list_row(const RowRef& rr, Keep keep, float* vals, int32_t* labs, uint32_t* counter,
+                                         uint32_t cap) {
+  if (rr.lab) list_row_t<true>(rr, keep, vals, labs, counter, cap);
+  else list_row_t<false>(rr, keep, vals, labs, counter, cap);
+}
+
 // Plain path: MSB-first radix select over the whole row in global memory.
 // Returns the threshold T with exactly `want` present keys >= T.
 __device__ unsigned long long radix_select_row(TopkShared& sh, const RowRef& rr, uint32_t want) {
@@ -310,16 +445,65 @@ __device__ unsigned long long radix_select_row(TopkShared& sh, const RowRef& rr,
   return prefix;
 }
 
-// MSB-first radix select over the `nc` keys of the candidate buffer.
+// MSB-first radix select over the `nc` keys of the candidate buffer.  It
+// starts at the highest bit where the candidates differ (their common high
+// bits are read off the smallest and largest key), so no pass is spent on
+// bits every candidate shares.
 __device__ unsigned long long radix_select_cand(TopkShared& sh, int nc, uint32_t want) {
-  unsigned long long prefix = 0ull;
-  for (int hi = 64; hi > 0; hi -= 8) {
-    const int shift = hi - 8;
-    for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
-    __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long kmin = ~0ull, kmax = 0ull;
+  for (int i = threadIdx.x; i < nc; i += kTopkThreads) {
+    const unsigned long long key = pack_key(sh.cand_val[i], sh.cand_lab[i]);
+    kmin = key < kmin ? key : kmin;
+    kmax = key > kmax ? key : kmax;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+    const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
+    kmin = a < kmin ? a : kmin;
+    kmax = b > kmax ? b : kmax;
+  }
+  if (lane == 0) {
+    sh.wmin[warp] = kmin;
+    sh.wmax[warp] = kmax;
+  }
+  for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    kmin = sh.wmin[lane];
+    kmax = sh.wmax[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+      const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
+      kmin = a < kmin ? a : kmin;
+      kmax = b > kmax ? b : kmax;
+    }
+    if (lane == 0) {
+      sh.wmin[0] = kmin;
+      sh.wmax[0] = kmax;
+    }
+  }
+  __syncthreads();
+  kmin = sh.wmin[0];
+  kmax = sh.wmax[0];
+  const unsigned long long diff = kmin ^ kmax;
+  int hi = diff ? 64 - __clzll(static_cast<long long>(diff)) : 0;
+  unsigned long long prefix = hi >= 64 ? 0ull : (kmin >> hi) << hi;  // bits every candidate shares
+  bool first = true;
+  while (hi > 0) {
+    const int width = hi < 8 ? hi : 8;
+    const int shift = hi - width;
+    if (!first) {
+      for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
+      __syncthreads();
+    }
+    first = false;
     for (int i = threadIdx.x; i < nc; i += kTopkThreads) {
-      const unsigned long long key = sh.cand_key[i];
-      if (hi >= 64 || (key >> hi) == (prefix >> hi)) atomicAdd(&sh.hist[(key >> shift) & 255u], 1u);
+      const unsigned long long key = pack_key(sh.cand_val[i], sh.cand_lab[i]);
+      if (hi >= 64 || (key >> hi) == (prefix >> hi))
+        atomicAdd(&sh.hist[static_cast<uint32_t>(key >> shift) & ((1u << width) - 1u)], 1u);
     }
     __syncthreads();
     if (threadIdx.x < 32) find_digit_256(sh, want);
@@ -328,6 +512,7 @@ __device__ unsigned long long radix_select_cand(TopkShared& sh, int nc, uint32_t
     want = sh.need;
     const uint32_t done = sh.done;
     __syncthreads();
+    hi = shift;
     if (done) break;
   }
   return prefix;
@@ -415,18 +600,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   if (kcap > 0 && !(exact_hist && hist_total == 0)) {
     {
       // ---- listing pass: every present entry in a bin >= blo -------------
-      const bool by_value = blo >= 4;
-      const float tlo = by_value ? code_floor_value(blo << (32 - kHistBits)) : 0.f;
-      for (int it = 0; it < chunks; ++it) {
-        Chunk c;
-        const uint32_t present = load_chunk(rr, it, c);
-        uint32_t flags = 0;
-#pragma unroll
-        for (int e = 0; e < kChunk; ++e) {
-          const bool in = by_value ? (c.v[e] >= tlo) : (hist_bin(order_code(c.v[e])) >= blo);
-          if ((present & (1u << e)) && in) flags |= 1u << e;
-        }
-        append_flagged(rr, it, c, flags, sh.cand_key, sh.cand_col, &sh.ccnt, kCandCap);
+      if (blo >= 4) {  // bins from 4 up start at finite values: compare the score itself
+        const float tlo = code_floor_value(blo << (32 - kHistBits));
+        list_row(rr, [&](float v, int32_t) { return v >= tlo; }, sh.cand_val, sh.cand_lab, &sh.ccnt, kCandCap);
+      } else {
+        list_row(rr, [&](float v, int32_t) { return hist_bin(order_code(v)) >= blo; }, sh.cand_val, sh.cand_lab,
+                 &sh.ccnt, kCandCap);
       }
       __syncthreads();
       const uint32_t listed = sh.ccnt;
@@ -454,24 +633,20 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       kk = static_cast<int>(min(kcap, sh.cnt));
       __syncthreads();
     }
-    if (tid == 0) sh.cnt = 0;
+    if (tid == 0) sh.ccnt = 0;
     __syncthreads();
+    unsigned long long thr = 0ull;
     if (kk > 0) {
-      const unsigned long long thr = radix_select_row(sh, rr, static_cast<uint32_t>(kk));
-      for (int it = 0; it < chunks; ++it) {
-        Chunk c;
-        const uint32_t present = load_chunk(rr, it, c);
-        uint32_t flags = 0;
-#pragma unroll
-        for (int e = 0; e < kChunk; ++e)
-          if ((present & (1u << e)) && pack_key(c.v[e], c.lab[e]) >= thr) flags |= 1u << e;
-        append_flagged(rr, it, c, flags, sh.sel_key, sh.sel_col, &sh.cnt, kMaxTopK);
-      }
+      thr = radix_select_row(sh, rr, static_cast<uint32_t>(kk));
+      // exactly kk entries pass: they become the candidate list
+      list_row(rr, [&](float v, int32_t lb) { return pack_key(v, lb) >= thr; }, sh.cand_val, sh.cand_lab, &sh.ccnt,
+               kCandCap);
     }
     __syncthreads();
-  } else if (kk > 0) {
+  }
+  if (kk > 0) {
     // ---- 4. select inside the candidate list ------------------------------
-    const int nc = static_cast<int>(sh.ccnt);
+    const int nc = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(kCandCap)));
     unsigned long long thr = 0ull;
     if (nc > kk) thr = radix_select_cand(sh, nc, static_cast<uint32_t>(kk));
     if (tid == 0) sh.cnt = 0;
@@ -479,15 +654,23 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     const int rounds = (nc + kTopkThreads - 1) / kTopkThreads;
     for (int rd = 0; rd < rounds; ++rd) {
       const int i = rd * kTopkThreads + tid;
-      const bool take = i < nc && sh.cand_key[i] >= thr;
+      unsigned long long key = 0ull;
+      float val = 0.f;
+      if (i < nc) {
+        val = sh.cand_val[i];
+        key = pack_key(val, sh.cand_lab[i]);
+      }
+      const bool take = i < nc && key >= thr;
       const uint32_t bal = __ballot_sync(0xffffffffu, take);
       uint32_t base = 0;
       if (lane == 0 && bal) base = atomicAdd(&sh.cnt, __popc(bal));
       base = __shfl_sync(0xffffffffu, base, 0);
       if (take) {
         const uint32_t s = base + __popc(bal & ((1u << lane) - 1u));
-        sh.sel_key[s] = sh.cand_key[i];
-        sh.sel_col[s] = sh.cand_col[i];
+        if (s < static_cast<uint32_t>(kMaxTopK)) {
+          sh.sel_key[s] = key;
+          sh.sel_val[s] = val;
+        }
       }
     }
     __syncthreads();
@@ -519,12 +702,24 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       sh.fill[i] = 0;
     }
     __syncthreads();
+    if (warp == 0) {
+      kmin = sh.wmin[lane];
+      kmax = sh.wmax[lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+        const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
+        kmin = a < kmin ? a : kmin;
+        kmax = b > kmax ? b : kmax;
+      }
+      if (lane == 0) {
+        sh.wmin[0] = kmin;
+        sh.wmax[0] = kmax;
+      }
+    }
+    __syncthreads();
     kmin = sh.wmin[0];
     kmax = sh.wmax[0];
-    for (int wi = 1; wi < kTopkWarps; ++wi) {
-      kmin = sh.wmin[wi] < kmin ? sh.wmin[wi] : kmin;
-      kmax = sh.wmax[wi] > kmax ? sh.wmax[wi] : kmax;
-    }
     const unsigned long long span = kmax - kmin;
     const int shift = span ? max(0, 64 - __clzll(static_cast<long long>(span)) - kHistBits) : 0;
     for (int i = tid; i < kk; i += kTopkThreads)
@@ -532,25 +727,25 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     __syncthreads();
     // bucket offsets from the top (largest keys first); fill holds the offsets
     scan_bins_2048(sh, sh.hist, sh.fill, 0u);
-    // scatter into buckets (the candidate buffer is free now)
+    // scatter into buckets
     for (int i = tid; i < kk; i += kTopkThreads) {
       const unsigned long long key = sh.sel_key[i];
       const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
       const uint32_t pos = atomicAdd(&sh.fill[bin], 1u);
-      sh.cand_key[pos] = key;
-      sh.cand_col[pos] = sh.sel_col[i];
+      sh.tmp_key[pos] = key;
+      sh.tmp_val[pos] = sh.sel_val[i];
     }
     __syncthreads();
     // rank inside the bucket: after the scatter fill[bin] is the bucket's end
     for (int i = tid; i < kk; i += kTopkThreads) {
-      const unsigned long long key = sh.cand_key[i];
+      const unsigned long long key = sh.tmp_key[i];
       const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
       const uint32_t end = sh.fill[bin];
       const uint32_t beg = end - sh.hist[bin];
       uint32_t rank = beg;
-      for (uint32_t j = beg; j < end; ++j) rank += (sh.cand_key[j] > key) ? 1u : 0u;
+      for (uint32_t j = beg; j < end; ++j) rank += (sh.tmp_key[j] > key) ? 1u : 0u;
       io[rank] = static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull));
-      if (vo) vo[rank] = rr.v[sh.cand_col[i]];
+      if (vo) vo[rank] = sh.tmp_val[i];
     }
   }
   for (int j = kk + tid; j < p.k; j += kTopkThreads) {
