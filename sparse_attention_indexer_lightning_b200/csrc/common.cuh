@@ -276,6 +276,12 @@ __device__ __forceinline__ void ffma2_acc(float& d0, float& d1, float a0, float 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// ReLU on the FMA pipe: x + |x| is 2 * max(x, 0) exactly (one FADD with an
+// absolute-value operand), where fmaxf would issue on the busier ALU pipe.
+// The factor 2 is taken out once per key at the end (a power of two, so the
+// result is bit-identical to summing w * max(x, 0)).
+__device__ __forceinline__ float relu2(float x) { return x + fabsf(x); }
+
 // Weighted-ReLU head reduction of one key's 32 head dot products:
 //   sum_h w[h] * max(0, scale * v[h])
 // with 8 independent partial sums updated two at a time by packed FMAs (a
@@ -290,16 +296,16 @@ __device__ __forceinline__ float head_reduce(const float (&v)[32], const float* 
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float a0 = fmaxf(SCALED ? scale * v[4 * i + 0] : v[4 * i + 0], 0.f);
-    const float a1 = fmaxf(SCALED ? scale * v[4 * i + 1] : v[4 * i + 1], 0.f);
-    const float a2 = fmaxf(SCALED ? scale * v[4 * i + 2] : v[4 * i + 2], 0.f);
-    const float a3 = fmaxf(SCALED ? scale * v[4 * i + 3] : v[4 * i + 3], 0.f);
+    const float a0 = relu2(SCALED ? scale * v[4 * i + 0] : v[4 * i + 0]);
+    const float a1 = relu2(SCALED ? scale * v[4 * i + 1] : v[4 * i + 1]);
+    const float a2 = relu2(SCALED ? scale * v[4 * i + 2] : v[4 * i + 2]);
+    const float a3 = relu2(SCALED ? scale * v[4 * i + 3] : v[4 * i + 3]);
     const int p = (2 * i) & 7;
     ffma2_acc(acc[p], acc[p + 1], a0, a1, wv[i].x, wv[i].y);
     const int q = (2 * i + 2) & 7;
     ffma2_acc(acc[q], acc[q + 1], a2, a3, wv[i].z, wv[i].w);
   }
-  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  return 0.5f * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
 }
 
 // head_reduce with the 32 head weights already in registers.
@@ -308,10 +314,9 @@ __device__ __forceinline__ float head_reduce_w(const uint32_t (&r)[32], const fl
 #pragma unroll
   for (int h = 0; h < 32; h += 2) {
     const int p = h & 7;
-    ffma2_acc(acc[p], acc[p + 1], fmaxf(__uint_as_float(r[h]), 0.f), fmaxf(__uint_as_float(r[h + 1]), 0.f), w[h],
-              w[h + 1]);
+    ffma2_acc(acc[p], acc[p + 1], relu2(__uint_as_float(r[h])), relu2(__uint_as_float(r[h + 1])), w[h], w[h + 1]);
   }
-  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  return 0.5f * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
 }
 
 // sum_h w[h] * max(0, sc * v[h]) for a per-key scale sc of either sign:

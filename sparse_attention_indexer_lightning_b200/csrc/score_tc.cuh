@@ -15,7 +15,8 @@
 // Roles (one persistent CTA per SM, contiguous runs of work units):
 //   warp 0      TMA producer (keys every unit, the query tile on group change)
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2..   epilogue (4 warps for QG = 1, 8 for QG = 8)
+//   warps 2..   epilogue (4 warps for QG = 1, 12 for QG = 8: three per TMEM
+//               lane quadrant, sharing the 8 queries of a group 3 / 3 / 2)
 // Pipelines: STAGES key buffers (full/empty mbarriers), 2 query-tile slots,
 // 2 TMEM accumulators so the epilogue of unit i overlaps the MMA of unit i+1.
 // Every wait is bounded; a wait that runs out raises the library fault word
@@ -43,9 +44,12 @@ struct TcCfg {
                                    : (ACC * ACC_COLS <= 64) ? 64
                                    : (ACC * ACC_COLS <= 128) ? 128
                                    : (ACC * ACC_COLS <= 256) ? 256 : 512;
-  static constexpr int EPI_WARPS = (QG == 1) ? 4 : 8;
+  // Epilogue warps come in sets of 4 (one per TMEM lane quadrant); the QG
+  // queries of a group are split between the EPI_SETS warps of a quadrant.
+  static constexpr int EPI_SETS = (QG == 1) ? 1 : 3;
+  static constexpr int EPI_WARPS = 4 * EPI_SETS;
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
-  static constexpr int Q_PER_EPI_WARP = (QG == 1) ? 1 : QG / 2;
+  static constexpr int Q_PER_EPI_WARP = (QG + EPI_SETS - 1) / EPI_SETS;
   static constexpr size_t SMEM_A = size_t(STAGES) * A_BYTES;
   static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
   static constexpr size_t SMEM_BAR = 512;
@@ -76,6 +80,16 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
       return;
     }
   }
+}
+
+// Keys of the whole history query (b, t) may see: a precomputed count, or
+// floor((q_pos + 1) / stride) capped at n_total (block-complete causal rule).
+__device__ __forceinline__ int eligible_keys(const ScoreParams& p, int b, int t) {
+  const int64_t row = static_cast<int64_t>(b) * p.T + t;
+  if (p.lim_rows) return __ldg(p.lim_rows + row);
+  const int64_t qp = __ldg(p.q_pos + row);
+  int64_t e = qp < 0 ? 0 : (qp + 1) / p.stride;
+  return static_cast<int>(e > p.n_total ? p.n_total : e);
 }
 
 template <int QG>
@@ -236,11 +250,15 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
     // soon as the last load of the unit has landed in registers.
     const int ew = warp - 2;                  // 0 .. EPI_WARPS-1
     const int quad = warp & 3;                // TMEM lane quadrant this warp may read
-    const int qset = (QG == 1) ? 0 : (ew >> 2);
+    const int qset = ew >> 2;                 // which share of the group's queries
     int acc = 0;
     uint32_t acc_phase = 0;
     long long w_row = -1;                     // QG == 1: row whose weights sit in wreg
     float wreg[32];
+    long long lim_bg = -1;                    // group whose per-query limits sit in elig
+    int elig[C::Q_PER_EPI_WARP];
+#pragma unroll
+    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) elig[i] = 0;
     UnitPos up;
     up.init(u_begin, NT, G);
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
@@ -249,7 +267,9 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
       const int n = tile * C::BM + quad * 32 + lane;       // key within this launch
       int lim = p.N;
       if (p.n_valid) lim = min(lim, __ldg(p.n_valid + b));
-      int nq = p.T - g * QG - qset * C::Q_PER_EPI_WARP;   // queries of this warp in the group
+      // queries of this warp in the group: its share of the QG columns blocks,
+      // cut by the group size and by the last group's end
+      int nq = min(p.T - g * QG, QG) - qset * C::Q_PER_EPI_WARP;
       nq = nq < 0 ? 0 : (nq > C::Q_PER_EPI_WARP ? C::Q_PER_EPI_WARP : nq);
       if (QG == 1 && w_row != bg) {                        // one query per sequence: weights per row
         const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * p.T * kHeads);
@@ -295,15 +315,12 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
             s = head_reduce<false>(v, p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads, 1.f);
           }
           int lim_t = lim;
-          if (p.lim_rows) {
-            const int rel = __ldg(p.lim_rows + static_cast<int64_t>(b) * p.T + t) - p.key_base;
+          if (p.lim_rows || p.q_pos) {
+            // eligible keys of this query (whole history), re-derived only when
+            // the query group changes
+            if (lim_bg != bg) elig[jq] = eligible_keys(p, b, t);
+            const int rel = elig[jq] - p.key_base;
             lim_t = rel < 0 ? 0 : (rel < lim_t ? rel : lim_t);
-          } else if (p.q_pos) {
-            const int64_t qp = p.q_pos[static_cast<int64_t>(b) * p.T + t];
-            int64_t e = qp < 0 ? 0 : (qp + 1) / p.stride;
-            if (e > p.n_total) e = p.n_total;
-            const int64_t rel = e - p.key_base;
-            lim_t = static_cast<int>(rel < 0 ? 0 : (rel < lim_t ? rel : lim_t));
           }
           if (n < p.N) {
             p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
@@ -319,6 +336,7 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
           }
         }
       }
+      lim_bg = bg;
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
       if (use_hist && (u + 1 == u_end || tile + 1 == NT)) {
         // the row (one query per sequence here) ends in this CTA: publish its counts
