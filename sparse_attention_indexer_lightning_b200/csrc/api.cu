@@ -177,6 +177,7 @@ ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_
   ls_status s = make_bf16_map(&qmap, q, static_cast<uint64_t>(q_rows_total), kHeads);
   if (s != LS_OK) return s;
   CvtParams p;
+  p.q = q;
   p.keys = keys;
   p.scale = scale;
   p.rows = rows;

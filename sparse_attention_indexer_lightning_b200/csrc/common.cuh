@@ -237,6 +237,30 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// Instruction descriptor, kind::f16: A = B = f16, D = f32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                                  // D format f32 (A, B format 0 = f16)
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// 2^e as a float, exactly, for -126 <= e <= 127 (clamped).
+__device__ __forceinline__ float exp2i(int e) {
+  e = e < -126 ? -126 : (e > 127 ? 127 : e);
+  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+// Shift that brings a head's largest |q| into [2^14, 2^15): q * 2^s is then
+// an fp16 value without overflow, and keeps full fp16 precision for every
+// element within 2^28 of that largest one.  0 for an all-zero or non-finite head.
+__device__ __forceinline__ int f16_head_shift(float maxabs) {
+  const uint32_t bits = __float_as_uint(maxabs);
+  const int e = static_cast<int>((bits >> 23) & 0xffu);
+  if (maxabs == 0.f || e == 0xff) return 0;
+  const int sh = 14 - (e - 127);
+  return sh > 126 ? 126 : sh;  // keeps 2^s and 2^-s both normal floats
+}
+
 // --------------------------------------------------------------------------
 // small helpers
 // --------------------------------------------------------------------------

@@ -48,6 +48,7 @@ enum SrcFormat : int { SRC_INT8 = 0, SRC_E4M3 = 1, SRC_BF16 = 2 };
 //   rows != nullptr : b*key_stride + rows[b*N + j] (gathered; < 0 = padding)
 //   out[b*N + j] = sum_h w[b,h] * relu(scale * (q[b,h] . code))   (or -inf)
 struct CvtParams {
+  const uint16_t* q;       // bf16 query rows (problem b, head h: row b*q_row_stride + h)
   const void* keys;        // base of the key rows
   const float* scale;      // per-key scale, indexed like the key rows (nullptr for bf16)
   const int32_t* rows;     // [B][N] gathered row ids or nullptr

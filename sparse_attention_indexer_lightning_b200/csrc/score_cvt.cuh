@@ -10,9 +10,13 @@
 //
 //   score = sum_h w[h] * max(0, scale * (q[h] . code))
 //
-// Both 8-bit formats widen to bf16 exactly (int8 magnitudes <= 128 and e4m3
-// values fit bf16's 8-bit significand and exponent range), so the contraction
-// runs as a bf16 x bf16 -> fp32 tcgen05 MMA with one key per TMEM lane.
+// Both 8-bit formats widen to fp16 exactly (int8 magnitudes <= 128; e4m3 is a
+// subset of fp16), and the query tile is rescaled per head by a power of two
+// (largest |q| into [2^14, 2^15)) and rounded to fp16 in shared memory, which
+// is exact for every element within 2^28 of its head's largest; the head
+// weights get the inverse power of two, so the contraction runs as an
+// f16 x f16 -> fp32 tcgen05 MMA with one key per TMEM lane and the scores
+// equal the bf16 formula.  Gathered bf16 keys use a bf16 x bf16 MMA.
 //
 // Roles (448 threads, one persistent CTA per SM):
 //   warp 0      producer: 1-D bulk copies of raw rows (one copy per tile when
@@ -99,6 +103,81 @@ __device__ __forceinline__ void i8x4_to_bf16x4(uint32_t x, uint32_t& lo, uint32_
                               *reinterpret_cast<const __nv_bfloat162*>(&o1));
   lo = *reinterpret_cast<uint32_t*>(&r0);
   hi = *reinterpret_cast<uint32_t*>(&r1);
+}
+
+// 4 signed bytes -> 4 fp16, exactly: the half pattern 0x6400 | (v + 128) is
+// 1024 + v + 128, and subtracting 1152 leaves v.
+__device__ __forceinline__ void i8x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  const uint32_t y = x ^ 0x80808080u;
+  const uint32_t t0 = __byte_perm(y, 0x64646464u, 0x4140);
+  const uint32_t t1 = __byte_perm(y, 0x64646464u, 0x4342);
+  const uint32_t m = 0x64806480u;  // 1152.0 in each half
+  __half2 r0 = __hsub2(*reinterpret_cast<const __half2*>(&t0), *reinterpret_cast<const __half2*>(&m));
+  __half2 r1 = __hsub2(*reinterpret_cast<const __half2*>(&t1), *reinterpret_cast<const __half2*>(&m));
+  lo = *reinterpret_cast<uint32_t*>(&r0);
+  hi = *reinterpret_cast<uint32_t*>(&r1);
+}
+
+// 4 e4m3 codes -> 4 fp16, exactly (one conversion per pair).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+// The query tile of one problem (32 heads x 128, K-major, 128-byte swizzle) in
+// shared memory: lane h rescales head h by 2^s_h and rounds it to fp16 in
+// place (the swizzle only permutes 16-byte chunks inside a head's row).
+__device__ __forceinline__ void q_tile_to_f16(uint8_t* tile, int half_bytes, int lane) {
+  float mx = 0.f;
+#pragma unroll
+  for (int pnl = 0; pnl < 2; ++pnl) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + pnl * half_bytes + lane * 128 + c * 16);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] << 16)));
+        mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] & 0xffff0000u)));
+      }
+    }
+  }
+  const float sc = exp2i(f16_head_shift(mx));
+#pragma unroll
+  for (int pnl = 0; pnl < 2; ++pnl) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint4* pp = reinterpret_cast<uint4*>(tile + pnl * half_bytes + lane * 128 + c * 16);
+      uint4 v = *pp;
+      uint32_t* w4 = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2 h = __floats2half2_rn(__uint_as_float(w4[i] << 16) * sc,
+                                            __uint_as_float(w4[i] & 0xffff0000u) * sc);
+        w4[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      *pp = v;
+    }
+  }
+}
+
+// The same head shift, derived from the bf16 query rows in global memory.
+__device__ __forceinline__ int q_head_shift_global(const uint16_t* row) {
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  float mx = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint4 v = __ldg(r4 + c);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] << 16)));
+      mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] & 0xffff0000u)));
+    }
+  }
+  return f16_head_shift(mx);
 }
 
 // 2 e4m3 codes (low 16 bits of x, element 0 in the low byte) -> bf16x2, exact.
@@ -268,32 +347,42 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::BN);
-      int as = 0;
-      uint32_t aphase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      int prev_b = -1;
-      int bslot = 1;
-      uint32_t bphase[2] = {0, 0};
-      const uint32_t a_base = smem_u32(sA);
-      const uint32_t b_base = smem_u32(sB);
-      UnitPos up;
-      up.init(u_begin, NT, 1);
-      for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
-        const int b = up.b;
-        if (b != prev_b) {
-          if (prev_b >= 0) umma_commit(&bars->bempty[bslot]);
-          bslot ^= 1;
-          if (!mbar_wait(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
-          bphase[bslot] ^= 1;
-          prev_b = b;
+    // The whole warp follows the units: on a problem change its lanes turn the
+    // new query tile into fp16 (8-bit keys); lane 0 issues the MMAs.
+    constexpr bool F16 = FMT != SRC_BF16;
+    constexpr uint32_t idesc = F16 ? idesc_f16_f32(C::BM, C::BN) : idesc_bf16_f32(C::BM, C::BN);
+    int as = 0;
+    uint32_t aphase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int prev_b = -1;
+    int bslot = 1;
+    uint32_t bphase[2] = {0, 0};
+    const uint32_t a_base = smem_u32(sA);
+    const uint32_t b_base = smem_u32(sB);
+    UnitPos up;
+    up.init(u_begin, NT, 1);
+    for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
+      const int b = up.b;
+      if (b != prev_b) {
+        if (prev_b >= 0 && lane == 0) umma_commit(&bars->bempty[bslot]);
+        bslot ^= 1;
+        // every lane observes the barrier itself: all of them read the tile next
+        const bool ok = mbar_wait(&bars->bfull[bslot], bphase[bslot], abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        bphase[bslot] ^= 1;
+        prev_b = b;
+        if (F16) {
+          q_tile_to_f16(sB + bslot * C::B_BYTES, C::B_HALF, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
         }
-        if (!mbar_wait(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
-        tc_fence_after();
-        if (!mbar_wait(&bars->afull[as], aphase, abort_flag)) break;
-        tc_fence_after();
+      }
+      if (!warp_wait(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
+      tc_fence_after();
+      if (!warp_wait(&bars->afull[as], aphase, abort_flag)) break;
+      tc_fence_after();
+      if (lane == 0) {
         const uint32_t a_addr = a_base + as * C::A_BYTES;
         const uint32_t b_addr = b_base + bslot * C::B_BYTES;
         const uint32_t d_tmem = tmem_base + acc * C::BN;
@@ -306,9 +395,12 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
         }
         umma_commit(&bars->aempty[as]);
         umma_commit(&bars->tfull[acc]);
-        if (++as == C::AS) { as = 0; aphase ^= 1; }
-        if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
       }
+      __syncwarp();
+      if (++as == C::AS) { as = 0; aphase ^= 1; }
+      if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
+    }
+    if (lane == 0) {
       umma_commit(&bars->drain);
       cvt_wait_drain(&bars->drain, 0);
     }
@@ -356,15 +448,15 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
           const int row = id >> 3, cc = id & 7;
           uint4 o0, o1;
           if (FMT == SRC_INT8) {
-            i8x4_to_bf16x4(v[i].x, o0.x, o0.y);
-            i8x4_to_bf16x4(v[i].y, o0.z, o0.w);
-            i8x4_to_bf16x4(v[i].z, o1.x, o1.y);
-            i8x4_to_bf16x4(v[i].w, o1.z, o1.w);
+            i8x4_to_f16x4(v[i].x, o0.x, o0.y);
+            i8x4_to_f16x4(v[i].y, o0.z, o0.w);
+            i8x4_to_f16x4(v[i].z, o1.x, o1.y);
+            i8x4_to_f16x4(v[i].w, o1.z, o1.w);
           } else {
-            e4m3x4_to_bf16x4(v[i].x, o0.x, o0.y);
-            e4m3x4_to_bf16x4(v[i].y, o0.z, o0.w);
-            e4m3x4_to_bf16x4(v[i].z, o1.x, o1.y);
-            e4m3x4_to_bf16x4(v[i].w, o1.z, o1.w);
+            e4m3x4_to_f16x4(v[i].x, o0.x, o0.y);
+            e4m3x4_to_f16x4(v[i].y, o0.z, o0.w);
+            e4m3x4_to_f16x4(v[i].z, o1.x, o1.y);
+            e4m3x4_to_f16x4(v[i].w, o1.z, o1.w);
           }
           const int panel = cc >> 2;
           const int j0 = (cc & 3) * 2;
@@ -419,15 +511,23 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
         if (tile + 1 == NT) fetch(b + 1, 0, nvalid, nsc);
         else fetch(b, tile + 1, nvalid, nsc);
       }
-      if (w_b != b) {                                // head weights of this problem, kept in registers
-        const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * kHeads);
+      if (w_b != b) {  // head weights of this problem, kept in registers
+        if (FMT != SRC_BF16) {
+          // lane h: head h's weight times 2^-s_h, the inverse of the query tile's shift
+          const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.q_row_stride + lane) * kDim;
+          const float wl = __ldg(p.w + static_cast<int64_t>(b) * kHeads + lane) * exp2i(-q_head_shift_global(qrow));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 t4 = __ldg(w4 + i);
-          wreg[4 * i] = t4.x;
-          wreg[4 * i + 1] = t4.y;
-          wreg[4 * i + 2] = t4.z;
-          wreg[4 * i + 3] = t4.w;
+          for (int i = 0; i < 32; ++i) wreg[i] = __shfl_sync(0xffffffffu, wl, i);
+        } else {
+          const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * kHeads);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 t4 = __ldg(w4 + i);
+            wreg[4 * i] = t4.x;
+            wreg[4 * i + 1] = t4.y;
+            wreg[4 * i + 2] = t4.z;
+            wreg[4 * i + 3] = t4.w;
+          }
         }
         w_b = b;
       }
