@@ -173,6 +173,42 @@ def to_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+
+def source_digest() -> str:
+    """sha256 (first 16 hex digits) over the CUDA sources and the C header: a
+    DRAM-traffic figure taken from an ncu capture counts only while it matches."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_attention_indexer_lightning_b200", "csrc")
+    files = [os.path.join(csrc, f) for f in sorted(os.listdir(csrc))]
+    files.append(os.path.join(ROOT, "include", "ls_indexer.h"))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload`, from the
+    ncu table in profiles/, or None when absent or taken from other sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            lines = f.read().splitlines()
+    except OSError:
+        return None
+    dig = source_digest()
+    for ln in lines:
+        if not ln.strip() or ln.startswith("#"):
+            continue
+        parts = ln.split("\t")
+        if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[3] == dig:
+            return float(parts[2])
+    return None
+
+
 def roofline(bound, achieved, peak, unit, traffic=None, peak_kind="measured"):
     return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind}
@@ -259,7 +295,7 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
         "breakdown_ms": {"scan": scan_ms, "topk": topk_ms},
         "kernels": {kname: {"total_ms": v[0], "launches": v[1]} for kname, v in prof.items()},
         "roofline": roofline("hbm", key_bytes / (scan_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
-                             traffic=args.scan_traffic, peak_kind=peak_kind),
+                             traffic=ncu_traffic("score_tc_kernel<1>", wl.name), peak_kind=peak_kind),
         "gpu_launches": launches,
         "clocks": clk,
     }
@@ -352,7 +388,8 @@ def bench_prefill(L, args, peaks, peak_kind):
     res = {
         "ms_per_step": ms, "positions_per_s": pairs / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
         "kernels": kern,
-        "roofline": roofline("tensor", flops_alg / (score_ms * 1e-3) / 1e12, peak_t, "TFLOP/s", peak_kind=peak_kind),
+        "roofline": roofline("tensor", flops_alg / (score_ms * 1e-3) / 1e12, peak_t, "TFLOP/s",
+                             traffic=ncu_traffic("score_tc_kernel<8>", wl.name), peak_kind=peak_kind),
         "algorithmic_flops": flops_alg, "eligible_pairs": pairs,
         "note": "step = 4 streamed 8192-key tiles (H2D on a copy stream) + causal top-512 of 4096 queries; "
                 "roofline over the 4 scoring launches of the step (score_tc_kernel<8>)",
@@ -389,7 +426,8 @@ def bench_bucket(L, args, peaks, peak_kind):
     peak_t = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
     res = {"ms_per_step": ms, "positions_per_s": T * (P_ + wl.budget) / (ms * 1e-3),
            "selections_per_s": T / (ms * 1e-3), "kernels": kern,
-           "roofline": roofline("tensor", flops / (cms * 1e-3) / 1e12, peak_t, "TFLOP/s", peak_kind=peak_kind),
+           "roofline": roofline("tensor", flops / (cms * 1e-3) / 1e12, peak_t, "TFLOP/s",
+                                traffic=ncu_traffic("score_tc_kernel<8>", wl.name), peak_kind=peak_kind),
            "algorithmic_flops_centroids": flops,
            "note": "positions = centroids scored + keys rescored per query; roofline of the centroid scoring"}
     del args_b, wsb
@@ -424,7 +462,7 @@ def bench_two_stage(L, args, peaks, peak_kind):
         "ms_per_step": ms, "positions_per_s": B * (N + wl.shortlist) / (ms * 1e-3),
         "selections_per_s": B / (ms * 1e-3), "kernels": kern,
         "roofline": roofline("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
-                             peak_kind=peak_kind),
+                             traffic=ncu_traffic("score_cvt_kernel<int8>", wl.name), peak_kind=peak_kind),
         "algorithmic_bytes_scan": scan_bytes,
         "note": "positions = compact keys scanned + shortlist re-ranked; roofline of the compact scan "
                 "(int8 codes + fp32 scales)",
@@ -508,8 +546,6 @@ def main(argv=None):
     ap.add_argument("--only", default=None, choices=["prefill_chunk", "bucket", "two_stage"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--scan-traffic", type=float, default=None,
-                    help="dram bytes per scan launch from an ncu capture of the current kernel")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

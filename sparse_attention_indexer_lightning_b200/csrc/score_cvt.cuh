@@ -47,8 +47,9 @@ struct CvtCfg {
   static constexpr int B_HALF = BN * 64 * 2;
   static constexpr int RS = (FMT == SRC_BF16) ? 3 : 6;   // raw stages
   static constexpr int AS = 3;                            // converted stages
-  static constexpr int ACC = 2;
-  static constexpr int TMEM_COLS = 64;
+  static constexpr int ACC = 8;  // accumulator stages in TMEM (32 columns each)
+  static constexpr int TMEM_COLS = ACC * BN;
+  static_assert(ACC <= 8 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation");
   static constexpr int CVT_WARPS = 8;
   static constexpr int CVT_GROUPS = 2;                       // tiles converted at once
   static constexpr int CVT_GROUP_WARPS = CVT_WARPS / CVT_GROUPS;
@@ -70,8 +71,8 @@ struct CvtBarriers {
   uint64_t aempty[4];
   uint64_t bfull[2];
   uint64_t bempty[2];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[8];
+  uint64_t tempty[8];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -231,6 +232,8 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->bfull[s], 1);
       mbar_init(&bars->bempty[s], 1);
+    }
+    for (int s = 0; s < C::ACC; ++s) {
       mbar_init(&bars->tfull[s], 1);
       mbar_init(&bars->tempty[s], C::EPI_WARPS);
     }
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp follows the units: on a problem change its lanes turn the
-    // new query tile into fp16 (8-bit keys); lane 0 issues the MMAs.
+    // new query tile into fp16 (8-bit keys); one elected lane issues the MMAs.
     constexpr bool F16 = FMT != SRC_BF16;
     constexpr uint32_t idesc = F16 ? idesc_f16_f32(C::BM, C::BN) : idesc_bf16_f32(C::BM, C::BN);
     int as = 0;
@@ -365,7 +368,7 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
       const int b = up.b;
       if (b != prev_b) {
-        if (prev_b >= 0 && lane == 0) umma_commit(&bars->bempty[bslot]);
+        if (prev_b >= 0) umma_commit_warp(&bars->bempty[bslot]);
         bslot ^= 1;
         // every lane observes the barrier itself: all of them read the tile next
         const bool ok = mbar_wait(&bars->bfull[bslot], bphase[bslot], abort_flag);
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
       tc_fence_after();
       if (!warp_wait(&bars->afull[as], aphase, abort_flag)) break;
       tc_fence_after();
-      if (lane == 0) {
+      {
         const uint32_t a_addr = a_base + as * C::A_BYTES;
         const uint32_t b_addr = b_base + bslot * C::B_BYTES;
         const uint32_t d_tmem = tmem_base + acc * C::BN;
@@ -391,19 +394,17 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
           const uint32_t koff = (kk & 3) * 32;
           const uint64_t adesc = sw128_kmajor_desc(a_addr + (kk >> 2) * C::A_HALF + koff);
           const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + koff);
-          umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+          umma_f16_warp(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->aempty[as]);
-        umma_commit(&bars->tfull[acc]);
+        umma_commit_warp(&bars->aempty[as]);
+        umma_commit_warp(&bars->tfull[acc]);
       }
-      __syncwarp();
       if (++as == C::AS) { as = 0; aphase ^= 1; }
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
     }
-    if (lane == 0) {
-      umma_commit(&bars->drain);
-      cvt_wait_drain(&bars->drain, 0);
-    }
+    umma_commit_warp(&bars->drain);
+    if (lane == 0) cvt_wait_drain(&bars->drain, 0);
+    __syncwarp();
   } else if (warp < 2 + C::CVT_WARPS) {
     // ------------------------------------------------------------ converters
     // CVT_GROUPS groups of warps take alternate units, so that many tiles are
@@ -435,17 +436,22 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
           *reinterpret_cast<uint4*>(a + panel * C::A_HALF + row * 128 + ((j ^ (row & 7)) << 4)) = v[i];
         }
       } else {
+        // A warp takes 4 rows x 8 input chunks per step.  Within each group of
+        // 8 lanes (one shared-memory wavefront) the even row's chunks 0-3 (or
+        // 4-7) pair with the odd row's other half: the 16-byte reads cover all
+        // 32 banks, and so do both widened stores, whose chunk indexes then
+        // differ in parity under the row swizzle.
         constexpr int PER = (C::BM * 8) / CT;
+        const int qg = (ct & 31) >> 3, rsel = (ct >> 2) & 1;
+        const int row0 = (ct >> 5) * 4 + 2 * (qg >> 1) + rsel;
+        const int cc = 4 * (rsel ^ (qg & 1)) + (ct & 3);
         uint4 v[PER];
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          const int id = i * CT + ct;
-          v[i] = *reinterpret_cast<const uint4*>(raw + (id >> 3) * 128 + (id & 7) * 16);
-        }
+        for (int i = 0; i < PER; ++i)
+          v[i] = *reinterpret_cast<const uint4*>(raw + (row0 + i * (CT / 8)) * 128 + cc * 16);
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-          const int id = i * CT + ct;
-          const int row = id >> 3, cc = id & 7;
+          const int row = row0 + i * (CT / 8);
           uint4 o0, o1;
           if (FMT == SRC_INT8) {
             i8x4_to_f16x4(v[i].x, o0.x, o0.y);

@@ -38,7 +38,7 @@ struct TcCfg {
   static constexpr int B_BYTES = BN * kDim * 2;
   static constexpr int B_HALF = BN * 64 * 2;
   static constexpr int STAGES = (QG == 1) ? 6 : 3;
-  static constexpr int ACC = 2;
+  static constexpr int ACC = (QG == 1) ? 8 : 2;       // accumulator stages in TMEM
   static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
   static constexpr int TMEM_COLS = (ACC * ACC_COLS <= 32) ? 32
                                    : (ACC * ACC_COLS <= 64) ? 64
@@ -56,6 +56,7 @@ struct TcCfg {
   static constexpr size_t SMEM_HIST = (QG == 1) ? kHistBins * 4 : 0;  // per-row selection histogram
   static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR + SMEM_HIST;
   static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
+  static_assert(ACC <= 8, "accumulator barriers");
 };
 
 struct TcBarriers {
@@ -63,8 +64,8 @@ struct TcBarriers {
   uint64_t empty[8];
   uint64_t bfull[2];
   uint64_t bempty[2];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[8];
+  uint64_t tempty[8];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -125,6 +126,8 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->bfull[s], 1);
       mbar_init(&bars->bempty[s], 1);
+    }
+    for (int s = 0; s < C::ACC; ++s) {
       mbar_init(&bars->tfull[s], 1);
       mbar_init(&bars->tempty[s], C::EPI_WARPS);
     }
@@ -197,51 +200,66 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::BN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      long long prev_bg = -1;
-      int bslot = 1;
-      uint32_t bphase[2] = {0, 0};
-      const uint32_t a_base = smem_u32(sA);
-      const uint32_t b_base = smem_u32(sB);
-      UnitPos up;
-      up.init(u_begin, NT, G);
-      for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
-        const long long bg = static_cast<long long>(up.b) * G + up.g;
-        if (bg != prev_bg) {
-          if (prev_bg >= 0) umma_commit(&bars->bempty[bslot]);
-          bslot ^= 1;
-          if (!mbar_wait(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
-          bphase[bslot] ^= 1;
-          prev_bg = bg;
+    // The whole warp runs the loop.  With one query per group (N = 32) the
+    // MMAs are short and one elected lane of the converged warp issues them;
+    // with eight (N = 256) the epilogue sets the pace and issuing from lane 0
+    // alone measured faster.
+    constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::BN);
+    constexpr bool ELECT = (QG == 1);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    long long prev_bg = -1;
+    int bslot = 1;
+    uint32_t bphase[2] = {0, 0};
+    const uint32_t a_base = smem_u32(sA);
+    const uint32_t b_base = smem_u32(sB);
+    UnitPos up;
+    up.init(u_begin, NT, G);
+    for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
+      const long long bg = static_cast<long long>(up.b) * G + up.g;
+      if (bg != prev_bg) {
+        if (prev_bg >= 0) {
+          if (ELECT) umma_commit_warp(&bars->bempty[bslot]);
+          else if (lane == 0) umma_commit(&bars->bempty[bslot]);
         }
-        if (!mbar_wait(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
-        tc_fence_after();
-        if (!mbar_wait(&bars->full[stage], phase, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a_addr = a_base + stage * C::A_BYTES;
-        const uint32_t b_addr = b_base + bslot * C::B_BYTES;
-        const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+        bslot ^= 1;
+        if (!warp_wait(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
+        bphase[bslot] ^= 1;
+        prev_bg = bg;
+      }
+      if (!warp_wait(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
+      tc_fence_after();
+      if (!warp_wait(&bars->full[stage], phase, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t a_addr = a_base + stage * C::A_BYTES;
+      const uint32_t b_addr = b_base + bslot * C::B_BYTES;
+      const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
 #pragma unroll
-        for (int kk = 0; kk < kDim / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside a 128 B swizzle row
-          const uint64_t adesc = sw128_kmajor_desc(a_addr + (kk >> 2) * C::A_HALF + koff);
-          const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + koff);
-          umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-        }
+      for (int kk = 0; kk < kDim / 16; ++kk) {
+        const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside a 128 B swizzle row
+        const uint64_t adesc = sw128_kmajor_desc(a_addr + (kk >> 2) * C::A_HALF + koff);
+        const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + koff);
+        if (ELECT) umma_f16_warp(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        else if (lane == 0) umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+      }
+      if (ELECT) {
+        umma_commit_warp(&bars->empty[stage]);
+        umma_commit_warp(&bars->tfull[acc]);
+      } else if (lane == 0) {
         umma_commit(&bars->empty[stage]);
         umma_commit(&bars->tfull[acc]);
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-        if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
       }
-      // All MMAs this thread issued are complete once `drain` flips.
-      umma_commit(&bars->drain);
-      mbar_wait_drain(&bars->drain, 0);
+      __syncwarp();
+      if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
     }
+    // All MMAs the issuing lane started are complete once `drain` flips.
+    if (ELECT) umma_commit_warp(&bars->drain);
+    else if (lane == 0) umma_commit(&bars->drain);
+    if (lane == 0) mbar_wait_drain(&bars->drain, 0);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     // Each warp owns the 32 keys of its TMEM lane quadrant and Q_PER_EPI_WARP
