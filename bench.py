@@ -456,13 +456,13 @@ def bench_two_stage(L, args, peaks, peak_kind):
         return None
 
     ms, kern = _profiled_loop(L, ts, steps, warm, st)
-    scan_ms = kern["score_cvt_kernel<int8>"]["ms_per_step"]
+    scan_ms = kern["score_q8_kernel<int8>"]["ms_per_step"]
     scan_bytes = B * N * (dd + 4)
     res = {
         "ms_per_step": ms, "positions_per_s": B * (N + wl.shortlist) / (ms * 1e-3),
         "selections_per_s": B / (ms * 1e-3), "kernels": kern,
         "roofline": roofline("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
-                             traffic=ncu_traffic("score_cvt_kernel<int8>", wl.name), peak_kind=peak_kind),
+                             traffic=ncu_traffic("score_q8_kernel<int8>", wl.name), peak_kind=peak_kind),
         "algorithmic_bytes_scan": scan_bytes,
         "note": "positions = compact keys scanned + shortlist re-ranked; roofline of the compact scan "
                 "(int8 codes + fp32 scales)",

@@ -18,6 +18,7 @@
 #include "ls_indexer.h"
 #include "misc.cuh"
 #include "score_cvt.cuh"
+#include "score_q8.cuh"
 #include "score_tc.cuh"
 #include "topk.cuh"
 
@@ -129,6 +130,22 @@ ls_status make_bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_
   return LS_OK;
 }
 
+// 2-D byte map over [rows][128] (one 8-bit key per row), box = 128 x 128 rows,
+// 128-byte swizzle.
+ls_status make_u8_map(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim), static_cast<cuuint32_t>(kTileKeys)};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LS_OK;
+}
+
 ls_status check_shape(int H, int d) {
   if (H != kHeads || d != kDim)
     return fail(LS_ERR_UNSUPPORTED, "only H=%d, d=%d are built (got H=%d, d=%d)", kHeads, kDim, H, d);
@@ -191,10 +208,20 @@ ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_
   p.N = N;
   p.fmt = fmt;
   p.hist = hist;
-  ProfScope prof(fmt == SRC_INT8 ? "score_cvt_kernel<int8>" : fmt == SRC_E4M3 ? "score_cvt_kernel<e4m3>"
-                                                                               : "score_cvt_kernel<bf16>",
-                 st);
-  LS_CUDA(launch_score_cvt(&qmap, p, num_sms_current(), st));
+  if (fmt == SRC_BF16) {
+    ProfScope prof("score_cvt_kernel<bf16>", st);
+    LS_CUDA(launch_score_cvt(&qmap, p, num_sms_current(), st));
+    return LS_OK;
+  }
+  // 8-bit keys: contiguous rows ([B][key_stride][128], key_stride == N) come in
+  // by 2-D TMA; gathered rows by per-row bulk copies (kmap unused)
+  CUtensorMap kmap = qmap;
+  if (rows == nullptr) {
+    s = make_u8_map(&kmap, keys, static_cast<uint64_t>(B) * static_cast<uint64_t>(key_stride));
+    if (s != LS_OK) return s;
+  }
+  ProfScope prof(fmt == SRC_INT8 ? "score_q8_kernel<int8>" : "score_q8_kernel<e4m3>", st);
+  LS_CUDA(launch_score_q8(&qmap, &kmap, p, num_sms_current(), st));
   return LS_OK;
 }
 

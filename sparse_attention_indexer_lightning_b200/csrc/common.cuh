@@ -183,6 +183,48 @@ __device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, f16 inputs: A is read from tensor memory
+// (row i in lane i, two 16-bit elements per 32-bit column).  Issued by a
+// converged warp through one elected lane, like umma_f16_warp.
+__device__ __forceinline__ void umma_f16_tmem_a_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                     uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit words from registers into TMEM: thread i of
+// the warp writes lane (base+i), columns col..col+31.
+__device__ __forceinline__ void tmem_st_32x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Wait until this thread's tcgen05.st writes are done.
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 4-byte asynchronous global -> shared copy (no register round trip).
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// The mbarrier gets one more pending arrival now, and receives it once every
+// cp.async this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -283,6 +325,84 @@ __device__ __forceinline__ int f16_head_shift(float maxabs) {
   if (maxabs == 0.f || e == 0xff) return 0;
   const int sh = 14 - (e - 127);
   return sh > 126 ? 126 : sh;  // keeps 2^s and 2^-s both normal floats
+}
+
+// --------------------------------------------------------------------------
+// 8-bit keys and the query tile in fp16
+// --------------------------------------------------------------------------
+// 4 signed bytes -> 4 fp16, exactly: the half pattern 0x6400 | (v + 128) is
+// 1024 + v + 128, and subtracting 1152 leaves v.
+__device__ __forceinline__ void i8x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  const uint32_t y = x ^ 0x80808080u;
+  const uint32_t t0 = __byte_perm(y, 0x64646464u, 0x4140);
+  const uint32_t t1 = __byte_perm(y, 0x64646464u, 0x4342);
+  const uint32_t m = 0x64806480u;  // 1152.0 in each half
+  __half2 r0 = __hsub2(*reinterpret_cast<const __half2*>(&t0), *reinterpret_cast<const __half2*>(&m));
+  __half2 r1 = __hsub2(*reinterpret_cast<const __half2*>(&t1), *reinterpret_cast<const __half2*>(&m));
+  lo = *reinterpret_cast<uint32_t*>(&r0);
+  hi = *reinterpret_cast<uint32_t*>(&r1);
+}
+
+// 4 e4m3 codes -> 4 fp16, exactly (one conversion per pair).
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+// The query tile of one problem (32 heads x 128, K-major, 128-byte swizzle) in
+// shared memory: lane h rescales head h by 2^s_h and rounds it to fp16 in
+// place (the swizzle only permutes 16-byte chunks inside a head's row).
+__device__ __forceinline__ void q_tile_to_f16(uint8_t* tile, int half_bytes, int lane) {
+  float mx = 0.f;
+#pragma unroll
+  for (int pnl = 0; pnl < 2; ++pnl) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + pnl * half_bytes + lane * 128 + c * 16);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] << 16)));
+        mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] & 0xffff0000u)));
+      }
+    }
+  }
+  const float sc = exp2i(f16_head_shift(mx));
+#pragma unroll
+  for (int pnl = 0; pnl < 2; ++pnl) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint4* pp = reinterpret_cast<uint4*>(tile + pnl * half_bytes + lane * 128 + c * 16);
+      uint4 v = *pp;
+      uint32_t* w4 = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half2 h = __floats2half2_rn(__uint_as_float(w4[i] << 16) * sc,
+                                            __uint_as_float(w4[i] & 0xffff0000u) * sc);
+        w4[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      *pp = v;
+    }
+  }
+}
+
+// The same head shift, derived from the bf16 query rows in global memory.
+__device__ __forceinline__ int q_head_shift_global(const uint16_t* row) {
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  float mx = 0.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint4 v = __ldg(r4 + c);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] << 16)));
+      mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] & 0xffff0000u)));
+    }
+  }
+  return f16_head_shift(mx);
 }
 
 // --------------------------------------------------------------------------

@@ -63,6 +63,10 @@ struct CvtParams {
   uint32_t* hist;          // [B][2048] selection histogram (counts added) or nullptr
 };
 cudaError_t launch_score_cvt(const CUtensorMap* qmap, const CvtParams& p, int num_sms, cudaStream_t st);
+// 8-bit keys (int8 / e4m3, fmt SRC_INT8 / SRC_E4M3); kmap covers the contiguous
+// key rows ([rows][128] bytes) and is ignored when p.rows gathers them.
+cudaError_t launch_score_q8(const CUtensorMap* qmap, const CUtensorMap* kmap, const CvtParams& p, int num_sms,
+                            cudaStream_t st);
 
 // ---------------------------------------------------------------- top-k
 // Row-wise top-k by (value desc, label asc); labels default to the column.

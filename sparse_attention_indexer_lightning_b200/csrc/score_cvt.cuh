@@ -106,81 +106,6 @@ __device__ __forceinline__ void i8x4_to_bf16x4(uint32_t x, uint32_t& lo, uint32_
   hi = *reinterpret_cast<uint32_t*>(&r1);
 }
 
-// 4 signed bytes -> 4 fp16, exactly: the half pattern 0x6400 | (v + 128) is
-// 1024 + v + 128, and subtracting 1152 leaves v.
-__device__ __forceinline__ void i8x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
-  const uint32_t y = x ^ 0x80808080u;
-  const uint32_t t0 = __byte_perm(y, 0x64646464u, 0x4140);
-  const uint32_t t1 = __byte_perm(y, 0x64646464u, 0x4342);
-  const uint32_t m = 0x64806480u;  // 1152.0 in each half
-  __half2 r0 = __hsub2(*reinterpret_cast<const __half2*>(&t0), *reinterpret_cast<const __half2*>(&m));
-  __half2 r1 = __hsub2(*reinterpret_cast<const __half2*>(&t1), *reinterpret_cast<const __half2*>(&m));
-  lo = *reinterpret_cast<uint32_t*>(&r0);
-  hi = *reinterpret_cast<uint32_t*>(&r1);
-}
-
-// 4 e4m3 codes -> 4 fp16, exactly (one conversion per pair).
-__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(x));
-}
-
-// The query tile of one problem (32 heads x 128, K-major, 128-byte swizzle) in
-// shared memory: lane h rescales head h by 2^s_h and rounds it to fp16 in
-// place (the swizzle only permutes 16-byte chunks inside a head's row).
-__device__ __forceinline__ void q_tile_to_f16(uint8_t* tile, int half_bytes, int lane) {
-  float mx = 0.f;
-#pragma unroll
-  for (int pnl = 0; pnl < 2; ++pnl) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(tile + pnl * half_bytes + lane * 128 + c * 16);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] << 16)));
-        mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] & 0xffff0000u)));
-      }
-    }
-  }
-  const float sc = exp2i(f16_head_shift(mx));
-#pragma unroll
-  for (int pnl = 0; pnl < 2; ++pnl) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint4* pp = reinterpret_cast<uint4*>(tile + pnl * half_bytes + lane * 128 + c * 16);
-      uint4 v = *pp;
-      uint32_t* w4 = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const __half2 h = __floats2half2_rn(__uint_as_float(w4[i] << 16) * sc,
-                                            __uint_as_float(w4[i] & 0xffff0000u) * sc);
-        w4[i] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-      *pp = v;
-    }
-  }
-}
-
-// The same head shift, derived from the bf16 query rows in global memory.
-__device__ __forceinline__ int q_head_shift_global(const uint16_t* row) {
-  const uint4* r4 = reinterpret_cast<const uint4*>(row);
-  float mx = 0.f;
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint4 v = __ldg(r4 + c);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] << 16)));
-      mx = fmaxf(mx, fabsf(__uint_as_float(w4[i] & 0xffff0000u)));
-    }
-  }
-  return f16_head_shift(mx);
-}
-
 // 2 e4m3 codes (low 16 bits of x, element 0 in the low byte) -> bf16x2, exact.
 __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t x) {
   uint32_t h2;
