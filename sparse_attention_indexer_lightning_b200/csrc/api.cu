@@ -130,16 +130,17 @@ ls_status make_bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_
   return LS_OK;
 }
 
-// 2-D byte map over [rows][128] (one 8-bit key per row), box = 128 x 128 rows,
-// 128-byte swizzle.
+// 2-D map over [rows][128 bytes] (one 8-bit key per row), box = 128 bytes x
+// 128 rows, 128-byte swizzle.  The bytes are described as 64 16-bit elements
+// per row: the copy and the swizzle act on bytes either way.
 ls_status make_u8_map(CUtensorMap* m, const void* base, uint64_t rows) {
   auto fn = encode_fn();
   if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim), static_cast<cuuint32_t>(kTileKeys)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim / 2), static_cast<cuuint32_t>(kTileKeys)};
   cuuint32_t es[2] = {1u, 1u};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));

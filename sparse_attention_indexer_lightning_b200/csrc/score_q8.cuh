@@ -17,6 +17,12 @@
 // rows written and read once and 8 KB of query-tile reads: the widened keys
 // never pass through it.
 //
+// A unit is HALVES x 128 keys of one problem: 256 for contiguous keys (one
+// pipeline hand-off per 32 KB; with 16 KB units the hand-offs alone held the
+// stream to ~4.6 TB/s in a producer-only measurement, 32 KB units ran at
+// ~6.1 TB/s), 128 for gathered rows.  Each 128-key half has its own TMEM lane
+// block (A and D columns), so a unit is 2 x 8 MMAs.
+//
 // Roles (448 threads, one persistent CTA per SM):
 //   warp 0      producer: raw rows (one 2-D TMA box with the 128-byte swizzle
 //               when the keys are contiguous; one 128-byte bulk copy per row at
@@ -36,19 +42,24 @@
 
 namespace lsi {
 
+template <int HALVES>
 struct Q8Cfg {
-  static constexpr int BM = kTileKeys;                  // keys per unit (TMEM lanes)
+  static constexpr int BM = kTileKeys;                  // keys per half (TMEM lanes)
+  static constexpr int KPU = HALVES * BM;               // keys per unit
   static constexpr int BN = kHeads;                     // one query per problem
   static constexpr int ROW = kDim;                      // bytes per 8-bit key row
-  static constexpr int PITCH_G = ROW + 16;              // gathered rows: 144-byte pitch
-  static constexpr int RAW_BYTES = BM * PITCH_G;        // 18 KB per raw stage (1024-multiple)
-  static constexpr int RS = 8;                          // raw stages
-  static constexpr int AS = 6;                          // widened stages in TMEM
-  static constexpr int ACC = 4;                         // accumulator stages in TMEM
-  static constexpr int A_COLS = kDim / 2;               // two fp16 per 32-bit column
-  static constexpr int A_COL0 = ACC * BN;
+  // gathered rows (HALVES == 1) land at a 144-byte pitch, contiguous ones as
+  // 128-byte rows under the TMA's 128-byte swizzle
+  static constexpr int PITCH = (HALVES == 1) ? ROW + 16 : ROW;
+  static constexpr int RAW_BYTES = KPU * PITCH;         // 1024-multiple
+  static constexpr int RS = (HALVES == 1) ? 8 : 6;      // raw stages
+  static constexpr int AS = 6 / HALVES;                 // widened stages in TMEM
+  static constexpr int ACC = 4 / HALVES;                // accumulator stages in TMEM
+  static constexpr int A_COLS = HALVES * (kDim / 2);    // two fp16 per 32-bit column
+  static constexpr int D_COLS = HALVES * BN;
+  static constexpr int A_COL0 = ACC * D_COLS;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SS = 8;                          // scale stages
+  static constexpr int SS = (HALVES == 1) ? 32 : 8;     // scale stages (the producer's lead over the epilogue)
   static constexpr int CVT_WARPS = 8;
   static constexpr int CVT_GROUPS = 2;
   static constexpr int CVT_GROUP_WARPS = CVT_WARPS / CVT_GROUPS;
@@ -58,32 +69,34 @@ struct Q8Cfg {
   static constexpr int B_HALF = BN * 64 * 2;
   static constexpr size_t SMEM_RAW = size_t(RS) * RAW_BYTES;
   static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
-  static constexpr size_t SMEM_S = size_t(SS) * BM * 8;  // per row: fp32 scale + int flag
-  static constexpr size_t SMEM_BAR = 512;
-  static constexpr size_t SMEM_HIST = kHistBins * 4;
-  static constexpr size_t SMEM_TOTAL = 1024 + SMEM_RAW + SMEM_B + SMEM_S + SMEM_BAR + SMEM_HIST;
+  static constexpr size_t S_BYTES = size_t(KPU) * 8;    // per key: fp32 scale + int flag
+  static constexpr size_t SMEM_S = size_t(SS) * S_BYTES;
+  static constexpr size_t SMEM_BAR = 1024;
+  static constexpr size_t SMEM_TOTAL = 1024 + SMEM_RAW + SMEM_B + SMEM_S + SMEM_BAR;
+  static_assert(HALVES == 1 || HALVES == 2, "128- or 256-key units");
   static_assert(RAW_BYTES % 1024 == 0, "swizzled stages need 1024-byte alignment");
   static_assert(A_COL0 + AS * A_COLS <= TMEM_COLS, "TMEM columns");
-  static_assert(CVT_GROUP_WARPS == 4, "one converter warp per TMEM lane quadrant");
+  static_assert(CVT_GROUP_WARPS == 4 && EPI_WARPS == 4, "one warp per TMEM lane quadrant");
+  static_assert(RS <= 8 && AS <= 6 && ACC <= 4 && SS <= 32, "barrier arrays");
   static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
 };
 
 struct Q8Barriers {
-  uint64_t rfull[Q8Cfg::RS];
-  uint64_t rempty[Q8Cfg::RS];
-  uint64_t afull[Q8Cfg::AS];
-  uint64_t aempty[Q8Cfg::AS];
+  uint64_t rfull[8];
+  uint64_t rempty[8];
+  uint64_t afull[6];
+  uint64_t aempty[6];
   uint64_t bfull[2];
   uint64_t bempty[2];
-  uint64_t tfull[Q8Cfg::ACC];
-  uint64_t tempty[Q8Cfg::ACC];
-  uint64_t sfull[Q8Cfg::SS];
-  uint64_t sempty[Q8Cfg::SS];
+  uint64_t tfull[4];
+  uint64_t tempty[4];
+  uint64_t sfull[32];
+  uint64_t sempty[32];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Q8Barriers) <= Q8Cfg::SMEM_BAR, "barrier block");
+static_assert(sizeof(Q8Barriers) <= 1024, "barrier block");
 
 // Drain wait: bounded by time only (used after an abort and at the end).
 __device__ __forceinline__ void q8_wait_drain(uint64_t* bar, uint32_t parity) {
@@ -113,30 +126,26 @@ __device__ __forceinline__ void widen16(const uint4& v, uint32_t* o) {
   }
 }
 
-template <int FMT>
-__global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
+template <int FMT, int HALVES>
+__global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
     score_q8_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                     const CvtParams p) {
-  using C = Q8Cfg;
+  using C = Q8Cfg<HALVES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sR = smem;
   uint8_t* sB = sR + C::SMEM_RAW;
   uint8_t* sS = sB + C::SMEM_B;
   Q8Barriers* bars = reinterpret_cast<Q8Barriers*>(sS + C::SMEM_S);
-  uint32_t* shist = reinterpret_cast<uint32_t*>(sS + C::SMEM_S + C::SMEM_BAR);
   volatile int* abort_flag = &bars->abort_flag;
-  const bool use_hist = p.hist != nullptr;
-  if (use_hist)
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) shist[i] = 0;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int NT = (p.N + C::BM - 1) / C::BM;
+  const int NT = (p.N + C::KPU - 1) / C::KPU;
   const long long units = static_cast<long long>(p.B) * NT;
   const long long u_begin = units * blockIdx.x / gridDim.x;
   const long long u_end = units * (blockIdx.x + 1) / gridDim.x;
-  const bool gathered = p.rows != nullptr;
+  const bool gathered = (HALVES == 1) && p.rows != nullptr;  // the launcher sends gathers to HALVES == 1
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::RS; ++s) {
@@ -227,16 +236,18 @@ __global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
       if (!warp_wait(&bars->rempty[rs], rphase ^ 1, abort_flag)) { ok = false; break; }
       if (!warp_wait(&bars->sempty[ss], sphase ^ 1, abort_flag)) { ok = false; break; }
       uint8_t* dst = sR + rs * C::RAW_BYTES;
-      float* ssc = reinterpret_cast<float*>(sS + ss * (C::BM * 8));
-      int* sok = reinterpret_cast<int*>(ssc + C::BM);
-      const int j0 = tile * C::BM;
+      float* ssc = reinterpret_cast<float*>(sS + ss * C::S_BYTES);
+      int* sok = reinterpret_cast<int*>(ssc + C::KPU);
+      const int j0 = tile * C::KPU;
       if (!gathered) {
         if (lane == 0) {
-          mbar_arrive_expect_tx(&bars->rfull[rs], C::BM * C::ROW);
-          tma_load_2d(dst, &kmap, &bars->rfull[rs], 0, b * p.N + j0);
+          mbar_arrive_expect_tx(&bars->rfull[rs], C::KPU * C::ROW);
+#pragma unroll
+          for (int h = 0; h < HALVES; ++h)
+            tma_load_2d(dst + h * C::BM * C::ROW, &kmap, &bars->rfull[rs], 0, b * p.N + j0 + h * C::BM);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4 * HALVES; ++i) {
           const int r = lane + 32 * i;
           const bool valid = j0 + r < nvb;
           sok[r] = valid ? 1 : 0;
@@ -271,7 +282,7 @@ __global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
           sok[r] = rid[i] >= 0 ? 1 : 0;
           if (rid[i] >= 0) {
             const int64_t src_row = static_cast<int64_t>(b) * p.key_stride + rid[i];
-            bulk_load(dst + r * C::PITCH_G, keys + src_row * C::ROW, C::ROW, &bars->rfull[rs]);
+            bulk_load(dst + r * C::PITCH, keys + src_row * C::ROW, C::ROW, &bars->rfull[rs]);
             cp_async_4(ssc + r, p.scale + src_row);
           }
         }
@@ -320,12 +331,15 @@ __global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
       if (!warp_wait(&bars->afull[as], aphase, abort_flag)) break;
       tc_fence_after();
       const uint32_t b_addr = b_base + bslot * C::B_BYTES;
-      const uint32_t d_tmem = tmem_base + acc * C::BN;
-      const uint32_t a_tmem = tmem_base + C::A_COL0 + as * C::A_COLS;
 #pragma unroll
-      for (int kk = 0; kk < kDim / 16; ++kk) {
-        const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + (kk & 3) * 32);
-        umma_f16_tmem_a_warp(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
+      for (int h = 0; h < HALVES; ++h) {
+        const uint32_t d_tmem = tmem_base + acc * C::D_COLS + h * C::BN;
+        const uint32_t a_tmem = tmem_base + C::A_COL0 + as * C::A_COLS + h * (kDim / 2);
+#pragma unroll
+        for (int kk = 0; kk < kDim / 16; ++kk) {
+          const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + (kk & 3) * 32);
+          umma_f16_tmem_a_warp(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
+        }
       }
       umma_commit_warp(&bars->aempty[as]);
       umma_commit_warp(&bars->tfull[acc]);
@@ -353,17 +367,20 @@ __global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
       const uint8_t* raw = sR + rs * C::RAW_BYTES;
       // contiguous: 128-byte rows, 16-byte chunk c stored at c ^ (row & 7);
       // gathered: 144-byte pitch, chunks in order
-      const uint8_t* rowp = gathered ? raw + row * C::PITCH_G : raw + row * C::ROW;
       const int sw = gathered ? 0 : (row & 7);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint4 v[4];
+      for (int h = 0; h < HALVES; ++h) {
+        const uint8_t* rowp = raw + (h * C::BM + row) * C::PITCH;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(rowp + (((half * 4 + c) ^ sw) << 4));
-        uint32_t o[32];
+        for (int part = 0; part < 2; ++part) {
+          uint4 v[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) widen16<FMT>(v[c], o + 8 * c);
-        tmem_st_32x32(t_row + as * C::A_COLS + half * 32, o);
+          for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(rowp + (((part * 4 + c) ^ sw) << 4));
+          uint32_t o[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) widen16<FMT>(v[c], o + 8 * c);
+          tmem_st_32x32(t_row + as * C::A_COLS + h * (kDim / 2) + part * 32, o);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -375,7 +392,6 @@ __global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    constexpr int EPI0 = (2 + C::CVT_WARPS) * 32;  // first epilogue thread
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     int acc = 0, ss = 0;
@@ -392,39 +408,44 @@ __global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
         const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.q_row_stride + lane) * kDim;
         const float wl = __ldg(p.w + static_cast<int64_t>(b) * kHeads + lane) * exp2i(-q_head_shift_global(qrow));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) wreg[i] = __shfl_sync(0xffffffffu, wl, i);
+        for (int h = 0; h < 32; ++h) wreg[h] = __shfl_sync(0xffffffffu, wl, h);
         w_b = b;
       }
       if (!warp_wait(&bars->sfull[ss], sphase, abort_flag)) break;
-      const float* ssc = reinterpret_cast<const float*>(sS + ss * (C::BM * 8));
-      const float sc = ssc[row];
-      const int valid = reinterpret_cast<const int*>(ssc + C::BM)[row];
+      const float* ssc = reinterpret_cast<const float*>(sS + ss * C::S_BYTES);
+      float sc[HALVES];
+      int valid[HALVES];
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) {
+        sc[h] = ssc[h * C::BM + row];
+        valid[h] = reinterpret_cast<const int*>(ssc + C::KPU)[h * C::BM + row];
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->sempty[ss]);
       if (++ss == C::SS) { ss = 0; sphase ^= 1; }
       if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_32x32_nowait(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::BN),
-                           v);
-      tmem_wait_ld(v);
+      const uint32_t t_d = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::D_COLS);
+      uint32_t v0[32], v1[32];
+      tmem_ld_32x32_nowait(t_d, v0);
+      if (HALVES == 2) tmem_ld_32x32_nowait(t_d + C::BN, v1);
+      tmem_wait_ld(v0);
+      if (HALVES == 2) tmem_wait_ld(v1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->tempty[acc]);
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
-      const int j = tile * C::BM + row;
-      if (j < p.N) {
-        float s = neg_inf();
-        if (valid) {
-          s = head_reduce_scaled(v, wreg, sc);
-          if (use_hist) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) {
+        const int j = tile * C::KPU + h * C::BM + row;
+        if (j < p.N) {
+          float s = neg_inf();
+          if (valid[h]) {
+            s = head_reduce_scaled(h == 0 ? v0 : v1, wreg, sc[h]);
+            if (p.hist) atomicAdd(p.hist + static_cast<int64_t>(b) * kHistBins + hist_bin(order_code(s)), 1u);
+          }
+          p.out[static_cast<int64_t>(b) * p.N + j] = s;
         }
-        p.out[static_cast<int64_t>(b) * p.N + j] = s;
-      }
-      if (use_hist && ((u + 1 == u_end) || (tile + 1 == NT))) {  // warp-uniform
-        role_barrier(1, C::EPI_WARPS * 32);
-        flush_hist(shist, p.hist + static_cast<int64_t>(b) * kHistBins, threadIdx.x - EPI0, C::EPI_WARPS * 32);
-        role_barrier(1, C::EPI_WARPS * 32);
       }
     }
   }
@@ -438,30 +459,36 @@ __global__ void __launch_bounds__(Q8Cfg::THREADS, 1)
   }
 }
 
-template <int FMT>
+template <int FMT, int HALVES>
 static cudaError_t launch_q8(const CUtensorMap* qmap, const CUtensorMap* kmap, const CvtParams& p, int num_sms,
                              cudaStream_t st) {
-  using C = Q8Cfg;
+  using C = Q8Cfg<HALVES>;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(score_q8_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(score_q8_kernel<FMT, HALVES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::SMEM_TOTAL));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const int NT = (p.N + C::BM - 1) / C::BM;
+  const int NT = (p.N + C::KPU - 1) / C::KPU;
   const long long units = static_cast<long long>(p.B) * NT;
   if (units == 0) return cudaSuccess;
   const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-  score_q8_kernel<FMT><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*qmap, *kmap, p);
+  score_q8_kernel<FMT, HALVES><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*qmap, *kmap, p);
   return cudaGetLastError();
 }
 
+// Contiguous keys take 256-key units, gathered rows 128-key units.
 cudaError_t launch_score_q8(const CUtensorMap* qmap, const CUtensorMap* kmap, const CvtParams& p, int num_sms,
                             cudaStream_t st) {
+  const bool gathered = p.rows != nullptr;
   switch (p.fmt) {
-    case SRC_INT8: return launch_q8<SRC_INT8>(qmap, kmap, p, num_sms, st);
-    case SRC_E4M3: return launch_q8<SRC_E4M3>(qmap, kmap, p, num_sms, st);
+    case SRC_INT8:
+      return gathered ? launch_q8<SRC_INT8, 1>(qmap, kmap, p, num_sms, st)
+                      : launch_q8<SRC_INT8, 2>(qmap, kmap, p, num_sms, st);
+    case SRC_E4M3:
+      return gathered ? launch_q8<SRC_E4M3, 1>(qmap, kmap, p, num_sms, st)
+                      : launch_q8<SRC_E4M3, 2>(qmap, kmap, p, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }
