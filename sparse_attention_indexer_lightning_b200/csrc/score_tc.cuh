@@ -46,7 +46,7 @@ struct TcCfg {
                                    : (ACC * ACC_COLS <= 256) ? 256 : 512;
   // Epilogue warps come in sets of 4 (one per TMEM lane quadrant); the QG
   // queries of a group are split between the EPI_SETS warps of a quadrant.
-  static constexpr int EPI_SETS = (QG == 1) ? 1 : 3;
+  static constexpr int EPI_SETS = (QG == 1) ? 1 : 4;
   static constexpr int EPI_WARPS = 4 * EPI_SETS;
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
   static constexpr int Q_PER_EPI_WARP = (QG + EPI_SETS - 1) / EPI_SETS;
@@ -263,9 +263,11 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     // Each warp owns the 32 keys of its TMEM lane quadrant and Q_PER_EPI_WARP
-    // queries of the group.  The TMEM load of query j+1 is issued before the
-    // reduction of query j; the accumulator is handed back to the MMA warp as
-    // soon as the last load of the unit has landed in registers.
+    // queries of the group.  One register buffer: a query's TMEM load, then
+    // its reduction (a second buffer for overlapping the next load measured
+    // slower: the registers it takes cost more than the overlap gives); the
+    // accumulator is handed back to the MMA warp as soon as the unit's last
+    // load has landed in registers.
     const int ew = warp - 2;                  // 0 .. EPI_WARPS-1
     const int quad = warp & 3;                // TMEM lane quadrant this warp may read
     const int qset = ew >> 2;                 // which share of the group's queries
@@ -305,13 +307,8 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * C::ACC_COLS + qset * C::Q_PER_EPI_WARP * kHeads);
-      // two register buffers, alternated by the fully unrolled query loop
-      uint32_t ra[32], rb[32];
-      if (nq > 0) {
-        tmem_ld_32x32_nowait(tbase, ra);
-        tmem_wait_ld(ra);
-      }
-      if (nq <= 1) {                                       // nothing more to read: release now
+      uint32_t cur[32];
+      if (nq == 0) {                                       // nothing to read: release now
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->tempty[acc]);
@@ -319,10 +316,14 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
 #pragma unroll
       for (int jq = 0; jq < C::Q_PER_EPI_WARP; ++jq) {
         if (jq < nq) {                                     // warp-uniform
-          uint32_t(&cur)[32] = (jq & 1) ? rb : ra;
-          uint32_t(&nxt)[32] = (jq & 1) ? ra : rb;
           const int t = g * QG + qset * C::Q_PER_EPI_WARP + jq;
-          if (jq + 1 < nq) tmem_ld_32x32_nowait(tbase + static_cast<uint32_t>((jq + 1) * kHeads), nxt);
+          tmem_ld_32x32_nowait(tbase + static_cast<uint32_t>(jq * kHeads), cur);
+          tmem_wait_ld(cur);
+          if (jq + 1 == nq) {                              // the unit's last load is in: release
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+          }
           float s;
           if (QG == 1) {
             s = head_reduce_w(cur, wreg);
@@ -343,14 +344,6 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
           if (n < p.N) {
             p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
             if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
-          }
-          if (jq + 1 < nq) {
-            tmem_wait_ld(nxt);
-            if (jq + 2 == nq) {                            // the unit's last load is in: release
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&bars->tempty[acc]);
-            }
           }
         }
       }
