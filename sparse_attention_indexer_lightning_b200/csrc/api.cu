@@ -243,7 +243,7 @@ ls_status topk(const float* scores, int64_t ld, const int32_t* n_valid, const in
   p.val_out = val;
   p.ld_out = ld_out;
   ProfScope prof("topk_kernel", st);
-  LS_CUDA(launch_topk(p, st));
+  LS_CUDA(launch_topk(p, st, num_sms_current()));
   return LS_OK;
 }
 

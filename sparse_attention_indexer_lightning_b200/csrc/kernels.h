@@ -83,7 +83,7 @@ struct TopkParams {
   float* val_out;          // [R][k] values (bit copies), -inf padding; may be nullptr
   int64_t ld_out;
 };
-cudaError_t launch_topk(const TopkParams& p, cudaStream_t st);
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t st, int num_sms);
 
 // ---------------------------------------------------------------- misc
 // n_valid[t] = clamp((q_pos[t] + 1) / stride, 0, n_total)

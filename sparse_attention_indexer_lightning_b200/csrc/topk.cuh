@@ -39,24 +39,24 @@
 
 namespace lsi {
 
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kCandCap = 8192;     // listed candidates kept in shared memory
 constexpr int kExactHistMax = 8192; // rows up to this length get an exact histogram
 constexpr int kVec = 4;            // float4 loads per thread per chunk
 constexpr int kChunk = kVec * 4;   // entries per thread per chunk
 
+// NT threads per CTA (one row each), KMAX the largest k the CTA holds.
+template <int NT, int KMAX>
 struct TopkShared {
   float cand_val[kCandCap];            // listed entries: value and label
   int32_t cand_lab[kCandCap];
-  unsigned long long sel_key[kMaxTopK];  // the k selected: packed key and value
-  float sel_val[kMaxTopK];
-  unsigned long long tmp_key[kMaxTopK];  // bucketed copy for the final order
-  float tmp_val[kMaxTopK];
+  unsigned long long sel_key[KMAX];    // the k selected: packed key and value
+  float sel_val[KMAX];
+  unsigned long long tmp_key[KMAX];    // bucketed copy for the final order
+  float tmp_val[KMAX];
   uint32_t hist[kHistBins];
   uint32_t fill[kHistBins];
-  uint32_t wsum[kTopkWarps];
-  unsigned long long wmin[kTopkWarps], wmax[kTopkWarps];
+  uint32_t wsum[NT / 32];
+  unsigned long long wmin[NT / 32], wmax[NT / 32];
   uint32_t digit, need, done, total, cnt, ccnt, eq;
 };
 
@@ -84,37 +84,40 @@ struct Chunk {
   int32_t lab[kChunk];  // label (the column when the row has none); < 0 = absent
 };
 
+template <int NT>
 __device__ __forceinline__ int chunk_count(const RowRef& rr) {
   if (rr.vec) {
     const int n4 = rr.n >> 2;
-    return (n4 + kVec * kTopkThreads - 1) / (kVec * kTopkThreads) + ((rr.n & 3) ? 1 : 0);
+    return (n4 + kVec * NT - 1) / (kVec * NT) + ((rr.n & 3) ? 1 : 0);
   }
-  return (rr.n + kChunk * kTopkThreads - 1) / (kChunk * kTopkThreads);
+  return (rr.n + kChunk * NT - 1) / (kChunk * NT);
 }
 
 // Column of entry e of chunk `it` for this thread.
+template <int NT>
 __device__ __forceinline__ int chunk_col(const RowRef& rr, int it, int e) {
   if (rr.vec) {
     const int n4 = rr.n >> 2;
-    const int body = (n4 + kVec * kTopkThreads - 1) / (kVec * kTopkThreads);
-    if (it < body) return 4 * ((it * kVec + (e >> 2)) * kTopkThreads + static_cast<int>(threadIdx.x)) + (e & 3);
+    const int body = (n4 + kVec * NT - 1) / (kVec * NT);
+    if (it < body) return 4 * ((it * kVec + (e >> 2)) * NT + static_cast<int>(threadIdx.x)) + (e & 3);
     return 4 * n4 + static_cast<int>(threadIdx.x);  // tail chunk: entry 0 only
   }
-  return (it * kChunk + e) * kTopkThreads + static_cast<int>(threadIdx.x);
+  return (it * kChunk + e) * NT + static_cast<int>(threadIdx.x);
 }
 
 // Loads chunk `it`; returns a bit per present entry.
+template <int NT>
 __device__ __forceinline__ uint32_t load_chunk(const RowRef& rr, int it, Chunk& c) {
   uint32_t present = 0;
   if (rr.vec) {
     const int n4 = rr.n >> 2;
-    const int body = (n4 + kVec * kTopkThreads - 1) / (kVec * kTopkThreads);
+    const int body = (n4 + kVec * NT - 1) / (kVec * NT);
     if (it < body) {
       float4 a[kVec];
       int4 b[kVec];
 #pragma unroll
       for (int u = 0; u < kVec; ++u) {
-        const int j = (it * kVec + u) * kTopkThreads + static_cast<int>(threadIdx.x);
+        const int j = (it * kVec + u) * NT + static_cast<int>(threadIdx.x);
         a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         b[u] = make_int4(-1, -1, -1, -1);
         if (j < n4) {
@@ -148,7 +151,7 @@ __device__ __forceinline__ uint32_t load_chunk(const RowRef& rr, int it, Chunk& 
   } else {
 #pragma unroll
     for (int e = 0; e < kChunk; ++e) {
-      const int i = (it * kChunk + e) * kTopkThreads + static_cast<int>(threadIdx.x);
+      const int i = (it * kChunk + e) * NT + static_cast<int>(threadIdx.x);
       c.v[e] = 0.f;
       c.lab[e] = -1;
       if (i < rr.n) {
@@ -165,7 +168,8 @@ __device__ __forceinline__ uint32_t load_chunk(const RowRef& rr, int it, Chunk& 
 
 // Warp 0: in a 256-bin histogram scanned from the top, find the digit d with
 // fewer than `want` keys above it and at least `want` at or above it.
-__device__ __forceinline__ void find_digit_256(TopkShared& sh, uint32_t want) {
+template <class SH>
+__device__ __forceinline__ void find_digit_256(SH& sh, uint32_t want) {
   const int lane = threadIdx.x;
   uint32_t c[8];
   uint32_t lsum = 0;
@@ -198,15 +202,22 @@ __device__ __forceinline__ void find_digit_256(TopkShared& sh, uint32_t want) {
 // All threads: exclusive prefix of a 2048-bin histogram taken from the top
 // (bin 2047 first) into `excl_out` (may alias nothing), the total into
 // sh.total, and for want = min(want_cap, total) > 0 the bin holding the
-// want-th entry (sh.digit / sh.need / sh.eq).
-__device__ __forceinline__ void scan_bins_2048(TopkShared& sh, const uint32_t* hist, uint32_t* excl_out,
+// want-th entry (sh.digit / sh.need / sh.eq).  Thread t takes the 2048 / NT
+// consecutive bins just below bin 2047 - t * (2048 / NT) + 1.
+template <int NT, class SH>
+__device__ __forceinline__ void scan_bins_2048(SH& sh, const uint32_t* hist, uint32_t* excl_out,
                                                uint32_t want_cap) {
+  constexpr int BPT = kHistBins / NT;
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  const int b0 = kHistBins - 1 - 2 * t, b1 = kHistBins - 2 - 2 * t;  // higher bin first
-  const uint32_t c0 = hist[b0], c1 = hist[b1];
-  const uint32_t c = c0 + c1;
-  uint32_t incl = c;
+  uint32_t c[BPT];
+  uint32_t csum = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    c[j] = hist[kHistBins - 1 - BPT * t - j];  // higher bin first
+    csum += c[j];
+  }
+  uint32_t incl = csum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -215,69 +226,31 @@ __device__ __forceinline__ void scan_bins_2048(TopkShared& sh, const uint32_t* h
   if (lane == 31) sh.wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t wv = sh.wsum[lane];
+    const uint32_t wv = lane < NT / 32 ? sh.wsum[lane] : 0u;
     uint32_t wi = wv;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t v = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += v;
     }
-    sh.wsum[lane] = wi - wv;
+    if (lane < NT / 32) sh.wsum[lane] = wi - wv;
     if (lane == 31) sh.total = wi;
   }
   __syncthreads();
-  const uint32_t excl = incl - c + sh.wsum[warp];
-  if (excl_out) {
-    excl_out[b0] = excl;
-    excl_out[b1] = excl + c0;
-  }
+  uint32_t excl = incl - csum + sh.wsum[warp];
   const uint32_t want = min(want_cap, sh.total);
-  if (want > 0 && excl < want && excl + c >= want) {
-    if (excl + c0 >= want) {
-      sh.digit = b0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    const int bin = kHistBins - 1 - BPT * t - j;
+    if (excl_out) excl_out[bin] = excl;
+    if (want > 0 && excl < want && excl + c[j] >= want) {
+      sh.digit = bin;
       sh.need = want - excl;
-      sh.eq = c0;
-    } else {
-      sh.digit = b1;
-      sh.need = want - excl - c0;
-      sh.eq = c1;
+      sh.eq = c[j];
     }
+    excl += c[j];
   }
   __syncthreads();
-}
-
-// Append the keys flagged in `flags` (bit e of the chunk) at slots handed out
-// by one atomic on `counter` per warp; slots >= cap are counted, not stored.
-// Warp-collective.
-__device__ __forceinline__ void append_flagged(const RowRef& rr, int it, const Chunk& c, uint32_t flags,
-                                               unsigned long long* keys, uint32_t* cols, uint32_t* counter,
-                                               uint32_t cap) {
-  if (!__any_sync(0xffffffffu, flags != 0u)) return;  // the common case in a listing pass
-  const uint32_t mine = __popc(flags);
-  uint32_t incl = mine;
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
-  if (tot == 0) return;
-  uint32_t base = 0;
-  if (lane == 31) base = atomicAdd(counter, tot);
-  base = __shfl_sync(0xffffffffu, base, 31);
-  if (!flags) return;
-  uint32_t slot = base + incl - mine;
-#pragma unroll
-  for (int e = 0; e < kChunk; ++e) {
-    if (flags & (1u << e)) {
-      if (slot < cap) {
-        keys[slot] = pack_key(c.v[e], c.lab[e]);
-        cols[slot] = static_cast<uint32_t>(chunk_col(rr, it, e));
-      }
-      ++slot;
-    }
-  }
 }
 
 __device__ __forceinline__ float f4at(const float4& a, int q) {
@@ -311,7 +284,7 @@ __device__ __forceinline__ uint32_t warp_slots(uint32_t flags, uint32_t* counter
 // labels when the row has them) per step; all threads run the same number of
 // steps.  Rows without labels skip every label computation until an entry is
 // flagged.
-template <bool HAS_LAB, class Keep>
+template <int NT, bool HAS_LAB, class Keep>
 __device__ __forceinline__ void list_row_t(const RowRef& rr, Keep keep, float* vals, int32_t* labs,
                                            uint32_t* counter, uint32_t cap) {
   const int tid = threadIdx.x;
@@ -319,13 +292,13 @@ __device__ __forceinline__ void list_row_t(const RowRef& rr, Keep keep, float* v
     const int n4 = rr.n >> 2;
     const float4* v4 = reinterpret_cast<const float4*>(rr.v);
     const int4* l4 = reinterpret_cast<const int4*>(rr.lab);
-    for (int base = 0; base < n4; base += kVec * kTopkThreads) {
+    for (int base = 0; base < n4; base += kVec * NT) {
       float4 a[kVec];
       int4 l[kVec];
       uint32_t inb = 0;  // bit u: vector u exists
 #pragma unroll
       for (int u = 0; u < kVec; ++u) {
-        const int j = base + u * kTopkThreads + tid;
+        const int j = base + u * NT + tid;
         a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (HAS_LAB) l[u] = make_int4(-1, -1, -1, -1);
         if (j < n4) {
@@ -338,7 +311,7 @@ __device__ __forceinline__ void list_row_t(const RowRef& rr, Keep keep, float* v
 #pragma unroll
       for (int e = 0; e < kChunk; ++e) {
         // label: the column when the row has none (dead code unless keep reads it)
-        const int32_t lb = HAS_LAB ? i4at(l[e >> 2], e & 3) : 4 * (base + (e >> 2) * kTopkThreads + tid) + (e & 3);
+        const int32_t lb = HAS_LAB ? i4at(l[e >> 2], e & 3) : 4 * (base + (e >> 2) * NT + tid) + (e & 3);
         const bool ok = HAS_LAB ? (lb >= 0) : ((inb >> (e >> 2)) & 1u);
         if (ok && keep(f4at(a[e >> 2], e & 3), lb)) flags |= 1u << e;
       }
@@ -349,7 +322,7 @@ __device__ __forceinline__ void list_row_t(const RowRef& rr, Keep keep, float* v
         if (flags & (1u << e)) {
           if (slot < cap) {
             vals[slot] = f4at(a[e >> 2], e & 3);
-            labs[slot] = HAS_LAB ? i4at(l[e >> 2], e & 3) : 4 * (base + (e >> 2) * kTopkThreads + tid) + (e & 3);
+            labs[slot] = HAS_LAB ? i4at(l[e >> 2], e & 3) : 4 * (base + (e >> 2) * NT + tid) + (e & 3);
           }
           ++slot;
         }
@@ -373,12 +346,12 @@ __device__ __forceinline__ void list_row_t(const RowRef& rr, Keep keep, float* v
       }
     }
   } else {
-    for (int base = 0; base < rr.n; base += kChunk * kTopkThreads) {
+    for (int base = 0; base < rr.n; base += kChunk * NT) {
       float a[kChunk];
       int32_t l[kChunk];
 #pragma unroll
       for (int e = 0; e < kChunk; ++e) {
-        const int i = base + e * kTopkThreads + tid;
+        const int i = base + e * NT + tid;
         a[e] = 0.f;
         l[e] = -1;
         if (i < rr.n) {
@@ -406,25 +379,26 @@ __device__ __forceinline__ void list_row_t(const RowRef& rr, Keep keep, float* v
   }
 }
 
-template <class Keep>
+template <int NT, class Keep>
 __device__ __forceinline__ void list_row(const RowRef& rr, Keep keep, float* vals, int32_t* labs, uint32_t* counter,
                                          uint32_t cap) {
-  if (rr.lab) list_row_t<true>(rr, keep, vals, labs, counter, cap);
-  else list_row_t<false>(rr, keep, vals, labs, counter, cap);
+  if (rr.lab) list_row_t<NT, true>(rr, keep, vals, labs, counter, cap);
+  else list_row_t<NT, false>(rr, keep, vals, labs, counter, cap);
 }
 
 // Plain path: MSB-first radix select over the whole row in global memory.
 // Returns the threshold T with exactly `want` present keys >= T.
-__device__ unsigned long long radix_select_row(TopkShared& sh, const RowRef& rr, uint32_t want) {
+template <int NT, class SH>
+__device__ unsigned long long radix_select_row(SH& sh, const RowRef& rr, uint32_t want) {
   unsigned long long prefix = 0ull;
-  const int chunks = chunk_count(rr);
+  const int chunks = chunk_count<NT>(rr);
   for (int hi = 64; hi > 0; hi -= 8) {
     const int shift = hi - 8;
-    for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
+    for (int i = threadIdx.x; i < 256; i += NT) sh.hist[i] = 0;
     __syncthreads();
     for (int it = 0; it < chunks; ++it) {
       Chunk c;
-      const uint32_t present = load_chunk(rr, it, c);
+      const uint32_t present = load_chunk<NT>(rr, it, c);
 #pragma unroll
       for (int e = 0; e < kChunk; ++e) {
         if (present & (1u << e)) {
@@ -449,10 +423,11 @@ __device__ unsigned long long radix_select_row(TopkShared& sh, const RowRef& rr,
 // starts at the highest bit where the candidates differ (their common high
 // bits are read off the smallest and largest key), so no pass is spent on
 // bits every candidate shares.
-__device__ unsigned long long radix_select_cand(TopkShared& sh, int nc, uint32_t want) {
+template <int NT, class SH>
+__device__ unsigned long long radix_select_cand(SH& sh, int nc, uint32_t want) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned long long kmin = ~0ull, kmax = 0ull;
-  for (int i = threadIdx.x; i < nc; i += kTopkThreads) {
+  for (int i = threadIdx.x; i < nc; i += NT) {
     const unsigned long long key = pack_key(sh.cand_val[i], sh.cand_lab[i]);
     kmin = key < kmin ? key : kmin;
     kmax = key > kmax ? key : kmax;
@@ -468,11 +443,11 @@ __device__ unsigned long long radix_select_cand(TopkShared& sh, int nc, uint32_t
     sh.wmin[warp] = kmin;
     sh.wmax[warp] = kmax;
   }
-  for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
+  for (int i = threadIdx.x; i < 256; i += NT) sh.hist[i] = 0;
   __syncthreads();
   if (warp == 0) {
-    kmin = sh.wmin[lane];
-    kmax = sh.wmax[lane];
+    kmin = lane < NT / 32 ? sh.wmin[lane] : ~0ull;
+    kmax = lane < NT / 32 ? sh.wmax[lane] : 0ull;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
@@ -496,11 +471,11 @@ __device__ unsigned long long radix_select_cand(TopkShared& sh, int nc, uint32_t
     const int width = hi < 8 ? hi : 8;
     const int shift = hi - width;
     if (!first) {
-      for (int i = threadIdx.x; i < 256; i += kTopkThreads) sh.hist[i] = 0;
+      for (int i = threadIdx.x; i < 256; i += NT) sh.hist[i] = 0;
       __syncthreads();
     }
     first = false;
-    for (int i = threadIdx.x; i < nc; i += kTopkThreads) {
+    for (int i = threadIdx.x; i < nc; i += NT) {
       const unsigned long long key = pack_key(sh.cand_val[i], sh.cand_lab[i]);
       if (hi >= 64 || (key >> hi) == (prefix >> hi))
         atomicAdd(&sh.hist[static_cast<uint32_t>(key >> shift) & ((1u << width) - 1u)], 1u);
@@ -518,9 +493,10 @@ __device__ unsigned long long radix_select_cand(TopkShared& sh, int nc, uint32_t
   return prefix;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
+template <int NT, int KMAX>
+__global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
+  TopkShared<NT, KMAX>& sh = *reinterpret_cast<TopkShared<NT, KMAX>*>(topk_smem);
   const int r = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -531,7 +507,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   if (p.n_valid) rr.n = max(0, min(rr.n, p.n_valid[r]));
   rr.vec = ((reinterpret_cast<uintptr_t>(rr.v) & 15u) == 0) &&
            (rr.lab == nullptr || (reinterpret_cast<uintptr_t>(rr.lab) & 15u) == 0);
-  const int chunks = chunk_count(rr);
+  const int chunks = chunk_count<NT>(rr);
   const uint32_t kcap = static_cast<uint32_t>(min(p.k, rr.n));  // k, or fewer entries
 
   // ---- 1. histogram of the top code bits ---------------------------------
@@ -543,12 +519,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   int S = 1;  // sampling period in groups of 8 entries
   if (p.hist) {
     const uint32_t* gh = p.hist + static_cast<int64_t>(r) * kHistBins;
-    for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = gh[i];
+    for (int i = tid; i < kHistBins; i += NT) sh.hist[i] = gh[i];
   } else {
-    for (int i = tid; i < kHistBins; i += kTopkThreads) sh.hist[i] = 0;
+    for (int i = tid; i < kHistBins; i += NT) sh.hist[i] = 0;
     __syncthreads();
     if (rr.n <= kExactHistMax) {
-      for (int i = tid; i < rr.n; i += kTopkThreads) {
+      for (int i = tid; i < rr.n; i += NT) {
         const int32_t l = rr.lab ? __ldg(rr.lab + i) : i;
         if (l >= 0) atomicAdd(&sh.hist[hist_bin(order_code(__ldg(rr.v + i)))], 1u);
       }
@@ -556,7 +532,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       exact_hist = false;
       while ((rr.n / S) > kExactHistMax) S <<= 1;
       const int groups = (rr.n + 7) >> 3;
-      for (int g = tid * S; g < groups; g += kTopkThreads * S) {
+      for (int g = tid * S; g < groups; g += NT * S) {
         const int i0 = g << 3;
         float v[8];
         int32_t l[8];
@@ -588,7 +564,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   // sample holds k/S entries with a 25% + 16 margin.
   uint32_t want_bins = kcap;
   if (!exact_hist) want_bins = (kcap + kcap / 4) / static_cast<uint32_t>(S) + 16u;
-  scan_bins_2048(sh, sh.hist, nullptr, max(want_bins, 1u));
+  scan_bins_2048<NT>(sh, sh.hist, nullptr, max(want_bins, 1u));
   uint32_t blo = sh.digit;
   const uint32_t hist_total = sh.total;
   if (hist_total == 0) blo = 0;                          // nothing present (or nothing sampled)
@@ -602,9 +578,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       // ---- listing pass: every present entry in a bin >= blo -------------
       if (blo >= 4) {  // bins from 4 up start at finite values: compare the score itself
         const float tlo = code_floor_value(blo << (32 - kHistBits));
-        list_row(rr, [&](float v, int32_t) { return v >= tlo; }, sh.cand_val, sh.cand_lab, &sh.ccnt, kCandCap);
+        list_row<NT>(rr, [&](float v, int32_t) { return v >= tlo; }, sh.cand_val, sh.cand_lab, &sh.ccnt, kCandCap);
       } else {
-        list_row(rr, [&](float v, int32_t) { return hist_bin(order_code(v)) >= blo; }, sh.cand_val, sh.cand_lab,
+        list_row<NT>(rr, [&](float v, int32_t) { return hist_bin(order_code(v)) >= blo; }, sh.cand_val, sh.cand_lab,
                  &sh.ccnt, kCandCap);
       }
       __syncthreads();
@@ -623,7 +599,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       __syncthreads();
       for (int it = 0; it < chunks; ++it) {
         Chunk c;
-        const uint32_t present = load_chunk(rr, it, c);
+        const uint32_t present = load_chunk<NT>(rr, it, c);
         uint32_t cnt = __popc(present);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
@@ -637,9 +613,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     __syncthreads();
     unsigned long long thr = 0ull;
     if (kk > 0) {
-      thr = radix_select_row(sh, rr, static_cast<uint32_t>(kk));
+      thr = radix_select_row<NT>(sh, rr, static_cast<uint32_t>(kk));
       // exactly kk entries pass: they become the candidate list
-      list_row(rr, [&](float v, int32_t lb) { return pack_key(v, lb) >= thr; }, sh.cand_val, sh.cand_lab, &sh.ccnt,
+      list_row<NT>(rr, [&](float v, int32_t lb) { return pack_key(v, lb) >= thr; }, sh.cand_val, sh.cand_lab, &sh.ccnt,
                kCandCap);
     }
     __syncthreads();
@@ -648,12 +624,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     // ---- 4. select inside the candidate list ------------------------------
     const int nc = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(kCandCap)));
     unsigned long long thr = 0ull;
-    if (nc > kk) thr = radix_select_cand(sh, nc, static_cast<uint32_t>(kk));
+    if (nc > kk) thr = radix_select_cand<NT>(sh, nc, static_cast<uint32_t>(kk));
     if (tid == 0) sh.cnt = 0;
     __syncthreads();
-    const int rounds = (nc + kTopkThreads - 1) / kTopkThreads;
+    const int rounds = (nc + NT - 1) / NT;
     for (int rd = 0; rd < rounds; ++rd) {
-      const int i = rd * kTopkThreads + tid;
+      const int i = rd * NT + tid;
       unsigned long long key = 0ull;
       float val = 0.f;
       if (i < nc) {
@@ -667,7 +643,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       base = __shfl_sync(0xffffffffu, base, 0);
       if (take) {
         const uint32_t s = base + __popc(bal & ((1u << lane) - 1u));
-        if (s < static_cast<uint32_t>(kMaxTopK)) {
+        if (s < static_cast<uint32_t>(KMAX)) {
           sh.sel_key[s] = key;
           sh.sel_val[s] = val;
         }
@@ -681,7 +657,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   float* vo = p.val_out ? p.val_out + static_cast<int64_t>(r) * p.ld_out : nullptr;
   if (kk > 0) {
     unsigned long long kmin = ~0ull, kmax = 0ull;
-    for (int i = tid; i < kk; i += kTopkThreads) {
+    for (int i = tid; i < kk; i += NT) {
       const unsigned long long key = sh.sel_key[i];
       kmin = key < kmin ? key : kmin;
       kmax = key > kmax ? key : kmax;
@@ -697,14 +673,14 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       sh.wmin[warp] = kmin;
       sh.wmax[warp] = kmax;
     }
-    for (int i = tid; i < kHistBins; i += kTopkThreads) {
+    for (int i = tid; i < kHistBins; i += NT) {
       sh.hist[i] = 0;
       sh.fill[i] = 0;
     }
     __syncthreads();
     if (warp == 0) {
-      kmin = sh.wmin[lane];
-      kmax = sh.wmax[lane];
+      kmin = lane < NT / 32 ? sh.wmin[lane] : ~0ull;
+      kmax = lane < NT / 32 ? sh.wmax[lane] : 0ull;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
@@ -722,13 +698,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     kmax = sh.wmax[0];
     const unsigned long long span = kmax - kmin;
     const int shift = span ? max(0, 64 - __clzll(static_cast<long long>(span)) - kHistBits) : 0;
-    for (int i = tid; i < kk; i += kTopkThreads)
+    for (int i = tid; i < kk; i += NT)
       atomicAdd(&sh.hist[static_cast<uint32_t>((sh.sel_key[i] - kmin) >> shift)], 1u);
     __syncthreads();
     // bucket offsets from the top (largest keys first); fill holds the offsets
-    scan_bins_2048(sh, sh.hist, sh.fill, 0u);
+    scan_bins_2048<NT>(sh, sh.hist, sh.fill, 0u);
     // scatter into buckets
-    for (int i = tid; i < kk; i += kTopkThreads) {
+    for (int i = tid; i < kk; i += NT) {
       const unsigned long long key = sh.sel_key[i];
       const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
       const uint32_t pos = atomicAdd(&sh.fill[bin], 1u);
@@ -737,7 +713,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     }
     __syncthreads();
     // rank inside the bucket: after the scatter fill[bin] is the bucket's end
-    for (int i = tid; i < kk; i += kTopkThreads) {
+    for (int i = tid; i < kk; i += NT) {
       const unsigned long long key = sh.tmp_key[i];
       const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
       const uint32_t end = sh.fill[bin];
@@ -748,23 +724,33 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       if (vo) vo[rank] = sh.tmp_val[i];
     }
   }
-  for (int j = kk + tid; j < p.k; j += kTopkThreads) {
+  for (int j = kk + tid; j < p.k; j += NT) {
     io[j] = -1;
     if (vo) vo[j] = neg_inf();
   }
 }
 
-cudaError_t launch_topk(const TopkParams& p, cudaStream_t st) {
+template <int NT, int KMAX>
+static cudaError_t launch_topk_t(const TopkParams& p, cudaStream_t st) {
+  using SH = TopkShared<NT, KMAX>;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(TopkShared)));
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel<NT, KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(SH)));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  if (p.R == 0) return cudaSuccess;
-  topk_kernel<<<p.R, kTopkThreads, sizeof(TopkShared), st>>>(p);
+  topk_kernel<NT, KMAX><<<p.R, NT, sizeof(SH), st>>>(p);
   return cudaGetLastError();
+}
+
+// More rows than SMs and k <= 1024: 512-thread CTAs, two per SM, so one
+// row's latency-bound phases overlap another's streaming pass.  Otherwise one
+// 1024-thread CTA per row.
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t st, int num_sms) {
+  if (p.R == 0) return cudaSuccess;
+  if (p.k <= 1024 && p.R > num_sms) return launch_topk_t<512, 1024>(p, st);
+  return launch_topk_t<1024, kMaxTopK>(p, st);
 }
 
 }  // namespace lsi
