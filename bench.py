@@ -334,7 +334,9 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
 def bench_variants(L, args, peaks, peak_kind, only=None):
     """Prefill chunk, two-stage and bucket searches: one timed loop each."""
     res = {}
-    for name, fn in (("prefill_chunk", bench_prefill), ("bucket", bench_bucket), ("two_stage", bench_two_stage)):
+    for name, fn in (("prefill_chunk", bench_prefill),
+                     ("prefill_chunk_running", lambda *a: bench_prefill(*a, full_scores=False)),
+                     ("bucket", bench_bucket), ("two_stage", bench_two_stage)):
         if only in (None, name):
             res[name] = fn(L, args, peaks, peak_kind)
     return res
@@ -353,7 +355,7 @@ def _profiled_loop(L, fn, steps, warm, st):
     return tot / steps, kern
 
 
-def bench_prefill(L, args, peaks, peak_kind):
+def bench_prefill(L, args, peaks, peak_kind, full_scores=True):
     """Prefill chunk: history streamed from pinned host memory in 8192-key
     tiles through two device buffers, causal top-512 of 4096 queries."""
     import torch
@@ -369,7 +371,8 @@ def bench_prefill(L, args, peaks, peak_kind):
     hist = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
     buf0 = torch.empty((wl.tile_keys, dd), dtype=torch.bfloat16, device="cuda")
     buf1 = torch.empty_like(buf0)
-    ws = torch.empty(L.lib().ls_prefill_select_workspace_size(T, N), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(L.lib().ls_prefill_select_workspace_size(T, N, wl.tile_keys, wl.k, int(full_scores)),
+                     dtype=torch.uint8, device="cuda")
     out = (torch.empty((T, wl.k), dtype=torch.int32, device="cuda"),
            torch.empty((T, wl.k), dtype=torch.float32, device="cuda"))
     cs = torch.cuda.Stream()
@@ -378,7 +381,7 @@ def bench_prefill(L, args, peaks, peak_kind):
 
     def pf(i, timed):
         L.ls_prefill_select_stream(q, w, qp, hist, buf0, buf1, k=wl.k, stride=wl.stride, tile_keys=wl.tile_keys,
-                                   ws=ws, out=out, copy_stream=cs)
+                                   full_scores=full_scores, ws=ws, out=out, copy_stream=cs)
         return None
 
     ms, kern = _profiled_loop(L, pf, steps, warm, st)
@@ -391,8 +394,12 @@ def bench_prefill(L, args, peaks, peak_kind):
         "roofline": roofline("tensor", flops_alg / (score_ms * 1e-3) / 1e12, peak_t, "TFLOP/s",
                              traffic=ncu_traffic("score_tc_kernel<8>", wl.name), peak_kind=peak_kind),
         "algorithmic_flops": flops_alg, "eligible_pairs": pairs,
-        "note": "step = 4 streamed 8192-key tiles (H2D on a copy stream) + causal top-512 of 4096 queries; "
-                "roofline over the 4 scoring launches of the step (score_tc_kernel<8>)",
+        "workspace_bytes": ws.numel(),
+        "note": ("step = 4 streamed 8192-key tiles (H2D on a copy stream) + causal top-512 of 4096 queries; "
+                 + ("full 4096 x 32768 score matrix, one top-k"
+                    if full_scores else "running top-512 across tiles (first tile in full, later tiles filtered "
+                                        "against each query's running 512th entry, merge per tile)")
+                 + "; roofline over the 4 scoring launches of the step (score_tc_kernel<8>)"),
     }
     del ws
     return res
@@ -543,7 +550,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_batch")
     ap.add_argument("--no-variants", action="store_true")
-    ap.add_argument("--only", default=None, choices=["prefill_chunk", "bucket", "two_stage"],
+    ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "bucket", "two_stage"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

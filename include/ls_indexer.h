@@ -181,13 +181,27 @@ ls_status ls_decode_select_noalloc(const uint16_t* q, const float* w, const uint
  * compute_stream with events; the outputs are complete when compute_stream
  * reaches the end of the call.  The call never blocks the host.  The first
  * copy waits for work already queued on compute_stream (buffers may be in use).
- * Workspace: ls_prefill_select_workspace_size(T, N) bytes.
+ *
+ * full_scores = 0: selection runs across the tiles (running top-k).  The
+ * first tile is scored in full and its exact top-k gives each query a running
+ * list; every later tile emits only the keys whose score beats the query's
+ * running k-th entry (strictly: a later key that ties it ranks lower) into up
+ * to 3k candidate slots, and a merge keeps the top k of running list +
+ * candidates.  A query that fills its slots gets that tile's exact top-k from
+ * the tile scored again in full (a launch that does nothing when no query
+ * overflowed).  No T x N score matrix is held: the workspace is one
+ * T x tile_keys tile plus the lists, so N is bounded by the history's host
+ * memory, not by the device.
+ * full_scores = 1: every tile's scores go into a T x N matrix in the
+ * workspace and one top-k runs at the end (fewer launches; needs T*N*4 B).
+ * Both forms return the same selection.
+ * Workspace: ls_prefill_select_workspace_size(T, N, tile_keys, k, full_scores) bytes.
  */
-size_t ls_prefill_select_workspace_size(int T, int N);
+size_t ls_prefill_select_workspace_size(int T, int N, int tile_keys, int k, int full_scores);
 ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int64_t* q_pos, int T, int H, int d,
                                    const uint16_t* hist_k, int N, int stride, int tile_keys, uint16_t* buf0,
-                                   uint16_t* buf1, int k, int32_t* idx_out, float* val_out, void* ws,
-                                   size_t ws_bytes, void* compute_stream, void* copy_stream);
+                                   uint16_t* buf1, int k, int full_scores, int32_t* idx_out, float* val_out,
+                                   void* ws, size_t ws_bytes, void* compute_stream, void* copy_stream);
 
 /*
  * ls_decode_two_stage_select -- LeanSparse two-stage decode search

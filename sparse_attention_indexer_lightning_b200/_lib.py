@@ -61,8 +61,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_topk_select": (I, [P, I64, P, P, I, I, I, P, P, P]),
         "ls_decode_select_workspace_size": (SZ, [I, I]),
         "ls_decode_select": (I, [P, P, P, P, I, I, I, I, I, P, P, P, SZ, P]),
-        "ls_prefill_select_workspace_size": (SZ, [I, I]),
-        "ls_prefill_select_stream": (I, [P, P, P, I, I, I, P, I, I, I, P, P, I, P, P, P, SZ, P, P]),
+        "ls_prefill_select_workspace_size": (SZ, [I, I, I, I, I]),
+        "ls_prefill_select_stream": (I, [P, P, P, I, I, I, P, I, I, I, P, P, I, I, P, P, P, SZ, P, P]),
         "ls_two_stage_workspace_size": (SZ, [I, I, I]),
         "ls_decode_two_stage_select": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P]),
         "ls_bucket_workspace_size": (SZ, [I, I, I, I]),
@@ -215,11 +215,14 @@ def ls_decode_select_noalloc(q, w, keys, k: int = 512, n_valid=None, out=None, s
 
 
 def ls_prefill_select_stream(q, w, q_pos, hist_k, buf0, buf1, k: int = 512, stride: int = 4,
-                             tile_keys: Optional[int] = None, ws=None, out=None, copy_stream=None, stream=None):
+                             tile_keys: Optional[int] = None, full_scores: bool = False, ws=None, out=None,
+                             copy_stream=None, stream=None):
     """Causal prefill selection with the history streamed from (pinned) host memory.
 
     q [T,H,d] bf16, w [T,H] f32, q_pos [T] int64 (device); hist_k [N,d] bf16 in
     pinned host memory (or on the device); buf0/buf1 [tile_keys, d] bf16 device.
+    full_scores=False keeps a running top-k across the tiles (workspace: one
+    tile of scores); True scores into a full T x N matrix and selects once.
     """
     _dev(q, torch.bfloat16, "q", 3)
     T, H, d = q.shape
@@ -235,7 +238,7 @@ def ls_prefill_select_stream(q, w, q_pos, hist_k, buf0, buf1, k: int = 512, stri
     tk = buf0.shape[0] if tile_keys is None else tile_keys
     if buf0.shape[0] < tk or buf1.shape[0] < tk:
         raise ValueError("buffers are shorter than tile_keys")
-    need = lib().ls_prefill_select_workspace_size(T, N)
+    need = lib().ls_prefill_select_workspace_size(T, N, tk, k, int(full_scores))
     if ws is None:
         ws = _workspace(need, q.device)
     if out is None:
@@ -245,8 +248,8 @@ def ls_prefill_select_stream(q, w, q_pos, hist_k, buf0, buf1, k: int = 512, stri
     cs = _stream(stream)
     xs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
     _check(lib().ls_prefill_select_stream(_ptr(q), _ptr(w), _ptr(q_pos), T, H, d, _ptr(hist_k), N, stride, tk,
-                                          _ptr(buf0), _ptr(buf1), k, _ptr(idx), _ptr(val), _ptr(ws), ws.numel(),
-                                          cs, xs))
+                                          _ptr(buf0), _ptr(buf1), k, int(full_scores), _ptr(idx), _ptr(val),
+                                          _ptr(ws), ws.numel(), cs, xs))
     return idx, val
 
 

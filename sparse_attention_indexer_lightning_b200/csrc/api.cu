@@ -155,11 +155,10 @@ ls_status check_shape(int H, int d) {
 
 cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 
-// Scores of bf16 keys on the tensor cores (the TMA path).
-ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid,
-                     const int64_t* q_pos, int stride, int B, int T, int N, int key_base, int n_total, float* out,
-                     int64_t ld_out, cudaStream_t st, uint32_t* hist = nullptr,
-                     const int32_t* lim_rows = nullptr) {
+// Scores of bf16 keys on the tensor cores (the TMA path), p filled by the
+// caller apart from the shape.
+ls_status score_tc_launch(const uint16_t* q, const uint16_t* keys, int B, int T, int N, ScoreParams p, cudaStream_t st,
+                          const char* prof_name = nullptr) {
   if (B == 0 || T == 0 || N == 0) return LS_OK;
   const int qg = (T == 1) ? 1 : 8;
   CUtensorMap kmap, qmap;
@@ -167,6 +166,18 @@ ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, co
   if (s != LS_OK) return s;
   s = make_bf16_map(&qmap, q, static_cast<uint64_t>(B) * T * kHeads, qg * kHeads);
   if (s != LS_OK) return s;
+  p.B = B;
+  p.T = T;
+  p.N = N;
+  ProfScope prof(prof_name ? prof_name : qg == 1 ? "score_tc_kernel<1>" : "score_tc_kernel<8>", st);
+  LS_CUDA(launch_score_tc(qg, &kmap, &qmap, p, num_sms_current(), st));
+  return LS_OK;
+}
+
+ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid,
+                     const int64_t* q_pos, int stride, int B, int T, int N, int key_base, int n_total, float* out,
+                     int64_t ld_out, cudaStream_t st, uint32_t* hist = nullptr,
+                     const int32_t* lim_rows = nullptr) {
   ScoreParams p;
   p.w = w;
   p.n_valid = n_valid;
@@ -177,13 +188,12 @@ ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, co
   p.B = B;
   p.T = T;
   p.N = N;
+  p.out_col0 = key_base;
   p.key_base = key_base;
   p.n_total = n_total;
   p.hist = hist;
   p.lim_rows = lim_rows;
-  ProfScope prof(qg == 1 ? "score_tc_kernel<1>" : "score_tc_kernel<8>", st);
-  LS_CUDA(launch_score_tc(qg, &kmap, &qmap, p, num_sms_current(), st));
-  return LS_OK;
+  return score_tc_launch(q, keys, B, T, N, p, st);
 }
 
 ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_total, const float* w,
@@ -226,6 +236,12 @@ ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_
   return LS_OK;
 }
 
+ls_status topk_launch(const TopkParams& p, cudaStream_t st, const char* prof_name = "topk_kernel") {
+  ProfScope prof(prof_name, st);
+  LS_CUDA(launch_topk(p, st, num_sms_current()));
+  return LS_OK;
+}
+
 ls_status topk(const float* scores, int64_t ld, const int32_t* n_valid, const int32_t* labels, int64_t ld_labels,
                int R, int N, int k, int32_t* idx, float* val, int64_t ld_out, cudaStream_t st,
                const uint32_t* hist = nullptr) {
@@ -242,9 +258,7 @@ ls_status topk(const float* scores, int64_t ld, const int32_t* n_valid, const in
   p.idx_out = idx;
   p.val_out = val;
   p.ld_out = ld_out;
-  ProfScope prof("topk_kernel", st);
-  LS_CUDA(launch_topk(p, st, num_sms_current()));
-  return LS_OK;
+  return topk_launch(p, st);
 }
 
 struct Carver {
@@ -344,15 +358,28 @@ ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* ke
   return topk(sc, N, n_valid, nullptr, 0, B, N, k, idx_out, val_out, k, S(stream));
 }
 
-size_t ls_prefill_select_workspace_size(int T, int N) {
-  if (T <= 0 || N <= 0) return 0;
-  return align_up(static_cast<size_t>(T) * N * sizeof(float)) + align_up(static_cast<size_t>(T) * sizeof(int32_t));
+// Candidate slots per row and tile in the running top-k of the prefill.
+int prefill_cand_cap(int k) { return 3 * k; }
+
+size_t ls_prefill_select_workspace_size(int T, int N, int tile_keys, int k, int full_scores) {
+  if (T <= 0 || N <= 0 || tile_keys <= 0 || k <= 0) return 0;
+  if (full_scores)  // the whole T x N score matrix, then one top-k
+    return align_up(static_cast<size_t>(T) * N * sizeof(float)) + align_up(static_cast<size_t>(T) * sizeof(int32_t));
+  const int tk = tile_keys < N ? tile_keys : N;
+  const int ntiles = (N + tile_keys - 1) / tile_keys;
+  const int64_t ldc = ntiles > 1 ? k + prefill_cand_cap(k) : 0;
+  return align_up(static_cast<size_t>(T) * tk * sizeof(float)) +    // one tile of scores
+         align_up(static_cast<size_t>(T) * ldc * sizeof(float)) +   // running top-k + candidates
+         align_up(static_cast<size_t>(T) * ldc * sizeof(int32_t)) +
+         align_up(static_cast<size_t>(T) * sizeof(int32_t)) +       // eligible counts
+         align_up(static_cast<size_t>(T) * sizeof(int32_t)) +       // merge counts
+         align_up(static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int));  // counters, overflow flags
 }
 
 ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int64_t* q_pos, int T, int H, int d,
                                    const uint16_t* hist_k, int N, int stride, int tile_keys, uint16_t* buf0,
-                                   uint16_t* buf1, int k, int32_t* idx_out, float* val_out, void* ws,
-                                   size_t ws_bytes, void* compute_stream, void* copy_stream) {
+                                   uint16_t* buf1, int k, int full_scores, int32_t* idx_out, float* val_out,
+                                   void* ws, size_t ws_bytes, void* compute_stream, void* copy_stream) {
   ls_status s = check_shape(H, d);
   if (s != LS_OK) return s;
   LS_CHECK_ARG(T >= 0 && N >= 0, "negative size");
@@ -362,74 +389,186 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
   if (T == 0) return LS_OK;
   LS_CHECK_ARG(q && w && q_pos && idx_out, "null tensor pointer");
   LS_CHECK_ARG(aligned16(q) && aligned16(w), "q and w must be 16-byte aligned");
-  const size_t need = ls_prefill_select_workspace_size(T, N);
-  if (ws_bytes < need || (need && !ws))
-    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
-  Carver cv(ws);
-  float* sc = cv.take<float>(static_cast<size_t>(T) * N);
-  int32_t* counts = cv.take<int32_t>(T);
   cudaStream_t cs = S(compute_stream);
   cudaStream_t xs = copy_stream ? S(copy_stream) : cs;
-  if (N > 0) {
-    LS_CHECK_ARG(hist_k && buf0 && buf1, "null history or buffer pointer");
-    LS_CHECK_ARG(aligned16(buf0) && aligned16(buf1) && aligned16(hist_k), "history and buffers must be 16-byte aligned");
-    cudaPointerAttributes attr;
-    LS_CUDA(cudaPointerGetAttributes(&attr, hist_k));
-    LS_CHECK_ARG(attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeDevice ||
-                     attr.type == cudaMemoryTypeManaged,
-                 "hist_k must be pinned host memory or device memory (pageable memory cannot be streamed)");
-    uint16_t* bufs[2] = {buf0, buf1};
-    cudaEvent_t start_ev, copied[2], freed[2];
-    LS_CUDA(cudaEventCreateWithFlags(&start_ev, cudaEventDisableTiming));
-    for (int i = 0; i < 2; ++i) {
-      LS_CUDA(cudaEventCreateWithFlags(&copied[i], cudaEventDisableTiming));
-      LS_CUDA(cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming));
-    }
-    ls_status st = LS_OK;
-    {
-      ProfScope prof("causal_counts_kernel", cs);
-      LS_CUDA(launch_causal_counts(q_pos, T, stride, N, counts, cs));
-    }
-    // Earlier work on the compute stream may still read the buffers.
-    cudaError_t e = cudaEventRecord(start_ev, cs);
-    if (e == cudaSuccess && xs != cs) e = cudaStreamWaitEvent(xs, start_ev, 0);
-    const int ntiles = (N + tile_keys - 1) / tile_keys;
-    for (int j = 0; j < ntiles && e == cudaSuccess && st == LS_OK; ++j) {
-      const int slot = j & 1;
-      const int k0 = j * tile_keys;
-      const int len = (N - k0 < tile_keys) ? (N - k0) : tile_keys;
-      if (j >= 2 && xs != cs) e = cudaStreamWaitEvent(xs, freed[slot], 0);
-      if (e != cudaSuccess) break;
-      e = cudaMemcpyAsync(bufs[slot], hist_k + static_cast<size_t>(k0) * kDim,
-                          static_cast<size_t>(len) * kDim * sizeof(uint16_t), cudaMemcpyDefault, xs);
-      if (e != cudaSuccess) break;
-      if (xs != cs) {
-        e = cudaEventRecord(copied[slot], xs);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, copied[slot], 0);
-        if (e != cudaSuccess) break;
-      }
-      st = score_bf16(q, w, bufs[slot], nullptr, q_pos, stride, 1, T, len, k0, N, sc, N, cs, nullptr, counts);
-      if (st != LS_OK) break;
-      if (xs != cs) e = cudaEventRecord(freed[slot], cs);
-    }
-    // The copy stream must not run ahead of this call's last kernels.
-    if (e == cudaSuccess && st == LS_OK && xs != cs) {
-      e = cudaEventRecord(start_ev, cs);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(xs, start_ev, 0);
-    }
-    cudaEventDestroy(start_ev);
-    for (int i = 0; i < 2; ++i) {
-      cudaEventDestroy(copied[i]);
-      cudaEventDestroy(freed[i]);
-    }
-    if (st != LS_OK) return st;
-    if (e != cudaSuccess) return fail(LS_ERR_CUDA, "history streaming: %s", cudaGetErrorString(e));
+  if (N == 0) {  // no history: every row is padding
+    TopkParams p;
+    p.R = T;
+    p.k = k;
+    p.idx_out = idx_out;
+    p.val_out = val_out;
+    p.ld_out = k;
+    return topk_launch(p, cs);
   }
-  if (N == 0) {
+  const size_t need = ls_prefill_select_workspace_size(T, N, tile_keys, k, full_scores);
+  if (ws_bytes < need || (need && !ws))
+    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  LS_CHECK_ARG(hist_k && buf0 && buf1, "null history or buffer pointer");
+  LS_CHECK_ARG(aligned16(buf0) && aligned16(buf1) && aligned16(hist_k), "history and buffers must be 16-byte aligned");
+  cudaPointerAttributes attr;
+  LS_CUDA(cudaPointerGetAttributes(&attr, hist_k));
+  LS_CHECK_ARG(attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeDevice ||
+                   attr.type == cudaMemoryTypeManaged,
+               "hist_k must be pinned host memory or device memory (pageable memory cannot be streamed)");
+  const int tk = full_scores ? N : (tile_keys < N ? tile_keys : N);
+  const int ntiles = (N + tile_keys - 1) / tile_keys;
+  const int cap = prefill_cand_cap(k);
+  const int64_t ldc = (!full_scores && ntiles > 1) ? k + cap : 0;
+  Carver cv(ws);
+  float* tile_sc = cv.take<float>(static_cast<size_t>(T) * tk);  // full_scores: the T x N matrix
+  float* run_val = cv.take<float>(static_cast<size_t>(T) * ldc);
+  int32_t* run_lab = cv.take<int32_t>(static_cast<size_t>(T) * ldc);
+  int32_t* counts = cv.take<int32_t>(T);
+  int32_t* nv = cv.take<int32_t>(T);
+  uint8_t* ctr = cv.take<uint8_t>(static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int));
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ctr);
+  int32_t* row_over = reinterpret_cast<int32_t*>(ctr) + T;
+  int* any_over = reinterpret_cast<int*>(ctr) + 2 * static_cast<size_t>(T);
+  const size_t ctr_bytes = static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int);
+
+  uint16_t* bufs[2] = {buf0, buf1};
+  cudaEvent_t start_ev, copied[2], freed[2];
+  LS_CUDA(cudaEventCreateWithFlags(&start_ev, cudaEventDisableTiming));
+  for (int i = 0; i < 2; ++i) {
+    LS_CUDA(cudaEventCreateWithFlags(&copied[i], cudaEventDisableTiming));
+    LS_CUDA(cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming));
+  }
+  ls_status st = LS_OK;
+  {
     ProfScope prof("causal_counts_kernel", cs);
     LS_CUDA(launch_causal_counts(q_pos, T, stride, N, counts, cs));
   }
-  return topk(sc, N, counts, nullptr, 0, T, N, k, idx_out, val_out, k, cs);
+  // Earlier work on the compute stream may still read the buffers.
+  cudaError_t e = cudaEventRecord(start_ev, cs);
+  if (e == cudaSuccess && xs != cs) e = cudaStreamWaitEvent(xs, start_ev, 0);
+  for (int j = 0; j < ntiles && e == cudaSuccess && st == LS_OK; ++j) {
+    const int slot = j & 1;
+    const int k0 = j * tile_keys;
+    const int len = (N - k0 < tile_keys) ? (N - k0) : tile_keys;
+    const bool last = j + 1 == ntiles;
+    if (j >= 2 && xs != cs) e = cudaStreamWaitEvent(xs, freed[slot], 0);
+    if (e != cudaSuccess) break;
+    e = cudaMemcpyAsync(bufs[slot], hist_k + static_cast<size_t>(k0) * kDim,
+                        static_cast<size_t>(len) * kDim * sizeof(uint16_t), cudaMemcpyDefault, xs);
+    if (e != cudaSuccess) break;
+    if (xs != cs) {
+      e = cudaEventRecord(copied[slot], xs);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, copied[slot], 0);
+      if (e != cudaSuccess) break;
+    }
+    ScoreParams sp;
+    sp.w = w;
+    sp.q_pos = q_pos;
+    sp.stride = stride;
+    sp.key_base = k0;
+    sp.n_total = N;
+    sp.lim_rows = counts;
+    TopkParams tp;                     // top-k of one full tile of scores
+    tp.scores = tile_sc;
+    tp.ld = tk;
+    tp.n_valid = counts;
+    tp.nv_offset = k0;
+    tp.label_base = k0;
+    tp.R = T;
+    tp.N = len;
+    tp.k = k;
+    if (full_scores) {
+      // every tile into its columns of the T x N matrix; one top-k at the end
+      sp.out = tile_sc;
+      sp.ld_out = N;
+      sp.out_col0 = k0;
+      st = score_tc_launch(q, bufs[slot], 1, T, len, sp, cs);
+      if (st != LS_OK) break;
+      if (last) {
+        TopkParams fp;
+        fp.scores = tile_sc;
+        fp.ld = N;
+        fp.n_valid = counts;
+        fp.R = T;
+        fp.N = N;
+        fp.k = k;
+        fp.idx_out = idx_out;
+        fp.val_out = val_out;
+        fp.ld_out = k;
+        st = topk_launch(fp, cs);
+        if (st != LS_OK) break;
+      }
+    } else if (j == 0) {
+      // the first tile is scored in full and gives every row its running top-k
+      sp.out = tile_sc;
+      sp.ld_out = tk;
+      st = score_tc_launch(q, bufs[slot], 1, T, len, sp, cs);
+      if (st != LS_OK) break;
+      tp.idx_out = last ? idx_out : run_lab;
+      tp.val_out = last ? val_out : run_val;
+      tp.ld_out = last ? k : ldc;
+      st = topk_launch(tp, cs);
+      if (st != LS_OK) break;
+    } else {
+      // later tiles append only keys that beat the row's running k-th entry
+      e = cudaMemsetAsync(ctr, 0, ctr_bytes, cs);
+      if (e != cudaSuccess) break;
+      ScoreParams fp = sp;
+      fp.cand_val = run_val;
+      fp.cand_lab = run_lab;
+      fp.ld_cand = ldc;
+      fp.run_k = k;
+      fp.cand_cap = cap;
+      fp.cand_cnt = cnt;
+      fp.row_over = row_over;
+      fp.any_over = any_over;
+      st = score_tc_launch(q, bufs[slot], 1, T, len, fp, cs);
+      if (st != LS_OK) break;
+      // rows that ran out of candidate slots: this tile again in full (the
+      // launches return at once when no row overflowed), its top-k into the
+      // row's candidate columns
+      sp.out = tile_sc;
+      sp.ld_out = tk;
+      sp.run_if = any_over;
+      st = score_tc_launch(q, bufs[slot], 1, T, len, sp, cs, "score_tc_kernel<8>:overflow");
+      if (st != LS_OK) break;
+      tp.run_if = any_over;
+      tp.row_flag = row_over;
+      tp.idx_out = run_lab + k;
+      tp.val_out = run_val + k;
+      tp.ld_out = ldc;
+      st = topk_launch(tp, cs, "topk_kernel:overflow");
+      if (st != LS_OK) break;
+      {
+        ProfScope prof("merge_counts_kernel", cs);
+        LS_CUDA(launch_merge_counts(cnt, row_over, T, k, cap, nv, cs));
+      }
+      // merge: running top-k + this tile's candidates -> the new running top-k
+      TopkParams mp;
+      mp.scores = run_val;
+      mp.ld = ldc;
+      mp.n_valid = nv;
+      mp.labels = run_lab;
+      mp.ld_labels = ldc;
+      mp.R = T;
+      mp.N = static_cast<int>(ldc);
+      mp.k = k;
+      mp.idx_out = last ? idx_out : run_lab;
+      mp.val_out = last ? val_out : run_val;
+      mp.ld_out = last ? k : ldc;
+      st = topk_launch(mp, cs);
+      if (st != LS_OK) break;
+    }
+    if (xs != cs) e = cudaEventRecord(freed[slot], cs);
+  }
+  // The copy stream must not run ahead of this call's last kernels.
+  if (e == cudaSuccess && st == LS_OK && xs != cs) {
+    e = cudaEventRecord(start_ev, cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(xs, start_ev, 0);
+  }
+  cudaEventDestroy(start_ev);
+  for (int i = 0; i < 2; ++i) {
+    cudaEventDestroy(copied[i]);
+    cudaEventDestroy(freed[i]);
+  }
+  if (st != LS_OK) return st;
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "history streaming: %s", cudaGetErrorString(e));
+  return LS_OK;
 }
 
 size_t ls_two_stage_workspace_size(int B, int N, int shortlist) {

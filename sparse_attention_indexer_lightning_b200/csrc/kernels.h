@@ -21,18 +21,38 @@ constexpr int kMaxTopK = 4096;
 // or -inf where the key is masked: n >= n_valid[b] (when given) or, with
 // q_pos, key_base + n >= (q_pos[b,t] + 1) / stride (block-complete causal rule),
 // capped at n_total.
+//
+// Filter form (out == nullptr): nothing is stored per key; instead every
+// eligible key whose score beats the row's running k-th entry (read from
+// cand_val / cand_lab columns run_k-1 of the row; a row whose list is not yet
+// full takes every eligible key) is appended as (score, key_base + n) to the
+// row's candidate columns run_k .. run_k+cand_cap-1 at the slot its counter
+// cand_cnt[row] hands out; a row that runs out of slots sets row_over[row]
+// and *any_over.  "Beats" compares order codes strictly: a later key that
+// ties the k-th entry ranks below it.
 struct ScoreParams {
-  const float* w;          // [B][T][H]
-  const int32_t* n_valid;  // [B] or nullptr
-  const int64_t* q_pos;    // [B][T] or nullptr
-  float* out;
-  int64_t ld_out;
-  int stride;
-  int B, T, N;
-  int key_base;
-  int n_total;             // causal cap: number of keys of the whole history
-  uint32_t* hist;          // [B*T][2048] selection histogram (counts added) or nullptr; qg == 1 only
-  const int32_t* lim_rows; // [B*T] eligible keys of the whole history per query (replaces q_pos) or nullptr
+  const float* w = nullptr;           // [B][T][H]
+  const int32_t* n_valid = nullptr;   // [B] or nullptr
+  const int64_t* q_pos = nullptr;     // [B][T] or nullptr
+  float* out = nullptr;
+  int64_t ld_out = 0;
+  int out_col0 = 0;                   // column of key n in out: out_col0 + n
+  int stride = 1;
+  int B = 0, T = 0, N = 0;
+  int key_base = 0;                   // position of key 0 of this launch in the history
+  int n_total = 0;                    // causal cap: number of keys of the whole history
+  uint32_t* hist = nullptr;           // [B*T][2048] selection histogram (counts added) or nullptr; qg == 1 only
+  const int32_t* lim_rows = nullptr;  // [B*T] eligible keys of the whole history per query (replaces q_pos)
+  // filter form
+  float* cand_val = nullptr;          // [B*T][ld_cand]
+  int32_t* cand_lab = nullptr;        // [B*T][ld_cand]
+  int64_t ld_cand = 0;
+  int run_k = 0;
+  int cand_cap = 0;
+  uint32_t* cand_cnt = nullptr;       // [B*T]
+  int32_t* row_over = nullptr;        // [B*T]
+  int* any_over = nullptr;
+  const int* run_if = nullptr;        // the launch does nothing unless *run_if != 0 (nullptr: always)
 };
 
 // qg = queries sharing one MMA B tile: 1 (one query per sequence) or 8.
@@ -71,17 +91,21 @@ cudaError_t launch_score_q8(const CUtensorMap* qmap, const CUtensorMap* kmap, co
 // ---------------------------------------------------------------- top-k
 // Row-wise top-k by (value desc, label asc); labels default to the column.
 struct TopkParams {
-  const float* scores;     // row r starts at scores + r*ld
-  int64_t ld;
-  const int32_t* n_valid;  // [R] or nullptr: columns >= n_valid[r] are absent
-  const int32_t* labels;   // [R][ld_labels] or nullptr; label < 0 = absent
-  int64_t ld_labels;
-  const uint32_t* hist;    // [R][2048] counts of the top 11 order-code bits of the
-                           // present entries (from the scoring epilogue) or nullptr
-  int R, N, k;
-  int32_t* idx_out;        // [R][k] labels, -1 padding
-  float* val_out;          // [R][k] values (bit copies), -inf padding; may be nullptr
-  int64_t ld_out;
+  const float* scores = nullptr;     // row r starts at scores + r*ld
+  int64_t ld = 0;
+  const int32_t* n_valid = nullptr;  // [R] or nullptr: columns >= n_valid[r] - nv_offset are absent
+  int nv_offset = 0;
+  const int32_t* labels = nullptr;   // [R][ld_labels] or nullptr; label < 0 = absent
+  int64_t ld_labels = 0;
+  int label_base = 0;                // without labels, entry j is labelled label_base + j
+  const uint32_t* hist = nullptr;    // [R][2048] counts of the top 11 order-code bits of the
+                                     // present entries (from the scoring epilogue) or nullptr
+  const int32_t* row_flag = nullptr; // [R] or nullptr: rows whose flag is 0 are left untouched
+  const int* run_if = nullptr;       // the launch does nothing unless *run_if != 0 (nullptr: always)
+  int R = 0, N = 0, k = 0;
+  int32_t* idx_out = nullptr;        // [R][k] labels, -1 padding
+  float* val_out = nullptr;          // [R][k] values (bit copies), -inf padding; may be nullptr
+  int64_t ld_out = 0;
 };
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t st, int num_sms);
 
@@ -94,6 +118,12 @@ cudaError_t launch_causal_counts(const int64_t* q_pos, int T, int stride, int n_
 // budget positions are held; cand[t][budget] padded with -1.
 cudaError_t launch_expand(const int32_t* picked, int T, int top_p, const int32_t* off, const int32_t* mem,
                           int P, int budget, int32_t* cand, cudaStream_t st);
+
+// Entries to merge per row after a filtered tile: the running k plus the
+// row's candidates (min(cnt, cap)), or plus the k entries of the row's
+// recomputed tile when it overflowed.
+cudaError_t launch_merge_counts(const uint32_t* cnt, const int32_t* row_over, int T, int k, int cap, int32_t* nv,
+                                cudaStream_t st);
 
 int read_and_clear_fault(cudaStream_t st, int* flags);
 cudaError_t launch_wait_probe(uint64_t limit_ns, int* waited, cudaStream_t st);

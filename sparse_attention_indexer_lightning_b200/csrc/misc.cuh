@@ -33,6 +33,21 @@ cudaError_t launch_causal_counts(const int64_t* q_pos, int T, int stride, int n_
   return cudaGetLastError();
 }
 
+__global__ void merge_counts_kernel(const uint32_t* cnt, const int32_t* row_over, int T, int k, int cap,
+                                    int32_t* nv) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const uint32_t c = cnt[t];
+  nv[t] = k + (row_over[t] ? k : static_cast<int32_t>(c < static_cast<uint32_t>(cap) ? c : cap));
+}
+
+cudaError_t launch_merge_counts(const uint32_t* cnt, const int32_t* row_over, int T, int k, int cap, int32_t* nv,
+                                cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  merge_counts_kernel<<<(T + 255) / 256, 256, 0, st>>>(cnt, row_over, T, k, cap, nv);
+  return cudaGetLastError();
+}
+
 // One warp per query.
 __global__ void expand_kernel(const int32_t* picked, int T, int top_p, const int32_t* off, const int32_t* mem,
                               int P, int budget, int32_t* cand) {

@@ -93,11 +93,14 @@ __device__ __forceinline__ int eligible_keys(const ScoreParams& p, int b, int t)
   return static_cast<int>(e > p.n_total ? p.n_total : e);
 }
 
-template <int QG>
+// FILTER: the filter form of ScoreParams (p.out == nullptr), built as its own
+// instantiation so the storing form keeps its registers.
+template <int QG, bool FILTER>
 __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const ScoreParams p) {
   using C = TcCfg<QG>;
+  if (p.run_if != nullptr && *p.run_if == 0) return;  // a conditional launch with nothing to do
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -275,13 +278,43 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
     uint32_t acc_phase = 0;
     long long w_row = -1;                     // QG == 1: row whose weights sit in wreg
     float wreg[32];
-    long long lim_bg = -1;                    // group whose per-query limits sit in elig
+    long long lim_bg = -1;                    // group whose per-query limits sit in elig / thr
     int elig[C::Q_PER_EPI_WARP];
+    uint32_t thr[C::Q_PER_EPI_WARP];          // filter form: order code a key must reach
 #pragma unroll
-    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) elig[i] = 0;
+    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) elig[i] = 0, thr[i] = 0;
+    constexpr bool filter = FILTER;
+    // Filter form: a query's slot reservation (one atomic per warp) is used
+    // one unit later, so the atomic's round trip overlaps the next unit.
+    float pend_s[C::Q_PER_EPI_WARP];
+    int32_t pend_lab[C::Q_PER_EPI_WARP];
+    uint32_t pend_bal[C::Q_PER_EPI_WARP], pend_base[C::Q_PER_EPI_WARP];
+    int64_t pend_at[C::Q_PER_EPI_WARP];
+#pragma unroll
+    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) pend_bal[i] = 0;
+    auto flush_pending = [&]() {
+#pragma unroll
+      for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) {
+        if (pend_bal[i]) {                                 // warp-uniform
+          const uint32_t base = __shfl_sync(0xffffffffu, pend_base[i], 0);
+          if ((pend_bal[i] >> lane) & 1u) {
+            const uint32_t slot = base + static_cast<uint32_t>(__popc(pend_bal[i] & ((1u << lane) - 1u)));
+            if (slot < static_cast<uint32_t>(p.cand_cap)) {
+              p.cand_val[pend_at[i] + slot] = pend_s[i];
+              p.cand_lab[pend_at[i] + slot] = pend_lab[i];
+            } else {
+              p.row_over[(pend_at[i] - p.run_k) / p.ld_cand] = 1;
+              *p.any_over = 1;
+            }
+          }
+          pend_bal[i] = 0;
+        }
+      }
+    };
     UnitPos up;
     up.init(u_begin, NT, G);
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
+      if (filter) flush_pending();
       const int tile = up.tile, g = up.g, b = up.b;
       const long long bg = static_cast<long long>(b) * G + g;
       const int n = tile * C::BM + quad * 32 + lane;       // key within this launch
@@ -341,9 +374,27 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
             const int rel = elig[jq] - p.key_base;
             lim_t = rel < 0 ? 0 : (rel < lim_t ? rel : lim_t);
           }
-          if (n < p.N) {
-            p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.key_base + n] = (n < lim_t) ? s : neg_inf();
-            if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
+          if (!filter) {
+            if (n < p.N) {
+              p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.out_col0 + n] = (n < lim_t) ? s : neg_inf();
+              if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
+            }
+          } else {
+            const int64_t row = static_cast<int64_t>(b) * p.T + t;
+            if (lim_bg != bg) {
+              // the row's running k-th entry; a list with padding takes every eligible key
+              const int64_t kth = row * p.ld_cand + p.run_k - 1;
+              thr[jq] = (p.cand_lab[kth] < 0) ? 0u : order_code(p.cand_val[kth]) + 1u;
+            }
+            const bool take = (n < p.N) && (n < lim_t) && order_code(s) >= thr[jq];
+            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+            pend_bal[jq] = bal;
+            if (bal) {
+              pend_base[jq] = (lane == 0) ? atomicAdd(p.cand_cnt + row, static_cast<uint32_t>(__popc(bal))) : 0u;
+              pend_s[jq] = s;
+              pend_lab[jq] = p.key_base + n;
+              pend_at[jq] = row * p.ld_cand + p.run_k;
+            }
           }
         }
       }
@@ -356,6 +407,7 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
         role_barrier(1, C::EPI_WARPS * 32);
       }
     }
+    if (filter) flush_pending();
   }
 
   tc_fence_before();
@@ -367,13 +419,13 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
   }
 }
 
-template <int QG>
+template <int QG, bool FILTER>
 static cudaError_t launch_tc(const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p, int num_sms,
                              cudaStream_t st) {
   using C = TcCfg<QG>;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<QG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<QG, FILTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::SMEM_TOTAL));
     if (e != cudaSuccess) return e;
     attr_done = true;
@@ -383,14 +435,15 @@ static cudaError_t launch_tc(const CUtensorMap* kmap, const CUtensorMap* qmap, c
   const long long units = static_cast<long long>(p.B) * G * NT;
   if (units == 0) return cudaSuccess;
   const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-  score_tc_kernel<QG><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*kmap, *qmap, p);
+  score_tc_kernel<QG, FILTER><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*kmap, *qmap, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_score_tc(int qg, const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p,
                             int num_sms, cudaStream_t st) {
-  if (qg == 1) return launch_tc<1>(kmap, qmap, p, num_sms, st);
-  if (qg == 8) return launch_tc<8>(kmap, qmap, p, num_sms, st);
+  const bool filter = p.out == nullptr;
+  if (qg == 1) return filter ? launch_tc<1, true>(kmap, qmap, p, num_sms, st) : launch_tc<1, false>(kmap, qmap, p, num_sms, st);
+  if (qg == 8) return filter ? launch_tc<8, true>(kmap, qmap, p, num_sms, st) : launch_tc<8, false>(kmap, qmap, p, num_sms, st);
   return cudaErrorInvalidValue;
 }
 

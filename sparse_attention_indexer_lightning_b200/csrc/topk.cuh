@@ -498,13 +498,15 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
   extern __shared__ __align__(16) uint8_t topk_smem[];
   TopkShared<NT, KMAX>& sh = *reinterpret_cast<TopkShared<NT, KMAX>*>(topk_smem);
   const int r = blockIdx.x;
+  if (p.run_if != nullptr && *p.run_if == 0) return;      // conditional launch with nothing to do
+  if (p.row_flag != nullptr && p.row_flag[r] == 0) return;  // row left untouched
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   RowRef rr;
   rr.v = p.scores + static_cast<int64_t>(r) * p.ld;
   rr.lab = p.labels ? p.labels + static_cast<int64_t>(r) * p.ld_labels : nullptr;
   rr.n = p.N;
-  if (p.n_valid) rr.n = max(0, min(rr.n, p.n_valid[r]));
+  if (p.n_valid) rr.n = max(0, min(rr.n, p.n_valid[r] - p.nv_offset));
   rr.vec = ((reinterpret_cast<uintptr_t>(rr.v) & 15u) == 0) &&
            (rr.lab == nullptr || (reinterpret_cast<uintptr_t>(rr.lab) & 15u) == 0);
   const int chunks = chunk_count<NT>(rr);
@@ -720,7 +722,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
       const uint32_t beg = end - sh.hist[bin];
       uint32_t rank = beg;
       for (uint32_t j = beg; j < end; ++j) rank += (sh.tmp_key[j] > key) ? 1u : 0u;
-      io[rank] = static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull));
+      io[rank] = static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull)) + (rr.lab ? 0 : p.label_base);
       if (vo) vo[rank] = sh.tmp_val[i];
     }
   }

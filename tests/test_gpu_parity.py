@@ -65,8 +65,10 @@ def _adversarial_rows(rng, R, N):
     return s
 
 
+# the last three shapes have more rows than SMs: the two-CTAs-per-SM form
 @pytest.mark.parametrize("R,N,k", [(7, 3000, 512), (6, 517, 512), (6, 40000, 4096), (3, 131072, 4096),
-                                   (8, 1000, 1), (6, 129, 64)])
+                                   (8, 1000, 1), (6, 129, 64), (300, 3000, 512), (300, 20000, 1024),
+                                   (160, 9000, 64)])
 def test_topk_bit_exact(L, R, N, k):
     rng = np.random.default_rng(100 + N)
     s = _adversarial_rows(rng, R, N)
@@ -183,7 +185,7 @@ def test_converted_key_scores(L, fmt):
 # --------------------------------------------------------------------------- #
 # prefill: streamed history, causal eligibility
 # --------------------------------------------------------------------------- #
-def _prefill_run(L, d, wl, use_copy_stream=True):
+def _prefill_run(L, d, wl, use_copy_stream=True, full_scores=False):
     T = d["q"].shape[0]
     q, w, qp = dev_bf16(d["q"]), dev(d["w"]), dev(d["q_pos"])
     hist = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -191,7 +193,7 @@ def _prefill_run(L, d, wl, use_copy_stream=True):
     buf1 = torch.empty_like(buf0)
     cs = torch.cuda.Stream() if use_copy_stream else None
     idx, val = L.ls_prefill_select_stream(q, w, qp, hist, buf0, buf1, k=wl.k, stride=wl.stride,
-                                          tile_keys=wl.tile_keys, copy_stream=cs)
+                                          tile_keys=wl.tile_keys, full_scores=full_scores, copy_stream=cs)
     torch.cuda.synchronize()
     return q, w, qp, idx.cpu().numpy(), val.cpu().numpy()
 
@@ -213,9 +215,43 @@ def test_prefill_stream_small(L):
                             stride=wl.stride)[0]
     ri, rv = L.ls_topk_select(sc, wl.k, n_valid=dev(n_t.astype(np.int32)))
     assert np.array_equal(ri.cpu().numpy(), idx) and f32_bits_equal(rv.cpu().numpy(), val)
-    # same answer on a single stream
+    # same answer on a single stream, and from the full-matrix form
     *_, idx2, val2 = _prefill_run(L, d, wl, use_copy_stream=False)
     assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
+    *_, idx3, val3 = _prefill_run(L, d, wl, full_scores=True)
+    assert np.array_equal(idx3, idx) and f32_bits_equal(val3, val)
+
+
+def test_prefill_stream_overflow(L):
+    """Queries whose scores rise with position beat their running list with
+    every key of every later tile, so they overflow the candidate slots and take
+    the full-tile path; the other queries score 0 everywhere (ties go to the
+    lower position), so nothing after the first tile enters their lists."""
+    from types import SimpleNamespace
+    from workloads.synth import to_bf16_bits
+    T, H, dd, N, k, stride = 24, 32, 128, 1000, 32, 4
+    rng = np.random.default_rng(7)
+    u = rng.standard_normal(dd)
+    u /= np.linalg.norm(u)
+    alpha = np.linspace(0.05, 1.0, N)
+    kbits = to_bf16_bits(alpha[:, None] * u[None, :])
+    sign = np.where(np.arange(T) < T // 2, 1.0, -1.0)
+    qbits = to_bf16_bits(np.broadcast_to(sign[:, None, None] * u[None, None, :], (T, H, dd)).copy())
+    w = (np.abs(rng.standard_normal((T, H))) + 0.1).astype(np.float32)
+    q_pos = (stride * N - 1 - rng.integers(0, 300, size=T)).astype(np.int64)
+    d = {"q": qbits, "w": w, "k": kbits, "q_pos": q_pos}
+    wl = SimpleNamespace(k=k, stride=stride, tile_keys=128)
+    q, wd, qp, idx, val = _prefill_run(L, d, wl)
+    n_t = eligible_count(q_pos, stride, N)
+    keys = bf16_to_f64(kbits)
+    for t in range(T):
+        n = int(n_t[t])
+        ref = indexer_scores(bf16_to_f64(qbits[t])[None], w[t].astype(np.float64)[None], keys[:n])[0]
+        check_selection(idx[t], val[t], np.arange(n), ref, k, RTOL_BF16, f"overflow t={t}")
+    sc = L.ls_indexer_score(q.view(1, T, H, dd), wd.view(1, T, H), dev_bf16(kbits)[None], q_pos=qp.view(1, T),
+                            stride=stride)[0]
+    ri, rv = L.ls_topk_select(sc, k, n_valid=dev(n_t.astype(np.int32)))
+    assert np.array_equal(ri.cpu().numpy(), idx) and f32_bits_equal(rv.cpu().numpy(), val)
 
 
 @pytest.mark.slow
@@ -223,6 +259,9 @@ def test_prefill_chunk_full_size_sampled(L):
     wl = get_workload("prefill_chunk")
     d = data("prefill_chunk")
     _, _, _, idx, val = _prefill_run(L, d, wl)
+    # the full-matrix form selects the same
+    *_, idx2, val2 = _prefill_run(L, d, wl, full_scores=True)
+    assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
     N = d["k"].shape[0]
     n_t = eligible_count(d["q_pos"], wl.stride, N)
     keys = bf16_to_f64(d["k"])
