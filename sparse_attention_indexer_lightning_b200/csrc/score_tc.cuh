@@ -29,7 +29,7 @@
 
 namespace lsi {
 
-template <int QG>
+template <int QG, bool FILTER = false>
 struct TcCfg {
   static constexpr int BM = kTileKeys;             // keys per tile
   static constexpr int BN = QG * kHeads;           // queries x heads per MMA
@@ -37,7 +37,7 @@ struct TcCfg {
   static constexpr int A_HALF = BM * 64 * 2;       // one 64-wide swizzle panel
   static constexpr int B_BYTES = BN * kDim * 2;
   static constexpr int B_HALF = BN * 64 * 2;
-  static constexpr int STAGES = (QG == 1) ? 6 : 3;
+  static constexpr int STAGES = (QG == 1) ? 6 : (FILTER ? 2 : 3);
   static constexpr int ACC = (QG == 1) ? 8 : 2;       // accumulator stages in TMEM
   static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
   static constexpr int TMEM_COLS = (ACC * ACC_COLS <= 32) ? 32
@@ -54,7 +54,10 @@ struct TcCfg {
   static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
   static constexpr size_t SMEM_BAR = 512;
   static constexpr size_t SMEM_HIST = (QG == 1) ? kHistBins * 4 : 0;  // per-row selection histogram
-  static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR + SMEM_HIST;
+  // filter form: each epilogue warp stages up to SBUF candidates per query
+  static constexpr int SBUF = 64;
+  static constexpr size_t SMEM_F = FILTER ? size_t(EPI_WARPS) * Q_PER_EPI_WARP * SBUF * 8 : 0;
+  static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR + SMEM_HIST + SMEM_F;
   static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
   static_assert(ACC <= 8, "accumulator barriers");
 };
@@ -96,10 +99,10 @@ __device__ __forceinline__ int eligible_keys(const ScoreParams& p, int b, int t)
 // FILTER: the filter form of ScoreParams (p.out == nullptr), built as its own
 // instantiation so the storing form keeps its registers.
 template <int QG, bool FILTER>
-__global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
+__global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const ScoreParams p) {
-  using C = TcCfg<QG>;
+  using C = TcCfg<QG, FILTER>;
   if (p.run_if != nullptr && *p.run_if == 0) return;  // a conditional launch with nothing to do
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -284,39 +287,46 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
 #pragma unroll
     for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) elig[i] = 0, thr[i] = 0;
     constexpr bool filter = FILTER;
-    // Filter form: a query's slot reservation (one atomic per warp) is used
-    // one unit later, so the atomic's round trip overlaps the next unit.
-    float pend_s[C::Q_PER_EPI_WARP];
-    int32_t pend_lab[C::Q_PER_EPI_WARP];
-    uint32_t pend_bal[C::Q_PER_EPI_WARP], pend_base[C::Q_PER_EPI_WARP];
-    int64_t pend_at[C::Q_PER_EPI_WARP];
+    // Filter form: each warp stages its queries' candidates in shared memory
+    // and reserves global slots for a whole batch with one atomic.
+    float* fbuf = reinterpret_cast<float*>(smem + C::SMEM_A + C::SMEM_B + C::SMEM_BAR + C::SMEM_HIST) +
+                  static_cast<size_t>(ew) * C::Q_PER_EPI_WARP * C::SBUF * 2;
+    uint32_t fcnt[C::Q_PER_EPI_WARP];
+    int64_t frow[C::Q_PER_EPI_WARP];
 #pragma unroll
-    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) pend_bal[i] = 0;
-    auto flush_pending = [&]() {
-#pragma unroll
-      for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) {
-        if (pend_bal[i]) {                                 // warp-uniform
-          const uint32_t base = __shfl_sync(0xffffffffu, pend_base[i], 0);
-          if ((pend_bal[i] >> lane) & 1u) {
-            const uint32_t slot = base + static_cast<uint32_t>(__popc(pend_bal[i] & ((1u << lane) - 1u)));
-            if (slot < static_cast<uint32_t>(p.cand_cap)) {
-              p.cand_val[pend_at[i] + slot] = pend_s[i];
-              p.cand_lab[pend_at[i] + slot] = pend_lab[i];
-            } else {
-              p.row_over[(pend_at[i] - p.run_k) / p.ld_cand] = 1;
-              *p.any_over = 1;
-            }
-          }
-          pend_bal[i] = 0;
+    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) fcnt[i] = 0, frow[i] = 0;
+    auto flush_q = [&](int i) {                            // warp-uniform
+      __syncwarp();
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(p.cand_cnt + frow[i], fcnt[i]);
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const float* bv = fbuf + i * C::SBUF * 2;
+      const int32_t* bl = reinterpret_cast<const int32_t*>(bv + C::SBUF);
+      for (uint32_t e = lane; e < fcnt[i]; e += 32) {
+        const uint32_t slot = base + e;
+        if (slot < static_cast<uint32_t>(p.cand_cap)) {
+          const int64_t at = frow[i] * p.ld_cand + p.run_k + slot;
+          p.cand_val[at] = bv[e];
+          p.cand_lab[at] = bl[e];
+        } else {
+          p.row_over[frow[i]] = 1;
+          *p.any_over = 1;
         }
       }
+      __syncwarp();
+      fcnt[i] = 0;
+    };
+    auto flush_all = [&]() {
+#pragma unroll
+      for (int i = 0; i < C::Q_PER_EPI_WARP; ++i)
+        if (fcnt[i]) flush_q(i);
     };
     UnitPos up;
     up.init(u_begin, NT, G);
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
-      if (filter) flush_pending();
       const int tile = up.tile, g = up.g, b = up.b;
       const long long bg = static_cast<long long>(b) * G + g;
+      if (filter && bg != lim_bg) flush_all();             // staged entries belong to the previous group
       const int n = tile * C::BM + quad * 32 + lane;       // key within this launch
       int lim = p.N;
       if (p.n_valid) lim = min(lim, __ldg(p.n_valid + b));
@@ -388,12 +398,17 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
             }
             const bool take = (n < p.N) && (n < lim_t) && order_code(s) >= thr[jq];
             const uint32_t bal = __ballot_sync(0xffffffffu, take);
-            pend_bal[jq] = bal;
             if (bal) {
-              pend_base[jq] = (lane == 0) ? atomicAdd(p.cand_cnt + row, static_cast<uint32_t>(__popc(bal))) : 0u;
-              pend_s[jq] = s;
-              pend_lab[jq] = p.key_base + n;
-              pend_at[jq] = row * p.ld_cand + p.run_k;
+              frow[jq] = row;
+              const uint32_t add = static_cast<uint32_t>(__popc(bal));
+              if (fcnt[jq] + add > static_cast<uint32_t>(C::SBUF)) flush_q(jq);
+              if (take) {
+                const uint32_t off = fcnt[jq] + static_cast<uint32_t>(__popc(bal & ((1u << lane) - 1u)));
+                float* bv = fbuf + jq * C::SBUF * 2;
+                bv[off] = s;
+                reinterpret_cast<int32_t*>(bv + C::SBUF)[off] = p.key_base + n;
+              }
+              fcnt[jq] += add;
             }
           }
         }
@@ -407,7 +422,7 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
         role_barrier(1, C::EPI_WARPS * 32);
       }
     }
-    if (filter) flush_pending();
+    if (filter) flush_all();
   }
 
   tc_fence_before();
@@ -422,7 +437,7 @@ __global__ void __launch_bounds__(TcCfg<QG>::THREADS, 1)
 template <int QG, bool FILTER>
 static cudaError_t launch_tc(const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p, int num_sms,
                              cudaStream_t st) {
-  using C = TcCfg<QG>;
+  using C = TcCfg<QG, FILTER>;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<QG, FILTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
