@@ -219,6 +219,12 @@ __device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
+// 16-byte asynchronous global -> shared copy, bypassing L1 (both addresses
+// 16-byte aligned).
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
 // The mbarrier gets one more pending arrival now, and receives it once every
 // cp.async this thread issued so far has landed.
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {

@@ -249,24 +249,31 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
             atomicOr(&g_fault, FAULT_BAD_INDEX);
             rid[i] = -1;
           }
-          cnt += (rid[i] >= 0);
         }
+        // 16-byte cp.async chunks, ROW_BYTES / 16 lanes per row: one warp
+        // instruction copies 512 contiguous-per-row bytes (a per-row bulk copy
+        // each would queue 128 small copies on the TMA unit)
+        constexpr int CPR = C::ROW_BYTES / 16;           // chunks per row
+        constexpr int RPI = 32 / CPR;                    // rows per warp instruction
+        const int chunk = lane % CPR, sub = lane / CPR;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0) mbar_arrive_expect_tx(&bars->rfull[rs], static_cast<uint32_t>(cnt) * C::ROW_BYTES);
+        for (int it = 0; it < C::BM / RPI; ++it) {
+          const int r = it * RPI + sub;
+          const int32_t rr = __shfl_sync(0xffffffffu, rid[(it * RPI) >> 5], r & 31);  // row r's id: lane r % 32
+          if (rr >= 0)
+            cp_async_16(dst + r * C::ROW_BYTES + chunk * 16,
+                        keys + (static_cast<int64_t>(b) * p.key_stride + rr) * C::ROW_BYTES + chunk * 16);
+        }
+        cp_async_mbar_arrive(&bars->rfull[rs]);
         __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (rid[i] >= 0) {
-            const uint8_t* src = keys + (static_cast<int64_t>(b) * p.key_stride + rid[i]) * C::ROW_BYTES;
-            bulk_load(dst + (lane + 32 * i) * C::ROW_BYTES, src, C::ROW_BYTES, &bars->rfull[rs]);
-          }
-        }
+        if (lane == 0) mbar_arrive(&bars->rfull[rs]);
+        (void)cnt;
       }
       issued[rs] = 1;
       issued_par[rs] = rphase;
       if (++rs == C::RS) { rs = 0; rphase ^= 1; }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (!ok && lane == 0) {
       for (int s = 0; s < C::RS; ++s)
         if (issued[s]) cvt_wait_drain(&bars->rfull[s], issued_par[s]);

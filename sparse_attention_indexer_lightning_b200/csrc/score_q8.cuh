@@ -254,10 +254,11 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
           if (valid) cp_async_4(ssc + r, p.scale + static_cast<int64_t>(b) * p.N + j0 + r);
         }
       } else {
-        // lane l copies rows l, l+32, l+64, l+96; the next unit's row ids are
-        // read now, so their latency overlaps this unit's copies
+        // lane l holds the row ids of rows l, l+32, l+64, l+96 (the next
+        // unit's are read now, so their latency overlaps this unit's copies);
+        // the rows move as 16-byte cp.async chunks, eight lanes per row, so a
+        // warp instruction copies four whole rows
         int32_t rid[4];
-        int cnt = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) rid[i] = rid_next[i];
         if (u + 1 < u_end) {
@@ -270,21 +271,24 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
             atomicOr(&g_fault, FAULT_BAD_INDEX);
             rid[i] = -1;
           }
-          cnt += (rid[i] >= 0);
         }
+        const int chunk = lane & 7, sub = lane >> 3;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0) mbar_arrive_expect_tx(&bars->rfull[rs], static_cast<uint32_t>(cnt) * C::ROW);
+        for (int it = 0; it < C::BM / 4; ++it) {
+          const int r = it * 4 + sub;
+          const int32_t rr = __shfl_sync(0xffffffffu, rid[it >> 3], r & 31);
+          if (rr >= 0)
+            cp_async_16(dst + r * C::PITCH + chunk * 16,
+                        keys + (static_cast<int64_t>(b) * p.key_stride + rr) * C::ROW + chunk * 16);
+        }
+        cp_async_mbar_arrive(&bars->rfull[rs]);
         __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->rfull[rs]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = lane + 32 * i;
           sok[r] = rid[i] >= 0 ? 1 : 0;
-          if (rid[i] >= 0) {
-            const int64_t src_row = static_cast<int64_t>(b) * p.key_stride + rid[i];
-            bulk_load(dst + r * C::PITCH, keys + src_row * C::ROW, C::ROW, &bars->rfull[rs]);
-            cp_async_4(ssc + r, p.scale + src_row);
-          }
+          if (rid[i] >= 0) cp_async_4(ssc + r, p.scale + static_cast<int64_t>(b) * p.key_stride + rid[i]);
         }
       }
       cp_async_mbar_arrive(&bars->sfull[ss]);
