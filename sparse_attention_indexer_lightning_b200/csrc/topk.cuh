@@ -40,7 +40,8 @@
 namespace lsi {
 
 constexpr int kCandCap = 8192;     // listed candidates kept in shared memory
-constexpr int kExactHistMax = 8192; // rows up to this length get an exact histogram
+constexpr int kExactHistMax = 2048; // rows up to this length get an exact histogram; longer rows
+                                    // sample about this many entries
 constexpr int kVec = 4;            // float4 loads per thread per chunk
 constexpr int kChunk = kVec * 4;   // entries per thread per chunk
 
@@ -622,9 +623,13 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
     }
     __syncthreads();
   }
+  int32_t* io = p.idx_out + static_cast<int64_t>(r) * p.ld_out;
+  float* vo = p.val_out ? p.val_out + static_cast<int64_t>(r) * p.ld_out : nullptr;
+  const int lab_add = rr.lab ? 0 : p.label_base;
+  const int nc_all = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(kCandCap)));
   if (kk > 0) {
     // ---- 4. select inside the candidate list ------------------------------
-    const int nc = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(kCandCap)));
+    const int nc = nc_all;
     unsigned long long thr = 0ull;
     if (nc > kk) thr = radix_select_cand<NT>(sh, nc, static_cast<uint32_t>(kk));
     if (tid == 0) sh.cnt = 0;
@@ -655,8 +660,6 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
   }
 
   // ---- 5. canonical order: bucket by key range, rank inside the bucket ----
-  int32_t* io = p.idx_out + static_cast<int64_t>(r) * p.ld_out;
-  float* vo = p.val_out ? p.val_out + static_cast<int64_t>(r) * p.ld_out : nullptr;
   if (kk > 0) {
     unsigned long long kmin = ~0ull, kmax = 0ull;
     for (int i = tid; i < kk; i += NT) {
@@ -722,7 +725,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
       const uint32_t beg = end - sh.hist[bin];
       uint32_t rank = beg;
       for (uint32_t j = beg; j < end; ++j) rank += (sh.tmp_key[j] > key) ? 1u : 0u;
-      io[rank] = static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull)) + (rr.lab ? 0 : p.label_base);
+      io[rank] = static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull)) + lab_add;
       if (vo) vo[rank] = sh.tmp_val[i];
     }
   }
