@@ -51,9 +51,9 @@ struct TopkShared {
   float cand_val[kCandCap];            // listed entries: value and label
   int32_t cand_lab[kCandCap];
   unsigned long long sel_key[KMAX];    // the k selected: packed key and value
-  float sel_val[KMAX];
   unsigned long long tmp_key[KMAX];    // bucketed copy for the final order
-  float tmp_val[KMAX];
+  float sel_val[KMAX];                 // (sel_key + tmp_key and sel_val + tmp_val are also
+  float tmp_val[KMAX];                 //  used as one 2*KMAX array by the bucket select)
   uint32_t hist[kHistBins];
   uint32_t fill[kHistBins];
   uint32_t wsum[NT / 32];
@@ -627,6 +627,94 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
   float* vo = p.val_out ? p.val_out + static_cast<int64_t>(r) * p.ld_out : nullptr;
   const int lab_add = rr.lab ? 0 : p.label_base;
   const int nc_all = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(kCandCap)));
+  // ---- 4'. bucket select: selection and canonical order in one pass -------
+  // The candidates are bucketed by their position in the [min, max] key range
+  // (2048 bins); the bins from the top hold the k largest keys up to the
+  // boundary bin.  Keys of the bins down to the boundary are scattered (in
+  // bin order) into a 2*KMAX buffer and ranked inside their bin; a key's rank
+  // is its output slot, kept if below k.  When the boundary bin reaches past
+  // the buffer, the radix path below runs instead.
+  if (kk > 0) {
+    unsigned long long kmin = ~0ull, kmax = 0ull;
+    for (int i = tid; i < nc_all; i += NT) {
+      const unsigned long long key = pack_key(sh.cand_val[i], sh.cand_lab[i]);
+      kmin = key < kmin ? key : kmin;
+      kmax = key > kmax ? key : kmax;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+      const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
+      kmin = a < kmin ? a : kmin;
+      kmax = b > kmax ? b : kmax;
+    }
+    if (lane == 0) {
+      sh.wmin[warp] = kmin;
+      sh.wmax[warp] = kmax;
+    }
+    for (int i = tid; i < kHistBins; i += NT) {
+      sh.hist[i] = 0;
+      sh.fill[i] = 0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      kmin = lane < NT / 32 ? sh.wmin[lane] : ~0ull;
+      kmax = lane < NT / 32 ? sh.wmax[lane] : 0ull;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+        const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
+        kmin = a < kmin ? a : kmin;
+        kmax = b > kmax ? b : kmax;
+      }
+      if (lane == 0) {
+        sh.wmin[0] = kmin;
+        sh.wmax[0] = kmax;
+      }
+    }
+    __syncthreads();
+    kmin = sh.wmin[0];
+    kmax = sh.wmax[0];
+    const unsigned long long span = kmax - kmin;
+    const int shift = span ? max(0, 64 - __clzll(static_cast<long long>(span)) - kHistBits) : 0;
+    for (int i = tid; i < nc_all; i += NT) {
+      const unsigned long long key = pack_key(sh.cand_val[i], sh.cand_lab[i]);
+      atomicAdd(&sh.hist[static_cast<uint32_t>((key - kmin) >> shift)], 1u);
+    }
+    __syncthreads();
+    scan_bins_2048<NT>(sh, sh.hist, sh.fill, static_cast<uint32_t>(kk));  // fill: offsets from the top
+    const uint32_t b_end = sh.fill[sh.digit] + sh.hist[sh.digit];         // end of the boundary bin
+    if (b_end <= 2u * KMAX) {
+      unsigned long long* bkey = sh.sel_key;  // 2*KMAX keys
+      float* bval = sh.sel_val;               // 2*KMAX values
+      for (int i = tid; i < nc_all; i += NT) {
+        const float v = sh.cand_val[i];
+        const unsigned long long key = pack_key(v, sh.cand_lab[i]);
+        const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
+        if (sh.fill[bin] < b_end) {  // a bin at or above the boundary (its offset only grows past b_end if not)
+          const uint32_t pos = atomicAdd(&sh.fill[bin], 1u);
+          bkey[pos] = key;
+          bval[pos] = v;
+        }
+      }
+      __syncthreads();
+      // after the scatter fill[bin] is the bin's end
+      for (int i = tid; i < static_cast<int>(b_end); i += NT) {
+        const unsigned long long key = bkey[i];
+        const uint32_t bin = static_cast<uint32_t>((key - kmin) >> shift);
+        const uint32_t end = sh.fill[bin];
+        const uint32_t beg = end - sh.hist[bin];
+        uint32_t rank = beg;
+        for (uint32_t j = beg; j < end; ++j) rank += (bkey[j] > key) ? 1u : 0u;
+        if (rank < static_cast<uint32_t>(kk)) {
+          io[rank] = static_cast<int32_t>(~static_cast<uint32_t>(key & 0xffffffffull)) + lab_add;
+          if (vo) vo[rank] = bval[i];
+        }
+      }
+      kk = -kk;  // done: only the padding is left
+    }
+    __syncthreads();
+  }
   if (kk > 0) {
     // ---- 4. select inside the candidate list ------------------------------
     const int nc = nc_all;
@@ -729,6 +817,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
       if (vo) vo[rank] = sh.tmp_val[i];
     }
   }
+  if (kk < 0) kk = -kk;
   for (int j = kk + tid; j < p.k; j += NT) {
     io[j] = -1;
     if (vo) vo[j] = neg_inf();
