@@ -392,7 +392,9 @@ def bench_prefill(L, args, peaks, peak_kind, full_scores=True):
         "ms_per_step": ms, "positions_per_s": pairs / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
         "kernels": kern,
         "roofline": roofline("tensor", flops_alg / (score_ms * 1e-3) / 1e12, peak_t, "TFLOP/s",
-                             traffic=ncu_traffic("score_tc_kernel<8>", wl.name), peak_kind=peak_kind),
+                             traffic=ncu_traffic("score_tc_kernel<8>",
+                                                 wl.name if full_scores else wl.name + "_running"),
+                             peak_kind=peak_kind),
         "algorithmic_flops": flops_alg, "eligible_pairs": pairs,
         "workspace_bytes": ws.numel(),
         "note": ("step = 4 streamed 8192-key tiles (H2D on a copy stream) + causal top-512 of 4096 queries; "
