@@ -29,7 +29,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .formats import bf16_to_f64, dequant
+from .formats import bf16_to_f64, dequant, pq_decode
 from .indexer import eligible_count, indexer_scores
 
 
@@ -108,19 +108,29 @@ def prefill_select(q_bits, w, q_pos, k_bits, stride: int = 4, k: int = 512, rows
     return idx, val
 
 
+def two_stage_pq_select(q_bits, w, pq_codes, pq_books, fk, fk_scale, n_valid, shortlist: int, k: int = 512,
+                        rows=None, return_detail: bool = False):
+    """The two-stage search with PQ compact keys: scores of the PQ-decoded keys
+    -> shortlist -> exact re-rank of the fp8 originals -> top-k."""
+    return two_stage_select(q_bits, w, None, None, fk, fk_scale, n_valid, shortlist, k, rows, return_detail,
+                            coarse=lambda b, n: pq_decode(pq_codes[b, :n], pq_books))
+
+
 def two_stage_select(q_bits, w, ck, ck_scale, fk, fk_scale, n_valid, shortlist: int, k: int = 512,
-                     rows=None, return_detail: bool = False):
-    """Compact scan -> shortlist -> exact re-rank of the originals -> top-k."""
+                     rows=None, return_detail: bool = False, coarse=None):
+    """Compact scan -> shortlist -> exact re-rank of the originals -> top-k.
+    ``coarse(b, n)`` gives the compact keys of row b (default: int8 x scale)."""
     B = q_bits.shape[0]
     rows = np.arange(B) if rows is None else np.asarray(rows)
     idx = np.empty((rows.size, k), dtype=np.int64)
     val = np.empty((rows.size, k), dtype=np.float64)
     detail = []
     for i, b in enumerate(rows):
-        n = int(n_valid[b]) if n_valid is not None else ck.shape[1]
+        n = int(n_valid[b]) if n_valid is not None else fk.shape[1]
         qb = bf16_to_f64(q_bits[b])[None]
         wb = np.asarray(w[b], np.float64)[None]
-        s_hat = indexer_scores(qb, wb, dequant(ck[b, :n], ck_scale[b, :n], "int8"))[0]
+        kc = dequant(ck[b, :n], ck_scale[b, :n], "int8") if coarse is None else coarse(b, n)
+        s_hat = indexer_scores(qb, wb, kc)[0]
         short, _ = select_topk(s_hat, np.arange(n), shortlist)
         short = short[short >= 0]
         exact = indexer_scores(qb, wb, dequant(fk[b, short], fk_scale[b, short], "e4m3"))[0]

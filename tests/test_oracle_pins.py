@@ -14,11 +14,11 @@ import pytest
 import torch
 
 from oracle import brute, sizes
-from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64
+from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64, f16_to_f64, pq_decode
 from oracle.indexer import eligible_blocks, eligible_count, indexer_scores
 from oracle.select import (
     bucket_select, decode_select, expand_buckets, prefill_select, recall_at_k, select_topk,
-    topk_rows, two_stage_select,
+    topk_rows, two_stage_pq_select, two_stage_select,
 )
 from workloads import make_workload
 from workloads.synth import make_bucket, make_decode, make_two_stage, to_bf16_bits
@@ -48,6 +48,73 @@ def test_e4m3_decode_all_codes():
     assert e4m3_to_f64(np.array([0x01]))[0] == 2.0 ** -9
     assert e4m3_to_f64(np.array([0x38]))[0] == 1.0
     assert e4m3_to_f64(np.array([0xB8]))[0] == -1.0
+
+
+def test_f16_decode_all_codes():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = f16_to_f64(bits)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert f16_to_f64(np.array([0x7BFF]))[0] == 65504.0
+    assert f16_to_f64(np.array([0x0001]))[0] == 2.0 ** -24
+    assert f16_to_f64(np.array([0x3C00]))[0] == 1.0
+    assert f16_to_f64(np.array([0xFC00]))[0] == -np.inf
+
+
+def test_pq_decode_brute_force():
+    rng = np.random.default_rng(21)
+    books = (rng.standard_normal((32, 256, 4)) * 0.1).astype(np.float16).view(np.uint16)
+    codes = rng.integers(0, 256, size=(5, 32)).astype(np.uint8)
+    got = pq_decode(codes, books)
+    for r in range(5):
+        want = []
+        for m in range(32):
+            for j in range(4):
+                want.append(float(np.float16(books[m, codes[r, m], j].view(np.float16))))
+        assert got[r].tolist() == want
+
+
+def test_pq_generator_codes_are_nearest_centroids():
+    d = make_two_stage(B=2, N=900, seed=22, plant_frac=0.05, ragged=200, pq=True, pq_sample=1200)
+    books = f16_to_f64(d["pq_books"])                                  # [32, 256, 4]
+    keys = dequant(d["fk"][1, :50], d["fk_scale"][1, :50], "e4m3")      # [50, 128]
+    for m in range(32):
+        x = keys[:, 4 * m: 4 * m + 4]
+        d2 = ((x[:, None, :] - books[m][None]) ** 2).sum(-1)            # [50, 256]
+        chosen = d2[np.arange(50), d["pq_codes"][1, :50, m].astype(np.int64)]
+        assert np.all(chosen <= d2.min(1) * (1 + 1e-5) + 1e-12)
+
+
+def test_two_stage_pq_full_shortlist_equals_exact():
+    d = make_two_stage(B=2, N=700, seed=23, plant_frac=0.05, ragged=100, pq=True, pq_sample=1000)
+    n = d["n_valid"]
+    got_i, got_v = two_stage_pq_select(d["q"], d["w"], d["pq_codes"], d["pq_books"], d["fk"], d["fk_scale"], n,
+                                       shortlist=700, k=32)
+    for b in range(2):
+        keys = dequant(d["fk"][b, : n[b]], d["fk_scale"][b, : n[b]], "e4m3")
+        s = indexer_scores(bf16_to_f64(d["q"][b])[None], d["w"][b].astype(np.float64)[None], keys)[0]
+        ei, ev = select_topk(s, np.arange(n[b]), 32)
+        assert np.array_equal(got_i[b], ei)
+        assert np.array_equal(got_v[b], ev)
+
+
+def test_two_stage_pq_brute_force_tiny():
+    d = make_two_stage(B=1, N=60, seed=24, plant_frac=0.1, pq=True, pq_sample=60)
+    gi, gv, det = two_stage_pq_select(d["q"], d["w"], d["pq_codes"], d["pq_books"], d["fk"], d["fk_scale"],
+                                      d["n_valid"], shortlist=12, k=5, return_detail=True)
+    qb = bf16_to_f64(d["q"][0]).tolist()
+    wb = d["w"][0].astype(np.float64).tolist()
+    books = d["pq_books"].view(np.float16)
+    ck = [[float(books[m, d["pq_codes"][0, s, m], j]) for m in range(32) for j in range(4)] for s in range(60)]
+    fk = e4m3_to_f64(d["fk"][0]) * d["fk_scale"][0].astype(np.float64)[:, None]
+    shat = [brute.score(qb, wb, ck[s]) for s in range(60)]
+    short, _ = brute.topk(shat, list(range(60)), 12)
+    ex = [brute.score(qb, wb, fk[s].tolist()) for s in short]
+    bp, _ = brute.topk(ex, short, 5)
+    assert gi[0].tolist() == bp
+    assert det[0]["shortlist"].tolist() == short
 
 
 def test_dequant_scales():

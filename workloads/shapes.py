@@ -81,6 +81,12 @@ WORKLOADS: Dict[str, Workload] = {
     "two_stage": Workload(
         "two_stage", "two_stage", B=32, N=131072, shortlist=4096, plant_frac=0.05, plant_cos=0.6
     ),
+    # the same search with 32-byte PQ compact keys (LeanSparse podcast
+    # transcript, 07:12-07:34) in place of the int8 ones
+    "two_stage_pq": Workload(
+        "two_stage_pq", "two_stage", B=32, N=131072, shortlist=4096, plant_frac=0.05, plant_cos=0.6,
+        extra={"pq": 1},
+    ),
     "bucket": Workload(
         "bucket", "bucket", T=256, clusters=32768, cluster_size=8, noise_rel=0.3, top_p=64, budget=512
     ),
@@ -91,6 +97,10 @@ WORKLOADS: Dict[str, Workload] = {
     ),
     "two_stage_s": Workload(
         "two_stage_s", "two_stage", B=3, N=9000, shortlist=1024, plant_frac=0.05, plant_cos=0.6, ragged=1500
+    ),
+    "two_stage_pq_s": Workload(
+        "two_stage_pq_s", "two_stage", B=3, N=9000, shortlist=1024, plant_frac=0.05, plant_cos=0.6, ragged=1500,
+        extra={"pq": 1},
     ),
     "bucket_s": Workload(
         "bucket_s", "bucket", T=19, clusters=1500, cluster_size=8, noise_rel=0.3, top_p=64, budget=512,

@@ -9,6 +9,9 @@ oracle read:
 * fp8 e4m3 tensors as ``uint8`` codes (torch's ``float8_e4m3fn`` cast, input
   clipped to +-448 first so nothing becomes NaN),
 * int8 tensors as ``int8``, scales and head weights as ``float32``,
+* product-quantisation (PQ) compact keys as ``uint8`` codes (32 per key, one
+  per 4-dimension sub-vector) with fp16 codebooks as ``uint16`` bit patterns
+  [32][256][4], the codebooks trained by k-means on a sample of the keys,
 * positions as ``int64`` / ``int32``.
 
 Distributions (all workloads): q, k ~ N(0, 1)/sqrt(d), w ~ N(0, 1)/sqrt(H).
@@ -59,6 +62,57 @@ def _normal(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------- #
+# product quantisation of the compact keys (LeanSparse podcast transcript,
+# 07:12-07:34: compact keys of 32 bytes): 32 sub-vectors of 4 dimensions, 256
+# centroids each
+# --------------------------------------------------------------------------- #
+PQ_M, PQ_K, PQ_SUB = 32, 256, 4
+
+
+def train_pq_books(x: np.ndarray, rng: np.random.Generator, iters: int = 10) -> np.ndarray:
+    """Lloyd k-means per sub-space on the rows of x [n, 128], centroids seeded
+    from sample rows (distinct when n >= 256; one draw per sub-space), empty
+    clusters keeping
+    their centroid; assignments by fp32 squared distance, means in fp64.
+    Returns the codebooks rounded to fp16, as bit patterns [32][256][4]."""
+    n = x.shape[0]
+    xs = np.ascontiguousarray(np.asarray(x, dtype=np.float64).reshape(n, PQ_M, PQ_SUB).transpose(1, 0, 2))
+    c = np.stack([xs[m, rng.choice(n, size=PQ_K, replace=n < PQ_K)] for m in range(PQ_M)])  # [32, 256, 4]
+    xt32 = torch.from_numpy(xs.astype(np.float32))
+    xt64 = torch.from_numpy(xs)
+    for _ in range(iters):
+        ct = torch.from_numpy(c.astype(np.float32))
+        a = ((ct * ct).sum(-1)[:, None, :] - 2.0 * torch.bmm(xt32, ct.transpose(1, 2))).argmin(-1)  # [32, n]
+        cnt = torch.zeros(PQ_M, PQ_K, dtype=torch.float64).scatter_add_(1, a, torch.ones_like(a, dtype=torch.float64))
+        sums = torch.zeros(PQ_M, PQ_K, PQ_SUB, dtype=torch.float64).scatter_add_(
+            1, a[..., None].expand(-1, -1, PQ_SUB), xt64)
+        cnt = cnt.numpy()
+        nz = cnt > 0
+        c[nz] = sums.numpy()[nz] / cnt[nz][:, None]
+    return c.astype(np.float16).view(np.uint16)
+
+
+def encode_pq(x: np.ndarray, books_bits: np.ndarray) -> np.ndarray:
+    """Rows of x [n, 128] -> the index of the nearest fp16 centroid (squared
+    Euclidean distance in fp32) per sub-vector: uint8 codes [n, 32].  Runs on
+    the GPU when one is present (the codes are an input like any other: both
+    the oracle and the CUDA path read the same array)."""
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    books = torch.from_numpy(books_bits.view(np.float16).astype(np.float32)).to(dev)  # [32, 256, 4]
+    bt = books.transpose(1, 2).contiguous()                                            # [32, 4, 256]
+    cn = (books * books).sum(-1)[:, None, :]                                           # [32, 1, 256]
+    n = x.shape[0]
+    codes = np.empty((n, PQ_M), dtype=np.uint8)
+    step = 1 << 15
+    for lo in range(0, n, step):
+        xs = torch.from_numpy(np.ascontiguousarray(x[lo: lo + step], dtype=np.float32)).to(dev)
+        xs = xs.view(-1, PQ_M, PQ_SUB).transpose(0, 1)                                  # [32, c, 4]
+        a = (cn - 2.0 * torch.bmm(xs, bt)).argmin(-1)                                   # [32, c]
+        codes[lo: lo + xs.shape[1]] = a.transpose(0, 1).to(torch.uint8).cpu().numpy()
+    return codes
+
+
+# --------------------------------------------------------------------------- #
 # decode: B sequences, one query each, bf16 keys
 # --------------------------------------------------------------------------- #
 def make_decode(
@@ -102,7 +156,7 @@ def make_prefill(
 # --------------------------------------------------------------------------- #
 def make_two_stage(
     B: int, N: int, H: int = 32, d: int = 128, seed: int = 0, plant_frac: float = 0.05,
-    plant_cos: float = 0.6, ragged: int = 0,
+    plant_cos: float = 0.6, ragged: int = 0, pq: bool = False, pq_sample: int = 8192,
 ) -> Dict[str, np.ndarray]:
     """Full keys: fp8 e4m3 codes with a per-key fp32 scale amax/448.
 
@@ -112,7 +166,10 @@ def make_two_stage(
     max(w_h, 0) q_h); the key keeps the norm of the Gaussian draw it replaces.
 
     Compact keys: int8 codes of the dequantised full key with a per-key fp32
-    scale amax/127, rounded half to even, clamped to +-127.
+    scale amax/127, rounded half to even, clamped to +-127.  With ``pq``, also
+    PQ codes of the dequantised full keys against codebooks trained on
+    ``pq_sample`` keys drawn (after everything above) uniformly from all
+    sequences' valid positions.
     """
     rng = np.random.default_rng(seed)
     q = to_bf16_bits(_normal(rng, (B, H, d), 1.0 / math.sqrt(d)))
@@ -150,10 +207,25 @@ def make_two_stage(
         n_valid = rng.integers(max(N - ragged, 0), N + 1, size=B)
     else:
         n_valid = np.full(B, N)
-    return {
+    out = {
         "q": q, "w": w, "fk": fk, "fk_scale": fk_scale, "ck": ck, "ck_scale": ck_scale,
         "n_valid": n_valid.astype(np.int32), "planted": planted,
     }
+    if pq:
+        def deq(b, sel=slice(None)):
+            return e4m3_codes_to_f32(fk[b, sel]).astype(np.float64) * fk_scale[b, sel].astype(np.float64)[:, None]
+        tot = int(n_valid.sum())
+        pick = np.sort(rng.choice(tot, size=min(pq_sample, tot), replace=False))
+        starts = np.concatenate([[0], np.cumsum(n_valid)])
+        bi = np.searchsorted(starts, pick, side="right") - 1
+        sample = np.concatenate([deq(b, pick[bi == b] - starts[b]) for b in range(B) if np.any(bi == b)])
+        books = train_pq_books(sample, rng)
+        codes = np.empty((B, N, PQ_M), dtype=np.uint8)
+        for b in range(B):
+            codes[b] = encode_pq(deq(b), books)
+        out["pq_codes"] = codes
+        out["pq_books"] = books
+    return out
 
 
 # --------------------------------------------------------------------------- #
@@ -218,7 +290,8 @@ def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
     if wl.kind == "prefill":
         return make_prefill(wl.T, wl.N, wl.q_pos0, wl.H, wl.d, s)
     if wl.kind == "two_stage":
-        return make_two_stage(wl.B, wl.N, wl.H, wl.d, s, wl.plant_frac, wl.plant_cos, ragged=wl.ragged)
+        return make_two_stage(wl.B, wl.N, wl.H, wl.d, s, wl.plant_frac, wl.plant_cos, ragged=wl.ragged,
+                              pq=bool(wl.extra.get("pq", 0)))
     if wl.kind == "bucket":
         return make_bucket(
             wl.T, wl.clusters, wl.cluster_size, wl.H, wl.d, s, wl.noise_rel,
