@@ -336,7 +336,8 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
     res = {}
     for name, fn in (("prefill_chunk", bench_prefill),
                      ("prefill_chunk_running", lambda *a: bench_prefill(*a, full_scores=False)),
-                     ("bucket", bench_bucket), ("two_stage", bench_two_stage)):
+                     ("bucket", bench_bucket), ("two_stage", bench_two_stage),
+                     ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True))):
         if only in (None, name):
             res[name] = fn(L, args, peaks, peak_kind)
     return res
@@ -443,38 +444,45 @@ def bench_bucket(L, args, peaks, peak_kind):
     return res
 
 
-def bench_two_stage(L, args, peaks, peak_kind):
-    """Two-stage decode search: compact scan, shortlist, exact re-rank."""
+def bench_two_stage(L, args, peaks, peak_kind, pq=False):
+    """Two-stage decode search: compact scan (int8 + scale, or 32-byte PQ codes), shortlist, exact re-rank."""
     import torch
     from workloads import get_workload, make_workload
     st = torch.cuda.current_stream()
     steps = max(3, args.steps)
     warm = max(3, args.warmup)
-    wl = get_workload("two_stage")
+    wl = get_workload("two_stage_pq" if pq else "two_stage")
     d = make_workload(wl)
     B, H, dd = d["q"].shape
-    N = d["ck"].shape[1]
-    a2 = [to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev(d["ck"]), to_dev(d["ck_scale"]),
-          to_dev(d["fk"]).view(torch.float8_e4m3fn), to_dev(d["fk_scale"])]
+    N = d["fk"].shape[1]
+    fk = [to_dev(d["fk"]).view(torch.float8_e4m3fn), to_dev(d["fk_scale"])]
+    if pq:
+        books = torch.from_numpy(d["pq_books"].view(np.int16)).view(torch.float16).cuda()
+        a2 = [to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev(d["pq_codes"]), books] + fk
+        call = L.ls_decode_two_stage_pq_select
+        scan_name, scan_bytes = "score_q8_kernel<pq>", B * N * 32
+    else:
+        a2 = [to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev(d["ck"]), to_dev(d["ck_scale"])] + fk
+        call = L.ls_decode_two_stage_select
+        scan_name, scan_bytes = "score_q8_kernel<int8>", B * N * (dd + 4)
     ws2 = torch.empty(L.lib().ls_two_stage_workspace_size(B, N, wl.shortlist), dtype=torch.uint8, device="cuda")
     out2 = (torch.empty((B, wl.k), dtype=torch.int32, device="cuda"),
             torch.empty((B, wl.k), dtype=torch.float32, device="cuda"))
 
     def ts(i, timed):
-        L.ls_decode_two_stage_select(*a2, shortlist=wl.shortlist, k=wl.k, ws=ws2, out=out2)
+        call(*a2, shortlist=wl.shortlist, k=wl.k, ws=ws2, out=out2)
         return None
 
     ms, kern = _profiled_loop(L, ts, steps, warm, st)
-    scan_ms = kern["score_q8_kernel<int8>"]["ms_per_step"]
-    scan_bytes = B * N * (dd + 4)
+    scan_ms = kern[scan_name]["ms_per_step"]
     res = {
         "ms_per_step": ms, "positions_per_s": B * (N + wl.shortlist) / (ms * 1e-3),
         "selections_per_s": B / (ms * 1e-3), "kernels": kern,
         "roofline": roofline("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
-                             traffic=ncu_traffic("score_q8_kernel<int8>", wl.name), peak_kind=peak_kind),
+                             traffic=ncu_traffic(scan_name, wl.name), peak_kind=peak_kind),
         "algorithmic_bytes_scan": scan_bytes,
         "note": "positions = compact keys scanned + shortlist re-ranked; roofline of the compact scan "
-                "(int8 codes + fp32 scales)",
+                + ("(32-byte PQ codes; codebooks stay in shared memory)" if pq else "(int8 codes + fp32 scales)"),
     }
     del a2, ws2
     torch.cuda.empty_cache()
@@ -552,7 +560,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_batch")
     ap.add_argument("--no-variants", action="store_true")
-    ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "bucket", "two_stage"],
+    ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "bucket", "two_stage",
+                                                     "two_stage_pq"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

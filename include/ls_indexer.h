@@ -225,6 +225,35 @@ ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const in
                                      int32_t* shortlist_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ls_decode_two_stage_pq_select -- the same search with 32-byte product-
+ * quantised compact keys, the LeanSparse compact-key form (podcast
+ * transcript, 07:12-07:34): a key is 32 one-byte codes, code m choosing row
+ * code[m] of codebook m, whose 4 values are dimensions 4m..4m+3 of the
+ * decoded key.  The coarse score is the indexer score of the decoded key;
+ * the shortlist is re-ranked exactly with the fp8 originals as above.
+ *
+ *   pq_codes [B][N][32] uint8
+ *   pq_books [32][256][4] fp16 (IEEE binary16 bit patterns), 16-byte aligned
+ * Other arguments, outputs, errors and workspace as ls_decode_two_stage_select.
+ */
+ls_status ls_decode_two_stage_pq_select(const uint16_t* q, const float* w, const uint8_t* pq_codes,
+                                        const uint16_t* pq_books, const uint8_t* fk, const float* fk_scale,
+                                        const int32_t* n_valid, int B, int H, int d, int N, int shortlist, int k,
+                                        int32_t* idx_out, float* val_out, int32_t* shortlist_out, void* ws,
+                                        size_t ws_bytes, void* stream);
+
+/*
+ * ls_indexer_score_pq -- coarse scores of PQ compact keys (one query per
+ * sequence): scores[b][n] = sum_h w[b,h] * max(0, q[b,h] . key(b,n)), key
+ * decoded from pq_codes[b][n] with pq_books as in
+ * ls_decode_two_stage_pq_select; -inf for n >= n_valid[b].
+ *   q [B][H][d] bf16, w [B][H] fp32, pq_codes [B][N][32], pq_books [32][256][4]
+ *   fp16, scores [B][N] fp32; all device pointers, 16-byte aligned.
+ */
+ls_status ls_indexer_score_pq(const uint16_t* q, const float* w, const uint8_t* pq_codes, const uint16_t* pq_books,
+                              const int32_t* n_valid, int B, int H, int d, int N, float* scores, void* stream);
+
+/*
  * ls_bucket_select -- LSA-style flat bucket search with indexer-form scoring
  * ("Latent Sparse Attention", "How LSA finds the keys" and "The method, term
  * by term", steps 5-6): score every bucket centroid, keep the top_p buckets,

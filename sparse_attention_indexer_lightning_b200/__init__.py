@@ -15,9 +15,11 @@ from ._lib import (  # noqa: F401
     ls_bucket_select,
     ls_decode_select,
     ls_decode_select_noalloc,
+    ls_decode_two_stage_pq_select,
     ls_decode_two_stage_select,
     ls_device_status,
     ls_indexer_score,
+    ls_indexer_score_pq,
     ls_prefill_select_stream,
     ls_profile_begin,
     ls_profile_end,

@@ -35,7 +35,8 @@ EXPORTED = (
     "ls_decode_select_workspace_size", "ls_decode_select", "ls_prefill_select_workspace_size",
     "ls_prefill_select_stream", "ls_two_stage_workspace_size", "ls_decode_two_stage_select",
     "ls_bucket_workspace_size", "ls_bucket_select", "ls_selftest_wait_probe", "ls_profile_begin",
-    "ls_profile_end", "ls_profile_kernel", "ls_decode_select_noalloc",
+    "ls_profile_end", "ls_profile_kernel", "ls_decode_select_noalloc", "ls_decode_two_stage_pq_select",
+    "ls_indexer_score_pq",
 )
 HIST_BINS = 2048
 
@@ -72,6 +73,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_profile_end": (I, [P]),
         "ls_profile_kernel": (I, [I, P, P, P]),
         "ls_decode_select_noalloc": (I, [P, P, P, P, I, I, I, I, I, P, P, P]),
+        "ls_decode_two_stage_pq_select": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P]),
+        "ls_indexer_score_pq": (I, [P, P, P, P, P, I, I, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -278,6 +281,62 @@ def ls_decode_two_stage_select(q, w, ck, ck_scale, fk, fk_scale, n_valid=None, s
     _check(lib().ls_decode_two_stage_select(_ptr(q), _ptr(w), _ptr(ck), _ptr(ck_scale), _ptr(fk), _ptr(fk_scale),
                                             _ptr(n_valid), B, H, d, N, shortlist, k, _ptr(idx), _ptr(val), _ptr(sl),
                                             _ptr(ws), ws.numel(), _stream(stream)))
+    if want_shortlist:
+        return idx, val, sl
+    return idx, val
+
+
+def _pq_args(pq_codes, pq_books):
+    _dev(pq_codes, torch.uint8, "pq_codes", 3)
+    if pq_codes.shape[2] != 32:
+        raise ValueError("pq_codes must be [B, N, 32]")
+    if pq_books.dtype == torch.int16:
+        pq_books = pq_books.view(torch.float16)
+    _dev(pq_books, torch.float16, "pq_books", 3)
+    if tuple(pq_books.shape) != (32, 256, 4):
+        raise ValueError("pq_books must be [32, 256, 4] fp16")
+    return pq_codes, pq_books
+
+
+def ls_indexer_score_pq(q, w, pq_codes, pq_books, n_valid=None, stream=None):
+    """q [B,H,d] bf16, w [B,H] f32, pq_codes [B,N,32] uint8, pq_books [32,256,4] fp16 -> scores [B,N] f32."""
+    _dev(q, torch.bfloat16, "q", 3)
+    B, H, d = q.shape
+    _dev(w, torch.float32, "w", 2)
+    pq_codes, pq_books = _pq_args(pq_codes, pq_books)
+    N = pq_codes.shape[1]
+    _opt(n_valid, torch.int32, "n_valid")
+    out = torch.empty((B, N), dtype=torch.float32, device=q.device)
+    _check(lib().ls_indexer_score_pq(_ptr(q), _ptr(w), _ptr(pq_codes), _ptr(pq_books), _ptr(n_valid), B, H, d, N,
+                                     _ptr(out), _stream(stream)))
+    return out
+
+
+def ls_decode_two_stage_pq_select(q, w, pq_codes, pq_books, fk, fk_scale, n_valid=None, shortlist: int = 4096,
+                                  k: int = 512, want_shortlist: bool = False, ws=None, out=None, stream=None):
+    """Two-stage decode search with PQ compact keys (pq_codes [B,N,32] uint8, pq_books [32,256,4] fp16) and the
+    fp8 originals fk e4m3 [B,N,d] + fk_scale [B,N] for the exact re-rank."""
+    _dev(q, torch.bfloat16, "q", 3)
+    B, H, d = q.shape
+    _dev(w, torch.float32, "w", 2)
+    pq_codes, pq_books = _pq_args(pq_codes, pq_books)
+    N = pq_codes.shape[1]
+    if fk.dtype == torch.uint8:
+        fk = fk.view(torch.float8_e4m3fn)
+    _dev(fk, torch.float8_e4m3fn, "fk", 3)
+    _dev(fk_scale, torch.float32, "fk_scale", 2)
+    _opt(n_valid, torch.int32, "n_valid")
+    need = lib().ls_two_stage_workspace_size(B, N, shortlist)
+    if ws is None:
+        ws = _workspace(need, q.device)
+    if out is None:
+        out = (torch.empty((B, k), dtype=torch.int32, device=q.device),
+               torch.empty((B, k), dtype=torch.float32, device=q.device))
+    idx, val = out
+    sl = torch.empty((B, shortlist), dtype=torch.int32, device=q.device) if want_shortlist else None
+    _check(lib().ls_decode_two_stage_pq_select(_ptr(q), _ptr(w), _ptr(pq_codes), _ptr(pq_books), _ptr(fk),
+                                               _ptr(fk_scale), _ptr(n_valid), B, H, d, N, shortlist, k, _ptr(idx),
+                                               _ptr(val), _ptr(sl), _ptr(ws), ws.numel(), _stream(stream)))
     if want_shortlist:
         return idx, val, sl
     return idx, val

@@ -147,6 +147,22 @@ ls_status make_u8_map(CUtensorMap* m, const void* base, uint64_t rows) {
   return LS_OK;
 }
 
+// 2-D map over [rows][32 bytes] (PQ codes, one key per row), box = 32 bytes x
+// 128 rows, no swizzle; the bytes are described as 16 16-bit elements.
+ls_status make_pq_map(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kPqSub / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kPqSub)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kPqSub / 2), static_cast<cuuint32_t>(kTileKeys)};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LS_OK;
+}
+
 ls_status check_shape(int H, int d) {
   if (H != kHeads || d != kDim)
     return fail(LS_ERR_UNSUPPORTED, "only H=%d, d=%d are built (got H=%d, d=%d)", kHeads, kDim, H, d);
@@ -199,7 +215,7 @@ ls_status score_bf16(const uint16_t* q, const float* w, const uint16_t* keys, co
 ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_total, const float* w,
                         const void* keys, const float* scale, const int32_t* rows, const int32_t* n_valid,
                         int64_t key_rows, int64_t key_stride, int B, int N, int fmt, float* out, cudaStream_t st,
-                        uint32_t* hist = nullptr) {
+                        uint32_t* hist = nullptr, const uint16_t* books = nullptr) {
   if (B == 0 || N == 0) return LS_OK;
   CUtensorMap qmap;
   ls_status s = make_bf16_map(&qmap, q, static_cast<uint64_t>(q_rows_total), kHeads);
@@ -208,6 +224,7 @@ ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_
   p.q = q;
   p.keys = keys;
   p.scale = scale;
+  p.books = books;
   p.rows = rows;
   p.n_valid = n_valid;
   p.w = w;
@@ -228,10 +245,13 @@ ls_status score_convert(const uint16_t* q, int64_t q_row_stride, int64_t q_rows_
   // by 2-D TMA; gathered rows by per-row bulk copies (kmap unused)
   CUtensorMap kmap = qmap;
   if (rows == nullptr) {
-    s = make_u8_map(&kmap, keys, static_cast<uint64_t>(B) * static_cast<uint64_t>(key_stride));
+    const uint64_t nrows = static_cast<uint64_t>(B) * static_cast<uint64_t>(key_stride);
+    s = fmt == SRC_PQ ? make_pq_map(&kmap, keys, nrows) : make_u8_map(&kmap, keys, nrows);
     if (s != LS_OK) return s;
   }
-  ProfScope prof(fmt == SRC_INT8 ? "score_q8_kernel<int8>" : "score_q8_kernel<e4m3>", st);
+  ProfScope prof(fmt == SRC_INT8 ? "score_q8_kernel<int8>" : fmt == SRC_PQ ? "score_q8_kernel<pq>"
+                                                                           : "score_q8_kernel<e4m3>",
+                 st);
   LS_CUDA(launch_score_q8(&qmap, &kmap, p, num_sms_current(), st));
   return LS_OK;
 }
@@ -579,10 +599,13 @@ size_t ls_two_stage_workspace_size(int B, int N, int shortlist) {
          align_up(static_cast<size_t>(B) * kHistBins * sizeof(uint32_t));
 }
 
-ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const int8_t* ck, const float* ck_scale,
-                                     const uint8_t* fk, const float* fk_scale, const int32_t* n_valid, int B,
-                                     int H, int d, int N, int shortlist, int k, int32_t* idx_out, float* val_out,
-                                     int32_t* shortlist_out, void* ws, size_t ws_bytes, void* stream) {
+// The two-stage search over either compact key form: int8 codes + per-key
+// scale (coarse_fmt SRC_INT8) or PQ codes + codebooks (SRC_PQ).
+static ls_status two_stage_run(const uint16_t* q, const float* w, const void* ck, const float* ck_scale,
+                               const uint16_t* books, int coarse_fmt, const uint8_t* fk, const float* fk_scale,
+                               const int32_t* n_valid, int B, int H, int d, int N, int shortlist, int k,
+                               int32_t* idx_out, float* val_out, int32_t* shortlist_out, void* ws, size_t ws_bytes,
+                               void* stream) {
   ls_status s = check_shape(H, d);
   if (s != LS_OK) return s;
   LS_CHECK_ARG(B >= 0 && N >= 0, "negative size");
@@ -598,18 +621,18 @@ ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const in
   float* s_hat = cv.take<float>(static_cast<size_t>(B) * N);
   int32_t* short_ws = cv.take<int32_t>(static_cast<size_t>(B) * shortlist);
   float* exact = cv.take<float>(static_cast<size_t>(B) * shortlist);
-  uint32_t* hist = cv.take<uint32_t>(static_cast<size_t>(B) * kHistBins);
   int32_t* sl = shortlist_out ? shortlist_out : short_ws;
   cudaStream_t st = S(stream);
   if (N > 0) {
-    LS_CHECK_ARG(q && w && ck && ck_scale && fk && fk_scale, "null tensor pointer");
-    LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(ck) && aligned16(fk) && aligned16(ck_scale) &&
-                     aligned16(fk_scale),
+    const bool pq = coarse_fmt == SRC_PQ;
+    LS_CHECK_ARG(q && w && ck && fk && fk_scale && (pq ? books != nullptr : ck_scale != nullptr),
+                 "null tensor pointer");
+    LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(ck) && aligned16(fk) && aligned16(fk_scale) &&
+                     (pq ? aligned16(books) : aligned16(ck_scale)),
                  "tensors must be 16-byte aligned");
-    // coarse pass over compact keys
-    (void)hist;
+    // coarse pass over the compact keys
     s = score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, ck, ck_scale, nullptr, n_valid, N, N, B, N,
-                      SRC_INT8, s_hat, st);
+                      coarse_fmt, s_hat, st, nullptr, books);
     if (s != LS_OK) return s;
   }
   // shortlist: top-S positions by coarse score
@@ -622,6 +645,36 @@ ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const in
     if (s != LS_OK) return s;
   }
   return topk(exact, shortlist, nullptr, sl, shortlist, B, shortlist, k, idx_out, val_out, k, st);
+}
+
+ls_status ls_decode_two_stage_select(const uint16_t* q, const float* w, const int8_t* ck, const float* ck_scale,
+                                     const uint8_t* fk, const float* fk_scale, const int32_t* n_valid, int B,
+                                     int H, int d, int N, int shortlist, int k, int32_t* idx_out, float* val_out,
+                                     int32_t* shortlist_out, void* ws, size_t ws_bytes, void* stream) {
+  return two_stage_run(q, w, ck, ck_scale, nullptr, SRC_INT8, fk, fk_scale, n_valid, B, H, d, N, shortlist, k,
+                       idx_out, val_out, shortlist_out, ws, ws_bytes, stream);
+}
+
+ls_status ls_decode_two_stage_pq_select(const uint16_t* q, const float* w, const uint8_t* pq_codes,
+                                        const uint16_t* pq_books, const uint8_t* fk, const float* fk_scale,
+                                        const int32_t* n_valid, int B, int H, int d, int N, int shortlist, int k,
+                                        int32_t* idx_out, float* val_out, int32_t* shortlist_out, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  return two_stage_run(q, w, pq_codes, nullptr, pq_books, SRC_PQ, fk, fk_scale, n_valid, B, H, d, N, shortlist, k,
+                       idx_out, val_out, shortlist_out, ws, ws_bytes, stream);
+}
+
+ls_status ls_indexer_score_pq(const uint16_t* q, const float* w, const uint8_t* pq_codes, const uint16_t* pq_books,
+                              const int32_t* n_valid, int B, int H, int d, int N, float* scores, void* stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(B >= 0 && N >= 0, "negative size (B=%d N=%d)", B, N);
+  if (B == 0 || N == 0) return LS_OK;
+  LS_CHECK_ARG(q && w && pq_codes && pq_books && scores, "null tensor pointer");
+  LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(pq_codes) && aligned16(pq_books),
+               "q, w, codes and codebooks must be 16-byte aligned");
+  return score_convert(q, kHeads, static_cast<int64_t>(B) * kHeads, w, pq_codes, nullptr, nullptr, n_valid, N, N, B,
+                       N, SRC_PQ, scores, S(stream), nullptr, pq_books);
 }
 
 size_t ls_bucket_workspace_size(int T, int P, int top_p, int budget) {

@@ -60,7 +60,10 @@ cudaError_t launch_score_tc(int qg, const CUtensorMap* kmap, const CUtensorMap* 
                             const ScoreParams& p, int num_sms, cudaStream_t st);
 
 // Source rows for the converting scorer.
-enum SrcFormat : int { SRC_INT8 = 0, SRC_E4M3 = 1, SRC_BF16 = 2 };
+enum SrcFormat : int { SRC_INT8 = 0, SRC_E4M3 = 1, SRC_BF16 = 2, SRC_PQ = 3 };
+// PQ compact keys: kPqSub one-byte codes per key, sub-vector m (dimensions
+// 4m..4m+3) = row code[m] of codebook m; codebooks fp16 [kPqSub][256][4].
+constexpr int kPqSub = 32;
 
 // Scoring of keys that are either int8 / fp8 e4m3 codes with a per-key fp32
 // scale, or gathered bf16 rows.  Row j of problem b is key
@@ -70,7 +73,8 @@ enum SrcFormat : int { SRC_INT8 = 0, SRC_E4M3 = 1, SRC_BF16 = 2 };
 struct CvtParams {
   const uint16_t* q;       // bf16 query rows (problem b, head h: row b*q_row_stride + h)
   const void* keys;        // base of the key rows
-  const float* scale;      // per-key scale, indexed like the key rows (nullptr for bf16)
+  const float* scale;      // per-key scale, indexed like the key rows (nullptr for bf16 / PQ)
+  const uint16_t* books;   // PQ codebooks (fp16 bits, [32][256][4], 16-byte aligned) or nullptr
   const int32_t* rows;     // [B][N] gathered row ids or nullptr
   const int32_t* n_valid;  // [B] or nullptr (contiguous form only)
   const float* w;          // [B][H]

@@ -42,17 +42,19 @@
 
 namespace lsi {
 
-template <int HALVES>
+template <int FMT, int HALVES>
 struct Q8Cfg {
+  static constexpr bool PQ = FMT == SRC_PQ;
   static constexpr int BM = kTileKeys;                  // keys per half (TMEM lanes)
   static constexpr int KPU = HALVES * BM;               // keys per unit
   static constexpr int BN = kHeads;                     // one query per problem
-  static constexpr int ROW = kDim;                      // bytes per 8-bit key row
+  static constexpr int ROW = PQ ? kPqSub : kDim;        // bytes per key row (8-bit codes / PQ codes)
   // gathered rows (HALVES == 1) land at a 144-byte pitch, contiguous ones as
-  // 128-byte rows under the TMA's 128-byte swizzle
+  // 128-byte rows under the TMA's 128-byte swizzle (PQ: 32-byte rows, no
+  // swizzle)
   static constexpr int PITCH = (HALVES == 1) ? ROW + 16 : ROW;
   static constexpr int RAW_BYTES = KPU * PITCH;         // 1024-multiple
-  static constexpr int RS = (HALVES == 1) ? 8 : 6;      // raw stages
+  static constexpr int RS = (HALVES == 1 || PQ) ? 8 : 6;  // raw stages
   static constexpr int AS = 6 / HALVES;                 // widened stages in TMEM
   static constexpr int ACC = 4 / HALVES;                // accumulator stages in TMEM
   static constexpr int A_COLS = HALVES * (kDim / 2);    // two fp16 per 32-bit column
@@ -72,7 +74,8 @@ struct Q8Cfg {
   static constexpr size_t S_BYTES = size_t(KPU) * 8;    // per key: fp32 scale + int flag
   static constexpr size_t SMEM_S = size_t(SS) * S_BYTES;
   static constexpr size_t SMEM_BAR = 1024;
-  static constexpr size_t SMEM_TOTAL = 1024 + SMEM_RAW + SMEM_B + SMEM_S + SMEM_BAR;
+  static constexpr size_t SMEM_CB = PQ ? size_t(kPqSub) * 256 * 8 : 0;  // PQ codebooks, fp16 [32][256][4]
+  static constexpr size_t SMEM_TOTAL = 1024 + SMEM_RAW + SMEM_B + SMEM_S + SMEM_BAR + SMEM_CB;
   static_assert(HALVES == 1 || HALVES == 2, "128- or 256-key units");
   static_assert(RAW_BYTES % 1024 == 0, "swizzled stages need 1024-byte alignment");
   static_assert(A_COL0 + AS * A_COLS <= TMEM_COLS, "TMEM columns");
@@ -93,6 +96,7 @@ struct Q8Barriers {
   uint64_t sfull[32];
   uint64_t sempty[32];
   uint64_t drain;
+  uint64_t cbfull;  // PQ codebooks landed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -113,7 +117,7 @@ __device__ __forceinline__ void q8_wait_drain(uint64_t* bar, uint32_t parity) {
 // fp16 pairs, element 2w in the low half of word w.
 template <int FMT>
 __device__ __forceinline__ void widen16(const uint4& v, uint32_t* o) {
-  if (FMT == SRC_INT8) {
+  if (FMT == SRC_INT8 || FMT == SRC_PQ) {
     i8x4_to_f16x4(v.x, o[0], o[1]);
     i8x4_to_f16x4(v.y, o[2], o[3]);
     i8x4_to_f16x4(v.z, o[4], o[5]);
@@ -127,16 +131,17 @@ __device__ __forceinline__ void widen16(const uint4& v, uint32_t* o) {
 }
 
 template <int FMT, int HALVES>
-__global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
+__global__ void __launch_bounds__(Q8Cfg<FMT, HALVES>::THREADS, 1)
     score_q8_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                     const CvtParams p) {
-  using C = Q8Cfg<HALVES>;
+  using C = Q8Cfg<FMT, HALVES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sR = smem;
   uint8_t* sB = sR + C::SMEM_RAW;
   uint8_t* sS = sB + C::SMEM_B;
   Q8Barriers* bars = reinterpret_cast<Q8Barriers*>(sS + C::SMEM_S);
+  uint8_t* sCB = sS + C::SMEM_S + C::SMEM_BAR;  // PQ codebooks
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -169,6 +174,7 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
       mbar_init(&bars->sempty[s], C::EPI_WARPS);
     }
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->cbfull, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
   }
@@ -179,6 +185,10 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&qmap);
     if (!gathered) tma_prefetch_desc(&kmap);
+  }
+  if (C::PQ && threadIdx.x == 0) {  // barrier init by this same thread above; the codebooks once per CTA
+    mbar_arrive_expect_tx(&bars->cbfull, static_cast<uint32_t>(C::SMEM_CB));
+    bulk_load(sCB, p.books, static_cast<uint32_t>(C::SMEM_CB), &bars->cbfull);
   }
   tc_fence_before();
   __syncthreads();
@@ -251,7 +261,8 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
           const int r = lane + 32 * i;
           const bool valid = j0 + r < nvb;
           sok[r] = valid ? 1 : 0;
-          if (valid) cp_async_4(ssc + r, p.scale + static_cast<int64_t>(b) * p.N + j0 + r);
+          if (C::PQ) ssc[r] = 1.f;  // PQ keys carry no scale
+          else if (valid) cp_async_4(ssc + r, p.scale + static_cast<int64_t>(b) * p.N + j0 + r);
         }
       } else {
         // lane l holds the row ids of rows l, l+32, l+64, l+96 (the next
@@ -362,7 +373,9 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
     const int row = qd * 32 + lane;
     const uint32_t t_row = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + C::A_COL0;
     const long long count = u_end - u_begin;
-    for (long long i = cg; i < count; i += C::CVT_GROUPS) {
+    bool cb_ok = true;
+    if (C::PQ) cb_ok = warp_wait(&bars->cbfull, 0, abort_flag);
+    for (long long i = cg; i < count && cb_ok; i += C::CVT_GROUPS) {
       const int rs = static_cast<int>(i % C::RS), as = static_cast<int>(i % C::AS);
       const uint32_t rphase = static_cast<uint32_t>((i / C::RS) & 1), aphase = static_cast<uint32_t>((i / C::AS) & 1);
       if (!warp_wait(&bars->rfull[rs], rphase, abort_flag)) break;
@@ -375,6 +388,25 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
 #pragma unroll
       for (int h = 0; h < HALVES; ++h) {
         const uint8_t* rowp = raw + (h * C::BM + row) * C::PITCH;
+        if (C::PQ) {
+          // 32 codes; sub-vector m is row code[m] of codebook m (4 fp16 = 8 bytes)
+          const uint2* cb = reinterpret_cast<const uint2*>(sCB);
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const uint4 cw = *reinterpret_cast<const uint4*>(rowp + part * 16);
+            const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+            uint32_t o[32];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const uint32_t code = (w4[c >> 2] >> (8 * (c & 3))) & 0xffu;
+              const uint2 e = cb[(part * 16 + c) * 256 + code];
+              o[2 * c] = e.x;
+              o[2 * c + 1] = e.y;
+            }
+            tmem_st_32x32(t_row + as * C::A_COLS + h * (kDim / 2) + part * 32, o);
+          }
+          continue;
+        }
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           uint4 v[4];
@@ -466,7 +498,7 @@ __global__ void __launch_bounds__(Q8Cfg<HALVES>::THREADS, 1)
 template <int FMT, int HALVES>
 static cudaError_t launch_q8(const CUtensorMap* qmap, const CUtensorMap* kmap, const CvtParams& p, int num_sms,
                              cudaStream_t st) {
-  using C = Q8Cfg<HALVES>;
+  using C = Q8Cfg<FMT, HALVES>;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(score_q8_kernel<FMT, HALVES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -493,6 +525,8 @@ cudaError_t launch_score_q8(const CUtensorMap* qmap, const CUtensorMap* kmap, co
     case SRC_E4M3:
       return gathered ? launch_q8<SRC_E4M3, 1>(qmap, kmap, p, num_sms, st)
                       : launch_q8<SRC_E4M3, 2>(qmap, kmap, p, num_sms, st);
+    case SRC_PQ:  // contiguous only
+      return gathered ? cudaErrorInvalidValue : launch_q8<SRC_PQ, 2>(qmap, kmap, p, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }

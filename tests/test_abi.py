@@ -79,6 +79,12 @@ def test_argument_checks_without_gpu(lib):
     st = lib.ls_decode_two_stage_select(dummy, dummy, dummy, dummy, dummy, dummy, None, 1, 32, 128, 100, 256, 512,
                                         dummy, None, None, dummy, 1 << 30, None)
     assert st == 1
+    # PQ two-stage: shortlist shorter than k; PQ scores: null codebooks, H != 32
+    st = lib.ls_decode_two_stage_pq_select(dummy, dummy, dummy, dummy, dummy, dummy, None, 1, 32, 128, 100, 256, 512,
+                                           dummy, None, None, dummy, 1 << 30, None)
+    assert st == 1
+    assert lib.ls_indexer_score_pq(dummy, dummy, dummy, None, None, 1, 32, 128, 64, dummy, None) == 1
+    assert lib.ls_indexer_score_pq(dummy, dummy, dummy, dummy, None, 1, 16, 128, 64, dummy, None) == 3
     # bucket: budget below k
     st = lib.ls_bucket_select(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 128, 10, 80, 4, 100, 512, dummy,
                               None, None, dummy, 1 << 30, None)

@@ -11,9 +11,11 @@ import numpy as np
 import pytest
 import torch
 
-from oracle.formats import bf16_to_f64, dequant
+from oracle.formats import bf16_to_f64, dequant, pq_decode
 from oracle.indexer import eligible_count, indexer_scores
-from oracle.select import bucket_select, expand_buckets, recall_at_k, select_topk, topk_rows, two_stage_select
+from oracle.select import (
+    bucket_select, expand_buckets, recall_at_k, select_topk, topk_rows, two_stage_pq_select, two_stage_select,
+)
 from parity_util import (
     RTOL_BF16, RTOL_FP8, check_scores, check_selection, check_set, dev, dev_bf16, dev_e4m3, f32_bits_equal,
 )
@@ -278,12 +280,20 @@ def _check_two_stage(L, name, rows):
     wl = get_workload(name)
     d = data(name)
     q, w = dev_bf16(d["q"]), dev(d["w"])
-    idx, val, sl = L.ls_decode_two_stage_select(q, w, dev(d["ck"]), dev(d["ck_scale"]), dev_e4m3(d["fk"]),
-                                                dev(d["fk_scale"]), dev(d["n_valid"]), shortlist=wl.shortlist,
-                                                k=wl.k, want_shortlist=True)
+    if wl.extra.get("pq"):
+        books = torch.from_numpy(d["pq_books"].view(np.int16)).view(torch.float16).cuda()
+        idx, val, sl = L.ls_decode_two_stage_pq_select(q, w, dev(d["pq_codes"]), books, dev_e4m3(d["fk"]),
+                                                       dev(d["fk_scale"]), dev(d["n_valid"]), shortlist=wl.shortlist,
+                                                       k=wl.k, want_shortlist=True)
+        _, _, det = two_stage_pq_select(d["q"], d["w"], d["pq_codes"], d["pq_books"], d["fk"], d["fk_scale"],
+                                        d["n_valid"], wl.shortlist, wl.k, rows=rows, return_detail=True)
+    else:
+        idx, val, sl = L.ls_decode_two_stage_select(q, w, dev(d["ck"]), dev(d["ck_scale"]), dev_e4m3(d["fk"]),
+                                                    dev(d["fk_scale"]), dev(d["n_valid"]), shortlist=wl.shortlist,
+                                                    k=wl.k, want_shortlist=True)
+        _, _, det = two_stage_select(d["q"], d["w"], d["ck"], d["ck_scale"], d["fk"], d["fk_scale"], d["n_valid"],
+                                     wl.shortlist, wl.k, rows=rows, return_detail=True)
     idx, val, sl = idx.cpu().numpy(), val.cpu().numpy(), sl.cpu().numpy()
-    _, _, det = two_stage_select(d["q"], d["w"], d["ck"], d["ck_scale"], d["fk"], d["fk_scale"], d["n_valid"],
-                                 wl.shortlist, wl.k, rows=rows, return_detail=True)
     recalls = []
     for i, b in enumerate(rows):
         n = int(d["n_valid"][b])
@@ -312,6 +322,31 @@ def test_two_stage_small(L):
 @pytest.mark.slow
 def test_two_stage_full_size_sampled(L):
     rec = _check_two_stage(L, "two_stage", [0, 17, 31])
+    assert min(rec) > 0.5
+
+
+def test_pq_scores(L):
+    wl = get_workload("two_stage_pq_s")
+    d = data("two_stage_pq_s")
+    books = torch.from_numpy(d["pq_books"].view(np.int16)).view(torch.float16).cuda()
+    sc = L.ls_indexer_score_pq(dev_bf16(d["q"]), dev(d["w"]), dev(d["pq_codes"]), books,
+                               n_valid=dev(d["n_valid"])).cpu().numpy()
+    for b in range(wl.B):
+        n = int(d["n_valid"][b])
+        ref = indexer_scores(bf16_to_f64(d["q"][b])[None], d["w"][b].astype(np.float64)[None],
+                             pq_decode(d["pq_codes"][b, :n], d["pq_books"]))[0]
+        check_scores(sc[b, :n], ref, RTOL_BF16, f"pq row {b}")
+        assert np.all(np.isneginf(sc[b, n:]))
+
+
+def test_two_stage_pq_small(L):
+    rec = _check_two_stage(L, "two_stage_pq_s", [0, 1, 2])
+    assert min(rec) > 0.5
+
+
+@pytest.mark.slow
+def test_two_stage_pq_full_size_sampled(L):
+    rec = _check_two_stage(L, "two_stage_pq", [0, 17, 31])
     assert min(rec) > 0.5
 
 
