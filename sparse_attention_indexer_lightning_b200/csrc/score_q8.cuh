@@ -405,17 +405,17 @@ __global__ void __launch_bounds__(Q8Cfg<FMT, HALVES>::THREADS, 1)
             }
             tmem_st_32x32(t_row + as * C::A_COLS + h * (kDim / 2) + part * 32, o);
           }
-          continue;
-        }
+        } else {
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          uint4 v[4];
+          for (int part = 0; part < 2; ++part) {
+            uint4 v[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(rowp + (((part * 4 + c) ^ sw) << 4));
-          uint32_t o[32];
+            for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(rowp + (((part * 4 + c) ^ sw) << 4));
+            uint32_t o[32];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) widen16<FMT>(v[c], o + 8 * c);
-          tmem_st_32x32(t_row + as * C::A_COLS + h * (kDim / 2) + part * 32, o);
+            for (int c = 0; c < 4; ++c) widen16<FMT>(v[c], o + 8 * c);
+            tmem_st_32x32(t_row + as * C::A_COLS + h * (kDim / 2) + part * 32, o);
+          }
         }
       }
       tmem_wait_st();
