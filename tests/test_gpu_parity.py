@@ -256,6 +256,26 @@ def test_prefill_stream_overflow(L):
     assert np.array_equal(ri.cpu().numpy(), idx) and f32_bits_equal(rv.cpu().numpy(), val)
 
 
+@pytest.mark.parametrize("T,N,tile,k", [(1, 2000, 256, 64), (40, 2000, 256, 1100), (9, 300, 512, 32)])
+def test_prefill_stream_shapes(L, T, N, tile, k):
+    """One query (the one-query scorer's filter form), k above 1024 (the wide
+    top-k and 5k-entry merge rows) and a history shorter than one tile: the
+    running form, the full-matrix form and the oracle agree."""
+    from types import SimpleNamespace
+    from workloads.synth import make_prefill
+    d = make_prefill(T, N, 4 * N - T - 37, seed=31)
+    wl = SimpleNamespace(k=k, stride=4, tile_keys=tile)
+    _, _, _, idx, val = _prefill_run(L, d, wl)
+    *_, idx2, val2 = _prefill_run(L, d, wl, full_scores=True)
+    assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
+    n_t = eligible_count(d["q_pos"], 4, N)
+    keys = bf16_to_f64(d["k"])
+    for t in range(T):
+        n = int(n_t[t])
+        ref = indexer_scores(bf16_to_f64(d["q"][t])[None], d["w"][t].astype(np.float64)[None], keys[:n])[0]
+        check_selection(idx[t], val[t], np.arange(n), ref, k, RTOL_BF16, f"shape ({T},{N},{tile},{k}) t={t}")
+
+
 @pytest.mark.slow
 def test_prefill_chunk_full_size_sampled(L):
     wl = get_workload("prefill_chunk")
