@@ -39,17 +39,17 @@
 
 namespace lsi {
 
-constexpr int kCandCap = 8192;     // listed candidates kept in shared memory
+constexpr int kCandCap = 8192;     // listed candidates kept in shared memory (the wide forms)
 constexpr int kExactHistMax = 2048; // rows up to this length get an exact histogram; longer rows
                                     // sample about this many entries
 constexpr int kVec = 4;            // float4 loads per thread per chunk
 constexpr int kChunk = kVec * 4;   // entries per thread per chunk
 
 // NT threads per CTA (one row each), KMAX the largest k the CTA holds.
-template <int NT, int KMAX>
+template <int NT, int KMAX, int CAP>
 struct TopkShared {
-  float cand_val[kCandCap];            // listed entries: value and label
-  int32_t cand_lab[kCandCap];
+  float cand_val[CAP];                 // listed entries: value and label
+  int32_t cand_lab[CAP];
   unsigned long long sel_key[KMAX];    // the k selected: packed key and value
   unsigned long long tmp_key[KMAX];    // bucketed copy for the final order
   float sel_val[KMAX];                 // (sel_key + tmp_key and sel_val + tmp_val are also
@@ -494,10 +494,13 @@ __device__ unsigned long long radix_select_cand(SH& sh, int nc, uint32_t want) {
   return prefix;
 }
 
-template <int NT, int KMAX>
-__global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p) {
+// NT threads, largest k KMAX, CAP listed candidates: <1024, 4096, 8192> one
+// CTA per SM; <512, 1024, 8192> two; <256, 512, 2048> four (rows of many
+// queries with k <= 512: more rows in flight hide the per-row latency).
+template <int NT, int KMAX, int CAP>
+__global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
-  TopkShared<NT, KMAX>& sh = *reinterpret_cast<TopkShared<NT, KMAX>*>(topk_smem);
+  TopkShared<NT, KMAX, CAP>& sh = *reinterpret_cast<TopkShared<NT, KMAX, CAP>*>(topk_smem);
   const int r = blockIdx.x;
   if (p.run_if != nullptr && *p.run_if == 0) return;      // conditional launch with nothing to do
   if (p.row_flag != nullptr && p.row_flag[r] == 0) return;  // row left untouched
@@ -581,16 +584,16 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
       // ---- listing pass: every present entry in a bin >= blo -------------
       if (blo >= 4) {  // bins from 4 up start at finite values: compare the score itself
         const float tlo = code_floor_value(blo << (32 - kHistBits));
-        list_row<NT>(rr, [&](float v, int32_t) { return v >= tlo; }, sh.cand_val, sh.cand_lab, &sh.ccnt, kCandCap);
+        list_row<NT>(rr, [&](float v, int32_t) { return v >= tlo; }, sh.cand_val, sh.cand_lab, &sh.ccnt, CAP);
       } else {
         list_row<NT>(rr, [&](float v, int32_t) { return hist_bin(order_code(v)) >= blo; }, sh.cand_val, sh.cand_lab,
-                 &sh.ccnt, kCandCap);
+                 &sh.ccnt, CAP);
       }
       __syncthreads();
       const uint32_t listed = sh.ccnt;
       // entries to select: exact when the histogram counted every present entry
       kk = static_cast<int>(exact_hist ? min(kcap, hist_total) : kcap);
-      if (listed > static_cast<uint32_t>(kCandCap) || listed < static_cast<uint32_t>(kk)) plain = true;
+      if (listed > static_cast<uint32_t>(CAP) || listed < static_cast<uint32_t>(kk)) plain = true;
     }
   }
 
@@ -619,14 +622,14 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
       thr = radix_select_row<NT>(sh, rr, static_cast<uint32_t>(kk));
       // exactly kk entries pass: they become the candidate list
       list_row<NT>(rr, [&](float v, int32_t lb) { return pack_key(v, lb) >= thr; }, sh.cand_val, sh.cand_lab, &sh.ccnt,
-               kCandCap);
+               CAP);
     }
     __syncthreads();
   }
   int32_t* io = p.idx_out + static_cast<int64_t>(r) * p.ld_out;
   float* vo = p.val_out ? p.val_out + static_cast<int64_t>(r) * p.ld_out : nullptr;
   const int lab_add = rr.lab ? 0 : p.label_base;
-  const int nc_all = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(kCandCap)));
+  const int nc_all = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(CAP)));
   // ---- 4'. bucket select: selection and canonical order in one pass -------
   // The candidates are bucketed by their position in the [min, max] key range
   // (2048 bins); the bins from the top hold the k largest keys up to the
@@ -824,17 +827,17 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_kernel(const TopkParams p)
   }
 }
 
-template <int NT, int KMAX>
+template <int NT, int KMAX, int CAP>
 static cudaError_t launch_topk_t(const TopkParams& p, cudaStream_t st) {
-  using SH = TopkShared<NT, KMAX>;
+  using SH = TopkShared<NT, KMAX, CAP>;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel<NT, KMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel<NT, KMAX, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(SH)));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  topk_kernel<NT, KMAX><<<p.R, NT, sizeof(SH), st>>>(p);
+  topk_kernel<NT, KMAX, CAP><<<p.R, NT, sizeof(SH), st>>>(p);
   return cudaGetLastError();
 }
 
@@ -843,8 +846,9 @@ static cudaError_t launch_topk_t(const TopkParams& p, cudaStream_t st) {
 // 1024-thread CTA per row.
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t st, int num_sms) {
   if (p.R == 0) return cudaSuccess;
-  if (p.k <= 1024 && p.R > num_sms) return launch_topk_t<512, 1024>(p, st);
-  return launch_topk_t<1024, kMaxTopK>(p, st);
+  if (p.k <= 512 && p.R >= 2 * num_sms) return launch_topk_t<256, 512, 2048>(p, st);
+  if (p.k <= 1024 && p.R > num_sms) return launch_topk_t<512, 1024, kCandCap>(p, st);
+  return launch_topk_t<1024, kMaxTopK, kCandCap>(p, st);
 }
 
 }  // namespace lsi

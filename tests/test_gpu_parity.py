@@ -67,10 +67,10 @@ def _adversarial_rows(rng, R, N):
     return s
 
 
-# the last three shapes have more rows than SMs: the two-CTAs-per-SM form
+# the last four shapes have more rows than SMs: the two- and four-CTAs-per-SM forms
 @pytest.mark.parametrize("R,N,k", [(7, 3000, 512), (6, 517, 512), (6, 40000, 4096), (3, 131072, 4096),
                                    (8, 1000, 1), (6, 129, 64), (300, 3000, 512), (300, 20000, 1024),
-                                   (160, 9000, 64)])
+                                   (160, 9000, 64), (400, 40000, 256)])
 def test_topk_bit_exact(L, R, N, k):
     rng = np.random.default_rng(100 + N)
     s = _adversarial_rows(rng, R, N)
