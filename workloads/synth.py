@@ -72,8 +72,8 @@ PQ_M, PQ_K, PQ_SUB = 32, 256, 4
 def train_pq_books(x: np.ndarray, rng: np.random.Generator, iters: int = 10) -> np.ndarray:
     """Lloyd k-means per sub-space on the rows of x [n, 128], centroids seeded
     from sample rows (distinct when n >= 256; one draw per sub-space), empty
-    clusters keeping
-    their centroid; assignments by fp32 squared distance, means in fp64.
+    clusters keeping their centroid; assignments by fp32 squared distance,
+    means in fp64.
     Returns the codebooks rounded to fp16, as bit patterns [32][256][4]."""
     n = x.shape[0]
     xs = np.ascontiguousarray(np.asarray(x, dtype=np.float64).reshape(n, PQ_M, PQ_SUB).transpose(1, 0, 2))
