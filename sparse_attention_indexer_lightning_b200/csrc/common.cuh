@@ -438,65 +438,84 @@ struct UnitPos {
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
-// d += a * b on a pair of fp32 lanes (packed fp32x2 FMA of sm_100a).
-__device__ __forceinline__ void ffma2_acc(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mov.b64 rd, {%0, %1};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+// Two fp32 lanes packed in one 64-bit register pair (the operand form of the
+// packed fp32x2 arithmetic of sm_100a).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
 }
 
-// ReLU on the FMA pipe: x + |x| is 2 * max(x, 0) exactly (one FADD with an
-// absolute-value operand), where fmaxf would issue on the busier ALU pipe.
-// The factor 2 is taken out once per key at the end (a power of two, so the
-// result is bit-identical to summing w * max(x, 0)).
-__device__ __forceinline__ float relu2(float x) { return x + fabsf(x); }
-
-// Weighted-ReLU head reduction of one key's 32 head dot products:
-//   sum_h w[h] * max(0, scale * v[h])
-// with 8 independent partial sums updated two at a time by packed FMAs (a
-// single running sum would serialise 32 dependent FMAs).  w must be 16-byte
-// aligned.
-template <bool SCALED>
-__device__ __forceinline__ float head_reduce(const float (&v)[32], const float* __restrict__ w, float scale) {
-  const float4* w4 = reinterpret_cast<const float4*>(w);
-  float4 wv[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) wv[i] = __ldg(w4 + i);
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float a0 = relu2(SCALED ? scale * v[4 * i + 0] : v[4 * i + 0]);
-    const float a1 = relu2(SCALED ? scale * v[4 * i + 1] : v[4 * i + 1]);
-    const float a2 = relu2(SCALED ? scale * v[4 * i + 2] : v[4 * i + 2]);
-    const float a3 = relu2(SCALED ? scale * v[4 * i + 3] : v[4 * i + 3]);
-    const int p = (2 * i) & 7;
-    ffma2_acc(acc[p], acc[p + 1], a0, a1, wv[i].x, wv[i].y);
-    const int q = (2 * i + 2) & 7;
-    ffma2_acc(acc[q], acc[q + 1], a2, a3, wv[i].z, wv[i].w);
-  }
-  return 0.5f * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 
-// head_reduce with the 32 head weights already in registers.
-__device__ __forceinline__ float head_reduce_w(const uint32_t (&r)[32], const float (&w)[32]) {
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+// acc += (x + |x|) * w on a pair of lanes.  x + |x| is 2 * max(x, 0) exactly
+// (one FADD with an absolute-value operand, on the FMA pipe); the factor 2 is
+// taken out once per key at the end (a power of two, so nothing is lost).
+// The two ReLU results are produced straight into the register pair the
+// packed FMA reads, and the accumulator and weights stay packed throughout,
+// so no register moves are needed between the steps.
+__device__ __forceinline__ void relu2_fma2(uint64_t& acc, uint32_t x0, uint32_t x1, uint64_t w) {
+  asm("{\n\t.reg .f32 a0, a1, t0, t1;\n\t.reg .b64 ra;\n\t"
+      "mov.b32 t0, %1;\n\t"
+      "mov.b32 t1, %2;\n\t"
+      "abs.f32 a0, t0;\n\t"
+      "abs.f32 a1, t1;\n\t"
+      "add.f32 a0, t0, a0;\n\t"
+      "add.f32 a1, t1, a1;\n\t"
+      "mov.b64 ra, {a0, a1};\n\t"
+      "fma.rn.f32x2 %0, ra, %3, %0;\n\t}"
+      : "+l"(acc)
+      : "r"(x0), "r"(x1), "l"(w));
+}
+
+// Sum of four packed partial sums, halved (see relu2_fma2).
+__device__ __forceinline__ float finish_pairs(const uint64_t (&acc)[4]) {
+  uint64_t s01, s23, s;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(s01) : "l"(acc[0]), "l"(acc[1]));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(s23) : "l"(acc[2]), "l"(acc[3]));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(s) : "l"(s01), "l"(s23));
+  float lo, hi;
+  unpack_f32x2(s, lo, hi);
+  return 0.5f * (lo + hi);
+}
+
+// The 32 head weights of one query as 16 packed pairs.
+struct HeadWeights {
+  uint64_t v[16];
+  __device__ __forceinline__ void load(const float* __restrict__ w) {  // 16-byte aligned
+    const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(w);
 #pragma unroll
-  for (int h = 0; h < 32; h += 2) {
-    const int p = h & 7;
-    ffma2_acc(acc[p], acc[p + 1], relu2(__uint_as_float(r[h])), relu2(__uint_as_float(r[h + 1])), w[h], w[h + 1]);
+    for (int i = 0; i < 8; ++i) {
+      const ulonglong2 t = __ldg(w2 + i);
+      v[2 * i] = t.x;
+      v[2 * i + 1] = t.y;
+    }
   }
-  return 0.5f * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+};
+
+// Weighted-ReLU head reduction of one key's 32 head dot products r (fp32 bit
+// patterns, one TMEM row):  sum_h w[h] * max(0, r[h]),  with four independent
+// packed partial sums (a single running sum would serialise 16 dependent FMAs).
+__device__ __forceinline__ float head_reduce_w(const uint32_t (&r)[32], const HeadWeights& w) {
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int h = 0; h < 32; h += 2) relu2_fma2(acc[(h >> 1) & 3], r[h], r[h + 1], w.v[h >> 1]);
+  return finish_pairs(acc);
+}
+
+// The same with the weights read from global memory (16-byte aligned).
+__device__ __forceinline__ float head_reduce(const uint32_t (&r)[32], const float* __restrict__ w) {
+  HeadWeights hw;
+  hw.load(w);
+  return head_reduce_w(r, hw);
 }
 
 // sum_h w[h] * max(0, sc * v[h]) for a per-key scale sc of either sign:
 // = |sc| * sum_h w[h] * max(0, sign(sc) * v[h]).  The sign is uniform across a
 // warp in practice (scales are magnitudes), so the branch does not diverge.
-__device__ __forceinline__ float head_reduce_scaled(const uint32_t (&r)[32], const float (&w)[32], float sc) {
+__device__ __forceinline__ float head_reduce_scaled(const uint32_t (&r)[32], const HeadWeights& w, float sc) {
   float base;
   if (sc >= 0.f) {
     base = head_reduce_w(r, w);

@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     up.init(u_begin, NT, 1);
     if (u_begin < u_end) fetch(up.b, up.tile, nvalid, nsc);
     int w_b = -1;
-    float wreg[32];
+    HeadWeights wreg;
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
       const int tile = up.tile;
       const int b = up.b;
@@ -455,17 +455,10 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
           const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.q_row_stride + lane) * kDim;
           const float wl = __ldg(p.w + static_cast<int64_t>(b) * kHeads + lane) * exp2i(-q_head_shift_global(qrow));
 #pragma unroll
-          for (int i = 0; i < 32; ++i) wreg[i] = __shfl_sync(0xffffffffu, wl, i);
+          for (int i = 0; i < 16; ++i)
+            wreg.v[i] = pack_f32x2(__shfl_sync(0xffffffffu, wl, 2 * i), __shfl_sync(0xffffffffu, wl, 2 * i + 1));
         } else {
-          const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * kHeads);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 t4 = __ldg(w4 + i);
-            wreg[4 * i] = t4.x;
-            wreg[4 * i + 1] = t4.y;
-            wreg[4 * i + 2] = t4.z;
-            wreg[4 * i + 3] = t4.w;
-          }
+          wreg.load(p.w + static_cast<int64_t>(b) * kHeads);
         }
         w_b = b;
       }

@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(Q8Cfg<FMT, HALVES>::THREADS, 1)
     int acc = 0, ss = 0;
     uint32_t acc_phase = 0, sphase = 0;
     int w_b = -1;
-    float wreg[32];
+    HeadWeights wreg;
     UnitPos up;
     up.init(u_begin, NT, 1);
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, 1)) {
@@ -444,7 +444,8 @@ __global__ void __launch_bounds__(Q8Cfg<FMT, HALVES>::THREADS, 1)
         const uint16_t* qrow = p.q + (static_cast<int64_t>(b) * p.q_row_stride + lane) * kDim;
         const float wl = __ldg(p.w + static_cast<int64_t>(b) * kHeads + lane) * exp2i(-q_head_shift_global(qrow));
 #pragma unroll
-        for (int h = 0; h < 32; ++h) wreg[h] = __shfl_sync(0xffffffffu, wl, h);
+        for (int i = 0; i < 16; ++i)
+          wreg.v[i] = pack_f32x2(__shfl_sync(0xffffffffu, wl, 2 * i), __shfl_sync(0xffffffffu, wl, 2 * i + 1));
         w_b = b;
       }
       if (!warp_wait(&bars->sfull[ss], sphase, abort_flag)) break;

@@ -279,13 +279,15 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
     const int qset = ew >> 2;                 // which share of the group's queries
     int acc = 0;
     uint32_t acc_phase = 0;
-    long long w_row = -1;                     // QG == 1: row whose weights sit in wreg
-    float wreg[32];
-    long long lim_bg = -1;                    // group whose per-query limits sit in elig / thr
-    int elig[C::Q_PER_EPI_WARP];
+    HeadWeights wreg;                         // QG == 1: the group's one query's weights
+    // Per-query data of the current group, derived once when the group changes
+    // (consecutive units of a CTA walk the key tiles of one group):
+    int limq[C::Q_PER_EPI_WARP];              // keys of this launch the query may see (<= N)
+    float* orow[C::Q_PER_EPI_WARP];           // storing form: the query's row at this launch's key 0
+    const float* wq[C::Q_PER_EPI_WARP];       // QG > 1: the query's head weights
     uint32_t thr[C::Q_PER_EPI_WARP];          // filter form: order code a key must reach
 #pragma unroll
-    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) elig[i] = 0, thr[i] = 0;
+    for (int i = 0; i < C::Q_PER_EPI_WARP; ++i) limq[i] = 0, orow[i] = nullptr, wq[i] = nullptr, thr[i] = 0;
     constexpr bool filter = FILTER;
     // Filter form: each warp stages its queries' candidates in shared memory
     // and reserves global slots for a whole batch with one atomic.
@@ -323,28 +325,45 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
     };
     UnitPos up;
     up.init(u_begin, NT, G);
+    int nq = 0;                                            // queries of this warp in the current group
+    int hb = 0;                                            // problem of the current group
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
-      const int tile = up.tile, g = up.g, b = up.b;
-      const long long bg = static_cast<long long>(b) * G + g;
-      if (filter && bg != lim_bg) flush_all();             // staged entries belong to the previous group
+      const int tile = up.tile;
       const int n = tile * C::BM + quad * 32 + lane;       // key within this launch
-      int lim = p.N;
-      if (p.n_valid) lim = min(lim, __ldg(p.n_valid + b));
-      // queries of this warp in the group: its share of the QG columns blocks,
-      // cut by the group size and by the last group's end
-      int nq = min(p.T - g * QG, QG) - qset * C::Q_PER_EPI_WARP;
-      nq = nq < 0 ? 0 : (nq > C::Q_PER_EPI_WARP ? C::Q_PER_EPI_WARP : nq);
-      if (QG == 1 && w_row != bg) {                        // one query per sequence: weights per row
-        const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(b) * p.T * kHeads);
+      if (u == u_begin || tile == 0) {                     // units run (b, g, tile): a new group
+        const int g = up.g, b = up.b;
+        hb = b;
+        if (filter) flush_all();                           // staged entries belong to the previous group
+        // this warp's share of the QG columns blocks, cut by the group size
+        // and by the last group's end
+        nq = min(p.T - g * QG, QG) - qset * C::Q_PER_EPI_WARP;
+        nq = nq < 0 ? 0 : (nq > C::Q_PER_EPI_WARP ? C::Q_PER_EPI_WARP : nq);
+        int lim = p.N;
+        if (p.n_valid) lim = min(lim, __ldg(p.n_valid + b));
+        if (QG == 1) wreg.load(p.w + (static_cast<int64_t>(b) * p.T + g) * kHeads);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 t4 = __ldg(w4 + i);
-          wreg[4 * i] = t4.x;
-          wreg[4 * i + 1] = t4.y;
-          wreg[4 * i + 2] = t4.z;
-          wreg[4 * i + 3] = t4.w;
+        for (int jq = 0; jq < C::Q_PER_EPI_WARP; ++jq) {
+          if (jq < nq) {
+            const int t = g * QG + qset * C::Q_PER_EPI_WARP + jq;
+            const int64_t row = static_cast<int64_t>(b) * p.T + t;
+            int lt = lim;
+            if (p.lim_rows || p.q_pos) {
+              // eligible keys of this query (whole history), relative to this launch
+              const int rel = eligible_keys(p, b, t) - p.key_base;
+              lt = rel < 0 ? 0 : (rel < lt ? rel : lt);
+            }
+            limq[jq] = lt;
+            wq[jq] = p.w + row * kHeads;
+            if (!filter) {
+              orow[jq] = p.out + row * p.ld_out + p.out_col0;
+            } else {
+              // the row's running k-th entry; a list with padding takes every eligible key
+              const int64_t kth = row * p.ld_cand + p.run_k - 1;
+              thr[jq] = (p.cand_lab[kth] < 0) ? 0u : order_code(p.cand_val[kth]) + 1u;
+              frow[jq] = row;
+            }
+          }
         }
-        w_row = bg;
       }
       if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
@@ -359,7 +378,6 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
 #pragma unroll
       for (int jq = 0; jq < C::Q_PER_EPI_WARP; ++jq) {
         if (jq < nq) {                                     // warp-uniform
-          const int t = g * QG + qset * C::Q_PER_EPI_WARP + jq;
           tmem_ld_32x32_nowait(tbase + static_cast<uint32_t>(jq * kHeads), cur);
           tmem_wait_ld(cur);
           if (jq + 1 == nq) {                              // the unit's last load is in: release
@@ -367,39 +385,16 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->tempty[acc]);
           }
-          float s;
-          if (QG == 1) {
-            s = head_reduce_w(cur, wreg);
-          } else {
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]);
-            s = head_reduce<false>(v, p.w + (static_cast<int64_t>(b) * p.T + t) * kHeads, 1.f);
-          }
-          int lim_t = lim;
-          if (p.lim_rows || p.q_pos) {
-            // eligible keys of this query (whole history), re-derived only when
-            // the query group changes
-            if (lim_bg != bg) elig[jq] = eligible_keys(p, b, t);
-            const int rel = elig[jq] - p.key_base;
-            lim_t = rel < 0 ? 0 : (rel < lim_t ? rel : lim_t);
-          }
+          const float s = (QG == 1) ? head_reduce_w(cur, wreg) : head_reduce(cur, wq[jq]);
           if (!filter) {
             if (n < p.N) {
-              p.out[(static_cast<int64_t>(b) * p.T + t) * p.ld_out + p.out_col0 + n] = (n < lim_t) ? s : neg_inf();
-              if (use_hist && n < lim_t) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
+              orow[jq][n] = (n < limq[jq]) ? s : neg_inf();
+              if (use_hist && n < limq[jq]) atomicAdd(&shist[hist_bin(order_code(s))], 1u);
             }
           } else {
-            const int64_t row = static_cast<int64_t>(b) * p.T + t;
-            if (lim_bg != bg) {
-              // the row's running k-th entry; a list with padding takes every eligible key
-              const int64_t kth = row * p.ld_cand + p.run_k - 1;
-              thr[jq] = (p.cand_lab[kth] < 0) ? 0u : order_code(p.cand_val[kth]) + 1u;
-            }
-            const bool take = (n < p.N) && (n < lim_t) && order_code(s) >= thr[jq];
+            const bool take = (n < limq[jq]) && order_code(s) >= thr[jq];
             const uint32_t bal = __ballot_sync(0xffffffffu, take);
             if (bal) {
-              frow[jq] = row;
               const uint32_t add = static_cast<uint32_t>(__popc(bal));
               if (fcnt[jq] + add > static_cast<uint32_t>(C::SBUF)) flush_q(jq);
               if (take) {
@@ -413,12 +408,11 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
           }
         }
       }
-      lim_bg = bg;
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
       if (use_hist && (u + 1 == u_end || tile + 1 == NT)) {
         // the row (one query per sequence here) ends in this CTA: publish its counts
         role_barrier(1, C::EPI_WARPS * 32);
-        flush_hist(shist, p.hist + static_cast<int64_t>(b) * p.T * kHistBins, ew * 32 + lane, C::EPI_WARPS * 32);
+        flush_hist(shist, p.hist + static_cast<int64_t>(hb) * p.T * kHistBins, ew * 32 + lane, C::EPI_WARPS * 32);
         role_barrier(1, C::EPI_WARPS * 32);
       }
     }
