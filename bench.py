@@ -336,6 +336,8 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
     res = {}
     for name, fn in (("prefill_chunk", bench_prefill),
                      ("prefill_chunk_running", lambda *a: bench_prefill(*a, full_scores=False)),
+                     ("prefill_chunk_fp8", lambda *a: bench_prefill(*a, fp8=True)),
+                     ("prefill_chunk_fp8_running", lambda *a: bench_prefill(*a, full_scores=False, fp8=True)),
                      ("bucket", bench_bucket), ("two_stage", bench_two_stage),
                      ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True))):
         if only in (None, name):
@@ -356,53 +358,75 @@ def _profiled_loop(L, fn, steps, warm, st):
     return tot / steps, kern
 
 
-def bench_prefill(L, args, peaks, peak_kind, full_scores=True):
+def bench_prefill(L, args, peaks, peak_kind, full_scores=True, fp8=False):
     """Prefill chunk: history streamed from pinned host memory in 8192-key
-    tiles through two device buffers, causal top-512 of 4096 queries."""
+    tiles through two device buffers, causal top-512 of 4096 queries; with
+    fp8, e4m3 queries and an e4m3 history (the indexer's FP8 form)."""
     import torch
     from workloads import get_workload, make_workload
     st = torch.cuda.current_stream()
     steps = max(3, args.steps)
     warm = max(3, args.warmup)
-    wl = get_workload("prefill_chunk")
+    wl = get_workload("prefill_chunk_fp8" if fp8 else "prefill_chunk")
     d = make_workload(wl)
     T, H, dd = d["q"].shape
     N = d["k"].shape[0]
-    q, w, qp = to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev(d["q_pos"])
-    hist = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
-    buf0 = torch.empty((wl.tile_keys, dd), dtype=torch.bfloat16, device="cuda")
-    buf1 = torch.empty_like(buf0)
-    ws = torch.empty(L.lib().ls_prefill_select_workspace_size(T, N, wl.tile_keys, wl.k, int(full_scores)),
-                     dtype=torch.uint8, device="cuda")
+    w, qp = to_dev(d["w"]), to_dev(d["q_pos"])
     out = (torch.empty((T, wl.k), dtype=torch.int32, device="cuda"),
            torch.empty((T, wl.k), dtype=torch.float32, device="cuda"))
     cs = torch.cuda.Stream()
     n_t = np.minimum((d["q_pos"] + 1) // wl.stride, N)
     pairs = int(n_t.sum())
+    if fp8:
+        q8, qs = to_dev(d["q8"]), to_dev(d["q_scale"])
+        hk = torch.from_numpy(np.ascontiguousarray(d["k8"])).pin_memory()
+        hs = torch.from_numpy(np.ascontiguousarray(d["k_scale"])).pin_memory()
+        buf0 = torch.empty(wl.tile_keys * (dd + 4), dtype=torch.uint8, device="cuda")
+        buf1 = torch.empty_like(buf0)
+        ws = torch.empty(L.lib().ls_prefill_select_fp8_workspace_size(T, N, wl.tile_keys, wl.k, int(full_scores)),
+                         dtype=torch.uint8, device="cuda")
 
-    def pf(i, timed):
-        L.ls_prefill_select_stream(q, w, qp, hist, buf0, buf1, k=wl.k, stride=wl.stride, tile_keys=wl.tile_keys,
-                                   full_scores=full_scores, ws=ws, out=out, copy_stream=cs)
-        return None
+        def pf(i, timed):
+            L.ls_prefill_select_stream_fp8(q8, qs, w, qp, hk, hs, buf0, buf1, k=wl.k, stride=wl.stride,
+                                           tile_keys=wl.tile_keys, full_scores=full_scores, ws=ws, out=out,
+                                           copy_stream=cs)
+            return None
+        kname = "score_tc_kernel<8,fp8>"
+    else:
+        q = to_dev_bf16(d["q"])
+        hist = torch.from_numpy(d["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        buf0 = torch.empty((wl.tile_keys, dd), dtype=torch.bfloat16, device="cuda")
+        buf1 = torch.empty_like(buf0)
+        ws = torch.empty(L.lib().ls_prefill_select_workspace_size(T, N, wl.tile_keys, wl.k, int(full_scores)),
+                         dtype=torch.uint8, device="cuda")
+
+        def pf(i, timed):
+            L.ls_prefill_select_stream(q, w, qp, hist, buf0, buf1, k=wl.k, stride=wl.stride,
+                                       tile_keys=wl.tile_keys, full_scores=full_scores, ws=ws, out=out,
+                                       copy_stream=cs)
+            return None
+        kname = "score_tc_kernel<8>"
 
     ms, kern = _profiled_loop(L, pf, steps, warm, st)
-    score_ms = kern["score_tc_kernel<8>"]["ms_per_step"]
+    score_ms = kern[kname]["ms_per_step"]
     flops_alg = pairs * 2 * H * dd
     peak_t = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    if fp8:
+        peak_t = 2 * peak_t   # fp8 dense = 2 x bf16 dense (4.5 vs 2.25 PFLOP/s nominal)
     res = {
         "ms_per_step": ms, "positions_per_s": pairs / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
         "kernels": kern,
         "roofline": roofline("tensor", flops_alg / (score_ms * 1e-3) / 1e12, peak_t, "TFLOP/s",
-                             traffic=ncu_traffic("score_tc_kernel<8>",
-                                                 wl.name if full_scores else wl.name + "_running"),
-                             peak_kind=peak_kind),
+                             traffic=ncu_traffic(kname, wl.name if full_scores else wl.name + "_running"),
+                             peak_kind=peak_kind + (" bf16 x 2 (fp8)" if fp8 else "")),
         "algorithmic_flops": flops_alg, "eligible_pairs": pairs,
         "workspace_bytes": ws.numel(),
         "note": ("step = 4 streamed 8192-key tiles (H2D on a copy stream) + causal top-512 of 4096 queries; "
+                 + ("fp8 e4m3 queries and history (one scale per query head / per key); " if fp8 else "")
                  + ("full 4096 x 32768 score matrix, one top-k"
                     if full_scores else "running top-512 across tiles (first tile in full, later tiles filtered "
                                         "against each query's running 512th entry, merge per tile)")
-                 + "; roofline over the 4 scoring launches of the step (score_tc_kernel<8>)"),
+                 + f"; roofline over the 4 scoring launches of the step ({kname})"),
     }
     del ws
     return res
@@ -560,7 +584,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_batch")
     ap.add_argument("--no-variants", action="store_true")
-    ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "bucket", "two_stage",
+    ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "prefill_chunk_fp8",
+                                                     "prefill_chunk_fp8_running", "bucket", "two_stage",
                                                      "two_stage_pq"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -204,6 +204,58 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
                                    void* ws, size_t ws_bytes, void* compute_stream, void* copy_stream);
 
 /*
+ * ls_indexer_score_fp8 -- the indexer's scores with fp8 e4m3 queries and keys
+ * (the FP8 GEMM of the indexer, "03 long context" lecture, section "Sparsity
+ * Is a Systems Feature: The Blast Radius", kernel layer; 128-dim FP8 keys
+ * with a 4 B scale, section "The Architectural Answer: Read Less of the
+ * Past", stage 1):
+ *
+ *   scores[b][t][n] = sum_h w[b,t,h] * max(0, (qs[b,t,h] * q8[b,t,h]) . (ks[b,n] * k8[b,n]))
+ *                   (or -inf where n is not eligible)
+ *
+ *   q8 [B][T][H][d] e4m3 codes, q_scale [B][T][H] fp32 (one scale per query head)
+ *   w  [B][T][H] fp32
+ *   k8 [B][N][d] e4m3 codes, k_scale [B][N] fp32 (one scale per key)
+ *   n_valid [B] or NULL, q_pos [B][T] int64 or NULL (causal eligibility
+ *   floor((q_pos + 1) / stride), as in ls_indexer_score)
+ *   scores [B][T][N] fp32
+ * Scales must be non-negative and finite (magnitudes, amax / 448): the
+ * kernel takes them out of the ReLU, scaling the head weights by q_scale and
+ * the head sum by k_scale.  The q8 . k8 products of e4m3 codes are exact and
+ * summed in fp32 on the tensor cores (kind::f8f6f4); the head-weighted ReLU
+ * sum runs in fp32, so the scores match the exact value of the formula to
+ * fp32 rounding.
+ * q8 and k8 must be 16-byte aligned; w, q_scale and k_scale 4-byte aligned.
+ * Workspace: ls_indexer_score_fp8_workspace_size(B, T) bytes, 16-byte aligned
+ * (w * q_scale, B*T*H floats).
+ */
+size_t ls_indexer_score_fp8_workspace_size(int B, int T);
+ls_status ls_indexer_score_fp8(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                               const float* k_scale, const int32_t* n_valid, const int64_t* q_pos, int stride, int B,
+                               int T, int H, int d, int N, float* scores, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ls_prefill_select_stream_fp8 -- ls_prefill_select_stream with fp8 queries
+ * and an fp8 history (the scores of ls_indexer_score_fp8):
+ *
+ *   q8 [T][H][d] e4m3, q_scale [T][H] fp32, w [T][H] fp32, q_pos [T] int64
+ *   hist_k8 [N][d] e4m3 codes and hist_kscale [N] fp32, both in PINNED host
+ *           memory (device memory is accepted too)
+ *   buf0, buf1  device buffers of tile_keys * (d + 4) bytes each, 16-B
+ *           aligned: a tile's codes, then its scales at byte tile_keys * d
+ * Streaming, the two forms (full_scores 0 / 1), outputs and ordering are as
+ * in ls_prefill_select_stream; both forms return the same selection.
+ * Workspace: ls_prefill_select_fp8_workspace_size(T, N, tile_keys, k,
+ * full_scores) bytes, 16-byte aligned.
+ */
+size_t ls_prefill_select_fp8_workspace_size(int T, int N, int tile_keys, int k, int full_scores);
+ls_status ls_prefill_select_stream_fp8(const uint8_t* q8, const float* q_scale, const float* w, const int64_t* q_pos,
+                                       int T, int H, int d, const uint8_t* hist_k8, const float* hist_kscale, int N,
+                                       int stride, int tile_keys, void* buf0, void* buf1, int k, int full_scores,
+                                       int32_t* idx_out, float* val_out, void* ws, size_t ws_bytes,
+                                       void* compute_stream, void* copy_stream);
+
+/*
  * ls_decode_two_stage_select -- LeanSparse two-stage decode search
  * (podcast transcript, 07:12-08:00): scan compact keys, keep a shortlist,
  * fetch the shortlist's original keys and re-rank exactly, keep the top k.

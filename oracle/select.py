@@ -15,6 +15,12 @@ Pipelines:
 
 * decode / prefill selection: exact scores of every eligible position, then
   top-k (k = 512; LeanSparse podcast transcript, 01:33-02:06).
+* fp8 prefill selection: the same with e4m3 queries (one fp32 scale per
+  query head) and e4m3 keys (one fp32 scale per key), decoded exactly from
+  their codes and scaled ("03 long context" lecture, section "Sparsity Is a
+  Systems Feature: The Blast Radius": the indexer scores as an FP8 GEMM over
+  the 128-dim keys; section "The Architectural Answer: Read Less of the
+  Past", stage 1: a 128-dim FP8 key with a 4 B scale).
 * two-stage decode search (LeanSparse podcast transcript, 07:12-08:00): scores
   from compact keys, keep a shortlist, score the shortlist's original keys
   exactly, keep the top k of those.
@@ -101,6 +107,30 @@ def prefill_select(q_bits, w, q_pos, k_bits, stride: int = 4, k: int = 512, rows
     for i, t in enumerate(rows):
         n = int(n_t[t])
         s = indexer_scores(bf16_to_f64(q_bits[t])[None], np.asarray(w[t], np.float64)[None], keys[:n])[0]
+        idx[i], val[i] = select_topk(s, np.arange(n), k)
+        all_scores.append(s)
+    if return_scores:
+        return idx, val, all_scores
+    return idx, val
+
+
+def prefill_select_fp8(q8, q_scale, w, q_pos, k8, k_scale, stride: int = 4, k: int = 512, rows=None,
+                       return_scores: bool = False):
+    """Causal prefill selection with fp8 inputs: query head h of query t is
+    e4m3(q8[t, h]) * q_scale[t, h], key n is e4m3(k8[n]) * k_scale[n]; the
+    scores and the selection are then those of prefill_select."""
+    T = q8.shape[0]
+    N = k8.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    n_t = eligible_count(q_pos, stride, N)
+    keys = dequant(k8, k_scale, "e4m3")
+    idx = np.empty((rows.size, k), dtype=np.int64)
+    val = np.empty((rows.size, k), dtype=np.float64)
+    all_scores = []
+    for i, t in enumerate(rows):
+        n = int(n_t[t])
+        qt = dequant(q8[t], q_scale[t], "e4m3")          # [H, d]
+        s = indexer_scores(qt[None], np.asarray(w[t], np.float64)[None], keys[:n])[0]
         idx[i], val[i] = select_topk(s, np.arange(n), k)
         all_scores.append(s)
     if return_scores:

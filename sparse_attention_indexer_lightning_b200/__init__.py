@@ -19,8 +19,10 @@ from ._lib import (  # noqa: F401
     ls_decode_two_stage_select,
     ls_device_status,
     ls_indexer_score,
+    ls_indexer_score_fp8,
     ls_indexer_score_pq,
     ls_prefill_select_stream,
+    ls_prefill_select_stream_fp8,
     ls_profile_begin,
     ls_profile_end,
     ls_selftest_wait_probe,

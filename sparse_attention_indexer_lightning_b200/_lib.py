@@ -36,7 +36,8 @@ EXPORTED = (
     "ls_prefill_select_stream", "ls_two_stage_workspace_size", "ls_decode_two_stage_select",
     "ls_bucket_workspace_size", "ls_bucket_select", "ls_selftest_wait_probe", "ls_profile_begin",
     "ls_profile_end", "ls_profile_kernel", "ls_decode_select_noalloc", "ls_decode_two_stage_pq_select",
-    "ls_indexer_score_pq",
+    "ls_indexer_score_pq", "ls_indexer_score_fp8_workspace_size", "ls_indexer_score_fp8",
+    "ls_prefill_select_fp8_workspace_size", "ls_prefill_select_stream_fp8",
 )
 HIST_BINS = 2048
 
@@ -75,6 +76,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_decode_select_noalloc": (I, [P, P, P, P, I, I, I, I, I, P, P, P]),
         "ls_decode_two_stage_pq_select": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, SZ, P]),
         "ls_indexer_score_pq": (I, [P, P, P, P, P, I, I, I, I, P, P]),
+        "ls_indexer_score_fp8_workspace_size": (SZ, [I, I]),
+        "ls_indexer_score_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, SZ, P]),
+        "ls_prefill_select_fp8_workspace_size": (SZ, [I, I, I, I, I]),
+        "ls_prefill_select_stream_fp8": (I, [P, P, P, P, I, I, I, P, P, I, I, I, P, P, I, I, P, P, P, SZ, P, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -253,6 +258,78 @@ def ls_prefill_select_stream(q, w, q_pos, hist_k, buf0, buf1, k: int = 512, stri
     _check(lib().ls_prefill_select_stream(_ptr(q), _ptr(w), _ptr(q_pos), T, H, d, _ptr(hist_k), N, stride, tk,
                                           _ptr(buf0), _ptr(buf1), k, int(full_scores), _ptr(idx), _ptr(val),
                                           _ptr(ws), ws.numel(), cs, xs))
+    return idx, val
+
+
+def _codes(t, name: str, ndim: int) -> torch.Tensor:
+    """fp8 e4m3 codes as a uint8 view (float8_e4m3fn tensors are viewed, not converted)."""
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    return _dev(t, torch.uint8, name, ndim)
+
+
+def ls_indexer_score_fp8(q8, q_scale, w, k8, k_scale, n_valid=None, q_pos=None, stride: int = 4, ws=None,
+                         stream=None):
+    """q8 [B,T,H,d] e4m3 (float8_e4m3fn or uint8 codes), q_scale [B,T,H] f32, w [B,T,H] f32,
+    k8 [B,N,d] e4m3, k_scale [B,N] f32 -> scores [B,T,N] f32 (the fp8 indexer; scales >= 0)."""
+    q8 = _codes(q8, "q8", 4)
+    B, T, H, d = q8.shape
+    _dev(q_scale, torch.float32, "q_scale", 3)
+    _dev(w, torch.float32, "w", 3)
+    k8 = _codes(k8, "k8", 3)
+    N = k8.shape[1]
+    _dev(k_scale, torch.float32, "k_scale", 2)
+    _opt(n_valid, torch.int32, "n_valid")
+    _opt(q_pos, torch.int64, "q_pos")
+    need = lib().ls_indexer_score_fp8_workspace_size(B, T)
+    if ws is None:
+        ws = _workspace(need, q8.device)
+    out = torch.empty((B, T, N), dtype=torch.float32, device=q8.device)
+    _check(lib().ls_indexer_score_fp8(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), _ptr(n_valid),
+                                      _ptr(q_pos), stride, B, T, H, d, N, _ptr(out), _ptr(ws), ws.numel(),
+                                      _stream(stream)))
+    return out
+
+
+def ls_prefill_select_stream_fp8(q8, q_scale, w, q_pos, hist_k8, hist_kscale, buf0, buf1, k: int = 512,
+                                 stride: int = 4, tile_keys: Optional[int] = None, full_scores: bool = False,
+                                 ws=None, out=None, copy_stream=None, stream=None):
+    """Causal prefill selection with fp8 queries and an fp8 history streamed from (pinned) host memory.
+
+    q8 [T,H,d] e4m3, q_scale [T,H] f32, w [T,H] f32, q_pos [T] int64 (device);
+    hist_k8 [N,d] e4m3 codes and hist_kscale [N] f32 in pinned host memory (or
+    on the device); buf0/buf1 uint8 device buffers of tile_keys * (d + 4) bytes.
+    """
+    q8 = _codes(q8, "q8", 3)
+    T, H, d = q8.shape
+    _dev(q_scale, torch.float32, "q_scale", 2)
+    _dev(w, torch.float32, "w", 2)
+    _dev(q_pos, torch.int64, "q_pos", 1)
+    if hist_k8.dtype == torch.float8_e4m3fn:
+        hist_k8 = hist_k8.view(torch.uint8)
+    for t, dt, nd, name in ((hist_k8, torch.uint8, 2, "hist_k8"), (hist_kscale, torch.float32, 1, "hist_kscale")):
+        if t.dtype != dt or t.dim() != nd or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {nd}-d {dt} tensor")
+        if t.device.type == "cpu" and not t.is_pinned():
+            raise ValueError(f"{name} must be in pinned host memory")
+    N = hist_k8.shape[0]
+    _dev(buf0, torch.uint8, "buf0", 1)
+    _dev(buf1, torch.uint8, "buf1", 1)
+    tk = buf0.numel() // (d + 4) if tile_keys is None else tile_keys
+    if buf0.numel() < tk * (d + 4) or buf1.numel() < tk * (d + 4):
+        raise ValueError("buffers are shorter than tile_keys * (d + 4) bytes")
+    need = lib().ls_prefill_select_fp8_workspace_size(T, N, tk, k, int(full_scores))
+    if ws is None:
+        ws = _workspace(need, q8.device)
+    if out is None:
+        out = (torch.empty((T, k), dtype=torch.int32, device=q8.device),
+               torch.empty((T, k), dtype=torch.float32, device=q8.device))
+    idx, val = out
+    cs = _stream(stream)
+    xs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
+    _check(lib().ls_prefill_select_stream_fp8(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(q_pos), T, H, d, _ptr(hist_k8),
+                                              _ptr(hist_kscale), N, stride, tk, _ptr(buf0), _ptr(buf1), k,
+                                              int(full_scores), _ptr(idx), _ptr(val), _ptr(ws), ws.numel(), cs, xs))
     return idx, val
 
 

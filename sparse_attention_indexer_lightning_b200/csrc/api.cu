@@ -130,15 +130,15 @@ ls_status make_bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_
   return LS_OK;
 }
 
-// 2-D map over [rows][128 bytes] (one 8-bit key per row), box = 128 bytes x
-// 128 rows, 128-byte swizzle.  The bytes are described as 64 16-bit elements
-// per row: the copy and the swizzle act on bytes either way.
-ls_status make_u8_map(CUtensorMap* m, const void* base, uint64_t rows) {
+// 2-D map over [rows][128 bytes] (one 8-bit key or query head per row), box =
+// 128 bytes x box_rows rows, 128-byte swizzle.  The bytes are described as 64
+// 16-bit elements per row: the copy and the swizzle act on bytes either way.
+ls_status make_u8_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows = kTileKeys) {
   auto fn = encode_fn();
   if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDim)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim / 2), static_cast<cuuint32_t>(kTileKeys)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim / 2), box_rows};
   cuuint32_t es[2] = {1u, 1u};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -187,6 +187,32 @@ ls_status score_tc_launch(const uint16_t* q, const uint16_t* keys, int B, int T,
   p.N = N;
   ProfScope prof(prof_name ? prof_name : qg == 1 ? "score_tc_kernel<1>" : "score_tc_kernel<8>", st);
   LS_CUDA(launch_score_tc(qg, &kmap, &qmap, p, num_sms_current(), st));
+  return LS_OK;
+}
+
+// The fp8 scorer's head weights: w * q_scale per (query, head), n values.
+ls_status fold_scales(const float* w, const float* q_scale, int64_t n, float* w_eff, cudaStream_t st) {
+  ProfScope prof("fold_scales_kernel", st);
+  LS_CUDA(launch_fold_scales(w, q_scale, n, w_eff, st));
+  return LS_OK;
+}
+
+// Scores of fp8 queries and keys on the tensor cores; p.w must hold w *
+// q_scale (fold_scales), p is filled by the caller apart from the shape.
+ls_status score_f8_launch(const uint8_t* q8, const uint8_t* keys, const float* key_scale, int B, int T, int N,
+                          ScoreParams p, cudaStream_t st, const char* prof_name = nullptr) {
+  if (B == 0 || T == 0 || N == 0) return LS_OK;
+  CUtensorMap kmap, qmap;
+  ls_status s = make_u8_map(&kmap, keys, static_cast<uint64_t>(B) * N, kTileKeys);
+  if (s != LS_OK) return s;
+  s = make_u8_map(&qmap, q8, static_cast<uint64_t>(B) * T * kHeads, 8 * kHeads);
+  if (s != LS_OK) return s;
+  p.B = B;
+  p.T = T;
+  p.N = N;
+  p.key_scale = key_scale;
+  ProfScope prof(prof_name ? prof_name : "score_tc_kernel<8,fp8>", st);
+  LS_CUDA(launch_score_tc_f8(&kmap, &qmap, p, num_sms_current(), st));
   return LS_OK;
 }
 
@@ -383,11 +409,10 @@ int prefill_cand_cap(int k) { return 3 * k; }
 
 size_t ls_prefill_select_workspace_size(int T, int N, int tile_keys, int k, int full_scores) {
   if (T <= 0 || N <= 0 || tile_keys <= 0 || k <= 0) return 0;
-  if (full_scores)  // the whole T x N score matrix, then one top-k
-    return align_up(static_cast<size_t>(T) * N * sizeof(float)) + align_up(static_cast<size_t>(T) * sizeof(int32_t));
-  const int tk = tile_keys < N ? tile_keys : N;
+  // full_scores: the whole T x N score matrix (one top-k at the end), no running lists
+  const int tk = full_scores ? N : (tile_keys < N ? tile_keys : N);
   const int ntiles = (N + tile_keys - 1) / tile_keys;
-  const int64_t ldc = ntiles > 1 ? k + prefill_cand_cap(k) : 0;
+  const int64_t ldc = (!full_scores && ntiles > 1) ? k + prefill_cand_cap(k) : 0;
   return align_up(static_cast<size_t>(T) * tk * sizeof(float)) +    // one tile of scores
          align_up(static_cast<size_t>(T) * ldc * sizeof(float)) +   // running top-k + candidates
          align_up(static_cast<size_t>(T) * ldc * sizeof(int32_t)) +
@@ -396,45 +421,60 @@ size_t ls_prefill_select_workspace_size(int T, int N, int tile_keys, int k, int 
          align_up(static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int));  // counters, overflow flags
 }
 
-ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int64_t* q_pos, int T, int H, int d,
-                                   const uint16_t* hist_k, int N, int stride, int tile_keys, uint16_t* buf0,
-                                   uint16_t* buf1, int k, int full_scores, int32_t* idx_out, float* val_out,
-                                   void* ws, size_t ws_bytes, void* compute_stream, void* copy_stream) {
-  ls_status s = check_shape(H, d);
-  if (s != LS_OK) return s;
-  LS_CHECK_ARG(T >= 0 && N >= 0, "negative size");
-  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
-  LS_CHECK_ARG(stride >= 1, "stride must be >= 1");
-  LS_CHECK_ARG(tile_keys >= 1, "tile_keys must be >= 1");
-  if (T == 0) return LS_OK;
-  LS_CHECK_ARG(q && w && q_pos && idx_out, "null tensor pointer");
-  LS_CHECK_ARG(aligned16(q) && aligned16(w), "q and w must be 16-byte aligned");
-  cudaStream_t cs = S(compute_stream);
-  cudaStream_t xs = copy_stream ? S(copy_stream) : cs;
-  if (N == 0) {  // no history: every row is padding
-    TopkParams p;
-    p.R = T;
-    p.k = k;
-    p.idx_out = idx_out;
-    p.val_out = val_out;
-    p.ld_out = k;
-    return topk_launch(p, cs);
+}  // extern "C"
+
+namespace {
+
+// History sources of the streamed prefill: how a tile of the history reaches
+// a device buffer and how the keys in a buffer are scored.
+struct Bf16History {
+  const uint16_t* q;
+  const uint16_t* hist;
+  uint16_t* bufs[2];
+  const char* overflow_name = "score_tc_kernel<8>:overflow";
+  cudaError_t copy(int slot, int k0, int len, cudaStream_t xs) const {
+    return cudaMemcpyAsync(bufs[slot], hist + static_cast<size_t>(k0) * kDim,
+                           static_cast<size_t>(len) * kDim * sizeof(uint16_t), cudaMemcpyDefault, xs);
   }
-  const size_t need = ls_prefill_select_workspace_size(T, N, tile_keys, k, full_scores);
-  if (ws_bytes < need || (need && !ws))
-    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
-  LS_CHECK_ARG(hist_k && buf0 && buf1, "null history or buffer pointer");
-  LS_CHECK_ARG(aligned16(buf0) && aligned16(buf1) && aligned16(hist_k), "history and buffers must be 16-byte aligned");
-  cudaPointerAttributes attr;
-  LS_CUDA(cudaPointerGetAttributes(&attr, hist_k));
-  LS_CHECK_ARG(attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeDevice ||
-                   attr.type == cudaMemoryTypeManaged,
-               "hist_k must be pinned host memory or device memory (pageable memory cannot be streamed)");
+  ls_status score(int slot, int T, int len, const ScoreParams& sp, cudaStream_t cs, const char* name) const {
+    return score_tc_launch(q, bufs[slot], 1, T, len, sp, cs, name);
+  }
+};
+
+// fp8 history: e4m3 codes [N][128] and fp32 scales [N]; a device buffer holds
+// a tile's codes followed by its scales (at tile_keys * 128 bytes).
+struct F8History {
+  const uint8_t* q8;
+  const uint8_t* hist;
+  const float* hist_scale;
+  uint8_t* bufs[2];
+  int tile_keys;
+  const char* overflow_name = "score_tc_kernel<8,fp8>:overflow";
+  cudaError_t copy(int slot, int k0, int len, cudaStream_t xs) const {
+    cudaError_t e = cudaMemcpyAsync(bufs[slot], hist + static_cast<size_t>(k0) * kDim, static_cast<size_t>(len) * kDim,
+                                    cudaMemcpyDefault, xs);
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyAsync(bufs[slot] + static_cast<size_t>(tile_keys) * kDim, hist_scale + k0,
+                           static_cast<size_t>(len) * sizeof(float), cudaMemcpyDefault, xs);
+  }
+  ls_status score(int slot, int T, int len, const ScoreParams& sp, cudaStream_t cs, const char* name) const {
+    const float* ks = reinterpret_cast<const float*>(bufs[slot] + static_cast<size_t>(tile_keys) * kDim);
+    return score_f8_launch(q8, bufs[slot], ks, 1, T, len, sp, cs, name);
+  }
+};
+
+// The streamed prefill over tiles of tile_keys history keys: copy tile j on
+// the copy stream while tile j-1 is scored; either every tile into the full
+// T x N matrix and one top-k at the end, or a running top-k (tile 0 in full,
+// later tiles through the filter form, then a merge).
+template <class Src>
+ls_status prefill_stream(const Src& src, Carver& cv, const float* w, const int64_t* q_pos, int T, int N, int stride,
+                         int tile_keys, int k, int full_scores, int32_t* idx_out, float* val_out, cudaStream_t cs,
+                         cudaStream_t xs) {
   const int tk = full_scores ? N : (tile_keys < N ? tile_keys : N);
   const int ntiles = (N + tile_keys - 1) / tile_keys;
   const int cap = prefill_cand_cap(k);
   const int64_t ldc = (!full_scores && ntiles > 1) ? k + cap : 0;
-  Carver cv(ws);
   float* tile_sc = cv.take<float>(static_cast<size_t>(T) * tk);  // full_scores: the T x N matrix
   float* run_val = cv.take<float>(static_cast<size_t>(T) * ldc);
   int32_t* run_lab = cv.take<int32_t>(static_cast<size_t>(T) * ldc);
@@ -446,7 +486,6 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
   int* any_over = reinterpret_cast<int*>(ctr) + 2 * static_cast<size_t>(T);
   const size_t ctr_bytes = static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int);
 
-  uint16_t* bufs[2] = {buf0, buf1};
   cudaEvent_t start_ev, copied[2], freed[2];
   LS_CUDA(cudaEventCreateWithFlags(&start_ev, cudaEventDisableTiming));
   for (int i = 0; i < 2; ++i) {
@@ -468,8 +507,7 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
     const bool last = j + 1 == ntiles;
     if (j >= 2 && xs != cs) e = cudaStreamWaitEvent(xs, freed[slot], 0);
     if (e != cudaSuccess) break;
-    e = cudaMemcpyAsync(bufs[slot], hist_k + static_cast<size_t>(k0) * kDim,
-                        static_cast<size_t>(len) * kDim * sizeof(uint16_t), cudaMemcpyDefault, xs);
+    e = src.copy(slot, k0, len, xs);
     if (e != cudaSuccess) break;
     if (xs != cs) {
       e = cudaEventRecord(copied[slot], xs);
@@ -497,7 +535,7 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
       sp.out = tile_sc;
       sp.ld_out = N;
       sp.out_col0 = k0;
-      st = score_tc_launch(q, bufs[slot], 1, T, len, sp, cs);
+      st = src.score(slot, T, len, sp, cs, nullptr);
       if (st != LS_OK) break;
       if (last) {
         TopkParams fp;
@@ -517,7 +555,7 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
       // the first tile is scored in full and gives every row its running top-k
       sp.out = tile_sc;
       sp.ld_out = tk;
-      st = score_tc_launch(q, bufs[slot], 1, T, len, sp, cs);
+      st = src.score(slot, T, len, sp, cs, nullptr);
       if (st != LS_OK) break;
       tp.idx_out = last ? idx_out : run_lab;
       tp.val_out = last ? val_out : run_val;
@@ -537,7 +575,7 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
       fp.cand_cnt = cnt;
       fp.row_over = row_over;
       fp.any_over = any_over;
-      st = score_tc_launch(q, bufs[slot], 1, T, len, fp, cs);
+      st = src.score(slot, T, len, fp, cs, nullptr);
       if (st != LS_OK) break;
       // rows that ran out of candidate slots: this tile again in full (the
       // launches return at once when no row overflowed), its top-k into the
@@ -545,7 +583,7 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
       sp.out = tile_sc;
       sp.ld_out = tk;
       sp.run_if = any_over;
-      st = score_tc_launch(q, bufs[slot], 1, T, len, sp, cs, "score_tc_kernel<8>:overflow");
+      st = src.score(slot, T, len, sp, cs, src.overflow_name);
       if (st != LS_OK) break;
       tp.run_if = any_over;
       tp.row_flag = row_over;
@@ -589,6 +627,137 @@ ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int6
   if (st != LS_OK) return st;
   if (e != cudaSuccess) return fail(LS_ERR_CUDA, "history streaming: %s", cudaGetErrorString(e));
   return LS_OK;
+}
+
+
+}  // namespace
+
+extern "C" {
+
+ls_status ls_prefill_select_stream(const uint16_t* q, const float* w, const int64_t* q_pos, int T, int H, int d,
+                                   const uint16_t* hist_k, int N, int stride, int tile_keys, uint16_t* buf0,
+                                   uint16_t* buf1, int k, int full_scores, int32_t* idx_out, float* val_out,
+                                   void* ws, size_t ws_bytes, void* compute_stream, void* copy_stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(T >= 0 && N >= 0, "negative size");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  LS_CHECK_ARG(stride >= 1, "stride must be >= 1");
+  LS_CHECK_ARG(tile_keys >= 1, "tile_keys must be >= 1");
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(q && w && q_pos && idx_out, "null tensor pointer");
+  LS_CHECK_ARG(aligned16(q) && aligned16(w), "q and w must be 16-byte aligned");
+  cudaStream_t cs = S(compute_stream);
+  cudaStream_t xs = copy_stream ? S(copy_stream) : cs;
+  if (N == 0) {  // no history: every row is padding
+    TopkParams p;
+    p.R = T;
+    p.k = k;
+    p.idx_out = idx_out;
+    p.val_out = val_out;
+    p.ld_out = k;
+    return topk_launch(p, cs);
+  }
+  const size_t need = ls_prefill_select_workspace_size(T, N, tile_keys, k, full_scores);
+  if (ws_bytes < need || (need && !ws))
+    return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  LS_CHECK_ARG(hist_k && buf0 && buf1, "null history or buffer pointer");
+  LS_CHECK_ARG(aligned16(buf0) && aligned16(buf1) && aligned16(hist_k), "history and buffers must be 16-byte aligned");
+  cudaPointerAttributes attr;
+  LS_CUDA(cudaPointerGetAttributes(&attr, hist_k));
+  LS_CHECK_ARG(attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeDevice ||
+                   attr.type == cudaMemoryTypeManaged,
+               "hist_k must be pinned host memory or device memory (pageable memory cannot be streamed)");
+  Carver cv(ws);
+  Bf16History src{q, hist_k, {buf0, buf1}};
+  return prefill_stream(src, cv, w, q_pos, T, N, stride, tile_keys, k, full_scores, idx_out, val_out, cs, xs);
+}
+
+size_t ls_indexer_score_fp8_workspace_size(int B, int T) {
+  if (B <= 0 || T <= 0) return 0;
+  return align_up(static_cast<size_t>(B) * T * kHeads * sizeof(float));  // w * q_scale
+}
+
+ls_status ls_indexer_score_fp8(const uint8_t* q8, const float* q_scale, const float* w, const uint8_t* k8,
+                               const float* k_scale, const int32_t* n_valid, const int64_t* q_pos, int stride, int B,
+                               int T, int H, int d, int N, float* scores, void* ws, size_t ws_bytes, void* stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(B >= 0 && T >= 0 && N >= 0, "negative size (B=%d T=%d N=%d)", B, T, N);
+  if (B == 0 || T == 0 || N == 0) return LS_OK;
+  LS_CHECK_ARG(q8 && q_scale && w && k8 && k_scale && scores, "null tensor pointer");
+  LS_CHECK_ARG(aligned16(q8) && aligned16(k8), "q8 and k8 must be 16-byte aligned");
+  LS_CHECK_ARG(q_pos == nullptr || stride >= 1, "stride must be >= 1 with q_pos");
+  const size_t need = ls_indexer_score_fp8_workspace_size(B, T);
+  if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  LS_CHECK_ARG(aligned16(ws), "workspace must be 16-byte aligned");
+  cudaStream_t st = S(stream);
+  float* w_eff = static_cast<float*>(ws);
+  s = fold_scales(w, q_scale, static_cast<int64_t>(B) * T * kHeads, w_eff, st);
+  if (s != LS_OK) return s;
+  ScoreParams p;
+  p.w = w_eff;
+  p.n_valid = n_valid;
+  p.q_pos = q_pos;
+  p.out = scores;
+  p.ld_out = N;
+  p.stride = stride;
+  p.n_total = N;
+  return score_f8_launch(q8, k8, k_scale, B, T, N, p, st);
+}
+
+size_t ls_prefill_select_fp8_workspace_size(int T, int N, int tile_keys, int k, int full_scores) {
+  const size_t base = ls_prefill_select_workspace_size(T, N, tile_keys, k, full_scores);
+  if (base == 0) return 0;
+  return base + align_up(static_cast<size_t>(T) * kHeads * sizeof(float));  // + w * q_scale, after the generic part
+}
+
+ls_status ls_prefill_select_stream_fp8(const uint8_t* q8, const float* q_scale, const float* w, const int64_t* q_pos,
+                                       int T, int H, int d, const uint8_t* hist_k8, const float* hist_kscale, int N,
+                                       int stride, int tile_keys, void* buf0, void* buf1, int k, int full_scores,
+                                       int32_t* idx_out, float* val_out, void* ws, size_t ws_bytes,
+                                       void* compute_stream, void* copy_stream) {
+  ls_status s = check_shape(H, d);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(T >= 0 && N >= 0, "negative size");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  LS_CHECK_ARG(stride >= 1, "stride must be >= 1");
+  LS_CHECK_ARG(tile_keys >= 1, "tile_keys must be >= 1");
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(q8 && q_scale && w && q_pos && idx_out, "null tensor pointer");
+  LS_CHECK_ARG(aligned16(q8), "q8 must be 16-byte aligned");
+  cudaStream_t cs = S(compute_stream);
+  cudaStream_t xs = copy_stream ? S(copy_stream) : cs;
+  if (N == 0) {  // no history: every row is padding
+    TopkParams p;
+    p.R = T;
+    p.k = k;
+    p.idx_out = idx_out;
+    p.val_out = val_out;
+    p.ld_out = k;
+    return topk_launch(p, cs);
+  }
+  const size_t need = ls_prefill_select_fp8_workspace_size(T, N, tile_keys, k, full_scores);
+  if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  LS_CHECK_ARG(aligned16(ws), "workspace must be 16-byte aligned");
+  LS_CHECK_ARG(hist_k8 && hist_kscale && buf0 && buf1, "null history or buffer pointer");
+  LS_CHECK_ARG(aligned16(buf0) && aligned16(buf1) && aligned16(hist_k8),
+               "history codes and buffers must be 16-byte aligned");
+  for (const void* hp : {static_cast<const void*>(hist_k8), static_cast<const void*>(hist_kscale)}) {
+    cudaPointerAttributes attr;
+    LS_CUDA(cudaPointerGetAttributes(&attr, hp));
+    LS_CHECK_ARG(attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeDevice ||
+                     attr.type == cudaMemoryTypeManaged,
+                 "the history must be pinned host memory or device memory (pageable memory cannot be streamed)");
+  }
+  // w * q_scale sits at the end of the workspace, after the generic part
+  float* w_eff = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + need -
+                                          align_up(static_cast<size_t>(T) * kHeads * sizeof(float)));
+  s = fold_scales(w, q_scale, static_cast<int64_t>(T) * kHeads, w_eff, cs);
+  if (s != LS_OK) return s;
+  Carver cv(ws);
+  F8History src{q8, hist_k8, hist_kscale, {static_cast<uint8_t*>(buf0), static_cast<uint8_t*>(buf1)}, tile_keys};
+  return prefill_stream(src, cv, w_eff, q_pos, T, N, stride, tile_keys, k, full_scores, idx_out, val_out, cs, xs);
 }
 
 size_t ls_two_stage_workspace_size(int B, int N, int shortlist) {

@@ -53,11 +53,21 @@ struct ScoreParams {
   int32_t* row_over = nullptr;        // [B*T]
   int* any_over = nullptr;
   const int* run_if = nullptr;        // the launch does nothing unless *run_if != 0 (nullptr: always)
+  const float* key_scale = nullptr;   // fp8 scorer: per-key scale [B][N] (scores are multiplied by it)
 };
 
 // qg = queries sharing one MMA B tile: 1 (one query per sequence) or 8.
 cudaError_t launch_score_tc(int qg, const CUtensorMap* kmap, const CUtensorMap* qmap,
                             const ScoreParams& p, int num_sms, cudaStream_t st);
+
+// fp8 queries and keys (e4m3 codes) on the tensor cores, eight queries per
+// group: kmap over the keys [B*N][128 B], qmap over the query heads
+// [B*T*H][128 B]; p.w holds w * q_scale (launch_fold_scales), p.key_scale the
+// per-key scales [B][N].
+cudaError_t launch_score_tc_f8(const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p, int num_sms,
+                               cudaStream_t st);
+// out[i] = w[i] * qs[i], i < n.
+cudaError_t launch_fold_scales(const float* w, const float* qs, int64_t n, float* out, cudaStream_t st);
 
 // Source rows for the converting scorer.
 enum SrcFormat : int { SRC_INT8 = 0, SRC_E4M3 = 1, SRC_BF16 = 2, SRC_PQ = 3 };

@@ -7,6 +7,8 @@
 //  * expand: best-first bucket expansion ("Latent Sparse Attention", "The
 //    method, term by term", step 6): read the picked buckets in score order,
 //    append their members until the budget is held, cut the last bucket short.
+//  * fold_scales: w[t, h] * q_scale[t, h] for the fp8 scorer, which takes the
+//    non-negative per-(query, head) scale out of the ReLU.
 //  * wait_probe: a kernel whose mbarrier is never signalled, used by the tests
 //    to show that a bounded wait returns with an error status.
 
@@ -30,6 +32,20 @@ cudaError_t launch_causal_counts(const int64_t* q_pos, int T, int stride, int n_
                                  cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   causal_counts_kernel<<<(T + 255) / 256, 256, 0, st>>>(q_pos, T, stride, n_total, out);
+  return cudaGetLastError();
+}
+
+__global__ void fold_scales_kernel(const float* __restrict__ w, const float* __restrict__ qs, int64_t n,
+                                   float* __restrict__ out) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = w[i] * qs[i];
+}
+
+cudaError_t launch_fold_scales(const float* w, const float* qs, int64_t n, float* out, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int64_t want = (n + 255) / 256;
+  fold_scales_kernel<<<static_cast<int>(want < 2048 ? want : 2048), 256, 0, st>>>(w, qs, n, out);
   return cudaGetLastError();
 }
 

@@ -1,4 +1,5 @@
-// Lightning-indexer scoring on the sm_100a tensor cores, bf16 keys.
+// Lightning-indexer scoring on the sm_100a tensor cores: bf16 queries and
+// keys, or (F8) fp8 e4m3 queries and keys.
 //
 // score(t, s) = sum_h w[t, h] * max(0, q[t, h] . k[s])   ("03 long context",
 // section "The Architectural Answer: Read Less of the Past", stage 1; the
@@ -12,11 +13,19 @@
 // owns a key reads its 32 head sums with one tcgen05.ld and reduces the heads
 // in registers: ReLU, multiply by w, add -- no shuffles.
 //
+// F8 (the indexer's FP8 GEMM, "03 long context" lecture, section "Sparsity
+// Is a Systems Feature: The Blast Radius", kernel layer): A and B are e4m3
+// codes, a 128-byte row per key or query head (one swizzle panel), K = 128
+// as 4 kind::f8f6f4 MMAs of K = 32; the code products are exact and summed
+// in fp32.  With non-negative scales the ReLU commutes with them: the host
+// passes w * q_scale as the head weights and the epilogue multiplies each
+// key's head sum by its scale.
+//
 // Roles (one persistent CTA per SM, contiguous runs of work units):
 //   warp 0      TMA producer (keys every unit, the query tile on group change)
 //   warp 1      TMEM allocator + single-thread MMA issuer
-//   warps 2..   epilogue (4 warps for QG = 1, 12 for QG = 8: three per TMEM
-//               lane quadrant, sharing the 8 queries of a group 3 / 3 / 2)
+//   warps 2..   epilogue (4 warps for QG = 1, 16 for QG = 8: four per TMEM
+//               lane quadrant, two of the group's 8 queries each)
 // Pipelines: STAGES key buffers (full/empty mbarriers), 2 query-tile slots,
 // 2 TMEM accumulators so the epilogue of unit i overlaps the MMA of unit i+1.
 // Every wait is bounded; a wait that runs out raises the library fault word
@@ -29,15 +38,20 @@
 
 namespace lsi {
 
-template <int QG, bool FILTER = false>
+// F8: fp8 e4m3 queries and keys (kind::f8f6f4 MMAs, K = 32 each; a 128-byte
+// row holds a whole key, so one swizzle panel); otherwise bf16 (two 64-wide
+// panels per row, K = 16 per MMA).
+template <int QG, bool FILTER = false, bool F8 = false>
 struct TcCfg {
   static constexpr int BM = kTileKeys;             // keys per tile
   static constexpr int BN = QG * kHeads;           // queries x heads per MMA
-  static constexpr int A_BYTES = BM * kDim * 2;    // 32 KB
-  static constexpr int A_HALF = BM * 64 * 2;       // one 64-wide swizzle panel
-  static constexpr int B_BYTES = BN * kDim * 2;
-  static constexpr int B_HALF = BN * 64 * 2;
-  static constexpr int STAGES = (QG == 1) ? 6 : (FILTER ? 2 : 3);
+  static constexpr int ESZ = F8 ? 1 : 2;           // bytes per element
+  static constexpr int A_BYTES = BM * kDim * ESZ;  // 32 KB (bf16), 16 KB (fp8)
+  static constexpr int A_HALF = BM * 128;          // one 128-byte swizzle panel of the tile
+  static constexpr int B_BYTES = BN * kDim * ESZ;
+  static constexpr int B_HALF = BN * 128;
+  static constexpr int PANELS = kDim * ESZ / 128;  // 2 (bf16) or 1 (fp8)
+  static constexpr int STAGES = (QG == 1) ? 6 : (FILTER ? 2 : (F8 ? 4 : 3));
   static constexpr int ACC = (QG == 1) ? 8 : 2;       // accumulator stages in TMEM
   static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
   static constexpr int TMEM_COLS = (ACC * ACC_COLS <= 32) ? 32
@@ -75,17 +89,6 @@ struct TcBarriers {
 };
 static_assert(sizeof(TcBarriers) <= 512, "barrier block");
 
-// Drain wait: bounded by time only (used after an abort).
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > LSI_WAIT_LIMIT_NS) {
-      atomicOr(&g_fault, FAULT_WAIT_TIMEOUT);
-      return;
-    }
-  }
-}
-
 // Keys of the whole history query (b, t) may see: a precomputed count, or
 // floor((q_pos + 1) / stride) capped at n_total (block-complete causal rule).
 __device__ __forceinline__ int eligible_keys(const ScoreParams& p, int b, int t) {
@@ -98,11 +101,11 @@ __device__ __forceinline__ int eligible_keys(const ScoreParams& p, int b, int t)
 
 // FILTER: the filter form of ScoreParams (p.out == nullptr), built as its own
 // instantiation so the storing form keeps its registers.
-template <int QG, bool FILTER>
-__global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
+template <int QG, bool FILTER, bool F8>
+__global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                     const ScoreParams p) {
-  using C = TcCfg<QG, FILTER>;
+  using C = TcCfg<QG, FILTER, F8>;
   if (p.run_if != nullptr && *p.run_if == 0) return;  // a conditional launch with nothing to do
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
           const int qrow = (b * p.T + g * QG) * kHeads;
           uint8_t* dst = sB + bslot * C::B_BYTES;
           tma_load_2d(dst, &qmap, &bars->bfull[bslot], 0, qrow);
-          tma_load_2d(dst + C::B_HALF, &qmap, &bars->bfull[bslot], 64, qrow);
+          if (C::PANELS == 2) tma_load_2d(dst + C::B_HALF, &qmap, &bars->bfull[bslot], 64, qrow);
           prev_bg = bg;
         }
         if (!mbar_wait(&bars->empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
         const int krow = b * p.N + tile * C::BM;
         uint8_t* dst = sA + stage * C::A_BYTES;
         tma_load_2d(dst, &kmap, &bars->full[stage], 0, krow);
-        tma_load_2d(dst + C::A_HALF, &kmap, &bars->full[stage], 64, krow);
+        if (C::PANELS == 2) tma_load_2d(dst + C::A_HALF, &kmap, &bars->full[stage], 64, krow);
         issued[stage] = 1;
         issued_par[stage] = phase;
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
     // MMAs are short and one elected lane of the converged warp issues them;
     // with eight (N = 256) the epilogue sets the pace and issuing from lane 0
     // alone measured faster.
-    constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::BN);
+    constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(C::BM, C::BN) : idesc_bf16_f32(C::BM, C::BN);
     constexpr bool ELECT = (QG == 1);
     int stage = 0;
     uint32_t phase = 0;
@@ -242,13 +245,19 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
       const uint32_t a_addr = a_base + stage * C::A_BYTES;
       const uint32_t b_addr = b_base + bslot * C::B_BYTES;
       const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+      // one MMA per 32 bytes of K: 16 bf16 or 32 e4m3 inside a 128-byte swizzle row
 #pragma unroll
-      for (int kk = 0; kk < kDim / 16; ++kk) {
-        const uint32_t koff = (kk & 3) * 32;  // 16 bf16 = 32 B inside a 128 B swizzle row
+      for (int kk = 0; kk < 4 * C::PANELS; ++kk) {
+        const uint32_t koff = (kk & 3) * 32;
         const uint64_t adesc = sw128_kmajor_desc(a_addr + (kk >> 2) * C::A_HALF + koff);
         const uint64_t bdesc = sw128_kmajor_desc(b_addr + (kk >> 2) * C::B_HALF + koff);
-        if (ELECT) umma_f16_warp(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-        else if (lane == 0) umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        if (F8) {
+          if (lane == 0) umma_e4m3(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        } else if (ELECT) {
+          umma_f16_warp(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        } else if (lane == 0) {
+          umma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+        }
       }
       if (ELECT) {
         umma_commit_warp(&bars->empty[stage]);
@@ -365,6 +374,8 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
           }
         }
       }
+      float ks = 1.f;                                      // fp8: the key's scale, loaded ahead of the wait
+      if (F8) ks = (n < p.N) ? __ldg(p.key_scale + static_cast<int64_t>(hb) * p.N + n) : 0.f;
       if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
@@ -385,7 +396,8 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->tempty[acc]);
           }
-          const float s = (QG == 1) ? head_reduce_w(cur, wreg) : head_reduce(cur, wq[jq]);
+          float s = (QG == 1) ? head_reduce_w(cur, wreg) : head_reduce(cur, wq[jq]);
+          if (F8) s *= ks;                                 // the key's scale (w holds w * q_scale)
           if (!filter) {
             if (n < p.N) {
               orow[jq][n] = (n < limq[jq]) ? s : neg_inf();
@@ -428,13 +440,13 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER>::THREADS, 1)
   }
 }
 
-template <int QG, bool FILTER>
+template <int QG, bool FILTER, bool F8 = false>
 static cudaError_t launch_tc(const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p, int num_sms,
                              cudaStream_t st) {
-  using C = TcCfg<QG, FILTER>;
+  using C = TcCfg<QG, FILTER, F8>;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<QG, FILTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<QG, FILTER, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::SMEM_TOTAL));
     if (e != cudaSuccess) return e;
     attr_done = true;
@@ -444,7 +456,7 @@ static cudaError_t launch_tc(const CUtensorMap* kmap, const CUtensorMap* qmap, c
   const long long units = static_cast<long long>(p.B) * G * NT;
   if (units == 0) return cudaSuccess;
   const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-  score_tc_kernel<QG, FILTER><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*kmap, *qmap, p);
+  score_tc_kernel<QG, FILTER, F8><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*kmap, *qmap, p);
   return cudaGetLastError();
 }
 
@@ -454,6 +466,15 @@ cudaError_t launch_score_tc(int qg, const CUtensorMap* kmap, const CUtensorMap* 
   if (qg == 1) return filter ? launch_tc<1, true>(kmap, qmap, p, num_sms, st) : launch_tc<1, false>(kmap, qmap, p, num_sms, st);
   if (qg == 8) return filter ? launch_tc<8, true>(kmap, qmap, p, num_sms, st) : launch_tc<8, false>(kmap, qmap, p, num_sms, st);
   return cudaErrorInvalidValue;
+}
+
+// fp8 queries and keys, eight queries per group: p.w holds w * q_scale per
+// (query, head) and p.key_scale the keys' scales.
+cudaError_t launch_score_tc_f8(const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p, int num_sms,
+                               cudaStream_t st) {
+  const bool filter = p.out == nullptr;
+  return filter ? launch_tc<8, true, true>(kmap, qmap, p, num_sms, st)
+                : launch_tc<8, false, true>(kmap, qmap, p, num_sms, st);
 }
 
 }  // namespace lsi

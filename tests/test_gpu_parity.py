@@ -294,6 +294,152 @@ def test_prefill_chunk_full_size_sampled(L):
 
 
 # --------------------------------------------------------------------------- #
+# fp8 indexer: fp8 queries and keys, the prefill streamed from an fp8 history
+# --------------------------------------------------------------------------- #
+def _fp8_ref(d, t, n):
+    qt = dequant(d["q8"][t], d["q_scale"][t], "e4m3")
+    return indexer_scores(qt[None], d["w"][t].astype(np.float64)[None],
+                          dequant(d["k8"][:n], d["k_scale"][:n], "e4m3"))[0]
+
+
+def _fp8_prefill_run(L, d, wl, full_scores=False, use_copy_stream=True):
+    q8 = dev(d["q8"])
+    qs, w, qp = dev(d["q_scale"]), dev(d["w"]), dev(d["q_pos"])
+    hk = torch.from_numpy(np.ascontiguousarray(d["k8"])).pin_memory()
+    hs = torch.from_numpy(np.ascontiguousarray(d["k_scale"])).pin_memory()
+    buf0 = torch.empty(wl.tile_keys * 132, dtype=torch.uint8, device="cuda")
+    buf1 = torch.empty_like(buf0)
+    cs = torch.cuda.Stream() if use_copy_stream else None
+    idx, val = L.ls_prefill_select_stream_fp8(q8, qs, w, qp, hk, hs, buf0, buf1, k=wl.k, stride=wl.stride,
+                                              tile_keys=wl.tile_keys, full_scores=full_scores, copy_stream=cs)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), val.cpu().numpy()
+
+
+def test_fp8_scores(L):
+    """Every (query, key) score of a 77-query chunk (a partial last group of 8)
+    against 1019 keys (a ragged last tile): within the fp8 tolerance and, since
+    the kernel sums exact code products in fp32, within the bf16 one too;
+    ineligible keys hold -inf."""
+    wl = get_workload("prefill_fp8_s")
+    d = data("prefill_fp8_s")
+    T, H, dd = d["q8"].shape
+    N = d["k8"].shape[0]
+    sc = L.ls_indexer_score_fp8(dev(d["q8"])[None], dev(d["q_scale"])[None], dev(d["w"])[None],
+                                dev(d["k8"])[None], dev(d["k_scale"])[None], q_pos=dev(d["q_pos"])[None],
+                                stride=wl.stride)[0].cpu().numpy()
+    n_t = eligible_count(d["q_pos"], wl.stride, N)
+    for t in range(T):
+        n = int(n_t[t])
+        ref = _fp8_ref(d, t, n)
+        check_scores(sc[t, :n], ref, RTOL_FP8, f"fp8 scores t={t}")
+        check_scores(sc[t, :n], ref, RTOL_BF16, f"fp8 scores (fp32 sums) t={t}")
+        assert np.all(np.isneginf(sc[t, n:]))
+
+
+def test_fp8_scores_batched_n_valid(L):
+    """Several problems in one call (B = 3, one query each and a group of 8),
+    n_valid cutting each problem's keys."""
+    d = data("prefill_fp8_s")
+    B, T, N = 3, 9, 300
+    rng = np.random.default_rng(5)
+    q8 = np.stack([d["q8"][rng.permutation(77)[:T]] for _ in range(B)])
+    qs = np.stack([d["q_scale"][:T]] * B)
+    w = np.stack([d["w"][b:b + T] for b in range(B)])
+    k8 = np.stack([d["k8"][b * 200:b * 200 + N] for b in range(B)])
+    ks = np.stack([d["k_scale"][b * 200:b * 200 + N] for b in range(B)])
+    nv = np.array([300, 129, 1], dtype=np.int32)
+    sc = L.ls_indexer_score_fp8(dev(q8), dev(qs), dev(w), dev(k8), dev(ks), n_valid=dev(nv)).cpu().numpy()
+    for b in range(B):
+        db = {"q8": q8[b], "q_scale": qs[b], "w": w[b], "k8": k8[b], "k_scale": ks[b]}
+        for t in range(T):
+            ref = _fp8_ref(db, t, int(nv[b]))
+            check_scores(sc[b, t, :nv[b]], ref, RTOL_FP8, f"fp8 batched b={b} t={t}")
+            assert np.all(np.isneginf(sc[b, t, nv[b]:]))
+
+
+def test_fp8_prefill_stream_small(L):
+    wl = get_workload("prefill_fp8_s")
+    d = data("prefill_fp8_s")
+    idx, val = _fp8_prefill_run(L, d, wl)
+    T = d["q8"].shape[0]
+    N = d["k8"].shape[0]
+    n_t = eligible_count(d["q_pos"], wl.stride, N)
+    for t in range(T):
+        n = int(n_t[t])
+        check_selection(idx[t], val[t], np.arange(n), _fp8_ref(d, t, n), wl.k, RTOL_FP8, f"fp8 prefill t={t}")
+    # the full-matrix form, a single stream, and scoring the resident history agree bit for bit
+    idx2, val2 = _fp8_prefill_run(L, d, wl, full_scores=True)
+    assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
+    idx3, val3 = _fp8_prefill_run(L, d, wl, use_copy_stream=False)
+    assert np.array_equal(idx3, idx) and f32_bits_equal(val3, val)
+    sc = L.ls_indexer_score_fp8(dev(d["q8"])[None], dev(d["q_scale"])[None], dev(d["w"])[None],
+                                dev(d["k8"])[None], dev(d["k_scale"])[None], q_pos=dev(d["q_pos"])[None],
+                                stride=wl.stride)[0]
+    ri, rv = L.ls_topk_select(sc, wl.k, n_valid=dev(n_t.astype(np.int32)))
+    assert np.array_equal(ri.cpu().numpy(), idx) and f32_bits_equal(rv.cpu().numpy(), val)
+
+
+@pytest.mark.parametrize("T,N,tile,k", [(1, 2000, 256, 64), (40, 2000, 256, 1100), (9, 300, 512, 32)])
+def test_fp8_prefill_stream_shapes(L, T, N, tile, k):
+    """One query (a group of 8 with 7 empty columns), k above 1024, a history
+    shorter than one tile: the running form, the full-matrix form and the
+    oracle agree."""
+    from types import SimpleNamespace
+    from workloads.synth import make_prefill
+    d = make_prefill(T, N, 4 * N - T - 37, seed=31, fp8=True)
+    wl = SimpleNamespace(k=k, stride=4, tile_keys=tile)
+    idx, val = _fp8_prefill_run(L, d, wl)
+    idx2, val2 = _fp8_prefill_run(L, d, wl, full_scores=True)
+    assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
+    n_t = eligible_count(d["q_pos"], 4, N)
+    for t in range(T):
+        n = int(n_t[t])
+        check_selection(idx[t], val[t], np.arange(n), _fp8_ref(d, t, n), k, RTOL_FP8,
+                        f"fp8 shape ({T},{N},{tile},{k}) t={t}")
+
+
+def test_fp8_prefill_stream_overflow(L):
+    """Rising scores overflow the candidate slots of half the queries (the
+    filter form's overflow path through the full tile); the rest score 0."""
+    from types import SimpleNamespace
+    from workloads.synth import quantize_e4m3_rows
+    T, H, dd, N, k, stride = 24, 32, 128, 1000, 32, 4
+    rng = np.random.default_rng(7)
+    u = rng.standard_normal(dd)
+    u /= np.linalg.norm(u)
+    alpha = np.linspace(0.05, 1.0, N)
+    k8, ks = quantize_e4m3_rows(alpha[:, None] * u[None, :])
+    sign = np.where(np.arange(T) < T // 2, 1.0, -1.0)
+    q8, qs = quantize_e4m3_rows(np.broadcast_to(sign[:, None, None] * u[None, None, :], (T, H, dd)).copy())
+    w = (np.abs(rng.standard_normal((T, H))) + 0.1).astype(np.float32)
+    q_pos = (stride * N - 1 - rng.integers(0, 300, size=T)).astype(np.int64)
+    d = {"q8": q8, "q_scale": qs, "w": w, "k8": k8, "k_scale": ks, "q_pos": q_pos}
+    wl = SimpleNamespace(k=k, stride=stride, tile_keys=128)
+    idx, val = _fp8_prefill_run(L, d, wl)
+    idx2, val2 = _fp8_prefill_run(L, d, wl, full_scores=True)
+    assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
+    n_t = eligible_count(q_pos, stride, N)
+    for t in range(T):
+        n = int(n_t[t])
+        check_selection(idx[t], val[t], np.arange(n), _fp8_ref(d, t, n), k, RTOL_FP8, f"fp8 overflow t={t}")
+
+
+@pytest.mark.slow
+def test_fp8_prefill_chunk_full_size_sampled(L):
+    wl = get_workload("prefill_chunk_fp8")
+    d = data("prefill_chunk_fp8")
+    idx, val = _fp8_prefill_run(L, d, wl)
+    idx2, val2 = _fp8_prefill_run(L, d, wl, full_scores=True)
+    assert np.array_equal(idx2, idx) and f32_bits_equal(val2, val)
+    N = d["k8"].shape[0]
+    n_t = eligible_count(d["q_pos"], wl.stride, N)
+    for t in (0, 1, 7, 8, 1023, 2048, 4093, 4094, 4095):
+        n = int(n_t[t])
+        check_selection(idx[t], val[t], np.arange(n), _fp8_ref(d, t, n), wl.k, RTOL_FP8, f"fp8 prefill t={t}")
+
+
+# --------------------------------------------------------------------------- #
 # two-stage decode search
 # --------------------------------------------------------------------------- #
 def _check_two_stage(L, name, rows):

@@ -17,7 +17,7 @@ from oracle import brute, sizes
 from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64, f16_to_f64, pq_decode
 from oracle.indexer import eligible_blocks, eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, decode_select, expand_buckets, prefill_select, recall_at_k, select_topk,
+    bucket_select, decode_select, expand_buckets, prefill_select, prefill_select_fp8, recall_at_k, select_topk,
     topk_rows, two_stage_pq_select, two_stage_select,
 )
 from workloads import make_workload
@@ -300,6 +300,71 @@ def test_prefill_select_brute_force_tiny():
         sc = [brute.score(bf16_to_f64(q[t]).tolist(), w[t].astype(np.float64).tolist(), kf[s]) for s in elig]
         bp, bv = brute.topk(sc, elig, 16)
         assert idx[t].tolist() == bp
+
+
+def _e4m3_code_of_int(v: int) -> int:
+    """The e4m3 code of an integer |v| <= 15, built from the field layout
+    (sign, exponent biased by 7, 3 mantissa bits)."""
+    v = int(v)
+    s = 0x80 if v < 0 else 0
+    a = abs(v)
+    if a == 0:
+        return s
+    e = a.bit_length() - 1
+    m = ((a - (1 << e)) * 8) >> e
+    return s | ((e + 7) << 3) | m
+
+
+def test_prefill_select_fp8_integer_codes_brute_force():
+    """fp8 codes of small integers with power-of-two scales: every product and
+    sum is exact in fp64, so the oracle's scores equal a pure-Python brute
+    force exactly; a scale applied to the wrong axis changes them."""
+    rng = np.random.default_rng(11)
+    T, H, d, N = 5, 3, 8, 40
+    qi = rng.integers(-15, 16, size=(T, H, d))
+    ki = rng.integers(-15, 16, size=(N, d))
+    q8 = np.vectorize(_e4m3_code_of_int)(qi).astype(np.uint8)
+    k8 = np.vectorize(_e4m3_code_of_int)(ki).astype(np.uint8)
+    assert np.array_equal(e4m3_to_f64(q8), qi) and np.array_equal(e4m3_to_f64(k8), ki)
+    qs = np.exp2(rng.integers(-3, 4, size=(T, H))).astype(np.float32)
+    ks = np.exp2(rng.integers(-3, 4, size=N)).astype(np.float32)
+    w = rng.standard_normal((T, H)).astype(np.float32)
+    q_pos = np.array([3, 40, 99, 150, 159], dtype=np.int64)
+    idx, val, scores = prefill_select_fp8(q8, qs, w, q_pos, k8, ks, stride=4, k=8, return_scores=True)
+    for t in range(T):
+        n = min((int(q_pos[t]) + 1) // 4, N)
+        qt = [[float(qi[t, h, j]) * float(qs[t, h]) for j in range(d)] for h in range(H)]
+        ref = [brute.score(qt, [float(x) for x in w[t]], [float(ki[s, j]) * float(ks[s]) for j in range(d)])
+               for s in range(n)]
+        assert scores[t].tolist() == ref
+        bp, _ = brute.topk(ref, list(range(n)), 8)
+        assert idx[t].tolist() == bp
+
+
+def test_prefill_select_fp8_equals_bf16_pipeline():
+    """Every e4m3 value times a power of two is a bf16 value: the fp8
+    selection must equal the bf16 selection of the decoded inputs."""
+    d = make_workload("prefill_fp8_s")
+    rows = np.array([0, 5, 40, 76])
+    qs = np.exp2(np.round(np.log2(d["q_scale"]))).astype(np.float32)
+    ks = np.exp2(np.round(np.log2(d["k_scale"]))).astype(np.float32)
+    qb = to_bf16_bits(e4m3_to_f64(d["q8"]) * qs[..., None])
+    kb = to_bf16_bits(e4m3_to_f64(d["k8"]) * ks[:, None])
+    assert np.array_equal(bf16_to_f64(qb), e4m3_to_f64(d["q8"]) * qs[..., None].astype(np.float64))
+    i8, v8 = prefill_select_fp8(d["q8"], qs, d["w"], d["q_pos"], d["k8"], ks, stride=4, k=64, rows=rows)
+    ib, vb = prefill_select(qb, d["w"], d["q_pos"], kb, stride=4, k=64, rows=rows)
+    assert np.array_equal(i8, ib) and np.array_equal(v8, vb)
+
+
+def test_fp8_prefill_generator_scales():
+    """The fp8 inputs are the bf16 draws quantised per row: scale = amax / 448
+    and every decoded value within half an e4m3 step of the original."""
+    d = make_workload("prefill_fp8_s")
+    qf = bf16_to_f64(d["q"])
+    amax = np.abs(qf).max(axis=-1)
+    assert np.allclose(d["q_scale"], (amax / 448.0).astype(np.float32))
+    deq = e4m3_to_f64(d["q8"]) * d["q_scale"].astype(np.float64)[..., None]
+    assert np.all(np.abs(deq - qf) <= np.abs(qf) * 2.0 ** -4 + d["q_scale"][..., None] * 2.0 ** -9)
 
 
 def test_two_stage_full_shortlist_equals_exact():

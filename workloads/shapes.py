@@ -9,6 +9,10 @@ Five full-size workloads follow the shapes the pages use:
   126976..131071 against 131072 history tokens (32768 positions), history
   streamed in 8192-key tiles through two device buffers (LeanSparse podcast
   transcript, 05:36-06:44).
+* ``prefill_chunk_fp8`` -- the same chunk with fp8 e4m3 queries (one scale
+  per query head) and an fp8 history (one scale per key), quantised from the
+  same draws: the indexer's FP8 form ("03 long context" lecture, section
+  "Sparsity Is a Systems Feature: The Blast Radius", kernel layer).
 * ``two_stage``     -- 32 sequences x 524288 tokens (131072 positions each):
   compact int8 scan, 4096-entry shortlist, exact re-rank of fp8 originals
   (LeanSparse podcast transcript, 07:12-08:00).
@@ -78,6 +82,12 @@ WORKLOADS: Dict[str, Workload] = {
     "prefill_chunk": Workload(
         "prefill_chunk", "prefill", T=4096, q_pos0=126976, N=32768, stride=4, tile_keys=8192
     ),
+    # the same chunk with fp8 queries (one scale per query head) and an fp8
+    # history (one scale per key): the indexer's FP8 form
+    "prefill_chunk_fp8": Workload(
+        "prefill_chunk_fp8", "prefill", T=4096, q_pos0=126976, N=32768, stride=4, tile_keys=8192,
+        extra={"fp8": 1},
+    ),
     "two_stage": Workload(
         "two_stage", "two_stage", B=32, N=131072, shortlist=4096, plant_frac=0.05, plant_cos=0.6
     ),
@@ -94,6 +104,9 @@ WORKLOADS: Dict[str, Workload] = {
     "decode_s": Workload("decode_s", "decode", B=5, N=3000, ragged=700),
     "prefill_s": Workload(
         "prefill_s", "prefill", T=77, q_pos0=4000, N=1019, stride=4, tile_keys=256
+    ),
+    "prefill_fp8_s": Workload(
+        "prefill_fp8_s", "prefill", T=77, q_pos0=4000, N=1019, stride=4, tile_keys=256, extra={"fp8": 1}
     ),
     "two_stage_s": Workload(
         "two_stage_s", "two_stage", B=3, N=9000, shortlist=1024, plant_frac=0.05, plant_cos=0.6, ragged=1500

@@ -136,9 +136,21 @@ def make_decode(
 # --------------------------------------------------------------------------- #
 # prefill: T queries at consecutive token positions, one history of N keys
 # --------------------------------------------------------------------------- #
+def quantize_e4m3_rows(x: np.ndarray):
+    """Rows of x (last axis) -> (e4m3 codes, fp32 scales): scale = amax / 448
+    per row (1.0 for an all-zero row), codes = e4m3(x / scale)."""
+    x = np.asarray(x, dtype=np.float64)
+    amax = np.abs(x).max(axis=-1)
+    sc = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32)
+    return to_e4m3_codes(x / sc.astype(np.float64)[..., None]), sc
+
+
 def make_prefill(
-    T: int, N: int, q_pos0: int, H: int = 32, d: int = 128, seed: int = 0
+    T: int, N: int, q_pos0: int, H: int = 32, d: int = 128, seed: int = 0, fp8: bool = False
 ) -> Dict[str, np.ndarray]:
+    """bf16 queries and history; with fp8 also their e4m3 forms (q8 with one
+    scale per (query, head), k8 with one scale per key) quantised from the
+    same values."""
     rng = np.random.default_rng(seed)
     q = to_bf16_bits(_normal(rng, (T, H, d), 1.0 / math.sqrt(d)))
     w = _normal(rng, (T, H), 1.0 / math.sqrt(H)).astype(np.float32)
@@ -148,7 +160,11 @@ def make_prefill(
         e = min(N, s + step)
         k[s:e] = to_bf16_bits(_normal(rng, (e - s, d), 1.0 / math.sqrt(d)))
     q_pos = (q_pos0 + np.arange(T)).astype(np.int64)
-    return {"q": q, "w": w, "k": k, "q_pos": q_pos}
+    out = {"q": q, "w": w, "k": k, "q_pos": q_pos}
+    if fp8:
+        out["q8"], out["q_scale"] = quantize_e4m3_rows(bf16_bits_to_f32(q))
+        out["k8"], out["k_scale"] = quantize_e4m3_rows(bf16_bits_to_f32(k))
+    return out
 
 
 # --------------------------------------------------------------------------- #
@@ -288,7 +304,7 @@ def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
     if wl.kind == "decode":
         return make_decode(wl.B, wl.N, wl.H, wl.d, s, ragged=wl.ragged)
     if wl.kind == "prefill":
-        return make_prefill(wl.T, wl.N, wl.q_pos0, wl.H, wl.d, s)
+        return make_prefill(wl.T, wl.N, wl.q_pos0, wl.H, wl.d, s, fp8=bool(wl.extra.get("fp8", 0)))
     if wl.kind == "two_stage":
         return make_two_stage(wl.B, wl.N, wl.H, wl.d, s, wl.plant_frac, wl.plant_cos, ragged=wl.ragged,
                               pq=bool(wl.extra.get("pq", 0)))
