@@ -338,7 +338,7 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
                      ("prefill_chunk_running", lambda *a: bench_prefill(*a, full_scores=False)),
                      ("prefill_chunk_fp8", lambda *a: bench_prefill(*a, fp8=True)),
                      ("prefill_chunk_fp8_running", lambda *a: bench_prefill(*a, full_scores=False, fp8=True)),
-                     ("bucket", bench_bucket), ("two_stage", bench_two_stage),
+                     ("bucket", bench_bucket), ("lsa_flat", bench_lsa), ("two_stage", bench_two_stage),
                      ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True))):
         if only in (None, name):
             res[name] = fn(L, args, peaks, peak_kind)
@@ -468,6 +468,47 @@ def bench_bucket(L, args, peaks, peak_kind):
     return res
 
 
+def bench_lsa(L, args, peaks, peak_kind):
+    """Native LSA flat search: 256 index queries over 131072 buckets of one
+    1048576-token sequence; top 1024 buckets, 4096 long-range keys."""
+    import torch
+    from workloads import get_workload, make_workload
+    st = torch.cuda.current_stream()
+    steps = max(3, args.steps)
+    warm = max(3, args.warmup)
+    wl = get_workload("lsa_flat")
+    d = make_workload(wl)
+    ex = wl.extra
+    T = d["q_idx"].shape[0]
+    P_ = d["centroids"].shape[0]
+    a = [to_dev_bf16(d["q_idx"]), to_dev(d["q_pos"]), to_dev_bf16(d["centroids"]), to_dev(d["bucket_off"]),
+         to_dev(d["bucket_mem"])]
+    ws = torch.empty(L.lib().ls_lsa_flat_workspace_size(T, P_, wl.top_p), dtype=torch.uint8, device="cuda")
+    row = ex["n_sink"] + ex["block_keys"] + wl.budget
+    out = (torch.empty((T, row), dtype=torch.int32, device="cuda"), torch.empty((T,), dtype=torch.int32, device="cuda"))
+
+    def run(i, timed):
+        L.ls_lsa_flat_select(*a, block_keys=ex["block_keys"], buckets_per_block=ex["bpb"], n_sink=ex["n_sink"],
+                             top_p=wl.top_p, budget=wl.budget, ws=ws, out=out)
+        return None
+
+    ms, kern = _profiled_loop(L, run, steps, warm, st)
+    dms = kern["dot_tc_kernel"]["ms_per_step"]
+    vis = np.minimum((d["q_pos"] // ex["block_keys"]) * ex["bpb"], P_)
+    scored = int(vis.sum())
+    bytes_dot = P_ * 128 + T * 128 + T * P_ * 4
+    peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    res = {"ms_per_step": ms, "positions_per_s": scored / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
+           "kernels": kern,
+           "roofline": roofline("hbm", bytes_dot / (dms * 1e-3) / 1e9, peak_b, "GB/s",
+                                traffic=ncu_traffic("dot_tc_kernel", wl.name), peak_kind=peak_kind),
+           "bytes_dot": bytes_dot, "visible_buckets_scored": scored,
+           "note": "positions = visible buckets scored per query (one 64-d dot each); roofline of the bucket "
+                   "scoring: centroids + queries read, the T x P score matrix written"}
+    del a, ws
+    return res
+
+
 def bench_two_stage(L, args, peaks, peak_kind, pq=False):
     """Two-stage decode search: compact scan (int8 + scale, or 32-byte PQ codes), shortlist, exact re-rank."""
     import torch
@@ -585,8 +626,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="decode_batch")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "prefill_chunk_fp8",
-                                                     "prefill_chunk_fp8_running", "bucket", "two_stage",
-                                                     "two_stage_pq"],
+                                                     "prefill_chunk_fp8_running", "bucket", "lsa_flat",
+                                                     "two_stage", "two_stage_pq"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

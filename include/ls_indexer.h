@@ -256,6 +256,44 @@ ls_status ls_prefill_select_stream_fp8(const uint8_t* q8, const float* q_scale, 
                                        void* compute_stream, void* copy_stream);
 
 /*
+ * ls_lsa_flat_select -- the native LSA flat search ("Latent Sparse
+ * Attention", sections "How LSA finds the keys" and "The method, term by
+ * term", steps 5-6): a query scores the unit centroid of every bucket of
+ * the blocks before its own with one 64-d dot product, keeps the best top_p
+ * buckets and reads them best first until it holds `budget` long-range keys,
+ * plus the sink keys and the window (its own, not yet clustered block).
+ *
+ *   q_idx      [T][64] bf16 index queries (unit vectors; the projection that
+ *              makes them is the caller's)
+ *   q_pos      [T] int64 token positions
+ *   centroids  [P][64] bf16 unit centroids, block-major: the buckets of key
+ *              block j (positions [j*block_keys, (j+1)*block_keys)) are
+ *              [j*buckets_per_block, (j+1)*buckets_per_block)
+ *   bucket_off [P+1] int32, bucket_mem [bucket_off[P]] int32: bucket p's
+ *              member positions, ascending, in bucket_mem[off[p] .. off[p+1])
+ *   n_sink     sink keys (positions 0 .. n_sink-1), block_keys the window
+ *   keys_out   [T][n_sink + block_keys + budget] int32: per query, the sinks
+ *              below its window, the window [block_start, t], then the
+ *              long-range keys in read order (members that fall in the sinks
+ *              or the window skipped, the last bucket cut short); -1 after
+ *              n_out[t] entries
+ *   n_out      [T] int32 entries per row
+ *   picked_out [T][top_p] int32 picked buckets, best first (or NULL); -1
+ *              where fewer than top_p buckets are visible
+ * Visible buckets of a query at position t: the first
+ * min(P, buckets_per_block * floor(t / block_keys)).  Bucket order: score
+ * descending, then bucket id ascending.  Only d = 64 is built.
+ * Workspace: ls_lsa_flat_workspace_size(T, P, top_p) bytes (a T x P score
+ * matrix among them).
+ */
+size_t ls_lsa_flat_workspace_size(int T, int P, int top_p);
+ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
+                             const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
+                             int block_keys, int buckets_per_block, int n_sink, int top_p, int budget,
+                             int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/*
  * ls_decode_two_stage_select -- LeanSparse two-stage decode search
  * (podcast transcript, 07:12-08:00): scan compact keys, keep a shortlist,
  * fetch the shortlist's original keys and re-rank exactly, keep the top k.

@@ -24,6 +24,13 @@ Pipelines:
 * two-stage decode search (LeanSparse podcast transcript, 07:12-08:00): scores
   from compact keys, keep a shortlist, score the shortlist's original keys
   exactly, keep the top k of those.
+* native LSA flat search ("Latent Sparse Attention", "How LSA finds the keys"
+  and "The method, term by term", steps 5-6): score the unit centroid of
+  every bucket of the blocks before the query's own with one 64-d dot
+  product, keep the top-p buckets, read them best first skipping members
+  that fall in the sinks or the window until the budget is held (the last
+  bucket cut short); the read list is the sinks, the window (the query's own
+  block up to the query) and those long-range keys.
 * bucket search ("Latent Sparse Attention", "How LSA finds the keys" and "The
   method, term by term", steps 5-6): score every bucket centroid with the
   indexer score, keep the top-p buckets, read them best first appending their
@@ -209,6 +216,58 @@ def bucket_select(q_bits, w, centroids, bucket_off, bucket_mem, key_bits, top_p:
     if return_detail:
         return idx, val, detail
     return idx, val
+
+
+def lsa_visible(q_pos, block_keys: int, buckets_per_block: int, n_buckets: int) -> np.ndarray:
+    """Buckets a query sees: those of the complete blocks before its own."""
+    q_pos = np.maximum(np.asarray(q_pos, dtype=np.int64), 0)
+    return np.minimum((q_pos // block_keys) * buckets_per_block, n_buckets)
+
+
+def lsa_read_list(picked, pos: int, bucket_off, bucket_mem, block_keys: int, n_sink: int, budget: int) -> np.ndarray:
+    """The keys a query at position ``pos`` reads, given its picked buckets in
+    pick order: the sinks below its window, the window (its own block up to
+    ``pos``), then the picked buckets' members in pick order and stored order,
+    members that fall in the sinks or the window skipped, until ``budget``
+    long-range keys are held."""
+    pos = max(int(pos), 0)
+    wstart = (pos // block_keys) * block_keys
+    sinks = [s for s in range(n_sink) if s < wstart]
+    window = list(range(wstart, pos + 1))
+    longr = []
+    for p in picked:
+        if p < 0 or len(longr) == budget:
+            break
+        for m in bucket_mem[bucket_off[p]: bucket_off[p + 1]]:
+            m = int(m)
+            if m < n_sink or m >= wstart:
+                continue
+            if len(longr) == budget:
+                break
+            longr.append(m)
+    return np.asarray(sinks + window + longr, dtype=np.int64)
+
+
+def lsa_flat_select(q_idx_bits, q_pos, centroid_bits, bucket_off, bucket_mem, block_keys: int,
+                    buckets_per_block: int, n_sink: int, top_p: int, budget: int, rows=None,
+                    return_detail: bool = False):
+    """Read lists of the native LSA flat search, one per query (``rows``,
+    default all)."""
+    T = q_idx_bits.shape[0]
+    P = centroid_bits.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    cent = bf16_to_f64(centroid_bits)
+    vis = lsa_visible(q_pos, block_keys, buckets_per_block, P)
+    out, detail = [], []
+    for t in rows:
+        v = int(vis[t])
+        scores = cent[:v] @ bf16_to_f64(q_idx_bits[t])          # one dot product per visible bucket
+        picked, _ = select_topk(scores, np.arange(v), top_p)
+        out.append(lsa_read_list(picked, q_pos[t], bucket_off, bucket_mem, block_keys, n_sink, budget))
+        detail.append({"scores": scores, "picked": picked, "visible": v})
+    if return_detail:
+        return out, detail
+    return out
 
 
 def recall_at_k(sel: np.ndarray, ref: np.ndarray) -> float:

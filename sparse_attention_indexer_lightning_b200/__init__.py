@@ -21,6 +21,7 @@ from ._lib import (  # noqa: F401
     ls_indexer_score,
     ls_indexer_score_fp8,
     ls_indexer_score_pq,
+    ls_lsa_flat_select,
     ls_prefill_select_stream,
     ls_prefill_select_stream_fp8,
     ls_profile_begin,

@@ -18,6 +18,7 @@
 #include "ls_indexer.h"
 #include "misc.cuh"
 #include "score_cvt.cuh"
+#include "score_dot.cuh"
 #include "score_q8.cuh"
 #include "score_tc.cuh"
 #include "topk.cuh"
@@ -187,6 +188,22 @@ ls_status score_tc_launch(const uint16_t* q, const uint16_t* keys, int B, int T,
   p.N = N;
   ProfScope prof(prof_name ? prof_name : qg == 1 ? "score_tc_kernel<1>" : "score_tc_kernel<8>", st);
   LS_CUDA(launch_score_tc(qg, &kmap, &qmap, p, num_sms_current(), st));
+  return LS_OK;
+}
+
+// 2-D map over [rows][64] bf16 vectors (128 bytes each: one swizzle row),
+// box = 64 x box_rows, 128-byte swizzle.
+ls_status make_vec64_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kLsaDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLsaDim * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kLsaDim), box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return LS_OK;
 }
 
@@ -895,6 +912,57 @@ ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* ce
     if (s != LS_OK) return s;
   }
   return topk(exact, budget, nullptr, cand, budget, T, budget, k, idx_out, val_out, k, st);
+}
+
+size_t ls_lsa_flat_workspace_size(int T, int P, int top_p) {
+  if (T <= 0 || top_p <= 0) return 0;
+  return align_up(static_cast<size_t>(T) * (P > 0 ? P : 0) * sizeof(float)) +   // bucket scores
+         align_up(static_cast<size_t>(T) * sizeof(int32_t)) +                  // visible buckets
+         align_up(static_cast<size_t>(T) * top_p * sizeof(int32_t));           // picked buckets
+}
+
+ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
+                             const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
+                             int block_keys, int buckets_per_block, int n_sink, int top_p, int budget,
+                             int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (d != kLsaDim) return fail(LS_ERR_UNSUPPORTED, "only d=%d is built for the LSA index space (got %d)", kLsaDim, d);
+  LS_CHECK_ARG(T >= 0 && P >= 0, "negative size");
+  LS_CHECK_ARG(block_keys >= 1 && buckets_per_block >= 1, "block_keys and buckets_per_block must be >= 1");
+  LS_CHECK_ARG(n_sink >= 0 && budget >= 1, "n_sink must be >= 0 and budget >= 1");
+  LS_CHECK_ARG(top_p >= 1 && top_p <= kMaxTopK, "top_p must be in [1, %d] (got %d)", kMaxTopK, top_p);
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(q_pos && keys_out && n_out, "null tensor pointer");
+  const size_t need = ls_lsa_flat_workspace_size(T, P, top_p);
+  if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  Carver cv(ws);
+  float* sc = cv.take<float>(static_cast<size_t>(T) * P);
+  int32_t* vis = cv.take<int32_t>(T);
+  int32_t* picked_ws = cv.take<int32_t>(static_cast<size_t>(T) * top_p);
+  int32_t* picked = picked_out ? picked_out : picked_ws;
+  cudaStream_t st = S(stream);
+  {
+    ProfScope prof("lsa_visible_kernel", st);
+    LS_CUDA(launch_lsa_visible(q_pos, T, block_keys, buckets_per_block, P, vis, st));
+  }
+  if (P > 0) {
+    LS_CHECK_ARG(q_idx && centroids && bucket_off && bucket_mem, "null tensor pointer");
+    LS_CHECK_ARG(aligned16(q_idx) && aligned16(centroids), "q_idx and centroids must be 16-byte aligned");
+    CUtensorMap cmap, qmap;
+    ls_status s = make_vec64_map(&cmap, centroids, static_cast<uint64_t>(P), kTileKeys);
+    if (s != LS_OK) return s;
+    s = make_vec64_map(&qmap, q_idx, static_cast<uint64_t>(T), DotCfg::QB);
+    if (s != LS_OK) return s;
+    ProfScope prof("dot_tc_kernel", st);
+    LS_CUDA(launch_dot_tc(&cmap, &qmap, T, P, sc, P, num_sms_current(), st));
+  }
+  // top-p of each row's visible prefix (padding -1 where fewer are visible)
+  ls_status s = topk(sc, P, vis, nullptr, 0, T, P, top_p, picked, nullptr, top_p, st);
+  if (s != LS_OK) return s;
+  ProfScope prof("lsa_expand_kernel", st);
+  LS_CUDA(launch_lsa_expand(picked, q_pos, T, top_p, bucket_off, bucket_mem, P, block_keys, n_sink, budget, keys_out,
+                            n_sink + block_keys + budget, n_out, st));
+  return LS_OK;
 }
 
 ls_status ls_profile_begin(void) {

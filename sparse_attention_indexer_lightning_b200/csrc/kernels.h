@@ -12,6 +12,7 @@ constexpr int kHeads = 32;   // indexer heads built
 constexpr int kDim = 128;    // indexer key / query width
 constexpr int kTileKeys = 128;
 constexpr int kMaxTopK = 4096;
+constexpr int kLsaDim = 64;    // native LSA index space width
 
 // ---------------------------------------------------------------- scoring
 // Tensor-core scoring of bf16 keys read by TMA.  One launch covers B
@@ -68,6 +69,19 @@ cudaError_t launch_score_tc_f8(const CUtensorMap* kmap, const CUtensorMap* qmap,
                                cudaStream_t st);
 // out[i] = w[i] * qs[i], i < n.
 cudaError_t launch_fold_scales(const float* w, const float* qs, int64_t n, float* out, cudaStream_t st);
+
+// Native LSA flat search: out[t][p] = q[t] . c[p] over 64-d bf16 vectors
+// (cmap over the centroids [P][128 B], qmap over the index queries [T][128 B]).
+cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, int T, int P, float* out, int64_t ld_out,
+                          int num_sms, cudaStream_t st);
+// vis[t] = min(P, bpb * floor(q_pos[t] / block_keys)).
+cudaError_t launch_lsa_visible(const int64_t* q_pos, int T, int block_keys, int bpb, int P, int32_t* vis,
+                               cudaStream_t st);
+// The read list of each query: sinks below its window, the window, then the
+// picked buckets' members best first (sinks and window skipped) up to budget.
+cudaError_t launch_lsa_expand(const int32_t* picked, const int64_t* q_pos, int T, int top_p, const int32_t* off,
+                              const int32_t* mem, int P, int block_keys, int n_sink, int budget, int32_t* keys_out,
+                              int row_len, int32_t* n_out, cudaStream_t st);
 
 // Source rows for the converting scorer.
 enum SrcFormat : int { SRC_INT8 = 0, SRC_E4M3 = 1, SRC_BF16 = 2, SRC_PQ = 3 };

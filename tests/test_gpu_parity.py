@@ -14,7 +14,8 @@ import torch
 from oracle.formats import bf16_to_f64, dequant, pq_decode
 from oracle.indexer import eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, expand_buckets, recall_at_k, select_topk, topk_rows, two_stage_pq_select, two_stage_select,
+    bucket_select, expand_buckets, lsa_flat_select, lsa_read_list, recall_at_k, select_topk, topk_rows,
+    two_stage_pq_select, two_stage_select,
 )
 from parity_util import (
     RTOL_BF16, RTOL_FP8, check_scores, check_selection, check_set, dev, dev_bf16, dev_e4m3, f32_bits_equal,
@@ -554,6 +555,44 @@ def test_bucket_small(L):
 def test_bucket_full_size_sampled(L):
     rec = _check_bucket(L, "bucket", [0, 100, 255])
     assert min(rec) > 0.3
+
+
+# --------------------------------------------------------------------------- #
+# native LSA flat search
+# --------------------------------------------------------------------------- #
+def _check_lsa(L, name, rows):
+    wl = get_workload(name)
+    d = data(name)
+    ex = wl.extra
+    keys, n, picked = L.ls_lsa_flat_select(dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]),
+                                           dev(d["bucket_off"]), dev(d["bucket_mem"]), block_keys=ex["block_keys"],
+                                           buckets_per_block=ex["bpb"], n_sink=ex["n_sink"], top_p=wl.top_p,
+                                           budget=wl.budget, want_picked=True)
+    keys, n, picked = keys.cpu().numpy(), n.cpu().numpy(), picked.cpu().numpy()
+    _, det = lsa_flat_select(d["q_idx"], d["q_pos"], d["centroids"], d["bucket_off"], d["bucket_mem"],
+                             ex["block_keys"], ex["bpb"], ex["n_sink"], wl.top_p, wl.budget, rows=rows,
+                             return_detail=True)
+    for i, t in enumerate(rows):
+        v = det[i]["visible"]
+        sc = det[i]["scores"]
+        check_set(picked[t], np.arange(v), sc, wl.top_p, RTOL_BF16, f"{name} picked row {t}")
+        got = picked[t][picked[t] >= 0]
+        # best first by the reference scores, up to the tolerance
+        gs = sc[got]
+        assert np.all(gs[:-1] >= gs[1:] - RTOL_BF16 * max(1e-3, float(np.abs(sc).max(initial=0)))), t
+        want = lsa_read_list(picked[t], d["q_pos"][t], d["bucket_off"], d["bucket_mem"], ex["block_keys"],
+                             ex["n_sink"], wl.budget)
+        assert n[t] == want.size and np.array_equal(keys[t, :n[t]], want), f"{name} read list row {t}"
+        assert np.all(keys[t, n[t]:] == -1)
+
+
+def test_lsa_flat_small(L):
+    _check_lsa(L, "lsa_flat_s", list(range(37)))
+
+
+@pytest.mark.slow
+def test_lsa_flat_full_size_sampled(L):
+    _check_lsa(L, "lsa_flat", [0, 1, 100, 254, 255])
 
 
 def test_bucket_bad_member_flagged(L):

@@ -17,8 +17,8 @@ from oracle import brute, sizes
 from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64, f16_to_f64, pq_decode
 from oracle.indexer import eligible_blocks, eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, decode_select, expand_buckets, prefill_select, prefill_select_fp8, recall_at_k, select_topk,
-    topk_rows, two_stage_pq_select, two_stage_select,
+    bucket_select, decode_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_visible, prefill_select,
+    prefill_select_fp8, recall_at_k, select_topk, topk_rows, two_stage_pq_select, two_stage_select,
 )
 from workloads import make_workload
 from workloads.synth import make_bucket, make_decode, make_two_stage, to_bf16_bits
@@ -365,6 +365,71 @@ def test_fp8_prefill_generator_scales():
     assert np.allclose(d["q_scale"], (amax / 448.0).astype(np.float32))
     deq = e4m3_to_f64(d["q8"]) * d["q_scale"].astype(np.float64)[..., None]
     assert np.all(np.abs(deq - qf) <= np.abs(qf) * 2.0 ** -4 + d["q_scale"][..., None] * 2.0 ** -9)
+
+
+def test_lsa_visibility_by_blocks():
+    """A bucket is visible iff its whole block ends at or before the start of
+    the query's own block (brute force over blocks)."""
+    block_keys, bpb, P = 16, 3, 3 * 7
+    for t in range(0, 16 * 9):
+        wstart = (t // block_keys) * block_keys
+        vis = [p for p in range(P) if (p // bpb + 1) * block_keys <= wstart]
+        assert lsa_visible([t], block_keys, bpb, P)[0] == len(vis)
+        assert vis == list(range(len(vis)))
+
+
+def test_lsa_dot_equals_two_head_indexer_score():
+    """The single dot product is the indexer score with heads q and -q,
+    weights 1 and -1: max(0, x) - max(0, -x) = x."""
+    d = make_workload("lsa_flat_s")
+    q = bf16_to_f64(d["q_idx"][:5])
+    c = bf16_to_f64(d["centroids"][:300])
+    qq = np.stack([q, -q], axis=1)                       # [5, 2, 64]
+    w = np.tile(np.array([1.0, -1.0]), (5, 1))
+    assert np.allclose(indexer_scores(qq, w, c), q @ c.T, rtol=0, atol=1e-15)
+    _, det = lsa_flat_select(d["q_idx"], d["q_pos"], d["centroids"], d["bucket_off"], d["bucket_mem"], 512, 64, 4,
+                             64, 512, rows=[11], return_detail=True)
+    assert np.allclose(det[0]["scores"], indexer_scores(np.stack([bf16_to_f64(d["q_idx"][11]),
+                                                                  -bf16_to_f64(d["q_idx"][11])])[None],
+                                                        np.array([[1.0, -1.0]]), bf16_to_f64(d["centroids"]))[0],
+                       rtol=0, atol=1e-15)
+
+
+def test_lsa_read_list_covers_history_with_full_budget():
+    """With every visible bucket picked and an unlimited budget, the read list
+    is exactly the positions 0 .. t, each once."""
+    d = make_workload("lsa_flat_s")
+    for t in (0, 3, 4, 511, 512, 1024, 5000, 39999):
+        qpos = d["q_pos"].copy()
+        qpos[0] = t
+        out = lsa_flat_select(d["q_idx"], qpos, d["centroids"], d["bucket_off"], d["bucket_mem"], 512, 64,
+                              4, 4096, 10 ** 6, rows=[0])[0]
+        if t // 512 * 64 <= 4096:
+            assert sorted(out.tolist()) == list(range(t + 1)), t
+
+
+def test_lsa_brute_force_tiny():
+    """Pure-Python dot products and a full sort pick the buckets; the read
+    list of the picked order is rebuilt by hand."""
+    d = make_workload("lsa_flat_s")
+    t = 5000
+    v = (t // 512) * 64
+    cent = bf16_to_f64(d["centroids"]).tolist()
+    q = bf16_to_f64(d["q_idx"][20:21])[0].tolist()
+    scores = [sum(a * b for a, b in zip(cent[p], q)) for p in range(v)]
+    bp, _ = brute.topk(scores, list(range(v)), 16)
+    qpos = d["q_pos"].copy()
+    qpos[20] = t
+    out, det = lsa_flat_select(d["q_idx"], qpos, d["centroids"], d["bucket_off"], d["bucket_mem"], 512, 64, 4, 16,
+                               100, rows=[20], return_detail=True)
+    assert det[0]["picked"].tolist() == bp
+    want = [0, 1, 2, 3] + list(range(4608, 5001))
+    for p in bp:
+        for m in d["bucket_mem"][d["bucket_off"][p]:d["bucket_off"][p + 1]]:
+            if 4 <= m < 4608 and len(want) < 4 + 393 + 100:
+                want.append(int(m))
+    assert out[0].tolist() == want
+    assert lsa_read_list(bp, t, d["bucket_off"], d["bucket_mem"], 512, 4, 100).tolist() == want
 
 
 def test_two_stage_full_shortlist_equals_exact():

@@ -16,6 +16,11 @@ Five full-size workloads follow the shapes the pages use:
 * ``two_stage``     -- 32 sequences x 524288 tokens (131072 positions each):
   compact int8 scan, 4096-entry shortlist, exact re-rank of fp8 originals
   (LeanSparse podcast transcript, 07:12-08:00).
+* ``lsa_flat``      -- the native LSA flat search over one sequence of
+  1048576 tokens: 131072 buckets (64 per 512-key block) with 64-d unit
+  centroids, 256 index queries, top 1024 buckets expanded to 4096 long-range
+  keys plus 4 sinks and the window ("Latent Sparse Attention", "How LSA finds
+  the keys").
 * ``bucket``        -- one sequence of 1048576 tokens (262144 keys) built as
   32768 clusters of 8 keys; 256 decode queries keep 64 buckets and expand them
   to 512 keys ("Latent Sparse Attention", "How LSA finds the keys").
@@ -38,7 +43,7 @@ from typing import Dict
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str  # "decode" | "prefill" | "two_stage" | "bucket"
+    kind: str  # "decode" | "prefill" | "two_stage" | "bucket" | "lsa"
     H: int = 32
     d: int = 128
     k: int = 512
@@ -100,6 +105,14 @@ WORKLOADS: Dict[str, Workload] = {
     "bucket": Workload(
         "bucket", "bucket", T=256, clusters=32768, cluster_size=8, noise_rel=0.3, top_p=64, budget=512
     ),
+    # native LSA flat search: one sequence of 1048576 tokens (2048 blocks of
+    # 512 keys, 64 buckets each), 256 index queries at positions spread over
+    # its second half; top 1024 buckets, 4096 long-range keys, 4 sinks
+    # ("Latent Sparse Attention", "How LSA finds the keys")
+    "lsa_flat": Workload(
+        "lsa_flat", "lsa", T=256, N=1048576, top_p=1024, budget=4096,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "spread": 2053},
+    ),
     # ---- reduced parity cases: several tiles, ragged tails ------------------
     "decode_s": Workload("decode_s", "decode", B=5, N=3000, ragged=700),
     "prefill_s": Workload(
@@ -114,6 +127,10 @@ WORKLOADS: Dict[str, Workload] = {
     "two_stage_pq_s": Workload(
         "two_stage_pq_s", "two_stage", B=3, N=9000, shortlist=1024, plant_frac=0.05, plant_cos=0.6, ragged=1500,
         extra={"pq": 1},
+    ),
+    "lsa_flat_s": Workload(
+        "lsa_flat_s", "lsa", T=37, N=40000, top_p=64, budget=512,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "edge": 1},
     ),
     "bucket_s": Workload(
         "bucket_s", "bucket", T=19, clusters=1500, cluster_size=8, noise_rel=0.3, top_p=64, budget=512,

@@ -295,6 +295,56 @@ def make_bucket(
     }
 
 
+def make_lsa(
+    T: int, L: int, block_keys: int = 512, bpb: int = 64, seed: int = 0, spread: int = 2053, edge: bool = False,
+) -> Dict[str, np.ndarray]:
+    """Native LSA index for one sequence of L tokens and T index queries.
+
+    Complete blocks of ``block_keys`` keys, each cut into pools of 4
+    consecutive keys that are grouped into ``bpb`` buckets of 1..4 pools
+    (4..16 keys; the grouping stands in for the Ward merges, drawn at random
+    here), members stored in ascending position order (CSR ``bucket_off`` /
+    ``bucket_mem``, buckets block-major).  Centroids and index queries are
+    random 64-d unit vectors rounded to bf16.  Query positions: the last
+    token and every ``spread``-th token before it, or (``edge``) the block
+    edges 0, 3, 4, 511, 512, ... followed by random positions."""
+    rng = np.random.default_rng(seed)
+    dim = 64
+    n_pool = block_keys // 4
+    nb = L // block_keys
+    P = nb * bpb
+    off = np.zeros(P + 1, dtype=np.int64)
+    members = np.empty(nb * block_keys, dtype=np.int32)
+    at = 0
+    for j in range(nb):
+        sizes = np.full(bpb, n_pool // bpb)
+        for _ in range(3 * bpb // 4):
+            a, b = rng.integers(bpb, size=2)
+            if a != b and sizes[a] > 1 and sizes[b] < 4:
+                sizes[a] -= 1
+                sizes[b] += 1
+        perm = rng.permutation(n_pool)
+        cuts = np.concatenate([[0], np.cumsum(sizes)])
+        for i in range(bpb):
+            pools = np.sort(perm[cuts[i]:cuts[i + 1]])
+            pos = (j * block_keys + 4 * pools[:, None] + np.arange(4)[None, :]).reshape(-1)
+            members[at:at + pos.size] = pos
+            at += pos.size
+            off[j * bpb + i + 1] = at
+    c = rng.standard_normal((P, dim))
+    c /= np.linalg.norm(c, axis=1, keepdims=True)
+    q = rng.standard_normal((T, dim))
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    if edge:
+        fixed = [0, 3, 4, 511, 512, 513, 1023, 1024, 1536, 2047, 2048, L - 1]
+        rest = np.sort(rng.integers(0, L, size=max(0, T - len(fixed))))
+        q_pos = np.concatenate([fixed, rest])[:T].astype(np.int64)
+    else:
+        q_pos = (L - 1 - spread * np.arange(T)).astype(np.int64)
+    return {"q_idx": to_bf16_bits(q), "q_pos": q_pos, "centroids": to_bf16_bits(c),
+            "bucket_off": off.astype(np.int32), "bucket_mem": members}
+
+
 def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
     """Inputs for a named workload (or a ``Workload``)."""
     if isinstance(wl, str):
@@ -313,4 +363,7 @@ def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
             wl.T, wl.clusters, wl.cluster_size, wl.H, wl.d, s, wl.noise_rel,
             wl.extra.get("min_size", 0), wl.extra.get("max_size", 0),
         )
+    if wl.kind == "lsa":
+        return make_lsa(wl.T, wl.N, wl.extra.get("block_keys", 512), wl.extra.get("bpb", 64), s,
+                        wl.extra.get("spread", 2053), bool(wl.extra.get("edge", 0)))
     raise ValueError(wl.kind)
