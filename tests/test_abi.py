@@ -28,7 +28,9 @@ def declared_functions():
 def test_header_declares_the_calls():
     names = declared_functions()
     for n in ("ls_indexer_score", "ls_topk_select", "ls_prefill_select_stream", "ls_decode_two_stage_select",
-              "ls_bucket_select", "ls_decode_select", "ls_last_error", "ls_device_status"):
+              "ls_bucket_select", "ls_decode_select", "ls_last_error", "ls_device_status", "ls_indexer_score_fp8",
+              "ls_prefill_select_stream_fp8", "ls_lsa_flat_select", "ls_indexer_score_pq",
+              "ls_decode_two_stage_pq_select"):
         assert n in names
 
 
@@ -50,6 +52,12 @@ def test_version_and_workspace_queries(lib):
     assert lib.ls_two_stage_workspace_size(32, 131072, 4096) >= 32 * 131072 * 4 + 2 * 32 * 4096 * 4
     assert lib.ls_bucket_workspace_size(256, 32768, 64, 512) >= 256 * 32768 * 4
     assert lib.ls_decode_select_workspace_size(0, 10) == 0
+    # fp8: w * q_scale per (query, head); the fp8 prefill adds it to the bf16 prefill's workspace
+    assert lib.ls_indexer_score_fp8_workspace_size(2, 9) >= 2 * 9 * 32 * 4
+    assert (lib.ls_prefill_select_fp8_workspace_size(4096, 32768, 8192, 512, 1)
+            >= lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 1) + 4096 * 32 * 4)
+    # LSA: the T x P bucket scores, visible counts and picks
+    assert lib.ls_lsa_flat_workspace_size(256, 131072, 1024) >= 256 * 131072 * 4 + 256 * 1024 * 4
 
 
 def test_argument_checks_without_gpu(lib):
@@ -85,6 +93,24 @@ def test_argument_checks_without_gpu(lib):
     assert st == 1
     assert lib.ls_indexer_score_pq(dummy, dummy, dummy, None, None, 1, 32, 128, 64, dummy, None) == 1
     assert lib.ls_indexer_score_pq(dummy, dummy, dummy, dummy, None, 1, 16, 128, 64, dummy, None) == 3
+    # fp8 indexer: H != 32, null scale, short workspace
+    assert lib.ls_indexer_score_fp8(dummy, dummy, dummy, dummy, dummy, None, None, 4, 1, 8, 16, 128, 64, dummy,
+                                    dummy, 1 << 20, None) == 3
+    assert lib.ls_indexer_score_fp8(dummy, None, dummy, dummy, dummy, None, None, 4, 1, 8, 32, 128, 64, dummy,
+                                    dummy, 1 << 20, None) == 1
+    assert lib.ls_indexer_score_fp8(dummy, dummy, dummy, dummy, dummy, None, None, 4, 1, 8, 32, 128, 64, dummy,
+                                    dummy, 16, None) == 2
+    # fp8 prefill: k out of range; LSA: d != 64, top_p too large, short workspace
+    assert lib.ls_prefill_select_stream_fp8(dummy, dummy, dummy, dummy, 4, 32, 128, dummy, dummy, 100, 4, 64,
+                                            dummy, dummy, 5000, 0, dummy, None, dummy, 1 << 30, None, None) == 1
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 128, 64, 512, 64, 4, 16, 64, dummy, dummy,
+                                  None, dummy, 1 << 30, None) == 3
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 5000, 64, dummy, dummy,
+                                  None, dummy, 1 << 30, None) == 1
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 16, 64, dummy, dummy,
+                                  None, dummy, 8, None) == 2
+    assert lib.ls_lsa_flat_select(None, None, None, None, None, 0, 64, 64, 512, 64, 4, 16, 64, None, None, None,
+                                  None, 0, None) == 0
     # bucket: budget below k
     st = lib.ls_bucket_select(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 128, 10, 80, 4, 100, 512, dummy,
                               None, None, dummy, 1 << 30, None)
