@@ -338,7 +338,9 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
                      ("prefill_chunk_running", lambda *a: bench_prefill(*a, full_scores=False)),
                      ("prefill_chunk_fp8", lambda *a: bench_prefill(*a, fp8=True)),
                      ("prefill_chunk_fp8_running", lambda *a: bench_prefill(*a, full_scores=False, fp8=True)),
-                     ("bucket", bench_bucket), ("lsa_flat", bench_lsa), ("two_stage", bench_two_stage),
+                     ("bucket", bench_bucket), ("lsa_flat", bench_lsa),
+                     ("lsa_flat_threshold", lambda *a: bench_lsa(*a, threshold=True)),
+                     ("two_stage", bench_two_stage),
                      ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True))):
         if only in (None, name):
             res[name] = fn(L, args, peaks, peak_kind)
@@ -346,13 +348,16 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
 
 
 def _profiled_loop(L, fn, steps, warm, st):
-    """Warm up, then time `steps` calls with the library's per-kernel events on."""
+    """Warm up, time `steps` calls, then run them again with the library's
+    per-kernel events on for the kernel breakdown (the step time is taken
+    without the events, which add a few microseconds per launch)."""
     import torch
     for i in range(warm):
         fn(i, None)
     torch.cuda.synchronize()
-    L.ls_profile_begin()
     tot, _ = time_loop(fn, steps, 0, st)
+    L.ls_profile_begin()
+    time_loop(fn, steps, 0, st)
     prof = L.ls_profile_end()
     kern = {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps} for k, v in prof.items()}
     return tot / steps, kern
@@ -468,9 +473,11 @@ def bench_bucket(L, args, peaks, peak_kind):
     return res
 
 
-def bench_lsa(L, args, peaks, peak_kind):
+def bench_lsa(L, args, peaks, peak_kind, threshold=False):
     """Native LSA flat search: 256 index queries over 131072 buckets of one
-    1048576-token sequence; top 1024 buckets, 4096 long-range keys."""
+    1048576-token sequence; top 1024 buckets, 4096 long-range keys.  With
+    threshold, the sampled-threshold scan lists only the buckets that clear
+    each query's threshold (else every score goes to a T x P matrix)."""
     import torch
     from workloads import get_workload, make_workload
     st = torch.cuda.current_stream()
@@ -483,28 +490,36 @@ def bench_lsa(L, args, peaks, peak_kind):
     P_ = d["centroids"].shape[0]
     a = [to_dev_bf16(d["q_idx"]), to_dev(d["q_pos"]), to_dev_bf16(d["centroids"]), to_dev(d["bucket_off"]),
          to_dev(d["bucket_mem"])]
-    ws = torch.empty(L.lib().ls_lsa_flat_workspace_size(T, P_, wl.top_p), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(L.lib().ls_lsa_flat_workspace_size(T, P_, wl.top_p, int(threshold)), dtype=torch.uint8,
+                     device="cuda")
     row = ex["n_sink"] + ex["block_keys"] + wl.budget
     out = (torch.empty((T, row), dtype=torch.int32, device="cuda"), torch.empty((T,), dtype=torch.int32, device="cuda"))
 
     def run(i, timed):
         L.ls_lsa_flat_select(*a, block_keys=ex["block_keys"], buckets_per_block=ex["bpb"], n_sink=ex["n_sink"],
-                             top_p=wl.top_p, budget=wl.budget, ws=ws, out=out)
+                             top_p=wl.top_p, budget=wl.budget, threshold=threshold, ws=ws, out=out)
         return None
 
     ms, kern = _profiled_loop(L, run, steps, warm, st)
-    dms = kern["dot_tc_kernel"]["ms_per_step"]
+    kname = "dot_tc_kernel:filter" if threshold else "dot_tc_kernel"
+    dms = kern[kname]["ms_per_step"]
     vis = np.minimum((d["q_pos"] // ex["block_keys"]) * ex["bpb"], P_)
     scored = int(vis.sum())
-    bytes_dot = P_ * 128 + T * 128 + T * P_ * 4
+    # centroids and queries read; the full form also writes the T x P score matrix
+    bytes_dot = P_ * 128 + T * 128 + (0 if threshold else T * P_ * 4)
     peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
     res = {"ms_per_step": ms, "positions_per_s": scored / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
            "kernels": kern,
            "roofline": roofline("hbm", bytes_dot / (dms * 1e-3) / 1e9, peak_b, "GB/s",
-                                traffic=ncu_traffic("dot_tc_kernel", wl.name), peak_kind=peak_kind),
+                                traffic=ncu_traffic(kname, wl.name + ("_threshold" if threshold else "")),
+                                peak_kind=peak_kind),
            "bytes_dot": bytes_dot, "visible_buckets_scored": scored,
-           "note": "positions = visible buckets scored per query (one 64-d dot each); roofline of the bucket "
-                   "scoring: centroids + queries read, the T x P score matrix written"}
+           "note": "positions = visible buckets scored per query (one 64-d dot each); "
+                   + ("sampled thresholds (every 128th bucket, 32nd best), the scan lists the buckets that clear "
+                      "them, top-1024 of each list, full-scoring fallback launches that return at once; roofline "
+                      "of the filtered scan over the centroid and query bytes it reads"
+                      if threshold else "full T x P score matrix; roofline of the scoring over the centroids and "
+                                        "queries read and the score matrix written")}
     del a, ws
     return res
 
@@ -627,7 +642,7 @@ def main(argv=None):
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "prefill_chunk_fp8",
                                                      "prefill_chunk_fp8_running", "bucket", "lsa_flat",
-                                                     "two_stage", "two_stage_pq"],
+                                                     "lsa_flat_threshold", "two_stage", "two_stage_pq"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -283,13 +283,23 @@ ls_status ls_prefill_select_stream_fp8(const uint8_t* q8, const float* q_scale, 
  * Visible buckets of a query at position t: the first
  * min(P, buckets_per_block * floor(t / block_keys)).  Bucket order: score
  * descending, then bucket id ascending.  Only d = 64 is built.
- * Workspace: ls_lsa_flat_workspace_size(T, P, top_p) bytes (a T x P score
- * matrix among them).
+ * threshold = 0: every (query, bucket) score is written to a T x P matrix in
+ * the workspace and the top_p of each row's visible prefix selected.
+ * threshold = 1: the LSA article's sampled threshold (section "What the
+ * kernels do about the top-p"): each query scores every (top_p / 8)-th
+ * bucket, its 32nd best sample becomes its threshold (about 4 * top_p
+ * buckets clear it), the scan appends only the visible buckets that reach
+ * the threshold to a list of up to 8 * top_p, and the top_p of the list is
+ * kept; a query whose list overflows or holds fewer than min(top_p, visible)
+ * buckets is scored in full instead.  Both forms pick the same buckets.
+ * Workspace: ls_lsa_flat_workspace_size(T, P, top_p, threshold) bytes (the
+ * T x P score matrix among them: the full form's scores and the threshold
+ * form's fallback).
  */
-size_t ls_lsa_flat_workspace_size(int T, int P, int top_p);
+size_t ls_lsa_flat_workspace_size(int T, int P, int top_p, int threshold);
 ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
                              const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
-                             int block_keys, int buckets_per_block, int n_sink, int top_p, int budget,
+                             int block_keys, int buckets_per_block, int n_sink, int top_p, int budget, int threshold,
                              int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws, size_t ws_bytes,
                              void* stream);
 

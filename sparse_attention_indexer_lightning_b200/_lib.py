@@ -81,8 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_indexer_score_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, SZ, P]),
         "ls_prefill_select_fp8_workspace_size": (SZ, [I, I, I, I, I]),
         "ls_prefill_select_stream_fp8": (I, [P, P, P, P, I, I, I, P, P, I, I, I, P, P, I, I, P, P, P, SZ, P, P]),
-        "ls_lsa_flat_workspace_size": (SZ, [I, I, I]),
-        "ls_lsa_flat_select": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
+        "ls_lsa_flat_workspace_size": (SZ, [I, I, I, I]),
+        "ls_lsa_flat_select": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -452,10 +452,11 @@ def ls_bucket_select(q, w, centroids, bucket_off, bucket_mem, keys, top_p: int =
 
 def ls_lsa_flat_select(q_idx, q_pos, centroids, bucket_off, bucket_mem, block_keys: int = 512,
                        buckets_per_block: int = 64, n_sink: int = 4, top_p: int = 1024, budget: int = 4096,
-                       want_picked: bool = False, ws=None, out=None, stream=None):
+                       threshold: bool = False, want_picked: bool = False, ws=None, out=None, stream=None):
     """Native LSA flat search.  q_idx [T,64] bf16, q_pos [T] int64, centroids [P,64] bf16 (block-major),
     bucket_off [P+1] / bucket_mem int32 (members ascending) -> (keys [T, n_sink+block_keys+budget] int32,
-    n [T] int32[, picked [T, top_p] int32])."""
+    n [T] int32[, picked [T, top_p] int32]).  threshold: the sampled-threshold scan with candidate lists (else
+    the full score matrix); both pick the same buckets."""
     _dev(q_idx, torch.bfloat16, "q_idx", 2)
     T, d = q_idx.shape
     _dev(q_pos, torch.int64, "q_pos", 1)
@@ -463,7 +464,7 @@ def ls_lsa_flat_select(q_idx, q_pos, centroids, bucket_off, bucket_mem, block_ke
     P = centroids.shape[0]
     _dev(bucket_off, torch.int32, "bucket_off", 1)
     _dev(bucket_mem, torch.int32, "bucket_mem", 1)
-    need = lib().ls_lsa_flat_workspace_size(T, P, top_p)
+    need = lib().ls_lsa_flat_workspace_size(T, P, top_p, int(threshold))
     if ws is None:
         ws = _workspace(need, q_idx.device)
     if out is None:
@@ -472,7 +473,8 @@ def ls_lsa_flat_select(q_idx, q_pos, centroids, bucket_off, bucket_mem, block_ke
     keys, n = out
     picked = torch.empty((T, top_p), dtype=torch.int32, device=q_idx.device) if want_picked else None
     _check(lib().ls_lsa_flat_select(_ptr(q_idx), _ptr(q_pos), _ptr(centroids), _ptr(bucket_off), _ptr(bucket_mem),
-                                    T, d, P, block_keys, buckets_per_block, n_sink, top_p, budget, _ptr(keys),
+                                    T, d, P, block_keys, buckets_per_block, n_sink, top_p, budget, int(threshold),
+                                    _ptr(keys),
                                     _ptr(n), _ptr(picked), _ptr(ws), ws.numel(), _stream(stream)))
     return (keys, n, picked) if want_picked else (keys, n)
 

@@ -7,6 +7,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -914,16 +915,94 @@ ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* ce
   return topk(exact, budget, nullptr, cand, budget, T, budget, k, idx_out, val_out, k, st);
 }
 
-size_t ls_lsa_flat_workspace_size(int T, int P, int top_p) {
-  if (T <= 0 || top_p <= 0) return 0;
-  return align_up(static_cast<size_t>(T) * (P > 0 ? P : 0) * sizeof(float)) +   // bucket scores
-         align_up(static_cast<size_t>(T) * sizeof(int32_t)) +                  // visible buckets
-         align_up(static_cast<size_t>(T) * top_p * sizeof(int32_t));           // picked buckets
+}  // extern "C"
+
+namespace {
+
+// Sampled-threshold parameters of the LSA search: every stride-th bucket is
+// sampled and the 32nd best sample sets the threshold, so about 4 * top_p
+// buckets of a row clear it; a row lists up to 8 * top_p.
+struct LsaThreshold {
+  int stride, rank, cap;
+  explicit LsaThreshold(int top_p)
+      : stride(top_p / 8 > 1 ? top_p / 8 : 1), rank(32), cap(8 * top_p) {}
+};
+
+// Per-CTA list segments of the filtered scan: nseg = the scan's grid, seg
+// entries each (about 4x the expected count of a CTA's share of 4 * top_p),
+// at most 2 * cap + 64 * nseg entries per row.
+struct LsaSegments {
+  int nseg, seg;
+  long long per_row;
+  LsaSegments(int T, int P, int cap) {
+    nseg = dot_tc_grid(T, P, num_sms_current());
+    if (nseg < 1) nseg = 1;
+    per_row = 2LL * cap + 64LL * nseg;
+    const int want = ((2 * cap / nseg + 31) / 32) * 32;
+    seg = static_cast<int>(std::min<long long>(std::max(32, want), per_row / nseg));
+  }
+};
+
+struct LsaWorkspace {
+  float* sc;        // [T][P] full scores (the full-matrix form, and the threshold form's fallback)
+  int32_t* vis;     // [T]
+  int32_t* nsamp;   // [T]
+  int32_t* picked;  // [T][top_p]
+  float* ss;        // [T][n_samp] sample scores
+  float* sv;        // [T][rank] best samples
+  int32_t* si;      // [T][rank]
+  float* sval;      // [T][nseg][seg] the scan's list segments
+  int32_t* slab;
+  uint32_t* scnt;   // [T][nseg]
+  float* cval;      // [T][cap] packed lists
+  int32_t* clab;
+  int32_t* nv;      // [T]
+  uint8_t* ctr;     // row_over [T], any_over
+  size_t ctr_bytes;
+  size_t scnt_bytes;
+  size_t used;
+};
+
+LsaWorkspace carve_lsa(void* ws, int T, int P, int top_p, int threshold) {
+  Carver cv(ws);
+  LsaWorkspace w{};
+  const LsaThreshold th(top_p);
+  const int n_samp = (P + th.stride - 1) / th.stride;
+  w.sc = cv.take<float>(static_cast<size_t>(T) * P);
+  w.vis = cv.take<int32_t>(T);
+  w.nsamp = cv.take<int32_t>(T);
+  w.picked = cv.take<int32_t>(static_cast<size_t>(T) * top_p);
+  if (threshold) {
+    w.ss = cv.take<float>(static_cast<size_t>(T) * n_samp);
+    w.sv = cv.take<float>(static_cast<size_t>(T) * th.rank);
+    w.si = cv.take<int32_t>(static_cast<size_t>(T) * th.rank);
+    const LsaSegments sg(T, P, th.cap);
+    w.sval = cv.take<float>(static_cast<size_t>(T) * sg.per_row);
+    w.slab = cv.take<int32_t>(static_cast<size_t>(T) * sg.per_row);
+    w.scnt_bytes = static_cast<size_t>(T) * sg.nseg * sizeof(uint32_t);
+    w.scnt = cv.take<uint32_t>(static_cast<size_t>(T) * sg.nseg);
+    w.cval = cv.take<float>(static_cast<size_t>(T) * th.cap);
+    w.clab = cv.take<int32_t>(static_cast<size_t>(T) * th.cap);
+    w.nv = cv.take<int32_t>(T);
+    w.ctr_bytes = static_cast<size_t>(T) * sizeof(int32_t) + sizeof(int);   // row flags, then the any-row flag
+    w.ctr = cv.take<uint8_t>(w.ctr_bytes);
+  }
+  w.used = cv.used;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ls_lsa_flat_workspace_size(int T, int P, int top_p, int threshold) {
+  if (T <= 0 || top_p <= 0 || P < 0) return 0;
+  return carve_lsa(nullptr, T, P, top_p, threshold).used;
 }
 
 ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
                              const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
-                             int block_keys, int buckets_per_block, int n_sink, int top_p, int budget,
+                             int block_keys, int buckets_per_block, int n_sink, int top_p, int budget, int threshold,
                              int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws, size_t ws_bytes,
                              void* stream) {
   if (d != kLsaDim) return fail(LS_ERR_UNSUPPORTED, "only d=%d is built for the LSA index space (got %d)", kLsaDim, d);
@@ -933,17 +1012,16 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
   LS_CHECK_ARG(top_p >= 1 && top_p <= kMaxTopK, "top_p must be in [1, %d] (got %d)", kMaxTopK, top_p);
   if (T == 0) return LS_OK;
   LS_CHECK_ARG(q_pos && keys_out && n_out, "null tensor pointer");
-  const size_t need = ls_lsa_flat_workspace_size(T, P, top_p);
+  const size_t need = ls_lsa_flat_workspace_size(T, P, top_p, threshold);
   if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
-  Carver cv(ws);
-  float* sc = cv.take<float>(static_cast<size_t>(T) * P);
-  int32_t* vis = cv.take<int32_t>(T);
-  int32_t* picked_ws = cv.take<int32_t>(static_cast<size_t>(T) * top_p);
-  int32_t* picked = picked_out ? picked_out : picked_ws;
+  const LsaWorkspace w = carve_lsa(ws, T, P, top_p, threshold);
+  const LsaThreshold th(top_p);
+  int32_t* picked = picked_out ? picked_out : w.picked;
   cudaStream_t st = S(stream);
   {
     ProfScope prof("lsa_visible_kernel", st);
-    LS_CUDA(launch_lsa_visible(q_pos, T, block_keys, buckets_per_block, P, vis, st));
+    LS_CUDA(launch_lsa_visible(q_pos, T, block_keys, buckets_per_block, P, th.stride, w.vis,
+                               threshold ? w.nsamp : nullptr, st));
   }
   if (P > 0) {
     LS_CHECK_ARG(q_idx && centroids && bucket_off && bucket_mem, "null tensor pointer");
@@ -953,12 +1031,109 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
     if (s != LS_OK) return s;
     s = make_vec64_map(&qmap, q_idx, static_cast<uint64_t>(T), DotCfg::QB);
     if (s != LS_OK) return s;
-    ProfScope prof("dot_tc_kernel", st);
-    LS_CUDA(launch_dot_tc(&cmap, &qmap, T, P, sc, P, num_sms_current(), st));
+    DotParams full;
+    full.T = T;
+    full.P = P;
+    full.out = w.sc;
+    full.ld_out = P;
+    TopkParams tp;                        // top-p of each row's visible prefix (padding -1)
+    tp.scores = w.sc;
+    tp.ld = P;
+    tp.n_valid = w.vis;
+    tp.R = T;
+    tp.N = P;
+    tp.k = top_p;
+    tp.idx_out = picked;
+    tp.ld_out = top_p;
+    if (!threshold) {
+      {
+        ProfScope prof("dot_tc_kernel", st);
+        LS_CUDA(launch_dot_tc(&cmap, &qmap, full, num_sms_current(), st));
+      }
+      s = topk_launch(tp, st);
+      if (s != LS_OK) return s;
+    } else {
+      // 1. thresholds from a sample of every stride-th bucket
+      const int n_samp = (P + th.stride - 1) / th.stride;
+      {
+        ProfScope prof("lsa_sample_kernel", st);
+        LS_CUDA(launch_lsa_sample(q_idx, centroids, T, n_samp, th.stride, w.ss, st));
+      }
+      TopkParams sp;
+      sp.scores = w.ss;
+      sp.ld = n_samp;
+      sp.n_valid = w.nsamp;
+      sp.R = T;
+      sp.N = n_samp;
+      sp.k = th.rank;
+      sp.idx_out = w.si;
+      sp.val_out = w.sv;
+      sp.ld_out = th.rank;
+      s = topk_launch(sp, st, "topk_kernel:sample");
+      if (s != LS_OK) return s;
+      // 2. the scan lists the buckets that reach the threshold
+      int32_t* row_over = reinterpret_cast<int32_t*>(w.ctr);
+      int* any_over = reinterpret_cast<int*>(w.ctr) + static_cast<size_t>(T);
+      LS_CUDA(cudaMemsetAsync(w.ctr, 0, w.ctr_bytes, st));
+      LS_CUDA(cudaMemsetAsync(w.scnt, 0, w.scnt_bytes, st));
+      const LsaSegments sg(T, P, th.cap);
+      DotParams fp;
+      fp.T = T;
+      fp.P = P;
+      fp.vis = w.vis;
+      fp.tau = w.sv + (th.rank - 1);
+      fp.ld_tau = th.rank;
+      fp.cand_val = w.sval;
+      fp.cand_lab = w.slab;
+      fp.nseg = sg.nseg;
+      fp.seg = sg.seg;
+      fp.cand_cnt = w.scnt;
+      fp.row_over = row_over;
+      fp.any_over = any_over;
+      {
+        ProfScope prof("dot_tc_kernel:filter", st);
+        LS_CUDA(launch_dot_tc(&cmap, &qmap, fp, num_sms_current(), st));
+      }
+      {
+        ProfScope prof("lsa_compact_kernel", st);
+        LS_CUDA(launch_lsa_compact(w.sval, w.slab, w.scnt, sg.nseg, sg.seg, w.vis, T, top_p, th.cap, w.cval, w.clab,
+                                   w.nv, row_over, any_over, st));
+      }
+      // 3. top-p of each list
+      TopkParams cp;
+      cp.scores = w.cval;
+      cp.ld = th.cap;
+      cp.n_valid = w.nv;
+      cp.labels = w.clab;
+      cp.ld_labels = th.cap;
+      cp.R = T;
+      cp.N = th.cap;
+      cp.k = top_p;
+      cp.idx_out = picked;
+      cp.ld_out = top_p;
+      s = topk_launch(cp, st);
+      if (s != LS_OK) return s;
+      // 4. rows whose list ran over or came up short: scored in full (launches
+      //    that return at once when no row is flagged)
+      full.run_if = any_over;
+      {
+        ProfScope prof("dot_tc_kernel:fallback", st);
+        LS_CUDA(launch_dot_tc(&cmap, &qmap, full, num_sms_current(), st));
+      }
+      tp.run_if = any_over;
+      tp.row_flag = row_over;
+      s = topk_launch(tp, st, "topk_kernel:fallback");
+      if (s != LS_OK) return s;
+    }
+  } else {
+    TopkParams tp;                        // nothing visible anywhere: every row is padding
+    tp.R = T;
+    tp.k = top_p;
+    tp.idx_out = picked;
+    tp.ld_out = top_p;
+    ls_status s = topk_launch(tp, st);
+    if (s != LS_OK) return s;
   }
-  // top-p of each row's visible prefix (padding -1 where fewer are visible)
-  ls_status s = topk(sc, P, vis, nullptr, 0, T, P, top_p, picked, nullptr, top_p, st);
-  if (s != LS_OK) return s;
   ProfScope prof("lsa_expand_kernel", st);
   LS_CUDA(launch_lsa_expand(picked, q_pos, T, top_p, bucket_off, bucket_mem, P, block_keys, n_sink, budget, keys_out,
                             n_sink + block_keys + budget, n_out, st));

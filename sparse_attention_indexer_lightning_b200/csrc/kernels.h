@@ -70,13 +70,43 @@ cudaError_t launch_score_tc_f8(const CUtensorMap* kmap, const CUtensorMap* qmap,
 // out[i] = w[i] * qs[i], i < n.
 cudaError_t launch_fold_scales(const float* w, const float* qs, int64_t n, float* out, cudaStream_t st);
 
-// Native LSA flat search: out[t][p] = q[t] . c[p] over 64-d bf16 vectors
-// (cmap over the centroids [P][128 B], qmap over the index queries [T][128 B]).
-cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, int T, int P, float* out, int64_t ld_out,
-                          int num_sms, cudaStream_t st);
-// vis[t] = min(P, bpb * floor(q_pos[t] / block_keys)).
-cudaError_t launch_lsa_visible(const int64_t* q_pos, int T, int block_keys, int bpb, int P, int32_t* vis,
-                               cudaStream_t st);
+// Native LSA flat search: scores q[t] . c[p] over 64-d bf16 vectors (cmap over
+// the centroids [P][128 B], qmap over the index queries [T][128 B]); stored
+// to out[t][p] (out != nullptr), or, the filter form (out == nullptr),
+// appended as (score, p) to row t's candidate list when p < vis[t] and the
+// score's order code reaches that of tau[t * ld_tau].
+struct DotParams {
+  int T = 0, P = 0;
+  float* out = nullptr;
+  int64_t ld_out = 0;
+  const int32_t* vis = nullptr;       // [T] visible buckets per row
+  const float* tau = nullptr;         // thresholds, tau[t * ld_tau]
+  int64_t ld_tau = 0;
+  // row t's list is split into nseg segments of seg entries, one per CTA
+  // (nseg = the grid size): [T][nseg][seg], counts [T][nseg] zeroed before the launch
+  float* cand_val = nullptr;
+  int32_t* cand_lab = nullptr;
+  int nseg = 0, seg = 0;
+  uint32_t* cand_cnt = nullptr;
+  int32_t* row_over = nullptr;        // [T]
+  int* any_over = nullptr;
+  const int* run_if = nullptr;        // the launch does nothing unless *run_if != 0 (nullptr: always)
+};
+cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, const DotParams& p, int num_sms,
+                          cudaStream_t st);
+// vis[t] = min(P, bpb * floor(q_pos[t] / block_keys)); n_samp[t] = ceil(vis[t] / stride) (if n_samp).
+cudaError_t launch_lsa_visible(const int64_t* q_pos, int T, int block_keys, int bpb, int P, int stride, int32_t* vis,
+                               int32_t* n_samp, cudaStream_t st);
+// ss[t][i] = q[t] . c[i * stride], i < n_samp.
+cudaError_t launch_lsa_sample(const uint16_t* q, const uint16_t* c, int T, int n_samp, int stride, float* ss,
+                              cudaStream_t st);
+// The grid size the LSA scan launches with (the filter form's segment count).
+int dot_tc_grid(int T, int P, int num_sms);
+// Pack each row's per-CTA segments into cval / clab [T][cap] (nv[t] entries);
+// flag rows that ran over or hold fewer than min(top_p, vis[t]).
+cudaError_t launch_lsa_compact(const float* sval, const int32_t* slab, const uint32_t* cnt, int nseg, int seg,
+                               const int32_t* vis, int T, int top_p, int cap, float* cval, int32_t* clab, int32_t* nv,
+                               int32_t* row_over, int* any_over, cudaStream_t st);
 // The read list of each query: sinks below its window, the window, then the
 // picked buckets' members best first (sinks and window skipped) up to budget.
 cudaError_t launch_lsa_expand(const int32_t* picked, const int64_t* q_pos, int T, int top_p, const int32_t* off,

@@ -63,10 +63,22 @@ struct DotBarriers {
 };
 static_assert(sizeof(DotBarriers) <= DotCfg::SMEM_BAR, "barrier block");
 
+// Threshold code of a row: a key is listed when its order code reaches it
+// (-inf, the padding of a short sample, lists every visible bucket).
+__device__ __forceinline__ uint32_t tau_code(float tau) { return order_code(tau); }
+
+
+// FILTER: instead of storing every score, append (score, bucket) to the
+// query's candidate list when the bucket is visible and its score reaches the
+// query's threshold (LSA's sampled threshold: "appends only those above it to
+// a short list"); a list that runs out of room flags its row.
+template <bool FILTER>
 __global__ void __launch_bounds__(DotCfg::THREADS, 1)
-    dot_tc_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap qmap, int T, int P,
-                  float* __restrict__ out, int64_t ld_out) {
+    dot_tc_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap qmap,
+                  const DotParams p) {
   using C = DotCfg;
+  if (p.run_if != nullptr && *p.run_if == 0) return;  // a conditional launch with nothing to do
+  const int T = p.T, P = p.P;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -208,11 +220,22 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
+    // filter form: lane l holds the threshold code and visible count of the
+    // warp's queries t0 + l and t0 + 32 + l (reloaded when the group changes)
+    uint32_t thr_a = 0xffffffffu, thr_b = 0xffffffffu;
+    int vis_a = 0, vis_b = 0;
     UnitPos up;
     up.init(u_begin, NT, G);
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
-      const int p = up.tile * C::BM + quad * 32 + lane;      // this thread's centroid
+      const int pc = up.tile * C::BM + quad * 32 + lane;     // this thread's centroid
       const int t0 = up.g * C::QB + cset * C::COLS_PER_WARP;
+      if (FILTER && (u == u_begin || up.tile == 0)) {
+        const int ta = t0 + lane, tb = t0 + 32 + lane;
+        thr_a = (ta < T) ? tau_code(p.tau[static_cast<int64_t>(ta) * p.ld_tau]) : 0xffffffffu;
+        thr_b = (tb < T) ? tau_code(p.tau[static_cast<int64_t>(tb) * p.ld_tau]) : 0xffffffffu;
+        vis_a = (ta < T) ? p.vis[ta] : 0;
+        vis_b = (tb < T) ? p.vis[tb] : 0;
+      }
       if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t col = tmem_base + lane_off + static_cast<uint32_t>(acc * C::ACC_COLS + cset * C::COLS_PER_WARP);
@@ -226,14 +249,66 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
       if (lane == 0) mbar_arrive(&bars->tempty[acc]);
       if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
       const int nt = min(C::COLS_PER_WARP, T - t0);          // queries of this warp that exist
-      if (p < P && nt > 0) {
-        float* o = out + static_cast<int64_t>(t0) * ld_out + p;
+      if (!FILTER) {
+        if (pc < P && nt > 0) {
+          float* o = p.out + static_cast<int64_t>(t0) * p.ld_out + pc;
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nt) o[static_cast<int64_t>(j) * ld_out] = __uint_as_float(v0[j]);
+          for (int j = 0; j < 32; ++j)
+            if (j < nt) o[static_cast<int64_t>(j) * p.ld_out] = __uint_as_float(v0[j]);
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (32 + j < nt) o[static_cast<int64_t>(32 + j) * ld_out] = __uint_as_float(v1[j]);
+          for (int j = 0; j < 32; ++j)
+            if (32 + j < nt) o[static_cast<int64_t>(32 + j) * p.ld_out] = __uint_as_float(v1[j]);
+        }
+      } else {
+        // Pass 1: one ballot per query column; lane j keeps the ballots of
+        // columns j and 32 + j.  Pass 2: every lane reserves its two columns'
+        // slots with one atomic each, all in flight together.  Pass 3: the
+        // listed lanes write (score, bucket) at their slots.
+        uint32_t bal_a = 0, bal_b = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const uint32_t thr = __shfl_sync(0xffffffffu, h ? thr_b : thr_a, j);
+            const int vis = __shfl_sync(0xffffffffu, h ? vis_b : vis_a, j);
+            const float sv = __uint_as_float(h ? v1[j] : v0[j]);
+            const bool take = (32 * h + j < nt) && (pc < vis) && order_code(sv) >= thr;
+            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+            if (lane == j) {
+              if (h) bal_b = bal;
+              else bal_a = bal;
+            }
+          }
+        }
+        uint32_t base_a = 0, base_b = 0;
+        // each CTA appends to its own segment of a row's list (few atomics per address)
+        if (bal_a)
+          base_a = atomicAdd(p.cand_cnt + static_cast<int64_t>(t0 + lane) * p.nseg + blockIdx.x,
+                             static_cast<uint32_t>(__popc(bal_a)));
+        if (bal_b)
+          base_b = atomicAdd(p.cand_cnt + static_cast<int64_t>(t0 + 32 + lane) * p.nseg + blockIdx.x,
+                             static_cast<uint32_t>(__popc(bal_b)));
+        const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const uint32_t bal = __shfl_sync(0xffffffffu, h ? bal_b : bal_a, j);
+            const uint32_t base = __shfl_sync(0xffffffffu, h ? base_b : base_a, j);
+            if ((bal >> lane) & 1u) {
+              const int t = t0 + 32 * h + j;
+              const uint32_t slot = base + static_cast<uint32_t>(__popc(bal & below));
+              if (slot < static_cast<uint32_t>(p.seg)) {
+                const int64_t at = (static_cast<int64_t>(t) * p.nseg + blockIdx.x) * p.seg + slot;
+                p.cand_val[at] = __uint_as_float(h ? v1[j] : v0[j]);
+                p.cand_lab[at] = pc;
+              } else {
+                p.row_over[t] = 1;
+                *p.any_over = 1;
+              }
+            }
+          }
+        }
       }
     }
   }
@@ -247,23 +322,32 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
   }
 }
 
-cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, int T, int P, float* out, int64_t ld_out,
-                          int num_sms, cudaStream_t st) {
+template <bool FILTER>
+static cudaError_t launch_dot(const CUtensorMap* cmap, const CUtensorMap* qmap, const DotParams& p, int num_sms,
+                              cudaStream_t st) {
   using C = DotCfg;
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(dot_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(dot_tc_kernel<FILTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(C::SMEM_TOTAL));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const int G = (T + C::QB - 1) / C::QB;
-  const int NT = (P + C::BM - 1) / C::BM;
-  const long long units = static_cast<long long>(G) * NT;
-  if (units == 0) return cudaSuccess;
-  const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-  dot_tc_kernel<<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*cmap, *qmap, T, P, out, ld_out);
+  const int grid = dot_tc_grid(p.T, p.P, num_sms);
+  if (grid == 0) return cudaSuccess;
+  if (FILTER && grid > p.nseg) return cudaErrorInvalidValue;   // one list segment per CTA
+  dot_tc_kernel<FILTER><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*cmap, *qmap, p);
   return cudaGetLastError();
+}
+
+int dot_tc_grid(int T, int P, int num_sms) {
+  const long long units = static_cast<long long>((T + DotCfg::QB - 1) / DotCfg::QB) * ((P + DotCfg::BM - 1) / DotCfg::BM);
+  return static_cast<int>(units < num_sms ? units : num_sms);
+}
+
+cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, const DotParams& p, int num_sms,
+                          cudaStream_t st) {
+  return p.out == nullptr ? launch_dot<true>(cmap, qmap, p, num_sms, st) : launch_dot<false>(cmap, qmap, p, num_sms, st);
 }
 
 // Visible buckets of each query (causal block visibility: the buckets of the
@@ -274,13 +358,106 @@ cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, int 
 //   best first, members that fall in the sinks or the window skipped, until
 //   `budget` are held (the last bucket cut short); -1 after the end; n_out[t]
 //   the row's length.  Bucket members are stored in ascending position order.
+// Sample scores for the thresholds: row t scores the buckets 0, stride,
+// 2*stride, ... below its visible count (the same positions for every row, so
+// the sampled centroids stay in L2): ss[t][i] = q[t] . c[i * stride].
+__global__ void lsa_sample_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ c, int T, int n_samp,
+                                  int stride, float* __restrict__ ss) {
+  const int t = blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  __shared__ float qs[kLsaDim];
+  if (threadIdx.x < kLsaDim) qs[threadIdx.x] = __uint_as_float(static_cast<uint32_t>(q[t * kLsaDim + threadIdx.x]) << 16);
+  __syncthreads();
+  if (i >= n_samp) return;
+  const uint4* row = reinterpret_cast<const uint4*>(c + static_cast<int64_t>(i) * stride * kLsaDim);
+  float acc = 0.f;
+#pragma unroll
+  for (int v = 0; v < kLsaDim / 8; ++v) {
+    const uint4 x = __ldg(row + v);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(__uint_as_float(w[e] << 16), qs[8 * v + 2 * e], acc);
+      acc = fmaf(__uint_as_float(w[e] & 0xffff0000u), qs[8 * v + 2 * e + 1], acc);
+    }
+  }
+  ss[static_cast<int64_t>(t) * n_samp + i] = acc;
+}
+
+// After the filtered scan, one CTA per row: the row's per-CTA segments are
+// packed into one list of up to `cap` entries (nv[t] of them).  A row falls
+// back to full scoring when a segment ran over (flagged in the scan), the
+// list would exceed cap, or it holds fewer than min(top_p, visible) buckets.
+__global__ void __launch_bounds__(256)
+    lsa_compact_kernel(const float* __restrict__ sval, const int32_t* __restrict__ slab,
+                       const uint32_t* __restrict__ cnt, int nseg, int seg, const int32_t* __restrict__ vis, int top_p,
+                       int cap, float* __restrict__ cval, int32_t* __restrict__ clab, int32_t* __restrict__ nv,
+                       int32_t* __restrict__ row_over, int* __restrict__ any_over) {
+  __shared__ int offs[1025];
+  __shared__ int wsum[8];
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, wid = tid >> 5;
+  // exclusive scan of the segment counts (nseg <= 1024: 4 per thread)
+  int c4[4];
+  int mine = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = tid * 4 + i;
+    c4[i] = (c < nseg) ? static_cast<int>(min(cnt[static_cast<int64_t>(t) * nseg + c], static_cast<uint32_t>(seg))) : 0;
+    mine += c4[i];
+  }
+  int incl = mine;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  int run = incl - mine;
+  for (int w = 0; w < wid; ++w) run += wsum[w];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = tid * 4 + i;
+    if (c < nseg) offs[c] = run;
+    run += c4[i];
+  }
+  if (tid == 255) offs[nseg] = run;
+  __syncthreads();
+  const int total = offs[nseg];
+  const int need = min(top_p, vis[t]);
+  if (tid == 0) {
+    nv[t] = min(total, cap);
+    if (total > cap || total < need) {
+      row_over[t] = 1;
+      *any_over = 1;
+    }
+  }
+  if (total > cap) return;
+  // output entry o comes from the segment c with offs[c] <= o < offs[c + 1]
+  for (int o = tid; o < total; o += 256) {
+    int lo = 0, hi = nseg;                      // offs[lo] <= o < offs[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (offs[mid] <= o) lo = mid;
+      else hi = mid;
+    }
+    const int64_t src = (static_cast<int64_t>(t) * nseg + lo) * seg + (o - offs[lo]);
+    cval[static_cast<int64_t>(t) * cap + o] = sval[src];
+    clab[static_cast<int64_t>(t) * cap + o] = slab[src];
+  }
+}
+
 __global__ void lsa_visible_kernel(const int64_t* __restrict__ q_pos, int T, int block_keys, int bpb, int P,
-                                   int32_t* __restrict__ vis) {
+                                   int stride, int32_t* __restrict__ vis, int32_t* __restrict__ n_samp) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
   const int64_t qp = q_pos[t] < 0 ? 0 : q_pos[t];
   const int64_t v = (qp / block_keys) * bpb;
-  vis[t] = static_cast<int32_t>(v < P ? v : P);
+  const int32_t vv = static_cast<int32_t>(v < P ? v : P);
+  vis[t] = vv;
+  if (n_samp) n_samp[t] = (vv + stride - 1) / stride;   // sampled buckets below the visible count
 }
 
 __device__ __forceinline__ int lower_bound_i32(const int32_t* __restrict__ a, int n, int64_t x) {
@@ -368,10 +545,27 @@ __global__ void __launch_bounds__(kExpandThreads)
   if (tid == 0) n_out[t] = used;
 }
 
-cudaError_t launch_lsa_visible(const int64_t* q_pos, int T, int block_keys, int bpb, int P, int32_t* vis,
-                               cudaStream_t st) {
+cudaError_t launch_lsa_visible(const int64_t* q_pos, int T, int block_keys, int bpb, int P, int stride, int32_t* vis,
+                               int32_t* n_samp, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  lsa_visible_kernel<<<(T + 255) / 256, 256, 0, st>>>(q_pos, T, block_keys, bpb, P, vis);
+  lsa_visible_kernel<<<(T + 255) / 256, 256, 0, st>>>(q_pos, T, block_keys, bpb, P, stride, vis, n_samp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsa_sample(const uint16_t* q, const uint16_t* c, int T, int n_samp, int stride, float* ss,
+                              cudaStream_t st) {
+  if (T == 0 || n_samp == 0) return cudaSuccess;
+  lsa_sample_kernel<<<dim3((n_samp + 255) / 256, T), 256, 0, st>>>(q, c, T, n_samp, stride, ss);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsa_compact(const float* sval, const int32_t* slab, const uint32_t* cnt, int nseg, int seg,
+                               const int32_t* vis, int T, int top_p, int cap, float* cval, int32_t* clab, int32_t* nv,
+                               int32_t* row_over, int* any_over, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (nseg > 1024) return cudaErrorInvalidValue;
+  lsa_compact_kernel<<<T, 256, 0, st>>>(sval, slab, cnt, nseg, seg, vis, top_p, cap, cval, clab, nv, row_over,
+                                        any_over);
   return cudaGetLastError();
 }
 

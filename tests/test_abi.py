@@ -57,7 +57,10 @@ def test_version_and_workspace_queries(lib):
     assert (lib.ls_prefill_select_fp8_workspace_size(4096, 32768, 8192, 512, 1)
             >= lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 1) + 4096 * 32 * 4)
     # LSA: the T x P bucket scores, visible counts and picks
-    assert lib.ls_lsa_flat_workspace_size(256, 131072, 1024) >= 256 * 131072 * 4 + 256 * 1024 * 4
+    assert lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) >= 256 * 131072 * 4 + 256 * 1024 * 4
+    # the threshold form adds the samples and the candidate lists (8 * top_p per row)
+    assert (lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 1)
+            >= lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) + 256 * 8192 * 8)
 
 
 def test_argument_checks_without_gpu(lib):
@@ -103,13 +106,13 @@ def test_argument_checks_without_gpu(lib):
     # fp8 prefill: k out of range; LSA: d != 64, top_p too large, short workspace
     assert lib.ls_prefill_select_stream_fp8(dummy, dummy, dummy, dummy, 4, 32, 128, dummy, dummy, 100, 4, 64,
                                             dummy, dummy, 5000, 0, dummy, None, dummy, 1 << 30, None, None) == 1
-    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 128, 64, 512, 64, 4, 16, 64, dummy, dummy,
-                                  None, dummy, 1 << 30, None) == 3
-    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 5000, 64, dummy, dummy,
-                                  None, dummy, 1 << 30, None) == 1
-    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 16, 64, dummy, dummy,
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 128, 64, 512, 64, 4, 16, 64, 1, dummy,
+                                  dummy, None, dummy, 1 << 30, None) == 3
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 5000, 64, 1, dummy,
+                                  dummy, None, dummy, 1 << 30, None) == 1
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 16, 64, 1, dummy, dummy,
                                   None, dummy, 8, None) == 2
-    assert lib.ls_lsa_flat_select(None, None, None, None, None, 0, 64, 64, 512, 64, 4, 16, 64, None, None, None,
+    assert lib.ls_lsa_flat_select(None, None, None, None, None, 0, 64, 64, 512, 64, 4, 16, 64, 1, None, None, None,
                                   None, 0, None) == 0
     # bucket: budget below k
     st = lib.ls_bucket_select(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 128, 10, 80, 4, 100, 512, dummy,

@@ -560,15 +560,23 @@ def test_bucket_full_size_sampled(L):
 # --------------------------------------------------------------------------- #
 # native LSA flat search
 # --------------------------------------------------------------------------- #
-def _check_lsa(L, name, rows):
-    wl = get_workload(name)
-    d = data(name)
+def _lsa_run(L, d, wl, threshold):
     ex = wl.extra
     keys, n, picked = L.ls_lsa_flat_select(dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]),
                                            dev(d["bucket_off"]), dev(d["bucket_mem"]), block_keys=ex["block_keys"],
                                            buckets_per_block=ex["bpb"], n_sink=ex["n_sink"], top_p=wl.top_p,
-                                           budget=wl.budget, want_picked=True)
-    keys, n, picked = keys.cpu().numpy(), n.cpu().numpy(), picked.cpu().numpy()
+                                           budget=wl.budget, threshold=threshold, want_picked=True)
+    return keys.cpu().numpy(), n.cpu().numpy(), picked.cpu().numpy()
+
+
+def _check_lsa(L, name, rows, d=None, wl=None):
+    wl = wl or get_workload(name)
+    d = d or data(name)
+    ex = wl.extra
+    keys, n, picked = _lsa_run(L, d, wl, threshold=True)
+    # the full-matrix form picks the same buckets, bit for bit
+    keys0, n0, picked0 = _lsa_run(L, d, wl, threshold=False)
+    assert np.array_equal(picked0, picked) and np.array_equal(keys0, keys) and np.array_equal(n0, n), name
     _, det = lsa_flat_select(d["q_idx"], d["q_pos"], d["centroids"], d["bucket_off"], d["bucket_mem"],
                              ex["block_keys"], ex["bpb"], ex["n_sink"], wl.top_p, wl.budget, rows=rows,
                              return_detail=True)
@@ -593,6 +601,29 @@ def test_lsa_flat_small(L):
 @pytest.mark.slow
 def test_lsa_flat_full_size_sampled(L):
     _check_lsa(L, "lsa_flat", [0, 1, 100, 254, 255])
+
+
+def test_lsa_threshold_fallbacks(L):
+    """Rows whose sampled threshold misses fall back to full scoring.  Every
+    query points along u; the sampled buckets (every top_p/8-th) point along
+    u and the rest along -u, so the sample's 32nd best clears only sampled
+    buckets: rows with fewer than top_p of them come up short; then all
+    centroids along u, so every visible bucket ties at the threshold and rows
+    with more than 8*top_p visible buckets overflow their lists."""
+    wl = get_workload("lsa_flat_s")
+    base = data("lsa_flat_s")
+    rng = np.random.default_rng(3)
+    u = rng.standard_normal(64)
+    u /= np.linalg.norm(u)
+    P = base["centroids"].shape[0]
+    stride = max(1, wl.top_p // 8)
+    sign = np.where(np.arange(P) % stride == 0, 1.0, -1.0)
+    from workloads.synth import to_bf16_bits
+    for cent in (sign[:, None] * u[None, :], np.broadcast_to(u, (P, 64)).copy()):
+        d = dict(base)
+        d["q_idx"] = to_bf16_bits(np.broadcast_to(u, base["q_idx"].shape).copy())
+        d["centroids"] = to_bf16_bits(cent)
+        _check_lsa(L, "lsa_flat_s", list(range(37)), d=d, wl=wl)
 
 
 def test_bucket_bad_member_flagged(L):
