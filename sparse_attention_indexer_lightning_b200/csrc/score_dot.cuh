@@ -45,7 +45,13 @@ struct DotCfg {
   static constexpr size_t SMEM_A = size_t(STAGES) * A_BYTES;
   static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
   static constexpr size_t SMEM_BAR = 512;
-  static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR;
+  // filter form, per epilogue warp: each column's ballot and list base (64 x
+  // 2 words) and each lane's listed (score, column) pairs (LIST per lane)
+  static constexpr int LIST = 16;
+  static constexpr size_t SMEM_COL = 64 * 2 * 4;
+  static constexpr size_t SMEM_LST = 32 * LIST * 8;
+  static constexpr size_t SMEM_F = size_t(EPI_WARPS) * (SMEM_COL + SMEM_LST);
+  static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR + SMEM_F;
   static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
   static_assert(DIM * 2 == 128, "one 128-byte swizzle row per vector");
 };
@@ -62,10 +68,6 @@ struct DotBarriers {
   int abort_flag;
 };
 static_assert(sizeof(DotBarriers) <= DotCfg::SMEM_BAR, "barrier block");
-
-// Threshold code of a row: a key is listed when its order code reaches it
-// (-inf, the padding of a short sample, lists every visible bucket).
-__device__ __forceinline__ uint32_t tau_code(float tau) { return order_code(tau); }
 
 
 // FILTER: instead of storing every score, append (score, bucket) to the
@@ -84,6 +86,7 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::SMEM_A;
   DotBarriers* bars = reinterpret_cast<DotBarriers*>(smem + C::SMEM_A + C::SMEM_B);
+  uint8_t* sfilt = smem + C::SMEM_A + C::SMEM_B + C::SMEM_BAR;
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -220,10 +223,11 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
-    // filter form: lane l holds the threshold code and visible count of the
-    // warp's queries t0 + l and t0 + 32 + l (reloaded when the group changes)
-    uint32_t thr_a = 0xffffffffu, thr_b = 0xffffffffu;
-    int vis_a = 0, vis_b = 0;
+    // filter form: lane l holds the threshold and visible count of the warp's
+    // queries t0 + l and t0 + 32 + l (reloaded when the group changes; a query
+    // past the end sees nothing), vis_min the smallest of the 64 counts
+    float thr_a = 0.f, thr_b = 0.f;
+    int vis_a = 0, vis_b = 0, vis_min = 0;
     UnitPos up;
     up.init(u_begin, NT, G);
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
@@ -231,25 +235,31 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
       const int t0 = up.g * C::QB + cset * C::COLS_PER_WARP;
       if (FILTER && (u == u_begin || up.tile == 0)) {
         const int ta = t0 + lane, tb = t0 + 32 + lane;
-        thr_a = (ta < T) ? tau_code(p.tau[static_cast<int64_t>(ta) * p.ld_tau]) : 0xffffffffu;
-        thr_b = (tb < T) ? tau_code(p.tau[static_cast<int64_t>(tb) * p.ld_tau]) : 0xffffffffu;
+        thr_a = (ta < T) ? p.tau[static_cast<int64_t>(ta) * p.ld_tau] : 0.f;
+        thr_b = (tb < T) ? p.tau[static_cast<int64_t>(tb) * p.ld_tau] : 0.f;
         vis_a = (ta < T) ? p.vis[ta] : 0;
         vis_b = (tb < T) ? p.vis[tb] : 0;
+        vis_min = min(vis_a, vis_b);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) vis_min = min(vis_min, __shfl_xor_sync(0xffffffffu, vis_min, d));
       }
       if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t col = tmem_base + lane_off + static_cast<uint32_t>(acc * C::ACC_COLS + cset * C::COLS_PER_WARP);
-      uint32_t v0[32], v1[32];
-      tmem_ld_32x32_nowait(col, v0);
-      tmem_ld_32x32_nowait(col + 32, v1);
-      tmem_wait_ld(v0);
-      tmem_wait_ld(v1);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->tempty[acc]);
-      if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
       const int nt = min(C::COLS_PER_WARP, T - t0);          // queries of this warp that exist
+      auto release = [&]() {                                  // the accumulator is read: hand it back
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->tempty[acc]);
+        if (++acc == C::ACC) { acc = 0; acc_phase ^= 1; }
+      };
       if (!FILTER) {
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32_nowait(col, v0);
+        tmem_ld_32x32_nowait(col + 32, v1);
+        tmem_wait_ld(v0);
+        tmem_wait_ld(v1);
+        release();
         if (pc < P && nt > 0) {
           float* o = p.out + static_cast<int64_t>(t0) * p.ld_out + pc;
 #pragma unroll
@@ -260,23 +270,44 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
             if (32 + j < nt) o[static_cast<int64_t>(32 + j) * p.ld_out] = __uint_as_float(v1[j]);
         }
       } else {
-        // Pass 1: one ballot per query column; lane j keeps the ballots of
-        // columns j and 32 + j.  Pass 2: every lane reserves its two columns'
-        // slots with one atomic each, all in flight together.  Pass 3: the
-        // listed lanes write (score, bucket) at their slots.
+        // Pass 1: one ballot per query column (lane j keeps the ballots of
+        // columns j and 32 + j); each lane notes its listed (score, column)
+        // pairs in shared memory.  Pass 2: every lane reserves its two
+        // columns' slots with one atomic each, all in flight together, and
+        // publishes ballot and base.  Pass 3: each lane writes its own pairs.
+        uint32_t* scol = reinterpret_cast<uint32_t*>(sfilt + (warp - 2) * (C::SMEM_COL + C::SMEM_LST));
+        uint2* slst = reinterpret_cast<uint2*>(sfilt + (warp - 2) * (C::SMEM_COL + C::SMEM_LST) + C::SMEM_COL) +
+                      lane * C::LIST;
         uint32_t bal_a = 0, bal_b = 0;
+        int nl = 0;                                     // this lane's listed pairs
+        // one 32-column half at a time, so only 32 scores are live in registers.
+        // Listed: visible and score >= threshold (as floats: -0 equals +0, a
+        // NaN is never listed, a -inf threshold lists every visible bucket).
+        // A tile below every column's visible count skips the per-column count.
+        const bool all_visible = up.tile * C::BM + C::BM <= vis_min;
+        uint32_t v[32];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+          tmem_ld_32x32_nowait(col + 32 * h, v);
+          tmem_wait_ld(v);
+          if (h == 1) release();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const uint32_t thr = __shfl_sync(0xffffffffu, h ? thr_b : thr_a, j);
-            const int vis = __shfl_sync(0xffffffffu, h ? vis_b : vis_a, j);
-            const float sv = __uint_as_float(h ? v1[j] : v0[j]);
-            const bool take = (32 * h + j < nt) && (pc < vis) && order_code(sv) >= thr;
+            const float thr = __shfl_sync(0xffffffffu, h ? thr_b : thr_a, j);
+            const uint32_t sv = v[j];
+            bool take = __uint_as_float(sv) >= thr;
+            if (!all_visible) {                          // warp-uniform: every lane takes part in the shuffle
+              const int vis = __shfl_sync(0xffffffffu, h ? vis_b : vis_a, j);
+              take = take && (pc < vis);
+            }
             const uint32_t bal = __ballot_sync(0xffffffffu, take);
             if (lane == j) {
               if (h) bal_b = bal;
               else bal_a = bal;
+            }
+            if (take) {
+              if (nl < C::LIST) slst[nl] = make_uint2(sv, static_cast<uint32_t>(32 * h + j));
+              ++nl;
             }
           }
         }
@@ -288,27 +319,46 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
         if (bal_b)
           base_b = atomicAdd(p.cand_cnt + static_cast<int64_t>(t0 + 32 + lane) * p.nseg + blockIdx.x,
                              static_cast<uint32_t>(__popc(bal_b)));
+        scol[lane] = bal_a;
+        scol[32 + lane] = bal_b;
+        scol[64 + lane] = base_a;
+        scol[96 + lane] = base_b;
+        __syncwarp();
         const uint32_t below = (1u << lane) - 1u;
+        for (int e = 0; e < nl && e < C::LIST; ++e) {
+          const uint2 pr = slst[e];
+          const int c = static_cast<int>(pr.y);
+          const int t = t0 + c;
+          const uint32_t slot = scol[64 + c] + static_cast<uint32_t>(__popc(scol[c] & below));
+          if (slot < static_cast<uint32_t>(p.seg)) {
+            const int64_t at = (static_cast<int64_t>(t) * p.nseg + blockIdx.x) * p.seg + slot;
+            p.cand_val[at] = __uint_as_float(pr.x);
+            p.cand_lab[at] = pc;
+          } else {
+            p.row_over[t] = 1;
+            *p.any_over = 1;
+          }
+        }
+        if (nl > C::LIST) {
+          // more listed pairs than the lane's buffer holds: rescan for the
+          // columns it could not note and send those rows to the fallback
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < 2; ++h) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const uint32_t bal = __shfl_sync(0xffffffffu, h ? bal_b : bal_a, j);
-            const uint32_t base = __shfl_sync(0xffffffffu, h ? base_b : base_a, j);
-            if ((bal >> lane) & 1u) {
-              const int t = t0 + 32 * h + j;
-              const uint32_t slot = base + static_cast<uint32_t>(__popc(bal & below));
-              if (slot < static_cast<uint32_t>(p.seg)) {
-                const int64_t at = (static_cast<int64_t>(t) * p.nseg + blockIdx.x) * p.seg + slot;
-                p.cand_val[at] = __uint_as_float(h ? v1[j] : v0[j]);
-                p.cand_lab[at] = pc;
-              } else {
-                p.row_over[t] = 1;
-                *p.any_over = 1;
+            for (int j = 0; j < 32; ++j) {
+              const int c = 32 * h + j;
+              if (((h ? scol[32 + j] : scol[j]) >> lane) & 1u) {
+                bool noted = false;
+                for (int e = 0; e < C::LIST; ++e) noted |= (static_cast<int>(slst[e].y) == c);
+                if (!noted) {
+                  p.row_over[t0 + c] = 1;
+                  *p.any_over = 1;
+                }
               }
             }
           }
         }
+        __syncwarp();                                   // the warp's shared area is reused next unit
       }
     }
   }
