@@ -363,6 +363,18 @@ def _profiled_loop(L, fn, steps, warm, st):
     return tot / steps, kern
 
 
+def _recall(sel, exact):
+    """Mean over rows of |selected ∩ exact| / |exact| (padding -1 ignored)."""
+    import torch
+    hits, tot = 0, 0
+    for r in range(sel.shape[0]):
+        e = exact[r][exact[r] >= 0]
+        a = sel[r][sel[r] >= 0]
+        hits += int(torch.isin(a, e).sum())
+        tot += int(e.numel())
+    return hits / max(tot, 1)
+
+
 def bench_prefill(L, args, peaks, peak_kind, full_scores=True, fp8=False):
     """Prefill chunk: history streamed from pinned host memory in 8192-key
     tiles through two device buffers, causal top-512 of 4096 queries; with
@@ -461,13 +473,19 @@ def bench_bucket(L, args, peaks, peak_kind):
 
     ms, kern = _profiled_loop(L, bk, steps, warm, st)
     cms = kern["score_tc_kernel<8>"]["ms_per_step"]
+    # recall@k against the exact scan of every key (outside the timed region)
+    N_ = d["keys"].shape[0]
+    exact = L.ls_indexer_score(args_b[0].view(1, T, H, dd), args_b[1].view(1, T, H), args_b[5].view(1, N_, dd))
+    ei, _ = L.ls_topk_select(exact.view(T, N_), wl.k)
+    recall = _recall(outb[0], ei)
+    del exact
     flops = T * P_ * 2 * H * dd
     peak_t = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
     res = {"ms_per_step": ms, "positions_per_s": T * (P_ + wl.budget) / (ms * 1e-3),
            "selections_per_s": T / (ms * 1e-3), "kernels": kern,
            "roofline": roofline("tensor", flops / (cms * 1e-3) / 1e12, peak_t, "TFLOP/s",
                                 traffic=ncu_traffic("score_tc_kernel<8>", wl.name), peak_kind=peak_kind),
-           "algorithmic_flops_centroids": flops,
+           "algorithmic_flops_centroids": flops, "recall_at_k": recall,
            "note": "positions = centroids scored + keys rescored per query; roofline of the centroid scoring"}
     del args_b, wsb
     return res
@@ -555,12 +573,18 @@ def bench_two_stage(L, args, peaks, peak_kind, pq=False):
 
     ms, kern = _profiled_loop(L, ts, steps, warm, st)
     scan_ms = kern[scan_name]["ms_per_step"]
+    # recall@k against the exact full scan of the fp8 keys (outside the timed region)
+    nv = to_dev(d["n_valid"]) if d.get("n_valid") is not None else None
+    exact = L.ls_indexer_score(a2[0].view(B, 1, H, dd), a2[1].view(B, 1, H), fk[0], key_scale=fk[1], n_valid=nv)
+    ei, _ = L.ls_topk_select(exact.view(B, N), wl.k, n_valid=nv)
+    recall = _recall(out2[0], ei)
+    del exact
     res = {
         "ms_per_step": ms, "positions_per_s": B * (N + wl.shortlist) / (ms * 1e-3),
         "selections_per_s": B / (ms * 1e-3), "kernels": kern,
         "roofline": roofline("hbm", scan_bytes / (scan_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                              traffic=ncu_traffic(scan_name, wl.name), peak_kind=peak_kind),
-        "algorithmic_bytes_scan": scan_bytes,
+        "algorithmic_bytes_scan": scan_bytes, "recall_at_k": recall,
         "note": "positions = compact keys scanned + shortlist re-ranked; roofline of the compact scan "
                 + ("(32-byte PQ codes; codebooks stay in shared memory)" if pq else "(int8 codes + fp32 scales)"),
     }
