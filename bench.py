@@ -176,14 +176,28 @@ def to_dev(a):
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
 
-def source_digest() -> str:
-    """sha256 (first 16 hex digits) over the CUDA sources and the C header: a
-    DRAM-traffic figure taken from an ncu capture counts only while it matches."""
+# The device code each measured kernel's DRAM traffic depends on: its own
+# source file, the shared device helpers and the parameter structs.
+KERNEL_SOURCES = {
+    "score_tc_kernel": ["common.cuh", "kernels.h", "score_tc.cuh"],
+    "score_q8_kernel": ["common.cuh", "kernels.h", "score_q8.cuh"],
+    "dot_tc_kernel": ["common.cuh", "kernels.h", "score_dot.cuh"],
+}
+
+
+def source_digest(kernel: str = None) -> str:
+    """sha256 (first 16 hex digits) over the CUDA sources a kernel is built
+    from (every CUDA source and the C header when the kernel is not listed):
+    a DRAM-traffic figure taken from an ncu capture counts only while it matches."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_attention_indexer_lightning_b200", "csrc")
-    files = [os.path.join(csrc, f) for f in sorted(os.listdir(csrc))]
-    files.append(os.path.join(ROOT, "include", "ls_indexer.h"))
+    base = None if kernel is None else kernel.split("<")[0].split(":")[0]
+    if base in KERNEL_SOURCES:
+        files = [os.path.join(csrc, f) for f in KERNEL_SOURCES[base]]
+    else:
+        files = [os.path.join(csrc, f) for f in sorted(os.listdir(csrc))]
+        files.append(os.path.join(ROOT, "include", "ls_indexer.h"))
     for f in files:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
@@ -199,7 +213,7 @@ def ncu_traffic(kernel: str, workload: str):
             lines = f.read().splitlines()
     except OSError:
         return None
-    dig = source_digest()
+    dig = source_digest(kernel)
     for ln in lines:
         if not ln.strip() or ln.startswith("#"):
             continue
