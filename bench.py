@@ -353,7 +353,7 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
                      ("prefill_chunk_fp8", lambda *a: bench_prefill(*a, fp8=True)),
                      ("prefill_chunk_fp8_running", lambda *a: bench_prefill(*a, full_scores=False, fp8=True)),
                      ("bucket", bench_bucket), ("lsa_flat", bench_lsa),
-                     ("lsa_flat_threshold", lambda *a: bench_lsa(*a, threshold=True)),
+                     ("lsa_flat_threshold", lambda *a: bench_lsa(*a, threshold=True)), ("lsa_tree", bench_lsa_tree),
                      ("two_stage", bench_two_stage),
                      ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True))):
         if only in (None, name):
@@ -556,6 +556,49 @@ def bench_lsa(L, args, peaks, peak_kind, threshold=False):
     return res
 
 
+def bench_lsa_tree(L, args, peaks, peak_kind):
+    """LSA tree search on the lsa_flat sequence: 32768 node buckets scored,
+    beam 2048, their 8192 child buckets scored, top 1024, read lists."""
+    import torch
+    from workloads import get_workload, make_workload
+    st = torch.cuda.current_stream()
+    steps = max(3, args.steps)
+    warm = max(3, args.warmup)
+    wl = get_workload("lsa_tree")
+    d = make_workload(wl)
+    ex = wl.extra
+    T = d["q_idx"].shape[0]
+    P1 = d["node_centroids"].shape[0]
+    a = [to_dev_bf16(d["q_idx"]), to_dev(d["q_pos"]), to_dev_bf16(d["centroids"]), to_dev_bf16(d["node_centroids"]),
+         to_dev(d["bucket_off"]), to_dev(d["bucket_mem"])]
+    ws = torch.empty(L.lib().ls_lsa_tree_workspace_size(T, P1, ex["beam"], ex["fanout"], ex["node_block"], wl.top_p),
+                     dtype=torch.uint8, device="cuda")
+    row = ex["n_sink"] + ex["block_keys"] + wl.budget
+    out = (torch.empty((T, row), dtype=torch.int32, device="cuda"), torch.empty((T,), dtype=torch.int32, device="cuda"))
+
+    def run(i, timed):
+        L.ls_lsa_tree_select(*a, block_keys=ex["block_keys"], buckets_per_block=ex["bpb"], node_block=ex["node_block"],
+                             fanout=ex["fanout"], beam=ex["beam"], n_sink=ex["n_sink"], top_p=wl.top_p,
+                             budget=wl.budget, ws=ws, out=out)
+        return None
+
+    ms, kern = _profiled_loop(L, run, steps, warm, st)
+    scored = T * (P1 + ex["beam"] * ex["fanout"])
+    nms = kern["dot_tc_kernel:nodes"]["ms_per_step"]
+    bytes_nodes = P1 * 128 + T * 128 + T * P1 * 4
+    peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    res = {"ms_per_step": ms, "positions_per_s": scored / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
+           "kernels": kern,
+           "roofline": roofline("hbm", bytes_nodes / (nms * 1e-3) / 1e9, peak_b, "GB/s",
+                                traffic=ncu_traffic("dot_tc_kernel", wl.name), peak_kind=peak_kind),
+           "vectors_scored_per_query": P1 + ex["beam"] * ex["fanout"],
+           "note": "positions = node buckets + child buckets scored per query (32768 + 8192 against 131072 for "
+                   "the flat search); roofline of the node scoring (node centroids and queries read, scores "
+                   "written)"}
+    del a, ws
+    return res
+
+
 def bench_two_stage(L, args, peaks, peak_kind, pq=False):
     """Two-stage decode search: compact scan (int8 + scale, or 32-byte PQ codes), shortlist, exact re-rank."""
     import torch
@@ -680,7 +723,8 @@ def main(argv=None):
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "prefill_chunk_fp8",
                                                      "prefill_chunk_fp8_running", "bucket", "lsa_flat",
-                                                     "lsa_flat_threshold", "two_stage", "two_stage_pq"],
+                                                     "lsa_flat_threshold", "lsa_tree", "two_stage",
+                                                     "two_stage_pq"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

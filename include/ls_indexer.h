@@ -304,6 +304,33 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
                              void* stream);
 
 /*
+ * ls_lsa_tree_select -- the LSA tree search's beam over one level of node
+ * buckets ("Latent Sparse Attention", section "The tree, step by step"):
+ * every node_block buckets form a node cluster block, grouped fanout to a
+ * node bucket (node n covers buckets fanout*n .. fanout*n + fanout - 1; nodes
+ * exist for complete node blocks only).  A query scores the node buckets of
+ * the complete node blocks among its visible buckets, keeps the best `beam`,
+ * steps down to their children plus the visible buckets no node covers yet,
+ * picks the best top_p of those and reads them as ls_lsa_flat_select does.
+ *
+ *   node_centroids [P1][64] bf16 unit centroids of the node buckets
+ *   beam_out [T][beam] int32 picked node buckets, best first (or NULL)
+ *   other arguments and outputs as in ls_lsa_flat_select
+ * With beam >= every visible node bucket the picks are those of the flat
+ * search.  Only d = 64 and one node level are built (the pages start the
+ * beam at the lowest level with at most 32768 node buckets: level 1 up to
+ * 1M tokens).
+ * Workspace: ls_lsa_tree_workspace_size(T, P1, beam, fanout, node_block, top_p) bytes.
+ */
+size_t ls_lsa_tree_workspace_size(int T, int P1, int beam, int fanout, int node_block, int top_p);
+ls_status ls_lsa_tree_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
+                             const uint16_t* node_centroids, const int32_t* bucket_off, const int32_t* bucket_mem,
+                             int T, int d, int P, int P1, int block_keys, int buckets_per_block, int node_block,
+                             int fanout, int beam, int n_sink, int top_p, int budget, int32_t* keys_out,
+                             int32_t* n_out, int32_t* picked_out, int32_t* beam_out, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/*
  * ls_decode_two_stage_select -- LeanSparse two-stage decode search
  * (podcast transcript, 07:12-08:00): scan compact keys, keep a shortlist,
  * fetch the shortlist's original keys and re-rank exactly, keep the top k.

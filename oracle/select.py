@@ -31,6 +31,10 @@ Pipelines:
   that fall in the sinks or the window until the budget is held (the last
   bucket cut short); the read list is the sinks, the window (the query's own
   block up to the query) and those long-range keys.
+* LSA tree search, one node level ("Latent Sparse Attention", "The tree, step
+  by step"): node buckets group 4 buckets of a complete 4096-bucket block;
+  the beam keeps the best node buckets, the search steps down to their
+  children plus the uncovered buckets and picks the top-p there.
 * bucket search ("Latent Sparse Attention", "How LSA finds the keys" and "The
   method, term by term", steps 5-6): score every bucket centroid with the
   indexer score, keep the top-p buckets, read them best first appending their
@@ -265,6 +269,41 @@ def lsa_flat_select(q_idx_bits, q_pos, centroid_bits, bucket_off, bucket_mem, bl
         picked, _ = select_topk(scores, np.arange(v), top_p)
         out.append(lsa_read_list(picked, q_pos[t], bucket_off, bucket_mem, block_keys, n_sink, budget))
         detail.append({"scores": scores, "picked": picked, "visible": v})
+    if return_detail:
+        return out, detail
+    return out
+
+
+def lsa_tree_select(q_idx_bits, q_pos, centroid_bits, node_bits, bucket_off, bucket_mem, block_keys: int,
+                    buckets_per_block: int, node_block: int, fanout: int, beam: int, n_sink: int, top_p: int,
+                    budget: int, rows=None, return_detail: bool = False):
+    """Read lists of the LSA tree search with one level of node buckets
+    ("Latent Sparse Attention", "The tree, step by step"): score the node
+    buckets of the complete node blocks among the query's visible buckets,
+    keep the best ``beam``, step down to their children plus the visible
+    buckets no node covers, pick the top-p of those, read them."""
+    T = q_idx_bits.shape[0]
+    P = centroid_bits.shape[0]
+    P1 = node_bits.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    cent = bf16_to_f64(centroid_bits)
+    nodes = bf16_to_f64(node_bits)
+    vis = lsa_visible(q_pos, block_keys, buckets_per_block, P)
+    out, detail = [], []
+    for t in rows:
+        v = int(vis[t])
+        vn = min((v // node_block) * (node_block // fanout), P1)
+        qv = bf16_to_f64(q_idx_bits[t])
+        node_scores = nodes[:vn] @ qv
+        kept, _ = select_topk(node_scores, np.arange(vn), beam)
+        kept = kept[kept >= 0]
+        cand = [int(n) * fanout + c for n in kept for c in range(fanout)] + list(range(vn * fanout, v))
+        cand = np.asarray(cand, dtype=np.int64)
+        scores = cent[cand] @ qv if cand.size else np.zeros(0)
+        picked, _ = select_topk(scores, cand, top_p)
+        out.append(lsa_read_list(picked, q_pos[t], bucket_off, bucket_mem, block_keys, n_sink, budget))
+        detail.append({"node_scores": node_scores, "beam": kept, "visible_nodes": vn, "candidates": cand,
+                       "scores": scores, "picked": picked, "visible": v})
     if return_detail:
         return out, detail
     return out

@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     ls_indexer_score_fp8,
     ls_indexer_score_pq,
     ls_lsa_flat_select,
+    ls_lsa_tree_select,
     ls_prefill_select_stream,
     ls_prefill_select_stream_fp8,
     ls_profile_begin,

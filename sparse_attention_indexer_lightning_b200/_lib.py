@@ -38,7 +38,7 @@ EXPORTED = (
     "ls_profile_end", "ls_profile_kernel", "ls_decode_select_noalloc", "ls_decode_two_stage_pq_select",
     "ls_indexer_score_pq", "ls_indexer_score_fp8_workspace_size", "ls_indexer_score_fp8",
     "ls_prefill_select_fp8_workspace_size", "ls_prefill_select_stream_fp8", "ls_lsa_flat_workspace_size",
-    "ls_lsa_flat_select",
+    "ls_lsa_flat_select", "ls_lsa_tree_workspace_size", "ls_lsa_tree_select",
 )
 HIST_BINS = 2048
 
@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_prefill_select_stream_fp8": (I, [P, P, P, P, I, I, I, P, P, I, I, I, P, P, I, I, P, P, P, SZ, P, P]),
         "ls_lsa_flat_workspace_size": (SZ, [I, I, I, I]),
         "ls_lsa_flat_select": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
+        "ls_lsa_tree_workspace_size": (SZ, [I, I, I, I, I, I]),
+        "ls_lsa_tree_select": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -477,6 +479,36 @@ def ls_lsa_flat_select(q_idx, q_pos, centroids, bucket_off, bucket_mem, block_ke
                                     _ptr(keys),
                                     _ptr(n), _ptr(picked), _ptr(ws), ws.numel(), _stream(stream)))
     return (keys, n, picked) if want_picked else (keys, n)
+
+
+def ls_lsa_tree_select(q_idx, q_pos, centroids, node_centroids, bucket_off, bucket_mem, block_keys: int = 512,
+                       buckets_per_block: int = 64, node_block: int = 4096, fanout: int = 4, beam: int = 2048,
+                       n_sink: int = 4, top_p: int = 1024, budget: int = 4096, want_picked: bool = False,
+                       ws=None, out=None, stream=None):
+    """LSA tree search over one level of node buckets.  As ls_lsa_flat_select, plus node_centroids [P1,64]
+    bf16; with want_picked also returns (picked [T, top_p], beam [T, beam]) int32."""
+    _dev(q_idx, torch.bfloat16, "q_idx", 2)
+    T, d = q_idx.shape
+    _dev(q_pos, torch.int64, "q_pos", 1)
+    _dev(centroids, torch.bfloat16, "centroids", 2)
+    _dev(node_centroids, torch.bfloat16, "node_centroids", 2)
+    P, P1 = centroids.shape[0], node_centroids.shape[0]
+    _dev(bucket_off, torch.int32, "bucket_off", 1)
+    _dev(bucket_mem, torch.int32, "bucket_mem", 1)
+    need = lib().ls_lsa_tree_workspace_size(T, P1, beam, fanout, node_block, top_p)
+    if ws is None:
+        ws = _workspace(need, q_idx.device)
+    if out is None:
+        out = (torch.empty((T, n_sink + block_keys + budget), dtype=torch.int32, device=q_idx.device),
+               torch.empty((T,), dtype=torch.int32, device=q_idx.device))
+    keys, n = out
+    picked = torch.empty((T, top_p), dtype=torch.int32, device=q_idx.device) if want_picked else None
+    bm = torch.empty((T, beam), dtype=torch.int32, device=q_idx.device) if want_picked else None
+    _check(lib().ls_lsa_tree_select(_ptr(q_idx), _ptr(q_pos), _ptr(centroids), _ptr(node_centroids),
+                                    _ptr(bucket_off), _ptr(bucket_mem), T, d, P, P1, block_keys, buckets_per_block,
+                                    node_block, fanout, beam, n_sink, top_p, budget, _ptr(keys), _ptr(n),
+                                    _ptr(picked), _ptr(bm), _ptr(ws), ws.numel(), _stream(stream)))
+    return (keys, n, picked, bm) if want_picked else (keys, n)
 
 
 def ls_device_status(stream=None) -> int:

@@ -20,6 +20,7 @@
 #include "misc.cuh"
 #include "score_cvt.cuh"
 #include "score_dot.cuh"
+#include "score_tree.cuh"
 #include "score_q8.cuh"
 #include "score_tc.cuh"
 #include "topk.cuh"
@@ -1134,6 +1135,108 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
     ls_status s = topk_launch(tp, st);
     if (s != LS_OK) return s;
   }
+  ProfScope prof("lsa_expand_kernel", st);
+  LS_CUDA(launch_lsa_expand(picked, q_pos, T, top_p, bucket_off, bucket_mem, P, block_keys, n_sink, budget, keys_out,
+                            n_sink + block_keys + budget, n_out, st));
+  return LS_OK;
+}
+
+size_t ls_lsa_tree_workspace_size(int T, int P1, int beam, int fanout, int node_block, int top_p) {
+  if (T <= 0 || beam <= 0 || fanout <= 0 || node_block <= 0 || top_p <= 0 || P1 < 0) return 0;
+  const size_t cap = static_cast<size_t>(beam) * fanout + node_block;
+  return align_up(static_cast<size_t>(T) * P1 * sizeof(float)) +       // node scores
+         align_up(static_cast<size_t>(T) * sizeof(int32_t)) * 3 +       // visible buckets, nodes, list lengths
+         align_up(static_cast<size_t>(T) * beam * sizeof(int32_t)) +    // the beam
+         align_up(static_cast<size_t>(T) * cap * sizeof(float)) +       // candidate scores
+         align_up(static_cast<size_t>(T) * cap * sizeof(int32_t)) +     // candidate buckets
+         align_up(static_cast<size_t>(T) * top_p * sizeof(int32_t));    // picked buckets
+}
+
+ls_status ls_lsa_tree_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
+                             const uint16_t* node_centroids, const int32_t* bucket_off, const int32_t* bucket_mem,
+                             int T, int d, int P, int P1, int block_keys, int buckets_per_block, int node_block,
+                             int fanout, int beam, int n_sink, int top_p, int budget, int32_t* keys_out,
+                             int32_t* n_out, int32_t* picked_out, int32_t* beam_out, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (d != kLsaDim) return fail(LS_ERR_UNSUPPORTED, "only d=%d is built for the LSA index space (got %d)", kLsaDim, d);
+  LS_CHECK_ARG(T >= 0 && P >= 0 && P1 >= 0, "negative size");
+  LS_CHECK_ARG(block_keys >= 1 && buckets_per_block >= 1, "block_keys and buckets_per_block must be >= 1");
+  LS_CHECK_ARG(fanout >= 1 && node_block >= fanout && node_block % fanout == 0,
+               "node_block must be a positive multiple of fanout");
+  LS_CHECK_ARG(static_cast<int64_t>(P1) * fanout <= P, "P1 * fanout (%lld) exceeds P (%d)",
+               static_cast<long long>(P1) * fanout, P);
+  LS_CHECK_ARG(n_sink >= 0 && budget >= 1, "n_sink must be >= 0 and budget >= 1");
+  LS_CHECK_ARG(top_p >= 1 && top_p <= kMaxTopK, "top_p must be in [1, %d] (got %d)", kMaxTopK, top_p);
+  LS_CHECK_ARG(beam >= 1 && beam <= kMaxTopK, "beam must be in [1, %d] (got %d)", kMaxTopK, beam);
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(q_idx && q_pos && centroids && bucket_off && bucket_mem && keys_out && n_out, "null tensor pointer");
+  LS_CHECK_ARG(P1 == 0 || node_centroids != nullptr, "null node_centroids");
+  LS_CHECK_ARG(aligned16(q_idx) && aligned16(centroids) && (P1 == 0 || aligned16(node_centroids)),
+               "q_idx and the centroids must be 16-byte aligned");
+  const size_t need = ls_lsa_tree_workspace_size(T, P1, beam, fanout, node_block, top_p);
+  if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  const int cap = beam * fanout + node_block;
+  Carver cv(ws);
+  float* sc1 = cv.take<float>(static_cast<size_t>(T) * P1);
+  int32_t* vis = cv.take<int32_t>(T);
+  int32_t* vis_nodes = cv.take<int32_t>(T);
+  int32_t* nv = cv.take<int32_t>(T);
+  int32_t* beam_ws = cv.take<int32_t>(static_cast<size_t>(T) * beam);
+  float* cval = cv.take<float>(static_cast<size_t>(T) * cap);
+  int32_t* clab = cv.take<int32_t>(static_cast<size_t>(T) * cap);
+  int32_t* picked_ws = cv.take<int32_t>(static_cast<size_t>(T) * top_p);
+  int32_t* bm = beam_out ? beam_out : beam_ws;
+  int32_t* picked = picked_out ? picked_out : picked_ws;
+  cudaStream_t st = S(stream);
+  {
+    ProfScope prof("lsa_tree_visible_kernel", st);
+    LS_CUDA(launch_lsa_tree_visible(q_pos, T, block_keys, buckets_per_block, P, node_block, fanout, P1, vis, vis_nodes,
+                                    st));
+  }
+  // the beam: the best node buckets among each query's visible ones
+  if (P1 > 0) {
+    CUtensorMap cmap, qmap;
+    ls_status s = make_vec64_map(&cmap, node_centroids, static_cast<uint64_t>(P1), kTileKeys);
+    if (s != LS_OK) return s;
+    s = make_vec64_map(&qmap, q_idx, static_cast<uint64_t>(T), DotCfg::QB);
+    if (s != LS_OK) return s;
+    DotParams dp;
+    dp.T = T;
+    dp.P = P1;
+    dp.out = sc1;
+    dp.ld_out = P1;
+    ProfScope prof("dot_tc_kernel:nodes", st);
+    LS_CUDA(launch_dot_tc(&cmap, &qmap, dp, num_sms_current(), st));
+  }
+  TopkParams bp;
+  bp.scores = sc1;
+  bp.ld = P1;
+  bp.n_valid = vis_nodes;
+  bp.R = T;
+  bp.N = P1;
+  bp.k = beam;
+  bp.idx_out = bm;
+  bp.ld_out = beam;
+  ls_status s = topk_launch(bp, st, "topk_kernel:beam");
+  if (s != LS_OK) return s;
+  // the beam's children and the uncovered buckets, scored; their top-p
+  {
+    ProfScope prof("lsa_tree_candidates_kernel", st);
+    LS_CUDA(launch_lsa_tree_candidates(q_idx, centroids, bm, beam, vis, vis_nodes, T, fanout, cap, cval, clab, nv, st));
+  }
+  TopkParams cp;
+  cp.scores = cval;
+  cp.ld = cap;
+  cp.n_valid = nv;
+  cp.labels = clab;
+  cp.ld_labels = cap;
+  cp.R = T;
+  cp.N = cap;
+  cp.k = top_p;
+  cp.idx_out = picked;
+  cp.ld_out = top_p;
+  s = topk_launch(cp, st);
+  if (s != LS_OK) return s;
   ProfScope prof("lsa_expand_kernel", st);
   LS_CUDA(launch_lsa_expand(picked, q_pos, T, top_p, bucket_off, bucket_mem, P, block_keys, n_sink, budget, keys_out,
                             n_sink + block_keys + budget, n_out, st));

@@ -14,8 +14,8 @@ import torch
 from oracle.formats import bf16_to_f64, dequant, pq_decode
 from oracle.indexer import eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, expand_buckets, lsa_flat_select, lsa_read_list, recall_at_k, select_topk, topk_rows,
-    two_stage_pq_select, two_stage_select,
+    bucket_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_select, recall_at_k, select_topk,
+    topk_rows, two_stage_pq_select, two_stage_select,
 )
 from parity_util import (
     RTOL_BF16, RTOL_FP8, check_scores, check_selection, check_set, dev, dev_bf16, dev_e4m3, f32_bits_equal,
@@ -624,6 +624,52 @@ def test_lsa_threshold_fallbacks(L):
         d["q_idx"] = to_bf16_bits(np.broadcast_to(u, base["q_idx"].shape).copy())
         d["centroids"] = to_bf16_bits(cent)
         _check_lsa(L, "lsa_flat_s", list(range(37)), d=d, wl=wl)
+
+
+def _check_lsa_tree(L, name, rows, beam=None):
+    wl = get_workload(name)
+    d = data(name)
+    ex = wl.extra
+    beam = beam or ex["beam"]
+    fan, nblk = ex["fanout"], ex["node_block"]
+    keys, n, picked, bm = L.ls_lsa_tree_select(
+        dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]), dev_bf16(d["node_centroids"]),
+        dev(d["bucket_off"]), dev(d["bucket_mem"]), block_keys=ex["block_keys"], buckets_per_block=ex["bpb"],
+        node_block=nblk, fanout=fan, beam=beam, n_sink=ex["n_sink"], top_p=wl.top_p, budget=wl.budget,
+        want_picked=True)
+    keys, n, picked, bm = keys.cpu().numpy(), n.cpu().numpy(), picked.cpu().numpy(), bm.cpu().numpy()
+    _, det = lsa_tree_select(d["q_idx"], d["q_pos"], d["centroids"], d["node_centroids"], d["bucket_off"],
+                             d["bucket_mem"], ex["block_keys"], ex["bpb"], nblk, fan, beam, ex["n_sink"], wl.top_p,
+                             wl.budget, rows=rows, return_detail=True)
+    cent = bf16_to_f64(d["centroids"])
+    for i, t in enumerate(rows):
+        vn, v = det[i]["visible_nodes"], det[i]["visible"]
+        check_set(bm[t], np.arange(vn), det[i]["node_scores"], beam, RTOL_BF16, f"{name} beam row {t}")
+        # candidates from the GPU's beam: its children, then the uncovered buckets
+        kept = bm[t][bm[t] >= 0]
+        cand = np.asarray([int(x) * fan + c for x in kept for c in range(fan)] + list(range(vn * fan, v)),
+                          dtype=np.int64)
+        ref = cent[cand] @ bf16_to_f64(d["q_idx"][t]) if cand.size else np.zeros(0)
+        check_set(picked[t], cand, ref, wl.top_p, RTOL_BF16, f"{name} picked row {t}")
+        want = lsa_read_list(picked[t], d["q_pos"][t], d["bucket_off"], d["bucket_mem"], ex["block_keys"],
+                             ex["n_sink"], wl.budget)
+        assert n[t] == want.size and np.array_equal(keys[t, :n[t]], want), f"{name} read list row {t}"
+        assert np.all(keys[t, n[t]:] == -1)
+
+
+def test_lsa_tree_small(L):
+    _check_lsa_tree(L, "lsa_flat_s", list(range(37)))
+
+
+def test_lsa_tree_full_beam_matches_flat(L):
+    """A beam covering every node bucket reads what the flat search reads
+    (band rule on the picks: the two paths score on different units)."""
+    _check_lsa_tree(L, "lsa_flat_s", list(range(37)), beam=4096)
+
+
+@pytest.mark.slow
+def test_lsa_tree_full_size_sampled(L):
+    _check_lsa_tree(L, "lsa_tree", [0, 1, 100, 254, 255])
 
 
 def test_bucket_bad_member_flagged(L):

@@ -17,7 +17,8 @@ from oracle import brute, sizes
 from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64, f16_to_f64, pq_decode
 from oracle.indexer import eligible_blocks, eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, decode_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_visible, prefill_select,
+    bucket_select, decode_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_select, lsa_visible,
+    prefill_select,
     prefill_select_fp8, recall_at_k, select_topk, topk_rows, two_stage_pq_select, two_stage_select,
 )
 from workloads import make_workload
@@ -430,6 +431,53 @@ def test_lsa_brute_force_tiny():
                 want.append(int(m))
     assert out[0].tolist() == want
     assert lsa_read_list(bp, t, d["bucket_off"], d["bucket_mem"], 512, 4, 100).tolist() == want
+
+
+def test_lsa_tree_with_full_beam_equals_flat():
+    """A beam holding every visible node bucket steps down to every visible
+    bucket: the tree search reads what the flat search reads."""
+    d = make_workload("lsa_flat_s")
+    args = (d["q_idx"], d["q_pos"], d["centroids"])
+    flat = lsa_flat_select(*args, d["bucket_off"], d["bucket_mem"], 512, 64, 4, 64, 512)
+    tree = lsa_tree_select(*args, d["node_centroids"], d["bucket_off"], d["bucket_mem"], 512, 64, 4096, 4, 4096,
+                           4, 64, 512)
+    for t in range(d["q_pos"].size):
+        assert np.array_equal(flat[t], tree[t]), t
+
+
+def test_lsa_tree_brute_force_tiny():
+    """Pure-Python node scores, beam, children + uncovered buckets, picks."""
+    d = make_workload("lsa_flat_s")
+    t = int(np.argmax(d["q_pos"]))
+    v = min((int(d["q_pos"][t]) // 512) * 64, d["centroids"].shape[0])
+    vn = (v // 4096) * 1024
+    assert vn > 0 and v > vn * 4
+    q = bf16_to_f64(d["q_idx"][t:t + 1])[0].tolist()
+    nodes = bf16_to_f64(d["node_centroids"]).tolist()
+    cent = bf16_to_f64(d["centroids"]).tolist()
+    ns = [sum(a * b for a, b in zip(nodes[n], q)) for n in range(vn)]
+    beam, _ = brute.topk(ns, list(range(vn)), 7)
+    cand = [4 * n + c for n in beam for c in range(4)] + list(range(vn * 4, v))
+    cs = [sum(a * b for a, b in zip(cent[p], q)) for p in cand]
+    picked, _ = brute.topk(cs, cand, 20)
+    out, det = lsa_tree_select(d["q_idx"], d["q_pos"], d["centroids"], d["node_centroids"], d["bucket_off"],
+                               d["bucket_mem"], 512, 64, 4096, 4, 7, 4, 20, 100, rows=[t], return_detail=True)
+    assert det[0]["beam"].tolist() == beam
+    assert det[0]["picked"].tolist() == picked
+    assert out[0].tolist() == lsa_read_list(picked, d["q_pos"][t], d["bucket_off"], d["bucket_mem"], 512, 4,
+                                            100).tolist()
+
+
+def test_lsa_generator_node_centroids():
+    """Node centroid = the normalised sum of its 4 children's key sums, each
+    taken as size x centroid."""
+    d = make_workload("lsa_flat_s")
+    sizes = np.diff(d["bucket_off"]).astype(np.float64)
+    c = bf16_to_f64(d["centroids"])
+    n = bf16_to_f64(d["node_centroids"])
+    for j in (0, 1, 511, 1023):
+        s = (c[4 * j:4 * j + 4] * sizes[4 * j:4 * j + 4, None]).sum(axis=0)
+        assert np.allclose(n[j], s / np.linalg.norm(s), atol=2 ** -8)
 
 
 def test_two_stage_full_shortlist_equals_exact():

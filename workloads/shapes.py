@@ -113,6 +113,13 @@ WORKLOADS: Dict[str, Workload] = {
         "lsa_flat", "lsa", T=256, N=1048576, top_p=1024, budget=4096,
         extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "spread": 2053},
     ),
+    # its tree search: 32768 node buckets (4 buckets each), beam 2048
+    # ("Latent Sparse Attention", "The tree, step by step")
+    "lsa_tree": Workload(
+        "lsa_tree", "lsa", T=256, N=1048576, top_p=1024, budget=4096,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "spread": 2053, "node_block": 4096, "fanout": 4,
+               "beam": 2048},
+    ),
     # ---- reduced parity cases: several tiles, ragged tails ------------------
     "decode_s": Workload("decode_s", "decode", B=5, N=3000, ragged=700),
     "prefill_s": Workload(
@@ -130,7 +137,7 @@ WORKLOADS: Dict[str, Workload] = {
     ),
     "lsa_flat_s": Workload(
         "lsa_flat_s", "lsa", T=37, N=40000, top_p=64, budget=512,
-        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "edge": 1},
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "edge": 1, "node_block": 4096, "fanout": 4, "beam": 96},
     ),
     "bucket_s": Workload(
         "bucket_s", "bucket", T=19, clusters=1500, cluster_size=8, noise_rel=0.3, top_p=64, budget=512,

@@ -305,7 +305,9 @@ def make_lsa(
     (4..16 keys; the grouping stands in for the Ward merges, drawn at random
     here), members stored in ascending position order (CSR ``bucket_off`` /
     ``bucket_mem``, buckets block-major).  Centroids and index queries are
-    random 64-d unit vectors rounded to bf16.  Query positions: the last
+    random 64-d unit vectors rounded to bf16; node buckets for the tree
+    search group every 4 buckets of each complete 4096-bucket block.  Query
+    positions: the last
     token and every ``spread``-th token before it, or (``edge``) the block
     edges 0, 3, 4, 511, 512, ... followed by random positions."""
     rng = np.random.default_rng(seed)
@@ -335,6 +337,17 @@ def make_lsa(
     c /= np.linalg.norm(c, axis=1, keepdims=True)
     q = rng.standard_normal((T, dim))
     q /= np.linalg.norm(q, axis=1, keepdims=True)
+    # node buckets for the tree search: every node_block buckets form a node
+    # cluster block grouped 4 to a node (complete node blocks only); a node's
+    # centroid is the normalised sum of its children's key sums, each child's
+    # key sum taken as size x centroid (the synthetic buckets have no keys)
+    node_block, fanout = 4096, 4
+    P1 = (P // node_block) * (node_block // fanout)
+    sizes = np.diff(off)[:P1 * fanout].astype(np.float64)
+    cb = bf16_bits_to_f32(to_bf16_bits(c[:P1 * fanout])).astype(np.float64)
+    nsum = (cb * sizes[:, None]).reshape(P1, fanout, dim).sum(axis=1)
+    norms = np.linalg.norm(nsum, axis=1, keepdims=True)
+    nc = nsum / np.where(norms > 0, norms, 1.0)
     if edge:
         fixed = [0, 3, 4, 511, 512, 513, 1023, 1024, 1536, 2047, 2048, L - 1]
         rest = np.sort(rng.integers(0, L, size=max(0, T - len(fixed))))
@@ -342,7 +355,8 @@ def make_lsa(
     else:
         q_pos = (L - 1 - spread * np.arange(T)).astype(np.int64)
     return {"q_idx": to_bf16_bits(q), "q_pos": q_pos, "centroids": to_bf16_bits(c),
-            "bucket_off": off.astype(np.int32), "bucket_mem": members}
+            "bucket_off": off.astype(np.int32), "bucket_mem": members,
+            "node_centroids": to_bf16_bits(nc) if P1 else np.zeros((0, dim), dtype=np.uint16)}
 
 
 def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
