@@ -558,8 +558,14 @@ __global__ void __launch_bounds__(kExpandThreads)
       if (pb >= 0 && pb < P) {
         o[i] = off[pb];
         const int n = max(0, off[pb + 1] - o[i]);
-        lo[i] = lower_bound_i32(mem + o[i], n, n_sink);             // members below the sinks' end
-        sz[i] = lower_bound_i32(mem + o[i], n, wstart) - lo[i];     // members before the window
+        // members below the sinks' end / before the window; members are
+        // ascending, so a bucket whose first member clears the sinks and whose
+        // last precedes the window (every bucket outside block 0) needs no search
+        if (n > 0) {
+          const int32_t first = mem[o[i]], last = mem[o[i] + n - 1];
+          lo[i] = (first >= n_sink) ? 0 : lower_bound_i32(mem + o[i], n, n_sink);
+          sz[i] = ((last < wstart) ? n : lower_bound_i32(mem + o[i], n, wstart)) - lo[i];
+        }
       }
       mine += sz[i];
     }
