@@ -29,7 +29,7 @@ def test_header_declares_the_calls():
     names = declared_functions()
     for n in ("ls_indexer_score", "ls_topk_select", "ls_prefill_select_stream", "ls_decode_two_stage_select",
               "ls_bucket_select", "ls_decode_select", "ls_last_error", "ls_device_status", "ls_indexer_score_fp8",
-              "ls_prefill_select_stream_fp8", "ls_lsa_flat_select", "ls_indexer_score_pq",
+              "ls_prefill_select_stream_fp8", "ls_lsa_flat_select", "ls_lsa_tree_select", "ls_indexer_score_pq",
               "ls_decode_two_stage_pq_select"):
         assert n in names
 
@@ -58,6 +58,8 @@ def test_version_and_workspace_queries(lib):
             >= lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 1) + 4096 * 32 * 4)
     # LSA: the T x P bucket scores, visible counts and picks
     assert lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) >= 256 * 131072 * 4 + 256 * 1024 * 4
+    # LSA tree: node scores, beam and candidates (beam * fanout + node_block per row)
+    assert lib.ls_lsa_tree_workspace_size(256, 32768, 2048, 4, 4096, 1024) >= 256 * 32768 * 4 + 256 * 12288 * 8
     # the threshold form adds the samples and the candidate lists (8 * top_p per row)
     assert (lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 1)
             >= lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) + 256 * 8192 * 8)
@@ -114,6 +116,18 @@ def test_argument_checks_without_gpu(lib):
                                   None, dummy, 8, None) == 2
     assert lib.ls_lsa_flat_select(None, None, None, None, None, 0, 64, 64, 512, 64, 4, 16, 64, 1, None, None, None,
                                   None, 0, None) == 0
+    # LSA tree: d != 64, beam too large, more node children than buckets, short workspace, empty batch
+    tree = lib.ls_lsa_tree_select
+    assert tree(dummy, dummy, dummy, dummy, dummy, dummy, 4, 128, 4096, 1024, 512, 64, 4096, 4, 96, 4, 64, 512, dummy,
+                dummy, None, None, dummy, 1 << 30, None) == 3
+    assert tree(dummy, dummy, dummy, dummy, dummy, dummy, 4, 64, 4096, 1024, 512, 64, 4096, 4, 5000, 4, 64, 512, dummy,
+                dummy, None, None, dummy, 1 << 30, None) == 1
+    assert tree(dummy, dummy, dummy, dummy, dummy, dummy, 4, 64, 4096, 1025, 512, 64, 4096, 4, 96, 4, 64, 512, dummy,
+                dummy, None, None, dummy, 1 << 30, None) == 1
+    assert tree(dummy, dummy, dummy, dummy, dummy, dummy, 4, 64, 4096, 1024, 512, 64, 4096, 4, 96, 4, 64, 512, dummy,
+                dummy, None, None, dummy, 16, None) == 2
+    assert tree(None, None, None, None, None, None, 0, 64, 4096, 1024, 512, 64, 4096, 4, 96, 4, 64, 512, None, None,
+                None, None, None, 0, None) == 0
     # bucket: budget below k
     st = lib.ls_bucket_select(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 128, 10, 80, 4, 100, 512, dummy,
                               None, None, dummy, 1 << 30, None)
