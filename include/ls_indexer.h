@@ -331,6 +331,26 @@ ls_status ls_lsa_tree_select(const uint16_t* q_idx, const int64_t* q_pos, const 
                              void* stream);
 
 /*
+ * ls_merge_select -- the combine step of a prefill whose history is split into
+ * S contiguous shards (one per GPU, say): each shard's exact top-k lists of
+ * the same T queries are merged into the top-k of the whole history (the
+ * top-k of the union of the shards' top-k lists is the global top-k, since
+ * every shard contributes its own best).
+ *
+ *   vals [S][T][k_in] fp32, idx [S][T][k_in] int32: list s of query t, in
+ *        canonical order, positions local to shard s, padded with -1 / -inf
+ *        at the end (the output form of ls_prefill_select_stream)
+ *   offsets [S] int32 (device): shard s's first position in the history
+ *   idx_out [T][k] int32 global positions, val_out [T][k] fp32 (or NULL)
+ * Ordering and padding as everywhere (score descending, position ascending;
+ * -1 / -inf past the end); values are bit copies of the inputs.
+ * Workspace: ls_merge_select_workspace_size(S, T, k_in) bytes.
+ */
+size_t ls_merge_select_workspace_size(int S, int T, int k_in);
+ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* offsets, int S, int T, int k_in,
+                          int k, int32_t* idx_out, float* val_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * ls_decode_two_stage_select -- LeanSparse two-stage decode search
  * (podcast transcript, 07:12-08:00): scan compact keys, keep a shortlist,
  * fetch the shortlist's original keys and re-rank exactly, keep the top k.

@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     ls_indexer_score_pq,
     ls_lsa_flat_select,
     ls_lsa_tree_select,
+    ls_merge_select,
     ls_prefill_select_stream,
     ls_prefill_select_stream_fp8,
     ls_profile_begin,
@@ -30,4 +31,5 @@ from ._lib import (  # noqa: F401
     ls_selftest_wait_probe,
     ls_topk_select,
     lib,
+    shard_plan,
 )

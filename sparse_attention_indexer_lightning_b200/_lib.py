@@ -38,7 +38,8 @@ EXPORTED = (
     "ls_profile_end", "ls_profile_kernel", "ls_decode_select_noalloc", "ls_decode_two_stage_pq_select",
     "ls_indexer_score_pq", "ls_indexer_score_fp8_workspace_size", "ls_indexer_score_fp8",
     "ls_prefill_select_fp8_workspace_size", "ls_prefill_select_stream_fp8", "ls_lsa_flat_workspace_size",
-    "ls_lsa_flat_select", "ls_lsa_tree_workspace_size", "ls_lsa_tree_select",
+    "ls_lsa_flat_select", "ls_lsa_tree_workspace_size", "ls_lsa_tree_select", "ls_merge_select_workspace_size",
+    "ls_merge_select",
 )
 HIST_BINS = 2048
 
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_lsa_flat_select": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
         "ls_lsa_tree_workspace_size": (SZ, [I, I, I, I, I, I]),
         "ls_lsa_tree_select": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]),
+        "ls_merge_select_workspace_size": (SZ, [I, I, I]),
+        "ls_merge_select": (I, [P, P, P, I, I, I, I, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -509,6 +512,37 @@ def ls_lsa_tree_select(q_idx, q_pos, centroids, node_centroids, bucket_off, buck
                                     node_block, fanout, beam, n_sink, top_p, budget, _ptr(keys), _ptr(n),
                                     _ptr(picked), _ptr(bm), _ptr(ws), ws.numel(), _stream(stream)))
     return (keys, n, picked, bm) if want_picked else (keys, n)
+
+
+def ls_merge_select(vals, idx, offsets, k: int = 512, ws=None, out=None, stream=None):
+    """Merge S shards' top-k lists of the same T queries into the global top-k.
+
+    vals [S,T,k_in] f32 and idx [S,T,k_in] int32 (positions local to each shard, -1 padded),
+    offsets [S] int32 (each shard's first history position) -> (idx [T,k] int32, val [T,k] f32)."""
+    _dev(vals, torch.float32, "vals", 3)
+    _dev(idx, torch.int32, "idx", 3)
+    _dev(offsets, torch.int32, "offsets", 1)
+    S, T, k_in = vals.shape
+    need = lib().ls_merge_select_workspace_size(S, T, k_in)
+    if ws is None:
+        ws = _workspace(need, vals.device)
+    if out is None:
+        out = (torch.empty((T, k), dtype=torch.int32, device=vals.device),
+               torch.empty((T, k), dtype=torch.float32, device=vals.device))
+    io, vo = out
+    _check(lib().ls_merge_select(_ptr(vals), _ptr(idx), _ptr(offsets), S, T, k_in, k, _ptr(io), _ptr(vo), _ptr(ws),
+                                 ws.numel(), _stream(stream)))
+    return io, vo
+
+
+def shard_plan(n_keys: int, n_shards: int):
+    """Contiguous shards of a history of n_keys compressed positions: [(first position, length), ...]."""
+    base, out = 0, []
+    for s in range(n_shards):
+        length = n_keys // n_shards + (1 if s < n_keys % n_shards else 0)
+        out.append((base, length))
+        base += length
+    return out
 
 
 def ls_device_status(stream=None) -> int:

@@ -21,6 +21,7 @@
 #include "score_cvt.cuh"
 #include "score_dot.cuh"
 #include "score_tree.cuh"
+#include "merge.cuh"
 #include "score_q8.cuh"
 #include "score_tc.cuh"
 #include "topk.cuh"
@@ -1241,6 +1242,35 @@ ls_status ls_lsa_tree_select(const uint16_t* q_idx, const int64_t* q_pos, const 
   LS_CUDA(launch_lsa_expand(picked, q_pos, T, top_p, bucket_off, bucket_mem, P, block_keys, n_sink, budget, keys_out,
                             n_sink + block_keys + budget, n_out, st));
   return LS_OK;
+}
+
+size_t ls_merge_select_workspace_size(int S, int T, int k_in) {
+  if (S <= 0 || T <= 0 || k_in <= 0) return 0;
+  const size_t n = static_cast<size_t>(T) * S * k_in;
+  return align_up(n * sizeof(float)) + align_up(n * sizeof(int32_t)) + align_up(static_cast<size_t>(T) * sizeof(int32_t));
+}
+
+ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* offsets, int S, int T, int k_in,
+                          int k, int32_t* idx_out, float* val_out, void* ws, size_t ws_bytes, void* stream) {
+  LS_CHECK_ARG(S >= 1 && T >= 0 && k_in >= 1, "S and k_in must be >= 1, T >= 0");
+  LS_CHECK_ARG(k >= 1 && k <= kMaxTopK, "k must be in [1, %d] (got %d)", kMaxTopK, k);
+  LS_CHECK_ARG(static_cast<int64_t>(S) * k_in <= (1LL << 30), "S * k_in too large");
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(vals && idx && offsets && idx_out, "null tensor pointer");
+  const size_t need = ls_merge_select_workspace_size(S, T, k_in);
+  if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  Carver cv(ws);
+  const size_t n = static_cast<size_t>(T) * S * k_in;
+  float* pv = cv.take<float>(n);
+  int32_t* pl = cv.take<int32_t>(n);
+  int32_t* nv = cv.take<int32_t>(T);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    ProfScope prof("merge_pack_kernel", st);
+    LS_CUDA(launch_merge_pack(vals, idx, offsets, S, T, k_in, pv, pl, nv, st));
+  }
+  return topk(pv, static_cast<int64_t>(S) * k_in, nv, pl, static_cast<int64_t>(S) * k_in, T, S * k_in, k, idx_out,
+              val_out, k, st);
 }
 
 ls_status ls_profile_begin(void) {

@@ -30,7 +30,7 @@ def test_header_declares_the_calls():
     for n in ("ls_indexer_score", "ls_topk_select", "ls_prefill_select_stream", "ls_decode_two_stage_select",
               "ls_bucket_select", "ls_decode_select", "ls_last_error", "ls_device_status", "ls_indexer_score_fp8",
               "ls_prefill_select_stream_fp8", "ls_lsa_flat_select", "ls_lsa_tree_select", "ls_indexer_score_pq",
-              "ls_decode_two_stage_pq_select"):
+              "ls_decode_two_stage_pq_select", "ls_merge_select"):
         assert n in names
 
 
@@ -60,6 +60,9 @@ def test_version_and_workspace_queries(lib):
     assert lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) >= 256 * 131072 * 4 + 256 * 1024 * 4
     # LSA tree: node scores, beam and candidates (beam * fanout + node_block per row)
     assert lib.ls_lsa_tree_workspace_size(256, 32768, 2048, 4, 4096, 1024) >= 256 * 32768 * 4 + 256 * 12288 * 8
+    # shard merge: the packed S * k_in candidates per row (values and positions) and the row counts
+    assert lib.ls_merge_select_workspace_size(4, 4096, 512) >= 4096 * 4 * 512 * 8 + 4096 * 4
+    assert lib.ls_merge_select_workspace_size(0, 4096, 512) == 0
     # the threshold form adds the samples and the candidate lists (8 * top_p per row)
     assert (lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 1)
             >= lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) + 256 * 8192 * 8)
@@ -128,6 +131,11 @@ def test_argument_checks_without_gpu(lib):
                 dummy, None, None, dummy, 16, None) == 2
     assert tree(None, None, None, None, None, None, 0, 64, 4096, 1024, 512, 64, 4096, 4, 96, 4, 64, 512, None, None,
                 None, None, None, 0, None) == 0
+    # shard merge: no shards, k above the limit, short workspace, empty batch
+    assert lib.ls_merge_select(dummy, dummy, dummy, 0, 4, 512, 512, dummy, None, dummy, 1 << 30, None) == 1
+    assert lib.ls_merge_select(dummy, dummy, dummy, 2, 4, 512, 100000, dummy, None, dummy, 1 << 30, None) == 1
+    assert lib.ls_merge_select(dummy, dummy, dummy, 2, 4, 512, 512, dummy, None, dummy, 16, None) == 2
+    assert lib.ls_merge_select(None, None, None, 2, 0, 512, 512, None, None, None, 0, None) == 0
     # bucket: budget below k
     st = lib.ls_bucket_select(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 128, 10, 80, 4, 100, 512, dummy,
                               None, None, dummy, 1 << 30, None)

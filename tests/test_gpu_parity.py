@@ -294,6 +294,35 @@ def test_prefill_chunk_full_size_sampled(L):
         check_selection(idx[t], val[t], np.arange(n), ref, wl.k, RTOL_BF16, f"prefill t={t}")
 
 
+def test_prefill_sharded_history_merge(L):
+    """A history split into S contiguous shards (one per GPU in a sharded
+    prefill): each shard's selection for the same queries, positions shifted
+    so the causal rule holds per shard, merged by ls_merge_select, equals the
+    selection over the whole history bit for bit."""
+    wl = get_workload("prefill_s")
+    d = data("prefill_s")
+    T, H, dd = d["q"].shape
+    N = d["k"].shape[0]
+    q, w, qp = dev_bf16(d["q"]), dev(d["w"]), dev(d["q_pos"])
+    _, _, _, idx0, val0 = _prefill_run(L, d, wl)
+    for S in (2, 3):
+        vals, idxs, offs = [], [], []
+        for base, length in L.shard_plan(N, S):
+            hist = torch.from_numpy(d["k"][base:base + length].view(np.int16)).view(torch.bfloat16).pin_memory()
+            buf0 = torch.empty((wl.tile_keys, 128), dtype=torch.bfloat16, device="cuda")
+            buf1 = torch.empty_like(buf0)
+            i_s, v_s = L.ls_prefill_select_stream(q, w, qp - base * wl.stride, hist, buf0, buf1, k=wl.k,
+                                                  stride=wl.stride, tile_keys=wl.tile_keys)
+            vals.append(v_s)
+            idxs.append(i_s)
+            offs.append(base)
+        mi, mv = L.ls_merge_select(torch.stack(vals), torch.stack(idxs), dev(np.asarray(offs, dtype=np.int32)),
+                                   k=wl.k)
+        torch.cuda.synchronize()
+        assert np.array_equal(mi.cpu().numpy(), idx0), S
+        assert f32_bits_equal(mv.cpu().numpy(), val0), S
+
+
 # --------------------------------------------------------------------------- #
 # fp8 indexer: fp8 queries and keys, the prefill streamed from an fp8 history
 # --------------------------------------------------------------------------- #
