@@ -22,11 +22,16 @@ Sources (page title, section):
   "What the kernels do about the top-p" (packed keys with the score above the
   inverted id).
 * Two-stage decode search: LeanSparse podcast transcript, 07:12-08:00.
+* Sparse main attention over the selected rows (absorbed MLA: the 576-element
+  latent row is the key of every head, its first 512 elements the value):
+  "03 long context", section "The Architectural Answer: Read Less of the
+  Past" (stage 2) and "Derivation 6" (576-element bf16 latent rows).
 * Bucket search: "Latent Sparse Attention", sections "How LSA finds the keys"
   and "The method, term by term" (steps 5 and 6).
 
 Modules: ``formats`` (byte formats), ``indexer`` (scores, eligibility),
-``select`` (top-k and the three search pipelines), ``brute`` (pure-Python
+``select`` (top-k and the three search pipelines), ``attention`` (sparse
+main attention and the online-softmax merge), ``brute`` (pure-Python
 loops for tiny inputs), ``sizes`` (the pages' size arithmetic).
 """
 

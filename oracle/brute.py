@@ -39,3 +39,30 @@ def topk(values, positions, k):
         pos.append(-1)
         val.append(-math.inf)
     return pos, val
+
+
+def attention(q_heads, rows, scale, d_v):
+    """Sparse attention of one query by loops: q_heads H lists of D floats,
+    rows n lists of D floats (the selected latent rows) -> (H lists of d_v
+    outputs, H log-sum-exps).  Softmax as written: exp of each scaled logit
+    over the sum of them all (no max subtraction; fine for tiny inputs)."""
+    outs, lses = [], []
+    for qh in q_heads:
+        if not rows:
+            outs.append([0.0] * d_v)
+            lses.append(-math.inf)
+            continue
+        weights = []
+        for row in rows:
+            dot = 0.0
+            for j in range(len(row)):
+                dot += qh[j] * row[j]
+            weights.append(math.exp(scale * dot))
+        total = sum(weights)
+        out = [0.0] * d_v
+        for w, row in zip(weights, rows):
+            for c in range(d_v):
+                out[c] += (w / total) * row[c]
+        outs.append(out)
+        lses.append(math.log(total))
+    return outs, lses

@@ -611,3 +611,105 @@ def test_ratio_readings():
     assert sizes.key_to_hot_buffer_ratio(524288) == pytest.approx(7.3333, abs=1e-3)
     assert sizes.key_to_hot_buffer_ratio(512000, with_scale=False) == pytest.approx(6.944, abs=1e-3)
     assert abs(sizes.key_to_hot_buffer_ratio(512000) - 7.2) <= 0.05
+
+
+# --------------------------------------------------------------------------- #
+# sparse main attention over the selected rows
+# --------------------------------------------------------------------------- #
+from oracle.attention import default_scale, merge_partials, sparse_attention  # noqa: E402
+from workloads.synth import make_attention  # noqa: E402
+
+
+def _attn_case(T=3, H=4, N=40, k=12, d=24, seed=5):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((T, H, d))
+    lat = rng.standard_normal((N, d))
+    idx = np.stack([rng.choice(N, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    return q, lat, idx
+
+
+def test_attention_brute_force_tiny():
+    q, lat, idx = _attn_case()
+    idx[1, 7:] = -1
+    idx[2, :] = -1
+    scale, d_v = 0.3, 16
+    o, lse = sparse_attention(q, lat, idx, scale, d_v)
+    for t in range(q.shape[0]):
+        rows = [list(lat[s]) for s in idx[t] if s >= 0]
+        bo, bl = brute.attention([list(x) for x in q[t]], rows, scale, d_v)
+        assert np.allclose(o[t], np.array(bo), rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse[t], np.array(bl), rtol=1e-12, atol=0) or (not rows and np.all(np.isneginf(lse[t])))
+    assert np.all(o[2] == 0.0) and np.all(np.isneginf(lse[2]))
+
+
+def test_attention_equals_dense_sdpa_when_every_row_is_selected():
+    """Selecting every row reduces to dense attention of one query over the
+    whole cache (MQA: every head attends to the same rows), computed here by
+    torch's scaled_dot_product_attention in fp64."""
+    q, lat, _ = _attn_case(T=2, H=3, N=50, d=32)
+    scale, d_v = 0.17, 20
+    idx = np.tile(np.arange(50, dtype=np.int32)[::-1], (2, 1))
+    o, lse = sparse_attention(q, lat, idx, scale, d_v)
+    qt = torch.from_numpy(q)[:, :, None, :]                                  # [T, H, 1, D]
+    kt = torch.from_numpy(lat)[None, None].expand(2, 3, 50, 32)
+    vt = torch.from_numpy(lat[:, :d_v])[None, None].expand(2, 3, 50, d_v)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)[:, :, 0].numpy()
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-13)
+    from scipy.special import logsumexp
+    assert np.allclose(lse, logsumexp(scale * np.einsum("thd,nd->thn", q, lat), axis=2), rtol=1e-13)
+
+
+def test_attention_closed_forms():
+    q, lat, idx = _attn_case(T=2, H=3, N=30, k=9, d=16)
+    scale = 0.5
+    # one selected row: the output is that row's value part, lse its logit
+    one = np.full_like(idx, -1)
+    one[:, 4] = idx[:, 0]
+    o, lse = sparse_attention(q, lat, one, scale, 10)
+    for t in range(2):
+        assert np.array_equal(o[t], np.tile(lat[idx[t, 0], :10], (3, 1)))
+        assert np.allclose(lse[t], scale * q[t] @ lat[idx[t, 0]], rtol=1e-14)
+    # a zero query: uniform weights, the mean of the selected values, lse = log n
+    o, lse = sparse_attention(np.zeros_like(q), lat, idx, scale, 10)
+    for t in range(2):
+        assert np.allclose(o[t], np.tile(lat[idx[t]][:, :10].mean(axis=0), (3, 1)), rtol=1e-13, atol=1e-15)
+        assert np.allclose(lse[t], math.log(9), rtol=1e-14)
+
+
+def test_attention_invariants():
+    """Slot order and where the unused slots sit do not matter; attention over
+    a union of disjoint selections is the online-softmax merge of the parts."""
+    q, lat, idx = _attn_case(T=3, H=4, N=60, k=20, d=24, seed=9)
+    scale = 0.4
+    o, lse = sparse_attention(q, lat, idx, scale, 16)
+    rng = np.random.default_rng(1)
+    perm = np.full((3, 27), -1, dtype=np.int32)
+    for t in range(3):
+        slots = rng.choice(27, size=20, replace=False)
+        perm[t, slots] = rng.permutation(idx[t])
+    o2, lse2 = sparse_attention(q, lat, perm, scale, 16)
+    assert np.allclose(o2, o, rtol=1e-12, atol=1e-14) and np.allclose(lse2, lse, rtol=1e-13)
+    a, b = idx.copy(), idx.copy()
+    a[:, 8:] = -1
+    b[:, :8] = -1
+    oa, la = sparse_attention(q, lat, a, scale, 16)
+    ob, lb = sparse_attention(q, lat, b, scale, 16)
+    om, lm = merge_partials(oa, la, ob, lb)
+    assert np.allclose(om, o, rtol=1e-12, atol=1e-14) and np.allclose(lm, lse, rtol=1e-13)
+    # merging with an empty part changes nothing
+    e = np.full_like(idx, -1)
+    oe, le = sparse_attention(q, lat, e, scale, 16)
+    om, lm = merge_partials(o, lse, oe, le)
+    assert np.array_equal(om, o) and np.array_equal(lm, lse)
+
+
+def test_attention_generator():
+    d = make_attention(7, 16, 3000, 300, ragged=250)
+    nv = (d["idx"] >= 0).sum(axis=1)
+    assert nv[0] == 0 and nv[1] == 1 and np.all(nv[2:] >= 50)
+    for t in range(7):   # distinct rows, a valid prefix
+        row = d["idx"][t]
+        assert np.all(row[:nv[t]] >= 0) and np.all(row[nv[t]:] == -1)
+        assert len(set(row[:nv[t]].tolist())) == nv[t]
+    lat = bf16_to_f64(d["latent"])
+    assert abs(lat.std() - 1.0) < 0.01 and abs(default_scale() - 1 / 24) < 1e-15

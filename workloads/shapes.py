@@ -43,7 +43,7 @@ from typing import Dict
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str  # "decode" | "prefill" | "two_stage" | "bucket" | "lsa"
+    kind: str  # "decode" | "prefill" | "two_stage" | "bucket" | "lsa" | "attention"
     H: int = 32
     d: int = 128
     k: int = 512
@@ -120,6 +120,12 @@ WORKLOADS: Dict[str, Workload] = {
         extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "spread": 2053, "node_block": 4096, "fanout": 4,
                "beam": 2048},
     ),
+    # sparse main attention after the decode selection: 64 decode queries of
+    # 128 heads, each over its 512 selected rows of a latent cache of
+    # 262144 rows x 576 bf16 (302 MB, larger than L2); H, d = heads, latent
+    # width ("03 long context", "The Architectural Answer: Read Less of the
+    # Past", stage 2)
+    "attn_decode": Workload("attn_decode", "attention", T=64, H=128, d=576, N=262144, k=512),
     # ---- reduced parity cases: several tiles, ragged tails ------------------
     "decode_s": Workload("decode_s", "decode", B=5, N=3000, ragged=700),
     "prefill_s": Workload(
@@ -139,6 +145,9 @@ WORKLOADS: Dict[str, Workload] = {
         "lsa_flat_s", "lsa", T=37, N=40000, top_p=64, budget=512,
         extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "edge": 1, "node_block": 4096, "fanout": 4, "beam": 96},
     ),
+    # 7 queries, 2 head groups, 300 slots (5 chunks, the last ragged); rows 0
+    # and 1 select nothing and one row, the others a ragged prefix
+    "attn_s": Workload("attn_s", "attention", T=7, H=16, d=576, N=3000, k=300, ragged=250),
     "bucket_s": Workload(
         "bucket_s", "bucket", T=19, clusters=1500, cluster_size=8, noise_rel=0.3, top_p=64, budget=512,
         extra={"min_size": 4, "max_size": 16},

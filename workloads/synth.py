@@ -359,6 +359,35 @@ def make_lsa(
             "node_centroids": to_bf16_bits(nc) if P1 else np.zeros((0, dim), dtype=np.uint16)}
 
 
+# --------------------------------------------------------------------------- #
+# sparse main attention: a latent cache of N rows x d bf16 (d = 576: 512
+# latent + 64 rotary elements), T queries of H heads, and per query k slots of
+# selected rows (distinct, -1 after the valid prefix)
+# --------------------------------------------------------------------------- #
+def make_attention(T: int, H: int, N: int, k: int, d: int = 576, seed: int = 0,
+                   ragged: int = 0, q_std: float = 2.0 / 24.0) -> Dict[str, np.ndarray]:
+    """q ~ N(0, q_std^2) and latent ~ N(0, 1) per element (logits of standard
+    deviation about q_std * sqrt(d) before the 1/sqrt(d) scale: 2 by default).
+    With ``ragged``, row 0 selects nothing, row 1 one row, the others a valid
+    prefix of length in [k - ragged, k]."""
+    rng = np.random.default_rng(seed)
+    q = to_bf16_bits(_normal(rng, (T, H, d), q_std))
+    latent = np.empty((N, d), dtype=np.uint16)
+    step = 1 << 16
+    for r0 in range(0, N, step):          # in chunks, to bound the fp64 working set
+        n = min(step, N - r0)
+        latent[r0:r0 + n] = to_bf16_bits(rng.standard_normal((n, d)))
+    idx = np.full((T, k), -1, dtype=np.int32)
+    for t in range(T):
+        if ragged:
+            nv = 0 if t == 0 else 1 if t == 1 else int(rng.integers(max(k - ragged, 0), k + 1))
+        else:
+            nv = k
+        nv = min(nv, N)
+        idx[t, :nv] = rng.choice(N, size=nv, replace=False)
+    return {"q": q, "latent": latent, "idx": idx}
+
+
 def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
     """Inputs for a named workload (or a ``Workload``)."""
     if isinstance(wl, str):
@@ -380,4 +409,6 @@ def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
     if wl.kind == "lsa":
         return make_lsa(wl.T, wl.N, wl.extra.get("block_keys", 512), wl.extra.get("bpb", 64), s,
                         wl.extra.get("spread", 2053), bool(wl.extra.get("edge", 0)))
+    if wl.kind == "attention":
+        return make_attention(wl.T, wl.H, wl.N, wl.k, wl.d, s, ragged=wl.ragged)
     raise ValueError(wl.kind)
