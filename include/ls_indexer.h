@@ -351,6 +351,35 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
                           int k, int32_t* idx_out, float* val_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ls_sparse_attention -- sparse main attention over the selected rows, stage
+ * 2 of DSA ("03 long context", section "The Architectural Answer: Read Less
+ * of the Past"): exact attention of every query head over only the k rows the
+ * indexer selected, in the absorbed MLA form where one cached latent row of
+ * d = 576 bf16 elements (512 latent + 64 rotary; "Derivation 6" of the same
+ * lecture) is the key of every head and its first d_v = 512 elements the
+ * value.  For query t, head h and the selected rows S_t:
+ *   logit(s) = scale * q[t,h,:] . latent[s,:]
+ *   lse[t,h] = log sum_{s in S_t} exp(logit(s))
+ *   out[t,h,:] = sum_{s in S_t} exp(logit(s) - lse[t,h]) * latent[s,:512]
+ *
+ *   q [T][H][576] bf16, latent [n_rows][576] bf16 (16-byte aligned)
+ *   idx [T][k] int32: selected positions, -1 = unused slot (anywhere in the row)
+ *   row_off [T] int64 or NULL: row of latent = idx + row_off[t] (one buffer
+ *        holding several sequences' caches); a row outside [0, n_rows) is
+ *        skipped and sets LS_FAULT_BAD_INDEX (see ls_device_status)
+ *   H a multiple of 8, k <= 2048; scale is the softmax scale (1/sqrt(576) is
+ *        the plain choice; the pages do not fix it)
+ *   out [T][H][512] fp32; lse [T][H] fp32 natural-log sum or NULL.  An empty
+ *        selection gives out = 0 and lse = -inf; partial results over
+ *        disjoint selections combine exactly by their lse (online softmax).
+ * Errors: LS_ERR_UNSUPPORTED for d != 576 or d_v != 512, LS_ERR_INVALID_ARG
+ * for the other limits.  No workspace; asynchronous on `stream`.
+ */
+ls_status ls_sparse_attention(const uint16_t* q, const uint16_t* latent, const int32_t* idx, const int64_t* row_off,
+                              int T, int H, int d, int d_v, int64_t n_rows, int k, float scale, float* out, float* lse,
+                              void* stream);
+
+/*
  * ls_decode_two_stage_select -- LeanSparse two-stage decode search
  * (podcast transcript, 07:12-08:00): scan compact keys, keep a shortlist,
  * fetch the shortlist's original keys and re-rank exactly, keep the top k.

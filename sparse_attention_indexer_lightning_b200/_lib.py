@@ -10,6 +10,7 @@ shared library and raises ImportError when it is missing or stale.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional
 
@@ -39,7 +40,7 @@ EXPORTED = (
     "ls_indexer_score_pq", "ls_indexer_score_fp8_workspace_size", "ls_indexer_score_fp8",
     "ls_prefill_select_fp8_workspace_size", "ls_prefill_select_stream_fp8", "ls_lsa_flat_workspace_size",
     "ls_lsa_flat_select", "ls_lsa_tree_workspace_size", "ls_lsa_tree_select", "ls_merge_select_workspace_size",
-    "ls_merge_select",
+    "ls_merge_select", "ls_sparse_attention",
 )
 HIST_BINS = 2048
 
@@ -88,6 +89,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_lsa_tree_select": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]),
         "ls_merge_select_workspace_size": (SZ, [I, I, I]),
         "ls_merge_select": (I, [P, P, P, I, I, I, I, P, P, P, SZ, P]),
+        "ls_sparse_attention": (I, [P, P, P, P, I, I, I, I, I64, I, ctypes.c_float, P, P, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -533,6 +535,34 @@ def ls_merge_select(vals, idx, offsets, k: int = 512, ws=None, out=None, stream=
     _check(lib().ls_merge_select(_ptr(vals), _ptr(idx), _ptr(offsets), S, T, k_in, k, _ptr(io), _ptr(vo), _ptr(ws),
                                  ws.numel(), _stream(stream)))
     return io, vo
+
+
+def ls_sparse_attention(q, latent, idx, scale: Optional[float] = None, row_off=None, want_lse: bool = True,
+                        out=None, stream=None):
+    """Sparse main attention over the selected latent rows.
+
+    q [T,H,576] bf16, latent [R,576] bf16, idx [T,k] int32 (-1 = unused slot),
+    row_off [T] int64 or None (row = idx + row_off[t]); scale defaults to
+    1/sqrt(576) -> (out [T,H,512] f32, lse [T,H] f32 or None)."""
+    _dev(q, torch.bfloat16, "q", 3)
+    _dev(latent, torch.bfloat16, "latent", 2)
+    _dev(idx, torch.int32, "idx", 2)
+    _opt(row_off, torch.int64, "row_off")
+    T, H, d = q.shape
+    R, d_lat = latent.shape
+    if d_lat != d:
+        raise ValueError(f"q has {d} elements per head, latent rows {d_lat}")
+    if idx.shape[0] != T:
+        raise ValueError(f"idx has {idx.shape[0]} rows for {T} queries")
+    k = idx.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, H, 512), dtype=torch.float32, device=q.device)
+    lse = torch.empty((T, H), dtype=torch.float32, device=q.device) if want_lse else None
+    _check(lib().ls_sparse_attention(_ptr(q), _ptr(latent), _ptr(idx), _ptr(row_off), T, H, d, 512, R, k, float(scale),
+                                     _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def shard_plan(n_keys: int, n_shards: int):

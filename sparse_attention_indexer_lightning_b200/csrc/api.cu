@@ -22,6 +22,7 @@
 #include "score_dot.cuh"
 #include "score_tree.cuh"
 #include "merge.cuh"
+#include "sparse_attn.cuh"
 #include "score_q8.cuh"
 #include "score_tc.cuh"
 #include "topk.cuh"
@@ -1271,6 +1272,30 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
   }
   return topk(pv, static_cast<int64_t>(S) * k_in, nv, pl, static_cast<int64_t>(S) * k_in, T, S * k_in, k, idx_out,
               val_out, k, st);
+}
+
+ls_status ls_sparse_attention(const uint16_t* q, const uint16_t* latent, const int32_t* idx, const int64_t* row_off,
+                              int T, int H, int d, int d_v, int64_t n_rows, int k, float scale, float* out, float* lse,
+                              void* stream) {
+  LS_CHECK_ARG(T >= 0 && H >= 0 && k >= 0 && n_rows >= 0, "negative size (T=%d H=%d k=%d)", T, H, k);
+  if (d != kAttnLatent || d_v != kAttnValue)
+    return fail(LS_ERR_UNSUPPORTED, "latent rows of %d elements with %d value elements are built (got d=%d d_v=%d)",
+                kAttnLatent, kAttnValue, d, d_v);
+  LS_CHECK_ARG(H >= kAttnHeads && H % kAttnHeads == 0 && H <= 1024, "H must be a multiple of %d in [%d, 1024] (got %d)",
+               kAttnHeads, kAttnHeads, H);
+  LS_CHECK_ARG(k >= 1 && k <= kAttnMaxK, "k must be in [1, %d] (got %d)", kAttnMaxK, k);
+  LS_CHECK_ARG(n_rows <= 0x7fffffffLL, "at most 2^31 - 1 latent rows");
+  LS_CHECK_ARG(static_cast<int64_t>(T) * (H / kAttnHeads) <= 0x7fffffffLL, "T * H / 8 too large");
+  LS_CHECK_ARG(scale == scale && scale > -3.4e38f && scale < 3.4e38f, "scale must be finite");
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(q && idx && out, "null tensor pointer");
+  LS_CHECK_ARG(latent || n_rows == 0, "null latent with n_rows > 0");
+  LS_CHECK_ARG(aligned16(q) && aligned16(out) && (!latent || aligned16(latent)),
+               "q, latent and out must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope prof("sparse_attn_kernel", st);
+  LS_CUDA(launch_sparse_attn(q, latent, idx, row_off, T, H, k, n_rows, scale, out, lse, st));
+  return LS_OK;
 }
 
 ls_status ls_profile_begin(void) {

@@ -1,0 +1,231 @@
+// Sparse main attention over the selected latent rows: stage 2 of DSA ("03
+// long context", section "The Architectural Answer: Read Less of the Past"),
+// in the absorbed MLA form where one cached latent row of 576 bf16 elements
+// (512 latent + 64 rotary; "Derivation 6" of the same lecture) is the key of
+// every query head and its first 512 elements are the value.  For query t and
+// head h over the selected rows S_t:
+//
+//   logit(s) = scale * q[t,h,:] . c[s,:],   lse = log sum_s exp(logit(s)),
+//   o[t,h,:] = sum_s exp(logit(s) - lse) * c[s,:512]
+//
+// One CTA per (query, group of 8 heads), 256 threads, on the CUDA cores:
+//
+//  1. the CTA's row ids (slot -> idx + row offset; -1 or out of range -> none)
+//     and its 8 query heads (fp32, [dimension][head]) go to shared memory;
+//  2. logits: the selected rows are staged 64 at a time (a row per 289-word
+//     stride, so 32 consecutive rows start on 32 different banks); thread
+//     (row j, quarter p) takes dimensions 144p .. 144p + 143 for all 8 heads,
+//     and the four quarters are added in a fixed order;
+//  3. softmax: warp h takes head h: max, exp(logit - max), sum, 1 / sum, lse;
+//  4. values: the value parts are staged again, 64 rows at a time; thread i
+//     owns output columns 2i and 2i + 1 of all 8 heads.
+//
+// The selection sits in shared memory in full (k <= 2048 slots), so the
+// softmax is exact in two passes, with no running rescale.  Unused slots
+// stage zeros and weigh 0.
+
+#pragma once
+
+#include "common.cuh"
+
+namespace lsi {
+
+constexpr int kAttnLatent = 576;                    // elements of a latent row (the key)
+constexpr int kAttnValue = 512;                     // leading elements that are the value
+constexpr int kAttnHeads = 8;                       // heads per CTA
+constexpr int kAttnChunk = 64;                      // selected rows staged per pass
+constexpr int kAttnThreads = 256;
+constexpr int kAttnMaxK = 2048;
+constexpr int kAttnRowWords = kAttnLatent / 2 + 1;  // 289 words: row r starts on bank r mod 32
+constexpr int kAttnQuarter = kAttnLatent / 4;       // 144 dimensions per partial dot product
+static_assert(kAttnValue / 2 == kAttnThreads, "one value column pair per thread");
+static_assert(kAttnThreads == 4 * kAttnChunk, "four dimension quarters per staged row");
+static_assert(kAttnThreads / 32 == kAttnHeads, "one warp per head in the softmax");
+
+__host__ __device__ constexpr int attn_kpad(int k) { return (k + kAttnChunk - 1) / kAttnChunk * kAttnChunk; }
+
+// Dynamic shared memory of one CTA for k slots (4-byte words throughout).
+__host__ __device__ constexpr size_t attn_smem_bytes(int k) {
+  return 4 * (static_cast<size_t>(kAttnLatent) * kAttnHeads      // query heads [d][h]
+              + static_cast<size_t>(kAttnChunk) * kAttnRowWords  // staged rows
+              + 4 * kAttnHeads * kAttnChunk                       // partial dot products [quarter][h][row]
+              + static_cast<size_t>(kAttnHeads) * attn_kpad(k)    // logits, then weights [h][slot]
+              + attn_kpad(k)                                      // row ids [slot]
+              + kAttnHeads);                                      // 1 / sum of weights [h]
+}
+
+__device__ __forceinline__ float attn_bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float attn_bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float attn_warp_max(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float attn_warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Stage the first `words` 32-bit words (bf16 pairs) of the rows in slots
+// c0 .. c0 + 63; an unused slot stages zeros.
+__device__ __forceinline__ void attn_stage(uint32_t* rows, const int32_t* ids, int c0,
+                                           const uint16_t* __restrict__ latent, int words) {
+  const int vecs = words / 4;                       // 16-byte loads per row
+  for (int i = threadIdx.x; i < kAttnChunk * vecs; i += kAttnThreads) {
+    const int r = i / vecs;
+    const int v = i - r * vecs;
+    const int32_t id = ids[c0 + r];
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (id >= 0) x = __ldg(reinterpret_cast<const uint4*>(latent + static_cast<int64_t>(id) * kAttnLatent) + v);
+    uint32_t* dst = rows + r * kAttnRowWords + 4 * v;
+    dst[0] = x.x;
+    dst[1] = x.y;
+    dst[2] = x.z;
+    dst[3] = x.w;
+  }
+}
+
+// grid: T * (H / 8) CTAs, CTA b = (query b / (H / 8), head group b % (H / 8)).
+__global__ void __launch_bounds__(kAttnThreads)
+    sparse_attn_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ latent,
+                       const int32_t* __restrict__ idx, const int64_t* __restrict__ row_off, int H, int k,
+                       int64_t n_rows, float scale, float* __restrict__ out, float* __restrict__ lse) {
+  extern __shared__ __align__(16) unsigned char attn_smem[];
+  const int kp = attn_kpad(k);
+  float* qs = reinterpret_cast<float*>(attn_smem);
+  uint32_t* rows = reinterpret_cast<uint32_t*>(qs + kAttnLatent * kAttnHeads);
+  float* part = reinterpret_cast<float*>(rows + kAttnChunk * kAttnRowWords);
+  float* sc = part + 4 * kAttnHeads * kAttnChunk;
+  int32_t* ids = reinterpret_cast<int32_t*>(sc + kAttnHeads * kp);
+  float* inv_l = reinterpret_cast<float*>(ids + kp);
+
+  const int tid = threadIdx.x;
+  const int groups = H / kAttnHeads;
+  const int t = blockIdx.x / groups;
+  const int h0 = (blockIdx.x - t * groups) * kAttnHeads;
+  const int64_t off = row_off ? row_off[t] : 0;
+
+  // 1. row ids and query heads
+  for (int i = tid; i < kp; i += kAttnThreads) {
+    int32_t id = -1;
+    if (i < k) {
+      const int32_t s = idx[static_cast<int64_t>(t) * k + i];
+      if (s >= 0) {
+        const int64_t r = off + s;
+        if (r >= 0 && r < n_rows)
+          id = static_cast<int32_t>(r);
+        else
+          atomicOr(&g_fault, FAULT_BAD_INDEX);      // never read: the slot stays unused
+      }
+    }
+    ids[i] = id;
+  }
+  const uint16_t* qt = q + (static_cast<int64_t>(t) * H + h0) * kAttnLatent;
+  for (int i = tid; i < kAttnHeads * kAttnLatent; i += kAttnThreads) {
+    const int hh = i / kAttnLatent;
+    const int d = i - hh * kAttnLatent;
+    qs[d * kAttnHeads + hh] = __uint_as_float(static_cast<uint32_t>(qt[i]) << 16);
+  }
+  __syncthreads();
+
+  // 2. logits
+  const int jj = tid & (kAttnChunk - 1);
+  const int qd = tid / kAttnChunk;
+  for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
+    attn_stage(rows, ids, c0, latent, kAttnLatent / 2);
+    __syncthreads();
+    float acc[kAttnHeads];
+#pragma unroll
+    for (int hh = 0; hh < kAttnHeads; ++hh) acc[hh] = 0.f;
+    const uint32_t* rw = rows + jj * kAttnRowWords + qd * (kAttnQuarter / 2);
+    const float* qq = qs + qd * kAttnQuarter * kAttnHeads;
+#pragma unroll 4
+    for (int w = 0; w < kAttnQuarter / 2; ++w) {
+      const uint32_t x = rw[w];
+      const float x0 = attn_bf16_lo(x);
+      const float x1 = attn_bf16_hi(x);
+      const float* q0 = qq + 2 * w * kAttnHeads;
+#pragma unroll
+      for (int hh = 0; hh < kAttnHeads; ++hh) acc[hh] = fmaf(x1, q0[kAttnHeads + hh], fmaf(x0, q0[hh], acc[hh]));
+    }
+#pragma unroll
+    for (int hh = 0; hh < kAttnHeads; ++hh) part[(qd * kAttnHeads + hh) * kAttnChunk + jj] = acc[hh];
+    __syncthreads();
+    for (int i = tid; i < kAttnHeads * kAttnChunk; i += kAttnThreads) {
+      const int hh = i / kAttnChunk;
+      const int j = i - hh * kAttnChunk;
+      const float s = ((part[(0 * kAttnHeads + hh) * kAttnChunk + j] + part[(1 * kAttnHeads + hh) * kAttnChunk + j]) +
+                       part[(2 * kAttnHeads + hh) * kAttnChunk + j]) +
+                      part[(3 * kAttnHeads + hh) * kAttnChunk + j];
+      sc[hh * kp + c0 + j] = ids[c0 + j] >= 0 ? s * scale : -INFINITY;
+    }
+    __syncthreads();
+  }
+
+  // 3. softmax, one warp per head (kp is a multiple of 32: every lane loops alike)
+  {
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    float* sh = sc + warp * kp;
+    float m = -INFINITY;
+    for (int j = lane; j < kp; j += 32) m = fmaxf(m, sh[j]);
+    m = attn_warp_max(m);
+    float l = 0.f;
+    for (int j = lane; j < kp; j += 32) {
+      const float x = sh[j];
+      const float e = (x == -INFINITY) ? 0.f : expf(x - m);
+      sh[j] = e;
+      l += e;
+    }
+    l = attn_warp_sum(l);
+    if (lane == 0) {
+      inv_l[warp] = l > 0.f ? 1.f / l : 0.f;
+      if (lse) lse[static_cast<int64_t>(t) * H + h0 + warp] = l > 0.f ? m + logf(l) : -INFINITY;
+    }
+  }
+  __syncthreads();
+
+  // 4. values
+  float o[kAttnHeads][2];
+#pragma unroll
+  for (int hh = 0; hh < kAttnHeads; ++hh) o[hh][0] = o[hh][1] = 0.f;
+  for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
+    attn_stage(rows, ids, c0, latent, kAttnValue / 2);
+    __syncthreads();
+    for (int j = 0; j < kAttnChunk; ++j) {
+      const uint32_t x = rows[j * kAttnRowWords + tid];
+      const float v0 = attn_bf16_lo(x);
+      const float v1 = attn_bf16_hi(x);
+#pragma unroll
+      for (int hh = 0; hh < kAttnHeads; ++hh) {
+        const float p = sc[hh * kp + c0 + j];
+        o[hh][0] = fmaf(p, v0, o[hh][0]);
+        o[hh][1] = fmaf(p, v1, o[hh][1]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int hh = 0; hh < kAttnHeads; ++hh) {
+    float* dst = out + (static_cast<int64_t>(t) * H + h0 + hh) * kAttnValue + 2 * tid;
+    const float il = inv_l[hh];
+    *reinterpret_cast<float2*>(dst) = make_float2(o[hh][0] * il, o[hh][1] * il);
+  }
+}
+
+cudaError_t launch_sparse_attn(const uint16_t* q, const uint16_t* latent, const int32_t* idx, const int64_t* row_off,
+                               int T, int H, int k, int64_t n_rows, float scale, float* out, float* lse,
+                               cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const size_t smem = attn_smem_bytes(k);
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = static_cast<int64_t>(T) * (H / kAttnHeads);
+  sparse_attn_kernel<<<static_cast<unsigned>(blocks), kAttnThreads, smem, st>>>(q, latent, idx, row_off, H, k, n_rows,
+                                                                                  scale, out, lse);
+  return cudaGetLastError();
+}
+
+}  // namespace lsi

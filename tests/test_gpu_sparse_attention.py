@@ -1,0 +1,156 @@
+"""Parity of the sparse main attention (CUDA, through the C ABI) with the fp64 oracle.
+
+Tolerance, from the arithmetic: each logit is an fp32 sum of 576 exact
+products of bf16 values (relative error a few 1e-7 of the sum of magnitudes),
+the weights come from fp32 exp and one division (a few ulp), and each output
+is an fp32 weighted sum of at most 2048 bf16 values.  Every error term is
+below 1e-5 of the largest value magnitude among the selected rows for these
+inputs (logits of standard deviation about 2), so the bound checked is
+|o - o_ref| <= 1e-4 * max |value| of the query's selected rows and
+|lse - lse_ref| <= 1e-4 * (1 + |lse_ref|).  A missed or doubled row moves an
+output by about its weight (>= 1e-3 here), a wrong scale or value slice far
+more.
+"""
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.attention import default_scale, merge_partials, sparse_attention
+from oracle.formats import bf16_to_f64
+from parity_util import dev, dev_bf16
+from workloads import get_workload, make_workload
+from workloads.synth import make_attention, make_decode
+
+pytestmark = pytest.mark.gpu
+
+ATTN_TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_indexer_lightning_b200 import build as b
+    b.build()
+    import sparse_attention_indexer_lightning_b200 as lib
+    return lib
+
+
+@functools.lru_cache(maxsize=None)
+def data(name):
+    return make_workload(name)
+
+
+def _check(out, lse, q_bits, lat_bits, gidx, scale, rows=None, what=""):
+    """Compare queries `rows` (all by default) of the GPU result with the oracle;
+    gidx holds latent row ids (-1 = unused)."""
+    rows = range(q_bits.shape[0]) if rows is None else rows
+    rows = list(rows)
+    ro, rl = sparse_attention(bf16_to_f64(q_bits[rows]), bf16_to_f64(lat_bits), gidx[rows], scale)
+    for i, t in enumerate(rows):
+        sel = gidx[t][gidx[t] >= 0]
+        if sel.size == 0:
+            assert np.all(out[t] == 0.0), f"{what} t={t}: empty selection must give zeros"
+            assert np.all(np.isneginf(lse[t])), f"{what} t={t}: empty selection must give lse = -inf"
+            continue
+        vmax = np.abs(bf16_to_f64(lat_bits[sel, :512])).max()
+        err = np.abs(out[t] - ro[i]).max()
+        assert err <= ATTN_TOL * vmax, f"{what} t={t}: output error {err:.3e} > {ATTN_TOL * vmax:.3e}"
+        lerr = np.abs(lse[t] - rl[i])
+        assert np.all(lerr <= ATTN_TOL * (1 + np.abs(rl[i]))), f"{what} t={t}: lse error {lerr.max():.3e}"
+
+
+def _run(L, d, scale=None, idx=None, row_off=None):
+    idx = d["idx"] if idx is None else idx
+    out, lse = L.ls_sparse_attention(dev_bf16(d["q"]), dev_bf16(d["latent"]), dev(idx.astype(np.int32)),
+                                     scale=scale, row_off=None if row_off is None else dev(row_off))
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+def test_sparse_attention_small(L):
+    """7 queries x 16 heads over 300 slots (5 chunks, the last ragged): empty,
+    one-row and ragged selections; the unused slots at the tail, then scattered."""
+    d = data("attn_s")
+    out, lse = _run(L, d)
+    _check(out, lse, d["q"], d["latent"], d["idx"], default_scale(), what="attn_s")
+    rng = np.random.default_rng(3)
+    idx = np.stack([rng.permutation(r) for r in d["idx"]])
+    out2, lse2 = _run(L, d, idx=idx)
+    _check(out2, lse2, d["q"], d["latent"], idx, default_scale(), what="scattered")
+
+
+def test_sparse_attention_shapes(L):
+    """k = 1, k = 1000 with a larger scale, the largest k (2048), many heads."""
+    for T, H, N, k, scale in ((3, 8, 100, 1, 0.5), (2, 8, 5000, 1000, 0.2), (2, 8, 5000, 2048, None),
+                              (2, 128, 5000, 512, None), (1, 24, 700, 130, 0.05)):
+        d = make_attention(T, H, N, k, seed=T * 1000 + k)
+        out, lse = _run(L, d, scale=scale)
+        _check(out, lse, d["q"], d["latent"], d["idx"], default_scale() if scale is None else scale,
+               what=f"T={T} H={H} k={k}")
+
+
+def test_sparse_attention_row_offsets_and_bad_rows(L):
+    """row = idx + row_off[t]; rows outside the cache are skipped and flagged."""
+    d = data("attn_s")
+    N = d["latent"].shape[0]
+    idx = np.where(d["idx"] >= 0, d["idx"] % 1000, -1).astype(np.int32)
+    off = np.array([0, 10, 2000, 1500, 0, 2999, 5], dtype=np.int64)
+    L.ls_device_status()
+    out, lse = _run(L, d, scale=0.07, idx=idx, row_off=off)
+    flags = L.ls_device_status()
+    g = np.where(idx >= 0, idx + off[:, None], -1)
+    bad = (idx >= 0) & (g >= N)
+    assert bad.any()
+    assert flags & 2        # LS_FAULT_BAD_INDEX
+    g = np.where(bad, -1, g)
+    _check(out, lse, d["q"], d["latent"], g, 0.07, what="row_off")
+
+
+def test_sparse_attention_lse_merges_disjoint_parts(L):
+    """Attention over the first and the last slots separately, merged by their
+    lse (online softmax), equals attention over all of them."""
+    d = make_attention(4, 16, 4000, 512, seed=11)
+    out, lse = _run(L, d)
+    a = d["idx"].copy()
+    a[:, 200:] = -1
+    b = d["idx"].copy()
+    b[:, :200] = -1
+    oa, la = _run(L, d, idx=a)
+    ob, lb = _run(L, d, idx=b)
+    om, lm = merge_partials(oa.astype(np.float64), la.astype(np.float64), ob.astype(np.float64),
+                            lb.astype(np.float64))
+    vmax = np.abs(bf16_to_f64(d["latent"][:, :512])).max()
+    assert np.abs(om - out).max() <= ATTN_TOL * vmax
+    assert np.all(np.abs(lm - lse) <= ATTN_TOL * (1 + np.abs(lse)))
+
+
+def test_sparse_attention_after_decode_selection(L):
+    """The decode indexer's top-512 of each sequence, fed as is to the sparse
+    attention over a cache holding every sequence's latent rows (row_off =
+    b * N): the two stages chained as DSA runs them."""
+    wl = get_workload("decode_s")
+    dd = make_decode(wl.B, wl.N, seed=wl.seed, ragged=wl.ragged)
+    idx, _ = L.ls_decode_select(dev_bf16(dd["q"]), dev(dd["w"]), dev_bf16(dd["k"]), k=wl.k,
+                                n_valid=dev(dd["n_valid"]))
+    att = make_attention(wl.B, 128, wl.B * wl.N, 1, seed=21)
+    off = (np.arange(wl.B, dtype=np.int64) * wl.N)
+    out, lse = L.ls_sparse_attention(dev_bf16(att["q"]), dev_bf16(att["latent"]), idx, row_off=dev(off))
+    torch.cuda.synchronize()
+    sel = idx.cpu().numpy()
+    assert np.all((sel >= 0).sum(axis=1) == np.minimum(dd["n_valid"], wl.k))
+    g = np.where(sel >= 0, sel + off[:, None], -1)
+    _check(out.cpu().numpy(), lse.cpu().numpy(), att["q"], att["latent"], g, default_scale(), what="chained")
+
+
+@pytest.mark.slow
+def test_sparse_attention_full_size_sampled(L):
+    """64 decode queries x 128 heads, 512 rows each of a 262144-row cache
+    (302 MB): every output finite, sampled queries against the oracle."""
+    d = data("attn_decode")
+    out, lse = _run(L, d)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    _check(out, lse, d["q"], d["latent"], d["idx"], default_scale(), rows=[0, 17, 40, 63], what="attn_decode")
