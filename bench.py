@@ -355,8 +355,15 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
                      ("bucket", bench_bucket), ("lsa_flat", bench_lsa),
                      ("lsa_flat_threshold", lambda *a: bench_lsa(*a, threshold=True)), ("lsa_tree", bench_lsa_tree),
                      ("two_stage", bench_two_stage),
-                     ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True))):
+                     ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True)),
+                     ("attn_decode", bench_attention)):
         if only in (None, name):
+            if name == "attn_decode" and only is None:
+                try:                       # the newest path: an error here must not lose the lines above
+                    res[name] = fn(L, args, peaks, peak_kind)
+                except Exception as e:     # noqa: BLE001
+                    res[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+                continue
             res[name] = fn(L, args, peaks, peak_kind)
     return res
 
@@ -599,6 +606,50 @@ def bench_lsa_tree(L, args, peaks, peak_kind):
     return res
 
 
+# fp32 FMA issue rate of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz (clocks.max.sm)
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bench_attention(L, args, peaks, peak_kind):
+    """Sparse main attention after the decode selection: 64 queries x 128
+    heads, each over its 512 selected rows of a 262144 x 576 bf16 latent cache
+    (302 MB).  Four selections are cycled so that consecutive steps gather
+    different rows (4 x 37.7 MB, more than L2)."""
+    import torch
+    from workloads import get_workload, make_workload
+    st = torch.cuda.current_stream()
+    steps = max(3, args.steps)
+    warm = max(3, args.warmup)
+    wl = get_workload("attn_decode")
+    d = make_workload(wl)
+    T, H, D = d["q"].shape
+    R = d["latent"].shape[0]
+    rng = np.random.default_rng(wl.seed + 1)
+    sets = [to_dev(d["idx"])] + [to_dev(np.stack([rng.choice(R, size=wl.k, replace=False) for _ in range(T)])
+                                        .astype(np.int32)) for _ in range(3)]
+    q, lat = to_dev_bf16(d["q"]), to_dev_bf16(d["latent"])
+    out = torch.empty((T, H, 512), dtype=torch.float32, device="cuda")
+
+    def run(i, timed):
+        L.ls_sparse_attention(q, lat, sets[i % len(sets)], out=out)
+        return None
+
+    ms, kern = _profiled_loop(L, run, steps, warm, st)
+    kms = kern["sparse_attn_kernel"]["ms_per_step"]
+    flops = T * H * wl.k * (D + 512) * 2
+    gathered = T * wl.k * D * 2
+    peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    res = {"ms_per_step": ms, "positions_per_s": T * wl.k / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
+           "kernels": kern,
+           "roofline": roofline("alu", flops / (kms * 1e-3) / 1e12, round(ALU_FP32_TFLOPS, 1), "TFLOP/s",
+                                peak_kind="derived: fp32 FMA issue rate at clocks.max.sm"),
+           "gather_hbm_frac": round(gathered / (kms * 1e-3) / 1e9 / peak_b, 4),
+           "note": "positions = selected rows attended per step; flops = T x H x k x (576 + 512) x 2 "
+                   "(logits and values); CUDA-core kernel"}
+    del sets, q, lat, out
+    return res
+
+
 def bench_two_stage(L, args, peaks, peak_kind, pq=False):
     """Two-stage decode search: compact scan (int8 + scale, or 32-byte PQ codes), shortlist, exact re-rank."""
     import torch
@@ -724,7 +775,7 @@ def main(argv=None):
     ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "prefill_chunk_fp8",
                                                      "prefill_chunk_fp8_running", "bucket", "lsa_flat",
                                                      "lsa_flat_threshold", "lsa_tree", "two_stage",
-                                                     "two_stage_pq"],
+                                                     "two_stage_pq", "attn_decode"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
