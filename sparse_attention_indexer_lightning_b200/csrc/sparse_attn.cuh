@@ -15,10 +15,12 @@
 //  2. logits: the selected rows are staged 64 at a time (a row per 289-word
 //     stride, so 32 consecutive rows start on 32 different banks); thread
 //     (row j, quarter p) takes dimensions 144p .. 144p + 143 for all 8 heads,
-//     and the four quarters are added in a fixed order;
+//     and the four quarters are added in a fixed order; logits are kept
+//     slot-major ([slot][head]);
 //  3. softmax: warp h takes head h: max, exp(logit - max), sum, 1 / sum, lse;
 //  4. values: the value parts are staged again, 64 rows at a time; thread i
-//     owns output columns 2i and 2i + 1 of all 8 heads.
+//     owns output columns 2i and 2i + 1 of all 8 heads and reads a row's 8
+//     weights as two 16-byte broadcasts.
 //
 // The selection sits in shared memory in full (k <= 2048 slots), so the
 // softmax is exact in two passes, with no running rescale.  Unused slots
@@ -41,6 +43,8 @@ constexpr int kAttnQuarter = kAttnLatent / 4;       // 144 dimensions per partia
 static_assert(kAttnValue / 2 == kAttnThreads, "one value column pair per thread");
 static_assert(kAttnThreads == 4 * kAttnChunk, "four dimension quarters per staged row");
 static_assert(kAttnThreads / 32 == kAttnHeads, "one warp per head in the softmax");
+static_assert((kAttnLatent * kAttnHeads + kAttnChunk * kAttnRowWords + 4 * kAttnHeads * kAttnChunk) % 4 == 0,
+              "the weights start on a 16-byte boundary (float4 reads)");
 
 __host__ __device__ constexpr int attn_kpad(int k) { return (k + kAttnChunk - 1) / kAttnChunk * kAttnChunk; }
 
@@ -48,8 +52,8 @@ __host__ __device__ constexpr int attn_kpad(int k) { return (k + kAttnChunk - 1)
 __host__ __device__ constexpr size_t attn_smem_bytes(int k) {
   return 4 * (static_cast<size_t>(kAttnLatent) * kAttnHeads      // query heads [d][h]
               + static_cast<size_t>(kAttnChunk) * kAttnRowWords  // staged rows
-              + 4 * kAttnHeads * kAttnChunk                       // partial dot products [quarter][h][row]
-              + static_cast<size_t>(kAttnHeads) * attn_kpad(k)    // logits, then weights [h][slot]
+              + 4 * kAttnHeads * kAttnChunk                       // partial dot products [quarter][row][h]
+              + static_cast<size_t>(kAttnHeads) * attn_kpad(k)    // logits, then weights [slot][h]
               + attn_kpad(k)                                      // row ids [slot]
               + kAttnHeads);                                      // 1 / sum of weights [h]
 }
@@ -149,16 +153,17 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
       for (int hh = 0; hh < kAttnHeads; ++hh) acc[hh] = fmaf(x1, q0[kAttnHeads + hh], fmaf(x0, q0[hh], acc[hh]));
     }
+    float* pp = part + (qd * kAttnChunk + jj) * kAttnHeads;
 #pragma unroll
-    for (int hh = 0; hh < kAttnHeads; ++hh) part[(qd * kAttnHeads + hh) * kAttnChunk + jj] = acc[hh];
+    for (int hh = 0; hh < kAttnHeads; ++hh) pp[hh] = acc[hh];
     __syncthreads();
     for (int i = tid; i < kAttnHeads * kAttnChunk; i += kAttnThreads) {
-      const int hh = i / kAttnChunk;
-      const int j = i - hh * kAttnChunk;
-      const float s = ((part[(0 * kAttnHeads + hh) * kAttnChunk + j] + part[(1 * kAttnHeads + hh) * kAttnChunk + j]) +
-                       part[(2 * kAttnHeads + hh) * kAttnChunk + j]) +
-                      part[(3 * kAttnHeads + hh) * kAttnChunk + j];
-      sc[hh * kp + c0 + j] = ids[c0 + j] >= 0 ? s * scale : -INFINITY;
+      const int j = i / kAttnHeads;
+      const int hh = i - j * kAttnHeads;
+      const float s = ((part[(0 * kAttnChunk + j) * kAttnHeads + hh] + part[(1 * kAttnChunk + j) * kAttnHeads + hh]) +
+                       part[(2 * kAttnChunk + j) * kAttnHeads + hh]) +
+                      part[(3 * kAttnChunk + j) * kAttnHeads + hh];
+      sc[(c0 + j) * kAttnHeads + hh] = ids[c0 + j] >= 0 ? s * scale : -INFINITY;
     }
     __syncthreads();
   }
@@ -167,15 +172,15 @@ __global__ void __launch_bounds__(kAttnThreads)
   {
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    float* sh = sc + warp * kp;
+    float* sh = sc + warp;                          // head `warp` of slot j at sh[j * 8]
     float m = -INFINITY;
-    for (int j = lane; j < kp; j += 32) m = fmaxf(m, sh[j]);
+    for (int j = lane; j < kp; j += 32) m = fmaxf(m, sh[j * kAttnHeads]);
     m = attn_warp_max(m);
     float l = 0.f;
     for (int j = lane; j < kp; j += 32) {
-      const float x = sh[j];
+      const float x = sh[j * kAttnHeads];
       const float e = (x == -INFINITY) ? 0.f : expf(x - m);
-      sh[j] = e;
+      sh[j * kAttnHeads] = e;
       l += e;
     }
     l = attn_warp_sum(l);
@@ -197,11 +202,14 @@ __global__ void __launch_bounds__(kAttnThreads)
       const uint32_t x = rows[j * kAttnRowWords + tid];
       const float v0 = attn_bf16_lo(x);
       const float v1 = attn_bf16_hi(x);
+      const float4* pj = reinterpret_cast<const float4*>(sc + (c0 + j) * kAttnHeads);   // 32-byte aligned
+      const float4 pa = pj[0];
+      const float4 pb = pj[1];
+      const float p[kAttnHeads] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
       for (int hh = 0; hh < kAttnHeads; ++hh) {
-        const float p = sc[hh * kp + c0 + j];
-        o[hh][0] = fmaf(p, v0, o[hh][0]);
-        o[hh][1] = fmaf(p, v1, o[hh][1]);
+        o[hh][0] = fmaf(p[hh], v0, o[hh][0]);
+        o[hh][1] = fmaf(p[hh], v1, o[hh][1]);
       }
     }
     __syncthreads();
