@@ -350,6 +350,8 @@ size_t ls_merge_select_workspace_size(int S, int T, int k_in);
 ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* offsets, int S, int T, int k_in,
                           int k, int32_t* idx_out, float* val_out, void* ws, size_t ws_bytes, void* stream);
 
+#define LS_ATTN_FOREIGN_ROWS 1   /* ls_sparse_attention: rows outside [0, n_rows) are another shard's */
+
 /*
  * ls_sparse_attention -- sparse main attention over the selected rows, stage
  * 2 of DSA ("03 long context", section "The Architectural Answer: Read Less
@@ -369,6 +371,9 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
  *        skipped and sets LS_FAULT_BAD_INDEX (see ls_device_status)
  *   H a multiple of 8, k <= 2048; scale is the softmax scale (1/sqrt(576) is
  *        the plain choice; the pages do not fix it)
+ *   flags: 0, or LS_ATTN_FOREIGN_ROWS when latent holds one shard of the
+ *        rows (row_off = -first row of the shard, n_rows = its length): rows
+ *        outside it belong to other shards and are skipped without the fault
  *   out [T][H][512] fp32; lse [T][H] fp32 natural-log sum or NULL.  An empty
  *        selection gives out = 0 and lse = -inf; partial results over
  *        disjoint selections combine exactly by their lse (online softmax).
@@ -376,8 +381,27 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
  * for the other limits.  No workspace; asynchronous on `stream`.
  */
 ls_status ls_sparse_attention(const uint16_t* q, const uint16_t* latent, const int32_t* idx, const int64_t* row_off,
-                              int T, int H, int d, int d_v, int64_t n_rows, int k, float scale, float* out, float* lse,
-                              void* stream);
+                              int T, int H, int d, int d_v, int64_t n_rows, int k, float scale, int flags, float* out,
+                              float* lse, void* stream);
+
+/*
+ * ls_attention_merge -- combine S partial attentions of the same T x H
+ * (query, head) rows over disjoint selected-row sets into the attention over
+ * their union, by the online-softmax rule (the merge of the ring-attention
+ * section of "03 long context", "Teamwork First: Ring Attention for the Giant
+ * Prefill"): with m = max_s lse_s and w_s = exp(lse_s - m),
+ *   o = sum_s w_s o_s / sum_s w_s,   lse = m + log sum_s w_s.
+ * The combine step of a history-sharded attention: each rank attends over the
+ * selected rows it holds (LS_ATTN_FOREIGN_ROWS), the (o, lse) parts are
+ * gathered, and this call merges them.
+ *
+ *   o_parts [S][rows][d_v] fp32 (8-byte aligned), lse_parts [S][rows] fp32
+ *   o [rows][d_v] fp32, lse [rows] fp32 or NULL; rows = T * H, d_v even
+ * A part with lse = -inf (an empty selection) weighs 0; when every part is
+ * empty, o = 0 and lse = -inf.  No workspace; asynchronous on `stream`.
+ */
+ls_status ls_attention_merge(const float* o_parts, const float* lse_parts, int S, int64_t rows, int d_v, float* o,
+                             float* lse, void* stream);
 
 /*
  * ls_decode_two_stage_select -- LeanSparse two-stage decode search

@@ -25,6 +25,7 @@ from ._lib import (  # noqa: F401
     ls_lsa_tree_select,
     ls_merge_select,
     ls_sparse_attention,
+    ls_attention_merge,
     ls_prefill_select_stream,
     ls_prefill_select_stream_fp8,
     ls_profile_begin,

@@ -40,7 +40,7 @@ EXPORTED = (
     "ls_indexer_score_pq", "ls_indexer_score_fp8_workspace_size", "ls_indexer_score_fp8",
     "ls_prefill_select_fp8_workspace_size", "ls_prefill_select_stream_fp8", "ls_lsa_flat_workspace_size",
     "ls_lsa_flat_select", "ls_lsa_tree_workspace_size", "ls_lsa_tree_select", "ls_merge_select_workspace_size",
-    "ls_merge_select", "ls_sparse_attention",
+    "ls_merge_select", "ls_sparse_attention", "ls_attention_merge",
 )
 HIST_BINS = 2048
 
@@ -89,7 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_lsa_tree_select": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]),
         "ls_merge_select_workspace_size": (SZ, [I, I, I]),
         "ls_merge_select": (I, [P, P, P, I, I, I, I, P, P, P, SZ, P]),
-        "ls_sparse_attention": (I, [P, P, P, P, I, I, I, I, I64, I, ctypes.c_float, P, P, P]),
+        "ls_sparse_attention": (I, [P, P, P, P, I, I, I, I, I64, I, ctypes.c_float, I, P, P, P]),
+        "ls_attention_merge": (I, [P, P, I, I64, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -537,13 +538,18 @@ def ls_merge_select(vals, idx, offsets, k: int = 512, ws=None, out=None, stream=
     return io, vo
 
 
+LS_ATTN_FOREIGN_ROWS = 1
+
+
 def ls_sparse_attention(q, latent, idx, scale: Optional[float] = None, row_off=None, want_lse: bool = True,
-                        out=None, stream=None):
+                        out=None, foreign_rows: bool = False, stream=None):
     """Sparse main attention over the selected latent rows.
 
     q [T,H,576] bf16, latent [R,576] bf16, idx [T,k] int32 (-1 = unused slot),
     row_off [T] int64 or None (row = idx + row_off[t]); scale defaults to
-    1/sqrt(576) -> (out [T,H,512] f32, lse [T,H] f32 or None)."""
+    1/sqrt(576) -> (out [T,H,512] f32, lse [T,H] f32 or None).  With
+    ``foreign_rows`` latent holds one shard of the rows (row_off = -its first
+    row) and rows outside it are skipped as another shard's."""
     _dev(q, torch.bfloat16, "q", 3)
     _dev(latent, torch.bfloat16, "latent", 2)
     _dev(idx, torch.int32, "idx", 2)
@@ -561,8 +567,28 @@ def ls_sparse_attention(q, latent, idx, scale: Optional[float] = None, row_off=N
         out = torch.empty((T, H, 512), dtype=torch.float32, device=q.device)
     lse = torch.empty((T, H), dtype=torch.float32, device=q.device) if want_lse else None
     _check(lib().ls_sparse_attention(_ptr(q), _ptr(latent), _ptr(idx), _ptr(row_off), T, H, d, 512, R, k, float(scale),
-                                     _ptr(out), _ptr(lse), _stream(stream)))
+                                     LS_ATTN_FOREIGN_ROWS if foreign_rows else 0, _ptr(out), _ptr(lse),
+                                     _stream(stream)))
     return out, lse
+
+
+def ls_attention_merge(o_parts, lse_parts, out=None, stream=None):
+    """Combine S partial attentions over disjoint row sets (online softmax).
+
+    o_parts [S,...,d_v] f32, lse_parts [S,...] f32 -> (o [...,d_v] f32, lse [...] f32)."""
+    _dev(o_parts, torch.float32, "o_parts")
+    _dev(lse_parts, torch.float32, "lse_parts")
+    S, d_v = o_parts.shape[0], o_parts.shape[-1]
+    if tuple(o_parts.shape[:-1]) != tuple(lse_parts.shape):
+        raise ValueError(f"o_parts {tuple(o_parts.shape)} and lse_parts {tuple(lse_parts.shape)} disagree")
+    rows = lse_parts[0].numel()
+    if out is None:
+        out = (torch.empty(o_parts.shape[1:], dtype=torch.float32, device=o_parts.device),
+               torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device))
+    o, lse = out
+    _check(lib().ls_attention_merge(_ptr(o_parts), _ptr(lse_parts), S, rows, d_v, _ptr(o), _ptr(lse),
+                                    _stream(stream)))
+    return o, lse
 
 
 def shard_plan(n_keys: int, n_shards: int):

@@ -1275,8 +1275,9 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
 }
 
 ls_status ls_sparse_attention(const uint16_t* q, const uint16_t* latent, const int32_t* idx, const int64_t* row_off,
-                              int T, int H, int d, int d_v, int64_t n_rows, int k, float scale, float* out, float* lse,
-                              void* stream) {
+                              int T, int H, int d, int d_v, int64_t n_rows, int k, float scale, int flags, float* out,
+                              float* lse, void* stream) {
+  LS_CHECK_ARG((flags & ~LS_ATTN_FOREIGN_ROWS) == 0, "unknown flags 0x%x", flags);
   LS_CHECK_ARG(T >= 0 && H >= 0 && k >= 0 && n_rows >= 0, "negative size (T=%d H=%d k=%d)", T, H, k);
   if (d != kAttnLatent || d_v != kAttnValue)
     return fail(LS_ERR_UNSUPPORTED, "latent rows of %d elements with %d value elements are built (got d=%d d_v=%d)",
@@ -1294,7 +1295,22 @@ ls_status ls_sparse_attention(const uint16_t* q, const uint16_t* latent, const i
                "q, latent and out must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ProfScope prof("sparse_attn_kernel", st);
-  LS_CUDA(launch_sparse_attn(q, latent, idx, row_off, T, H, k, n_rows, scale, out, lse, st));
+  LS_CUDA(launch_sparse_attn(q, latent, idx, row_off, T, H, k, n_rows, scale, (flags & LS_ATTN_FOREIGN_ROWS) ? 1 : 0,
+                             out, lse, st));
+  return LS_OK;
+}
+
+ls_status ls_attention_merge(const float* o_parts, const float* lse_parts, int S, int64_t rows, int d_v, float* o,
+                             float* lse, void* stream) {
+  LS_CHECK_ARG(S >= 1 && rows >= 0, "S must be >= 1 and rows >= 0 (S=%d)", S);
+  LS_CHECK_ARG(d_v >= 2 && d_v % 2 == 0, "d_v must be even (got %d)", d_v);
+  if (rows == 0) return LS_OK;
+  LS_CHECK_ARG(o_parts && lse_parts && o, "null tensor pointer");
+  LS_CHECK_ARG((reinterpret_cast<uintptr_t>(o_parts) & 7u) == 0 && (reinterpret_cast<uintptr_t>(o) & 7u) == 0,
+               "o_parts and o must be 8-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope prof("attn_merge_kernel", st);
+  LS_CUDA(launch_attn_merge(o_parts, lse_parts, S, rows, d_v, o, lse, num_sms_current(), st));
   return LS_OK;
 }
 

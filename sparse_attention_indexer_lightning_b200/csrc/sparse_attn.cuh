@@ -10,7 +10,8 @@
 //
 // One CTA per (query, group of 8 heads), 256 threads, on the CUDA cores:
 //
-//  1. the CTA's row ids (slot -> idx + row offset; -1 or out of range -> none)
+//  1. the CTA's row ids (slot -> idx + row offset; -1 or out of range -> none;
+//     out of range is flagged unless the caller holds one shard of the rows)
 //     and its 8 query heads (fp32, [dimension][head]) go to shared memory;
 //  2. logits: the selected rows are staged 64 at a time (a row per 289-word
 //     stride, so 32 consecutive rows start on 32 different banks); thread
@@ -94,7 +95,8 @@ __device__ __forceinline__ void attn_stage(uint32_t* rows, const int32_t* ids, i
 __global__ void __launch_bounds__(kAttnThreads)
     sparse_attn_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ latent,
                        const int32_t* __restrict__ idx, const int64_t* __restrict__ row_off, int H, int k,
-                       int64_t n_rows, float scale, float* __restrict__ out, float* __restrict__ lse) {
+                       int64_t n_rows, float scale, int foreign_ok, float* __restrict__ out,
+                       float* __restrict__ lse) {
   extern __shared__ __align__(16) unsigned char attn_smem[];
   const int kp = attn_kpad(k);
   float* qs = reinterpret_cast<float*>(attn_smem);
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(kAttnThreads)
         const int64_t r = off + s;
         if (r >= 0 && r < n_rows)
           id = static_cast<int32_t>(r);
-        else
+        else if (!foreign_ok)
           atomicOr(&g_fault, FAULT_BAD_INDEX);      // never read: the slot stays unused
       }
     }
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 }
 
 cudaError_t launch_sparse_attn(const uint16_t* q, const uint16_t* latent, const int32_t* idx, const int64_t* row_off,
-                               int T, int H, int k, int64_t n_rows, float scale, float* out, float* lse,
+                               int T, int H, int k, int64_t n_rows, float scale, int foreign_ok, float* out, float* lse,
                                cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const size_t smem = attn_smem_bytes(k);
@@ -232,7 +234,51 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint16_t* latent, const 
   if (e != cudaSuccess) return e;
   const int64_t blocks = static_cast<int64_t>(T) * (H / kAttnHeads);
   sparse_attn_kernel<<<static_cast<unsigned>(blocks), kAttnThreads, smem, st>>>(q, latent, idx, row_off, H, k, n_rows,
-                                                                                  scale, out, lse);
+                                                                                  scale, foreign_ok, out, lse);
+  return cudaGetLastError();
+}
+
+// Combine of S partial attentions of the same queries over disjoint row sets
+// (the online-softmax rule): with m = max_s lse_s and w_s = exp(lse_s - m),
+// o = sum_s w_s o_s / sum_s w_s and lse = m + log sum_s w_s.  One thread per
+// (query, head, pair of output columns); a part with lse = -inf weighs 0, and
+// all parts empty give o = 0, lse = -inf.
+__global__ void __launch_bounds__(256)
+    attn_merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int S, int64_t rows,
+                      int d_v, float* __restrict__ o, float* __restrict__ lse) {
+  const int pairs = d_v / 2;
+  const int64_t n = rows * pairs;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / pairs;
+    const int c = static_cast<int>(i - r * pairs) * 2;
+    float m = -INFINITY;
+    for (int s = 0; s < S; ++s) m = fmaxf(m, lse_parts[s * rows + r]);
+    float den = 0.f, a0 = 0.f, a1 = 0.f;
+    if (m != -INFINITY) {
+      for (int s = 0; s < S; ++s) {
+        const float ls = lse_parts[s * rows + r];
+        if (ls == -INFINITY) continue;
+        const float w = expf(ls - m);
+        const float2 v = *reinterpret_cast<const float2*>(o_parts + (s * rows + r) * d_v + c);
+        den += w;
+        a0 = fmaf(w, v.x, a0);
+        a1 = fmaf(w, v.y, a1);
+      }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    *reinterpret_cast<float2*>(o + r * d_v + c) = make_float2(a0 * inv, a1 * inv);
+    if (c == 0 && lse) lse[r] = den > 0.f ? m + logf(den) : -INFINITY;
+  }
+}
+
+cudaError_t launch_attn_merge(const float* o_parts, const float* lse_parts, int S, int64_t rows, int d_v, float* o,
+                              float* lse, int num_sms, cudaStream_t st) {
+  const int64_t n = rows * (d_v / 2);
+  if (n == 0) return cudaSuccess;
+  const int64_t want = (n + 255) / 256;
+  const int blocks = static_cast<int>(want < 8LL * num_sms ? want : 8LL * num_sms);
+  attn_merge_kernel<<<blocks, 256, 0, st>>>(o_parts, lse_parts, S, rows, d_v, o, lse);
   return cudaGetLastError();
 }
 

@@ -30,7 +30,7 @@ def test_header_declares_the_calls():
     for n in ("ls_indexer_score", "ls_topk_select", "ls_prefill_select_stream", "ls_decode_two_stage_select",
               "ls_bucket_select", "ls_decode_select", "ls_last_error", "ls_device_status", "ls_indexer_score_fp8",
               "ls_prefill_select_stream_fp8", "ls_lsa_flat_select", "ls_lsa_tree_select", "ls_indexer_score_pq",
-              "ls_decode_two_stage_pq_select", "ls_merge_select", "ls_sparse_attention"):
+              "ls_decode_two_stage_pq_select", "ls_merge_select", "ls_sparse_attention", "ls_attention_merge"):
         assert n in names
 
 
@@ -139,12 +139,18 @@ def test_argument_checks_without_gpu(lib):
     # sparse attention: latent width not built, heads not a multiple of 8, k above 2048, misaligned q,
     # empty batch
     att = lib.ls_sparse_attention
-    assert att(dummy, dummy, dummy, None, 4, 128, 128, 512, 1000, 512, 0.04, dummy, None, None) == 3
-    assert att(dummy, dummy, dummy, None, 4, 12, 576, 512, 1000, 512, 0.04, dummy, None, None) == 1
-    assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 4096, 0.04, dummy, None, None) == 1
-    assert att(P(8), dummy, dummy, None, 4, 128, 576, 512, 1000, 512, 0.04, dummy, None, None) == 1
-    assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 512, float("nan"), dummy, None, None) == 1
-    assert att(None, None, None, None, 0, 128, 576, 512, 1000, 512, 0.04, None, None, None) == 0
+    assert att(dummy, dummy, dummy, None, 4, 128, 128, 512, 1000, 512, 0.04, 0, dummy, None, None) == 3
+    assert att(dummy, dummy, dummy, None, 4, 12, 576, 512, 1000, 512, 0.04, 0, dummy, None, None) == 1
+    assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 4096, 0.04, 0, dummy, None, None) == 1
+    assert att(P(8), dummy, dummy, None, 4, 128, 576, 512, 1000, 512, 0.04, 0, dummy, None, None) == 1
+    assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 512, float("nan"), 0, dummy, None, None) == 1
+    assert att(None, None, None, None, 0, 128, 576, 512, 1000, 512, 0.04, 0, None, None, None) == 0
+    assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 512, 0.04, 6, dummy, None, None) == 1
+    # attention merge: no parts, odd value width, empty
+    mg = lib.ls_attention_merge
+    assert mg(dummy, dummy, 0, 10, 512, dummy, None, None) == 1
+    assert mg(dummy, dummy, 2, 10, 511, dummy, None, None) == 1
+    assert mg(None, None, 2, 0, 512, None, None, None) == 0
     # bucket: budget below k
     st = lib.ls_bucket_select(dummy, dummy, dummy, dummy, dummy, dummy, 1, 32, 128, 10, 80, 4, 100, 512, dummy,
                               None, None, dummy, 1 << 30, None)

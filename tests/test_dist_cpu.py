@@ -88,3 +88,56 @@ def test_history_shards_cover_the_history_once(n_keys):
         assert base == pos and length > 0
         pos += length
     assert pos == n_keys
+
+
+def _attn_shard_worker(rank, world, port, q):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from oracle.attention import default_scale, merge_partials, sparse_attention
+    from oracle.formats import bf16_to_f64
+    from sparse_attention_indexer_lightning_b200 import shard_plan
+    from workloads.synth import make_attention
+    d = make_attention(5, 8, 900, 120, ragged=100, seed=4)
+    lat = bf16_to_f64(d["latent"])
+    base, length = shard_plan(lat.shape[0], world)[rank]
+    # this rank holds rows [base, base + length): the selection shifted by
+    # -base, rows outside its range skipped (another rank's)
+    local = d["idx"].astype(np.int64) - base
+    local = np.where((d["idx"] >= 0) & (local >= 0) & (local < length), local, -1)
+    o, lse = sparse_attention(bf16_to_f64(d["q"]), lat[base:base + length], local, default_scale())
+    o_all = [torch.zeros_like(torch.from_numpy(o)) for _ in range(world)]
+    l_all = [torch.zeros_like(torch.from_numpy(lse)) for _ in range(world)]
+    dist.all_gather(o_all, torch.from_numpy(o))
+    dist.all_gather(l_all, torch.from_numpy(lse))
+    mo, ml = o_all[0].numpy(), l_all[0].numpy()
+    for r in range(1, world):
+        mo, ml = merge_partials(mo, ml, o_all[r].numpy(), l_all[r].numpy())
+    ro, rl = sparse_attention(bf16_to_f64(d["q"]), lat, d["idx"], default_scale())
+    ok = (np.allclose(mo, ro, rtol=1e-12, atol=1e-13) and np.array_equal(np.isneginf(ml), np.isneginf(rl))
+          and np.allclose(ml[np.isfinite(rl)], rl[np.isfinite(rl)], rtol=1e-12))
+    q.put((rank, bool(ok)))
+    dist.destroy_process_group()
+
+
+def test_history_sharded_attention_merges_to_the_full_attention():
+    """Two gloo ranks each hold half of the latent rows, attend over the
+    selected rows they hold, all-gather (o, lse) and merge by the
+    online-softmax rule: every rank ends with the attention over the whole
+    selection (the protocol of the sharded decode, computed by the oracle)."""
+    import multiprocessing as mp_
+    ctx = mp_.get_context("spawn")
+    q = ctx.Queue()
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    procs = [ctx.Process(target=_attn_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == {0: True, 1: True}

@@ -128,6 +128,59 @@ def test_sparse_attention_lse_merges_disjoint_parts(L):
     assert np.all(np.abs(lm - lse) <= ATTN_TOL * (1 + np.abs(lse)))
 
 
+def test_attention_merge_kernel(L):
+    """ls_attention_merge against the oracle's online-softmax rule on random
+    parts, with empty parts (lse = -inf) mixed in and one row empty in every part."""
+    rng = np.random.default_rng(5)
+    S, T, H, dv = 4, 3, 16, 512
+    o = rng.standard_normal((S, T, H, dv)).astype(np.float32)
+    lse = (rng.standard_normal((S, T, H)) * 3).astype(np.float32)
+    lse[1, 0, :] = -np.inf
+    lse[:, 2, 5] = -np.inf
+    o[:, 2, 5] = 0.0
+    mo, ml = L.ls_attention_merge(dev(o), dev(lse))
+    torch.cuda.synchronize()
+    mo, ml = mo.cpu().numpy(), ml.cpu().numpy()
+    ro, rl = o[0].astype(np.float64), lse[0].astype(np.float64)
+    for s in range(1, S):
+        ro, rl = merge_partials(ro, rl, o[s].astype(np.float64), lse[s].astype(np.float64))
+    assert np.all(mo[2, 5] == 0.0) and np.isneginf(ml[2, 5])
+    assert np.abs(mo - ro).max() <= 1e-5 * np.abs(o).max()
+    fin = np.isfinite(rl)
+    assert np.array_equal(np.isneginf(ml), np.isneginf(rl))
+    assert np.all(np.abs(ml[fin] - rl[fin]) <= 1e-5 * (1 + np.abs(rl[fin])))
+
+
+def test_sparse_attention_history_shards_merge(L):
+    """The latent rows split into 3 contiguous shards (one per GPU in a
+    history-sharded decode): each shard attends over the selected rows it
+    holds (row_off = -its first row; other shards' rows are skipped without
+    the fault), and ls_attention_merge combines the (o, lse) parts into the
+    attention over the whole selection."""
+    d = data("attn_s")
+    N = d["latent"].shape[0]
+    T = d["q"].shape[0]
+    q, idx = dev_bf16(d["q"]), dev(d["idx"])
+    full_o, full_l = _run(L, d)
+    L.ls_device_status()
+    parts_o, parts_l = [], []
+    for base, length in L.shard_plan(N, 3):
+        lat = dev_bf16(np.ascontiguousarray(d["latent"][base:base + length]))
+        off = dev(np.full(T, -base, dtype=np.int64))
+        o, lse = L.ls_sparse_attention(q, lat, idx, row_off=off, foreign_rows=True)
+        parts_o.append(o)
+        parts_l.append(lse)
+    mo, ml = L.ls_attention_merge(torch.stack(parts_o), torch.stack(parts_l))
+    torch.cuda.synchronize()
+    assert L.ls_device_status() == 0
+    mo, ml = mo.cpu().numpy(), ml.cpu().numpy()
+    vmax = np.abs(bf16_to_f64(d["latent"][:, :512])).max()
+    assert np.abs(mo - full_o).max() <= ATTN_TOL * vmax
+    fin = np.isfinite(full_l)
+    assert np.array_equal(np.isneginf(ml), np.isneginf(full_l))
+    assert np.all(np.abs(ml[fin] - full_l[fin]) <= ATTN_TOL * (1 + np.abs(full_l[fin])))
+
+
 def test_sparse_attention_after_decode_selection(L):
     """The decode indexer's top-512 of each sequence, fed as is to the sparse
     attention over a cache holding every sequence's latent rows (row_off =
