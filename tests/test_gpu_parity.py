@@ -323,6 +323,37 @@ def test_prefill_sharded_history_merge(L):
         assert f32_bits_equal(mv.cpu().numpy(), val0), S
 
 
+def test_merge_select_edge_cases(L):
+    """ls_merge_select on hand-made shard lists: one shard (the identity), a
+    shard whose lists are all padding, lists shorter than k (fewer
+    candidates than k: the result is padded), equal values across shards
+    (the lower global position first), compared with the top-k of the union
+    of the valid entries."""
+    rng = np.random.default_rng(8)
+    T, k_in = 6, 40
+    for S, k, empty_shard in ((1, 40, None), (3, 40, 1), (2, 100, None), (4, 64, 3)):
+        offs = np.array([1000 * s for s in range(S)], dtype=np.int32)
+        vals = np.full((S, T, k_in), -np.inf, dtype=np.float32)
+        idx = np.full((S, T, k_in), -1, dtype=np.int32)
+        for s in range(S):
+            for t in range(T):
+                n = 0 if s == empty_shard else int(rng.integers(0, k_in + 1))
+                pos = np.sort(rng.choice(900, size=n, replace=False))
+                v = np.round(rng.standard_normal(n) * 2).astype(np.float32)   # many equal values
+                sel_pos, sel_val = select_topk(v, pos, k_in)                   # each list in canonical order
+                idx[s, t], vals[s, t] = sel_pos.astype(np.int32), sel_val.astype(np.float32)
+        mi, mv = L.ls_merge_select(dev(vals), dev(idx), dev(offs), k=k)
+        torch.cuda.synchronize()
+        mi, mv = mi.cpu().numpy(), mv.cpu().numpy()
+        for t in range(T):
+            ok = idx[:, t] >= 0
+            gpos = (idx[:, t] + offs[:, None])[ok]
+            gval = vals[:, t][ok]
+            rp, rv = select_topk(gval, gpos, k)
+            assert np.array_equal(mi[t], rp), (S, k, t)
+            assert f32_bits_equal(mv[t], rv.astype(np.float32)), (S, k, t)
+
+
 # --------------------------------------------------------------------------- #
 # fp8 indexer: fp8 queries and keys, the prefill streamed from an fp8 history
 # --------------------------------------------------------------------------- #
