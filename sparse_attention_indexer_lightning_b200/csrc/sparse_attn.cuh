@@ -14,10 +14,10 @@
 //     out of range is flagged unless the caller holds one shard of the rows)
 //     and its 8 query heads (fp32, [dimension][head]) go to shared memory;
 //  2. logits: the selected rows are staged 64 at a time (a row per 289-word
-//     stride, so 32 consecutive rows start on 32 different banks); thread
-//     (row j, quarter p) takes dimensions 144p .. 144p + 143 for all 8 heads,
-//     and the four quarters are added in a fixed order; logits are kept
-//     slot-major ([slot][head]);
+//     stride, so 32 consecutive rows start on 32 different banks); warp p
+//     takes dimensions 72p .. 72p + 71 (its query loads are broadcasts) and
+//     its lane g rows g and g + 32, for all 8 heads; the eight partial sums
+//     are added in a fixed order; logits are kept slot-major ([slot][head]);
 //  3. softmax: warp h takes head h: max, exp(logit - max), sum, 1 / sum, lse;
 //  4. values: the value parts are staged again, 64 rows at a time; thread i
 //     owns output columns 2i and 2i + 1 of all 8 heads and reads a row's 8
@@ -40,11 +40,13 @@ constexpr int kAttnChunk = 64;                      // selected rows staged per 
 constexpr int kAttnThreads = 256;
 constexpr int kAttnMaxK = 2048;
 constexpr int kAttnRowWords = kAttnLatent / 2 + 1;  // 289 words: row r starts on bank r mod 32
-constexpr int kAttnQuarter = kAttnLatent / 4;       // 144 dimensions per partial dot product
+constexpr int kAttnParts = kAttnThreads / 32;      // dimension slices, one per warp
+constexpr int kAttnSlice = kAttnLatent / kAttnParts;  // 72 dimensions per partial dot product
 static_assert(kAttnValue / 2 == kAttnThreads, "one value column pair per thread");
-static_assert(kAttnThreads == 4 * kAttnChunk, "four dimension quarters per staged row");
+static_assert(kAttnChunk == 64, "a lane scores staged rows g and g + 32");
+static_assert(kAttnSlice % 2 == 0, "slices of whole bf16 pairs");
 static_assert(kAttnThreads / 32 == kAttnHeads, "one warp per head in the softmax");
-static_assert((kAttnLatent * kAttnHeads + kAttnChunk * kAttnRowWords + 4 * kAttnHeads * kAttnChunk) % 4 == 0,
+static_assert((kAttnLatent * kAttnHeads + kAttnChunk * kAttnRowWords + kAttnParts * kAttnHeads * kAttnChunk) % 4 == 0,
               "the weights start on a 16-byte boundary (float4 reads)");
 
 __host__ __device__ constexpr int attn_kpad(int k) { return (k + kAttnChunk - 1) / kAttnChunk * kAttnChunk; }
@@ -53,7 +55,7 @@ __host__ __device__ constexpr int attn_kpad(int k) { return (k + kAttnChunk - 1)
 __host__ __device__ constexpr size_t attn_smem_bytes(int k) {
   return 4 * (static_cast<size_t>(kAttnLatent) * kAttnHeads      // query heads [d][h]
               + static_cast<size_t>(kAttnChunk) * kAttnRowWords  // staged rows
-              + 4 * kAttnHeads * kAttnChunk                       // partial dot products [quarter][row][h]
+              + kAttnParts * kAttnHeads * kAttnChunk              // partial dot products [slice][row][h]
               + static_cast<size_t>(kAttnHeads) * attn_kpad(k)    // logits, then weights [slot][h]
               + attn_kpad(k)                                      // row ids [slot]
               + kAttnHeads);                                      // 1 / sum of weights [h]
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   float* qs = reinterpret_cast<float*>(attn_smem);
   uint32_t* rows = reinterpret_cast<uint32_t*>(qs + kAttnLatent * kAttnHeads);
   float* part = reinterpret_cast<float*>(rows + kAttnChunk * kAttnRowWords);
-  float* sc = part + 4 * kAttnHeads * kAttnChunk;
+  float* sc = part + kAttnParts * kAttnHeads * kAttnChunk;
   int32_t* ids = reinterpret_cast<int32_t*>(sc + kAttnHeads * kp);
   float* inv_l = reinterpret_cast<float*>(ids + kp);
 
@@ -136,35 +138,48 @@ __global__ void __launch_bounds__(kAttnThreads)
   __syncthreads();
 
   // 2. logits
-  const int jj = tid & (kAttnChunk - 1);
-  const int qd = tid / kAttnChunk;
+  const int g = tid & 31;                             // staged rows g and g + 32
+  const int sl = tid >> 5;                            // dimension slice of this warp
   for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
     attn_stage(rows, ids, c0, latent, kAttnLatent / 2);
     __syncthreads();
-    float acc[kAttnHeads];
+    float a0[kAttnHeads], a1[kAttnHeads];
 #pragma unroll
-    for (int hh = 0; hh < kAttnHeads; ++hh) acc[hh] = 0.f;
-    const uint32_t* rw = rows + jj * kAttnRowWords + qd * (kAttnQuarter / 2);
-    const float* qq = qs + qd * kAttnQuarter * kAttnHeads;
-#pragma unroll 4
-    for (int w = 0; w < kAttnQuarter / 2; ++w) {
-      const uint32_t x = rw[w];
+    for (int hh = 0; hh < kAttnHeads; ++hh) a0[hh] = a1[hh] = 0.f;
+    const uint32_t* r0 = rows + g * kAttnRowWords + sl * (kAttnSlice / 2);
+    const uint32_t* r1 = r0 + 32 * kAttnRowWords;
+    const float* qq = qs + sl * kAttnSlice * kAttnHeads;
+#pragma unroll 2
+    for (int w = 0; w < kAttnSlice / 2; ++w) {
+      const uint32_t x = r0[w];
+      const uint32_t y = r1[w];
       const float x0 = attn_bf16_lo(x);
       const float x1 = attn_bf16_hi(x);
+      const float y0 = attn_bf16_lo(y);
+      const float y1 = attn_bf16_hi(y);
       const float* q0 = qq + 2 * w * kAttnHeads;
 #pragma unroll
-      for (int hh = 0; hh < kAttnHeads; ++hh) acc[hh] = fmaf(x1, q0[kAttnHeads + hh], fmaf(x0, q0[hh], acc[hh]));
+      for (int hh = 0; hh < kAttnHeads; ++hh) {
+        const float qa = q0[hh];
+        const float qb = q0[kAttnHeads + hh];
+        a0[hh] = fmaf(x1, qb, fmaf(x0, qa, a0[hh]));
+        a1[hh] = fmaf(y1, qb, fmaf(y0, qa, a1[hh]));
+      }
     }
-    float* pp = part + (qd * kAttnChunk + jj) * kAttnHeads;
+    float* p0 = part + (sl * kAttnChunk + g) * kAttnHeads;
+    float* p1 = p0 + 32 * kAttnHeads;
 #pragma unroll
-    for (int hh = 0; hh < kAttnHeads; ++hh) pp[hh] = acc[hh];
+    for (int hh = 0; hh < kAttnHeads; ++hh) {
+      p0[hh] = a0[hh];
+      p1[hh] = a1[hh];
+    }
     __syncthreads();
     for (int i = tid; i < kAttnHeads * kAttnChunk; i += kAttnThreads) {
       const int j = i / kAttnHeads;
       const int hh = i - j * kAttnHeads;
-      const float s = ((part[(0 * kAttnChunk + j) * kAttnHeads + hh] + part[(1 * kAttnChunk + j) * kAttnHeads + hh]) +
-                       part[(2 * kAttnChunk + j) * kAttnHeads + hh]) +
-                      part[(3 * kAttnChunk + j) * kAttnHeads + hh];
+      float s = part[j * kAttnHeads + hh];
+#pragma unroll
+      for (int q = 1; q < kAttnParts; ++q) s += part[(q * kAttnChunk + j) * kAttnHeads + hh];
       sc[(c0 + j) * kAttnHeads + hh] = ids[c0 + j] >= 0 ? s * scale : -INFINITY;
     }
     __syncthreads();
