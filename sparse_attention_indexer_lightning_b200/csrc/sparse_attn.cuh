@@ -19,9 +19,11 @@
 //     its lane g rows g and g + 32, for all 8 heads; the eight partial sums
 //     are added in a fixed order; logits are kept slot-major ([slot][head]);
 //  3. softmax: warp h takes head h: max, exp(logit - max), sum, 1 / sum, lse;
-//  4. values: the value parts are staged again, 64 rows at a time; thread i
-//     owns output columns 2i and 2i + 1 of all 8 heads and reads a row's 8
-//     weights as two 16-byte broadcasts.
+//  4. values: the value parts are staged again, 64 rows at a time, densely
+//     (256 words a row); thread i of each half owns output columns 4i .. 4i + 3
+//     of all 8 heads, the lower half takes the even rows and the upper half
+//     the odd ones, reading a row's 8 weights as two 16-byte broadcasts; the
+//     two halves' sums are added at the end.
 //
 // The selection sits in shared memory in full (k <= 2048 slots), so the
 // softmax is exact in two passes, with no running rescale.  Unused slots
@@ -42,7 +44,9 @@ constexpr int kAttnMaxK = 2048;
 constexpr int kAttnRowWords = kAttnLatent / 2 + 1;  // 289 words: row r starts on bank r mod 32
 constexpr int kAttnParts = kAttnThreads / 32;      // dimension slices, one per warp
 constexpr int kAttnSlice = kAttnLatent / kAttnParts;  // 72 dimensions per partial dot product
-static_assert(kAttnValue / 2 == kAttnThreads, "one value column pair per thread");
+static_assert(kAttnValue / 4 == kAttnThreads / 2, "four value columns per thread of each half");
+static_assert(kAttnThreads / 2 * 4 * kAttnHeads <= kAttnParts * kAttnHeads * kAttnChunk,
+              "the upper half's sums fit the partial-sum buffer");
 static_assert(kAttnChunk == 64, "a lane scores staged rows g and g + 32");
 static_assert(kAttnSlice % 2 == 0, "slices of whole bf16 pairs");
 static_assert(kAttnThreads / 32 == kAttnHeads, "one warp per head in the softmax");
@@ -75,9 +79,9 @@ __device__ __forceinline__ float attn_warp_sum(float v) {
 }
 
 // Stage the first `words` 32-bit words (bf16 pairs) of the rows in slots
-// c0 .. c0 + 63; an unused slot stages zeros.
+// c0 .. c0 + 63, a row every `stride` words; an unused slot stages zeros.
 __device__ __forceinline__ void attn_stage(uint32_t* rows, const int32_t* ids, int c0,
-                                           const uint16_t* __restrict__ latent, int words) {
+                                           const uint16_t* __restrict__ latent, int words, int stride) {
   const int vecs = words / 4;                       // 16-byte loads per row
   for (int i = threadIdx.x; i < kAttnChunk * vecs; i += kAttnThreads) {
     const int r = i / vecs;
@@ -85,7 +89,7 @@ __device__ __forceinline__ void attn_stage(uint32_t* rows, const int32_t* ids, i
     const int32_t id = ids[c0 + r];
     uint4 x = make_uint4(0u, 0u, 0u, 0u);
     if (id >= 0) x = __ldg(reinterpret_cast<const uint4*>(latent + static_cast<int64_t>(id) * kAttnLatent) + v);
-    uint32_t* dst = rows + r * kAttnRowWords + 4 * v;
+    uint32_t* dst = rows + r * stride + 4 * v;
     dst[0] = x.x;
     dst[1] = x.y;
     dst[2] = x.z;
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   const int g = tid & 31;                             // staged rows g and g + 32
   const int sl = tid >> 5;                            // dimension slice of this warp
   for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
-    attn_stage(rows, ids, c0, latent, kAttnLatent / 2);
+    attn_stage(rows, ids, c0, latent, kAttnLatent / 2, kAttnRowWords);
     __syncthreads();
     float a0[kAttnHeads], a1[kAttnHeads];
 #pragma unroll
@@ -209,16 +213,21 @@ __global__ void __launch_bounds__(kAttnThreads)
   __syncthreads();
 
   // 4. values
-  float o[kAttnHeads][2];
+  constexpr int kValWords = kAttnValue / 2;           // dense staging: row j at word 256 j (8-byte aligned)
+  const int cg = tid & (kAttnThreads / 2 - 1);        // columns 4 cg .. 4 cg + 3
+  const int half = tid / (kAttnThreads / 2);          // rows of this parity
+  float o[kAttnHeads][4];
 #pragma unroll
-  for (int hh = 0; hh < kAttnHeads; ++hh) o[hh][0] = o[hh][1] = 0.f;
+  for (int hh = 0; hh < kAttnHeads; ++hh) o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
   for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
-    attn_stage(rows, ids, c0, latent, kAttnValue / 2);
+    attn_stage(rows, ids, c0, latent, kValWords, kValWords);
     __syncthreads();
-    for (int j = 0; j < kAttnChunk; ++j) {
-      const uint32_t x = rows[j * kAttnRowWords + tid];
-      const float v0 = attn_bf16_lo(x);
-      const float v1 = attn_bf16_hi(x);
+    for (int j = half; j < kAttnChunk; j += 2) {
+      const uint2 x = *reinterpret_cast<const uint2*>(rows + j * kValWords + 2 * cg);
+      const float v0 = attn_bf16_lo(x.x);
+      const float v1 = attn_bf16_hi(x.x);
+      const float v2 = attn_bf16_lo(x.y);
+      const float v3 = attn_bf16_hi(x.y);
       const float4* pj = reinterpret_cast<const float4*>(sc + (c0 + j) * kAttnHeads);   // 32-byte aligned
       const float4 pa = pj[0];
       const float4 pb = pj[1];
@@ -227,15 +236,29 @@ __global__ void __launch_bounds__(kAttnThreads)
       for (int hh = 0; hh < kAttnHeads; ++hh) {
         o[hh][0] = fmaf(p[hh], v0, o[hh][0]);
         o[hh][1] = fmaf(p[hh], v1, o[hh][1]);
+        o[hh][2] = fmaf(p[hh], v2, o[hh][2]);
+        o[hh][3] = fmaf(p[hh], v3, o[hh][3]);
       }
     }
     __syncthreads();
   }
+  // the odd rows' sums go through shared memory (the partial-sum buffer is free) to the even rows' threads
+  float4* xfer = reinterpret_cast<float4*>(part) + cg;   // head hh at xfer[hh * 128]
+  if (half == 1) {
 #pragma unroll
-  for (int hh = 0; hh < kAttnHeads; ++hh) {
-    float* dst = out + (static_cast<int64_t>(t) * H + h0 + hh) * kAttnValue + 2 * tid;
-    const float il = inv_l[hh];
-    *reinterpret_cast<float2*>(dst) = make_float2(o[hh][0] * il, o[hh][1] * il);
+    for (int hh = 0; hh < kAttnHeads; ++hh)
+      xfer[hh * (kAttnThreads / 2)] = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
+  }
+  __syncthreads();
+  if (half == 0) {
+#pragma unroll
+    for (int hh = 0; hh < kAttnHeads; ++hh) {
+      const float4 u = xfer[hh * (kAttnThreads / 2)];
+      const float il = inv_l[hh];
+      float* dst = out + (static_cast<int64_t>(t) * H + h0 + hh) * kAttnValue + 4 * cg;
+      *reinterpret_cast<float4*>(dst) =
+          make_float4((o[hh][0] + u.x) * il, (o[hh][1] + u.y) * il, (o[hh][2] + u.z) * il, (o[hh][3] + u.w) * il);
+    }
   }
 }
 
