@@ -27,7 +27,9 @@
 //
 // The selection sits in shared memory in full (k <= 2048 slots), so the
 // softmax is exact in two passes, with no running rescale.  Unused slots
-// stage zeros and weigh 0.
+// stage zeros and weigh 0.  Rows are gathered a chunk ahead into registers
+// (the next chunk's loads are in flight while the current one is computed;
+// the value pass's first chunk while the softmax runs).
 
 #pragma once
 
@@ -78,22 +80,46 @@ __device__ __forceinline__ float attn_warp_sum(float v) {
   return v;
 }
 
-// Stage the first `words` 32-bit words (bf16 pairs) of the rows in slots
-// c0 .. c0 + 63, a row every `stride` words; an unused slot stages zeros.
-__device__ __forceinline__ void attn_stage(uint32_t* rows, const int32_t* ids, int c0,
-                                           const uint16_t* __restrict__ latent, int words, int stride) {
-  const int vecs = words / 4;                       // 16-byte loads per row
-  for (int i = threadIdx.x; i < kAttnChunk * vecs; i += kAttnThreads) {
-    const int r = i / vecs;
-    const int v = i - r * vecs;
+// One thread's share of a chunk of 64 staged rows, `WORDS` 32-bit words
+// (bf16 pairs) of each, held in registers between the global loads and the
+// shared-memory stores, so that the next chunk's gather is in flight while
+// the current one is computed.
+template <int WORDS>
+struct AttnChunk {
+  static constexpr int kVecs = WORDS / 4;                               // 16-byte loads per row
+  static constexpr int kPer = kAttnChunk * kVecs / kAttnThreads;        // loads per thread
+  static_assert(kAttnChunk * kVecs % kAttnThreads == 0, "whole loads per thread");
+  uint4 v[kPer];
+};
+
+// Gather rows of slots c0 .. c0 + 63 (an unused slot gives zeros).
+template <int WORDS>
+__device__ __forceinline__ void attn_fetch(AttnChunk<WORDS>& c, const int32_t* ids, int c0,
+                                           const uint16_t* __restrict__ latent) {
+#pragma unroll
+  for (int m = 0; m < AttnChunk<WORDS>::kPer; ++m) {
+    const int i = threadIdx.x + m * kAttnThreads;
+    const int r = i / AttnChunk<WORDS>::kVecs;
+    const int v = i - r * AttnChunk<WORDS>::kVecs;
     const int32_t id = ids[c0 + r];
-    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-    if (id >= 0) x = __ldg(reinterpret_cast<const uint4*>(latent + static_cast<int64_t>(id) * kAttnLatent) + v);
+    c.v[m] = make_uint4(0u, 0u, 0u, 0u);
+    if (id >= 0) c.v[m] = __ldg(reinterpret_cast<const uint4*>(latent + static_cast<int64_t>(id) * kAttnLatent) + v);
+  }
+}
+
+// Store a fetched chunk into shared memory, a row every `stride` words.
+template <int WORDS>
+__device__ __forceinline__ void attn_put(const AttnChunk<WORDS>& c, uint32_t* rows, int stride) {
+#pragma unroll
+  for (int m = 0; m < AttnChunk<WORDS>::kPer; ++m) {
+    const int i = threadIdx.x + m * kAttnThreads;
+    const int r = i / AttnChunk<WORDS>::kVecs;
+    const int v = i - r * AttnChunk<WORDS>::kVecs;
     uint32_t* dst = rows + r * stride + 4 * v;
-    dst[0] = x.x;
-    dst[1] = x.y;
-    dst[2] = x.z;
-    dst[3] = x.w;
+    dst[0] = c.v[m].x;
+    dst[1] = c.v[m].y;
+    dst[2] = c.v[m].z;
+    dst[3] = c.v[m].w;
   }
 }
 
@@ -144,50 +170,60 @@ __global__ void __launch_bounds__(kAttnThreads)
   // 2. logits
   const int g = tid & 31;                             // staged rows g and g + 32
   const int sl = tid >> 5;                            // dimension slice of this warp
-  for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
-    attn_stage(rows, ids, c0, latent, kAttnLatent / 2, kAttnRowWords);
-    __syncthreads();
-    float a0[kAttnHeads], a1[kAttnHeads];
+  {
+    AttnChunk<kAttnLatent / 2> next;
+    attn_fetch(next, ids, 0, latent);
+    for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
+      attn_put(next, rows, kAttnRowWords);
+      __syncthreads();
+      if (c0 + kAttnChunk < kp) attn_fetch(next, ids, c0 + kAttnChunk, latent);   // in flight during the math
+      float a0[kAttnHeads], a1[kAttnHeads];
 #pragma unroll
-    for (int hh = 0; hh < kAttnHeads; ++hh) a0[hh] = a1[hh] = 0.f;
-    const uint32_t* r0 = rows + g * kAttnRowWords + sl * (kAttnSlice / 2);
-    const uint32_t* r1 = r0 + 32 * kAttnRowWords;
-    const float* qq = qs + sl * kAttnSlice * kAttnHeads;
+      for (int hh = 0; hh < kAttnHeads; ++hh) a0[hh] = a1[hh] = 0.f;
+      const uint32_t* r0 = rows + g * kAttnRowWords + sl * (kAttnSlice / 2);
+      const uint32_t* r1 = r0 + 32 * kAttnRowWords;
+      const float* qq = qs + sl * kAttnSlice * kAttnHeads;
 #pragma unroll 2
-    for (int w = 0; w < kAttnSlice / 2; ++w) {
-      const uint32_t x = r0[w];
-      const uint32_t y = r1[w];
-      const float x0 = attn_bf16_lo(x);
-      const float x1 = attn_bf16_hi(x);
-      const float y0 = attn_bf16_lo(y);
-      const float y1 = attn_bf16_hi(y);
-      const float* q0 = qq + 2 * w * kAttnHeads;
+      for (int w = 0; w < kAttnSlice / 2; ++w) {
+        const uint32_t x = r0[w];
+        const uint32_t y = r1[w];
+        const float x0 = attn_bf16_lo(x);
+        const float x1 = attn_bf16_hi(x);
+        const float y0 = attn_bf16_lo(y);
+        const float y1 = attn_bf16_hi(y);
+        const float* q0 = qq + 2 * w * kAttnHeads;
+#pragma unroll
+        for (int hh = 0; hh < kAttnHeads; ++hh) {
+          const float qa = q0[hh];
+          const float qb = q0[kAttnHeads + hh];
+          a0[hh] = fmaf(x1, qb, fmaf(x0, qa, a0[hh]));
+          a1[hh] = fmaf(y1, qb, fmaf(y0, qa, a1[hh]));
+        }
+      }
+      float* p0 = part + (sl * kAttnChunk + g) * kAttnHeads;
+      float* p1 = p0 + 32 * kAttnHeads;
 #pragma unroll
       for (int hh = 0; hh < kAttnHeads; ++hh) {
-        const float qa = q0[hh];
-        const float qb = q0[kAttnHeads + hh];
-        a0[hh] = fmaf(x1, qb, fmaf(x0, qa, a0[hh]));
-        a1[hh] = fmaf(y1, qb, fmaf(y0, qa, a1[hh]));
+        p0[hh] = a0[hh];
+        p1[hh] = a1[hh];
       }
-    }
-    float* p0 = part + (sl * kAttnChunk + g) * kAttnHeads;
-    float* p1 = p0 + 32 * kAttnHeads;
+      __syncthreads();
+      for (int i = tid; i < kAttnHeads * kAttnChunk; i += kAttnThreads) {
+        const int j = i / kAttnHeads;
+        const int hh = i - j * kAttnHeads;
+        float s = part[j * kAttnHeads + hh];
 #pragma unroll
-    for (int hh = 0; hh < kAttnHeads; ++hh) {
-      p0[hh] = a0[hh];
-      p1[hh] = a1[hh];
+        for (int sp = 1; sp < kAttnParts; ++sp) s += part[(sp * kAttnChunk + j) * kAttnHeads + hh];
+        sc[(c0 + j) * kAttnHeads + hh] = ids[c0 + j] >= 0 ? s * scale : -INFINITY;
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    for (int i = tid; i < kAttnHeads * kAttnChunk; i += kAttnThreads) {
-      const int j = i / kAttnHeads;
-      const int hh = i - j * kAttnHeads;
-      float s = part[j * kAttnHeads + hh];
-#pragma unroll
-      for (int q = 1; q < kAttnParts; ++q) s += part[(q * kAttnChunk + j) * kAttnHeads + hh];
-      sc[(c0 + j) * kAttnHeads + hh] = ids[c0 + j] >= 0 ? s * scale : -INFINITY;
-    }
-    __syncthreads();
   }
+
+  // the value pass's first gather overlaps the softmax
+  constexpr int kValWords = kAttnValue / 2;           // dense staging: row j at word 256 j (8-byte aligned)
+  AttnChunk<kValWords> vnext;
+  attn_fetch(vnext, ids, 0, latent);
 
   // 3. softmax, one warp per head (kp is a multiple of 32: every lane loops alike)
   {
@@ -213,15 +249,15 @@ __global__ void __launch_bounds__(kAttnThreads)
   __syncthreads();
 
   // 4. values
-  constexpr int kValWords = kAttnValue / 2;           // dense staging: row j at word 256 j (8-byte aligned)
   const int cg = tid & (kAttnThreads / 2 - 1);        // columns 4 cg .. 4 cg + 3
   const int half = tid / (kAttnThreads / 2);          // rows of this parity
   float o[kAttnHeads][4];
 #pragma unroll
   for (int hh = 0; hh < kAttnHeads; ++hh) o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
   for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
-    attn_stage(rows, ids, c0, latent, kValWords, kValWords);
+    attn_put(vnext, rows, kValWords);
     __syncthreads();
+    if (c0 + kAttnChunk < kp) attn_fetch(vnext, ids, c0 + kAttnChunk, latent);
     for (int j = half; j < kAttnChunk; j += 2) {
       const uint2 x = *reinterpret_cast<const uint2*>(rows + j * kValWords + 2 * cg);
       const float v0 = attn_bf16_lo(x.x);
