@@ -168,3 +168,24 @@ def test_missing_library_fails_loudly(tmp_path):
     from sparse_attention_indexer_lightning_b200 import _lib
     with pytest.raises(ImportError):
         _lib.load_library(str(tmp_path / "libls_indexer.so"))
+
+
+def test_bindings_refuse_host_tensors():
+    """The Python calls only marshal device tensors into the C ABI: host
+    tensors are refused before anything runs (there is no CPU path)."""
+    import torch
+    import sparse_attention_indexer_lightning_b200 as L
+    q = torch.zeros((2, 8, 576), dtype=torch.bfloat16)
+    lat = torch.zeros((10, 576), dtype=torch.bfloat16)
+    idx = torch.zeros((2, 4), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.ls_sparse_attention(q, lat, idx)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.ls_attention_merge(torch.zeros((2, 3, 512)), torch.zeros((2, 3)))
+    with pytest.raises(ValueError, match="CUDA"):
+        L.ls_merge_select(torch.zeros((2, 3, 8)), torch.zeros((2, 3, 8), dtype=torch.int32),
+                          torch.zeros(2, dtype=torch.int32))
+    w = torch.zeros((2, 32), dtype=torch.float32)
+    keys = torch.zeros((2, 64, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.ls_decode_select(torch.zeros((2, 32, 128), dtype=torch.bfloat16), w, keys)
