@@ -1,0 +1,65 @@
+// Host stand-ins for the CUDA features the attention kernels use, so that
+// their source compiles with g++ and runs on the CPU for the kernel-logic
+// tests: one OS thread per CUDA thread of a block, std::barrier for
+// __syncthreads and for the two halves of a warp shuffle, a mutex for atomics.
+// Shared memory is a buffer of the launch's dynamic size (AddressSanitizer
+// sees its end).  Test infrastructure only.
+#pragma once
+#include <barrier>
+#include <cmath>
+#include <cstddef>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#define __global__
+#define __device__
+#define __host__
+#define __forceinline__ inline
+#define __restrict__ __restrict
+#define __launch_bounds__(x)
+#define __shared__
+#define __align__(x)
+
+struct uint4 { uint32_t x, y, z, w; };
+struct alignas(8) uint2 { uint32_t x, y; };
+struct float2 { float x, y; };
+struct alignas(16) float4 { float x, y, z, w; };
+inline uint4 make_uint4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) { return {a, b, c, d}; }
+inline float2 make_float2(float a, float b) { return {a, b}; }
+inline float4 make_float4(float a, float b, float c, float d) { return {a, b, c, d}; }
+
+struct Dim3 { unsigned x, y, z; };
+extern thread_local Dim3 threadIdx, blockIdx;
+extern Dim3 blockDim, gridDim;
+
+inline uint4 __ldg(const uint4* p) { return *p; }
+inline float __uint_as_float(uint32_t u) { float f; std::memcpy(&f, &u, 4); return f; }
+
+extern std::barrier<>* g_block_bar;
+extern std::barrier<>* g_warp_bar[32];
+extern float g_xbuf[32][32];
+extern std::mutex g_atomic_mu;
+extern unsigned char* g_smem;
+
+inline void __syncthreads() { g_block_bar->arrive_and_wait(); }
+inline float __shfl_xor_sync(unsigned, float v, int o) {
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  g_xbuf[w][l] = v;
+  g_warp_bar[w]->arrive_and_wait();
+  const float r = g_xbuf[w][l ^ o];
+  g_warp_bar[w]->arrive_and_wait();
+  return r;
+}
+inline int atomicOr(int* p, int v) {
+  std::lock_guard<std::mutex> g(g_atomic_mu);
+  const int old = *p;
+  *p |= v;
+  return old;
+}
+typedef int cudaError_t;
+
+namespace lsi {
+enum : int { FAULT_NONE = 0, FAULT_WAIT_TIMEOUT = 1, FAULT_BAD_INDEX = 2 };
+extern int g_fault;
+}  // namespace lsi
