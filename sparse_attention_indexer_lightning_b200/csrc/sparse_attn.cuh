@@ -8,28 +8,31 @@
 //   logit(s) = scale * q[t,h,:] . c[s,:],   lse = log sum_s exp(logit(s)),
 //   o[t,h,:] = sum_s exp(logit(s) - lse) * c[s,:512]
 //
-// One CTA per (query, group of 8 heads), 256 threads, on the CUDA cores:
+// One CTA per (query, group of 8 heads), 256 threads, on the CUDA cores.  The
+// selection streams through in chunks of 64 slots, each row gathered once
+// (its first 512 elements serve as the value from the same staged copy), with
+// the online-softmax recurrence per head (running max m and sum l; a chunk
+// that raises m rescales what was accumulated by exp(m_old - m_new)):
 //
-//  1. the CTA's row ids (slot -> idx + row offset; -1 or out of range -> none;
-//     out of range is flagged unless the caller holds one shard of the rows)
-//     and its 8 query heads (fp32, [dimension][head]) go to shared memory;
-//  2. logits: the selected rows are staged 64 at a time (a row per 289-word
-//     stride, so 32 consecutive rows start on 32 different banks); warp p
-//     takes dimensions 72p .. 72p + 71 (its query loads are broadcasts) and
-//     its lane g rows g and g + 32, for all 8 heads; the eight partial sums
-//     are added in a fixed order; logits are kept slot-major ([slot][head]);
-//  3. softmax: warp h takes head h: max, exp(logit - max), sum, 1 / sum, lse;
-//  4. values: the value parts are staged again, 64 rows at a time, densely
-//     (256 words a row); thread i of each half owns output columns 4i .. 4i + 3
-//     of all 8 heads, the lower half takes the even rows and the upper half
-//     the odd ones, reading a row's 8 weights as two 16-byte broadcasts; the
-//     two halves' sums are added at the end.
+//  1. the chunk's row ids (slot -> idx + row offset; -1 or out of range ->
+//     none; out of range is flagged unless the caller holds one shard of the
+//     rows), double-buffered so the next chunk's ids and rows can be fetched
+//     while this one is computed;
+//  2. logits: rows staged with a 289-word stride (32 consecutive rows start on
+//     32 different banks); warp p takes dimensions 72p .. 72p + 71 (its query
+//     loads are broadcasts) and its lane g rows g and g + 32, for all 8 heads;
+//     the eight partial sums are added in a fixed order;
+//  3. softmax step, warp h for head h: chunk max, new running max, rescale
+//     factor, weights exp(logit - m), running sum;
+//  4. values: thread i of each half of the CTA owns output columns 2i, 2i + 1,
+//     256 + 2i, 257 + 2i of all 8 heads, rescales them, and adds its parity's
+//     rows (the lower half the even rows, the upper half the odd ones),
+//     reading a row's 8 weights as two 16-byte broadcasts; the halves' sums
+//     meet in shared memory at the end.
 //
-// The selection sits in shared memory in full (k <= 2048 slots), so the
-// softmax is exact in two passes, with no running rescale.  Unused slots
-// stage zeros and weigh 0.  Rows are gathered a chunk ahead into registers
-// (the next chunk's loads are in flight while the current one is computed;
-// the value pass's first chunk while the softmax runs).
+// Rows are gathered a chunk ahead into registers, so the next chunk's loads
+// are in flight while the current one is computed.  Unused slots stage zeros
+// and weigh 0.  Shared memory does not depend on k.
 
 #pragma once
 
@@ -40,32 +43,30 @@ namespace lsi {
 constexpr int kAttnLatent = 576;                    // elements of a latent row (the key)
 constexpr int kAttnValue = 512;                     // leading elements that are the value
 constexpr int kAttnHeads = 8;                       // heads per CTA
-constexpr int kAttnChunk = 64;                      // selected rows staged per pass
+constexpr int kAttnChunk = 64;                      // selected rows staged per step
 constexpr int kAttnThreads = 256;
-constexpr int kAttnMaxK = 2048;
+constexpr int kAttnMaxK = 1 << 16;                  // slots per query (the selection streams through)
 constexpr int kAttnRowWords = kAttnLatent / 2 + 1;  // 289 words: row r starts on bank r mod 32
-constexpr int kAttnParts = kAttnThreads / 32;      // dimension slices, one per warp
+constexpr int kAttnParts = kAttnThreads / 32;       // dimension slices, one per warp
 constexpr int kAttnSlice = kAttnLatent / kAttnParts;  // 72 dimensions per partial dot product
-static_assert(kAttnValue / 4 == kAttnThreads / 2, "four value columns per thread of each half");
-static_assert(kAttnThreads / 2 * 4 * kAttnHeads <= kAttnParts * kAttnHeads * kAttnChunk,
-              "the upper half's sums fit the partial-sum buffer");
-static_assert(kAttnChunk == 64, "a lane scores staged rows g and g + 32");
+constexpr int kAttnHalf = kAttnThreads / 2;         // threads per half (value pass)
+static_assert(kAttnValue / 2 == 2 * kAttnHalf, "two column pairs per thread of each half");
+static_assert(kAttnChunk == 64, "a lane scores staged rows g and g + 32 and the softmax takes two per lane");
 static_assert(kAttnSlice % 2 == 0, "slices of whole bf16 pairs");
-static_assert(kAttnThreads / 32 == kAttnHeads, "one warp per head in the softmax");
-static_assert((kAttnLatent * kAttnHeads + kAttnChunk * kAttnRowWords + kAttnParts * kAttnHeads * kAttnChunk) % 4 == 0,
-              "the weights start on a 16-byte boundary (float4 reads)");
+static_assert(kAttnThreads / 32 == kAttnHeads, "one warp per head in the softmax step");
+static_assert(kAttnHalf * kAttnHeads * 4 <= kAttnParts * kAttnHeads * kAttnChunk,
+              "the upper half's sums fit the partial-sum buffer");
 
-__host__ __device__ constexpr int attn_kpad(int k) { return (k + kAttnChunk - 1) / kAttnChunk * kAttnChunk; }
+// Shared memory layout (4-byte words), fixed for every k.
+constexpr int kAttnOffRows = kAttnLatent * kAttnHeads;                       // query heads [d][h]
+constexpr int kAttnOffPart = kAttnOffRows + kAttnChunk * kAttnRowWords;      // staged rows
+constexpr int kAttnOffW = kAttnOffPart + kAttnParts * kAttnChunk * kAttnHeads;  // partial sums [slice][row][h]
+constexpr int kAttnOffIds = kAttnOffW + kAttnChunk * kAttnHeads;             // chunk logits / weights [row][h]
+constexpr int kAttnOffStat = kAttnOffIds + 2 * kAttnChunk;                   // row ids, two chunks
+constexpr int kAttnWords = kAttnOffStat + 2 * kAttnHeads;                    // rescale factors, 1 / sums
+static_assert(kAttnOffW % 4 == 0 && kAttnOffPart % 4 == 0, "float4 access to the weights and the exchange");
 
-// Dynamic shared memory of one CTA for k slots (4-byte words throughout).
-__host__ __device__ constexpr size_t attn_smem_bytes(int k) {
-  return 4 * (static_cast<size_t>(kAttnLatent) * kAttnHeads      // query heads [d][h]
-              + static_cast<size_t>(kAttnChunk) * kAttnRowWords  // staged rows
-              + kAttnParts * kAttnHeads * kAttnChunk              // partial dot products [slice][row][h]
-              + static_cast<size_t>(kAttnHeads) * attn_kpad(k)    // logits, then weights [slot][h]
-              + attn_kpad(k)                                      // row ids [slot]
-              + kAttnHeads);                                      // 1 / sum of weights [h]
-}
+__host__ __device__ constexpr size_t attn_smem_bytes() { return 4 * static_cast<size_t>(kAttnWords); }
 
 __device__ __forceinline__ float attn_bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float attn_bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -80,42 +81,55 @@ __device__ __forceinline__ float attn_warp_sum(float v) {
   return v;
 }
 
-// One thread's share of a chunk of 64 staged rows, `WORDS` 32-bit words
-// (bf16 pairs) of each, held in registers between the global loads and the
-// shared-memory stores, so that the next chunk's gather is in flight while
-// the current one is computed.
-template <int WORDS>
+// One thread's share of a chunk of 64 rows (the whole 576-element rows), held
+// in registers between the global loads and the shared-memory stores.
 struct AttnChunk {
-  static constexpr int kVecs = WORDS / 4;                               // 16-byte loads per row
+  static constexpr int kVecs = kAttnLatent / 8;                         // 16-byte loads per row
   static constexpr int kPer = kAttnChunk * kVecs / kAttnThreads;        // loads per thread
   static_assert(kAttnChunk * kVecs % kAttnThreads == 0, "whole loads per thread");
   uint4 v[kPer];
 };
 
-// Gather rows of slots c0 .. c0 + 63 (an unused slot gives zeros).
-template <int WORDS>
-__device__ __forceinline__ void attn_fetch(AttnChunk<WORDS>& c, const int32_t* ids, int c0,
-                                           const uint16_t* __restrict__ latent) {
+// Row ids of slots c0 .. c0 + 63 of query t (threads 0..63, one slot each).
+__device__ __forceinline__ void attn_resolve(int32_t* ids, const int32_t* __restrict__ idx, int t, int k, int c0,
+                                             int64_t off, int64_t n_rows, int foreign_ok) {
+  const int i = threadIdx.x;
+  if (i >= kAttnChunk) return;
+  int32_t id = -1;
+  if (c0 + i < k) {
+    const int32_t s = idx[static_cast<int64_t>(t) * k + c0 + i];
+    if (s >= 0) {
+      const int64_t r = off + s;
+      if (r >= 0 && r < n_rows)
+        id = static_cast<int32_t>(r);
+      else if (!foreign_ok)
+        atomicOr(&g_fault, FAULT_BAD_INDEX);          // never read: the slot stays unused
+    }
+  }
+  ids[i] = id;
+}
+
+// Gather the chunk's rows (an unused slot gives zeros).
+__device__ __forceinline__ void attn_fetch(AttnChunk& c, const int32_t* ids, const uint16_t* __restrict__ latent) {
 #pragma unroll
-  for (int m = 0; m < AttnChunk<WORDS>::kPer; ++m) {
+  for (int m = 0; m < AttnChunk::kPer; ++m) {
     const int i = threadIdx.x + m * kAttnThreads;
-    const int r = i / AttnChunk<WORDS>::kVecs;
-    const int v = i - r * AttnChunk<WORDS>::kVecs;
-    const int32_t id = ids[c0 + r];
+    const int r = i / AttnChunk::kVecs;
+    const int v = i - r * AttnChunk::kVecs;
+    const int32_t id = ids[r];
     c.v[m] = make_uint4(0u, 0u, 0u, 0u);
     if (id >= 0) c.v[m] = __ldg(reinterpret_cast<const uint4*>(latent + static_cast<int64_t>(id) * kAttnLatent) + v);
   }
 }
 
-// Store a fetched chunk into shared memory, a row every `stride` words.
-template <int WORDS>
-__device__ __forceinline__ void attn_put(const AttnChunk<WORDS>& c, uint32_t* rows, int stride) {
+// Store a fetched chunk into shared memory, a row every 289 words.
+__device__ __forceinline__ void attn_put(const AttnChunk& c, uint32_t* rows) {
 #pragma unroll
-  for (int m = 0; m < AttnChunk<WORDS>::kPer; ++m) {
+  for (int m = 0; m < AttnChunk::kPer; ++m) {
     const int i = threadIdx.x + m * kAttnThreads;
-    const int r = i / AttnChunk<WORDS>::kVecs;
-    const int v = i - r * AttnChunk<WORDS>::kVecs;
-    uint32_t* dst = rows + r * stride + 4 * v;
+    const int r = i / AttnChunk::kVecs;
+    const int v = i - r * AttnChunk::kVecs;
+    uint32_t* dst = rows + r * kAttnRowWords + 4 * v;
     dst[0] = c.v[m].x;
     dst[1] = c.v[m].y;
     dst[2] = c.v[m].z;
@@ -130,53 +144,53 @@ __global__ void __launch_bounds__(kAttnThreads)
                        int64_t n_rows, float scale, int foreign_ok, float* __restrict__ out,
                        float* __restrict__ lse) {
   extern __shared__ __align__(16) unsigned char attn_smem[];
-  const int kp = attn_kpad(k);
   float* qs = reinterpret_cast<float*>(attn_smem);
-  uint32_t* rows = reinterpret_cast<uint32_t*>(qs + kAttnLatent * kAttnHeads);
-  float* part = reinterpret_cast<float*>(rows + kAttnChunk * kAttnRowWords);
-  float* sc = part + kAttnParts * kAttnHeads * kAttnChunk;
-  int32_t* ids = reinterpret_cast<int32_t*>(sc + kAttnHeads * kp);
-  float* inv_l = reinterpret_cast<float*>(ids + kp);
+  uint32_t* rows = reinterpret_cast<uint32_t*>(qs + kAttnOffRows);
+  float* part = qs + kAttnOffPart;
+  float* wts = qs + kAttnOffW;
+  int32_t* ids = reinterpret_cast<int32_t*>(qs + kAttnOffIds);
+  float* stat = qs + kAttnOffStat;                    // [0, 8): rescale factors, [8, 16): 1 / sums
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int groups = H / kAttnHeads;
   const int t = blockIdx.x / groups;
   const int h0 = (blockIdx.x - t * groups) * kAttnHeads;
   const int64_t off = row_off ? row_off[t] : 0;
+  const int nchunks = (k + kAttnChunk - 1) / kAttnChunk;
 
-  // 1. row ids and query heads
-  for (int i = tid; i < kp; i += kAttnThreads) {
-    int32_t id = -1;
-    if (i < k) {
-      const int32_t s = idx[static_cast<int64_t>(t) * k + i];
-      if (s >= 0) {
-        const int64_t r = off + s;
-        if (r >= 0 && r < n_rows)
-          id = static_cast<int32_t>(r);
-        else if (!foreign_ok)
-          atomicOr(&g_fault, FAULT_BAD_INDEX);      // never read: the slot stays unused
-      }
-    }
-    ids[i] = id;
-  }
   const uint16_t* qt = q + (static_cast<int64_t>(t) * H + h0) * kAttnLatent;
   for (int i = tid; i < kAttnHeads * kAttnLatent; i += kAttnThreads) {
     const int hh = i / kAttnLatent;
     const int d = i - hh * kAttnLatent;
     qs[d * kAttnHeads + hh] = __uint_as_float(static_cast<uint32_t>(qt[i]) << 16);
   }
+  attn_resolve(ids, idx, t, k, 0, off, n_rows, foreign_ok);
   __syncthreads();
+  AttnChunk next;
+  attn_fetch(next, ids, latent);
 
-  // 2. logits
-  const int g = tid & 31;                             // staged rows g and g + 32
-  const int sl = tid >> 5;                            // dimension slice of this warp
-  {
-    AttnChunk<kAttnLatent / 2> next;
-    attn_fetch(next, ids, 0, latent);
-    for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
-      attn_put(next, rows, kAttnRowWords);
-      __syncthreads();
-      if (c0 + kAttnChunk < kp) attn_fetch(next, ids, c0 + kAttnChunk, latent);   // in flight during the math
+  const int g = lane;                                 // logits: staged rows g and g + 32
+  const int sl = warp;                                // logits: this warp's dimension slice
+  const int cg = tid & (kAttnHalf - 1);               // values: columns 2cg, 2cg + 1, 256 + 2cg, 257 + 2cg
+  const int half = tid / kAttnHalf;                   // values: rows of this parity
+  float m_run = -INFINITY;                            // softmax state of head `warp` (same in every lane)
+  float l_run = 0.f;
+  float o[kAttnHeads][4];
+#pragma unroll
+  for (int hh = 0; hh < kAttnHeads; ++hh) o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int32_t* cid = ids + (c & 1) * kAttnChunk;
+    attn_put(next, rows);
+    if (c + 1 < nchunks)
+      attn_resolve(ids + ((c + 1) & 1) * kAttnChunk, idx, t, k, (c + 1) * kAttnChunk, off, n_rows, foreign_ok);
+    __syncthreads();
+    if (c + 1 < nchunks) attn_fetch(next, ids + ((c + 1) & 1) * kAttnChunk, latent);   // in flight during the math
+
+    // 2. logits
+    {
       float a0[kAttnHeads], a1[kAttnHeads];
 #pragma unroll
       for (int hh = 0; hh < kAttnHeads; ++hh) a0[hh] = a1[hh] = 0.f;
@@ -207,64 +221,51 @@ __global__ void __launch_bounds__(kAttnThreads)
         p0[hh] = a0[hh];
         p1[hh] = a1[hh];
       }
-      __syncthreads();
-      for (int i = tid; i < kAttnHeads * kAttnChunk; i += kAttnThreads) {
-        const int j = i / kAttnHeads;
-        const int hh = i - j * kAttnHeads;
-        float s = part[j * kAttnHeads + hh];
-#pragma unroll
-        for (int sp = 1; sp < kAttnParts; ++sp) s += part[(sp * kAttnChunk + j) * kAttnHeads + hh];
-        sc[(c0 + j) * kAttnHeads + hh] = ids[c0 + j] >= 0 ? s * scale : -INFINITY;
-      }
-      __syncthreads();
     }
-  }
-
-  // the value pass's first gather overlaps the softmax
-  constexpr int kValWords = kAttnValue / 2;           // dense staging: row j at word 256 j (8-byte aligned)
-  AttnChunk<kValWords> vnext;
-  attn_fetch(vnext, ids, 0, latent);
-
-  // 3. softmax, one warp per head (kp is a multiple of 32: every lane loops alike)
-  {
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
-    float* sh = sc + warp;                          // head `warp` of slot j at sh[j * 8]
-    float m = -INFINITY;
-    for (int j = lane; j < kp; j += 32) m = fmaxf(m, sh[j * kAttnHeads]);
-    m = attn_warp_max(m);
-    float l = 0.f;
-    for (int j = lane; j < kp; j += 32) {
-      const float x = sh[j * kAttnHeads];
-      const float e = (x == -INFINITY) ? 0.f : expf(x - m);
-      sh[j * kAttnHeads] = e;
-      l += e;
-    }
-    l = attn_warp_sum(l);
-    if (lane == 0) {
-      inv_l[warp] = l > 0.f ? 1.f / l : 0.f;
-      if (lse) lse[static_cast<int64_t>(t) * H + h0 + warp] = l > 0.f ? m + logf(l) : -INFINITY;
-    }
-  }
-  __syncthreads();
-
-  // 4. values
-  const int cg = tid & (kAttnThreads / 2 - 1);        // columns 4 cg .. 4 cg + 3
-  const int half = tid / (kAttnThreads / 2);          // rows of this parity
-  float o[kAttnHeads][4];
-#pragma unroll
-  for (int hh = 0; hh < kAttnHeads; ++hh) o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
-  for (int c0 = 0; c0 < kp; c0 += kAttnChunk) {
-    attn_put(vnext, rows, kValWords);
     __syncthreads();
-    if (c0 + kAttnChunk < kp) attn_fetch(vnext, ids, c0 + kAttnChunk, latent);
+    for (int i = tid; i < kAttnHeads * kAttnChunk; i += kAttnThreads) {
+      const int j = i / kAttnHeads;
+      const int hh = i - j * kAttnHeads;
+      float s = part[j * kAttnHeads + hh];
+#pragma unroll
+      for (int sp = 1; sp < kAttnParts; ++sp) s += part[(sp * kAttnChunk + j) * kAttnHeads + hh];
+      wts[j * kAttnHeads + hh] = cid[j] >= 0 ? s * scale : -INFINITY;
+    }
+    __syncthreads();
+
+    // 3. softmax step for head `warp` (every lane takes slots lane and lane + 32)
+    {
+      const float x0 = wts[lane * kAttnHeads + warp];
+      const float x1 = wts[(lane + 32) * kAttnHeads + warp];
+      const float m_new = fmaxf(m_run, attn_warp_max(fmaxf(x0, x1)));
+      const float alpha = (m_new == -INFINITY) ? 1.f : expf(m_run - m_new);   // exp(-inf) = 0 on the first rows
+      const float e0 = (x0 == -INFINITY) ? 0.f : expf(x0 - m_new);
+      const float e1 = (x1 == -INFINITY) ? 0.f : expf(x1 - m_new);
+      wts[lane * kAttnHeads + warp] = e0;
+      wts[(lane + 32) * kAttnHeads + warp] = e1;
+      l_run = l_run * alpha + attn_warp_sum(e0 + e1);
+      m_run = m_new;
+      if (lane == 0) stat[warp] = alpha;
+    }
+    __syncthreads();
+
+    // 4. values
+#pragma unroll
+    for (int hh = 0; hh < kAttnHeads; ++hh) {
+      const float al = stat[hh];
+      o[hh][0] *= al;
+      o[hh][1] *= al;
+      o[hh][2] *= al;
+      o[hh][3] *= al;
+    }
     for (int j = half; j < kAttnChunk; j += 2) {
-      const uint2 x = *reinterpret_cast<const uint2*>(rows + j * kValWords + 2 * cg);
-      const float v0 = attn_bf16_lo(x.x);
-      const float v1 = attn_bf16_hi(x.x);
-      const float v2 = attn_bf16_lo(x.y);
-      const float v3 = attn_bf16_hi(x.y);
-      const float4* pj = reinterpret_cast<const float4*>(sc + (c0 + j) * kAttnHeads);   // 32-byte aligned
+      const uint32_t xa = rows[j * kAttnRowWords + cg];
+      const uint32_t xb = rows[j * kAttnRowWords + kAttnHalf + cg];
+      const float v0 = attn_bf16_lo(xa);
+      const float v1 = attn_bf16_hi(xa);
+      const float v2 = attn_bf16_lo(xb);
+      const float v3 = attn_bf16_hi(xb);
+      const float4* pj = reinterpret_cast<const float4*>(wts + j * kAttnHeads);   // 32-byte aligned
       const float4 pa = pj[0];
       const float4 pb = pj[1];
       const float p[kAttnHeads] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
@@ -276,24 +277,30 @@ __global__ void __launch_bounds__(kAttnThreads)
         o[hh][3] = fmaf(p[hh], v3, o[hh][3]);
       }
     }
-    __syncthreads();
+    __syncthreads();                                  // rows, weights and factors are rewritten next chunk
   }
-  // the odd rows' sums go through shared memory (the partial-sum buffer is free) to the even rows' threads
+
+  if (lane == 0) {
+    stat[kAttnHeads + warp] = l_run > 0.f ? 1.f / l_run : 0.f;
+    if (lse) lse[static_cast<int64_t>(t) * H + h0 + warp] = l_run > 0.f ? m_run + logf(l_run) : -INFINITY;
+  }
+  // the upper half's sums go through shared memory (the partial-sum buffer is free) to the lower half
   float4* xfer = reinterpret_cast<float4*>(part) + cg;   // head hh at xfer[hh * 128]
   if (half == 1) {
 #pragma unroll
     for (int hh = 0; hh < kAttnHeads; ++hh)
-      xfer[hh * (kAttnThreads / 2)] = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
+      xfer[hh * kAttnHalf] = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
   }
   __syncthreads();
   if (half == 0) {
 #pragma unroll
     for (int hh = 0; hh < kAttnHeads; ++hh) {
-      const float4 u = xfer[hh * (kAttnThreads / 2)];
-      const float il = inv_l[hh];
-      float* dst = out + (static_cast<int64_t>(t) * H + h0 + hh) * kAttnValue + 4 * cg;
-      *reinterpret_cast<float4*>(dst) =
-          make_float4((o[hh][0] + u.x) * il, (o[hh][1] + u.y) * il, (o[hh][2] + u.z) * il, (o[hh][3] + u.w) * il);
+      const float4 u = xfer[hh * kAttnHalf];
+      const float il = stat[kAttnHeads + hh];
+      float* dst = out + (static_cast<int64_t>(t) * H + h0 + hh) * kAttnValue;
+      *reinterpret_cast<float2*>(dst + 2 * cg) = make_float2((o[hh][0] + u.x) * il, (o[hh][1] + u.y) * il);
+      *reinterpret_cast<float2*>(dst + 2 * kAttnHalf + 2 * cg) =
+          make_float2((o[hh][2] + u.z) * il, (o[hh][3] + u.w) * il);
     }
   }
 }
@@ -302,7 +309,7 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint16_t* latent, const 
                                int T, int H, int k, int64_t n_rows, float scale, int foreign_ok, float* out, float* lse,
                                cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const size_t smem = attn_smem_bytes(k);
+  const size_t smem = attn_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

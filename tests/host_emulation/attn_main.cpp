@@ -51,7 +51,7 @@ static int run_attn(char** a) {
   std::vector<int64_t> off;
   if (has_off) off = load<int64_t>(dir, "off.bin", T);
   std::vector<float> out(static_cast<size_t>(T) * H * 512, 12345.f), lse(static_cast<size_t>(T) * H, 12345.f);
-  const size_t smem = lsi::attn_smem_bytes(k);
+  const size_t smem = lsi::attn_smem_bytes();
   std::vector<unsigned char> smem_buf(smem);
   g_smem = smem_buf.data();
   const int blocks = T * (H / 8);

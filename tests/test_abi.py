@@ -141,7 +141,7 @@ def test_argument_checks_without_gpu(lib):
     att = lib.ls_sparse_attention
     assert att(dummy, dummy, dummy, None, 4, 128, 128, 512, 1000, 512, 0.04, 0, dummy, None, None) == 3
     assert att(dummy, dummy, dummy, None, 4, 12, 576, 512, 1000, 512, 0.04, 0, dummy, None, None) == 1
-    assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 4096, 0.04, 0, dummy, None, None) == 1
+    assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 100000, 0.04, 0, dummy, None, None) == 1
     assert att(P(8), dummy, dummy, None, 4, 128, 576, 512, 1000, 512, 0.04, 0, dummy, None, None) == 1
     assert att(dummy, dummy, dummy, None, 4, 128, 576, 512, 1000, 512, float("nan"), 0, dummy, None, None) == 1
     assert att(None, None, None, None, 0, 128, 576, 512, 1000, 512, 0.04, 0, None, None, None) == 0

@@ -129,9 +129,9 @@ def test_host_kernel_row_offsets_bad_rows_and_shards(runner):
     _compare(out, lse, d["q"], d["latent"][base:base + length], local, default_scale())
 
 
-def test_host_kernel_largest_k_and_many_heads(runner):
+def test_host_kernel_long_selections_and_many_heads(runner):
     attn, _ = runner
-    for T, H, N, k in ((1, 8, 5000, 2048), (1, 24, 3000, 130)):
+    for T, H, N, k in ((1, 8, 5000, 2048), (1, 24, 3000, 130), (1, 8, 6000, 4612)):
         d = make_attention(T, H, N, k, seed=k)
         out, lse, fault = attn(d["q"], d["latent"], d["idx"], default_scale())
         assert fault == 0

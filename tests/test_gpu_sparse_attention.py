@@ -3,7 +3,8 @@
 Tolerance, from the arithmetic: each logit is an fp32 sum of 576 exact
 products of bf16 values (relative error a few 1e-7 of the sum of magnitudes),
 the weights come from fp32 exp and one division (a few ulp), and each output
-is an fp32 weighted sum of at most 2048 bf16 values.  Every error term is
+is an fp32 weighted sum of at most a few thousand bf16 values (with the
+online rescaling, one more rounding per chunk of 64).  Every error term is
 below 1e-5 of the largest value magnitude among the selected rows for these
 inputs (logits of standard deviation about 2), so the bound checked is
 |o - o_ref| <= 1e-4 * max |value| of the query's selected rows and
@@ -84,9 +85,10 @@ def test_sparse_attention_small(L):
 
 
 def test_sparse_attention_shapes(L):
-    """k = 1, k = 1000 with a larger scale, the largest k (2048), many heads."""
+    """k = 1, k = 1000 with a larger scale, k = 2048 and 4612 (the LSA read
+    list: 4 sinks, a 512-key window, 4096 long-range keys), many heads."""
     for T, H, N, k, scale in ((3, 8, 100, 1, 0.5), (2, 8, 5000, 1000, 0.2), (2, 8, 5000, 2048, None),
-                              (2, 128, 5000, 512, None), (1, 24, 700, 130, 0.05)):
+                              (2, 8, 9000, 4612, None), (2, 128, 5000, 512, None), (1, 24, 700, 130, 0.05)):
         d = make_attention(T, H, N, k, seed=T * 1000 + k)
         out, lse = _run(L, d, scale=scale)
         _check(out, lse, d["q"], d["latent"], d["idx"], default_scale() if scale is None else scale,
@@ -197,6 +199,27 @@ def test_sparse_attention_after_decode_selection(L):
     assert np.all((sel >= 0).sum(axis=1) == np.minimum(dd["n_valid"], wl.k))
     g = np.where(sel >= 0, sel + off[:, None], -1)
     _check(out.cpu().numpy(), lse.cpu().numpy(), att["q"], att["latent"], g, default_scale(), what="chained")
+
+
+def test_sparse_attention_over_lsa_read_lists(L):
+    """The LSA flat search's read lists (sinks, the window, the long-range
+    keys of the picked buckets, -1 after the row's count) fed as is to the
+    sparse attention over a latent cache of the sequence's tokens."""
+    wl = get_workload("lsa_flat_s")
+    d = data("lsa_flat_s")
+    ex = wl.extra
+    keys, n = L.ls_lsa_flat_select(dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]),
+                                   dev(d["bucket_off"]), dev(d["bucket_mem"]), block_keys=ex["block_keys"],
+                                   buckets_per_block=ex["bpb"], n_sink=ex["n_sink"], top_p=wl.top_p,
+                                   budget=wl.budget)[:2]
+    T = keys.shape[0]
+    att = make_attention(T, 16, wl.N, 1, seed=31)
+    out, lse = L.ls_sparse_attention(dev_bf16(att["q"]), dev_bf16(att["latent"]), keys)
+    torch.cuda.synchronize()
+    sel = keys.cpu().numpy()
+    nn = n.cpu().numpy()
+    assert np.all((sel >= 0).sum(axis=1) == nn) and nn.max() > ex["n_sink"]
+    _check(out.cpu().numpy(), lse.cpu().numpy(), att["q"], att["latent"], sel, default_scale(), what="lsa")
 
 
 @pytest.mark.slow
