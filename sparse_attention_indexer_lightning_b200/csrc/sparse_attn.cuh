@@ -57,13 +57,19 @@ static_assert(kAttnThreads / 32 == kAttnHeads, "one warp per head in the softmax
 static_assert(kAttnHalf * kAttnHeads * 4 <= kAttnParts * kAttnHeads * kAttnChunk,
               "the upper half's sums fit the partial-sum buffer");
 
-// Shared memory layout (4-byte words), fixed for every k.
-constexpr int kAttnOffRows = kAttnLatent * kAttnHeads;                       // query heads [d][h]
-constexpr int kAttnOffPart = kAttnOffRows + kAttnChunk * kAttnRowWords;      // staged rows
-constexpr int kAttnOffW = kAttnOffPart + kAttnParts * kAttnChunk * kAttnHeads;  // partial sums [slice][row][h]
-constexpr int kAttnOffIds = kAttnOffW + kAttnChunk * kAttnHeads;             // chunk logits / weights [row][h]
-constexpr int kAttnOffStat = kAttnOffIds + 2 * kAttnChunk;                   // row ids, two chunks
-constexpr int kAttnWords = kAttnOffStat + 2 * kAttnHeads;                    // rescale factors, 1 / sums
+// Shared memory layout in 4-byte words, the same for every k:
+//   [0, OffRows)         query heads, fp32 [d][h]
+//   [OffRows, OffPart)   staged rows, 289 words each
+//   [OffPart, OffW)      partial sums [slice][row][h], at the end the halves' exchange
+//   [OffW, OffIds)       the chunk's logits, then its weights [row][h]
+//   [OffIds, OffStat)    row ids of two chunks
+//   [OffStat, Words)     rescale factors [h], then 1 / sums [h]
+constexpr int kAttnOffRows = kAttnLatent * kAttnHeads;
+constexpr int kAttnOffPart = kAttnOffRows + kAttnChunk * kAttnRowWords;
+constexpr int kAttnOffW = kAttnOffPart + kAttnParts * kAttnChunk * kAttnHeads;
+constexpr int kAttnOffIds = kAttnOffW + kAttnChunk * kAttnHeads;
+constexpr int kAttnOffStat = kAttnOffIds + 2 * kAttnChunk;
+constexpr int kAttnWords = kAttnOffStat + 2 * kAttnHeads;
 static_assert(kAttnOffW % 4 == 0 && kAttnOffPart % 4 == 0, "float4 access to the weights and the exchange");
 
 __host__ __device__ constexpr size_t attn_smem_bytes() { return 4 * static_cast<size_t>(kAttnWords); }
