@@ -294,18 +294,13 @@ def test_prefill_chunk_full_size_sampled(L):
         check_selection(idx[t], val[t], np.arange(n), ref, wl.k, RTOL_BF16, f"prefill t={t}")
 
 
-def test_prefill_sharded_history_merge(L):
-    """A history split into S contiguous shards (one per GPU in a sharded
-    prefill): each shard's selection for the same queries, positions shifted
-    so the causal rule holds per shard, merged by ls_merge_select, equals the
-    selection over the whole history bit for bit."""
-    wl = get_workload("prefill_s")
-    d = data("prefill_s")
-    T, H, dd = d["q"].shape
+def _sharded_prefill_matches(L, name, shard_counts):
+    wl = get_workload(name)
+    d = data(name)
     N = d["k"].shape[0]
     q, w, qp = dev_bf16(d["q"]), dev(d["w"]), dev(d["q_pos"])
     _, _, _, idx0, val0 = _prefill_run(L, d, wl)
-    for S in (2, 3):
+    for S in shard_counts:
         vals, idxs, offs = [], [], []
         for base, length in L.shard_plan(N, S):
             hist = torch.from_numpy(d["k"][base:base + length].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -319,8 +314,24 @@ def test_prefill_sharded_history_merge(L):
         mi, mv = L.ls_merge_select(torch.stack(vals), torch.stack(idxs), dev(np.asarray(offs, dtype=np.int32)),
                                    k=wl.k)
         torch.cuda.synchronize()
-        assert np.array_equal(mi.cpu().numpy(), idx0), S
-        assert f32_bits_equal(mv.cpu().numpy(), val0), S
+        assert np.array_equal(mi.cpu().numpy(), idx0), (name, S)
+        assert f32_bits_equal(mv.cpu().numpy(), val0), (name, S)
+
+
+def test_prefill_sharded_history_merge(L):
+    """A history split into S contiguous shards (one per GPU in a sharded
+    prefill): each shard's selection for the same queries, positions shifted
+    so the causal rule holds per shard, merged by ls_merge_select, equals the
+    selection over the whole history bit for bit."""
+    _sharded_prefill_matches(L, "prefill_s", (2, 3))
+
+
+@pytest.mark.slow
+def test_prefill_sharded_history_merge_full_size(L):
+    """The 4096-query prefill chunk over 32768 keys in 4 and 3 history shards
+    (one 8192-key tile each, and ragged shards) merges to the unsharded
+    selection bit for bit."""
+    _sharded_prefill_matches(L, "prefill_chunk", (4, 3))
 
 
 def test_merge_select_edge_cases(L):
