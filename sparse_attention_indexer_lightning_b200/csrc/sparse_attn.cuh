@@ -77,6 +77,12 @@ __host__ __device__ constexpr size_t attn_smem_bytes() { return 4 * static_cast<
 __device__ __forceinline__ float attn_bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float attn_bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// acc = a * b + acc on both fp32 halves of the pairs: two fused multiply-adds,
+// each rounded once (the packed form halves the FMA instructions issued).
+__device__ __forceinline__ void attn_fma2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
 __device__ __forceinline__ float attn_warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
@@ -183,9 +189,9 @@ __global__ void __launch_bounds__(kAttnThreads)
   const int half = tid / kAttnHalf;                   // values: rows of this parity
   float m_run = -INFINITY;                            // softmax state of head `warp` (same in every lane)
   float l_run = 0.f;
-  float o[kAttnHeads][4];
+  uint64_t o[kAttnHeads / 2][4];                      // head pair (2i, 2i + 1) of this thread's 4 columns
 #pragma unroll
-  for (int hh = 0; hh < kAttnHeads; ++hh) o[hh][0] = o[hh][1] = o[hh][2] = o[hh][3] = 0.f;
+  for (int i = 0; i < kAttnHeads / 2; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0ull;
 
   for (int c = 0; c < nchunks; ++c) {
     const int32_t* cid = ids + (c & 1) * kAttnChunk;
@@ -195,37 +201,39 @@ __global__ void __launch_bounds__(kAttnThreads)
     __syncthreads();
     if (c + 1 < nchunks) attn_fetch(next, ids + ((c + 1) & 1) * kAttnChunk, latent);   // in flight during the math
 
-    // 2. logits
+    // 2. logits (accumulators hold the head pairs (2i, 2i + 1) of rows g and g + 32)
     {
-      float a0[kAttnHeads], a1[kAttnHeads];
+      uint64_t a0[kAttnHeads / 2], a1[kAttnHeads / 2];
 #pragma unroll
-      for (int hh = 0; hh < kAttnHeads; ++hh) a0[hh] = a1[hh] = 0.f;
+      for (int i = 0; i < kAttnHeads / 2; ++i) a0[i] = a1[i] = 0ull;
       const uint32_t* r0 = rows + g * kAttnRowWords + sl * (kAttnSlice / 2);
       const uint32_t* r1 = r0 + 32 * kAttnRowWords;
-      const float* qq = qs + sl * kAttnSlice * kAttnHeads;
+      const uint64_t* qq = reinterpret_cast<const uint64_t*>(qs + sl * kAttnSlice * kAttnHeads);
 #pragma unroll 2
       for (int w = 0; w < kAttnSlice / 2; ++w) {
         const uint32_t x = r0[w];
         const uint32_t y = r1[w];
-        const float x0 = attn_bf16_lo(x);
-        const float x1 = attn_bf16_hi(x);
-        const float y0 = attn_bf16_lo(y);
-        const float y1 = attn_bf16_hi(y);
-        const float* q0 = qq + 2 * w * kAttnHeads;
+        const uint64_t x0 = pack_f32x2(attn_bf16_lo(x), attn_bf16_lo(x));
+        const uint64_t x1 = pack_f32x2(attn_bf16_hi(x), attn_bf16_hi(x));
+        const uint64_t y0 = pack_f32x2(attn_bf16_lo(y), attn_bf16_lo(y));
+        const uint64_t y1 = pack_f32x2(attn_bf16_hi(y), attn_bf16_hi(y));
+        const uint64_t* q0 = qq + w * kAttnHeads;       // dimension 2w: 4 head pairs, then dimension 2w + 1
 #pragma unroll
-        for (int hh = 0; hh < kAttnHeads; ++hh) {
-          const float qa = q0[hh];
-          const float qb = q0[kAttnHeads + hh];
-          a0[hh] = fmaf(x1, qb, fmaf(x0, qa, a0[hh]));
-          a1[hh] = fmaf(y1, qb, fmaf(y0, qa, a1[hh]));
+        for (int i = 0; i < kAttnHeads / 2; ++i) {
+          const uint64_t qa = q0[i];
+          const uint64_t qb = q0[kAttnHeads / 2 + i];
+          attn_fma2(a0[i], qa, x0);
+          attn_fma2(a0[i], qb, x1);
+          attn_fma2(a1[i], qa, y0);
+          attn_fma2(a1[i], qb, y1);
         }
       }
       float* p0 = part + (sl * kAttnChunk + g) * kAttnHeads;
       float* p1 = p0 + 32 * kAttnHeads;
 #pragma unroll
-      for (int hh = 0; hh < kAttnHeads; ++hh) {
-        p0[hh] = a0[hh];
-        p1[hh] = a1[hh];
+      for (int i = 0; i < kAttnHeads / 2; ++i) {
+        unpack_f32x2(a0[i], p0[2 * i], p0[2 * i + 1]);
+        unpack_f32x2(a1[i], p1[2 * i], p1[2 * i + 1]);
       }
     }
     __syncthreads();
@@ -257,30 +265,31 @@ __global__ void __launch_bounds__(kAttnThreads)
 
     // 4. values
 #pragma unroll
-    for (int hh = 0; hh < kAttnHeads; ++hh) {
-      const float al = stat[hh];
-      o[hh][0] *= al;
-      o[hh][1] *= al;
-      o[hh][2] *= al;
-      o[hh][3] *= al;
+    for (int i = 0; i < kAttnHeads / 2; ++i) {
+      const float al0 = stat[2 * i];
+      const float al1 = stat[2 * i + 1];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float lo, hi;
+        unpack_f32x2(o[i][cc], lo, hi);
+        o[i][cc] = pack_f32x2(lo * al0, hi * al1);
+      }
     }
     for (int j = half; j < kAttnChunk; j += 2) {
       const uint32_t xa = rows[j * kAttnRowWords + cg];
       const uint32_t xb = rows[j * kAttnRowWords + kAttnHalf + cg];
-      const float v0 = attn_bf16_lo(xa);
-      const float v1 = attn_bf16_hi(xa);
-      const float v2 = attn_bf16_lo(xb);
-      const float v3 = attn_bf16_hi(xb);
-      const float4* pj = reinterpret_cast<const float4*>(wts + j * kAttnHeads);   // 32-byte aligned
-      const float4 pa = pj[0];
-      const float4 pb = pj[1];
-      const float p[kAttnHeads] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+      const uint64_t v[4] = {pack_f32x2(attn_bf16_lo(xa), attn_bf16_lo(xa)),
+                             pack_f32x2(attn_bf16_hi(xa), attn_bf16_hi(xa)),
+                             pack_f32x2(attn_bf16_lo(xb), attn_bf16_lo(xb)),
+                             pack_f32x2(attn_bf16_hi(xb), attn_bf16_hi(xb))};
+      const ulonglong2* pj = reinterpret_cast<const ulonglong2*>(wts + j * kAttnHeads);   // 32-byte aligned
+      const ulonglong2 pa = pj[0];                    // head pairs (0, 1) and (2, 3)
+      const ulonglong2 pb = pj[1];                    // head pairs (4, 5) and (6, 7)
+      const uint64_t p[kAttnHeads / 2] = {pa.x, pa.y, pb.x, pb.y};
 #pragma unroll
-      for (int hh = 0; hh < kAttnHeads; ++hh) {
-        o[hh][0] = fmaf(p[hh], v0, o[hh][0]);
-        o[hh][1] = fmaf(p[hh], v1, o[hh][1]);
-        o[hh][2] = fmaf(p[hh], v2, o[hh][2]);
-        o[hh][3] = fmaf(p[hh], v3, o[hh][3]);
+      for (int i = 0; i < kAttnHeads / 2; ++i) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) attn_fma2(o[i][cc], p[i], v[cc]);
       }
     }
     __syncthreads();                                  // rows, weights and factors are rewritten next chunk
@@ -291,11 +300,17 @@ __global__ void __launch_bounds__(kAttnThreads)
     if (lse) lse[static_cast<int64_t>(t) * H + h0 + warp] = l_run > 0.f ? m_run + logf(l_run) : -INFINITY;
   }
   // the upper half's sums go through shared memory (the partial-sum buffer is free) to the lower half
+  float oh[kAttnHeads][4];                            // the pairs split per head
+#pragma unroll
+  for (int i = 0; i < kAttnHeads / 2; ++i) {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) unpack_f32x2(o[i][cc], oh[2 * i][cc], oh[2 * i + 1][cc]);
+  }
   float4* xfer = reinterpret_cast<float4*>(part) + cg;   // head hh at xfer[hh * 128]
   if (half == 1) {
 #pragma unroll
     for (int hh = 0; hh < kAttnHeads; ++hh)
-      xfer[hh * kAttnHalf] = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
+      xfer[hh * kAttnHalf] = make_float4(oh[hh][0], oh[hh][1], oh[hh][2], oh[hh][3]);
   }
   __syncthreads();
   if (half == 0) {
@@ -304,9 +319,9 @@ __global__ void __launch_bounds__(kAttnThreads)
       const float4 u = xfer[hh * kAttnHalf];
       const float il = stat[kAttnHeads + hh];
       float* dst = out + (static_cast<int64_t>(t) * H + h0 + hh) * kAttnValue;
-      *reinterpret_cast<float2*>(dst + 2 * cg) = make_float2((o[hh][0] + u.x) * il, (o[hh][1] + u.y) * il);
+      *reinterpret_cast<float2*>(dst + 2 * cg) = make_float2((oh[hh][0] + u.x) * il, (oh[hh][1] + u.y) * il);
       *reinterpret_cast<float2*>(dst + 2 * kAttnHalf + 2 * cg) =
-          make_float2((o[hh][2] + u.z) * il, (o[hh][3] + u.w) * il);
+          make_float2((oh[hh][2] + u.z) * il, (oh[hh][3] + u.w) * il);
     }
   }
 }

@@ -25,6 +25,7 @@ struct uint4 { uint32_t x, y, z, w; };
 struct alignas(8) uint2 { uint32_t x, y; };
 struct float2 { float x, y; };
 struct alignas(16) float4 { float x, y, z, w; };
+struct alignas(16) ulonglong2 { unsigned long long x, y; };
 inline uint4 make_uint4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) { return {a, b, c, d}; }
 inline float2 make_float2(float a, float b) { return {a, b}; }
 inline float4 make_float4(float a, float b, float c, float d) { return {a, b, c, d}; }
@@ -59,7 +60,31 @@ inline int atomicOr(int* p, int v) {
 }
 typedef int cudaError_t;
 
+// fma.rn.f32x2: a correctly rounded fused multiply-add on each fp32 half
+inline uint64_t host_fma2(uint64_t acc, uint64_t a, uint64_t b) {
+  float c[2], x[2], y[2];
+  std::memcpy(c, &acc, 8);
+  std::memcpy(x, &a, 8);
+  std::memcpy(y, &b, 8);
+  c[0] = std::fma(x[0], y[0], c[0]);
+  c[1] = std::fma(x[1], y[1], c[1]);
+  std::memcpy(&acc, c, 8);
+  return acc;
+}
+
 namespace lsi {
 enum : int { FAULT_NONE = 0, FAULT_WAIT_TIMEOUT = 1, FAULT_BAD_INDEX = 2 };
 extern int g_fault;
+inline uint64_t pack_f32x2(float lo, float hi) {   // low half first, as mov.b64 {lo, hi}
+  const float v[2] = {lo, hi};
+  uint64_t r;
+  std::memcpy(&r, v, 8);
+  return r;
+}
+inline void unpack_f32x2(uint64_t r, float& lo, float& hi) {
+  float v[2];
+  std::memcpy(v, &r, 8);
+  lo = v[0];
+  hi = v[1];
+}
 }  // namespace lsi

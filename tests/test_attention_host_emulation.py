@@ -1,7 +1,8 @@
 """The attention kernels' own source, compiled for the host and checked against the oracle (no GPU).
 
-`csrc/sparse_attn.cuh` is preprocessed (launchers removed, the CUDA features
-it uses supplied by `host_emulation/cuda_shim.h`) and built with g++ under
+`csrc/sparse_attn.cuh` is preprocessed (launchers removed, its one packed-FMA
+instruction mapped to two correctly rounded fused multiply-adds, the CUDA
+features it uses supplied by `host_emulation/cuda_shim.h`) and built with g++ under
 AddressSanitizer; each CUDA thread of a block runs as an OS thread, with real
 barriers for `__syncthreads` and the warp shuffles.  This checks the kernels'
 index arithmetic, staging, barriers, softmax and combine on every CPU run,
@@ -33,7 +34,10 @@ def _host_source(src: str) -> str:
     src = re.sub(r"cudaError_t launch_\w+\(.*?\n}\n", "", src, flags=re.S)
     src = src.replace("extern __shared__ __align__(16) unsigned char attn_smem[];",
                       "unsigned char* attn_smem = ::g_smem;")
-    assert "<<<" not in src and "attn_smem = ::g_smem" in src
+    fma2 = 'asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));'
+    assert fma2 in src
+    src = src.replace(fma2, "acc = host_fma2(acc, a, b);")
+    assert "<<<" not in src and "asm(" not in src and "attn_smem = ::g_smem" in src
     return src
 
 
