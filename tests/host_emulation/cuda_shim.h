@@ -3,7 +3,9 @@
 // tests: one OS thread per CUDA thread of a block, std::barrier for
 // __syncthreads and for the two halves of a warp shuffle, a mutex for atomics.
 // Shared memory is a buffer of the launch's dynamic size (AddressSanitizer
-// sees its end).  Test infrastructure only.
+// sees its end); a kernel's static __shared__ variables become static locals,
+// shared by the threads of the one block that runs at a time.  Test
+// infrastructure only.
 #pragma once
 #include <barrier>
 #include <cmath>
@@ -51,6 +53,12 @@ inline float __shfl_xor_sync(unsigned, float v, int o) {
   const float r = g_xbuf[w][l ^ o];
   g_warp_bar[w]->arrive_and_wait();
   return r;
+}
+inline int atomicMin(int* p, int v) {
+  std::lock_guard<std::mutex> g(g_atomic_mu);
+  const int old = *p;
+  if (v < old) *p = v;
+  return old;
 }
 inline int atomicOr(int* p, int v) {
   std::lock_guard<std::mutex> g(g_atomic_mu);
