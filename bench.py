@@ -8,9 +8,11 @@ One step is one decode selection over the batch workload: 64 sequences x
 exact top-512 per sequence -- the scan (ls_indexer_score) then the selection
 (ls_topk_select).  Inputs (537 MB of keys) are larger than the 126 MB L2, so
 no flush is needed between steps.  The metric is query-positions scored per
-second (selections per second alongside).  The prefill, two-stage and bucket
-searches are timed the same way and reported under "variants", each with the
-roofline of its dominant kernel.
+second (selections per second alongside).  The prefill, two-stage, bucket
+and LSA searches, and the sparse attention that follows a decode selection
+(`attn_decode`, last; an error there is recorded in its own entry), are
+timed the same way and reported under "variants", each with the roofline of
+its dominant kernel.
 
 With N > 1 (torchrun) every rank runs its own batch (weak scaling, no
 collective on the data path); the reported time is the max over ranks.
