@@ -358,10 +358,11 @@ def bench_variants(L, args, peaks, peak_kind, only=None):
                      ("lsa_flat_threshold", lambda *a: bench_lsa(*a, threshold=True)), ("lsa_tree", bench_lsa_tree),
                      ("two_stage", bench_two_stage),
                      ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True)),
+                     ("prefill_shard_merge", bench_shard_merge),
                      ("attn_decode", bench_attention)):
         if only in (None, name):
-            if name == "attn_decode" and only is None:
-                try:                       # the newest path: an error here must not lose the lines above
+            if name in ("prefill_shard_merge", "attn_decode") and only is None:
+                try:                       # the newest paths: an error here must not lose the lines above
                     res[name] = fn(L, args, peaks, peak_kind)
                 except Exception as e:     # noqa: BLE001
                     res[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
@@ -608,6 +609,58 @@ def bench_lsa_tree(L, args, peaks, peak_kind):
     return res
 
 
+def bench_shard_merge(L, args, peaks, peak_kind, shards: int = 4):
+    """Combine step of a history-sharded prefill: the prefill chunk's history
+    in 4 contiguous shards, each shard's top-512 lists computed once outside
+    the timed region, then ls_merge_select (pack the valid prefixes with the
+    shards' first positions, exact top-512 of 4 x 512 candidates per query)
+    timed per step."""
+    import torch
+    from sparse_attention_indexer_lightning_b200 import shard_plan
+    from workloads import get_workload, make_workload
+    st = torch.cuda.current_stream()
+    steps = max(3, args.steps)
+    warm = max(3, args.warmup)
+    wl = get_workload("prefill_chunk")
+    d = make_workload(wl)
+    T = d["q"].shape[0]
+    N = d["k"].shape[0]
+    q, w, qp = to_dev_bf16(d["q"]), to_dev(d["w"]), to_dev(d["q_pos"])
+    vals, idxs, offs = [], [], []
+    for base, length in shard_plan(N, shards):
+        hist = torch.from_numpy(np.ascontiguousarray(d["k"][base:base + length]).view(np.int16)).view(
+            torch.bfloat16).pin_memory()
+        buf0 = torch.empty((wl.tile_keys, 128), dtype=torch.bfloat16, device="cuda")
+        buf1 = torch.empty_like(buf0)
+        i_s, v_s = L.ls_prefill_select_stream(q, w, qp - base * wl.stride, hist, buf0, buf1, k=wl.k,
+                                              stride=wl.stride, tile_keys=wl.tile_keys)
+        vals.append(v_s)
+        idxs.append(i_s)
+        offs.append(base)
+    vals, idxs = torch.stack(vals), torch.stack(idxs)
+    offs = to_dev(np.asarray(offs, dtype=np.int32))
+    ws = torch.empty(L.lib().ls_merge_select_workspace_size(shards, T, wl.k), dtype=torch.uint8, device="cuda")
+    out = (torch.empty((T, wl.k), dtype=torch.int32, device="cuda"),
+           torch.empty((T, wl.k), dtype=torch.float32, device="cuda"))
+
+    def run(i, timed):
+        L.ls_merge_select(vals, idxs, offs, k=wl.k, ws=ws, out=out)
+        return None
+
+    ms, kern = _profiled_loop(L, run, steps, warm, st)
+    tk = kern["topk_kernel"]["ms_per_step"]
+    cand = shards * T * wl.k
+    peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    res = {"ms_per_step": ms, "selections_per_s": T / (ms * 1e-3), "candidates_per_s": cand / (ms * 1e-3),
+           "kernels": kern,
+           "roofline": roofline("hbm", (cand * 8 + T * wl.k * 8) / (tk * 1e-3) / 1e9, peak_b, "GB/s",
+                                peak_kind=peak_kind),
+           "note": "top-k of the packed candidates: 8 bytes per candidate read (value, position) and 8 per "
+                   "selected entry written; the shards' own selections are outside the timed region"}
+    del vals, idxs, ws, out
+    return res
+
+
 # fp32 FMA issue rate of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz (clocks.max.sm)
 ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
@@ -777,7 +830,7 @@ def main(argv=None):
     ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "prefill_chunk_fp8",
                                                      "prefill_chunk_fp8_running", "bucket", "lsa_flat",
                                                      "lsa_flat_threshold", "lsa_tree", "two_stage",
-                                                     "two_stage_pq", "attn_decode"],
+                                                     "two_stage_pq", "prefill_shard_merge", "attn_decode"],
                     help="time one variant only and skip the decode line (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -54,8 +54,8 @@ def test_digest_covers_the_kernel_sources():
 
 def test_attention_line_error_keeps_the_other_lines(monkeypatch):
     """The attention line runs last and an exception there is recorded in its
-    own entry; the variants before it are kept."""
-    names = ["bench_prefill", "bench_bucket", "bench_lsa", "bench_lsa_tree", "bench_two_stage"]
+    own entry; the variants before it (the shard merge just before) are kept."""
+    names = ["bench_prefill", "bench_bucket", "bench_lsa", "bench_lsa_tree", "bench_two_stage", "bench_shard_merge"]
     for n in names:
         monkeypatch.setattr(bench, n, lambda *a, **k: {"ms_per_step": 1.0})
 
@@ -64,7 +64,8 @@ def test_attention_line_error_keeps_the_other_lines(monkeypatch):
 
     monkeypatch.setattr(bench, "bench_attention", boom)
     res = bench.bench_variants(None, None, {}, "measured")
-    assert list(res)[-1] == "attn_decode" and "attention failed" in res["attn_decode"]["error"]
+    assert list(res)[-2:] == ["prefill_shard_merge", "attn_decode"]
+    assert "attention failed" in res["attn_decode"]["error"]
     assert all(v == {"ms_per_step": 1.0} for k, v in res.items() if k != "attn_decode")
     with pytest.raises(RuntimeError):                       # asked for alone, it fails loudly
         bench.bench_variants(None, None, {}, "measured", only="attn_decode")
