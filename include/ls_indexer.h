@@ -369,9 +369,10 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
  *   row_off [T] int64 or NULL: row of latent = idx + row_off[t] (one buffer
  *        holding several sequences' caches); a row outside [0, n_rows) is
  *        skipped and sets LS_FAULT_BAD_INDEX (see ls_device_status)
- *   H a multiple of 8, k <= 65536 (the selection streams through in chunks
- *        of 64 slots: an LSA read list of 4612 slots fits); scale is the softmax scale (1/sqrt(576) is
- *        the plain choice; the pages do not fix it)
+ *   H a multiple of 8; k <= 65536 (the selection streams through in chunks
+ *        of 64 slots: an LSA read list of 4612 slots fits)
+ *   scale: the softmax scale (1/sqrt(576) is the plain choice; the pages do
+ *        not fix it)
  *   flags: 0, or LS_ATTN_FOREIGN_ROWS when latent holds one shard of the
  *        rows (row_off = -first row of the shard, n_rows = its length): rows
  *        outside it belong to other shards and are skipped without the fault
