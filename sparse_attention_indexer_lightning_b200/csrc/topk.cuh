@@ -687,6 +687,12 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
     __syncthreads();
     scan_bins_2048<NT>(sh, sh.hist, sh.fill, static_cast<uint32_t>(kk));  // fill: offsets from the top
     const uint32_t b_end = sh.fill[sh.digit] + sh.hist[sh.digit];         // end of the boundary bin
+    // Every thread holds b_end before any thread's scatter moves fill[]: a
+    // thread that read fill[digit] after another warp's atomics would see a
+    // larger end, rank slots the scatter never wrote (a bin index taken from
+    // uninitialised shared memory) and take the other branch around the
+    // barriers below.
+    __syncthreads();
     if (b_end <= 2u * KMAX) {
       unsigned long long* bkey = sh.sel_key;  // 2*KMAX keys
       float* bval = sh.sel_val;               // 2*KMAX values

@@ -19,7 +19,7 @@
 #define __host__
 #define __forceinline__ inline
 #define __restrict__ __restrict
-#define __launch_bounds__(x)
+#define __launch_bounds__(...)
 #define __shared__
 #define __align__(x)
 
@@ -36,8 +36,16 @@ struct Dim3 { unsigned x, y, z; };
 extern thread_local Dim3 threadIdx, blockIdx;
 extern Dim3 blockDim, gridDim;
 
-inline uint4 __ldg(const uint4* p) { return *p; }
+struct alignas(16) int4 { int x, y, z, w; };
+inline int4 make_int4(int a, int b, int c, int d) { return {a, b, c, d}; }
+
+template <class T>
+inline T __ldg(const T* p) { return *p; }
 inline float __uint_as_float(uint32_t u) { float f; std::memcpy(&f, &u, 4); return f; }
+inline uint32_t __float_as_uint(float f) { uint32_t u; std::memcpy(&u, &f, 4); return u; }
+inline float __int_as_float(int i) { float f; std::memcpy(&f, &i, 4); return f; }
+inline int __popc(uint32_t v) { return __builtin_popcount(v); }
+inline int __clzll(long long v) { return v == 0 ? 64 : __builtin_clzll(static_cast<unsigned long long>(v)); }
 
 extern std::barrier<>* g_block_bar;
 extern std::barrier<>* g_warp_bar[32];
@@ -53,6 +61,48 @@ inline float __shfl_xor_sync(unsigned, float v, int o) {
   const float r = g_xbuf[w][l ^ o];
   g_warp_bar[w]->arrive_and_wait();
   return r;
+}
+// Warp collectives beyond the float butterfly: every lane of the warp posts
+// its 64-bit value, a barrier of the warp's 32 threads, then each lane reads.
+inline uint64_t g_x64[32][32];
+template <class F>
+inline uint64_t warp_gather(uint64_t mine, F pick) {
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  g_x64[w][l] = mine;
+  g_warp_bar[w]->arrive_and_wait();
+  const uint64_t r = pick(g_x64[w], l);
+  g_warp_bar[w]->arrive_and_wait();
+  return r;
+}
+inline uint32_t __shfl_sync(unsigned, uint32_t v, int src) {
+  return static_cast<uint32_t>(warp_gather(v, [&](const uint64_t* x, int) { return x[src & 31]; }));
+}
+inline uint32_t __shfl_up_sync(unsigned, uint32_t v, int d) {
+  return static_cast<uint32_t>(warp_gather(v, [&](const uint64_t* x, int l) { return l >= d ? x[l - d] : x[l]; }));
+}
+inline unsigned long long __shfl_xor_sync(unsigned, unsigned long long v, int o) {
+  return warp_gather(v, [&](const uint64_t* x, int l) { return x[l ^ o]; });
+}
+inline uint32_t __shfl_xor_sync(unsigned, uint32_t v, int o) {
+  return static_cast<uint32_t>(warp_gather(v, [&](const uint64_t* x, int l) { return x[l ^ o]; }));
+}
+template <class T>
+inline T min(T a, T b) { return b < a ? b : a; }
+template <class T>
+inline T max(T a, T b) { return a < b ? b : a; }
+inline uint32_t __ballot_sync(unsigned, int pred) {
+  return static_cast<uint32_t>(warp_gather(pred ? 1u : 0u, [&](const uint64_t* x, int) {
+    uint32_t b = 0;
+    for (int i = 0; i < 32; ++i) b |= static_cast<uint32_t>(x[i] & 1u) << i;
+    return static_cast<uint64_t>(b);
+  }));
+}
+inline int __any_sync(unsigned m, int pred) { return __ballot_sync(m, pred) != 0u; }
+inline unsigned atomicAdd(unsigned* p, unsigned v) {
+  std::lock_guard<std::mutex> g(g_atomic_mu);
+  const unsigned old = *p;
+  *p += v;
+  return old;
 }
 inline int atomicMin(int* p, int v) {
   std::lock_guard<std::mutex> g(g_atomic_mu);
