@@ -1,7 +1,8 @@
 """Benchmark of the lightning-indexer selection path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_batch] [--no-variants] [--no-cpu-baseline]
+                    [--workload decode_batch] [--no-variants] [--variants default|all|A,B]
+                    [--only NAME] [--no-cpu-baseline]
 
 One step is one decode selection over the batch workload: 64 sequences x
 32768 stride-4 compressed bf16 keys (131072 tokens each), 32 heads x 128 dims,
@@ -10,9 +11,10 @@ exact top-512 per sequence -- the scan (ls_indexer_score) then the selection
 no flush is needed between steps.  The metric is query-positions scored per
 second (selections per second alongside).  The prefill, two-stage, bucket
 and LSA searches, and the sparse attention that follows a decode selection
-(`attn_decode`, last; an error there is recorded in its own entry), are
-timed the same way and reported under "variants", each with the roofline of
-its dominant kernel.
+(`attn_decode`), are timed the same way, each in a child process of its own
+(`bench.py --only NAME`), and reported under "variants", each with the
+roofline of its dominant kernel; a child that fails leaves an error entry and
+the decode line is printed whatever the variants do.
 
 With N > 1 (torchrun) every rank runs its own batch (weak scaling, no
 collective on the data path); the reported time is the max over ranks.
@@ -347,27 +349,64 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
     return out, d
 
 
-def bench_variants(L, args, peaks, peak_kind, only=None):
-    """Prefill chunk, two-stage and bucket searches: one timed loop each."""
+VARIANTS = {
+    "prefill_chunk": lambda *a: bench_prefill(*a),
+    "prefill_chunk_running": lambda *a: bench_prefill(*a, full_scores=False),
+    "prefill_chunk_fp8": lambda *a: bench_prefill(*a, fp8=True),
+    "prefill_chunk_fp8_running": lambda *a: bench_prefill(*a, full_scores=False, fp8=True),
+    "bucket": lambda *a: bench_bucket(*a),
+    "lsa_flat": lambda *a: bench_lsa(*a),
+    "lsa_flat_threshold": lambda *a: bench_lsa(*a, threshold=True),
+    "lsa_tree": lambda *a: bench_lsa_tree(*a),
+    "two_stage": lambda *a: bench_two_stage(*a),
+    "two_stage_pq": lambda *a: bench_two_stage(*a, pq=True),
+    "prefill_shard_merge": lambda *a: bench_shard_merge(*a),
+    "attn_decode": lambda *a: bench_attention(*a),
+}
+# The lines a plain run times, each in a child process of its own: a fault in
+# one (a sticky CUDA error ends its process) becomes an error entry and cannot
+# reach the decode line or another variant.  A variant joins this list once it
+# has run clean on a B200.
+DEFAULT_VARIANTS = list(VARIANTS)
+
+
+def bench_one_variant(L, args, peaks, peak_kind, name):
+    """One variant in this process (``--only NAME``)."""
+    return {name: VARIANTS[name](L, args, peaks, peak_kind)}
+
+
+def bench_variants(args, names=None, timeout_s: float = 900.0):
+    """Every variant in `names` in a child process of its own (``bench.py
+    --only NAME``), one after another; each child's JSON line becomes that
+    variant's entry, a child that fails leaves an error entry."""
+    import subprocess
     res = {}
-    for name, fn in (("prefill_chunk", bench_prefill),
-                     ("prefill_chunk_running", lambda *a: bench_prefill(*a, full_scores=False)),
-                     ("prefill_chunk_fp8", lambda *a: bench_prefill(*a, fp8=True)),
-                     ("prefill_chunk_fp8_running", lambda *a: bench_prefill(*a, full_scores=False, fp8=True)),
-                     ("bucket", bench_bucket), ("lsa_flat", bench_lsa),
-                     ("lsa_flat_threshold", lambda *a: bench_lsa(*a, threshold=True)), ("lsa_tree", bench_lsa_tree),
-                     ("two_stage", bench_two_stage),
-                     ("two_stage_pq", lambda *a: bench_two_stage(*a, pq=True)),
-                     ("prefill_shard_merge", bench_shard_merge),
-                     ("attn_decode", bench_attention)):
-        if only in (None, name):
-            if name in ("prefill_shard_merge", "attn_decode") and only is None:
-                try:                       # the newest paths: an error here must not lose the lines above
-                    res[name] = fn(L, args, peaks, peak_kind)
-                except Exception as e:     # noqa: BLE001
-                    res[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
-                continue
-            res[name] = fn(L, args, peaks, peak_kind)
+    for name in (DEFAULT_VARIANTS if names is None else names):
+        cmd = [sys.executable, os.path.abspath(__file__), "--only", name, "--steps", str(args.steps),
+               "--warmup", str(args.warmup)]
+        env = dict(os.environ)
+        for v in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "LOCAL_WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT"):
+            env.pop(v, None)
+        t0 = time.perf_counter()
+        try:
+            r = subprocess.run(cmd, capture_output=True, text=True, timeout=timeout_s, env=env, cwd=ROOT)
+        except subprocess.TimeoutExpired:
+            res[name] = {"error": f"timed out after {timeout_s:.0f} s"}
+            continue
+        entry = None
+        for ln in reversed(r.stdout.splitlines()):
+            if ln.startswith("{"):
+                try:
+                    entry = json.loads(ln).get(name)
+                except ValueError:
+                    entry = None
+                break
+        if r.returncode != 0 or not isinstance(entry, dict):
+            tail = (r.stderr or r.stdout).strip().splitlines()[-3:]
+            res[name] = {"error": f"exit {r.returncode}: " + " | ".join(tail)[-400:]}
+        else:
+            entry["child_wall_s"] = round(time.perf_counter() - t0, 1)
+            res[name] = entry
     return res
 
 
@@ -827,11 +866,11 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_batch")
     ap.add_argument("--no-variants", action="store_true")
-    ap.add_argument("--only", default=None, choices=["prefill_chunk", "prefill_chunk_running", "prefill_chunk_fp8",
-                                                     "prefill_chunk_fp8_running", "bucket", "lsa_flat",
-                                                     "lsa_flat_threshold", "lsa_tree", "two_stage",
-                                                     "two_stage_pq", "prefill_shard_merge", "attn_decode"],
-                    help="time one variant only and skip the decode line (profiling)")
+    ap.add_argument("--variants", default="default",
+                    help="'default' (the lines that have run clean on a B200), 'all', or a comma-separated list")
+    ap.add_argument("--only", default=None, choices=sorted(VARIANTS),
+                    help="time one variant in this process and skip the decode line (profiling, and the "
+                         "child processes of a plain run)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -844,16 +883,22 @@ def main(argv=None):
     import sparse_attention_indexer_lightning_b200 as L
     peaks, peak_kind = load_peaks()
     if args.only:
-        print(json.dumps({"variant": args.only, **bench_variants(L, args, peaks, peak_kind, args.only)}))
+        print(json.dumps({"variant": args.only, **bench_one_variant(L, args, peaks, peak_kind, args.only)}))
         return 0
     out, d = bench_decode(L, args, world, rank, peaks, peak_kind)
-    if not args.no_variants and world == 1:
-        out["variants"] = bench_variants(L, args, peaks, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n_seq, el = oracle_decode_rate(d, 12.0, 512)
         out["cpu_baseline"] = {"value": rate, "unit": "positions/s", "cores": blas_threads(), "kind": "oracle",
                                "sample": f"{n_seq} whole sequences x {d['k'].shape[1]} positions "
                                          f"({el:.1f} s of fp64 oracle work)"}
+    del d
+    if not args.no_variants and world == 1:
+        names = (None if args.variants == "default" else sorted(VARIANTS) if args.variants == "all"
+                 else [v for v in args.variants.split(",") if v])
+        try:
+            out["variants"] = bench_variants(args, names)
+        except Exception as e:  # noqa: BLE001 -- the decode line is printed whatever happens here
+            out["variants"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -153,13 +153,14 @@ ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* ke
  * Same arguments and results as ls_decode_select, without (ws, ws_bytes):
  * the scratch is a fixed 10 MiB device array inside the library, held on
  * every device that loads it until the process exits.  Sizes whose
- * ls_decode_select_workspace_size(B, N) exceeds 10 MiB (B*N above about
- * 2.5 million with B rows of histograms) return LS_ERR_WORKSPACE.  The first
- * call on a device looks up the array's device address (cudaGetSymbolAddress)
- * with that device current; make it before any stream capture.  The call
- * allocates nothing.  All calls share the array: calls that overlap on the
- * GPU race and must be serialised by the caller; the part that must start at
- * zero is cleared by every call.
+ * ls_decode_select_workspace_size(B, N) exceeds 10 MiB (B*N above 2,621,440
+ * scores) return LS_ERR_WORKSPACE.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current and
+ * keeps it; make that call before any stream capture, and do not call again
+ * on a device after cudaDeviceReset (the kept address belonged to the ended
+ * context).  The call allocates nothing.  All calls share the array: calls
+ * that overlap on the GPU race and must be serialised by the caller; nothing
+ * in it needs clearing (each call overwrites the score rows it reads).
  */
 ls_status ls_decode_select_noalloc(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid,
                                    int B, int H, int d, int N, int k, int32_t* idx_out, float* val_out,

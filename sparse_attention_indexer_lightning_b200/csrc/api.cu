@@ -394,8 +394,7 @@ ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid
 
 size_t ls_decode_select_workspace_size(int B, int N) {
   if (B <= 0 || N <= 0) return 0;
-  return align_up(static_cast<size_t>(B) * N * sizeof(float)) +
-         align_up(static_cast<size_t>(B) * kHistBins * sizeof(uint32_t));
+  return align_up(static_cast<size_t>(B) * N * sizeof(float));  // the score rows
 }
 
 ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* keys, const int32_t* n_valid, int B,
@@ -412,13 +411,11 @@ ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* ke
     return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
   Carver cv(ws);
   float* sc = cv.take<float>(static_cast<size_t>(B) * N);
-  uint32_t* hist = cv.take<uint32_t>(static_cast<size_t>(B) * kHistBins);
   if (N > 0) {
     LS_CHECK_ARG(q && w && keys, "null tensor pointer");
     LS_CHECK_ARG(aligned16(q) && aligned16(w) && aligned16(keys), "q, w and keys must be 16-byte aligned");
     // The top-k samples its own threshold; counting a histogram in the scan
     // epilogue costs the scan more than it saves the selection.
-    (void)hist;
     s = score_bf16(q, w, keys, n_valid, nullptr, 1, B, 1, N, 0, N, sc, N, S(stream));
     if (s != LS_OK) return s;
   }
@@ -1379,19 +1376,21 @@ ls_status ls_selftest_wait_probe(uint64_t limit_ns, int* gave_up_dev, void* stre
 // allocator, or a latency-critical loop where the implicit device-wide
 // synchronisation of cudaMalloc / cudaFree is not acceptable.  For them,
 // ls_decode_select_noalloc runs the same decode selection as
-// ls_decode_select with its scratch (the score rows and the selection
-// histograms) in the fixed device array below, which the library holds on
-// every device that loads it until the process exits.
+// ls_decode_select with its scratch (the score rows) in the fixed device
+// array below, which the library holds on every device that loads it until
+// the process exits.
 //
 // The array's host-side name is not a device address, so the first call on
 // each device (with that device current) asks the runtime for the address
 // with cudaGetSymbolAddress and caches it.  That first call should therefore
-// be made before any stream capture is started on that device.  Nothing else
-// is allocated: no cudaMalloc, cudaFree or allocating library call.
+// be made before any stream capture is started on that device.  A
+// cudaDeviceReset ends the context the cached address belongs to: a process
+// that resets a device must not call this entry point on it again.  Nothing
+// else is allocated: no cudaMalloc, cudaFree or allocating library call.
 //
 // All calls share the one array and it keeps the contents of the last call.
-// The histogram part, which must start at zero, is cleared on the stream by
-// every call; the score part is fully overwritten.  Calls whose work overlaps
+// Nothing in it has to start at zero: every call overwrites the score rows it
+// reads (the decode selection keeps no counters there).  Calls whose work overlaps
 // on the GPU (on different streams, or from different host threads) race on
 // the array: order them on one stream or serialise them.
 // ---------------------------------------------------------------------------
@@ -1413,7 +1412,7 @@ extern "C" ls_status ls_decode_select_noalloc(const uint16_t* q, const float* w,
   if (need > kNoAllocScratchBytes)
     return fail(LS_ERR_WORKSPACE,
                 "B=%d x N=%d needs %zu B of scratch; the fixed scratch of ls_decode_select_noalloc holds %zu B "
-                "(about 2.5M score entries in all); use ls_decode_select with a workspace",
+                "(2,621,440 score entries in all); use ls_decode_select with a workspace",
                 B, N, need, kNoAllocScratchBytes);
   int dev = 0;
   LS_CUDA(cudaGetDevice(&dev));

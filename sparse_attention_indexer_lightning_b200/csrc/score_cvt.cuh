@@ -502,12 +502,10 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
 template <int FMT>
 static cudaError_t launch_cvt(const CUtensorMap* qmap, const CvtParams& p, int num_sms, cudaStream_t st) {
   using C = CvtCfg<FMT>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(score_cvt_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::SMEM_TOTAL));
+  static std::atomic<uint64_t> attr_done{0};
+  {
+    const cudaError_t e = smem_limit_once(attr_done, reinterpret_cast<const void*>(&score_cvt_kernel<FMT>), C::SMEM_TOTAL);
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   const int NT = (p.N + C::BM - 1) / C::BM;
   const long long units = static_cast<long long>(p.B) * NT;

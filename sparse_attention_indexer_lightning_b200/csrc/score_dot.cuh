@@ -376,12 +376,10 @@ template <bool FILTER>
 static cudaError_t launch_dot(const CUtensorMap* cmap, const CUtensorMap* qmap, const DotParams& p, int num_sms,
                               cudaStream_t st) {
   using C = DotCfg;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(dot_tc_kernel<FILTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::SMEM_TOTAL));
+  static std::atomic<uint64_t> attr_done{0};
+  {
+    const cudaError_t e = smem_limit_once(attr_done, reinterpret_cast<const void*>(&dot_tc_kernel<FILTER>), C::SMEM_TOTAL);
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   const int grid = dot_tc_grid(p.T, p.P, num_sms);
   if (grid == 0) return cudaSuccess;

@@ -500,12 +500,10 @@ template <int FMT, int HALVES>
 static cudaError_t launch_q8(const CUtensorMap* qmap, const CUtensorMap* kmap, const CvtParams& p, int num_sms,
                              cudaStream_t st) {
   using C = Q8Cfg<FMT, HALVES>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(score_q8_kernel<FMT, HALVES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::SMEM_TOTAL));
+  static std::atomic<uint64_t> attr_done{0};
+  {
+    const cudaError_t e = smem_limit_once(attr_done, reinterpret_cast<const void*>(&score_q8_kernel<FMT, HALVES>), C::SMEM_TOTAL);
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   const int NT = (p.N + C::KPU - 1) / C::KPU;
   const long long units = static_cast<long long>(p.B) * NT;

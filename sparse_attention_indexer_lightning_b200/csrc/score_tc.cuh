@@ -444,12 +444,10 @@ template <int QG, bool FILTER, bool F8 = false>
 static cudaError_t launch_tc(const CUtensorMap* kmap, const CUtensorMap* qmap, const ScoreParams& p, int num_sms,
                              cudaStream_t st) {
   using C = TcCfg<QG, FILTER, F8>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<QG, FILTER, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::SMEM_TOTAL));
+  static std::atomic<uint64_t> attr_done{0};
+  {
+    const cudaError_t e = smem_limit_once(attr_done, reinterpret_cast<const void*>(&score_tc_kernel<QG, FILTER, F8>), C::SMEM_TOTAL);
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   const int G = (p.T + QG - 1) / QG;
   const int NT = (p.N + C::BM - 1) / C::BM;

@@ -836,12 +836,10 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
 template <int NT, int KMAX, int CAP>
 static cudaError_t launch_topk_t(const TopkParams& p, cudaStream_t st) {
   using SH = TopkShared<NT, KMAX, CAP>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel<NT, KMAX, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(SH)));
+  static std::atomic<uint64_t> attr_done{0};
+  {
+    const cudaError_t e = smem_limit_once(attr_done, reinterpret_cast<const void*>(&topk_kernel<NT, KMAX, CAP>), sizeof(SH));
     if (e != cudaSuccess) return e;
-    attr_done = true;
   }
   topk_kernel<NT, KMAX, CAP><<<p.R, NT, sizeof(SH), st>>>(p);
   return cudaGetLastError();

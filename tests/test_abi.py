@@ -43,7 +43,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_workspace_queries(lib):
     assert lib.ls_version() == 100
-    assert lib.ls_decode_select_workspace_size(64, 32768) == 64 * 32768 * 4 + 64 * 2048 * 4
+    assert lib.ls_decode_select_workspace_size(64, 32768) == 64 * 32768 * 4   # the score rows only
     # one 8192-key tile of scores plus running lists of k + 3k entries (values and labels)
     assert lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 0) >= 4096 * 8192 * 4 + 4096 * 2048 * 8
     assert lib.ls_prefill_select_workspace_size(4096, 8192, 8192, 512, 0) < 4096 * 8192 * 4 + 4096 * 64

@@ -52,20 +52,35 @@ def test_digest_covers_the_kernel_sources():
     assert bench.source_digest("topk_kernel") == bench.source_digest(None)
 
 
-def test_attention_line_error_keeps_the_other_lines(monkeypatch):
-    """The attention line runs last and an exception there is recorded in its
-    own entry; the variants before it (the shard merge just before) are kept."""
-    names = ["bench_prefill", "bench_bucket", "bench_lsa", "bench_lsa_tree", "bench_two_stage", "bench_shard_merge"]
-    for n in names:
-        monkeypatch.setattr(bench, n, lambda *a, **k: {"ms_per_step": 1.0})
+def test_variant_children_isolate_failures(monkeypatch):
+    """Each variant runs in a child process; a child that dies (a sticky CUDA
+    error ends its process), prints no line, or runs out of time leaves an
+    error entry, and the variants after it still run."""
+    import subprocess
+    import types
 
-    def boom(*a, **k):
-        raise RuntimeError("attention failed")
+    calls = []
 
-    monkeypatch.setattr(bench, "bench_attention", boom)
-    res = bench.bench_variants(None, None, {}, "measured")
-    assert list(res)[-2:] == ["prefill_shard_merge", "attn_decode"]
-    assert "attention failed" in res["attn_decode"]["error"]
-    assert all(v == {"ms_per_step": 1.0} for k, v in res.items() if k != "attn_decode")
-    with pytest.raises(RuntimeError):                       # asked for alone, it fails loudly
-        bench.bench_variants(None, None, {}, "measured", only="attn_decode")
+    def fake_run(cmd, **kw):
+        name = cmd[cmd.index("--only") + 1]
+        calls.append(name)
+        if name == "prefill_chunk_fp8_running":
+            return types.SimpleNamespace(returncode=1, stdout="",
+                                         stderr="torch.AcceleratorError: CUDA error: an illegal memory access")
+        if name == "bucket":
+            raise subprocess.TimeoutExpired(cmd, 1)
+        if name == "lsa_flat":
+            return types.SimpleNamespace(returncode=0, stdout="no json here\n", stderr="")
+        return types.SimpleNamespace(returncode=0, stdout="log line\n" + bench.json.dumps(
+            {"variant": name, name: {"ms_per_step": 1.0}}) + "\n", stderr="")
+
+    monkeypatch.setattr(subprocess, "run", fake_run)
+    args = types.SimpleNamespace(steps=3, warmup=3)
+    names = ["prefill_chunk", "prefill_chunk_fp8_running", "bucket", "lsa_flat", "two_stage"]
+    res = bench.bench_variants(args, names)
+    assert calls == names
+    assert res["prefill_chunk"]["ms_per_step"] == 1.0 and res["two_stage"]["ms_per_step"] == 1.0
+    assert "illegal memory access" in res["prefill_chunk_fp8_running"]["error"]
+    assert "timed out" in res["bucket"]["error"]
+    assert "exit 0" in res["lsa_flat"]["error"]
+    assert set(bench.DEFAULT_VARIANTS) <= set(bench.VARIANTS)

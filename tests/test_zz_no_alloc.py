@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import RTOL_BF16, dev, dev_bf16
+from parity_util import dev, dev_bf16
 from workloads.synth import make_decode
 
 pytestmark = pytest.mark.gpu
@@ -69,11 +69,9 @@ def test_noalloc_matches_workspace_call_twice(lib):
         i1, v1 = _with_workspace(lib, q, w, k, nv, 512, stream)
         torch.cuda.synchronize()
         i0, v0, i1, v1 = (t.cpu().numpy() for t in (i0, v0, i1, v1))
+        # the same kernels on the same inputs: indices and values bit for bit
         assert np.array_equal(i0, i1)
-        fin = np.isfinite(v1)
-        assert np.array_equal(np.isfinite(v0), fin)
-        floor = np.median(np.abs(v1[fin])) if fin.any() else 0.0
-        assert np.all(np.abs(v0[fin] - v1[fin]) <= RTOL_BF16 * np.maximum(np.abs(v1[fin]), floor))
+        assert np.array_equal(v0.view(np.uint32), v1.view(np.uint32))
 
 
 def test_noalloc_refuses_oversized_problem(lib):
