@@ -184,15 +184,18 @@ ls_status ls_decode_select_noalloc(const uint16_t* q, const float* w, const uint
  * copy waits for work already queued on compute_stream (buffers may be in use).
  *
  * full_scores = 0: selection runs across the tiles (running top-k).  The
- * first tile is scored in full and its exact top-k gives each query a running
- * list; every later tile emits only the keys whose score beats the query's
- * running k-th entry (strictly: a later key that ties it ranks lower) into up
- * to 3k candidate slots, and a merge keeps the top k of running list +
- * candidates.  A query that fills its slots gets that tile's exact top-k from
- * the tile scored again in full (a launch that does nothing when no query
- * overflowed).  No T x N score matrix is held: the workspace is one
- * T x tile_keys tile plus the lists, so N is bounded by the history's host
- * memory, not by the device.
+ * first tile is scored in full; its exact top-k starts each query's list and
+ * the list's k-th entry is the query's threshold for the rest of the call.
+ * Every later tile emits only the keys whose score beats that threshold
+ * (strictly: a later key that ties it ranks lower) into the query's 2k
+ * candidate slots for that tile; a query that fills them gets that tile's
+ * exact top-k instead, from the tile scored again in full (a launch that does
+ * nothing when no query overflowed).  After the last tile each query's lists
+ * are packed and one exact top-k selects from them: every key of the true
+ * top k scores at least the threshold, so it is in a list.  No T x N score
+ * matrix is held: the workspace is one T x tile_keys tile plus
+ * T x (k + 2k * (tiles - 1)) list entries, so N is bounded by the history's
+ * host memory, not by the device.
  * full_scores = 1: every tile's scores go into a T x N matrix in the
  * workspace and one top-k runs at the end (fewer launches; needs T*N*4 B).
  * Both forms return the same selection.

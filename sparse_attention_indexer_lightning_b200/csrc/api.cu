@@ -422,21 +422,30 @@ ls_status ls_decode_select(const uint16_t* q, const float* w, const uint16_t* ke
   return topk(sc, N, n_valid, nullptr, 0, B, N, k, idx_out, val_out, k, S(stream));
 }
 
-// Candidate slots per row and tile in the running top-k of the prefill.
-int prefill_cand_cap(int k) { return 3 * k; }
+// Candidate slots per row for each tile after the first in the running top-k
+// of the prefill.
+int prefill_cand_cap(int k) { return 2 * k; }
+
+// Row width of the running form's lists: the first tile's top-k, then one
+// candidate segment per later tile.
+int64_t prefill_list_width(int N, int tile_keys, int k) {
+  const int ntiles = (N + tile_keys - 1) / tile_keys;
+  return ntiles > 1 ? k + static_cast<int64_t>(ntiles - 1) * prefill_cand_cap(k) : 0;
+}
 
 size_t ls_prefill_select_workspace_size(int T, int N, int tile_keys, int k, int full_scores) {
   if (T <= 0 || N <= 0 || tile_keys <= 0 || k <= 0) return 0;
-  // full_scores: the whole T x N score matrix (one top-k at the end), no running lists
+  // full_scores: the whole T x N score matrix (one top-k at the end), no lists
   const int tk = full_scores ? N : (tile_keys < N ? tile_keys : N);
   const int ntiles = (N + tile_keys - 1) / tile_keys;
-  const int64_t ldc = (!full_scores && ntiles > 1) ? k + prefill_cand_cap(k) : 0;
+  const int64_t ldc = full_scores ? 0 : prefill_list_width(N, tile_keys, k);
+  const int64_t S = full_scores ? 0 : ntiles - 1;  // later tiles, each with its counters
   return align_up(static_cast<size_t>(T) * tk * sizeof(float)) +    // one tile of scores
-         align_up(static_cast<size_t>(T) * ldc * sizeof(float)) +   // running top-k + candidates
+         align_up(static_cast<size_t>(T) * ldc * sizeof(float)) +   // first tile's top-k + candidate segments
          align_up(static_cast<size_t>(T) * ldc * sizeof(int32_t)) +
          align_up(static_cast<size_t>(T) * sizeof(int32_t)) +       // eligible counts
-         align_up(static_cast<size_t>(T) * sizeof(int32_t)) +       // merge counts
-         align_up(static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int));  // counters, overflow flags
+         align_up(static_cast<size_t>(T) * sizeof(int32_t)) +       // packed list lengths
+         align_up(static_cast<size_t>(S) * (static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int)));  // counters, overflow flags
 }
 
 }  // extern "C"
@@ -492,17 +501,20 @@ ls_status prefill_stream(const Src& src, Carver& cv, const float* w, const int64
   const int tk = full_scores ? N : (tile_keys < N ? tile_keys : N);
   const int ntiles = (N + tile_keys - 1) / tile_keys;
   const int cap = prefill_cand_cap(k);
-  const int64_t ldc = (!full_scores && ntiles > 1) ? k + cap : 0;
+  const int64_t ldc = full_scores ? 0 : prefill_list_width(N, tile_keys, k);
+  const int S = full_scores ? 0 : ntiles - 1;
   float* tile_sc = cv.take<float>(static_cast<size_t>(T) * tk);  // full_scores: the T x N matrix
   float* run_val = cv.take<float>(static_cast<size_t>(T) * ldc);
   int32_t* run_lab = cv.take<int32_t>(static_cast<size_t>(T) * ldc);
   int32_t* counts = cv.take<int32_t>(T);
   int32_t* nv = cv.take<int32_t>(T);
-  uint8_t* ctr = cv.take<uint8_t>(static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int));
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(ctr);
-  int32_t* row_over = reinterpret_cast<int32_t*>(ctr) + T;
-  int* any_over = reinterpret_cast<int*>(ctr) + 2 * static_cast<size_t>(T);
-  const size_t ctr_bytes = static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int);
+  // per later tile j (1..S): candidate counters [T], overflow flags [T], and
+  // one "some row overflowed" word, zeroed once per call
+  const size_t ctr_bytes = static_cast<size_t>(S) * (static_cast<size_t>(T) * 2 * sizeof(int32_t) + sizeof(int));
+  uint8_t* ctr = cv.take<uint8_t>(ctr_bytes);
+  uint32_t* cnt_all = reinterpret_cast<uint32_t*>(ctr);
+  int32_t* over_all = reinterpret_cast<int32_t*>(ctr) + static_cast<size_t>(S) * T;
+  int* any_all = reinterpret_cast<int*>(ctr) + static_cast<size_t>(S) * 2 * T;
 
   cudaEvent_t start_ev, copied[2], freed[2];
   LS_CUDA(cudaEventCreateWithFlags(&start_ev, cudaEventDisableTiming));
@@ -515,8 +527,10 @@ ls_status prefill_stream(const Src& src, Carver& cv, const float* w, const int64
     ProfScope prof("causal_counts_kernel", cs);
     LS_CUDA(launch_causal_counts(q_pos, T, stride, N, counts, cs));
   }
+  cudaError_t e = cudaSuccess;
+  if (S > 0) e = cudaMemsetAsync(ctr, 0, ctr_bytes, cs);
   // Earlier work on the compute stream may still read the buffers.
-  cudaError_t e = cudaEventRecord(start_ev, cs);
+  if (e == cudaSuccess) e = cudaEventRecord(start_ev, cs);
   if (e == cudaSuccess && xs != cs) e = cudaStreamWaitEvent(xs, start_ev, 0);
   for (int j = 0; j < ntiles && e == cudaSuccess && st == LS_OK; ++j) {
     const int slot = j & 1;
@@ -570,7 +584,8 @@ ls_status prefill_stream(const Src& src, Carver& cv, const float* w, const int64
         if (st != LS_OK) break;
       }
     } else if (j == 0) {
-      // the first tile is scored in full and gives every row its running top-k
+      // the first tile is scored in full; its exact top-k starts every row's
+      // list, and the row's k-th entry there is its threshold for the rest
       sp.out = tile_sc;
       sp.ld_out = tk;
       st = src.score(slot, T, len, sp, cs, nullptr);
@@ -581,23 +596,28 @@ ls_status prefill_stream(const Src& src, Carver& cv, const float* w, const int64
       st = topk_launch(tp, cs);
       if (st != LS_OK) break;
     } else {
-      // later tiles append only keys that beat the row's running k-th entry
-      e = cudaMemsetAsync(ctr, 0, ctr_bytes, cs);
-      if (e != cudaSuccess) break;
+      // later tiles append the keys that beat the row's threshold to the
+      // row's segment for this tile
+      const size_t seg = static_cast<size_t>(k) + static_cast<size_t>(j - 1) * cap;
+      uint32_t* cnt = cnt_all + static_cast<size_t>(j - 1) * T;
+      int32_t* row_over = over_all + static_cast<size_t>(j - 1) * T;
+      int* any_over = any_all + (j - 1);
       ScoreParams fp = sp;
-      fp.cand_val = run_val;
-      fp.cand_lab = run_lab;
+      fp.cand_val = run_val + seg;
+      fp.cand_lab = run_lab + seg;
       fp.ld_cand = ldc;
-      fp.run_k = k;
       fp.cand_cap = cap;
+      fp.kth_val = run_val + (k - 1);
+      fp.kth_lab = run_lab + (k - 1);
+      fp.ld_kth = ldc;
       fp.cand_cnt = cnt;
       fp.row_over = row_over;
       fp.any_over = any_over;
       st = src.score(slot, T, len, fp, cs, nullptr);
       if (st != LS_OK) break;
-      // rows that ran out of candidate slots: this tile again in full (the
-      // launches return at once when no row overflowed), its top-k into the
-      // row's candidate columns
+      // rows that ran out of slots: this tile again in full (the launches
+      // return at once when no row overflowed), its top-k into the row's
+      // segment
       sp.out = tile_sc;
       sp.ld_out = tk;
       sp.run_if = any_over;
@@ -605,30 +625,32 @@ ls_status prefill_stream(const Src& src, Carver& cv, const float* w, const int64
       if (st != LS_OK) break;
       tp.run_if = any_over;
       tp.row_flag = row_over;
-      tp.idx_out = run_lab + k;
-      tp.val_out = run_val + k;
+      tp.idx_out = run_lab + seg;
+      tp.val_out = run_val + seg;
       tp.ld_out = ldc;
       st = topk_launch(tp, cs, "topk_kernel:overflow");
       if (st != LS_OK) break;
-      {
-        ProfScope prof("merge_counts_kernel", cs);
-        LS_CUDA(launch_merge_counts(cnt, row_over, T, k, cap, nv, cs));
+      if (last) {
+        // every row's lists packed into one prefix, then one exact top-k
+        {
+          ProfScope prof("pack_segments_kernel", cs);
+          LS_CUDA(launch_pack_segments(run_val, run_lab, ldc, T, k, S, cap, cnt_all, over_all, nv, cs));
+        }
+        TopkParams mp;
+        mp.scores = run_val;
+        mp.ld = ldc;
+        mp.n_valid = nv;
+        mp.labels = run_lab;
+        mp.ld_labels = ldc;
+        mp.R = T;
+        mp.N = static_cast<int>(ldc);
+        mp.k = k;
+        mp.idx_out = idx_out;
+        mp.val_out = val_out;
+        mp.ld_out = k;
+        st = topk_launch(mp, cs);
+        if (st != LS_OK) break;
       }
-      // merge: running top-k + this tile's candidates -> the new running top-k
-      TopkParams mp;
-      mp.scores = run_val;
-      mp.ld = ldc;
-      mp.n_valid = nv;
-      mp.labels = run_lab;
-      mp.ld_labels = ldc;
-      mp.R = T;
-      mp.N = static_cast<int>(ldc);
-      mp.k = k;
-      mp.idx_out = last ? idx_out : run_lab;
-      mp.val_out = last ? val_out : run_val;
-      mp.ld_out = last ? k : ldc;
-      st = topk_launch(mp, cs);
-      if (st != LS_OK) break;
     }
     if (xs != cs) e = cudaEventRecord(freed[slot], cs);
   }

@@ -24,13 +24,14 @@ constexpr int kLsaDim = 64;    // native LSA index space width
 // capped at n_total.
 //
 // Filter form (out == nullptr): nothing is stored per key; instead every
-// eligible key whose score beats the row's running k-th entry (read from
-// cand_val / cand_lab columns run_k-1 of the row; a row whose list is not yet
-// full takes every eligible key) is appended as (score, key_base + n) to the
-// row's candidate columns run_k .. run_k+cand_cap-1 at the slot its counter
-// cand_cnt[row] hands out; a row that runs out of slots sets row_over[row]
-// and *any_over.  "Beats" compares order codes strictly: a later key that
-// ties the k-th entry ranks below it.
+// eligible key whose score beats the row's threshold entry (kth_val /
+// kth_lab[row * ld_kth]: the k-th entry of the row's list so far; a label < 0
+// means the list is not full and every eligible key is taken) is appended as
+// (score, key_base + n) to the row's candidate columns 0 .. cand_cap-1 of
+// cand_val / cand_lab at the slot its counter cand_cnt[row] hands out; a row
+// that runs out of slots sets row_over[row] and *any_over.  "Beats" compares
+// order codes strictly: a later key that ties the threshold entry ranks
+// below it.
 struct ScoreParams {
   const float* w = nullptr;           // [B][T][H]
   const int32_t* n_valid = nullptr;   // [B] or nullptr
@@ -45,11 +46,13 @@ struct ScoreParams {
   uint32_t* hist = nullptr;           // [B*T][2048] selection histogram (counts added) or nullptr; qg == 1 only
   const int32_t* lim_rows = nullptr;  // [B*T] eligible keys of the whole history per query (replaces q_pos)
   // filter form
-  float* cand_val = nullptr;          // [B*T][ld_cand]
-  int32_t* cand_lab = nullptr;        // [B*T][ld_cand]
+  float* cand_val = nullptr;          // row r's slots at cand_val + r * ld_cand
+  int32_t* cand_lab = nullptr;
   int64_t ld_cand = 0;
-  int run_k = 0;
   int cand_cap = 0;
+  const float* kth_val = nullptr;     // row r's threshold entry at kth_val[r * ld_kth]
+  const int32_t* kth_lab = nullptr;
+  int64_t ld_kth = 0;
   uint32_t* cand_cnt = nullptr;       // [B*T]
   int32_t* row_over = nullptr;        // [B*T]
   int* any_over = nullptr;
@@ -177,11 +180,14 @@ cudaError_t launch_causal_counts(const int64_t* q_pos, int T, int stride, int n_
 cudaError_t launch_expand(const int32_t* picked, int T, int top_p, const int32_t* off, const int32_t* mem,
                           int P, int budget, int32_t* cand, cudaStream_t st);
 
-// Entries to merge per row after a filtered tile: the running k plus the
-// row's candidates (min(cnt, cap)), or plus the k entries of the row's
-// recomputed tile when it overflowed.
-cudaError_t launch_merge_counts(const uint32_t* cnt, const int32_t* row_over, int T, int k, int cap, int32_t* nv,
-                                cudaStream_t st);
+// Packs each row of the running prefill selection in place: row t of
+// (val, lab) [T][ld] holds the first tile's top-k in columns [0, k) and, for
+// each later tile j = 1 .. S, a segment of cap candidate slots at column
+// k + (j-1)*cap with cnt[(j-1)*T + t] entries (min(cnt, cap); k entries -- the
+// tile's recomputed top-k -- when row_over[(j-1)*T + t] is set).  The row's
+// present entries are moved to its first nv[t] columns, in that order.
+cudaError_t launch_pack_segments(float* val, int32_t* lab, int64_t ld, int T, int k, int S, int cap,
+                                 const uint32_t* cnt, const int32_t* row_over, int32_t* nv, cudaStream_t st);
 
 int read_and_clear_fault(cudaStream_t st, int* flags);
 cudaError_t launch_wait_probe(uint64_t limit_ns, int* waited, cudaStream_t st);

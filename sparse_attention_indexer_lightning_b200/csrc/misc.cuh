@@ -9,6 +9,9 @@
 //    append their members until the budget is held, cut the last bucket short.
 //  * fold_scales: w[t, h] * q_scale[t, h] for the fp8 scorer, which takes the
 //    non-negative per-(query, head) scale out of the ReLU.
+//  * pack_segments: the running prefill selection's per-row lists (the first
+//    tile's top-k and each later tile's candidate segment) moved to one
+//    contiguous prefix per row for the final top-k.
 //  * wait_probe: a kernel whose mbarrier is never signalled, used by the tests
 //    to show that a bounded wait returns with an error status.
 
@@ -49,18 +52,50 @@ cudaError_t launch_fold_scales(const float* w, const float* qs, int64_t n, float
   return cudaGetLastError();
 }
 
-__global__ void merge_counts_kernel(const uint32_t* cnt, const int32_t* row_over, int T, int k, int cap,
-                                    int32_t* nv) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  const uint32_t c = cnt[t];
-  nv[t] = k + (row_over[t] ? k : static_cast<int32_t>(c < static_cast<uint32_t>(cap) ? c : cap));
+// One CTA per row.  The first tile's top-k stays in place; each later
+// segment is moved down to the end of what precedes it, 256 entries at a
+// time: every thread reads its entry, a barrier, then every thread writes.
+// The source of a segment never starts before its destination, so a chunk's
+// writes land below every entry a later chunk still has to read.
+constexpr int kPackThreads = 256;
+
+__global__ void __launch_bounds__(kPackThreads)
+    pack_segments_kernel(float* __restrict__ val, int32_t* __restrict__ lab, int64_t ld, int T, int k, int S,
+                         int cap, const uint32_t* __restrict__ cnt, const int32_t* __restrict__ row_over,
+                         int32_t* __restrict__ nv) {
+  const int t = blockIdx.x;
+  const int64_t row = static_cast<int64_t>(t) * ld;
+  int total = k;                                   // the same in every thread
+  for (int j = 1; j <= S; ++j) {
+    const int64_t c = static_cast<int64_t>(j - 1) * T + t;
+    const int64_t src = row + k + static_cast<int64_t>(j - 1) * cap;
+    const int n = row_over[c] ? k : static_cast<int>(min(cnt[c], static_cast<uint32_t>(cap)));
+    const int64_t dst = row + total;
+    if (src != dst) {
+      for (int c0 = 0; c0 < n; c0 += kPackThreads) {
+        const int e = c0 + static_cast<int>(threadIdx.x);
+        float v = 0.f;
+        int32_t l = -1;
+        if (e < n) {
+          v = val[src + e];
+          l = lab[src + e];
+        }
+        __syncthreads();
+        if (e < n) {
+          val[dst + e] = v;
+          lab[dst + e] = l;
+        }
+      }
+    }
+    total += n;
+  }
+  if (threadIdx.x == 0) nv[t] = total;
 }
 
-cudaError_t launch_merge_counts(const uint32_t* cnt, const int32_t* row_over, int T, int k, int cap, int32_t* nv,
-                                cudaStream_t st) {
+cudaError_t launch_pack_segments(float* val, int32_t* lab, int64_t ld, int T, int k, int S, int cap,
+                                 const uint32_t* cnt, const int32_t* row_over, int32_t* nv, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  merge_counts_kernel<<<(T + 255) / 256, 256, 0, st>>>(cnt, row_over, T, k, cap, nv);
+  pack_segments_kernel<<<T, kPackThreads, 0, st>>>(val, lab, ld, T, k, S, cap, cnt, row_over, nv);
   return cudaGetLastError();
 }
 

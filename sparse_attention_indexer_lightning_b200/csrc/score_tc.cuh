@@ -26,7 +26,7 @@
 //   warp 1      TMEM allocator + single-thread MMA issuer
 //   warps 2..   epilogue (4 warps for QG = 1, 16 for QG = 8: four per TMEM
 //               lane quadrant, two of the group's 8 queries each)
-// Pipelines: STAGES key buffers (full/empty mbarriers), 2 query-tile slots,
+// Pipelines: STAGES key buffers (full/empty mbarriers), BSLOTS query-tile slots,
 // 2 TMEM accumulators so the epilogue of unit i overlaps the MMA of unit i+1.
 // Every wait is bounded; a wait that runs out raises the library fault word
 // and the CTA drains its copies and MMAs before it frees TMEM and exits.
@@ -51,7 +51,12 @@ struct TcCfg {
   static constexpr int B_BYTES = BN * kDim * ESZ;
   static constexpr int B_HALF = BN * 128;
   static constexpr int PANELS = kDim * ESZ / 128;  // 2 (bf16) or 1 (fp8)
-  static constexpr int STAGES = (QG == 1) ? 6 : (FILTER ? 2 : (F8 ? 4 : 3));
+  static constexpr int STAGES = (QG == 1) ? 6 : (F8 ? 4 : 3);
+  // query-tile slots: 2 lets the next group's tile land during the current
+  // group's last MMAs; 1 frees its space for key stages (the bf16 filter form,
+  // whose candidate staging would otherwise leave room for 2 key stages: 3
+  // stages and 1 slot measured faster)
+  static constexpr int BSLOTS = (FILTER && !F8) ? 1 : 2;
   static constexpr int ACC = (QG == 1) ? 8 : 2;       // accumulator stages in TMEM
   static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
   static constexpr int TMEM_COLS = (ACC * ACC_COLS <= 32) ? 32
@@ -65,7 +70,7 @@ struct TcCfg {
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
   static constexpr int Q_PER_EPI_WARP = (QG + EPI_SETS - 1) / EPI_SETS;
   static constexpr size_t SMEM_A = size_t(STAGES) * A_BYTES;
-  static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
+  static constexpr size_t SMEM_B = size_t(BSLOTS) * B_BYTES;
   static constexpr size_t SMEM_BAR = 512;
   static constexpr size_t SMEM_HIST = (QG == 1) ? kHistBins * 4 : 0;  // per-row selection histogram
   // filter form: each epilogue warp stages up to SBUF candidates per query
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long long prev_bg = -1;
-      int bslot = 1;
+      int bslot = C::BSLOTS - 1;
       uint32_t bphase[2] = {0, 0};
       int issued[8];
       uint32_t issued_par[8];
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
         const int tile = up.tile, g = up.g, b = up.b;
         const long long bg = static_cast<long long>(b) * G + g;
         if (bg != prev_bg) {
-          bslot ^= 1;
+          bslot = (bslot + 1 == C::BSLOTS) ? 0 : bslot + 1;
           if (!mbar_wait(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
           b_par[bslot] = bphase[bslot];
           b_issued[bslot] = 1;
@@ -220,7 +225,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     long long prev_bg = -1;
-    int bslot = 1;
+    int bslot = C::BSLOTS - 1;
     uint32_t bphase[2] = {0, 0};
     const uint32_t a_base = smem_u32(sA);
     const uint32_t b_base = smem_u32(sB);
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
           if (ELECT) umma_commit_warp(&bars->bempty[bslot]);
           else if (lane == 0) umma_commit(&bars->bempty[bslot]);
         }
-        bslot ^= 1;
+        bslot = (bslot + 1 == C::BSLOTS) ? 0 : bslot + 1;
         if (!warp_wait(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
         bphase[bslot] ^= 1;
         prev_bg = bg;
@@ -316,7 +321,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
       for (uint32_t e = lane; e < fcnt[i]; e += 32) {
         const uint32_t slot = base + e;
         if (slot < static_cast<uint32_t>(p.cand_cap)) {
-          const int64_t at = frow[i] * p.ld_cand + p.run_k + slot;
+          const int64_t at = frow[i] * p.ld_cand + slot;
           p.cand_val[at] = bv[e];
           p.cand_lab[at] = bl[e];
         } else {
@@ -366,9 +371,9 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
             if (!filter) {
               orow[jq] = p.out + row * p.ld_out + p.out_col0;
             } else {
-              // the row's running k-th entry; a list with padding takes every eligible key
-              const int64_t kth = row * p.ld_cand + p.run_k - 1;
-              thr[jq] = (p.cand_lab[kth] < 0) ? 0u : order_code(p.cand_val[kth]) + 1u;
+              // the row's threshold entry; a list with padding takes every eligible key
+              const int64_t kth = row * p.ld_kth;
+              thr[jq] = (p.kth_lab[kth] < 0) ? 0u : order_code(p.kth_val[kth]) + 1u;
               frow[jq] = row;
             }
           }

@@ -44,8 +44,8 @@ def test_every_declared_symbol_is_exported(lib):
 def test_version_and_workspace_queries(lib):
     assert lib.ls_version() == 100
     assert lib.ls_decode_select_workspace_size(64, 32768) == 64 * 32768 * 4   # the score rows only
-    # one 8192-key tile of scores plus running lists of k + 3k entries (values and labels)
-    assert lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 0) >= 4096 * 8192 * 4 + 4096 * 2048 * 8
+    # one 8192-key tile of scores plus lists of k + 2k entries per later tile (values and labels)
+    assert lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 0) >= 4096 * 8192 * 4 + 4096 * (512 + 3 * 1024) * 8
     assert lib.ls_prefill_select_workspace_size(4096, 8192, 8192, 512, 0) < 4096 * 8192 * 4 + 4096 * 64
     # full_scores: the whole T x N matrix
     assert lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 1) >= 4096 * 32768 * 4
