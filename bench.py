@@ -102,7 +102,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 break
-            time.sleep(0.0005)
+            time.sleep(0.0001)
 
     def stop(self):
         if self._nvml is None:

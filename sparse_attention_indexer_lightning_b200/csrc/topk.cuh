@@ -497,13 +497,16 @@ __device__ unsigned long long radix_select_cand(SH& sh, int nc, uint32_t want) {
 // NT threads, largest k KMAX, CAP listed candidates: <1024, 4096, 8192> one
 // CTA per SM; <512, 1024, 8192> two; <256, 512, 2048> four (rows of many
 // queries with k <= 512: more rows in flight hide the per-row latency).
-template <int NT, int KMAX, int CAP>
+// LOOP: the CTAs walk the rows (launches with row flags, where most rows are
+// left untouched); otherwise one CTA per row.
+template <int NT, int KMAX, int CAP, bool LOOP>
 __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
   TopkShared<NT, KMAX, CAP>& sh = *reinterpret_cast<TopkShared<NT, KMAX, CAP>*>(topk_smem);
-  const int r = blockIdx.x;
   if (p.run_if != nullptr && *p.run_if == 0) return;      // conditional launch with nothing to do
-  if (p.row_flag != nullptr && p.row_flag[r] == 0) return;  // row left untouched
+  // rows blockIdx.x, blockIdx.x + gridDim.x, ... (LOOP), else row blockIdx.x
+  for (int r = blockIdx.x; r < p.R; r += (LOOP ? gridDim.x : p.R)) {
+  if (p.row_flag != nullptr && p.row_flag[r] == 0) continue;  // row left untouched
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   RowRef rr;
@@ -831,17 +834,26 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
     io[j] = -1;
     if (vo) vo[j] = neg_inf();
   }
+  if (LOOP) __syncthreads();  // the next row reuses the shared block
+  }
 }
 
 template <int NT, int KMAX, int CAP>
-static cudaError_t launch_topk_t(const TopkParams& p, cudaStream_t st) {
+static cudaError_t launch_topk_t(const TopkParams& p, cudaStream_t st, int num_sms) {
   using SH = TopkShared<NT, KMAX, CAP>;
-  static std::atomic<uint64_t> attr_done{0};
+  // flagged launches walk the rows with at most as many CTAs as fit the SMs
+  // at once, so a launch with few (or no) flagged rows costs one wave
+  constexpr int kCtasPerSm = (NT == 256) ? 4 : 1024 / NT;
+  const bool loop = p.row_flag != nullptr && p.R > num_sms * kCtasPerSm;
+  static std::atomic<uint64_t> attr_done[2] = {{0}, {0}};
+  const void* fn = loop ? reinterpret_cast<const void*>(&topk_kernel<NT, KMAX, CAP, true>)
+                        : reinterpret_cast<const void*>(&topk_kernel<NT, KMAX, CAP, false>);
   {
-    const cudaError_t e = smem_limit_once(attr_done, reinterpret_cast<const void*>(&topk_kernel<NT, KMAX, CAP>), sizeof(SH));
+    const cudaError_t e = smem_limit_once(attr_done[loop ? 1 : 0], fn, sizeof(SH));
     if (e != cudaSuccess) return e;
   }
-  topk_kernel<NT, KMAX, CAP><<<p.R, NT, sizeof(SH), st>>>(p);
+  if (loop) topk_kernel<NT, KMAX, CAP, true><<<num_sms * kCtasPerSm, NT, sizeof(SH), st>>>(p);
+  else topk_kernel<NT, KMAX, CAP, false><<<p.R, NT, sizeof(SH), st>>>(p);
   return cudaGetLastError();
 }
 
@@ -850,9 +862,9 @@ static cudaError_t launch_topk_t(const TopkParams& p, cudaStream_t st) {
 // 1024-thread CTA per row.
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t st, int num_sms) {
   if (p.R == 0) return cudaSuccess;
-  if (p.k <= 512 && p.R >= 2 * num_sms) return launch_topk_t<256, 512, 2048>(p, st);
-  if (p.k <= 1024 && p.R > num_sms) return launch_topk_t<512, 1024, kCandCap>(p, st);
-  return launch_topk_t<1024, kMaxTopK, kCandCap>(p, st);
+  if (p.k <= 512 && p.R >= 2 * num_sms) return launch_topk_t<256, 512, 2048>(p, st, num_sms);
+  if (p.k <= 1024 && p.R > num_sms) return launch_topk_t<512, 1024, kCandCap>(p, st, num_sms);
+  return launch_topk_t<1024, kMaxTopK, kCandCap>(p, st, num_sms);
 }
 
 }  // namespace lsi

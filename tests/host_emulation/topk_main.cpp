@@ -4,6 +4,8 @@
 // block is allocated at exactly the kernel's size so AddressSanitizer sees its
 // end.  Test infrastructure only.
 //   DIR FORM R N k ld has_labels has_nvalid nv_offset label_base ld_out rows...
+//   (a negative first "row" -G instead runs a grid of G blocks over all rows
+//   with the row flags of flags.bin [R] i32: the flagged-launch form)
 //   FORM 0: <256, 512, 2048>   1: <512, 1024, 8192>   2: <1024, 4096, 8192>
 //   (scores.bin [R][ld] f32, labels.bin [R][ld] i32, nvalid.bin [R] i32)
 //   -> idx.bin, val.bin [R][ld_out]
@@ -44,10 +46,10 @@ static void save(const char* dir, const char* name, const std::vector<T>& v) {
 }
 
 template <int NT, int KMAX, int CAP>
-static void run_rows(const lsi::TopkParams& p, const std::vector<int>& rows) {
+static void run_rows(const lsi::TopkParams& p, const std::vector<int>& rows, int grid) {
   using SH = lsi::TopkShared<NT, KMAX, CAP>;
   blockDim = {static_cast<unsigned>(NT), 1, 1};
-  gridDim = {static_cast<unsigned>(p.R), 1, 1};
+  gridDim = {static_cast<unsigned>(grid > 0 ? grid : p.R), 1, 1};
   std::vector<std::barrier<>*> wb;
   for (int w = 0; w < NT / 32; ++w) g_warp_bar[w] = new std::barrier<>(32);
   for (int r : rows) {
@@ -62,7 +64,8 @@ static void run_rows(const lsi::TopkParams& p, const std::vector<int>& rows) {
       th.emplace_back([&, t] {
         threadIdx = {static_cast<unsigned>(t), 0, 0};
         blockIdx = {static_cast<unsigned>(r), 0, 0};
-        lsi::topk_kernel<NT, KMAX, CAP>(p);
+        if (grid > 0) lsi::topk_kernel<NT, KMAX, CAP, true>(p);
+        else lsi::topk_kernel<NT, KMAX, CAP, false>(p);
       });
     for (auto& x : th) x.join();
     std::free(smem);
@@ -80,7 +83,13 @@ int main(int argc, char** argv) {
   const int nv_offset = std::atoi(argv[9]), label_base = std::atoi(argv[10]);
   const long long ld_out = std::atoll(argv[11]);
   std::vector<int> rows;
+  int grid = 0;
   for (int i = 12; i < argc; ++i) rows.push_back(std::atoi(argv[i]));
+  if (!rows.empty() && rows[0] < 0) {
+    grid = -rows[0];
+    rows.clear();
+    for (int b = 0; b < grid; ++b) rows.push_back(b);
+  }
   // the inputs live in exactly-sized heap blocks, so reads past a row's end
   // or the array's end are reported
   auto sc = load<float>(dir, "scores.bin", static_cast<size_t>(R) * ld);
@@ -103,9 +112,14 @@ int main(int argc, char** argv) {
   p.idx_out = idx.data();
   p.val_out = val.data();
   p.ld_out = ld_out;
-  if (form == 0) run_rows<256, 512, 2048>(p, rows);
-  else if (form == 1) run_rows<512, 1024, 8192>(p, rows);
-  else run_rows<1024, 4096, 8192>(p, rows);
+  std::vector<int32_t> flags;
+  if (grid > 0) {
+    flags = load<int32_t>(dir, "flags.bin", static_cast<size_t>(R));
+    p.row_flag = flags.data();
+  }
+  if (form == 0) run_rows<256, 512, 2048>(p, rows, grid);
+  else if (form == 1) run_rows<512, 1024, 8192>(p, rows, grid);
+  else run_rows<1024, 4096, 8192>(p, rows, grid);
   save(dir, "idx.bin", idx);
   save(dir, "val.bin", val);
   return 0;

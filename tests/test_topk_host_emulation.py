@@ -78,15 +78,19 @@ def topk_host(tmp_path_factory):
     assert r.returncode == 0, r.stderr[-3000:]
     env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
 
-    def run(form, scores, labels, n_valid, k):
+    def run(form, scores, labels, n_valid, k, flags=None, grid=0):
         R, ld = scores.shape
         scores.astype(np.float32).tofile(d / "scores.bin")
         if labels is not None:
             labels.astype(np.int32).tofile(d / "labels.bin")
         if n_valid is not None:
             n_valid.astype(np.int32).tofile(d / "nvalid.bin")
+        rows = [str(r) for r in range(R)]
+        if flags is not None:
+            flags.astype(np.int32).tofile(d / "flags.bin")
+            rows = [str(-grid)]
         cmd = [str(exe), str(d), str(form), str(R), str(ld), str(k), str(ld), str(int(labels is not None)),
-               str(int(n_valid is not None)), "0", "0", str(k)] + [str(r) for r in range(R)]
+               str(int(n_valid is not None)), "0", "0", str(k)] + rows
         r = subprocess.run(cmd, capture_output=True, text=True, env=env, timeout=300)
         assert r.returncode == 0, r.stderr[-3000:]
         return (np.fromfile(d / "idx.bin", dtype=np.int32).reshape(R, k),
@@ -176,3 +180,23 @@ def test_host_topk_merge_rows(topk_host):
     want = _expect(sc, lab, nv, k)
     for _ in range(3):
         _check(topk_host(0, sc, lab, nv, k), want)
+
+
+def test_host_topk_flagged_rows_grid_stride(topk_host):
+    """A launch with row flags walks the rows with fewer CTAs than rows: the
+    flagged rows get their top-k, the others are left as they were."""
+    k = 64
+    rng = np.random.default_rng(11)
+    R, ld = 13, 700
+    sc = np.stack([_row(rng, ld, ("normal", "ties", "coarse")[r % 3]) for r in range(R)])
+    nv = rng.integers(0, ld + 1, R).astype(np.int32)
+    flags = (rng.random(R) < 0.5).astype(np.int32)
+    flags[0], flags[R - 1] = 1, 1
+    gi, gv = topk_host(0, sc, None, nv, k, flags=flags, grid=4)
+    wi, wv = _expect(sc, None, nv, k)
+    for r in range(R):
+        if flags[r]:
+            assert np.array_equal(gi[r], wi[r])
+            assert np.array_equal(gv[r].view(np.uint32), wv[r].astype(np.float32).view(np.uint32))
+        else:
+            assert np.all(gi[r] == 777)          # untouched
