@@ -728,18 +728,30 @@ def bench_attention(L, args, peaks, peak_kind):
         L.ls_sparse_attention(q, lat, sets[i % len(sets)], out=out)
         return None
 
+    def run_cc(i, timed):
+        L.ls_sparse_attention(q, lat, sets[i % len(sets)], out=out, cuda_cores=True)
+        return None
+
     ms, kern = _profiled_loop(L, run, steps, warm, st)
-    kms = kern["sparse_attn_kernel"]["ms_per_step"]
+    kname = "sparse_attn_tc_kernel" if "sparse_attn_tc_kernel" in kern else "sparse_attn_kernel"
+    kms = kern[kname]["ms_per_step"]
+    ms_cc, kern_cc = _profiled_loop(L, run_cc, steps, warm, st)
     flops = T * H * wl.k * (D + 512) * 2
     gathered = T * wl.k * D * 2
     peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    peak_t = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
     res = {"ms_per_step": ms, "positions_per_s": T * wl.k / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
            "kernels": kern,
-           "roofline": roofline("alu", flops / (kms * 1e-3) / 1e12, round(ALU_FP32_TFLOPS, 1), "TFLOP/s",
-                                peak_kind="derived: fp32 FMA issue rate at clocks.max.sm"),
+           "roofline": roofline("tensor", flops / (kms * 1e-3) / 1e12, peak_t, "TFLOP/s",
+                                peak_kind=peak_kind),
            "gather_hbm_frac": round(gathered / (kms * 1e-3) / 1e9 / peak_b, 4),
-           "note": "positions = selected rows attended per step; flops = T x H x k x (576 + 512) x 2 "
-                   "(logits and values); CUDA-core kernel"}
+           "cuda_core_kernel": {"ms_per_step": ms_cc, "kernels": kern_cc,
+                                "alu_frac": round(flops / (kern_cc["sparse_attn_kernel"]["ms_per_step"] * 1e-3)
+                                                  / 1e12 / ALU_FP32_TFLOPS, 4)},
+           "note": "positions = selected rows attended per step; flops = T x H x k x (576 + 512) x 2 (logits and "
+                   "values, counted once; the tensor-core kernel computes the logits in both CTAs of a query); "
+                   "tensor-core kernel (bf16 weights in the value contraction), the fp32 CUDA-core kernel timed "
+                   "beside it on the same selections"}
     del sets, q, lat, out
     return res
 

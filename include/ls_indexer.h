@@ -355,6 +355,7 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
                           int k, int32_t* idx_out, float* val_out, void* ws, size_t ws_bytes, void* stream);
 
 #define LS_ATTN_FOREIGN_ROWS 1   /* ls_sparse_attention: rows outside [0, n_rows) are another shard's */
+#define LS_ATTN_CUDA_CORES 2     /* ls_sparse_attention: take the CUDA-core kernel even where the tensor-core one applies */
 
 /*
  * ls_sparse_attention -- sparse main attention over the selected rows, stage
@@ -379,7 +380,13 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
  *        not fix it)
  *   flags: 0, or LS_ATTN_FOREIGN_ROWS when latent holds one shard of the
  *        rows (row_off = -first row of the shard, n_rows = its length): rows
- *        outside it belong to other shards and are skipped without the fault
+ *        outside it belong to other shards and are skipped without the fault;
+ *        LS_ATTN_CUDA_CORES forces the CUDA-core kernel (below)
+ * Kernels: H a multiple of 128 and k <= 512 run on the tensor cores (tcgen05:
+ *        logits and the value contraction as MMAs, the weights rounded to
+ *        bf16 for the value contraction, so an output is within 2^-8 of the
+ *        largest selected value magnitude; lse in fp32); other shapes, or
+ *        LS_ATTN_CUDA_CORES, take the fp32 CUDA-core kernel (within 1e-4).
  *   out [T][H][512] fp32; lse [T][H] fp32 natural-log sum or NULL.  An empty
  *        selection gives out = 0 and lse = -inf; partial results over
  *        disjoint selections combine exactly by their lse (online softmax).

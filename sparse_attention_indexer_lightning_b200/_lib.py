@@ -30,6 +30,8 @@ LS_KEY_FP8_E4M3 = 1
 LS_KEY_INT8 = 2
 LS_FAULT_WAIT_TIMEOUT = 1
 LS_FAULT_BAD_INDEX = 2
+LS_ATTN_FOREIGN_ROWS = 1
+LS_ATTN_CUDA_CORES = 2
 
 EXPORTED = (
     "ls_last_error", "ls_version", "ls_device_status", "ls_indexer_score", "ls_topk_select",
@@ -538,18 +540,18 @@ def ls_merge_select(vals, idx, offsets, k: int = 512, ws=None, out=None, stream=
     return io, vo
 
 
-LS_ATTN_FOREIGN_ROWS = 1
 
 
 def ls_sparse_attention(q, latent, idx, scale: Optional[float] = None, row_off=None, want_lse: bool = True,
-                        out=None, foreign_rows: bool = False, stream=None):
+                        out=None, foreign_rows: bool = False, cuda_cores: bool = False, stream=None):
     """Sparse main attention over the selected latent rows.
 
     q [T,H,576] bf16, latent [R,576] bf16, idx [T,k] int32 (-1 = unused slot),
     row_off [T] int64 or None (row = idx + row_off[t]); scale defaults to
     1/sqrt(576) -> (out [T,H,512] f32, lse [T,H] f32 or None).  With
     ``foreign_rows`` latent holds one shard of the rows (row_off = -its first
-    row) and rows outside it are skipped as another shard's."""
+    row) and rows outside it are skipped as another shard's.  ``cuda_cores``
+    forces the fp32 CUDA-core kernel where the tensor-core one would run."""
     _dev(q, torch.bfloat16, "q", 3)
     _dev(latent, torch.bfloat16, "latent", 2)
     _dev(idx, torch.int32, "idx", 2)
@@ -567,7 +569,8 @@ def ls_sparse_attention(q, latent, idx, scale: Optional[float] = None, row_off=N
         out = torch.empty((T, H, 512), dtype=torch.float32, device=q.device)
     lse = torch.empty((T, H), dtype=torch.float32, device=q.device) if want_lse else None
     _check(lib().ls_sparse_attention(_ptr(q), _ptr(latent), _ptr(idx), _ptr(row_off), T, H, d, 512, R, k, float(scale),
-                                     LS_ATTN_FOREIGN_ROWS if foreign_rows else 0, _ptr(out), _ptr(lse),
+                                     (LS_ATTN_FOREIGN_ROWS if foreign_rows else 0)
+                                     | (LS_ATTN_CUDA_CORES if cuda_cores else 0), _ptr(out), _ptr(lse),
                                      _stream(stream)))
     return out, lse
 

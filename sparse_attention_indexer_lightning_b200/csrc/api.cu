@@ -23,6 +23,7 @@
 #include "score_tree.cuh"
 #include "merge.cuh"
 #include "sparse_attn.cuh"
+#include "sparse_attn_tc.cuh"
 #include "score_q8.cuh"
 #include "score_tc.cuh"
 #include "topk.cuh"
@@ -203,6 +204,22 @@ ls_status make_vec64_map(CUtensorMap* m, const void* base, uint64_t rows, uint32
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(kLsaDim), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLsaDim * 2)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(kLsaDim), box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LS_OK;
+}
+
+// 2-D bf16 map over the latent / query rows [rows][576], box = 64 elements x
+// box_rows, 128-byte swizzle (one 128-byte panel of box_rows rows per copy).
+ls_status make_latent_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kAttnLatent), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kAttnLatent * 2)};
+  cuuint32_t box[2] = {64u, box_rows};
   cuuint32_t es[2] = {1u, 1u};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1296,7 +1313,7 @@ ls_status ls_merge_select(const float* vals, const int32_t* idx, const int32_t* 
 ls_status ls_sparse_attention(const uint16_t* q, const uint16_t* latent, const int32_t* idx, const int64_t* row_off,
                               int T, int H, int d, int d_v, int64_t n_rows, int k, float scale, int flags, float* out,
                               float* lse, void* stream) {
-  LS_CHECK_ARG((flags & ~LS_ATTN_FOREIGN_ROWS) == 0, "unknown flags 0x%x", flags);
+  LS_CHECK_ARG((flags & ~(LS_ATTN_FOREIGN_ROWS | LS_ATTN_CUDA_CORES)) == 0, "unknown flags 0x%x", flags);
   LS_CHECK_ARG(T >= 0 && H >= 0 && k >= 0 && n_rows >= 0, "negative size (T=%d H=%d k=%d)", T, H, k);
   if (d != kAttnLatent || d_v != kAttnValue)
     return fail(LS_ERR_UNSUPPORTED, "latent rows of %d elements with %d value elements are built (got d=%d d_v=%d)",
@@ -1313,9 +1330,18 @@ ls_status ls_sparse_attention(const uint16_t* q, const uint16_t* latent, const i
   LS_CHECK_ARG(aligned16(q) && aligned16(out) && (!latent || aligned16(latent)),
                "q, latent and out must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int foreign_ok = (flags & LS_ATTN_FOREIGN_ROWS) ? 1 : 0;
+  if (H % kTcHeads == 0 && k <= kTcMaxK && n_rows > 0 && !(flags & LS_ATTN_CUDA_CORES)) {
+    // groups of 128 heads over at most 512 slots: the tensor-core kernel
+    CUtensorMap qmap;
+    ls_status s = make_latent_map(&qmap, q, static_cast<uint64_t>(T) * H, kTcHeads);
+    if (s != LS_OK) return s;
+    ProfScope prof("sparse_attn_tc_kernel", st);
+    LS_CUDA(launch_sparse_attn_tc(&qmap, latent, idx, row_off, T, H, k, n_rows, scale, foreign_ok, out, lse, st));
+    return LS_OK;
+  }
   ProfScope prof("sparse_attn_kernel", st);
-  LS_CUDA(launch_sparse_attn(q, latent, idx, row_off, T, H, k, n_rows, scale, (flags & LS_ATTN_FOREIGN_ROWS) ? 1 : 0,
-                             out, lse, st));
+  LS_CUDA(launch_sparse_attn(q, latent, idx, row_off, T, H, k, n_rows, scale, foreign_ok, out, lse, st));
   return LS_OK;
 }
 

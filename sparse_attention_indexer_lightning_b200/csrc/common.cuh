@@ -265,6 +265,15 @@ __device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
+// Close the group of cp.async copies this thread issued since the last one.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // The mbarrier gets one more pending arrival now, and receives it once every
 // cp.async this thread issued so far has landed.
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
@@ -334,6 +343,21 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   uint64_t desc = 0;
   desc |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
   desc |= static_cast<uint64_t>(1) << 16;
+  desc |= static_cast<uint64_t>(1024 >> 4) << 32;
+  desc |= static_cast<uint64_t>(1) << 46;
+  desc |= static_cast<uint64_t>(2) << 61;
+  return desc;
+}
+
+// Shared-memory matrix descriptor for an MN-major operand under the 128-byte
+// swizzle: atoms of 64 MN-elements (128 B, 16-bit types) x 8 K-rows, rows
+// 128 B apart inside an atom (the same bytes as a K-major SW128 staging of
+// the K-rows); `lbo` = bytes between atoms along MN, 1024 between atoms
+// along K.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
+  desc |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
   desc |= static_cast<uint64_t>(1024 >> 4) << 32;
   desc |= static_cast<uint64_t>(1) << 46;
   desc |= static_cast<uint64_t>(2) << 61;

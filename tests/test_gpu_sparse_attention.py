@@ -11,6 +11,15 @@ inputs (logits of standard deviation about 2), so the bound checked is
 |lse - lse_ref| <= 1e-4 * (1 + |lse_ref|).  A missed or doubled row moves an
 output by about its weight (>= 1e-3 here), a wrong scale or value slice far
 more.
+
+Groups of 128 heads over at most 512 slots run on the tensor cores, where
+the weights enter the value contraction rounded to bf16 (relative error at
+most 2^-9 each; dividing by the sum of the rounded weights keeps them a
+convex combination, so each weight is off by at most 2 * 2^-9 of itself):
+there the output bound is |o - o_ref| <= 2^-8 * max |value|, and, sharper,
+within 2e-3 * max |value| of the same attention with the oracle's weights
+rounded to bf16 (fp32 logits can move a weight across a rounding boundary).
+lse keeps the 1e-4 bound (it is computed from the unrounded fp32 weights).
 """
 
 import functools
@@ -28,6 +37,12 @@ from workloads.synth import make_attention, make_decode
 pytestmark = pytest.mark.gpu
 
 ATTN_TOL = 1e-4
+ATTN_TOL_TC = 2.0 ** -8
+ATTN_TOL_TC_EMUL = 2e-3
+
+
+def _on_tensor_cores(H, k):
+    return H % 128 == 0 and k <= 512
 
 
 @pytest.fixture(scope="module")
@@ -45,12 +60,34 @@ def data(name):
     return make_workload(name)
 
 
+def _bf16_weight_attention(q, lat, gidx, scale):
+    """The attention with each weight exp(logit - max) rounded to fp32 and then
+    to bf16 (nearest even) before the weighted sum and its normalisation:
+    the tensor-core kernel's rounding applied to the fp64 logits (test-side
+    emulation, not the oracle)."""
+    out = np.zeros((q.shape[0], q.shape[1], 512))
+    for t in range(q.shape[0]):
+        sel = gidx[t][gidx[t] >= 0]
+        if sel.size == 0:
+            continue
+        c = lat[sel]
+        lg = scale * (q[t] @ c.T)
+        p = np.exp(lg - lg.max(axis=1, keepdims=True)).astype(np.float32)
+        pb = (torch.from_numpy(p).to(torch.bfloat16).to(torch.float64)).numpy()
+        out[t] = (pb @ c[:, :512]) / pb.sum(axis=1, keepdims=True)
+    return out
+
+
 def _check(out, lse, q_bits, lat_bits, gidx, scale, rows=None, what=""):
     """Compare queries `rows` (all by default) of the GPU result with the oracle;
-    gidx holds latent row ids (-1 = unused)."""
+    gidx holds latent row ids (-1 = unused).  The tolerance follows the path
+    the call took (see the module docstring)."""
     rows = range(q_bits.shape[0]) if rows is None else rows
     rows = list(rows)
+    tc = _on_tensor_cores(q_bits.shape[1], gidx.shape[1])
+    tol = ATTN_TOL_TC if tc else ATTN_TOL
     ro, rl = sparse_attention(bf16_to_f64(q_bits[rows]), bf16_to_f64(lat_bits), gidx[rows], scale)
+    re = _bf16_weight_attention(bf16_to_f64(q_bits[rows]), bf16_to_f64(lat_bits), gidx[rows], scale) if tc else None
     for i, t in enumerate(rows):
         sel = gidx[t][gidx[t] >= 0]
         if sel.size == 0:
@@ -59,7 +96,10 @@ def _check(out, lse, q_bits, lat_bits, gidx, scale, rows=None, what=""):
             continue
         vmax = np.abs(bf16_to_f64(lat_bits[sel, :512])).max()
         err = np.abs(out[t] - ro[i]).max()
-        assert err <= ATTN_TOL * vmax, f"{what} t={t}: output error {err:.3e} > {ATTN_TOL * vmax:.3e}"
+        assert err <= tol * vmax, f"{what} t={t}: output error {err:.3e} > {tol * vmax:.3e}"
+        if tc:
+            err = np.abs(out[t] - re[i]).max()
+            assert err <= ATTN_TOL_TC_EMUL * vmax, f"{what} t={t}: error {err:.3e} against bf16 weights"
         lerr = np.abs(lse[t] - rl[i])
         assert np.all(lerr <= ATTN_TOL * (1 + np.abs(rl[i]))), f"{what} t={t}: lse error {lerr.max():.3e}"
 
@@ -230,3 +270,51 @@ def test_sparse_attention_full_size_sampled(L):
     out, lse = _run(L, d)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
     _check(out, lse, d["q"], d["latent"], d["idx"], default_scale(), rows=[0, 17, 40, 63], what="attn_decode")
+
+
+def test_sparse_attention_tensor_cores(L):
+    """The tensor-core path: 128 and 256 heads, k from 1 to 512 (not multiples
+    of the 32- and 64-slot chunks), empty queries, unused slots at the tail and
+    scattered, a row offset per query, and attention over two disjoint halves
+    merged by their lse."""
+    for T, H, N, k, scale in ((3, 128, 3000, 512, None), (2, 128, 700, 1, 0.3), (2, 256, 4000, 300, None),
+                              (3, 128, 5000, 33, 0.05), (2, 128, 2000, 97, None)):
+        d = make_attention(T, H, N, k, seed=7 * T + k + H)
+        idx = d["idx"].copy()
+        if T > 2:
+            idx[0, :] = -1                                # an empty query
+            idx[1, ::3] = -1                              # scattered unused slots
+        out, lse = _run(L, d, scale=scale, idx=idx)
+        _check(out, lse, d["q"], d["latent"], idx, default_scale() if scale is None else scale,
+               what=f"tc T={T} H={H} k={k}")
+    d = make_attention(3, 128, 6000, 512, seed=99)
+    off = np.array([0, 100, 2500], dtype=np.int64)
+    idx = np.where(d["idx"] >= 0, d["idx"] % 3000, -1).astype(np.int32)
+    out, lse = _run(L, d, idx=idx, row_off=off)
+    _check(out, lse, d["q"], d["latent"], np.where(idx >= 0, idx + off[:, None], -1), default_scale(),
+           what="tc row_off")
+    a = idx.copy()
+    a[:, 200:] = -1
+    b = idx.copy()
+    b[:, :200] = -1
+    oa, la = _run(L, d, idx=a, row_off=off)
+    ob, lb = _run(L, d, idx=b, row_off=off)
+    om, lm = merge_partials(oa.astype(np.float64), la.astype(np.float64), ob.astype(np.float64),
+                            lb.astype(np.float64))
+    vmax = np.abs(bf16_to_f64(d["latent"][:, :512])).max()
+    assert np.abs(om - out).max() <= 2 * ATTN_TOL_TC * vmax
+    assert np.all(np.abs(lm - lse) <= ATTN_TOL * (1 + np.abs(lse)))
+
+
+def test_sparse_attention_tensor_cores_match_cuda_cores(L):
+    """Both kernels on the same 128-head inputs: lse agree to fp32 rounding,
+    outputs within the tensor-core bound of each other."""
+    d = make_attention(4, 128, 6000, 512, seed=5)
+    q, lat, idx = dev_bf16(d["q"]), dev_bf16(d["latent"]), dev(d["idx"])
+    ot, lt = L.ls_sparse_attention(q, lat, idx)
+    oc, lc = L.ls_sparse_attention(q, lat, idx, cuda_cores=True)
+    torch.cuda.synchronize()
+    ot, lt, oc, lc = (x.cpu().numpy() for x in (ot, lt, oc, lc))
+    vmax = np.abs(bf16_to_f64(d["latent"][:, :512])).max()
+    assert np.abs(ot - oc).max() <= ATTN_TOL_TC * vmax
+    assert np.all(np.abs(lt - lc) <= ATTN_TOL * (1 + np.abs(lc)))
