@@ -34,7 +34,9 @@ Pipelines:
 * LSA tree search, one node level ("Latent Sparse Attention", "The tree, step
   by step"): node buckets group 4 buckets of a complete 4096-bucket block;
   the beam keeps the best node buckets, the search steps down to their
-  children plus the uncovered buckets and picks the top-p there.
+  children plus the uncovered buckets and picks the top-p there.  Several
+  levels: the beam starts at the lowest level with at most 32768 node
+  buckets and steps down one level at a time the same way.
 * bucket search ("Latent Sparse Attention", "How LSA finds the keys" and "The
   method, term by term", steps 5-6): score every bucket centroid with the
   indexer score, keep the top-p buckets, read them best first appending their
@@ -304,6 +306,67 @@ def lsa_tree_select(q_idx_bits, q_pos, centroid_bits, node_bits, bucket_off, buc
         out.append(lsa_read_list(picked, q_pos[t], bucket_off, bucket_mem, block_keys, n_sink, budget))
         detail.append({"node_scores": node_scores, "beam": kept, "visible_nodes": vn, "candidates": cand,
                        "scores": scores, "picked": picked, "visible": v})
+    if return_detail:
+        return out, detail
+    return out
+
+
+def lsa_tree_levels(vis_buckets: int, level_sizes, node_block: int, fanout: int):
+    """Visible entries of every level for a query that sees ``vis_buckets``
+    buckets: level l's nodes exist for the complete node blocks of level
+    l - 1 ("Latent Sparse Attention", "The tree, step by step": every
+    node_block entries of a level form a node cluster block, grouped fanout to
+    a node of the level above)."""
+    v = [int(vis_buckets)]
+    for size in level_sizes:
+        v.append(min(int(size), (v[-1] // node_block) * (node_block // fanout)))
+    return v
+
+
+def lsa_tree_levels_select(q_idx_bits, q_pos, centroid_bits, level_bits, bucket_off, bucket_mem, block_keys: int,
+                           buckets_per_block: int, node_block: int, fanout: int, beam: int, start_nodes: int,
+                           n_sink: int, top_p: int, budget: int, rows=None, return_detail: bool = False):
+    """Read lists of the LSA tree search over several levels of node buckets
+    ("Latent Sparse Attention", "The tree, step by step"): node n of level l
+    covers entries fanout*n .. fanout*n + fanout - 1 of level l - 1 (level 0:
+    the buckets).  The beam starts at the lowest level with at most
+    ``start_nodes`` node buckets (the top level if none has so few) and
+    scores every visible node there, keeps the best ``beam``; at each level
+    below it scores the kept nodes' children plus the level's visible entries
+    no node above covers, keeps the best ``beam`` again; at the bucket level it
+    picks the top-p of the last beam's children and the uncovered buckets,
+    which are read as in the flat search.  ``level_bits``: the node centroids
+    of levels 1..L (bf16 bits), L >= 1."""
+    T = q_idx_bits.shape[0]
+    P = centroid_bits.shape[0]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    levels = [centroid_bits] + list(level_bits)
+    sizes = [lv.shape[0] for lv in levels]
+    L = len(level_bits)
+    assert L >= 1
+    start = next((lv for lv in range(1, L + 1) if sizes[lv] <= start_nodes), L)
+    vis = lsa_visible(q_pos, block_keys, buckets_per_block, P)
+    out, detail = [], []
+    for t in rows:
+        v = lsa_tree_levels(vis[t], sizes[1:], node_block, fanout)
+        qv = bf16_to_f64(q_idx_bits[t])
+        beams, counts = {}, {}
+        for lv in range(start, -1, -1):
+            if lv == start:                                  # every visible node of the start level
+                cand = np.arange(v[start], dtype=np.int64)
+            else:                                            # children of the beam, then the uncovered entries
+                cand = np.asarray([fanout * int(n) + c for n in beams[lv + 1] for c in range(fanout)]
+                                  + list(range(fanout * v[lv + 1], v[lv])), dtype=np.int64)
+            scores = bf16_to_f64(levels[lv][cand]) @ qv if cand.size else np.zeros(0)
+            counts[lv] = int(cand.size)
+            if lv > 0:
+                kept, _ = select_topk(scores, cand, beam)
+                beams[lv] = kept[kept >= 0]
+            else:
+                picked, _ = select_topk(scores, cand, top_p)
+        out.append(lsa_read_list(picked, q_pos[t], bucket_off, bucket_mem, block_keys, n_sink, budget))
+        detail.append({"start": start, "visible": v, "beams": beams, "counts": counts, "candidates": cand,
+                       "scores": scores, "picked": picked})
     if return_detail:
         return out, detail
     return out

@@ -17,11 +17,11 @@ from oracle import brute, sizes
 from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64, f16_to_f64, pq_decode
 from oracle.indexer import eligible_blocks, eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, decode_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_select, lsa_visible,
-    prefill_select,
+    bucket_select, decode_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_levels_select,
+    lsa_tree_select, lsa_visible, prefill_select,
     prefill_select_fp8, recall_at_k, select_topk, topk_rows, two_stage_pq_select, two_stage_select,
 )
-from workloads import make_workload
+from workloads import get_workload, make_workload
 from workloads.synth import make_bucket, make_decode, make_two_stage, to_bf16_bits
 
 
@@ -478,6 +478,124 @@ def test_lsa_generator_node_centroids():
     for j in (0, 1, 511, 1023):
         s = (c[4 * j:4 * j + 4] * sizes[4 * j:4 * j + 4, None]).sum(axis=0)
         assert np.allclose(n[j], s / np.linalg.norm(s), atol=2 ** -8)
+
+
+def _levels_args(d, ex):
+    return (d["q_idx"], d["q_pos"], d["centroids"], d["node_levels"], d["bucket_off"], d["bucket_mem"],
+            ex["block_keys"], ex["bpb"], ex["node_block"], ex["fanout"])
+
+
+@pytest.mark.parametrize("start_nodes", [100, 500, 5000])
+def test_lsa_tree_levels_with_full_beam_equals_flat(start_nodes):
+    """A beam holding every visible entry of each level steps down to every
+    visible bucket, from whichever level it starts: the tree reads what the
+    flat search reads."""
+    wl = get_workload("lsa_tree_levels_s")
+    d = make_workload("lsa_tree_levels_s")
+    ex = wl.extra
+    flat = lsa_flat_select(d["q_idx"], d["q_pos"], d["centroids"], d["bucket_off"], d["bucket_mem"],
+                           ex["block_keys"], ex["bpb"], ex["n_sink"], wl.top_p, wl.budget)
+    tree, det = lsa_tree_levels_select(*_levels_args(d, ex), 5000, start_nodes, ex["n_sink"], wl.top_p, wl.budget,
+                                       return_detail=True)
+    assert det[0]["start"] == {100: 3, 500: 2, 5000: 1}[start_nodes]
+    for t in range(d["q_pos"].size):
+        assert np.array_equal(flat[t], tree[t]), t
+
+
+def test_lsa_tree_levels_one_level_equals_one_level_search():
+    """With one node level the search is the one-level tree search."""
+    wl = get_workload("lsa_flat_s")
+    d = make_workload("lsa_flat_s")
+    ex = wl.extra
+    args = (d["q_idx"], d["q_pos"], d["centroids"])
+    one = lsa_tree_select(*args, d["node_centroids"], d["bucket_off"], d["bucket_mem"], 512, 64, 4096, 4, 96, 4,
+                          64, 512)
+    lv = lsa_tree_levels_select(*args, [d["node_centroids"]], d["bucket_off"], d["bucket_mem"], 512, 64, 4096, 4,
+                                96, 32768, 4, 64, 512)
+    for t in range(d["q_pos"].size):
+        assert np.array_equal(one[t], lv[t]), t
+
+
+@pytest.mark.parametrize("start_nodes,beam", [(100, 5), (500, 7), (5000, 9)])
+def test_lsa_tree_levels_brute_force_tiny(start_nodes, beam):
+    """Pure-Python levels: the visible entries of a level are those whose
+    block of node_block entries below is complete and visible; an entry is
+    covered when its parent is visible; the start level is scored in full,
+    every level below over the beam's children and the uncovered entries."""
+    wl = get_workload("lsa_tree_levels_s")
+    d = make_workload("lsa_tree_levels_s")
+    ex = wl.extra
+    fan, blk = ex["fanout"], ex["node_block"]
+    lv_bits = [d["centroids"]] + d["node_levels"]
+    start = {100: 3, 500: 2, 5000: 1}[start_nodes]
+    rows = [t for t in range(d["q_pos"].size) if d["q_pos"][t] >= 9000][:5] + [4, 8, 11, 0]
+    out, det = lsa_tree_levels_select(*_levels_args(d, ex), beam, start_nodes, ex["n_sink"], wl.top_p, wl.budget,
+                                      rows=rows, return_detail=True)
+    for i, t in enumerate(rows):
+        q = bf16_to_f64(d["q_idx"][t:t + 1])[0].tolist()
+        vis = [min(int(d["q_pos"][t]) // 512 * 64, d["centroids"].shape[0])]
+        for lv in range(1, 4):
+            n_up = lv_bits[lv].shape[0]
+            # node n exists for the query when all of its block's entries below are visible
+            vis.append(sum(1 for n in range(n_up) if ((n * fan) // blk + 1) * blk <= vis[lv - 1]))
+        kept = None
+        for lv in range(start, -1, -1):
+            if kept is None:
+                cand = list(range(vis[lv]))
+            else:
+                cand = [c for c in range(vis[lv]) if c // fan in kept or c // fan >= vis[lv + 1]]
+            rows_f = bf16_to_f64(lv_bits[lv][cand]).tolist() if cand else []
+            sc = [sum(a * b for a, b in zip(r, q)) for r in rows_f]
+            k = beam if lv > 0 else wl.top_p
+            sel, _ = brute.topk(sc, cand, k)
+            sel = [x for x in sel if x >= 0]
+            if lv > 0:
+                assert sorted(det[i]["beams"][lv].tolist()) == sorted(sel), (t, lv)
+                kept = set(sel)
+            else:
+                assert [x for x in det[i]["picked"].tolist() if x >= 0] == sel, t
+        want = lsa_read_list(np.asarray(sel + [-1] * (wl.top_p - len(sel))), d["q_pos"][t], d["bucket_off"],
+                             d["bucket_mem"], 512, ex["n_sink"], wl.budget)
+        assert out[i].tolist() == want.tolist(), t
+
+
+def test_lsa_tree_levels_counts_match_page_figures(golden_dir):
+    """The beam rule replayed at 1M and 10M tokens: start level and the number
+    of vectors scored for a query that sees the whole index are the pages'."""
+    g = _golden(golden_dir)
+    rng = np.random.default_rng(5)
+    for key in ("lsa_tree_1m", "lsa_tree_10m"):
+        f = g[key]
+        P = f["tokens"] // 512 * 64
+        assert P == f["buckets"]
+        sizes_ = [P]
+        while len(sizes_) < 4:
+            sizes_.append(sizes_[-1] // f["node_block"] * (f["node_block"] // f["fanout"]))
+        bits = [to_bf16_bits(rng.standard_normal((n, 64)) * 0.1) for n in sizes_]
+        q = to_bf16_bits(rng.standard_normal((1, 64)))
+        off = np.zeros(P + 1, dtype=np.int32)
+        _, det = lsa_tree_levels_select(q, np.asarray([f["tokens"]]), bits[0], bits[1:], off,
+                                        np.zeros(0, dtype=np.int32), 512, 64, f["node_block"], f["fanout"],
+                                        f["beam"], f["start_nodes"], 4, 1024, 4096, return_detail=True)
+        assert det[0]["start"] == f["start_level"]
+        if "level1_nodes" in f:
+            assert sizes_[1] == f["level1_nodes"]
+        if "start_level_nodes" in f:
+            assert sizes_[f["start_level"]] == f["start_level_nodes"]
+        assert sum(det[0]["counts"].values()) == f["scored"], key
+
+
+def test_lsa_generator_node_levels():
+    """A level-2 node centroid is the normalised sum of the key sums of the 16
+    buckets beneath it (size x centroid each): the levels sum keys, not
+    normalised centroids."""
+    d = make_workload("lsa_tree_levels_s")
+    sizes_ = np.diff(d["bucket_off"]).astype(np.float64)
+    c = bf16_to_f64(d["centroids"])
+    n2 = bf16_to_f64(d["node_levels"][1])
+    for j in (0, 1, 100, 287):
+        s = (c[16 * j:16 * j + 16] * sizes_[16 * j:16 * j + 16, None]).sum(axis=0)
+        assert np.allclose(n2[j], s / np.linalg.norm(s), atol=2 ** -8)
 
 
 def test_two_stage_full_shortlist_equals_exact():

@@ -21,6 +21,12 @@ Five full-size workloads follow the shapes the pages use:
   centroids, 256 index queries, top 1024 buckets expanded to 4096 long-range
   keys plus 4 sinks and the window ("Latent Sparse Attention", "How LSA finds
   the keys").
+* ``lsa_tree_10m``  -- the tree search at 10485760 tokens: three node
+  levels over 1310720 buckets, 256 index queries ("Latent Sparse Attention",
+  "The tree, step by step").
+* ``lsa_prefill_10m`` -- the sampled-threshold flat search for one prefill
+  chunk of 32768 queries at 10485760 tokens ("Latent Sparse Attention",
+  "What the kernels do about the top-p").
 * ``bucket``        -- one sequence of 1048576 tokens (262144 keys) built as
   32768 clusters of 8 keys; 256 decode queries keep 64 buckets and expand them
   to 512 keys ("Latent Sparse Attention", "How LSA finds the keys").
@@ -120,6 +126,23 @@ WORKLOADS: Dict[str, Workload] = {
         extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "spread": 2053, "node_block": 4096, "fanout": 4,
                "beam": 2048},
     ),
+    # the tree at 10485760 tokens: 1310720 buckets under three node levels
+    # (327680, 81920, 20480 node buckets); the beam starts at level 3, the
+    # lowest with at most 32768 node buckets, and scores 20480 + 3 x 8192
+    # vectors per query ("Latent Sparse Attention", "The tree, step by step")
+    "lsa_tree_10m": Workload(
+        "lsa_tree_10m", "lsa", T=256, N=10485760, top_p=1024, budget=4096,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "spread": 20531, "node_block": 4096, "fanout": 4,
+               "beam": 2048, "levels": 3, "start_nodes": 32768},
+    ),
+    # the sampled-threshold flat search on one prefill chunk: 32768 queries
+    # (the sequence's last 32768 tokens) against 1310720 buckets at
+    # 10485760 tokens, top 1024 buckets each ("Latent Sparse Attention",
+    # "What the kernels do about the top-p")
+    "lsa_prefill_10m": Workload(
+        "lsa_prefill_10m", "lsa", T=32768, N=10485760, top_p=1024, budget=4096,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "chunk": 1},
+    ),
     # sparse main attention after the decode selection: 64 decode queries of
     # 128 heads, each over its 512 selected rows of a latent cache of
     # 262144 rows x 576 bf16 (302 MB, larger than L2); H, d = heads, latent
@@ -144,6 +167,20 @@ WORKLOADS: Dict[str, Workload] = {
     "lsa_flat_s": Workload(
         "lsa_flat_s", "lsa", T=37, N=40000, top_p=64, budget=512,
         extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "edge": 1, "node_block": 4096, "fanout": 4, "beam": 96},
+    ),
+    # the tree with three node levels at a reduced size: node blocks of 128
+    # entries (two key blocks' buckets, so a query can see half a node
+    # block), 4992 buckets, 1248 / 288 / 64 node buckets
+    "lsa_tree_levels_s": Workload(
+        "lsa_tree_levels_s", "lsa", T=37, N=40000, top_p=64, budget=512,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "edge": 1, "node_block": 128, "fanout": 4, "beam": 24,
+               "levels": 3, "start_nodes": 500},
+    ),
+    # a prefill chunk at a reduced size: 3000 queries (the last 3000 tokens of
+    # 262144) against 32768 buckets
+    "lsa_prefill_s": Workload(
+        "lsa_prefill_s", "lsa", T=3000, N=262144, top_p=256, budget=1024,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "chunk": 1},
     ),
     # 7 queries, 2 head groups, 300 slots (5 chunks, the last ragged); rows 0
     # and 1 select nothing and one row, the others a ragged prefix

@@ -297,6 +297,7 @@ def make_bucket(
 
 def make_lsa(
     T: int, L: int, block_keys: int = 512, bpb: int = 64, seed: int = 0, spread: int = 2053, edge: bool = False,
+    node_block: int = 4096, fanout: int = 4, levels: int = 1, chunk: bool = False,
 ) -> Dict[str, np.ndarray]:
     """Native LSA index for one sequence of L tokens and T index queries.
 
@@ -305,11 +306,12 @@ def make_lsa(
     (4..16 keys; the grouping stands in for the Ward merges, drawn at random
     here), members stored in ascending position order (CSR ``bucket_off`` /
     ``bucket_mem``, buckets block-major).  Centroids and index queries are
-    random 64-d unit vectors rounded to bf16; node buckets for the tree
-    search group every 4 buckets of each complete 4096-bucket block.  Query
-    positions: the last
-    token and every ``spread``-th token before it, or (``edge``) the block
-    edges 0, 3, 4, 511, 512, ... followed by random positions."""
+    random 64-d unit vectors rounded to bf16.  Node buckets for the tree
+    search, ``levels`` levels of them: every ``node_block`` entries of a level
+    (complete blocks only) are grouped ``fanout`` to a node of the level
+    above.  Query positions: the last token and every ``spread``-th token
+    before it, or (``edge``) the block edges 0, 3, 4, 511, 512, ... followed
+    by random positions, or (``chunk``) the last T tokens, one prefill chunk."""
     rng = np.random.default_rng(seed)
     dim = 64
     n_pool = block_keys // 4
@@ -318,6 +320,7 @@ def make_lsa(
     off = np.zeros(P + 1, dtype=np.int64)
     members = np.empty(nb * block_keys, dtype=np.int32)
     at = 0
+    bucket_of_rank = np.empty(n_pool, dtype=np.int64)
     for j in range(nb):
         sizes = np.full(bpb, n_pool // bpb)
         for _ in range(3 * bpb // 4):
@@ -327,36 +330,41 @@ def make_lsa(
                 sizes[b] += 1
         perm = rng.permutation(n_pool)
         cuts = np.concatenate([[0], np.cumsum(sizes)])
-        for i in range(bpb):
-            pools = np.sort(perm[cuts[i]:cuts[i + 1]])
-            pos = (j * block_keys + 4 * pools[:, None] + np.arange(4)[None, :]).reshape(-1)
-            members[at:at + pos.size] = pos
-            at += pos.size
-            off[j * bpb + i + 1] = at
+        # bucket i takes the pools perm[cuts[i]:cuts[i+1]], in ascending order
+        bucket_of_rank[:] = np.repeat(np.arange(bpb), sizes)
+        pools = perm[np.lexsort((perm, bucket_of_rank))]
+        pos = (j * block_keys + 4 * pools[:, None] + np.arange(4)[None, :]).reshape(-1)
+        members[at:at + pos.size] = pos
+        off[j * bpb + 1:(j + 1) * bpb + 1] = at + 4 * cuts[1:]
+        at += pos.size
     c = rng.standard_normal((P, dim))
     c /= np.linalg.norm(c, axis=1, keepdims=True)
     q = rng.standard_normal((T, dim))
     q /= np.linalg.norm(q, axis=1, keepdims=True)
-    # node buckets for the tree search: every node_block buckets form a node
-    # cluster block grouped 4 to a node (complete node blocks only); a node's
-    # centroid is the normalised sum of its children's key sums, each child's
-    # key sum taken as size x centroid (the synthetic buckets have no keys)
-    node_block, fanout = 4096, 4
-    P1 = (P // node_block) * (node_block // fanout)
-    sizes = np.diff(off)[:P1 * fanout].astype(np.float64)
-    cb = bf16_bits_to_f32(to_bf16_bits(c[:P1 * fanout])).astype(np.float64)
-    nsum = (cb * sizes[:, None]).reshape(P1, fanout, dim).sum(axis=1)
-    norms = np.linalg.norm(nsum, axis=1, keepdims=True)
-    nc = nsum / np.where(norms > 0, norms, 1.0)
+    # node buckets: a node's centroid is the normalised sum of every key
+    # beneath it; the synthetic buckets have no keys, so a bucket's key sum
+    # is taken as its size x its (bf16) centroid and a node's as the sum of
+    # its children's
+    node_levels = []
+    ksum = bf16_bits_to_f32(to_bf16_bits(c)).astype(np.float64) * np.diff(off)[:, None].astype(np.float64)
+    for _ in range(levels):
+        n_up = (ksum.shape[0] // node_block) * (node_block // fanout)
+        ksum = ksum[:n_up * fanout].reshape(n_up, fanout, dim).sum(axis=1)
+        norms = np.linalg.norm(ksum, axis=1, keepdims=True)
+        node_levels.append(to_bf16_bits(ksum / np.where(norms > 0, norms, 1.0)) if n_up
+                           else np.zeros((0, dim), dtype=np.uint16))
     if edge:
         fixed = [0, 3, 4, 511, 512, 513, 1023, 1024, 1536, 2047, 2048, L - 1]
         rest = np.sort(rng.integers(0, L, size=max(0, T - len(fixed))))
         q_pos = np.concatenate([fixed, rest])[:T].astype(np.int64)
+    elif chunk:
+        q_pos = np.arange(L - T, L, dtype=np.int64)
     else:
         q_pos = (L - 1 - spread * np.arange(T)).astype(np.int64)
     return {"q_idx": to_bf16_bits(q), "q_pos": q_pos, "centroids": to_bf16_bits(c),
             "bucket_off": off.astype(np.int32), "bucket_mem": members,
-            "node_centroids": to_bf16_bits(nc) if P1 else np.zeros((0, dim), dtype=np.uint16)}
+            "node_centroids": node_levels[0] if levels else np.zeros((0, dim), dtype=np.uint16),
+            "node_levels": node_levels}
 
 
 # --------------------------------------------------------------------------- #
@@ -407,8 +415,10 @@ def make_workload(wl, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
             wl.extra.get("min_size", 0), wl.extra.get("max_size", 0),
         )
     if wl.kind == "lsa":
-        return make_lsa(wl.T, wl.N, wl.extra.get("block_keys", 512), wl.extra.get("bpb", 64), s,
-                        wl.extra.get("spread", 2053), bool(wl.extra.get("edge", 0)))
+        ex = wl.extra
+        return make_lsa(wl.T, wl.N, ex.get("block_keys", 512), ex.get("bpb", 64), s, ex.get("spread", 2053),
+                        bool(ex.get("edge", 0)), ex.get("node_block", 4096), ex.get("fanout", 4), ex.get("levels", 1),
+                        bool(ex.get("chunk", 0)))
     if wl.kind == "attention":
         return make_attention(wl.T, wl.H, wl.N, wl.k, wl.d, s, ragged=wl.ragged)
     raise ValueError(wl.kind)
