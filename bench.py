@@ -358,6 +358,9 @@ VARIANTS = {
     "lsa_flat": lambda *a: bench_lsa(*a),
     "lsa_flat_threshold": lambda *a: bench_lsa(*a, threshold=True),
     "lsa_tree": lambda *a: bench_lsa_tree(*a),
+    "lsa_tree_10m": lambda *a: bench_lsa_tree_levels(*a),
+    "lsa_prefill_10m": lambda *a: bench_lsa(*a, threshold=True, workload="lsa_prefill_10m"),
+    "lsa_prefill_10m_q4096": lambda *a: bench_lsa(*a, threshold=True, workload="lsa_prefill_10m_q4096"),
     "two_stage": lambda *a: bench_two_stage(*a),
     "two_stage_pq": lambda *a: bench_two_stage(*a, pq=True),
     "prefill_shard_merge": lambda *a: bench_shard_merge(*a),
@@ -367,7 +370,8 @@ VARIANTS = {
 # one (a sticky CUDA error ends its process) becomes an error entry and cannot
 # reach the decode line or another variant.  A variant joins this list once it
 # has run clean on a B200.
-DEFAULT_VARIANTS = list(VARIANTS)
+# the 4096-query LSA chunk is the scan's profile case, not a bench line
+DEFAULT_VARIANTS = [v for v in VARIANTS if v != "lsa_prefill_10m_q4096"]
 
 
 def bench_one_variant(L, args, peaks, peak_kind, name):
@@ -554,24 +558,26 @@ def bench_bucket(L, args, peaks, peak_kind):
     return res
 
 
-def bench_lsa(L, args, peaks, peak_kind, threshold=False):
+def bench_lsa(L, args, peaks, peak_kind, threshold=False, workload="lsa_flat"):
     """Native LSA flat search: 256 index queries over 131072 buckets of one
     1048576-token sequence; top 1024 buckets, 4096 long-range keys.  With
     threshold, the sampled-threshold scan lists only the buckets that clear
-    each query's threshold (else every score goes to a T x P matrix)."""
+    each query's threshold (else every score goes to a T x P matrix).  The
+    prefill workload: 32768 queries over 1310720 buckets (threshold form
+    only), a compute-bound scan reported against the bf16 tensor peak."""
     import torch
     from workloads import get_workload, make_workload
     st = torch.cuda.current_stream()
     steps = max(3, args.steps)
     warm = max(3, args.warmup)
-    wl = get_workload("lsa_flat")
+    wl = get_workload(workload)
     d = make_workload(wl)
     ex = wl.extra
     T = d["q_idx"].shape[0]
     P_ = d["centroids"].shape[0]
     a = [to_dev_bf16(d["q_idx"]), to_dev(d["q_pos"]), to_dev_bf16(d["centroids"]), to_dev(d["bucket_off"]),
          to_dev(d["bucket_mem"])]
-    ws = torch.empty(L.lib().ls_lsa_flat_workspace_size(T, P_, wl.top_p, int(threshold)), dtype=torch.uint8,
+    ws = torch.empty(L.lib().ls_lsa_flat_workspace_size(T, P_, wl.top_p, int(threshold), 0), dtype=torch.uint8,
                      device="cuda")
     row = ex["n_sink"] + ex["block_keys"] + wl.budget
     out = (torch.empty((T, row), dtype=torch.int32, device="cuda"), torch.empty((T,), dtype=torch.int32, device="cuda"))
@@ -589,11 +595,16 @@ def bench_lsa(L, args, peaks, peak_kind, threshold=False):
     # centroids and queries read; the full form also writes the T x P score matrix
     bytes_dot = P_ * 128 + T * 128 + (0 if threshold else T * P_ * 4)
     peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    traffic = ncu_traffic(kname, wl.name + ("_threshold" if threshold else ""))
+    if T >= 4096:
+        # prefill scale: the scan is a dense contraction (2 x 64 flops per visible (query, bucket) pair)
+        rl = roofline("tensor", 128.0 * scored / (dms * 1e-3) / 1e12,
+                      peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]), "TFLOP/s", traffic=traffic,
+                      peak_kind=peak_kind)
+    else:
+        rl = roofline("hbm", bytes_dot / (dms * 1e-3) / 1e9, peak_b, "GB/s", traffic=traffic, peak_kind=peak_kind)
     res = {"ms_per_step": ms, "positions_per_s": scored / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
-           "kernels": kern,
-           "roofline": roofline("hbm", bytes_dot / (dms * 1e-3) / 1e9, peak_b, "GB/s",
-                                traffic=ncu_traffic(kname, wl.name + ("_threshold" if threshold else "")),
-                                peak_kind=peak_kind),
+           "kernels": kern, "roofline": rl, "queries": T, "buckets": P_,
            "bytes_dot": bytes_dot, "visible_buckets_scored": scored,
            "note": "positions = visible buckets scored per query (one 64-d dot each); "
                    + ("sampled thresholds (every 128th bucket, 32nd best), the scan lists the buckets that clear "
@@ -645,6 +656,64 @@ def bench_lsa_tree(L, args, peaks, peak_kind):
                    "the flat search); roofline of the node scoring (node centroids and queries read, scores "
                    "written)"}
     del a, ws
+    return res
+
+
+def bench_lsa_tree_levels(L, args, peaks, peak_kind, workload="lsa_tree_10m"):
+    """LSA tree search over three node levels at 10485760 tokens: 256 index
+    queries; the beam starts at level 3 (20480 node buckets), keeps 2048,
+    steps down through levels 2 and 1 to the buckets, top 1024, read lists."""
+    import torch
+    from workloads import get_workload, make_workload
+    st = torch.cuda.current_stream()
+    steps = max(3, args.steps)
+    warm = max(3, args.warmup)
+    wl = get_workload(workload)
+    d = make_workload(wl)
+    ex = wl.extra
+    T = d["q_idx"].shape[0]
+    P_ = d["centroids"].shape[0]
+    levels = [to_dev_bf16(x) for x in d["node_levels"]]
+    sizes = [x.shape[0] for x in d["node_levels"]]
+    a = [to_dev_bf16(d["q_idx"]), to_dev(d["q_pos"]), to_dev_bf16(d["centroids"]), levels, to_dev(d["bucket_off"]),
+         to_dev(d["bucket_mem"])]
+    kw = dict(node_block=ex["node_block"], fanout=ex["fanout"], beam=ex["beam"], start_nodes=ex["start_nodes"],
+              top_p=wl.top_p)
+    ws = torch.empty(L.ls_lsa_tree_levels_workspace_size(T, P_, sizes, **kw), dtype=torch.uint8, device="cuda")
+    row = ex["n_sink"] + ex["block_keys"] + wl.budget
+    out = (torch.empty((T, row), dtype=torch.int32, device="cuda"), torch.empty((T,), dtype=torch.int32, device="cuda"))
+
+    def run(i, timed):
+        L.ls_lsa_tree_levels_select(*a, block_keys=ex["block_keys"], buckets_per_block=ex["bpb"],
+                                    n_sink=ex["n_sink"], budget=wl.budget, ws=ws, out=out, **kw)
+        return None
+
+    ms, kern = _profiled_loop(L, run, steps, warm, st)
+    # vectors scored per query: the start level's visible nodes, then the beam's children (and any
+    # uncovered entries) at each level below, from the level sizes the oracle's visibility rule gives
+    start = next((i + 1 for i, n in enumerate(sizes) if n <= ex["start_nodes"]), len(sizes))
+    vis0 = np.minimum((d["q_pos"] // ex["block_keys"]) * ex["bpb"], P_)
+    per_query, cand_rows = [], 0
+    for v0 in vis0:
+        v = [int(v0)]
+        for n in sizes:
+            v.append(min(n, v[-1] // ex["node_block"] * (ex["node_block"] // ex["fanout"])))
+        below = sum(min(ex["beam"], v[lv + 1]) * ex["fanout"] + (v[lv] - ex["fanout"] * v[lv + 1])
+                    for lv in range(start - 1, -1, -1))
+        per_query.append(v[start] + below)
+        cand_rows += below
+    scored = int(np.sum(per_query))
+    cand_ms = kern["lsa_tree_candidates_kernel"]["ms_per_step"]
+    peak_b = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    res = {"ms_per_step": ms, "positions_per_s": scored / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
+           "kernels": kern, "start_level": start, "level_sizes": [P_] + sizes,
+           "vectors_scored_per_query": float(np.mean(per_query)), "flat_vectors_per_query": float(np.mean(vis0)),
+           "roofline": roofline("hbm", cand_rows * 136 / (cand_ms * 1e-3) / 1e9, peak_b, "GB/s", peak_kind=peak_kind),
+           "note": "positions = vectors scored per query (start-level nodes, then each level's candidates), "
+                   "summed; roofline of the candidate scoring below the start level (136 bytes per candidate: "
+                   "its 128-byte centroid gathered, score and label written); inputs 168 MB of bucket centroids "
+                   "(larger than L2) of which each step gathers a part; no flush"}
+    del a, ws, levels
     return res
 
 

@@ -296,16 +296,24 @@ ls_status ls_prefill_select_stream_fp8(const uint8_t* q8, const float* q_scale, 
  * the threshold to a list of up to 8 * top_p, and the top_p of the list is
  * kept; a query whose list overflows or holds fewer than min(top_p, visible)
  * buckets is scored in full instead.  Both forms pick the same buckets.
- * Workspace: ls_lsa_flat_workspace_size(T, P, top_p, threshold) bytes (the
- * T x P score matrix among them: the full form's scores and the threshold
- * form's fallback).
+ * The threshold form never holds the T x P matrix: the missed queries are
+ * listed on the device and scored in full fallback_rows at a time (a few
+ * launches per chunk of rows, which return at once when the chunk holds
+ * none); fallback_rows <= 0 takes the default, the most rows whose scores
+ * fit 4 GiB (a multiple of 256 when that many fit), at most T.  The launches
+ * for every chunk are queued whether or not a row misses: ceil(T /
+ * fallback_rows) chunks.
+ * Workspace: ls_lsa_flat_workspace_size(T, P, top_p, threshold,
+ * fallback_rows) bytes: threshold = 0 holds the T x P matrix; threshold = 1
+ * holds the samples (T x P / (top_p / 8)), the lists (about T x 16 top_p
+ * entries of 8 bytes) and fallback_rows x P scores.
  */
-size_t ls_lsa_flat_workspace_size(int T, int P, int top_p, int threshold);
+size_t ls_lsa_flat_workspace_size(int T, int P, int top_p, int threshold, int fallback_rows);
 ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
                              const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
                              int block_keys, int buckets_per_block, int n_sink, int top_p, int budget, int threshold,
-                             int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws, size_t ws_bytes,
-                             void* stream);
+                             int fallback_rows, int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /*
  * ls_lsa_tree_select -- the LSA tree search's beam over one level of node
@@ -321,9 +329,8 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
  *   beam_out [T][beam] int32 picked node buckets, best first (or NULL)
  *   other arguments and outputs as in ls_lsa_flat_select
  * With beam >= every visible node bucket the picks are those of the flat
- * search.  Only d = 64 and one node level are built (the pages start the
- * beam at the lowest level with at most 32768 node buckets: level 1 up to
- * 1M tokens).
+ * search.  Only d = 64 is built; ls_lsa_tree_levels_select is the search
+ * over several node levels.
  * Workspace: ls_lsa_tree_workspace_size(T, P1, beam, fanout, node_block, top_p) bytes.
  */
 size_t ls_lsa_tree_workspace_size(int T, int P1, int beam, int fanout, int node_block, int top_p);
@@ -333,6 +340,50 @@ ls_status ls_lsa_tree_select(const uint16_t* q_idx, const int64_t* q_pos, const 
                              int fanout, int beam, int n_sink, int top_p, int budget, int32_t* keys_out,
                              int32_t* n_out, int32_t* picked_out, int32_t* beam_out, void* ws, size_t ws_bytes,
                              void* stream);
+
+/*
+ * ls_lsa_tree_levels_select -- the LSA tree search over L >= 1 levels of node
+ * buckets ("Latent Sparse Attention", section "The tree, step by step").
+ * Level 0 is the buckets; every node_block entries of level l - 1 (complete
+ * blocks only) are grouped fanout to a node of level l, node n covering
+ * entries fanout*n .. fanout*n + fanout - 1.  A query sees, at each level,
+ * the nodes of the complete node blocks among its visible entries below.  The
+ * beam starts at the lowest level with at most start_nodes node buckets (the
+ * top level if none has so few), scores every visible node there and keeps
+ * the best `beam`; at each level below it scores the kept nodes' children
+ * plus the visible entries no node of the level above covers and keeps the
+ * best `beam` again; at the bucket level it keeps the best top_p and reads
+ * them as ls_lsa_flat_select does.
+ *
+ *   node_centroids  HOST array of L device pointers: level l's node
+ *                   centroids [level_sizes[l-1]][64] bf16 at node_centroids[l-1]
+ *   level_sizes     HOST array of L ints, P1 .. PL; fanout * P_l <= P_{l-1}
+ *   L               1 .. 16
+ *   beam            1 .. 4096; start_nodes >= 1 (the pages: 32768)
+ *   picked_out      [T][top_p] int32 picked buckets, best first (or NULL)
+ *   beams_out       [L][T][beam] int32: level l's beam at [l-1], best first,
+ *                   -1 past its end (or NULL); levels above the start level
+ *                   are not written
+ *   other arguments and outputs as in ls_lsa_flat_select
+ * Ties go to the lower entry at every level.  With beam >= every level's
+ * visible entries the picks are those of the flat search.  The host arrays
+ * are read before the call returns; the device buffers must stay valid until
+ * the stream's work ends.
+ * Errors: LS_ERR_INVALID_ARG for sizes out of range, a level larger than its
+ * children allow, null or misaligned pointers; LS_ERR_UNSUPPORTED for d != 64;
+ * LS_ERR_WORKSPACE below the size returned by
+ * ls_lsa_tree_levels_workspace_size(T, P, level_sizes, L, node_block, fanout,
+ * beam, start_nodes, top_p) (0 for invalid arguments).
+ */
+size_t ls_lsa_tree_levels_workspace_size(int T, int P, const int* level_sizes, int L, int node_block, int fanout,
+                                         int beam, int start_nodes, int top_p);
+ls_status ls_lsa_tree_levels_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
+                                    const uint16_t* const* node_centroids, const int* level_sizes, int L,
+                                    const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
+                                    int block_keys, int buckets_per_block, int node_block, int fanout, int beam,
+                                    int start_nodes, int n_sink, int top_p, int budget, int32_t* keys_out,
+                                    int32_t* n_out, int32_t* picked_out, int32_t* beams_out, void* ws,
+                                    size_t ws_bytes, void* stream);
 
 /*
  * ls_merge_select -- the combine step of a prefill whose history is split into

@@ -22,6 +22,8 @@ from ._lib import (  # noqa: F401
     ls_indexer_score_fp8,
     ls_indexer_score_pq,
     ls_lsa_flat_select,
+    ls_lsa_tree_levels_select,
+    ls_lsa_tree_levels_workspace_size,
     ls_lsa_tree_select,
     ls_merge_select,
     ls_sparse_attention,

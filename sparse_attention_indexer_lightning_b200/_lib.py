@@ -42,7 +42,8 @@ EXPORTED = (
     "ls_indexer_score_pq", "ls_indexer_score_fp8_workspace_size", "ls_indexer_score_fp8",
     "ls_prefill_select_fp8_workspace_size", "ls_prefill_select_stream_fp8", "ls_lsa_flat_workspace_size",
     "ls_lsa_flat_select", "ls_lsa_tree_workspace_size", "ls_lsa_tree_select", "ls_merge_select_workspace_size",
-    "ls_merge_select", "ls_sparse_attention", "ls_attention_merge",
+    "ls_merge_select", "ls_sparse_attention", "ls_attention_merge", "ls_lsa_tree_levels_workspace_size",
+    "ls_lsa_tree_levels_select",
 )
 HIST_BINS = 2048
 
@@ -85,10 +86,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ls_indexer_score_fp8": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, SZ, P]),
         "ls_prefill_select_fp8_workspace_size": (SZ, [I, I, I, I, I]),
         "ls_prefill_select_stream_fp8": (I, [P, P, P, P, I, I, I, P, P, I, I, I, P, P, I, I, P, P, P, SZ, P, P]),
-        "ls_lsa_flat_workspace_size": (SZ, [I, I, I, I]),
-        "ls_lsa_flat_select": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
+        "ls_lsa_flat_workspace_size": (SZ, [I, I, I, I, I]),
+        "ls_lsa_flat_select": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, P, P, P, P, SZ, P]),
         "ls_lsa_tree_workspace_size": (SZ, [I, I, I, I, I, I]),
         "ls_lsa_tree_select": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]),
+        "ls_lsa_tree_levels_workspace_size": (SZ, [I, I, P, I, I, I, I, I, I]),
+        "ls_lsa_tree_levels_select": (I, [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P,
+                                          P, SZ, P]),
         "ls_merge_select_workspace_size": (SZ, [I, I, I]),
         "ls_merge_select": (I, [P, P, P, I, I, I, I, P, P, P, SZ, P]),
         "ls_sparse_attention": (I, [P, P, P, P, I, I, I, I, I64, I, ctypes.c_float, I, P, P, P]),
@@ -462,11 +466,13 @@ def ls_bucket_select(q, w, centroids, bucket_off, bucket_mem, keys, top_p: int =
 
 def ls_lsa_flat_select(q_idx, q_pos, centroids, bucket_off, bucket_mem, block_keys: int = 512,
                        buckets_per_block: int = 64, n_sink: int = 4, top_p: int = 1024, budget: int = 4096,
-                       threshold: bool = False, want_picked: bool = False, ws=None, out=None, stream=None):
+                       threshold: bool = False, fallback_rows: int = 0, want_picked: bool = False, ws=None, out=None,
+                       stream=None):
     """Native LSA flat search.  q_idx [T,64] bf16, q_pos [T] int64, centroids [P,64] bf16 (block-major),
     bucket_off [P+1] / bucket_mem int32 (members ascending) -> (keys [T, n_sink+block_keys+budget] int32,
     n [T] int32[, picked [T, top_p] int32]).  threshold: the sampled-threshold scan with candidate lists (else
-    the full score matrix); both pick the same buckets."""
+    the full score matrix); both pick the same buckets.  fallback_rows: queries the threshold form's fallback
+    scores in full at a time (0: the default bound)."""
     _dev(q_idx, torch.bfloat16, "q_idx", 2)
     T, d = q_idx.shape
     _dev(q_pos, torch.int64, "q_pos", 1)
@@ -474,7 +480,7 @@ def ls_lsa_flat_select(q_idx, q_pos, centroids, bucket_off, bucket_mem, block_ke
     P = centroids.shape[0]
     _dev(bucket_off, torch.int32, "bucket_off", 1)
     _dev(bucket_mem, torch.int32, "bucket_mem", 1)
-    need = lib().ls_lsa_flat_workspace_size(T, P, top_p, int(threshold))
+    need = lib().ls_lsa_flat_workspace_size(T, P, top_p, int(threshold), int(fallback_rows))
     if ws is None:
         ws = _workspace(need, q_idx.device)
     if out is None:
@@ -484,8 +490,8 @@ def ls_lsa_flat_select(q_idx, q_pos, centroids, bucket_off, bucket_mem, block_ke
     picked = torch.empty((T, top_p), dtype=torch.int32, device=q_idx.device) if want_picked else None
     _check(lib().ls_lsa_flat_select(_ptr(q_idx), _ptr(q_pos), _ptr(centroids), _ptr(bucket_off), _ptr(bucket_mem),
                                     T, d, P, block_keys, buckets_per_block, n_sink, top_p, budget, int(threshold),
-                                    _ptr(keys),
-                                    _ptr(n), _ptr(picked), _ptr(ws), ws.numel(), _stream(stream)))
+                                    int(fallback_rows), _ptr(keys), _ptr(n), _ptr(picked), _ptr(ws), ws.numel(),
+                                    _stream(stream)))
     return (keys, n, picked) if want_picked else (keys, n)
 
 
@@ -517,6 +523,49 @@ def ls_lsa_tree_select(q_idx, q_pos, centroids, node_centroids, bucket_off, buck
                                     node_block, fanout, beam, n_sink, top_p, budget, _ptr(keys), _ptr(n),
                                     _ptr(picked), _ptr(bm), _ptr(ws), ws.numel(), _stream(stream)))
     return (keys, n, picked, bm) if want_picked else (keys, n)
+
+
+def ls_lsa_tree_levels_workspace_size(T: int, P: int, level_sizes, node_block: int = 4096, fanout: int = 4,
+                                      beam: int = 2048, start_nodes: int = 32768, top_p: int = 1024) -> int:
+    L = len(level_sizes)
+    sizes = (ctypes.c_int * max(L, 1))(*[int(x) for x in level_sizes])
+    return lib().ls_lsa_tree_levels_workspace_size(T, P, sizes, L, node_block, fanout, beam, start_nodes, top_p)
+
+
+def ls_lsa_tree_levels_select(q_idx, q_pos, centroids, node_levels, bucket_off, bucket_mem, block_keys: int = 512,
+                              buckets_per_block: int = 64, node_block: int = 4096, fanout: int = 4,
+                              beam: int = 2048, start_nodes: int = 32768, n_sink: int = 4, top_p: int = 1024,
+                              budget: int = 4096, want_picked: bool = False, ws=None, out=None, stream=None):
+    """LSA tree search over several node levels.  As ls_lsa_flat_select, plus node_levels: a list of L
+    [P_l,64] bf16 tensors (levels 1..L); with want_picked also returns (picked [T, top_p],
+    beams [L, T, beam]) int32 (levels above the start level are left unwritten)."""
+    _dev(q_idx, torch.bfloat16, "q_idx", 2)
+    T, d = q_idx.shape
+    _dev(q_pos, torch.int64, "q_pos", 1)
+    _dev(centroids, torch.bfloat16, "centroids", 2)
+    for i, nc in enumerate(node_levels):
+        _dev(nc, torch.bfloat16, f"node_levels[{i}]", 2)
+    _dev(bucket_off, torch.int32, "bucket_off", 1)
+    _dev(bucket_mem, torch.int32, "bucket_mem", 1)
+    P, L = centroids.shape[0], len(node_levels)
+    sizes = [int(nc.shape[0]) for nc in node_levels]
+    need = ls_lsa_tree_levels_workspace_size(T, P, sizes, node_block, fanout, beam, start_nodes, top_p)
+    if ws is None:
+        ws = _workspace(need, q_idx.device)
+    if out is None:
+        out = (torch.empty((T, n_sink + block_keys + budget), dtype=torch.int32, device=q_idx.device),
+               torch.empty((T,), dtype=torch.int32, device=q_idx.device))
+    keys, n = out
+    picked = torch.empty((T, top_p), dtype=torch.int32, device=q_idx.device) if want_picked else None
+    beams = torch.full((max(L, 1), T, beam), -2, dtype=torch.int32, device=q_idx.device) if want_picked else None
+    ptrs = (ctypes.c_void_p * max(L, 1))(*[nc.data_ptr() for nc in node_levels])
+    csizes = (ctypes.c_int * max(L, 1))(*sizes)
+    _check(lib().ls_lsa_tree_levels_select(_ptr(q_idx), _ptr(q_pos), _ptr(centroids), ptrs, csizes, L,
+                                           _ptr(bucket_off), _ptr(bucket_mem), T, d, P, block_keys,
+                                           buckets_per_block, node_block, fanout, beam, start_nodes, n_sink, top_p,
+                                           budget, _ptr(keys), _ptr(n), _ptr(picked), _ptr(beams), _ptr(ws),
+                                           ws.numel(), _stream(stream)))
+    return (keys, n, picked, beams) if want_picked else (keys, n)
 
 
 def ls_merge_select(vals, idx, offsets, k: int = 512, ws=None, out=None, stream=None):

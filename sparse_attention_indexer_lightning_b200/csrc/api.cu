@@ -198,11 +198,12 @@ ls_status score_tc_launch(const uint16_t* q, const uint16_t* keys, int B, int T,
 
 // 2-D map over [rows][64] bf16 vectors (128 bytes each: one swizzle row),
 // box = 64 x box_rows, 128-byte swizzle.
-ls_status make_vec64_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+ls_status make_vec64_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows,
+                         uint64_t row_step = 1) {
   auto fn = encode_fn();
   if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(kLsaDim), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLsaDim * 2)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLsaDim * 2 * row_step)};   // row i at base + i * row_step * 128 B
   cuuint32_t box[2] = {static_cast<cuuint32_t>(kLsaDim), box_rows};
   cuuint32_t es[2] = {1u, 1u};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
@@ -967,47 +968,74 @@ struct LsaThreshold {
       : stride(top_p / 8 > 1 ? top_p / 8 : 1), rank(32), cap(8 * top_p) {}
 };
 
-// Per-CTA list segments of the filtered scan: nseg = the scan's grid, seg
-// entries each (about 4x the expected count of a CTA's share of 4 * top_p),
-// at most 2 * cap + 64 * nseg entries per row.
+// List segments of the filtered scan: each row's list holds 2 * cap entries
+// shared out among the scan's CTAs in proportion to the centroid tiles of
+// the row each one scores (about 2x the expected count of its share of the
+// 4 * top_p listed buckets), plus 64 slack entries per CTA.
 struct LsaSegments {
-  int nseg, seg;
+  int grid, nseg, cap2, slack;
   long long per_row;
   LsaSegments(int T, int P, int cap) {
-    nseg = dot_tc_grid(T, P, num_sms_current());
-    if (nseg < 1) nseg = 1;
-    per_row = 2LL * cap + 64LL * nseg;
-    const int want = ((2 * cap / nseg + 31) / 32) * 32;
-    seg = static_cast<int>(std::min<long long>(std::max(32, want), per_row / nseg));
+    grid = dot_tc_grid(T, P, num_sms_current());
+    const int NT = (P + DotCfg::BM - 1) / DotCfg::BM;
+    const long long units = static_cast<long long>((T + DotCfg::QB - 1) / DotCfg::QB) * NT;
+    nseg = grid > 0 ? lsa_max_segments(units, grid, NT) : 1;
+    cap2 = 2 * cap;
+    slack = 64;
+    per_row = cap2 + static_cast<long long>(slack) * nseg;
+  }
+};
+
+// The threshold form's fallback scores the missed rows in full, `rows` of
+// them at a time: at most kLsaFallbackBytes of scores (a multiple of the
+// scorer's 256-query group when that many fit), unless the caller asks for
+// fewer rows.
+constexpr size_t kLsaFallbackBytes = size_t(4) << 30;
+struct LsaFallback {
+  int rows, chunks;
+  LsaFallback(int T, int P, int fallback_rows) {
+    long long r = static_cast<long long>(kLsaFallbackBytes / (sizeof(float) * static_cast<size_t>(P > 0 ? P : 1)));
+    if (r >= DotCfg::QB) r -= r % DotCfg::QB;
+    if (fallback_rows > 0 && fallback_rows < r) r = fallback_rows;
+    if (r > T) r = T;
+    if (r < 1) r = 1;
+    rows = static_cast<int>(r);
+    chunks = (T + rows - 1) / rows;
   }
 };
 
 struct LsaWorkspace {
-  float* sc;        // [T][P] full scores (the full-matrix form, and the threshold form's fallback)
+  float* sc;        // the full-matrix form: [T][P] scores; the threshold form: [rows][P] of the fallback
   int32_t* vis;     // [T]
   int32_t* nsamp;   // [T]
   int32_t* picked;  // [T][top_p]
   float* ss;        // [T][n_samp] sample scores
   float* sv;        // [T][rank] best samples
   int32_t* si;      // [T][rank]
-  float* sval;      // [T][nseg][seg] the scan's list segments
-  int32_t* slab;
-  uint32_t* scnt;   // [T][nseg]
+  uint2* slist;     // [T][per_row] the scan's list segments, (score bits, bucket) pairs
+  uint32_t* scnt;   // [T][nseg][4]
   float* cval;      // [T][cap] packed lists
   int32_t* clab;
   int32_t* nv;      // [T]
   uint8_t* ctr;     // row_over [T], any_over
+  int32_t* fb_list; // [T] missed rows, then the count, then the chunk flags
+  int32_t* fb_count;
+  int32_t* fb_run;
+  uint16_t* fb_q;   // [rows][64] their index queries
+  int32_t* fb_vis;  // [rows]
+  int32_t* fb_pick; // [rows][top_p]
   size_t ctr_bytes;
   size_t scnt_bytes;
   size_t used;
 };
 
-LsaWorkspace carve_lsa(void* ws, int T, int P, int top_p, int threshold) {
+LsaWorkspace carve_lsa(void* ws, int T, int P, int top_p, int threshold, int fallback_rows) {
   Carver cv(ws);
   LsaWorkspace w{};
   const LsaThreshold th(top_p);
   const int n_samp = (P + th.stride - 1) / th.stride;
-  w.sc = cv.take<float>(static_cast<size_t>(T) * P);
+  const LsaFallback fb(T, P, fallback_rows);
+  w.sc = cv.take<float>(static_cast<size_t>(threshold ? fb.rows : T) * P);
   w.vis = cv.take<int32_t>(T);
   w.nsamp = cv.take<int32_t>(T);
   w.picked = cv.take<int32_t>(static_cast<size_t>(T) * top_p);
@@ -1016,15 +1044,20 @@ LsaWorkspace carve_lsa(void* ws, int T, int P, int top_p, int threshold) {
     w.sv = cv.take<float>(static_cast<size_t>(T) * th.rank);
     w.si = cv.take<int32_t>(static_cast<size_t>(T) * th.rank);
     const LsaSegments sg(T, P, th.cap);
-    w.sval = cv.take<float>(static_cast<size_t>(T) * sg.per_row);
-    w.slab = cv.take<int32_t>(static_cast<size_t>(T) * sg.per_row);
-    w.scnt_bytes = static_cast<size_t>(T) * sg.nseg * sizeof(uint32_t);
-    w.scnt = cv.take<uint32_t>(static_cast<size_t>(T) * sg.nseg);
+    w.slist = cv.take<uint2>(static_cast<size_t>(T) * sg.per_row);
+    w.scnt_bytes = static_cast<size_t>(T) * sg.nseg * 4 * sizeof(uint32_t);
+    w.scnt = cv.take<uint32_t>(static_cast<size_t>(T) * sg.nseg * 4);
     w.cval = cv.take<float>(static_cast<size_t>(T) * th.cap);
     w.clab = cv.take<int32_t>(static_cast<size_t>(T) * th.cap);
     w.nv = cv.take<int32_t>(T);
     w.ctr_bytes = static_cast<size_t>(T) * sizeof(int32_t) + sizeof(int);   // row flags, then the any-row flag
     w.ctr = cv.take<uint8_t>(w.ctr_bytes);
+    w.fb_list = cv.take<int32_t>(T);
+    w.fb_count = cv.take<int32_t>(1);
+    w.fb_run = cv.take<int32_t>(fb.chunks);
+    w.fb_q = cv.take<uint16_t>(static_cast<size_t>(fb.rows) * kLsaDim);
+    w.fb_vis = cv.take<int32_t>(fb.rows);
+    w.fb_pick = cv.take<int32_t>(static_cast<size_t>(fb.rows) * top_p);
   }
   w.used = cv.used;
   return w;
@@ -1034,16 +1067,16 @@ LsaWorkspace carve_lsa(void* ws, int T, int P, int top_p, int threshold) {
 
 extern "C" {
 
-size_t ls_lsa_flat_workspace_size(int T, int P, int top_p, int threshold) {
+size_t ls_lsa_flat_workspace_size(int T, int P, int top_p, int threshold, int fallback_rows) {
   if (T <= 0 || top_p <= 0 || P < 0) return 0;
-  return carve_lsa(nullptr, T, P, top_p, threshold).used;
+  return carve_lsa(nullptr, T, P, top_p, threshold, fallback_rows).used;
 }
 
 ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
                              const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
                              int block_keys, int buckets_per_block, int n_sink, int top_p, int budget, int threshold,
-                             int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws, size_t ws_bytes,
-                             void* stream) {
+                             int fallback_rows, int32_t* keys_out, int32_t* n_out, int32_t* picked_out, void* ws,
+                             size_t ws_bytes, void* stream) {
   if (d != kLsaDim) return fail(LS_ERR_UNSUPPORTED, "only d=%d is built for the LSA index space (got %d)", kLsaDim, d);
   LS_CHECK_ARG(T >= 0 && P >= 0, "negative size");
   LS_CHECK_ARG(block_keys >= 1 && buckets_per_block >= 1, "block_keys and buckets_per_block must be >= 1");
@@ -1051,9 +1084,9 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
   LS_CHECK_ARG(top_p >= 1 && top_p <= kMaxTopK, "top_p must be in [1, %d] (got %d)", kMaxTopK, top_p);
   if (T == 0) return LS_OK;
   LS_CHECK_ARG(q_pos && keys_out && n_out, "null tensor pointer");
-  const size_t need = ls_lsa_flat_workspace_size(T, P, top_p, threshold);
+  const size_t need = ls_lsa_flat_workspace_size(T, P, top_p, threshold, fallback_rows);
   if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
-  const LsaWorkspace w = carve_lsa(ws, T, P, top_p, threshold);
+  const LsaWorkspace w = carve_lsa(ws, T, P, top_p, threshold, fallback_rows);
   const LsaThreshold th(top_p);
   int32_t* picked = picked_out ? picked_out : w.picked;
   cudaStream_t st = S(stream);
@@ -1092,11 +1125,21 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
       s = topk_launch(tp, st);
       if (s != LS_OK) return s;
     } else {
-      // 1. thresholds from a sample of every stride-th bucket
+      // 1. thresholds from a sample of every stride-th bucket, scored by the
+      //    same tensor-core scorer through a map that steps stride rows
       const int n_samp = (P + th.stride - 1) / th.stride;
       {
-        ProfScope prof("lsa_sample_kernel", st);
-        LS_CUDA(launch_lsa_sample(q_idx, centroids, T, n_samp, th.stride, w.ss, st));
+        CUtensorMap smap;
+        s = make_vec64_map(&smap, centroids, static_cast<uint64_t>(n_samp), kTileKeys,
+                           static_cast<uint64_t>(th.stride));
+        if (s != LS_OK) return s;
+        DotParams sd;
+        sd.T = T;
+        sd.P = n_samp;
+        sd.out = w.ss;
+        sd.ld_out = n_samp;
+        ProfScope prof("dot_tc_kernel:sample", st);
+        LS_CUDA(launch_dot_tc(&smap, &qmap, sd, num_sms_current(), st));
       }
       TopkParams sp;
       sp.scores = w.ss;
@@ -1122,10 +1165,11 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
       fp.vis = w.vis;
       fp.tau = w.sv + (th.rank - 1);
       fp.ld_tau = th.rank;
-      fp.cand_val = w.sval;
-      fp.cand_lab = w.slab;
+      fp.cand_list = w.slist;
+      fp.ld_cand = sg.per_row;
       fp.nseg = sg.nseg;
-      fp.seg = sg.seg;
+      fp.cap2 = sg.cap2;
+      fp.slack = sg.slack;
       fp.cand_cnt = w.scnt;
       fp.row_over = row_over;
       fp.any_over = any_over;
@@ -1135,7 +1179,7 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
       }
       {
         ProfScope prof("lsa_compact_kernel", st);
-        LS_CUDA(launch_lsa_compact(w.sval, w.slab, w.scnt, sg.nseg, sg.seg, w.vis, T, top_p, th.cap, w.cval, w.clab,
+        LS_CUDA(launch_lsa_compact(w.slist, w.scnt, fp, sg.grid, w.vis, T, top_p, th.cap, w.cval, w.clab,
                                    w.nv, row_over, any_over, st));
       }
       // 3. top-p of each list
@@ -1152,17 +1196,50 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
       cp.ld_out = top_p;
       s = topk_launch(cp, st);
       if (s != LS_OK) return s;
-      // 4. rows whose list ran over or came up short: scored in full (launches
-      //    that return at once when no row is flagged)
-      full.run_if = any_over;
+      // 4. rows whose list ran over or came up short, listed and scored in
+      //    full fb.rows at a time (the launches of a chunk that holds none of
+      //    them return at once)
+      const LsaFallback fb(T, P, fallback_rows);
       {
-        ProfScope prof("dot_tc_kernel:fallback", st);
-        LS_CUDA(launch_dot_tc(&cmap, &qmap, full, num_sms_current(), st));
+        ProfScope prof("lsa_flag_list_kernel", st);
+        LS_CUDA(launch_lsa_flag_list(row_over, T, fb.rows, fb.chunks, w.fb_list, w.fb_count, w.fb_run, st));
       }
-      tp.run_if = any_over;
-      tp.row_flag = row_over;
-      s = topk_launch(tp, st, "topk_kernel:fallback");
+      CUtensorMap fqmap;
+      s = make_vec64_map(&fqmap, w.fb_q, static_cast<uint64_t>(fb.rows), DotCfg::QB);
       if (s != LS_OK) return s;
+      for (int c = 0; c < fb.chunks; ++c) {
+        const int32_t* run = w.fb_run + c;
+        const int c0 = c * fb.rows;
+        {
+          ProfScope prof("lsa_gather_rows_kernel", st);
+          LS_CUDA(launch_lsa_gather_rows(w.fb_list, w.fb_count, c0, fb.rows, q_idx, w.vis, run, w.fb_q, w.fb_vis,
+                                         st));
+        }
+        DotParams fd;
+        fd.T = fb.rows;
+        fd.P = P;
+        fd.out = w.sc;
+        fd.ld_out = P;
+        fd.run_if = run;
+        {
+          ProfScope prof("dot_tc_kernel:fallback", st);
+          LS_CUDA(launch_dot_tc(&cmap, &fqmap, fd, num_sms_current(), st));
+        }
+        TopkParams fk;
+        fk.scores = w.sc;
+        fk.ld = P;
+        fk.n_valid = w.fb_vis;
+        fk.R = fb.rows;
+        fk.N = P;
+        fk.k = top_p;
+        fk.idx_out = w.fb_pick;
+        fk.ld_out = top_p;
+        fk.run_if = run;
+        s = topk_launch(fk, st, "topk_kernel:fallback");
+        if (s != LS_OK) return s;
+        ProfScope prof("lsa_scatter_rows_kernel", st);
+        LS_CUDA(launch_lsa_scatter_rows(w.fb_list, w.fb_count, c0, fb.rows, w.fb_pick, top_p, run, picked, st));
+      }
     }
   } else {
     TopkParams tp;                        // nothing visible anywhere: every row is padding
@@ -1275,6 +1352,187 @@ ls_status ls_lsa_tree_select(const uint16_t* q_idx, const int64_t* q_pos, const 
   cp.ld_out = top_p;
   s = topk_launch(cp, st);
   if (s != LS_OK) return s;
+  ProfScope prof("lsa_expand_kernel", st);
+  LS_CUDA(launch_lsa_expand(picked, q_pos, T, top_p, bucket_off, bucket_mem, P, block_keys, n_sink, budget, keys_out,
+                            n_sink + block_keys + budget, n_out, st));
+  return LS_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// The shape of a tree search over several node levels: level sizes
+// (size[0] = P), the start level (the lowest with at most start_nodes node
+// buckets, else the top one) and the candidate list width of the levels
+// below it (the beam's children plus the most uncovered entries a level can
+// hold: less than a node block, or what the level above leaves uncovered when
+// it is cut short).
+struct TreePlan {
+  int L = 0, start = 0;
+  int size[kMaxTreeLevels + 1] = {};
+  long long cap = 0;
+};
+
+ls_status tree_plan(int P, const int* level_sizes, int L, int node_block, int fanout, int beam, int start_nodes,
+                    TreePlan* tp) {
+  LS_CHECK_ARG(L >= 1 && L <= kMaxTreeLevels, "L must be in [1, %d] (got %d)", kMaxTreeLevels, L);
+  LS_CHECK_ARG(level_sizes != nullptr, "null level_sizes");
+  LS_CHECK_ARG(P >= 0, "negative size");
+  LS_CHECK_ARG(fanout >= 1 && node_block >= fanout && node_block % fanout == 0,
+               "node_block must be a positive multiple of fanout");
+  LS_CHECK_ARG(beam >= 1 && beam <= kMaxTopK, "beam must be in [1, %d] (got %d)", kMaxTopK, beam);
+  LS_CHECK_ARG(start_nodes >= 1, "start_nodes must be >= 1");
+  tp->L = L;
+  tp->size[0] = P;
+  for (int l = 1; l <= L; ++l) {
+    tp->size[l] = level_sizes[l - 1];
+    LS_CHECK_ARG(tp->size[l] >= 0 && static_cast<int64_t>(tp->size[l]) * fanout <= tp->size[l - 1],
+                 "level %d: %d nodes of %d children each exceed the %d entries below", l, tp->size[l], fanout,
+                 tp->size[l - 1]);
+  }
+  tp->start = L;
+  for (int l = 1; l <= L; ++l)
+    if (tp->size[l] <= start_nodes) {
+      tp->start = l;
+      break;
+    }
+  long long ucap = 0;
+  for (int l = 0; l < tp->start; ++l)
+    ucap = std::max(ucap, std::max<long long>(node_block - 1,
+                                              tp->size[l] - static_cast<long long>(fanout) * tp->size[l + 1]));
+  tp->cap = static_cast<long long>(beam) * fanout + ucap;
+  LS_CHECK_ARG(tp->cap <= (1LL << 30), "candidate lists of %lld entries are too wide", tp->cap);
+  return LS_OK;
+}
+
+struct TreeWorkspace {
+  int32_t* vis;     // [L + 1][T] visible entries per level
+  float* sc;        // [T][size[start]] start-level scores
+  int32_t* beams;   // [2][T][beam] the beams of alternate levels
+  float* cval;      // [T][cap] candidates of one level
+  int32_t* clab;
+  int32_t* nv;      // [T]
+  int32_t* picked;  // [T][top_p]
+  size_t used;
+};
+
+TreeWorkspace carve_tree(void* ws, int T, const TreePlan& tp, int beam, int top_p) {
+  Carver cv(ws);
+  TreeWorkspace w{};
+  w.vis = cv.take<int32_t>(static_cast<size_t>(tp.L + 1) * T);
+  w.sc = cv.take<float>(static_cast<size_t>(T) * tp.size[tp.start]);
+  w.beams = cv.take<int32_t>(2 * static_cast<size_t>(T) * beam);
+  w.cval = cv.take<float>(static_cast<size_t>(T) * tp.cap);
+  w.clab = cv.take<int32_t>(static_cast<size_t>(T) * tp.cap);
+  w.nv = cv.take<int32_t>(T);
+  w.picked = cv.take<int32_t>(static_cast<size_t>(T) * top_p);
+  w.used = cv.used;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ls_lsa_tree_levels_workspace_size(int T, int P, const int* level_sizes, int L, int node_block, int fanout,
+                                         int beam, int start_nodes, int top_p) {
+  if (T <= 0 || top_p <= 0) return 0;
+  TreePlan tp;
+  if (tree_plan(P, level_sizes, L, node_block, fanout, beam, start_nodes, &tp) != LS_OK) return 0;
+  return carve_tree(nullptr, T, tp, beam, top_p).used;
+}
+
+ls_status ls_lsa_tree_levels_select(const uint16_t* q_idx, const int64_t* q_pos, const uint16_t* centroids,
+                                    const uint16_t* const* node_centroids, const int* level_sizes, int L,
+                                    const int32_t* bucket_off, const int32_t* bucket_mem, int T, int d, int P,
+                                    int block_keys, int buckets_per_block, int node_block, int fanout, int beam,
+                                    int start_nodes, int n_sink, int top_p, int budget, int32_t* keys_out,
+                                    int32_t* n_out, int32_t* picked_out, int32_t* beams_out, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  if (d != kLsaDim) return fail(LS_ERR_UNSUPPORTED, "only d=%d is built for the LSA index space (got %d)", kLsaDim, d);
+  LS_CHECK_ARG(T >= 0, "negative size");
+  TreePlan tp;
+  ls_status s = tree_plan(P, level_sizes, L, node_block, fanout, beam, start_nodes, &tp);
+  if (s != LS_OK) return s;
+  LS_CHECK_ARG(block_keys >= 1 && buckets_per_block >= 1, "block_keys and buckets_per_block must be >= 1");
+  LS_CHECK_ARG(n_sink >= 0 && budget >= 1, "n_sink must be >= 0 and budget >= 1");
+  LS_CHECK_ARG(top_p >= 1 && top_p <= kMaxTopK, "top_p must be in [1, %d] (got %d)", kMaxTopK, top_p);
+  if (T == 0) return LS_OK;
+  LS_CHECK_ARG(q_idx && q_pos && centroids && bucket_off && bucket_mem && keys_out && n_out && node_centroids,
+               "null tensor pointer");
+  LS_CHECK_ARG(aligned16(q_idx) && aligned16(centroids), "q_idx and the centroids must be 16-byte aligned");
+  for (int l = 1; l <= L; ++l)
+    LS_CHECK_ARG(tp.size[l] == 0 || (node_centroids[l - 1] != nullptr && aligned16(node_centroids[l - 1])),
+                 "level %d node centroids must be non-null and 16-byte aligned", l);
+  const size_t need = ls_lsa_tree_levels_workspace_size(T, P, level_sizes, L, node_block, fanout, beam, start_nodes,
+                                                        top_p);
+  if (ws_bytes < need || !ws) return fail(LS_ERR_WORKSPACE, "workspace %zu B < %zu B", ws_bytes, need);
+  const TreeWorkspace w = carve_tree(ws, T, tp, beam, top_p);
+  const int cap = static_cast<int>(tp.cap);
+  int32_t* picked = picked_out ? picked_out : w.picked;
+  auto beam_of = [&](int l) {   // level l's beam (1 <= l <= start)
+    return beams_out ? beams_out + static_cast<size_t>(l - 1) * T * beam
+                     : w.beams + ((l & 1) ? static_cast<size_t>(T) * beam : 0);
+  };
+  auto vis_of = [&](int l) { return w.vis + static_cast<size_t>(l) * T; };
+  cudaStream_t st = S(stream);
+  {
+    ProfScope prof("lsa_tree_levels_visible_kernel", st);
+    LS_CUDA(launch_lsa_tree_levels_visible(q_pos, T, block_keys, buckets_per_block, node_block, fanout, tp.size, L,
+                                           w.vis, st));
+  }
+  // the start level: every visible node scored, the best `beam` kept
+  const int S0 = tp.start;
+  const int PS = tp.size[S0];
+  if (PS > 0) {
+    CUtensorMap cmap, qmap;
+    s = make_vec64_map(&cmap, node_centroids[S0 - 1], static_cast<uint64_t>(PS), kTileKeys);
+    if (s != LS_OK) return s;
+    s = make_vec64_map(&qmap, q_idx, static_cast<uint64_t>(T), DotCfg::QB);
+    if (s != LS_OK) return s;
+    DotParams dp;
+    dp.T = T;
+    dp.P = PS;
+    dp.out = w.sc;
+    dp.ld_out = PS;
+    ProfScope prof("dot_tc_kernel:nodes", st);
+    LS_CUDA(launch_dot_tc(&cmap, &qmap, dp, num_sms_current(), st));
+  }
+  TopkParams bp;
+  bp.scores = w.sc;
+  bp.ld = PS;
+  bp.n_valid = vis_of(S0);
+  bp.R = T;
+  bp.N = PS;
+  bp.k = beam;
+  bp.idx_out = beam_of(S0);
+  bp.ld_out = beam;
+  s = topk_launch(bp, st, "topk_kernel:beam");
+  if (s != LS_OK) return s;
+  // each level below: the beam's children and the uncovered entries, scored;
+  // the best `beam` of them (top_p at the bucket level)
+  for (int l = S0 - 1; l >= 0; --l) {
+    const uint16_t* c = (l == 0) ? centroids : node_centroids[l - 1];
+    {
+      ProfScope prof("lsa_tree_candidates_kernel", st);
+      LS_CUDA(launch_lsa_tree_candidates(q_idx, c, beam_of(l + 1), beam, vis_of(l), vis_of(l + 1), T, fanout, cap,
+                                         w.cval, w.clab, w.nv, st));
+    }
+    TopkParams cp;
+    cp.scores = w.cval;
+    cp.ld = cap;
+    cp.n_valid = w.nv;
+    cp.labels = w.clab;
+    cp.ld_labels = cap;
+    cp.R = T;
+    cp.N = cap;
+    cp.k = (l > 0) ? beam : top_p;
+    cp.idx_out = (l > 0) ? beam_of(l) : picked;
+    cp.ld_out = cp.k;
+    s = topk_launch(cp, st, l > 0 ? "topk_kernel:beam" : "topk_kernel");
+    if (s != LS_OK) return s;
+  }
   ProfScope prof("lsa_expand_kernel", st);
   LS_CUDA(launch_lsa_expand(picked, q_pos, T, top_p, bucket_off, bucket_mem, P, block_keys, n_sink, budget, keys_out,
                             n_sink + block_keys + budget, n_out, st));

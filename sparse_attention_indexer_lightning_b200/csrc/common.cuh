@@ -77,6 +77,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// The dynamic shared block rounded up to a 1024-byte boundary by pointer
+// arithmetic on the shared array itself, so accesses through the result (and
+// pointers derived from it) stay shared loads, stores and atomics rather than
+// generic ones.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* raw) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
+  return raw + ((1024u - (a & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -89,14 +98,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, letting the thread sleep up to suspend_ns while the phase is
+// incomplete (it wakes as soon as the phase completes): a waiting warp then
+// takes no issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+constexpr uint32_t kWaitSuspendNs = 20000;
+
 // Bounded wait for the phase with the given parity.  Returns false (and sets
 // the CTA abort flag and the global fault word) when the limit runs out or
 // another role of the CTA has already aborted.
+// kSleep = false keeps the plain test (the indexer scorer, whose short
+// units measured a little faster with it).
+template <bool kSleep = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (kSleep ? mbar_try_wait_sleep(bar, parity, kWaitSuspendNs) : mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > LSI_WAIT_LIMIT_NS) {
       *abort_flag = 1;
@@ -109,7 +137,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // Drain wait: bounded by time only (used after an abort).
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, kWaitSuspendNs)) {
     if (globaltimer_ns() - t0 > LSI_WAIT_LIMIT_NS) {
       atomicOr(&g_fault, FAULT_WAIT_TIMEOUT);
       return;
@@ -119,9 +147,10 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 
 // Warp-uniform bounded wait: lane 0 waits, every lane gets its verdict, so
 // warp-collective instructions after the wait never see a partial warp.
+template <bool kSleep = true>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait<kSleep>(bar, parity, abort_flag);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 

@@ -13,6 +13,7 @@ constexpr int kDim = 128;    // indexer key / query width
 constexpr int kTileKeys = 128;
 constexpr int kMaxTopK = 4096;
 constexpr int kLsaDim = 64;    // native LSA index space width
+constexpr int kMaxTreeLevels = 16;   // node levels of the LSA tree search
 
 // ---------------------------------------------------------------- scoring
 // Tensor-core scoring of bf16 keys read by TMA.  One launch covers B
@@ -85,11 +86,14 @@ struct DotParams {
   const int32_t* vis = nullptr;       // [T] visible buckets per row
   const float* tau = nullptr;         // thresholds, tau[t * ld_tau]
   int64_t ld_tau = 0;
-  // row t's list is split into nseg segments of seg entries, one per CTA
-  // (nseg = the grid size): [T][nseg][seg], counts [T][nseg] zeroed before the launch
-  float* cand_val = nullptr;
-  int32_t* cand_lab = nullptr;
-  int nseg = 0, seg = 0;
+  // row t's list (ld_cand (score bits, bucket) pairs at t * ld_cand) is
+  // split into the segments lsa_segment() gives, one per CTA that scores the
+  // row, each in four quarters (one per TMEM lane quadrant: the epilogue
+  // warps that read it); counts [T][nseg][4] (nseg: the most CTAs one query
+  // group meets), zeroed before the launch
+  uint2* cand_list = nullptr;
+  int64_t ld_cand = 0;
+  int nseg = 0, cap2 = 0, slack = 0;
   uint32_t* cand_cnt = nullptr;
   int32_t* row_over = nullptr;        // [T]
   int* any_over = nullptr;
@@ -97,19 +101,63 @@ struct DotParams {
 };
 cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, const DotParams& p, int num_sms,
                           cudaStream_t st);
+
+// The filter form's list segments.  The scan's `grid` CTAs take contiguous
+// runs of its units = G * NT (query group major, NT centroid tiles per
+// group), so a query group is scored by a few consecutive CTAs, or by all of
+// them when there is one group.  CTA c's segment of a row of group g holds
+// cap2 * (the group's tiles it scores) / NT entries plus `slack`, the
+// segments of one row laid out in order of c (index j = c - the group's
+// first CTA); len = 0 when c scores none of the group.
+struct LsaSeg {
+  int64_t off;
+  int len, j;
+};
+__host__ __device__ inline int lsa_first_cta(long long units, int grid, int NT, int g) {
+  // the last CTA whose run starts at or before the group's first unit
+  const long long x = static_cast<long long>(g) * NT;
+  const long long c = ((x + 1) * grid + units - 1) / units - 1;
+  return static_cast<int>(c < 0 ? 0 : (c >= grid ? grid - 1 : c));
+}
+__host__ __device__ inline LsaSeg lsa_segment(long long units, int grid, int NT, int g, int c, int cap2, int slack) {
+  const long long gl = static_cast<long long>(g) * NT;
+  const long long ub = units * c / grid, ue = units * (c + 1) / grid;
+  const long long lo = (ub > gl ? ub : gl) - gl;
+  const long long hi = (ue < gl + NT ? ue : gl + NT) - gl;
+  LsaSeg s{0, 0, c - lsa_first_cta(units, grid, NT, g)};
+  if (hi <= lo) return s;
+  const long long a = static_cast<long long>(cap2) * lo / NT, b = static_cast<long long>(cap2) * hi / NT;
+  s.off = a + static_cast<long long>(slack) * s.j;
+  s.len = static_cast<int>(b - a) + slack;
+  return s;
+}
+// The most CTAs one query group can meet (each CTA takes at least
+// floor(units / grid) units).
+inline int lsa_max_segments(long long units, int grid, int NT) {
+  const long long per = units / grid > 0 ? units / grid : 1;
+  const long long k = NT / per + 2;
+  return static_cast<int>(k < grid ? k : grid);
+}
 // vis[t] = min(P, bpb * floor(q_pos[t] / block_keys)); n_samp[t] = ceil(vis[t] / stride) (if n_samp).
 cudaError_t launch_lsa_visible(const int64_t* q_pos, int T, int block_keys, int bpb, int P, int stride, int32_t* vis,
                                int32_t* n_samp, cudaStream_t st);
-// ss[t][i] = q[t] . c[i * stride], i < n_samp.
-cudaError_t launch_lsa_sample(const uint16_t* q, const uint16_t* c, int T, int n_samp, int stride, float* ss,
-                              cudaStream_t st);
 // The grid size the LSA scan launches with (the filter form's segment count).
 int dot_tc_grid(int T, int P, int num_sms);
-// Pack each row's per-CTA segments into cval / clab [T][cap] (nv[t] entries);
+// Pack each row's segments into cval / clab [T][cap] (nv[t] entries);
 // flag rows that ran over or hold fewer than min(top_p, vis[t]).
-cudaError_t launch_lsa_compact(const float* sval, const int32_t* slab, const uint32_t* cnt, int nseg, int seg,
+cudaError_t launch_lsa_compact(const uint2* slist, const uint32_t* cnt, const DotParams& fp, int grid,
                                const int32_t* vis, int T, int top_p, int cap, float* cval, int32_t* clab, int32_t* nv,
                                int32_t* row_over, int* any_over, cudaStream_t st);
+// The threshold form's fallback: the missed rows listed (ascending), then
+// scored in full `rows` at a time: their queries gathered, the chunk's picks
+// written back (launches that return at once when run_if[0] == 0).
+cudaError_t launch_lsa_flag_list(const int32_t* row_over, int T, int rows, int n_chunks, int32_t* list,
+                                 int32_t* count, int32_t* run, cudaStream_t st);
+cudaError_t launch_lsa_gather_rows(const int32_t* list, const int32_t* count, int c0, int rows, const uint16_t* q,
+                                   const int32_t* vis, const int32_t* run_if, uint16_t* qbuf, int32_t* vbuf,
+                                   cudaStream_t st);
+cudaError_t launch_lsa_scatter_rows(const int32_t* list, const int32_t* count, int c0, int rows, const int32_t* pbuf,
+                                    int top_p, const int32_t* run_if, int32_t* picked, cudaStream_t st);
 // The read list of each query: sinks below its window, the window, then the
 // picked buckets' members best first (sinks and window skipped) up to budget.
 cudaError_t launch_lsa_expand(const int32_t* picked, const int64_t* q_pos, int T, int top_p, const int32_t* off,

@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(CvtCfg<FMT>::THREADS, 1)
     score_cvt_kernel(const __grid_constant__ CUtensorMap qmap, const CvtParams p) {
   using C = CvtCfg<FMT>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* sR = smem;
   uint8_t* sA = smem + C::SMEM_RAW;
   uint8_t* sB = sA + C::SMEM_A;

@@ -45,12 +45,13 @@ struct DotCfg {
   static constexpr size_t SMEM_A = size_t(STAGES) * A_BYTES;
   static constexpr size_t SMEM_B = size_t(2) * B_BYTES;
   static constexpr size_t SMEM_BAR = 512;
-  // filter form, per epilogue warp: each column's ballot and list base (64 x
-  // 2 words) and each lane's listed (score, column) pairs (LIST per lane)
-  static constexpr int LIST = 16;
-  static constexpr size_t SMEM_COL = 64 * 2 * 4;
-  static constexpr size_t SMEM_LST = 32 * LIST * 8;
-  static constexpr size_t SMEM_F = size_t(EPI_WARPS) * (SMEM_COL + SMEM_LST);
+  // filter form, per epilogue warp: its 64 queries' negated thresholds and
+  // visible counts, its slot counters of their list segments, a copy of each
+  // lane's 32 scores of a half (read back for the listed ones) and a queue of
+  // QUEUE listed (score bits, bucket, column) entries
+  static constexpr int QUEUE = 64;
+  static constexpr size_t SMEM_FW = 64 * 4 * 3 + 32 * 32 * 4 + QUEUE * 4 * 3;
+  static constexpr size_t SMEM_F = size_t(EPI_WARPS) * SMEM_FW;
   static constexpr size_t SMEM_TOTAL = 1024 /*align slack*/ + SMEM_A + SMEM_B + SMEM_BAR + SMEM_F;
   static_assert(SMEM_TOTAL <= 232448, "shared memory budget");
   static_assert(DIM * 2 == 128, "one 128-byte swizzle row per vector");
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
   if (p.run_if != nullptr && *p.run_if == 0) return;  // a conditional launch with nothing to do
   const int T = p.T, P = p.P;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::SMEM_A;
   DotBarriers* bars = reinterpret_cast<DotBarriers*>(smem + C::SMEM_A + C::SMEM_B);
@@ -223,25 +224,80 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
-    // filter form: lane l holds the threshold and visible count of the warp's
-    // queries t0 + l and t0 + 32 + l (reloaded when the group changes; a query
-    // past the end sees nothing), vis_min the smallest of the 64 counts
-    float thr_a = 0.f, thr_b = 0.f;
-    int vis_a = 0, vis_b = 0, vis_min = 0;
+    // filter form: the warp's 64 queries' negated thresholds and visible
+    // counts in shared memory (reloaded when the group changes; a query past the end
+    // sees nothing), vis_min the smallest count; the warp appends to its own
+    // quarter (by lane quadrant) of this CTA's segment of each row's list,
+    // with slot counters in shared memory that no other warp touches, written
+    // out when the group changes and at the end.
+    float* thr_s = reinterpret_cast<float*>(sfilt + (warp - 2) * C::SMEM_FW);
+    int* vis_s = reinterpret_cast<int*>(thr_s + 64);
+    uint32_t* cnt_s = reinterpret_cast<uint32_t*>(vis_s + 64);
+    // lane l's scores at row l (128 bytes), 16-byte chunk q stored at chunk
+    // q ^ (l & 7) so that the 32 lanes' 16-byte stores spread over the banks
+    uint4* spill = reinterpret_cast<uint4*>(cnt_s + 64) + lane * 8;
+    uint32_t* q_val = reinterpret_cast<uint32_t*>(reinterpret_cast<uint4*>(cnt_s + 64) + 32 * 8);
+    int32_t* q_pc = reinterpret_cast<int32_t*>(q_val + C::QUEUE);
+    int32_t* q_col = q_pc + C::QUEUE;
+    int qn = 0;                               // queued entries (warp-uniform)
+    int vis_min = 0;
+    LsaSeg seg{0, 0, 0};
+    int64_t sub_off = 0;
+    uint32_t sub_len = 0;
+    int cur_t0 = -1;                          // the rows whose counters are live
+    // the queued entries take their slots (one shared atomic each, up to 32
+    // at a time) and go to the current group's list segments
+    auto drain = [&](int t0d) {
+      __syncwarp();
+      for (int e = lane; e < qn; e += 32) {
+        const int c = q_col[e];
+        const int t = t0d + c;
+        const uint32_t slot = atomicAdd(&cnt_s[c], 1u);
+        if (slot < sub_len) {
+          p.cand_list[static_cast<int64_t>(t) * p.ld_cand + sub_off + slot] =
+              make_uint2(q_val[e], static_cast<uint32_t>(q_pc[e]));
+        } else {
+          p.row_over[t] = 1;
+          *p.any_over = 1;
+        }
+      }
+      qn = 0;
+      __syncwarp();
+    };
+    auto flush = [&](int t0f) {
+      drain(t0f);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = t0f + 32 * h + lane;
+        if (t < T && seg.j < p.nseg)
+          p.cand_cnt[(static_cast<int64_t>(t) * p.nseg + seg.j) * 4 + quad] = cnt_s[32 * h + lane];
+      }
+    };
     UnitPos up;
     up.init(u_begin, NT, G);
     for (long long u = u_begin; u < u_end; ++u, up.next(NT, G)) {
       const int pc = up.tile * C::BM + quad * 32 + lane;     // this thread's centroid
       const int t0 = up.g * C::QB + cset * C::COLS_PER_WARP;
       if (FILTER && (u == u_begin || up.tile == 0)) {
-        const int ta = t0 + lane, tb = t0 + 32 + lane;
-        thr_a = (ta < T) ? p.tau[static_cast<int64_t>(ta) * p.ld_tau] : 0.f;
-        thr_b = (tb < T) ? p.tau[static_cast<int64_t>(tb) * p.ld_tau] : 0.f;
-        vis_a = (ta < T) ? p.vis[ta] : 0;
-        vis_b = (tb < T) ? p.vis[tb] : 0;
-        vis_min = min(vis_a, vis_b);
+        if (cur_t0 >= 0) flush(cur_t0);
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int t = t0 + 32 * h + lane;
+          thr_s[32 * h + lane] = (t < T) ? -p.tau[static_cast<int64_t>(t) * p.ld_tau] : 0.f;   // negated
+          vis_s[32 * h + lane] = (t < T) ? p.vis[t] : 0;
+          cnt_s[32 * h + lane] = 0;
+        }
+        vis_min = min(vis_s[lane], vis_s[32 + lane]);
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) vis_min = min(vis_min, __shfl_xor_sync(0xffffffffu, vis_min, d));
+        seg = lsa_segment(units, static_cast<int>(gridDim.x), NT, up.g, static_cast<int>(blockIdx.x), p.cap2,
+                          p.slack);
+        if (seg.j >= p.nseg) seg.len = 0;     // no counter for it: every listed pair flags its row
+        sub_len = static_cast<uint32_t>(seg.len / 4);
+        sub_off = seg.off + static_cast<int64_t>(quad) * sub_len;
+        cur_t0 = t0;
+        __syncwarp();
       }
       if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
@@ -270,97 +326,87 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
             if (32 + j < nt) o[static_cast<int64_t>(32 + j) * p.ld_out] = __uint_as_float(v1[j]);
         }
       } else {
-        // Pass 1: one ballot per query column (lane j keeps the ballots of
-        // columns j and 32 + j); each lane notes its listed (score, column)
-        // pairs in shared memory.  Pass 2: every lane reserves its two
-        // columns' slots with one atomic each, all in flight together, and
-        // publishes ballot and base.  Pass 3: each lane writes its own pairs.
-        uint32_t* scol = reinterpret_cast<uint32_t*>(sfilt + (warp - 2) * (C::SMEM_COL + C::SMEM_LST));
-        uint2* slst = reinterpret_cast<uint2*>(sfilt + (warp - 2) * (C::SMEM_COL + C::SMEM_LST) + C::SMEM_COL) +
-                      lane * C::LIST;
-        uint32_t bal_a = 0, bal_b = 0;
-        int nl = 0;                                     // this lane's listed pairs
-        // one 32-column half at a time, so only 32 scores are live in registers.
-        // Listed: visible and score >= threshold (as floats: -0 equals +0, a
-        // NaN is never listed, a -inf threshold lists every visible bucket).
-        // A tile below every column's visible count skips the per-column count.
+        // One 32-column half at a time: this lane's listed columns as a bit
+        // mask.  A score is listed when it is visible and not below its
+        // column's threshold in the top-k's key order: the sign bit of
+        // fl(score + (-threshold)) (one rounding, so it is set exactly when
+        // score < threshold, -0 below +0, a NaN score listed like the top
+        // key it is; a -inf threshold lists every visible bucket).  The
+        // sums go two at a time through the packed fp32 adder, their sign
+        // bits are shifted into four 8-bit words (column 4 * i + r at bit
+        // 8 * r + 7 - i of the combined word); a tile below every column's
+        // visible count skips the count.
         const bool all_visible = up.tile * C::BM + C::BM <= vis_min;
+        const float4* nthr4 = reinterpret_cast<const float4*>(thr_s);
+        const int4* vis4 = reinterpret_cast<const int4*>(vis_s);
         uint32_t v[32];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           tmem_ld_32x32_nowait(col + 32 * h, v);
           tmem_wait_ld(v);
           if (h == 1) release();
+          uint32_t neg[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float thr = __shfl_sync(0xffffffffu, h ? thr_b : thr_a, j);
-            const uint32_t sv = v[j];
-            bool take = __uint_as_float(sv) >= thr;
-            if (!all_visible) {                          // warp-uniform: every lane takes part in the shuffle
-              const int vis = __shfl_sync(0xffffffffu, h ? vis_b : vis_a, j);
-              take = take && (pc < vis);
-            }
-            const uint32_t bal = __ballot_sync(0xffffffffu, take);
-            if (lane == j) {
-              if (h) bal_b = bal;
-              else bal_a = bal;
-            }
-            if (take) {
-              if (nl < C::LIST) slst[nl] = make_uint2(sv, static_cast<uint32_t>(32 * h + j));
-              ++nl;
-            }
+          for (int i = 0; i < 8; ++i) {
+            const float4 nt = nthr4[8 * h + i];
+            uint64_t d01, d23;
+            asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d01)
+                : "l"(pack_f32x2(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]))),
+                  "l"(pack_f32x2(nt.x, nt.y)));
+            asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d23)
+                : "l"(pack_f32x2(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]))),
+                  "l"(pack_f32x2(nt.z, nt.w)));
+            float e0, e1, e2, e3;
+            unpack_f32x2(d01, e0, e1);
+            unpack_f32x2(d23, e2, e3);
+            neg[0] = __funnelshift_l(__float_as_uint(e0), neg[0], 1);
+            neg[1] = __funnelshift_l(__float_as_uint(e1), neg[1], 1);
+            neg[2] = __funnelshift_l(__float_as_uint(e2), neg[2], 1);
+            neg[3] = __funnelshift_l(__float_as_uint(e3), neg[3], 1);
           }
-        }
-        uint32_t base_a = 0, base_b = 0;
-        // each CTA appends to its own segment of a row's list (few atomics per address)
-        if (bal_a)
-          base_a = atomicAdd(p.cand_cnt + static_cast<int64_t>(t0 + lane) * p.nseg + blockIdx.x,
-                             static_cast<uint32_t>(__popc(bal_a)));
-        if (bal_b)
-          base_b = atomicAdd(p.cand_cnt + static_cast<int64_t>(t0 + 32 + lane) * p.nseg + blockIdx.x,
-                             static_cast<uint32_t>(__popc(bal_b)));
-        scol[lane] = bal_a;
-        scol[32 + lane] = bal_b;
-        scol[64 + lane] = base_a;
-        scol[96 + lane] = base_b;
-        __syncwarp();
-        const uint32_t below = (1u << lane) - 1u;
-        for (int e = 0; e < nl && e < C::LIST; ++e) {
-          const uint2 pr = slst[e];
-          const int c = static_cast<int>(pr.y);
-          const int t = t0 + c;
-          const uint32_t slot = scol[64 + c] + static_cast<uint32_t>(__popc(scol[c] & below));
-          if (slot < static_cast<uint32_t>(p.seg)) {
-            const int64_t at = (static_cast<int64_t>(t) * p.nseg + blockIdx.x) * p.seg + slot;
-            p.cand_val[at] = __uint_as_float(pr.x);
-            p.cand_lab[at] = pc;
-          } else {
-            p.row_over[t] = 1;
-            *p.any_over = 1;
+          uint32_t mask = ~(neg[0] | (neg[1] << 8) | (neg[2] << 16) | (neg[3] << 24));
+          if (!all_visible) {                           // visible: pc - vis < 0
+            uint32_t vis_neg[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int4 vv = vis4[8 * h + i];
+              vis_neg[0] = __funnelshift_l(static_cast<uint32_t>(pc - vv.x), vis_neg[0], 1);
+              vis_neg[1] = __funnelshift_l(static_cast<uint32_t>(pc - vv.y), vis_neg[1], 1);
+              vis_neg[2] = __funnelshift_l(static_cast<uint32_t>(pc - vv.z), vis_neg[2], 1);
+              vis_neg[3] = __funnelshift_l(static_cast<uint32_t>(pc - vv.w), vis_neg[3], 1);
+            }
+            mask &= vis_neg[0] | (vis_neg[1] << 8) | (vis_neg[2] << 16) | (vis_neg[3] << 24);
           }
-        }
-        if (nl > C::LIST) {
-          // more listed pairs than the lane's buffer holds: rescan for the
-          // columns it could not note and send those rows to the fallback
+          // listed pairs: each lane's next one per round, queued in lane
+          // order (a round rarely repeats: few lanes list two in a half)
+          if (__any_sync(0xffffffffu, mask != 0)) {
+            if (mask) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = 32 * h + j;
-              if (((h ? scol[32 + j] : scol[j]) >> lane) & 1u) {
-                bool noted = false;
-                for (int e = 0; e < C::LIST; ++e) noted |= (static_cast<int>(slst[e].y) == c);
-                if (!noted) {
-                  p.row_over[t0 + c] = 1;
-                  *p.any_over = 1;
-                }
+              for (int q = 0; q < 8; ++q)
+                spill[q ^ (lane & 7)] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+            while (true) {
+              const uint32_t bal = __ballot_sync(0xffffffffu, mask != 0);
+              if (bal == 0) break;
+              const int n = __popc(bal);
+              if (qn + n > C::QUEUE) drain(t0);
+              if (mask) {
+                const int bit = __ffs(mask) - 1;
+                mask &= mask - 1;
+                const int j = 4 * (7 - (bit & 7)) + (bit >> 3);
+                const int e = qn + __popc(bal & ((1u << lane) - 1u));
+                q_val[e] = reinterpret_cast<const uint32_t*>(spill + ((j >> 2) ^ (lane & 7)))[j & 3];
+                q_pc[e] = pc;
+                q_col[e] = 32 * h + j;
               }
+              qn += n;
             }
+            if (qn >= C::QUEUE / 2) drain(t0);
           }
         }
-        __syncwarp();                                   // the warp's shared area is reused next unit
       }
     }
+    if (FILTER && cur_t0 >= 0) flush(cur_t0);
   }
 
   tc_fence_before();
@@ -383,7 +429,13 @@ static cudaError_t launch_dot(const CUtensorMap* cmap, const CUtensorMap* qmap, 
   }
   const int grid = dot_tc_grid(p.T, p.P, num_sms);
   if (grid == 0) return cudaSuccess;
-  if (FILTER && grid > p.nseg) return cudaErrorInvalidValue;   // one list segment per CTA
+  if (FILTER) {                            // the segments must fit the counters and the rows
+    const long long units = static_cast<long long>((p.T + C::QB - 1) / C::QB) * ((p.P + C::BM - 1) / C::BM);
+    const int NT = (p.P + C::BM - 1) / C::BM;
+    if (lsa_max_segments(units, grid, NT) > p.nseg ||
+        p.cap2 + static_cast<long long>(p.slack) * p.nseg > p.ld_cand)
+      return cudaErrorInvalidValue;
+  }
   dot_tc_kernel<FILTER><<<grid, C::THREADS, C::SMEM_TOTAL, st>>>(*cmap, *qmap, p);
   return cudaGetLastError();
 }
@@ -398,61 +450,40 @@ cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, cons
   return p.out == nullptr ? launch_dot<true>(cmap, qmap, p, num_sms, st) : launch_dot<false>(cmap, qmap, p, num_sms, st);
 }
 
-// Visible buckets of each query (causal block visibility: the buckets of the
-// complete blocks before the query's own block) and the LSA read list
-// ("Latent Sparse Attention", section "The method, term by term", steps 5-6):
-//   row t of keys_out: the sinks below the window, then the window
-//   [block_start(t), t], then the long-range keys of the picked buckets read
-//   best first, members that fall in the sinks or the window skipped, until
-//   `budget` are held (the last bucket cut short); -1 after the end; n_out[t]
-//   the row's length.  Bucket members are stored in ascending position order.
-// Sample scores for the thresholds: row t scores the buckets 0, stride,
-// 2*stride, ... below its visible count (the same positions for every row, so
-// the sampled centroids stay in L2): ss[t][i] = q[t] . c[i * stride].
-__global__ void lsa_sample_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ c, int T, int n_samp,
-                                  int stride, float* __restrict__ ss) {
-  const int t = blockIdx.y;
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  __shared__ float qs[kLsaDim];
-  if (threadIdx.x < kLsaDim) qs[threadIdx.x] = __uint_as_float(static_cast<uint32_t>(q[t * kLsaDim + threadIdx.x]) << 16);
-  __syncthreads();
-  if (i >= n_samp) return;
-  const uint4* row = reinterpret_cast<const uint4*>(c + static_cast<int64_t>(i) * stride * kLsaDim);
-  float acc = 0.f;
-#pragma unroll
-  for (int v = 0; v < kLsaDim / 8; ++v) {
-    const uint4 x = __ldg(row + v);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      acc = fmaf(__uint_as_float(w[e] << 16), qs[8 * v + 2 * e], acc);
-      acc = fmaf(__uint_as_float(w[e] & 0xffff0000u), qs[8 * v + 2 * e + 1], acc);
-    }
-  }
-  ss[static_cast<int64_t>(t) * n_samp + i] = acc;
-}
-
-// After the filtered scan, one CTA per row: the row's per-CTA segments are
+// After the filtered scan, one CTA per row: the row's segments (one per CTA
+// of the scan that scored it) are
 // packed into one list of up to `cap` entries (nv[t] of them).  A row falls
 // back to full scoring when a segment ran over (flagged in the scan), the
 // list would exceed cap, or it holds fewer than min(top_p, visible) buckets.
 __global__ void __launch_bounds__(256)
-    lsa_compact_kernel(const float* __restrict__ sval, const int32_t* __restrict__ slab,
-                       const uint32_t* __restrict__ cnt, int nseg, int seg, const int32_t* __restrict__ vis, int top_p,
-                       int cap, float* __restrict__ cval, int32_t* __restrict__ clab, int32_t* __restrict__ nv,
-                       int32_t* __restrict__ row_over, int* __restrict__ any_over) {
+    lsa_compact_kernel(const uint2* __restrict__ slist, const uint32_t* __restrict__ cnt, int64_t ld_cand, int nseg,
+                       int cap2, int slack, int grid, int NT, long long units, const int32_t* __restrict__ vis,
+                       int top_p, int cap, float* __restrict__ cval, int32_t* __restrict__ clab,
+                       int32_t* __restrict__ nv, int32_t* __restrict__ row_over, int* __restrict__ any_over) {
   __shared__ int offs[1025];
+  __shared__ int64_t soff[1024];
   __shared__ int wsum[8];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31, wid = tid >> 5;
-  // exclusive scan of the segment counts (nseg <= 1024: 4 per thread)
+  const int g = t / DotCfg::QB;
+  const int c0 = lsa_first_cta(units, grid, NT, g);
+  const int nsub = 4 * nseg;                  // segment j's quarter q is sub-segment 4 * j + q
+  // exclusive scan of the sub-segment counts (nsub <= 1024: 4 per thread);
+  // a count past its sub-segment's length was flagged by the scan
   int c4[4];
   int mine = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int c = tid * 4 + i;
-    c4[i] = (c < nseg) ? static_cast<int>(min(cnt[static_cast<int64_t>(t) * nseg + c], static_cast<uint32_t>(seg))) : 0;
+    const int sidx = tid * 4 + i;
+    const int j = sidx >> 2, q = sidx & 3;
+    c4[i] = 0;
+    if (sidx < nsub && c0 + j < grid) {
+      const LsaSeg sg = lsa_segment(units, grid, NT, g, c0 + j, cap2, slack);
+      const int sub_len = sg.len / 4;
+      soff[sidx] = sg.off + static_cast<int64_t>(q) * sub_len;
+      c4[i] = static_cast<int>(min(cnt[static_cast<int64_t>(t) * nsub + sidx], static_cast<uint32_t>(sub_len)));
+    }
     mine += c4[i];
   }
   int incl = mine;
@@ -467,13 +498,13 @@ __global__ void __launch_bounds__(256)
   for (int w = 0; w < wid; ++w) run += wsum[w];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int c = tid * 4 + i;
-    if (c < nseg) offs[c] = run;
+    const int sidx = tid * 4 + i;
+    if (sidx < nsub) offs[sidx] = run;
     run += c4[i];
   }
-  if (tid == 255) offs[nseg] = run;
+  if (tid == 255) offs[nsub] = run;
   __syncthreads();
-  const int total = offs[nseg];
+  const int total = offs[nsub];
   const int need = min(top_p, vis[t]);
   if (tid == 0) {
     nv[t] = min(total, cap);
@@ -483,20 +514,94 @@ __global__ void __launch_bounds__(256)
     }
   }
   if (total > cap) return;
-  // output entry o comes from the segment c with offs[c] <= o < offs[c + 1]
+  // output entry o comes from the sub-segment s with offs[s] <= o < offs[s + 1]
   for (int o = tid; o < total; o += 256) {
-    int lo = 0, hi = nseg;                      // offs[lo] <= o < offs[hi]
+    int lo = 0, hi = nsub;                      // offs[lo] <= o < offs[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (offs[mid] <= o) lo = mid;
       else hi = mid;
     }
-    const int64_t src = (static_cast<int64_t>(t) * nseg + lo) * seg + (o - offs[lo]);
-    cval[static_cast<int64_t>(t) * cap + o] = sval[src];
-    clab[static_cast<int64_t>(t) * cap + o] = slab[src];
+    const uint2 e = slist[static_cast<int64_t>(t) * ld_cand + soff[lo] + (o - offs[lo])];
+    cval[static_cast<int64_t>(t) * cap + o] = __uint_as_float(e.x);
+    clab[static_cast<int64_t>(t) * cap + o] = static_cast<int32_t>(e.y);
   }
 }
 
+// The rows the sampled threshold missed, in ascending order: list[0, count)
+// (one CTA); run[c] = 1 when chunk c (rows [c * rows, (c + 1) * rows) of the
+// list) holds any, for c < n_chunks.
+__global__ void __launch_bounds__(1024)
+    lsa_flag_list_kernel(const int32_t* __restrict__ row_over, int T, int rows, int n_chunks,
+                         int32_t* __restrict__ list, int32_t* __restrict__ count, int32_t* __restrict__ run) {
+  __shared__ int wsum[32];
+  __shared__ int base_s;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) base_s = 0;
+  __syncthreads();
+  for (int t0 = 0; t0 < T; t0 += 1024) {
+    const int t = t0 + tid;
+    const int f = (t < T && row_over[t] != 0) ? 1 : 0;
+    const uint32_t bal = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) wsum[wid] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < 32; ++w) {
+      before += (w < wid) ? wsum[w] : 0;
+      total += wsum[w];
+    }
+    const int base = base_s;
+    if (f) list[base + before + __popc(bal & ((1u << lane) - 1u))] = t;
+    __syncthreads();                            // every thread has read base_s and wsum
+    if (tid == 0) base_s = base + total;
+    __syncthreads();
+  }
+  const int n = base_s;
+  if (tid == 0) *count = n;
+  for (int c = tid; c < n_chunks; c += 1024) run[c] = (static_cast<long long>(c) * rows < n) ? 1 : 0;
+}
+
+// Chunk c0 / rows of the missed rows: their index queries and visible counts
+// gathered into qbuf [rows][64] and vbuf [rows] (zeros past the list's end).
+__global__ void lsa_gather_rows_kernel(const int32_t* __restrict__ list, const int32_t* __restrict__ count, int c0,
+                                       int rows, const uint16_t* __restrict__ q, const int32_t* __restrict__ vis,
+                                       const int32_t* __restrict__ run_if, uint16_t* __restrict__ qbuf,
+                                       int32_t* __restrict__ vbuf) {
+  if (*run_if == 0) return;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;   // one 16-byte piece: row i / 8, piece i % 8
+  if (i >= rows * 8) return;
+  const int r = i >> 3, piece = i & 7;
+  const bool live = c0 + r < *count;
+  const int t = live ? list[c0 + r] : 0;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (live) v = reinterpret_cast<const uint4*>(q + static_cast<int64_t>(t) * kLsaDim)[piece];
+  reinterpret_cast<uint4*>(qbuf + static_cast<int64_t>(r) * kLsaDim)[piece] = v;
+  if (piece == 0) vbuf[r] = live ? vis[t] : 0;
+}
+
+// The picks of that chunk written back to the rows they belong to.
+__global__ void lsa_scatter_rows_kernel(const int32_t* __restrict__ list, const int32_t* __restrict__ count, int c0,
+                                        int rows, const int32_t* __restrict__ pbuf, int top_p,
+                                        const int32_t* __restrict__ run_if, int32_t* __restrict__ picked) {
+  if (*run_if == 0) return;
+  const int r = blockIdx.x;
+  if (r >= rows || c0 + r >= *count) return;
+  const int t = list[c0 + r];
+  for (int j = threadIdx.x; j < top_p; j += blockDim.x)
+    picked[static_cast<int64_t>(t) * top_p + j] = pbuf[static_cast<int64_t>(r) * top_p + j];
+}
+
+// Visible buckets of each query (causal block visibility: the buckets of the
+// complete blocks before the query's own block) and the LSA read list
+// ("Latent Sparse Attention", section "The method, term by term", steps 5-6):
+//   row t of keys_out: the sinks below the window, then the window
+//   [block_start(t), t], then the long-range keys of the picked buckets read
+//   best first, members that fall in the sinks or the window skipped, until
+//   `budget` are held (the last bucket cut short); -1 after the end; n_out[t]
+//   the row's length.  Bucket members are stored in ascending position order.
+// The sample scores for the thresholds are the tensor-core scorer's, over the
+// buckets 0, stride, 2*stride, ...; n_samp[t] counts those below row t's
+// visible count.
 __global__ void lsa_visible_kernel(const int64_t* __restrict__ q_pos, int T, int block_keys, int bpb, int P,
                                    int stride, int32_t* __restrict__ vis, int32_t* __restrict__ n_samp) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -606,20 +711,37 @@ cudaError_t launch_lsa_visible(const int64_t* q_pos, int T, int block_keys, int 
   return cudaGetLastError();
 }
 
-cudaError_t launch_lsa_sample(const uint16_t* q, const uint16_t* c, int T, int n_samp, int stride, float* ss,
-                              cudaStream_t st) {
-  if (T == 0 || n_samp == 0) return cudaSuccess;
-  lsa_sample_kernel<<<dim3((n_samp + 255) / 256, T), 256, 0, st>>>(q, c, T, n_samp, stride, ss);
+cudaError_t launch_lsa_compact(const uint2* slist, const uint32_t* cnt, const DotParams& fp, int grid,
+                               const int32_t* vis, int T, int top_p, int cap, float* cval, int32_t* clab, int32_t* nv,
+                               int32_t* row_over, int* any_over, cudaStream_t st) {
+  if (T == 0 || grid == 0) return cudaSuccess;
+  if (4 * fp.nseg > 1024) return cudaErrorInvalidValue;
+  const int NT = (fp.P + DotCfg::BM - 1) / DotCfg::BM;
+  const long long units = static_cast<long long>((T + DotCfg::QB - 1) / DotCfg::QB) * NT;
+  lsa_compact_kernel<<<T, 256, 0, st>>>(slist, cnt, fp.ld_cand, fp.nseg, fp.cap2, fp.slack, grid, NT, units, vis,
+                                        top_p, cap, cval, clab, nv, row_over, any_over);
   return cudaGetLastError();
 }
 
-cudaError_t launch_lsa_compact(const float* sval, const int32_t* slab, const uint32_t* cnt, int nseg, int seg,
-                               const int32_t* vis, int T, int top_p, int cap, float* cval, int32_t* clab, int32_t* nv,
-                               int32_t* row_over, int* any_over, cudaStream_t st) {
+cudaError_t launch_lsa_flag_list(const int32_t* row_over, int T, int rows, int n_chunks, int32_t* list,
+                                 int32_t* count, int32_t* run, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  if (nseg > 1024) return cudaErrorInvalidValue;
-  lsa_compact_kernel<<<T, 256, 0, st>>>(sval, slab, cnt, nseg, seg, vis, top_p, cap, cval, clab, nv, row_over,
-                                        any_over);
+  lsa_flag_list_kernel<<<1, 1024, 0, st>>>(row_over, T, rows, n_chunks, list, count, run);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsa_gather_rows(const int32_t* list, const int32_t* count, int c0, int rows, const uint16_t* q,
+                                   const int32_t* vis, const int32_t* run_if, uint16_t* qbuf, int32_t* vbuf,
+                                   cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  lsa_gather_rows_kernel<<<(rows * 8 + 255) / 256, 256, 0, st>>>(list, count, c0, rows, q, vis, run_if, qbuf, vbuf);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsa_scatter_rows(const int32_t* list, const int32_t* count, int c0, int rows, const int32_t* pbuf,
+                                    int top_p, const int32_t* run_if, int32_t* picked, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  lsa_scatter_rows_kernel<<<rows, 256, 0, st>>>(list, count, c0, rows, pbuf, top_p, run_if, picked);
   return cudaGetLastError();
 }
 

@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(Q8Cfg<FMT, HALVES>::THREADS, 1)
                     const CvtParams p) {
   using C = Q8Cfg<FMT, HALVES>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* sR = smem;
   uint8_t* sB = sR + C::SMEM_RAW;
   uint8_t* sS = sB + C::SMEM_B;

@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
   using C = TcCfg<QG, FILTER, F8>;
   if (p.run_if != nullptr && *p.run_if == 0) return;  // a conditional launch with nothing to do
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::SMEM_A;
   TcBarriers* bars = reinterpret_cast<TcBarriers*>(smem + C::SMEM_A + C::SMEM_B);
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
         const long long bg = static_cast<long long>(b) * G + g;
         if (bg != prev_bg) {
           bslot = (bslot + 1 == C::BSLOTS) ? 0 : bslot + 1;
-          if (!mbar_wait(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait<false>(&bars->bempty[bslot], bphase[bslot] ^ 1, abort_flag)) { ok = false; break; }
           b_par[bslot] = bphase[bslot];
           b_issued[bslot] = 1;
           bphase[bslot] ^= 1;
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
           if (C::PANELS == 2) tma_load_2d(dst + C::B_HALF, &qmap, &bars->bfull[bslot], 64, qrow);
           prev_bg = bg;
         }
-        if (!mbar_wait(&bars->empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait<false>(&bars->empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars->full[stage], C::A_BYTES);
         const int krow = b * p.N + tile * C::BM;
         uint8_t* dst = sA + stage * C::A_BYTES;
@@ -239,13 +239,13 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
           else if (lane == 0) umma_commit(&bars->bempty[bslot]);
         }
         bslot = (bslot + 1 == C::BSLOTS) ? 0 : bslot + 1;
-        if (!warp_wait(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
+        if (!warp_wait<false>(&bars->bfull[bslot], bphase[bslot], abort_flag)) break;
         bphase[bslot] ^= 1;
         prev_bg = bg;
       }
-      if (!warp_wait(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
+      if (!warp_wait<false>(&bars->tempty[acc], acc_phase ^ 1, abort_flag)) break;
       tc_fence_after();
-      if (!warp_wait(&bars->full[stage], phase, abort_flag)) break;
+      if (!warp_wait<false>(&bars->full[stage], phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t a_addr = a_base + stage * C::A_BYTES;
       const uint32_t b_addr = b_base + bslot * C::B_BYTES;
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(TcCfg<QG, FILTER, F8>::THREADS, 1)
       }
       float ks = 1.f;                                      // fp8: the key's scale, loaded ahead of the wait
       if (F8) ks = (n < p.N) ? __ldg(p.key_scale + static_cast<int64_t>(hb) * p.N + n) : 0.f;
-      if (!warp_wait(&bars->tfull[acc], acc_phase, abort_flag)) break;
+      if (!warp_wait<false>(&bars->tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * C::ACC_COLS + qset * C::Q_PER_EPI_WARP * kHeads);

@@ -11,9 +11,11 @@
 //  * lsa_tree_visible: per query, visible buckets (complete key blocks
 //    before its own) and visible node buckets (complete node blocks among
 //    those).
+//  * lsa_tree_levels_visible: the same per level of a tree of several node
+//    levels (level l groups the complete node blocks of level l - 1).
 //  * lsa_tree_candidates: one CTA per query lists and scores its candidate
-//    buckets: the children of its beam, then the visible buckets past the
-//    last complete node block.
+//    entries of one level: the children of its beam (nodes of the level
+//    above), then the visible entries past the last complete node block.
 
 #pragma once
 
@@ -33,6 +35,31 @@ __global__ void lsa_tree_visible_kernel(const int64_t* __restrict__ q_pos, int T
   vis[t] = vv;
   const int64_t vn = static_cast<int64_t>(vv / node_block) * (node_block / fanout);
   vis_nodes[t] = static_cast<int32_t>(vn < P1 ? vn : P1);
+}
+
+// Visible entries of every level of a tree of several node levels:
+// vis[0][t] = visible buckets, vis[l][t] = the level-l nodes of the complete
+// node blocks among the query's visible level-(l-1) entries, capped at the
+// level's size (size[l]; size[0] = P).  vis is [n + 1][T].
+struct TreeLevels {
+  int n = 0;
+  int size[kMaxTreeLevels + 1] = {};
+};
+
+__global__ void lsa_tree_levels_visible_kernel(const int64_t* __restrict__ q_pos, int T, int block_keys, int bpb,
+                                               int node_block, int fanout, const TreeLevels lv,
+                                               int32_t* __restrict__ vis) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int64_t qp = q_pos[t] < 0 ? 0 : q_pos[t];
+  int64_t v = (qp / block_keys) * bpb;
+  v = v < lv.size[0] ? v : lv.size[0];
+  vis[t] = static_cast<int32_t>(v);
+  for (int l = 1; l <= lv.n; ++l) {
+    v = (v / node_block) * (node_block / fanout);
+    v = v < lv.size[l] ? v : lv.size[l];
+    vis[static_cast<int64_t>(l) * T + t] = static_cast<int32_t>(v);
+  }
 }
 
 // q . c over 64 bf16 dimensions with the query held as 32 packed fp32 pairs:
@@ -105,6 +132,19 @@ cudaError_t launch_lsa_tree_visible(const int64_t* q_pos, int T, int block_keys,
   if (T == 0) return cudaSuccess;
   lsa_tree_visible_kernel<<<(T + 255) / 256, 256, 0, st>>>(q_pos, T, block_keys, bpb, P, node_block, fanout, P1, vis,
                                                            vis_nodes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lsa_tree_levels_visible(const int64_t* q_pos, int T, int block_keys, int bpb, int node_block,
+                                           int fanout, const int* sizes, int n_levels, int32_t* vis,
+                                           cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (n_levels < 1 || n_levels > kMaxTreeLevels) return cudaErrorInvalidValue;
+  TreeLevels lv;
+  lv.n = n_levels;
+  for (int l = 0; l <= n_levels; ++l) lv.size[l] = sizes[l];
+  lsa_tree_levels_visible_kernel<<<(T + 255) / 256, 256, 0, st>>>(q_pos, T, block_keys, bpb, node_block, fanout, lv,
+                                                                  vis);
   return cudaGetLastError();
 }
 

@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           int64_t n_rows, float scale, int foreign_ok, float* __restrict__ out,
                           float* __restrict__ lse) {
   extern __shared__ uint8_t attn_tc_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(attn_tc_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(attn_tc_raw);
   int32_t* ids = reinterpret_cast<int32_t*>(smem + kTcOffIds);
   AttnTcBars* bars = reinterpret_cast<AttnTcBars*>(smem + kTcOffBars);
   volatile int* abort_flag = &bars->abort_flag;

@@ -30,7 +30,8 @@ def test_header_declares_the_calls():
     for n in ("ls_indexer_score", "ls_topk_select", "ls_prefill_select_stream", "ls_decode_two_stage_select",
               "ls_bucket_select", "ls_decode_select", "ls_last_error", "ls_device_status", "ls_indexer_score_fp8",
               "ls_prefill_select_stream_fp8", "ls_lsa_flat_select", "ls_lsa_tree_select", "ls_indexer_score_pq",
-              "ls_decode_two_stage_pq_select", "ls_merge_select", "ls_sparse_attention", "ls_attention_merge"):
+              "ls_decode_two_stage_pq_select", "ls_merge_select", "ls_sparse_attention", "ls_attention_merge",
+              "ls_lsa_tree_levels_select"):
         assert n in names
 
 
@@ -57,15 +58,30 @@ def test_version_and_workspace_queries(lib):
     assert (lib.ls_prefill_select_fp8_workspace_size(4096, 32768, 8192, 512, 1)
             >= lib.ls_prefill_select_workspace_size(4096, 32768, 8192, 512, 1) + 4096 * 32 * 4)
     # LSA: the T x P bucket scores, visible counts and picks
-    assert lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) >= 256 * 131072 * 4 + 256 * 1024 * 4
+    assert lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0, 0) >= 256 * 131072 * 4 + 256 * 1024 * 4
     # LSA tree: node scores, beam and candidates (beam * fanout + node_block per row)
     assert lib.ls_lsa_tree_workspace_size(256, 32768, 2048, 4, 4096, 1024) >= 256 * 32768 * 4 + 256 * 12288 * 8
+    # LSA tree over three node levels at 10M tokens: starts at level 3 (20480 nodes); candidate rows of
+    # beam * fanout + node_block - 1 entries; invalid level sizes answer 0
+    import ctypes
+    sizes = (ctypes.c_int * 3)(327680, 81920, 20480)
+    ws3 = lib.ls_lsa_tree_levels_workspace_size(256, 1310720, sizes, 3, 4096, 4, 2048, 32768, 1024)
+    assert ws3 >= 256 * 20480 * 4 + 256 * (8192 + 4095) * 8 + 2 * 256 * 2048 * 4 + 4 * 256 * 4
+    assert ws3 < 256 * 81920 * 4                # the level-2 scores are never held
+    bad = (ctypes.c_int * 3)(327681, 81920, 20480)
+    assert lib.ls_lsa_tree_levels_workspace_size(256, 1310720, bad, 3, 4096, 4, 2048, 32768, 1024) == 0
+    assert lib.ls_lsa_tree_levels_workspace_size(256, 1310720, sizes, 0, 4096, 4, 2048, 32768, 1024) == 0
     # shard merge: the packed S * k_in candidates per row (values and positions) and the row counts
     assert lib.ls_merge_select_workspace_size(4, 4096, 512) >= 4096 * 4 * 512 * 8 + 4096 * 4
     assert lib.ls_merge_select_workspace_size(0, 4096, 512) == 0
     # the threshold form adds the samples and the candidate lists (8 * top_p per row)
-    assert (lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 1)
-            >= lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0) + 256 * 8192 * 8)
+    assert (lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 1, 0)
+            >= lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0, 0) + 256 * 8192 * 8)
+    # ... but never the T x P matrix at prefill scale: 32768 queries x 1310720 buckets (172 GB) fit in
+    # about 20 GB, the fallback's scores within 4 GiB (or fallback_rows x P)
+    big = lib.ls_lsa_flat_workspace_size(32768, 1310720, 1024, 1, 0)
+    assert 0 < big < 20 * 2 ** 30
+    assert big - lib.ls_lsa_flat_workspace_size(32768, 1310720, 1024, 1, 256) >= (768 - 256) * 1310720 * 4
 
 
 def test_argument_checks_without_gpu(lib):
@@ -111,14 +127,14 @@ def test_argument_checks_without_gpu(lib):
     # fp8 prefill: k out of range; LSA: d != 64, top_p too large, short workspace
     assert lib.ls_prefill_select_stream_fp8(dummy, dummy, dummy, dummy, 4, 32, 128, dummy, dummy, 100, 4, 64,
                                             dummy, dummy, 5000, 0, dummy, None, dummy, 1 << 30, None, None) == 1
-    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 128, 64, 512, 64, 4, 16, 64, 1, dummy,
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 128, 64, 512, 64, 4, 16, 64, 1, 0, dummy,
                                   dummy, None, dummy, 1 << 30, None) == 3
-    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 5000, 64, 1, dummy,
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 5000, 64, 1, 0, dummy,
                                   dummy, None, dummy, 1 << 30, None) == 1
-    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 16, 64, 1, dummy, dummy,
-                                  None, dummy, 8, None) == 2
-    assert lib.ls_lsa_flat_select(None, None, None, None, None, 0, 64, 64, 512, 64, 4, 16, 64, 1, None, None, None,
-                                  None, 0, None) == 0
+    assert lib.ls_lsa_flat_select(dummy, dummy, dummy, dummy, dummy, 4, 64, 64, 512, 64, 4, 16, 64, 1, 0, dummy,
+                                  dummy, None, dummy, 8, None) == 2
+    assert lib.ls_lsa_flat_select(None, None, None, None, None, 0, 64, 64, 512, 64, 4, 16, 64, 1, 0, None, None,
+                                  None, None, 0, None) == 0
     # LSA tree: d != 64, beam too large, more node children than buckets, short workspace, empty batch
     tree = lib.ls_lsa_tree_select
     assert tree(dummy, dummy, dummy, dummy, dummy, dummy, 4, 128, 4096, 1024, 512, 64, 4096, 4, 96, 4, 64, 512, dummy,

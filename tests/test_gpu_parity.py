@@ -14,7 +14,8 @@ import torch
 from oracle.formats import bf16_to_f64, dequant, pq_decode
 from oracle.indexer import eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_select, recall_at_k, select_topk,
+    bucket_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_levels_select, lsa_tree_select,
+    recall_at_k, select_topk,
     topk_rows, two_stage_pq_select, two_stage_select,
 )
 from parity_util import (
@@ -631,23 +632,25 @@ def test_bucket_full_size_sampled(L):
 # --------------------------------------------------------------------------- #
 # native LSA flat search
 # --------------------------------------------------------------------------- #
-def _lsa_run(L, d, wl, threshold):
+def _lsa_run(L, d, wl, threshold, fallback_rows=0):
     ex = wl.extra
     keys, n, picked = L.ls_lsa_flat_select(dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]),
                                            dev(d["bucket_off"]), dev(d["bucket_mem"]), block_keys=ex["block_keys"],
                                            buckets_per_block=ex["bpb"], n_sink=ex["n_sink"], top_p=wl.top_p,
-                                           budget=wl.budget, threshold=threshold, want_picked=True)
+                                           budget=wl.budget, threshold=threshold, fallback_rows=fallback_rows,
+                                           want_picked=True)
     return keys.cpu().numpy(), n.cpu().numpy(), picked.cpu().numpy()
 
 
-def _check_lsa(L, name, rows, d=None, wl=None):
+def _check_lsa(L, name, rows, d=None, wl=None, fallback_rows=0, compare_full=True):
     wl = wl or get_workload(name)
     d = d or data(name)
     ex = wl.extra
-    keys, n, picked = _lsa_run(L, d, wl, threshold=True)
-    # the full-matrix form picks the same buckets, bit for bit
-    keys0, n0, picked0 = _lsa_run(L, d, wl, threshold=False)
-    assert np.array_equal(picked0, picked) and np.array_equal(keys0, keys) and np.array_equal(n0, n), name
+    keys, n, picked = _lsa_run(L, d, wl, threshold=True, fallback_rows=fallback_rows)
+    if compare_full:
+        # the full-matrix form picks the same buckets, bit for bit
+        keys0, n0, picked0 = _lsa_run(L, d, wl, threshold=False)
+        assert np.array_equal(picked0, picked) and np.array_equal(keys0, keys) and np.array_equal(n0, n), name
     _, det = lsa_flat_select(d["q_idx"], d["q_pos"], d["centroids"], d["bucket_off"], d["bucket_mem"],
                              ex["block_keys"], ex["bpb"], ex["n_sink"], wl.top_p, wl.budget, rows=rows,
                              return_detail=True)
@@ -674,27 +677,58 @@ def test_lsa_flat_full_size_sampled(L):
     _check_lsa(L, "lsa_flat", [0, 1, 100, 254, 255])
 
 
-def test_lsa_threshold_fallbacks(L):
-    """Rows whose sampled threshold misses fall back to full scoring.  Every
-    query points along u; the sampled buckets (every top_p/8-th) point along
-    u and the rest along -u, so the sample's 32nd best clears only sampled
-    buckets: rows with fewer than top_p of them come up short; then all
-    centroids along u, so every visible bucket ties at the threshold and rows
-    with more than 8*top_p visible buckets overflow their lists."""
-    wl = get_workload("lsa_flat_s")
-    base = data("lsa_flat_s")
+def _missing_threshold_cases(base, top_p):
+    """Every query points along u.  First: the sampled buckets (every
+    top_p/8-th) point along u and the rest along -u, so the sample's 32nd
+    best clears only sampled buckets: rows with fewer than top_p of them come
+    up short.  Then all centroids along u, so every visible bucket ties at the
+    threshold and rows with more than 8*top_p visible buckets overflow their
+    lists."""
+    from workloads.synth import to_bf16_bits
     rng = np.random.default_rng(3)
     u = rng.standard_normal(64)
     u /= np.linalg.norm(u)
     P = base["centroids"].shape[0]
-    stride = max(1, wl.top_p // 8)
+    stride = max(1, top_p // 8)
     sign = np.where(np.arange(P) % stride == 0, 1.0, -1.0)
-    from workloads.synth import to_bf16_bits
     for cent in (sign[:, None] * u[None, :], np.broadcast_to(u, (P, 64)).copy()):
         d = dict(base)
         d["q_idx"] = to_bf16_bits(np.broadcast_to(u, base["q_idx"].shape).copy())
         d["centroids"] = to_bf16_bits(cent)
-        _check_lsa(L, "lsa_flat_s", list(range(37)), d=d, wl=wl)
+        yield d
+
+
+@pytest.mark.parametrize("fallback_rows", [0, 5])
+def test_lsa_threshold_fallbacks(L, fallback_rows):
+    """Rows whose sampled threshold misses fall back to full scoring, in one
+    chunk of rows or in eight."""
+    wl = get_workload("lsa_flat_s")
+    for d in _missing_threshold_cases(data("lsa_flat_s"), wl.top_p):
+        _check_lsa(L, "lsa_flat_s", list(range(37)), d=d, wl=wl, fallback_rows=fallback_rows)
+
+
+def test_lsa_prefill_chunk_small(L):
+    """A prefill chunk of 3000 queries: thirteen 256-query groups, each scored
+    by a few of the scan's CTAs, so every row's list is shared among a few
+    segments (proportional to the tiles each CTA scores)."""
+    _check_lsa(L, "lsa_prefill_s", [0, 1, 255, 256, 1000, 2047, 2048, 2999])
+
+
+@pytest.mark.parametrize("fallback_rows", [0, 256, 700])
+def test_lsa_prefill_chunk_fallbacks(L, fallback_rows):
+    """Every row of the 3000-query chunk misses its threshold and is scored in
+    full, 3000, 256 (12 chunks, the last ragged) or 700 rows at a time."""
+    wl = get_workload("lsa_prefill_s")
+    rows = [0, 1, 255, 256, 1000, 2999]
+    for d in _missing_threshold_cases(data("lsa_prefill_s"), wl.top_p):
+        _check_lsa(L, "lsa_prefill_s", rows, d=d, wl=wl, fallback_rows=fallback_rows)
+
+
+@pytest.mark.slow
+def test_lsa_prefill_10m_sampled(L):
+    """The 32768-query chunk at 10M tokens: the threshold form only (the full
+    matrix would take 172 GB), sampled rows against the oracle."""
+    _check_lsa(L, "lsa_prefill_10m", [0, 1, 255, 256, 16383, 32767], compare_full=False)
 
 
 def _check_lsa_tree(L, name, rows, beam=None):
@@ -741,6 +775,82 @@ def test_lsa_tree_full_beam_matches_flat(L):
 @pytest.mark.slow
 def test_lsa_tree_full_size_sampled(L):
     _check_lsa_tree(L, "lsa_tree", [0, 1, 100, 254, 255])
+
+
+def _check_lsa_tree_levels(L, name, rows, beam=None, start_nodes=None, d=None):
+    """Level by level against the oracle's scores of the candidates the GPU's
+    own beam of the level above gives (band rule on each beam and on the
+    picks), then the read lists exactly."""
+    wl = get_workload(name)
+    d = d or data(name)
+    ex = wl.extra
+    beam = beam or ex["beam"]
+    start_nodes = start_nodes or ex["start_nodes"]
+    fan, nblk = ex["fanout"], ex["node_block"]
+    levels = d["node_levels"]
+    keys, n, picked, bms = L.ls_lsa_tree_levels_select(
+        dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]), [dev_bf16(x) for x in levels],
+        dev(d["bucket_off"]), dev(d["bucket_mem"]), block_keys=ex["block_keys"], buckets_per_block=ex["bpb"],
+        node_block=nblk, fanout=fan, beam=beam, start_nodes=start_nodes, n_sink=ex["n_sink"], top_p=wl.top_p,
+        budget=wl.budget, want_picked=True)
+    keys, n, picked, bms = keys.cpu().numpy(), n.cpu().numpy(), picked.cpu().numpy(), bms.cpu().numpy()
+    _, det = lsa_tree_levels_select(d["q_idx"], d["q_pos"], d["centroids"], levels, d["bucket_off"],
+                                    d["bucket_mem"], ex["block_keys"], ex["bpb"], nblk, fan, beam, start_nodes,
+                                    ex["n_sink"], wl.top_p, wl.budget, rows=rows, return_detail=True)
+    bits = [d["centroids"]] + list(levels)
+    S = det[0]["start"]
+    assert np.all(bms[S:] == -2), "levels above the start level are written"
+    for i, t in enumerate(rows):
+        v = det[i]["visible"]
+        q = bf16_to_f64(d["q_idx"][t])
+        cand = np.arange(v[S], dtype=np.int64)
+        for lv in range(S, -1, -1):
+            if lv < S:
+                kept = bms[lv][t][bms[lv][t] >= 0]
+                cand = np.asarray([int(x) * fan + c for x in kept for c in range(fan)]
+                                  + list(range(fan * v[lv + 1], v[lv])), dtype=np.int64)
+            ref = bf16_to_f64(bits[lv][cand]) @ q if cand.size else np.zeros(0)
+            got = bms[lv - 1][t] if lv > 0 else picked[t]
+            check_set(got, cand, ref, beam if lv > 0 else wl.top_p, RTOL_BF16, f"{name} level {lv} row {t}")
+        want = lsa_read_list(picked[t], d["q_pos"][t], d["bucket_off"], d["bucket_mem"], ex["block_keys"],
+                             ex["n_sink"], wl.budget)
+        assert n[t] == want.size and np.array_equal(keys[t, :n[t]], want), f"{name} read list row {t}"
+        assert np.all(keys[t, n[t]:] == -1)
+    return keys, n, picked
+
+
+@pytest.mark.parametrize("start_nodes", [100, 500, 5000])
+def test_lsa_tree_levels_small(L, start_nodes):
+    _check_lsa_tree_levels(L, "lsa_tree_levels_s", list(range(37)), start_nodes=start_nodes)
+
+
+def test_lsa_tree_levels_full_beam_matches_flat(L):
+    """A beam holding every visible entry of each level reads what the flat
+    search reads (band rule on the picks; read lists exactly)."""
+    wl = get_workload("lsa_tree_levels_s")
+    keys, n, picked = _check_lsa_tree_levels(L, "lsa_tree_levels_s", list(range(37)), beam=1248, start_nodes=100)
+    _check_lsa(L, "lsa_tree_levels_s", list(range(37)), wl=wl)
+
+
+def test_lsa_tree_levels_one_level_matches_one_level_search(L):
+    """One node level: the same picks and read lists as the one-level search, bit for bit."""
+    wl = get_workload("lsa_flat_s")
+    d = data("lsa_flat_s")
+    ex = wl.extra
+    args = (dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]))
+    kw = dict(block_keys=ex["block_keys"], buckets_per_block=ex["bpb"], node_block=ex["node_block"],
+              fanout=ex["fanout"], beam=ex["beam"], n_sink=ex["n_sink"], top_p=wl.top_p, budget=wl.budget,
+              want_picked=True)
+    k1, n1, p1, _ = L.ls_lsa_tree_select(*args, dev_bf16(d["node_centroids"]), dev(d["bucket_off"]),
+                                         dev(d["bucket_mem"]), **kw)
+    k2, n2, p2, _ = L.ls_lsa_tree_levels_select(*args, [dev_bf16(d["node_centroids"])], dev(d["bucket_off"]),
+                                                dev(d["bucket_mem"]), start_nodes=32768, **kw)
+    assert torch.equal(p1, p2) and torch.equal(k1, k2) and torch.equal(n1, n2)
+
+
+@pytest.mark.slow
+def test_lsa_tree_levels_10m_sampled(L):
+    _check_lsa_tree_levels(L, "lsa_tree_10m", [0, 1, 100, 254, 255])
 
 
 def test_bucket_bad_member_flagged(L):

@@ -143,6 +143,12 @@ WORKLOADS: Dict[str, Workload] = {
         "lsa_prefill_10m", "lsa", T=32768, N=10485760, top_p=1024, budget=4096,
         extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "chunk": 1},
     ),
+    # a 4096-query chunk of the same sequence (the scan's profile case: the
+    # 168 MB of centroids still exceed L2, the workspace stays near 1.5 GB)
+    "lsa_prefill_10m_q4096": Workload(
+        "lsa_prefill_10m_q4096", "lsa", T=4096, N=10485760, top_p=1024, budget=4096,
+        extra={"block_keys": 512, "bpb": 64, "n_sink": 4, "chunk": 1},
+    ),
     # sparse main attention after the decode selection: 64 decode queries of
     # 128 heads, each over its 512 selected rows of a latent cache of
     # 262144 rows x 576 bf16 (302 MB, larger than L2); H, d = heads, latent
