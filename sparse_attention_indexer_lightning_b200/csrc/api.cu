@@ -1018,12 +1018,11 @@ struct LsaWorkspace {
   int32_t* clab;
   int32_t* nv;      // [T]
   uint8_t* ctr;     // row_over [T], any_over
-  int32_t* fb_list; // [T] missed rows, then the count, then the chunk flags
+  int32_t* fb_list; // [T] missed rows (-1 after the count), then the count, then the chunk flags
   int32_t* fb_count;
   int32_t* fb_run;
-  uint16_t* fb_q;   // [rows][64] their index queries
-  int32_t* fb_vis;  // [rows]
-  int32_t* fb_pick; // [rows][top_p]
+  uint16_t* fb_q;   // [T][64] their index queries, in list order
+  int32_t* fb_vis;  // [T] their visible counts
   size_t ctr_bytes;
   size_t scnt_bytes;
   size_t used;
@@ -1055,9 +1054,8 @@ LsaWorkspace carve_lsa(void* ws, int T, int P, int top_p, int threshold, int fal
     w.fb_list = cv.take<int32_t>(T);
     w.fb_count = cv.take<int32_t>(1);
     w.fb_run = cv.take<int32_t>(fb.chunks);
-    w.fb_q = cv.take<uint16_t>(static_cast<size_t>(fb.rows) * kLsaDim);
-    w.fb_vis = cv.take<int32_t>(fb.rows);
-    w.fb_pick = cv.take<int32_t>(static_cast<size_t>(fb.rows) * top_p);
+    w.fb_q = cv.take<uint16_t>(static_cast<size_t>(T) * kLsaDim);
+    w.fb_vis = cv.take<int32_t>(T);
   }
   w.used = cv.used;
   return w;
@@ -1196,27 +1194,29 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
       cp.ld_out = top_p;
       s = topk_launch(cp, st);
       if (s != LS_OK) return s;
-      // 4. rows whose list ran over or came up short, listed and scored in
-      //    full fb.rows at a time (the launches of a chunk that holds none of
-      //    them return at once)
+      // 4. rows whose list ran over or came up short: listed, their queries
+      //    gathered, then scored in full fb.rows at a time, each chunk's
+      //    top-p written to its listed rows (the two launches of a chunk that
+      //    holds none of them return at once)
       const LsaFallback fb(T, P, fallback_rows);
       {
         ProfScope prof("lsa_flag_list_kernel", st);
         LS_CUDA(launch_lsa_flag_list(row_over, T, fb.rows, fb.chunks, w.fb_list, w.fb_count, w.fb_run, st));
       }
-      CUtensorMap fqmap;
-      s = make_vec64_map(&fqmap, w.fb_q, static_cast<uint64_t>(fb.rows), DotCfg::QB);
-      if (s != LS_OK) return s;
+      {
+        ProfScope prof("lsa_gather_rows_kernel", st);
+        LS_CUDA(launch_lsa_gather_rows(w.fb_list, w.fb_count, T, q_idx, w.vis, any_over, w.fb_q, w.fb_vis, st));
+      }
       for (int c = 0; c < fb.chunks; ++c) {
         const int32_t* run = w.fb_run + c;
         const int c0 = c * fb.rows;
-        {
-          ProfScope prof("lsa_gather_rows_kernel", st);
-          LS_CUDA(launch_lsa_gather_rows(w.fb_list, w.fb_count, c0, fb.rows, q_idx, w.vis, run, w.fb_q, w.fb_vis,
-                                         st));
-        }
+        const int rows = std::min(fb.rows, T - c0);
+        CUtensorMap fqmap;
+        s = make_vec64_map(&fqmap, w.fb_q + static_cast<size_t>(c0) * kLsaDim, static_cast<uint64_t>(rows),
+                           DotCfg::QB);
+        if (s != LS_OK) return s;
         DotParams fd;
-        fd.T = fb.rows;
+        fd.T = rows;
         fd.P = P;
         fd.out = w.sc;
         fd.ld_out = P;
@@ -1228,17 +1228,16 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
         TopkParams fk;
         fk.scores = w.sc;
         fk.ld = P;
-        fk.n_valid = w.fb_vis;
-        fk.R = fb.rows;
+        fk.n_valid = w.fb_vis + c0;
+        fk.R = rows;
         fk.N = P;
         fk.k = top_p;
-        fk.idx_out = w.fb_pick;
+        fk.out_row = w.fb_list + c0;
+        fk.idx_out = picked;
         fk.ld_out = top_p;
         fk.run_if = run;
         s = topk_launch(fk, st, "topk_kernel:fallback");
         if (s != LS_OK) return s;
-        ProfScope prof("lsa_scatter_rows_kernel", st);
-        LS_CUDA(launch_lsa_scatter_rows(w.fb_list, w.fb_count, c0, fb.rows, w.fb_pick, top_p, run, picked, st));
       }
     }
   } else {

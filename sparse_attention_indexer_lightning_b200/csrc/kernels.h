@@ -148,16 +148,16 @@ int dot_tc_grid(int T, int P, int num_sms);
 cudaError_t launch_lsa_compact(const uint2* slist, const uint32_t* cnt, const DotParams& fp, int grid,
                                const int32_t* vis, int T, int top_p, int cap, float* cval, int32_t* clab, int32_t* nv,
                                int32_t* row_over, int* any_over, cudaStream_t st);
-// The threshold form's fallback: the missed rows listed (ascending), then
-// scored in full `rows` at a time: their queries gathered, the chunk's picks
-// written back (launches that return at once when run_if[0] == 0).
+// The threshold form's fallback: the missed rows listed (ascending; -1 past
+// the count) with run[c] = 1 for the chunks of `rows` list entries that hold
+// any, then their queries and visible counts gathered into qbuf / vbuf [T]
+// (zeros past the count), each chunk then scored in full and its picks
+// written to the listed rows (launches that return at once when run_if[0] == 0).
 cudaError_t launch_lsa_flag_list(const int32_t* row_over, int T, int rows, int n_chunks, int32_t* list,
                                  int32_t* count, int32_t* run, cudaStream_t st);
-cudaError_t launch_lsa_gather_rows(const int32_t* list, const int32_t* count, int c0, int rows, const uint16_t* q,
-                                   const int32_t* vis, const int32_t* run_if, uint16_t* qbuf, int32_t* vbuf,
+cudaError_t launch_lsa_gather_rows(const int32_t* list, const int32_t* count, int T, const uint16_t* q,
+                                   const int32_t* vis, const int* run_if, uint16_t* qbuf, int32_t* vbuf,
                                    cudaStream_t st);
-cudaError_t launch_lsa_scatter_rows(const int32_t* list, const int32_t* count, int c0, int rows, const int32_t* pbuf,
-                                    int top_p, const int32_t* run_if, int32_t* picked, cudaStream_t st);
 // The read list of each query: sinks below its window, the window, then the
 // picked buckets' members best first (sinks and window skipped) up to budget.
 cudaError_t launch_lsa_expand(const int32_t* picked, const int64_t* q_pos, int T, int top_p, const int32_t* off,
@@ -210,6 +210,7 @@ struct TopkParams {
   const uint32_t* hist = nullptr;    // [R][2048] counts of the top 11 order-code bits of the
                                      // present entries (from the scoring epilogue) or nullptr
   const int32_t* row_flag = nullptr; // [R] or nullptr: rows whose flag is 0 are left untouched
+  const int32_t* out_row = nullptr;  // [R] or nullptr: row r's output goes to row out_row[r] (< 0: none)
   const int* run_if = nullptr;       // the launch does nothing unless *run_if != 0 (nullptr: always)
   int R = 0, N = 0, k = 0;
   int32_t* idx_out = nullptr;        // [R][k] labels, -1 padding

@@ -528,9 +528,9 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// The rows the sampled threshold missed, in ascending order: list[0, count)
-// (one CTA); run[c] = 1 when chunk c (rows [c * rows, (c + 1) * rows) of the
-// list) holds any, for c < n_chunks.
+// The rows the sampled threshold missed, in ascending order: list[0, count),
+// -1 after (one CTA); run[c] = 1 when chunk c (list entries [c * rows,
+// (c + 1) * rows)) holds any, for c < n_chunks.
 __global__ void __launch_bounds__(1024)
     lsa_flag_list_kernel(const int32_t* __restrict__ row_over, int T, int rows, int n_chunks,
                          int32_t* __restrict__ list, int32_t* __restrict__ count, int32_t* __restrict__ run) {
@@ -557,38 +557,28 @@ __global__ void __launch_bounds__(1024)
     __syncthreads();
   }
   const int n = base_s;
+  for (int i = n + tid; i < T; i += 1024) list[i] = -1;
   if (tid == 0) *count = n;
   for (int c = tid; c < n_chunks; c += 1024) run[c] = (static_cast<long long>(c) * rows < n) ? 1 : 0;
 }
 
-// Chunk c0 / rows of the missed rows: their index queries and visible counts
-// gathered into qbuf [rows][64] and vbuf [rows] (zeros past the list's end).
-__global__ void lsa_gather_rows_kernel(const int32_t* __restrict__ list, const int32_t* __restrict__ count, int c0,
-                                       int rows, const uint16_t* __restrict__ q, const int32_t* __restrict__ vis,
-                                       const int32_t* __restrict__ run_if, uint16_t* __restrict__ qbuf,
+// The missed rows' index queries and visible counts, in list order, into
+// qbuf [T][64] and vbuf [T] (zeros past the count).
+__global__ void lsa_gather_rows_kernel(const int32_t* __restrict__ list, const int32_t* __restrict__ count, int T,
+                                       const uint16_t* __restrict__ q, const int32_t* __restrict__ vis,
+                                       const int* __restrict__ run_if, uint16_t* __restrict__ qbuf,
                                        int32_t* __restrict__ vbuf) {
   if (*run_if == 0) return;
+  const int n = *count;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;   // one 16-byte piece: row i / 8, piece i % 8
-  if (i >= rows * 8) return;
+  if (i >= T * 8) return;
   const int r = i >> 3, piece = i & 7;
-  const bool live = c0 + r < *count;
-  const int t = live ? list[c0 + r] : 0;
+  const bool live = r < n;
+  const int t = live ? list[r] : 0;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (live) v = reinterpret_cast<const uint4*>(q + static_cast<int64_t>(t) * kLsaDim)[piece];
   reinterpret_cast<uint4*>(qbuf + static_cast<int64_t>(r) * kLsaDim)[piece] = v;
   if (piece == 0) vbuf[r] = live ? vis[t] : 0;
-}
-
-// The picks of that chunk written back to the rows they belong to.
-__global__ void lsa_scatter_rows_kernel(const int32_t* __restrict__ list, const int32_t* __restrict__ count, int c0,
-                                        int rows, const int32_t* __restrict__ pbuf, int top_p,
-                                        const int32_t* __restrict__ run_if, int32_t* __restrict__ picked) {
-  if (*run_if == 0) return;
-  const int r = blockIdx.x;
-  if (r >= rows || c0 + r >= *count) return;
-  const int t = list[c0 + r];
-  for (int j = threadIdx.x; j < top_p; j += blockDim.x)
-    picked[static_cast<int64_t>(t) * top_p + j] = pbuf[static_cast<int64_t>(r) * top_p + j];
 }
 
 // Visible buckets of each query (causal block visibility: the buckets of the
@@ -635,8 +625,11 @@ __global__ void __launch_bounds__(kExpandThreads)
                       const int32_t* __restrict__ off, const int32_t* __restrict__ mem, int P, int block_keys,
                       int n_sink, int budget, int32_t* __restrict__ keys_out, int row_len,
                       int32_t* __restrict__ n_out) {
+  constexpr int kItems = kExpandThreads * kExpandItems;       // buckets per round
   __shared__ int warp_sum[kExpandThreads / 32];
   __shared__ int round_total;
+  __shared__ int s_start[kItems + 1];                          // a round's output start of each bucket
+  __shared__ int s_src[kItems];                                // and where its members begin in mem
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31, wid = tid >> 5;
@@ -688,14 +681,31 @@ __global__ void __launch_bounds__(kExpandThreads)
       before += (w < wid) ? v : 0;
       total += v;
     }
-    int start = base + before + incl - mine;
+    int start = before + incl - mine;
 #pragma unroll
     for (int i = 0; i < kExpandItems; ++i) {
-      for (int m = 0; m < sz[i] && start + m < budget; ++m) lr[start + m] = mem[o[i] + lo[i] + m];
+      s_start[tid * kExpandItems + i] = start;
+      s_src[tid * kExpandItems + i] = o[i] + lo[i];
       start += sz[i];
     }
-    if (tid == 0) round_total = total;
-    __syncthreads();                                   // warp_sum is reused by the next round
+    if (tid == 0) {
+      round_total = total;
+      s_start[kItems] = total;
+    }
+    __syncthreads();
+    // the round's members, block-wide: output q comes from the last bucket
+    // whose start is <= q (empty buckets share their successor's start)
+    const int take = min(total, budget - base);
+    for (int q = tid; q < take; q += kExpandThreads) {
+      int a = 0, b = kItems;                          // s_start[a] <= q < s_start[b]
+      while (b - a > 1) {
+        const int mid = (a + b) >> 1;
+        if (s_start[mid] <= q) a = mid;
+        else b = mid;
+      }
+      lr[base + q] = mem[s_src[a] + (q - s_start[a])];
+    }
+    __syncthreads();                                   // the tables are reused by the next round
     base += round_total;
   }
   const int n_lr = base < budget ? base : budget;
@@ -730,18 +740,11 @@ cudaError_t launch_lsa_flag_list(const int32_t* row_over, int T, int rows, int n
   return cudaGetLastError();
 }
 
-cudaError_t launch_lsa_gather_rows(const int32_t* list, const int32_t* count, int c0, int rows, const uint16_t* q,
-                                   const int32_t* vis, const int32_t* run_if, uint16_t* qbuf, int32_t* vbuf,
+cudaError_t launch_lsa_gather_rows(const int32_t* list, const int32_t* count, int T, const uint16_t* q,
+                                   const int32_t* vis, const int* run_if, uint16_t* qbuf, int32_t* vbuf,
                                    cudaStream_t st) {
-  if (rows == 0) return cudaSuccess;
-  lsa_gather_rows_kernel<<<(rows * 8 + 255) / 256, 256, 0, st>>>(list, count, c0, rows, q, vis, run_if, qbuf, vbuf);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_lsa_scatter_rows(const int32_t* list, const int32_t* count, int c0, int rows, const int32_t* pbuf,
-                                    int top_p, const int32_t* run_if, int32_t* picked, cudaStream_t st) {
-  if (rows == 0) return cudaSuccess;
-  lsa_scatter_rows_kernel<<<rows, 256, 0, st>>>(list, count, c0, rows, pbuf, top_p, run_if, picked);
+  if (T == 0) return cudaSuccess;
+  lsa_gather_rows_kernel<<<(T * 8 + 255) / 256, 256, 0, st>>>(list, count, T, q, vis, run_if, qbuf, vbuf);
   return cudaGetLastError();
 }
 

@@ -507,6 +507,8 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
   // rows blockIdx.x, blockIdx.x + gridDim.x, ... (LOOP), else row blockIdx.x
   for (int r = blockIdx.x; r < p.R; r += (LOOP ? gridDim.x : p.R)) {
   if (p.row_flag != nullptr && p.row_flag[r] == 0) continue;  // row left untouched
+  const int orow = p.out_row ? p.out_row[r] : r;               // where the row's output goes
+  if (orow < 0) continue;
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   RowRef rr;
@@ -629,8 +631,8 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
     }
     __syncthreads();
   }
-  int32_t* io = p.idx_out + static_cast<int64_t>(r) * p.ld_out;
-  float* vo = p.val_out ? p.val_out + static_cast<int64_t>(r) * p.ld_out : nullptr;
+  int32_t* io = p.idx_out + static_cast<int64_t>(orow) * p.ld_out;
+  float* vo = p.val_out ? p.val_out + static_cast<int64_t>(orow) * p.ld_out : nullptr;
   const int lab_add = rr.lab ? 0 : p.label_base;
   const int nc_all = static_cast<int>(min(sh.ccnt, static_cast<uint32_t>(CAP)));
   // ---- 4'. bucket select: selection and canonical order in one pass -------

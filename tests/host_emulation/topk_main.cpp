@@ -5,7 +5,8 @@
 // end.  Test infrastructure only.
 //   DIR FORM R N k ld has_labels has_nvalid nv_offset label_base ld_out rows...
 //   (a negative first "row" -G instead runs a grid of G blocks over all rows
-//   with the row flags of flags.bin [R] i32: the flagged-launch form)
+//   with the row flags of flags.bin [R] i32: the flagged-launch form; with
+//   outrow.bin [R] i32 present, row r's output goes to row out_row[r])
 //   FORM 0: <256, 512, 2048>   1: <512, 1024, 8192>   2: <1024, 4096, 8192>
 //   (scores.bin [R][ld] f32, labels.bin [R][ld] i32, nvalid.bin [R] i32)
 //   -> idx.bin, val.bin [R][ld_out]
@@ -112,6 +113,17 @@ int main(int argc, char** argv) {
   p.idx_out = idx.data();
   p.val_out = val.data();
   p.ld_out = ld_out;
+  // an out_row map [R] i32 when DIR/outrow.bin exists: row r's output goes to row out_row[r]
+  std::vector<int32_t> outrow;
+  {
+    char path[1024];
+    std::snprintf(path, sizeof path, "%s/outrow.bin", dir);
+    if (FILE* f = std::fopen(path, "rb")) {
+      std::fclose(f);
+      outrow = load<int32_t>(dir, "outrow.bin", static_cast<size_t>(R));
+      p.out_row = outrow.data();
+    }
+  }
   std::vector<int32_t> flags;
   if (grid > 0) {
     flags = load<int32_t>(dir, "flags.bin", static_cast<size_t>(R));

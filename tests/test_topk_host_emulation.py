@@ -78,9 +78,13 @@ def topk_host(tmp_path_factory):
     assert r.returncode == 0, r.stderr[-3000:]
     env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
 
-    def run(form, scores, labels, n_valid, k, flags=None, grid=0):
+    def run(form, scores, labels, n_valid, k, flags=None, grid=0, out_row=None):
         R, ld = scores.shape
         scores.astype(np.float32).tofile(d / "scores.bin")
+        if out_row is not None:
+            out_row.astype(np.int32).tofile(d / "outrow.bin")
+        elif (d / "outrow.bin").exists():
+            (d / "outrow.bin").unlink()
         if labels is not None:
             labels.astype(np.int32).tofile(d / "labels.bin")
         if n_valid is not None:
@@ -200,3 +204,22 @@ def test_host_topk_flagged_rows_grid_stride(topk_host):
             assert np.array_equal(gv[r].view(np.uint32), wv[r].astype(np.float32).view(np.uint32))
         else:
             assert np.all(gi[r] == 777)          # untouched
+
+
+def test_host_topk_out_row_map(topk_host):
+    """With an output row map, row r's top-k lands in row out_row[r]; rows
+    mapped to -1 write nothing, rows no input maps to are left as they were."""
+    k = 64
+    rng = np.random.default_rng(12)
+    R, ld = 9, 500
+    sc = np.stack([_row(rng, ld, ("normal", "ties", "coarse")[r % 3]) for r in range(R)])
+    nv = rng.integers(0, ld + 1, R).astype(np.int32)
+    out_row = np.array([3, -1, 0, 8, 1, -1, 2, 7, 4], dtype=np.int32)
+    gi, gv = topk_host(0, sc, None, nv, k, out_row=out_row)
+    wi, wv = _expect(sc, None, nv, k)
+    for r in range(R):
+        if out_row[r] >= 0:
+            assert np.array_equal(gi[out_row[r]], wi[r])
+            assert np.array_equal(gv[out_row[r]].view(np.uint32), wv[r].astype(np.float32).view(np.uint32))
+    for o in set(range(R)) - set(out_row.tolist()):
+        assert np.all(gi[o] == 777)
