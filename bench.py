@@ -186,6 +186,7 @@ KERNEL_SOURCES = {
     "score_tc_kernel": ["common.cuh", "kernels.h", "score_tc.cuh"],
     "score_q8_kernel": ["common.cuh", "kernels.h", "score_q8.cuh"],
     "dot_tc_kernel": ["common.cuh", "kernels.h", "score_dot.cuh"],
+    "sparse_attn_tc_kernel": ["common.cuh", "kernels.h", "sparse_attn_tc.cuh"],
 }
 
 
@@ -812,7 +813,7 @@ def bench_attention(L, args, peaks, peak_kind):
     res = {"ms_per_step": ms, "positions_per_s": T * wl.k / (ms * 1e-3), "selections_per_s": T / (ms * 1e-3),
            "kernels": kern,
            "roofline": roofline("tensor", flops / (kms * 1e-3) / 1e12, peak_t, "TFLOP/s",
-                                peak_kind=peak_kind),
+                                traffic=ncu_traffic("sparse_attn_tc_kernel", wl.name), peak_kind=peak_kind),
            "gather_hbm_frac": round(gathered / (kms * 1e-3) / 1e9 / peak_b, 4),
            "cuda_core_kernel": {"ms_per_step": ms_cc, "kernels": kern_cc,
                                 "alu_frac": round(flops / (kern_cc["sparse_attn_kernel"]["ms_per_step"] * 1e-3)
