@@ -330,8 +330,9 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
         // mask.  A score is listed when it is visible and not below its
         // column's threshold in the top-k's key order: the sign bit of
         // fl(score + (-threshold)) (one rounding, so it is set exactly when
-        // score < threshold, -0 below +0, a NaN score listed like the top
-        // key it is; a -inf threshold lists every visible bucket).  The
+        // score < threshold, -0 below +0; a NaN score is listed too, which
+        // changes nothing since the top-k ranks it last; a -inf threshold
+        // lists every visible bucket).  The
         // sums go two at a time through the packed fp32 adder, their sign
         // bits are shifted into four 8-bit words (column 4 * i + r at bit
         // 8 * r + 7 - i of the combined word); a tile below every column's
