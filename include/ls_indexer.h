@@ -290,10 +290,11 @@ ls_status ls_prefill_select_stream_fp8(const uint8_t* q8, const float* q_scale, 
  * threshold = 0: every (query, bucket) score is written to a T x P matrix in
  * the workspace and the top_p of each row's visible prefix selected.
  * threshold = 1: the LSA article's sampled threshold (section "What the
- * kernels do about the top-p"): each query scores every (top_p / 8)-th
- * bucket, its 32nd best sample becomes its threshold (about 4 * top_p
- * buckets clear it), the scan appends only the visible buckets that reach
- * the threshold to a list of up to 8 * top_p, and the top_p of the list is
+ * kernels do about the top-p"): each query scores every (top_p / 16)-th
+ * bucket, its 32nd best sample becomes its threshold (about 2 * top_p
+ * buckets clear it; the article measures lists of about 1.7 * top_p), the
+ * scan appends only the visible buckets that reach the threshold to a list
+ * of up to 4 * top_p, and the top_p of the list is
  * kept; a query whose list overflows or holds fewer than min(top_p, visible)
  * buckets is scored in full instead.  Both forms pick the same buckets.
  * The threshold form never holds the T x P matrix: the missed queries are
@@ -305,7 +306,7 @@ ls_status ls_prefill_select_stream_fp8(const uint8_t* q8, const float* q_scale, 
  * fallback_rows) chunks.
  * Workspace: ls_lsa_flat_workspace_size(T, P, top_p, threshold,
  * fallback_rows) bytes: threshold = 0 holds the T x P matrix; threshold = 1
- * holds the samples (T x P / (top_p / 8)), the lists (about T x 16 top_p
+ * holds the samples (T x P / (top_p / 16)), the lists (about T x 8 top_p
  * entries of 8 bytes) and fallback_rows x P scores.
  */
 size_t ls_lsa_flat_workspace_size(int T, int P, int top_p, int threshold, int fallback_rows);

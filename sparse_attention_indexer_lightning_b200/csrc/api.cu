@@ -960,18 +960,20 @@ ls_status ls_bucket_select(const uint16_t* q, const float* w, const uint16_t* ce
 namespace {
 
 // Sampled-threshold parameters of the LSA search: every stride-th bucket is
-// sampled and the 32nd best sample sets the threshold, so about 4 * top_p
-// buckets of a row clear it; a row lists up to 8 * top_p.
+// sampled (stride = top_p / 16) and the 32nd best sample sets the threshold,
+// so about 2 * top_p buckets of a row clear it (the count's relative spread is
+// about 1/sqrt(32): a row comes up short with a probability of a few in a
+// thousand); a row lists up to 4 * top_p.
 struct LsaThreshold {
   int stride, rank, cap;
   explicit LsaThreshold(int top_p)
-      : stride(top_p / 8 > 1 ? top_p / 8 : 1), rank(32), cap(8 * top_p) {}
+      : stride(top_p / 16 > 1 ? top_p / 16 : 1), rank(32), cap(4 * top_p) {}
 };
 
 // List segments of the filtered scan: each row's list holds 2 * cap entries
 // shared out among the scan's CTAs in proportion to the centroid tiles of
-// the row each one scores (about 2x the expected count of its share of the
-// 4 * top_p listed buckets), plus 64 slack entries per CTA.
+// the row each one scores (about 4x the expected count of its share of the
+// 2 * top_p listed buckets), plus 64 slack entries per CTA.
 struct LsaSegments {
   int grid, nseg, cap2, slack;
   long long per_row;
@@ -1221,6 +1223,8 @@ ls_status ls_lsa_flat_select(const uint16_t* q_idx, const int64_t* q_pos, const 
         fd.out = w.sc;
         fd.ld_out = P;
         fd.run_if = run;
+        fd.live_rows = w.fb_count;            // only the chunk's listed rows are scored
+        fd.live_base = c0;
         {
           ProfScope prof("dot_tc_kernel:fallback", st);
           LS_CUDA(launch_dot_tc(&cmap, &fqmap, fd, num_sms_current(), st));

@@ -98,6 +98,9 @@ struct DotParams {
   int32_t* row_over = nullptr;        // [T]
   int* any_over = nullptr;
   const int* run_if = nullptr;        // the launch does nothing unless *run_if != 0 (nullptr: always)
+  // storing form: only rows t < *live_rows - live_base are scored (nullptr: all T)
+  const int* live_rows = nullptr;
+  int live_base = 0;
 };
 cudaError_t launch_dot_tc(const CUtensorMap* cmap, const CUtensorMap* qmap, const DotParams& p, int num_sms,
                           cudaStream_t st);

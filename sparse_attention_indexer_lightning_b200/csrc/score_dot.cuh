@@ -81,7 +81,13 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
                   const DotParams p) {
   using C = DotCfg;
   if (p.run_if != nullptr && *p.run_if == 0) return;  // a conditional launch with nothing to do
-  const int T = p.T, P = p.P;
+  int T = p.T;
+  if (!FILTER && p.live_rows != nullptr) {            // rows past the live count are not scored
+    const int live = *p.live_rows - p.live_base;
+    T = live < 0 ? 0 : (live < T ? live : T);
+    if (T == 0) return;
+  }
+  const int P = p.P;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* sA = smem;
@@ -284,7 +290,11 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int t = t0 + 32 * h + lane;
-          thr_s[32 * h + lane] = (t < T) ? -p.tau[static_cast<int64_t>(t) * p.ld_tau] : 0.f;   // negated
+          // negated; a zero threshold (either sign) becomes +0, so that a
+          // score of -0 or +0 sums to +0 and is listed, as the top-k's keys
+          // (which give -0 and +0 one code) require
+          const float th = (t < T) ? p.tau[static_cast<int64_t>(t) * p.ld_tau] : 0.f;
+          thr_s[32 * h + lane] = (th == 0.f) ? 0.f : -th;
           vis_s[32 * h + lane] = (t < T) ? p.vis[t] : 0;
           cnt_s[32 * h + lane] = 0;
         }
@@ -330,9 +340,9 @@ __global__ void __launch_bounds__(DotCfg::THREADS, 1)
         // mask.  A score is listed when it is visible and not below its
         // column's threshold in the top-k's key order: the sign bit of
         // fl(score + (-threshold)) (one rounding, so it is set exactly when
-        // score < threshold, -0 below +0; a NaN score is listed too, which
-        // changes nothing since the top-k ranks it last; a -inf threshold
-        // lists every visible bucket).  The
+        // score < threshold; -0 and +0 equal; a NaN score is listed too,
+        // which changes nothing since the top-k ranks it last; a -inf
+        // threshold lists every visible bucket).  The
         // sums go two at a time through the packed fp32 adder, their sign
         // bits are shifted into four 8-bit words (column 4 * i + r at bit
         // 8 * r + 7 - i of the combined word); a tile below every column's

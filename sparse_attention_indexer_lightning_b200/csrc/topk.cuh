@@ -542,6 +542,9 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
     } else {
       exact_hist = false;
       while ((rr.n / S) > kExactHistMax) S <<= 1;
+      // the list's margin (16 sampled entries, 16 * S row entries) must stay
+      // well inside the candidate capacity: long rows are sampled more densely
+      if (S > CAP / 64) S = CAP / 64 > 1 ? CAP / 64 : 1;
       const int groups = (rr.n + 7) >> 3;
       for (int g = tid * S; g < groups; g += NT * S) {
         const int i0 = g << 3;
@@ -580,6 +583,36 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
   const uint32_t hist_total = sh.total;
   if (hist_total == 0) blo = 0;                          // nothing present (or nothing sampled)
   if (!exact_hist && hist_total <= want_bins) blo = 0;   // the sample cannot place the bin: list everything
+  // Sampled rows whose boundary bin is coarse (the entries estimated at or
+  // above it would crowd the candidate list): refine the boundary by the next
+  // 11 code bits of the sampled entries inside that bin.  The list's lower
+  // bound becomes a 22-bit code prefix.
+  uint32_t lo_code = blo << (32 - kHistBits);
+  if (!exact_hist && blo >= 4 && hist_total > want_bins) {
+    const uint32_t above = max(want_bins, 1u) - sh.need;  // sampled entries in bins above blo
+    if ((static_cast<uint64_t>(above) + sh.eq) * static_cast<uint64_t>(S) > static_cast<uint64_t>(CAP / 2)) {
+      const uint32_t need_in = sh.need;                  // sampled entries wanted from bin blo
+      __syncthreads();                                   // every thread has read sh.need / sh.eq
+      for (int i = tid; i < kHistBins; i += NT) sh.fill[i] = 0;
+      __syncthreads();
+      const int groups = (rr.n + 7) >> 3;
+      for (int g = tid * S; g < groups; g += NT * S) {
+        const int i0 = g << 3;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (i0 + e < rr.n) {
+            const int32_t l = rr.lab ? __ldg(rr.lab + i0 + e) : i0 + e;
+            const uint32_t c = order_code(__ldg(rr.v + i0 + e));
+            if (l >= 0 && hist_bin(c) == blo) atomicAdd(&sh.fill[(c >> (32 - 2 * kHistBits)) & (kHistBins - 1)], 1u);
+          }
+        }
+      }
+      __syncthreads();
+      scan_bins_2048<NT>(sh, sh.fill, nullptr, max(need_in, 1u));
+      if (sh.total >= need_in)                           // the bin's sampled entries place the sub-bin
+        lo_code = (blo << (32 - kHistBits)) | (sh.digit << (32 - 2 * kHistBits));
+    }
+  }
   __syncthreads();
 
   int kk = 0;
@@ -588,7 +621,7 @@ __global__ void __launch_bounds__(NT, (NT == 256) ? 4 : 1024 / NT) topk_kernel(c
     {
       // ---- listing pass: every present entry in a bin >= blo -------------
       if (blo >= 4) {  // bins from 4 up start at finite values: compare the score itself
-        const float tlo = code_floor_value(blo << (32 - kHistBits));
+        const float tlo = code_floor_value(lo_code);
         list_row<NT>(rr, [&](float v, int32_t) { return v >= tlo; }, sh.cand_val, sh.cand_lab, &sh.ccnt, CAP);
       } else {
         list_row<NT>(rr, [&](float v, int32_t) { return hist_bin(order_code(v)) >= blo; }, sh.cand_val, sh.cand_lab,

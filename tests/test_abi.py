@@ -74,7 +74,7 @@ def test_version_and_workspace_queries(lib):
     # shard merge: the packed S * k_in candidates per row (values and positions) and the row counts
     assert lib.ls_merge_select_workspace_size(4, 4096, 512) >= 4096 * 4 * 512 * 8 + 4096 * 4
     assert lib.ls_merge_select_workspace_size(0, 4096, 512) == 0
-    # the threshold form adds the samples and the candidate lists (8 * top_p per row)
+    # the threshold form adds the samples and the candidate lists (4 * top_p per row, segments of twice that)
     assert (lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 1, 0)
             >= lib.ls_lsa_flat_workspace_size(256, 131072, 1024, 0, 0) + 256 * 8192 * 8)
     # ... but never the T x P matrix at prefill scale: 32768 queries x 1310720 buckets (172 GB) fit in

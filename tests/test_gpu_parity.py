@@ -679,17 +679,17 @@ def test_lsa_flat_full_size_sampled(L):
 
 def _missing_threshold_cases(base, top_p):
     """Every query points along u.  First: the sampled buckets (every
-    top_p/8-th) point along u and the rest along -u, so the sample's 32nd
+    top_p/16-th) point along u and the rest along -u, so the sample's 32nd
     best clears only sampled buckets: rows with fewer than top_p of them come
     up short.  Then all centroids along u, so every visible bucket ties at the
-    threshold and rows with more than 8*top_p visible buckets overflow their
+    threshold and rows with more than 4*top_p visible buckets overflow their
     lists."""
     from workloads.synth import to_bf16_bits
     rng = np.random.default_rng(3)
     u = rng.standard_normal(64)
     u /= np.linalg.norm(u)
     P = base["centroids"].shape[0]
-    stride = max(1, top_p // 8)
+    stride = max(1, top_p // 16)
     sign = np.where(np.arange(P) % stride == 0, 1.0, -1.0)
     for cent in (sign[:, None] * u[None, :], np.broadcast_to(u, (P, 64)).copy()):
         d = dict(base)

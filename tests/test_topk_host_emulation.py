@@ -110,6 +110,10 @@ def _row(rng, n, kind):
         return rng.integers(0, 8, n).astype(np.float32)
     if kind == "coarse":                       # quarter steps, like sums of fp8 products
         return (np.round(rng.standard_normal(n) * 4) / 4).astype(np.float32)
+    if kind == "narrow":                       # one narrow cluster: a handful of the 2048 coarse bins
+        return (0.3 + 1e-3 * rng.standard_normal(n)).astype(np.float32)
+    if kind == "tail":                         # a long Gaussian row: the k-th entry deep in the tail
+        return (0.125 * rng.standard_normal(n)).astype(np.float32)
     if kind == "special":
         v = rng.standard_normal(n).astype(np.float32)
         m = rng.integers(0, 6, n)
@@ -223,3 +227,16 @@ def test_host_topk_out_row_map(topk_host):
             assert np.array_equal(gv[out_row[r]].view(np.uint32), wv[r].astype(np.float32).view(np.uint32))
     for o in set(range(R)) - set(out_row.tolist()):
         assert np.all(gi[o] == 777)
+
+
+@pytest.mark.parametrize("form,ld,k", [(1, 200000, 1000), (2, 60000, 3000), (0, 50000, 512)])
+def test_host_topk_long_rows_refined_boundary(topk_host, form, ld, k):
+    """Long rows whose k-th entry sits in a coarse histogram bin (a narrow
+    cluster, a deep Gaussian tail): the sampled boundary is refined by the next
+    code bits so that the list fits, and the selection stays exact."""
+    rng = np.random.default_rng(ld + k)
+    R = 4
+    sc = np.stack([_row(rng, ld, ("narrow", "tail")[r % 2]) for r in range(R)])
+    nv = np.full(R, ld, dtype=np.int32)
+    nv[3] = ld - 12345
+    _check(topk_host(form, sc, None, nv, k), _expect(sc, None, nv, k))
