@@ -848,6 +848,15 @@ def test_lsa_tree_levels_one_level_matches_one_level_search(L):
     assert torch.equal(p1, p2) and torch.equal(k1, k2) and torch.equal(n1, n2)
 
 
+def test_lsa_tree_levels_empty_start_level(L):
+    """The start level holds no node (level sizes 1024 and 0, start_nodes 1):
+    an empty beam, every level-1 node uncovered, then the buckets."""
+    from workloads.synth import make_lsa
+    d = make_lsa(37, 40000, 512, 64, 0, 2053, True, node_block=4096, fanout=4, levels=2)
+    assert [x.shape[0] for x in d["node_levels"]] == [1024, 0]
+    _check_lsa_tree_levels(L, "lsa_flat_s", list(range(37)), beam=96, start_nodes=1, d=d)
+
+
 @pytest.mark.slow
 def test_lsa_tree_levels_10m_sampled(L):
     _check_lsa_tree_levels(L, "lsa_tree_10m", [0, 1, 100, 254, 255])

@@ -559,6 +559,23 @@ def test_lsa_tree_levels_brute_force_tiny(start_nodes, beam):
         assert out[i].tolist() == want.tolist(), t
 
 
+def test_lsa_tree_levels_empty_start_level_equals_flat_with_full_beam():
+    """A tree whose top level has no node (4992 buckets, node blocks of 4096:
+    1024 level-1 nodes, none at level 2) started there: every level-1 node is
+    uncovered and joins the level-1 candidates, so a full beam still reads
+    what the flat search reads."""
+    from workloads.synth import make_lsa
+    d = make_lsa(37, 40000, 512, 64, 0, 2053, True, node_block=4096, fanout=4, levels=2)
+    assert [x.shape[0] for x in d["node_levels"]] == [1024, 0]
+    flat = lsa_flat_select(d["q_idx"], d["q_pos"], d["centroids"], d["bucket_off"], d["bucket_mem"], 512, 64, 4,
+                           64, 512)
+    tree, det = lsa_tree_levels_select(d["q_idx"], d["q_pos"], d["centroids"], d["node_levels"], d["bucket_off"],
+                                       d["bucket_mem"], 512, 64, 4096, 4, 5000, 1, 4, 64, 512, return_detail=True)
+    assert det[0]["start"] == 2
+    for t in range(d["q_pos"].size):
+        assert np.array_equal(flat[t], tree[t]), t
+
+
 def test_lsa_tree_levels_counts_match_page_figures(golden_dir):
     """The beam rule replayed at 1M and 10M tokens: start level and the number
     of vectors scored for a query that sees the whole index are the pages'."""
