@@ -714,6 +714,14 @@ def test_lsa_prefill_chunk_small(L):
     _check_lsa(L, "lsa_prefill_s", [0, 1, 255, 256, 1000, 2047, 2048, 2999])
 
 
+def test_lsa_prefill_chunk_largest_top_p(L):
+    """The 3000-query chunk with the largest top_p (4096): samples every
+    256th bucket, lists of up to 16384, the 4096-entry top-k form."""
+    from dataclasses import replace
+    wl = replace(get_workload("lsa_prefill_s"), top_p=4096, budget=4096)
+    _check_lsa(L, "lsa_prefill_s", [0, 1, 1000, 2999], wl=wl)
+
+
 @pytest.mark.parametrize("fallback_rows", [0, 256, 700])
 def test_lsa_prefill_chunk_fallbacks(L, fallback_rows):
     """Every row of the 3000-query chunk misses its threshold and is scored in
@@ -824,11 +832,13 @@ def test_lsa_tree_levels_small(L, start_nodes):
     _check_lsa_tree_levels(L, "lsa_tree_levels_s", list(range(37)), start_nodes=start_nodes)
 
 
-def test_lsa_tree_levels_full_beam_matches_flat(L):
-    """A beam holding every visible entry of each level reads what the flat
-    search reads (band rule on the picks; read lists exactly)."""
+@pytest.mark.parametrize("beam", [1248, 4096])
+def test_lsa_tree_levels_full_beam_matches_flat(L, beam):
+    """A beam holding every visible entry of each level (1248, or the
+    largest beam, 4096) reads what the flat search reads (band rule on the
+    picks; read lists exactly)."""
     wl = get_workload("lsa_tree_levels_s")
-    keys, n, picked = _check_lsa_tree_levels(L, "lsa_tree_levels_s", list(range(37)), beam=1248, start_nodes=100)
+    keys, n, picked = _check_lsa_tree_levels(L, "lsa_tree_levels_s", list(range(37)), beam=beam, start_nodes=100)
     _check_lsa(L, "lsa_tree_levels_s", list(range(37)), wl=wl)
 
 
