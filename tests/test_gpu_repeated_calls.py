@@ -12,6 +12,9 @@ last tile), a chunk with k = 32 (many filtered candidates per tile), queries
 whose scores rise with position (every later tile overflows the candidate
 slots of half the rows: the full-tile fallback), and a 600-query chunk whose
 merge rows take the four-CTAs-per-SM top-k form the benchmark's chunk uses.
+The LSA sampled-threshold search gets the same treatment (one workspace,
+0xFF-filled, ten calls, bit-equal to its full-matrix form), with and without
+every row falling back.
 """
 
 from types import SimpleNamespace
@@ -157,3 +160,43 @@ def test_prefill_running_repeated_calls(L, case, fp8):
 def f32_bits_equal_rows(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return (np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
             == np.ascontiguousarray(b, dtype=np.float32).view(np.uint32)).all(axis=1)
+
+
+@pytest.mark.parametrize("case", ["plain", "all_fall_back"])
+def test_lsa_threshold_repeated_calls(L, case):
+    """Back-to-back calls of the LSA sampled-threshold search on the
+    3000-query chunk with one workspace (0xFF-filled first) and one set of
+    output buffers: every call's picks and read lists equal the full-matrix
+    form's bit for bit and the fault word stays clear.  The second case makes
+    every row miss its threshold (all centroids and queries along one
+    direction, so every visible bucket ties), which runs the device-listed
+    fallback in 256-row chunks on every call."""
+    wl = get_workload("lsa_prefill_s")
+    d = dict(make_workload("lsa_prefill_s"))
+    ex = wl.extra
+    if case == "all_fall_back":
+        rng = np.random.default_rng(4)
+        u = rng.standard_normal(64)
+        u /= np.linalg.norm(u)
+        d["q_idx"] = to_bf16_bits(np.broadcast_to(u, d["q_idx"].shape).copy())
+        d["centroids"] = to_bf16_bits(np.broadcast_to(u, d["centroids"].shape).copy())
+    fb_rows = 256 if case == "all_fall_back" else 0
+    args = (dev_bf16(d["q_idx"]), dev(d["q_pos"]), dev_bf16(d["centroids"]), dev(d["bucket_off"]),
+            dev(d["bucket_mem"]))
+    kw = dict(block_keys=ex["block_keys"], buckets_per_block=ex["bpb"], n_sink=ex["n_sink"], top_p=wl.top_p,
+              budget=wl.budget, want_picked=True)
+    k0, n0, p0 = L.ls_lsa_flat_select(*args, threshold=False, **kw)
+    T, P = d["q_idx"].shape[0], d["centroids"].shape[0]
+    need = L.lib().ls_lsa_flat_workspace_size(T, P, wl.top_p, 1, fb_rows)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    row = ex["n_sink"] + ex["block_keys"] + wl.budget
+    out = (torch.empty((T, row), dtype=torch.int32, device="cuda"), torch.empty((T,), dtype=torch.int32, device="cuda"))
+    L.ls_device_status()
+    results = []
+    for _ in range(10):
+        keys, n, picked = L.ls_lsa_flat_select(*args, threshold=True, fallback_rows=fb_rows, ws=ws, out=out, **kw)
+        results.append((keys.clone(), n.clone(), picked.clone()))
+    torch.cuda.synchronize()
+    for i, (keys, n, picked) in enumerate(results):
+        assert torch.equal(picked, p0) and torch.equal(n, n0) and torch.equal(keys, k0), f"call {i}"
+    assert L.ls_device_status() == 0
