@@ -626,8 +626,9 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* __restrict__ a, in
 
 // One CTA of 256 threads per query: the picked buckets are taken 1024 at a
 // time (4 per thread, every load of a round in flight together), their kept
-// member counts scanned across the block, and each thread copies its own
-// buckets' members to their offsets.
+// member counts scanned across the block, and the round's members copied by
+// the whole block (output slot q from the bucket whose start is the last one
+// at or below q), so that the stores are coalesced.
 constexpr int kExpandThreads = 256;
 constexpr int kExpandItems = 4;
 
@@ -671,7 +672,9 @@ __global__ void __launch_bounds__(kExpandThreads)
         if (n > 0) {
           const int32_t first = mem[o[i]], last = mem[o[i] + n - 1];
           lo[i] = (first >= n_sink) ? 0 : lower_bound_i32(mem + o[i], n, n_sink);
-          sz[i] = ((last < wstart) ? n : lower_bound_i32(mem + o[i], n, wstart)) - lo[i];
+          // (a bucket of the query's own block 0 can put the window's start
+          // below the sinks' end: nothing of it is kept then)
+          sz[i] = max(0, ((last < wstart) ? n : lower_bound_i32(mem + o[i], n, wstart)) - lo[i]);
         }
       }
       mine += sz[i];
