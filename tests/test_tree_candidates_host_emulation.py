@@ -1,0 +1,113 @@
+"""The LSA tree search's candidate-scoring kernel, compiled for the host (no GPU).
+
+`lsa_tree_candidates_kernel` (`csrc/score_tree.cuh`) lists a query's
+candidates at one level -- the children of its beam (nodes of the level
+above, -1 padding past the visible ones), then the level's visible entries
+that no node covers -- and scores each as its centroid's 64-d dot product
+with the index query.  Its source is preprocessed (the packed FMA through the
+shim's host version, the static shared query row a function static: the
+emulator runs one CTA at a time) and built with g++ under AddressSanitizer.
+Inputs: the three-level reduced index's level-1 centroids with level-2 beams
+(full, partial and empty), and the bucket level with level-1 beams.
+Expected: the candidate labels in that order, exactly, and scores within
+fp32 rounding of the oracle's fp64 dot products.  Test infrastructure only.
+"""
+
+import os
+import re
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle.formats import bf16_to_f64
+from oracle.select import lsa_tree_levels, lsa_visible
+from workloads import get_workload, make_workload
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(os.path.dirname(HERE), "sparse_attention_indexer_lightning_b200", "csrc")
+
+
+def _host_source() -> str:
+    with open(os.path.join(CSRC, "score_tree.cuh")) as f:
+        src = f.read()
+    parts = []
+    for pat in (r"__device__ __forceinline__ float dot64_bf16\(.*?\n\}\n",
+                r"__global__ void __launch_bounds__\(256\)\n    lsa_tree_candidates_kernel\(.*?\n\}\n"):
+        m = re.search(pat, src, flags=re.S)
+        assert m, pat
+        parts.append(m.group(0))
+    body = "".join(parts).replace("__shared__ ", "static ")
+    fma = 'asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc[e]) : "l"(cw), "l"(q2[4 * v + e]));'
+    assert fma in body
+    body = body.replace(fma, "acc[e] = host_fma2(acc[e], cw, q2[4 * v + e]);")
+    assert "asm(" not in body
+    return ('#pragma once\n#include "cuda_shim.h"\nnamespace lsi {\nconstexpr int kLsaDim = 64;\n' + body + "}\n")
+
+
+@pytest.fixture(scope="module")
+def cand_host(tmp_path_factory):
+    cxx = shutil.which("g++")
+    if cxx is None:
+        pytest.skip("no host C++ compiler")
+    d = tmp_path_factory.mktemp("tree_cand_host")
+    (d / "tree_cand_host.h").write_text(_host_source())
+    exe = d / "tree_cand_host"
+    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
+            os.path.join(HERE, "host_emulation", "tree_candidates_main.cpp")]
+    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
+                                   "-fno-omit-frame-pointer"] + base[1:], capture_output=True, text=True)
+    if r.returncode != 0:
+        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-3000:]
+    return d, exe, dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+
+
+@pytest.mark.parametrize("level", [0, 1])
+def test_candidates_and_scores(cand_host, level):
+    d, exe, env = cand_host
+    wl = get_workload("lsa_tree_levels_s")
+    ex = wl.extra
+    data = make_workload("lsa_tree_levels_s")
+    fan, blk, beam_w = ex["fanout"], ex["node_block"], 24
+    levels = [data["centroids"]] + list(data["node_levels"])
+    sizes = [x.shape[0] for x in levels]
+    q = data["q_idx"]
+    T = q.shape[0]
+    vis0 = lsa_visible(data["q_pos"], 512, 64, sizes[0])
+    rng = np.random.default_rng(level)
+    beam = np.full((T, beam_w), -1, dtype=np.int32)
+    vis = np.zeros(T, np.int32)
+    visn = np.zeros(T, np.int32)
+    for t in range(T):
+        v = lsa_tree_levels(vis0[t], sizes[1:], blk, fan)
+        vis[t], visn[t] = v[level], v[level + 1]
+        nb = min(beam_w, v[level + 1]) - (t % 4 == 1) * 3         # some beams shorter than the visible nodes
+        if nb > 0:
+            beam[t, :nb] = rng.permutation(v[level + 1])[:nb]
+    cap = beam_w * fan + blk
+    c = levels[level]
+    q.astype(np.uint16).tofile(d / "q.bin")
+    c.astype(np.uint16).tofile(d / "c.bin")
+    beam.tofile(d / "beam.bin")
+    vis.tofile(d / "vis.bin")
+    visn.tofile(d / "visn.bin")
+    r = subprocess.run([str(exe), str(d), str(T), str(c.shape[0]), str(beam_w), str(fan), str(cap)],
+                       capture_output=True, text=True, env=env, timeout=900)
+    assert r.returncode == 0, r.stderr[-3000:]
+    cval = np.fromfile(d / "cval.bin", dtype=np.float32).reshape(T, cap)
+    clab = np.fromfile(d / "clab.bin", dtype=np.int32).reshape(T, cap)
+    nv = np.fromfile(d / "nv.bin", dtype=np.int32)
+    cf = bf16_to_f64(c)
+    for t in range(T):
+        nb = min(beam_w, int(visn[t]))
+        labs = [int(beam[t, i // fan]) * fan + i % fan if beam[t, i // fan] >= 0 else -1 for i in range(nb * fan)]
+        labs += list(range(fan * int(visn[t]), int(vis[t])))
+        assert nv[t] == len(labs), t
+        assert np.array_equal(clab[t, :nv[t]], np.asarray(labs, dtype=np.int32)), t
+        ok = np.asarray(labs) >= 0
+        ref = cf[np.asarray(labs)[ok]] @ bf16_to_f64(q[t]) if ok.any() else np.zeros(0)
+        got = cval[t, :nv[t]][ok]
+        assert np.allclose(got, ref, rtol=1e-5, atol=1e-6), t
+        assert np.all(np.isneginf(cval[t, :nv[t]][~ok])), t
