@@ -1,15 +1,19 @@
-// Runs the LSA tree search's candidate-scoring kernel (lsa_tree_candidates_kernel,
-// the library's source made host-compilable by cuda_shim.h and the test's
-// preprocessing) on files of inputs, one OS thread per CUDA thread, one
-// query (CTA) at a time.  Test infrastructure only.
+// Runs the LSA tree search's candidate-scoring kernel (lsa_tree_candidates_kernel)
+// and its level-visibility kernel (lsa_tree_levels_visible_kernel), the library's
+// source made host-compilable by cuda_shim.h and the test's preprocessing, on
+// files of inputs, one OS thread per CUDA thread, one CTA at a time.  Test
+// infrastructure only.
 //   DIR T R beam_w fanout cap
 //   inputs: q.bin [T][64] u16 (bf16), c.bin [R][64] u16, beam.bin [T][beam_w] i32,
 //           vis.bin [T] i32, visn.bin [T] i32
 //   outputs: cval.bin [T][cap] f32, clab.bin [T][cap] i32, nv.bin [T] i32
+//   DIR vis T block_keys bpb node_block fanout n size_0 .. size_n
+//   inputs: pos.bin [T] i64; output: lvis.bin [n + 1][T] i32
 #include "tree_cand_host.h"
 
 #include <cstdio>
 #include <cstdlib>
+#include <string>
 #include <thread>
 #include <vector>
 
@@ -42,9 +46,36 @@ static void save(const char* dir, const char* name, const std::vector<T>& v) {
   std::fclose(f);
 }
 
+static int run_visible(const char* dir, int argc, char** argv) {
+  const int T = std::atoi(argv[3]), block_keys = std::atoi(argv[4]), bpb = std::atoi(argv[5]);
+  const int node_block = std::atoi(argv[6]), fanout = std::atoi(argv[7]), n = std::atoi(argv[8]);
+  if (n < 1 || n > lsi::kMaxTreeLevels || argc != 10 + n) return 2;
+  lsi::TreeLevels lv;
+  lv.n = n;
+  for (int l = 0; l <= n; ++l) lv.size[l] = std::atoi(argv[9 + l]);
+  auto pos = load<int64_t>(dir, "pos.bin", static_cast<size_t>(T));
+  std::vector<int32_t> vis(static_cast<size_t>(n + 1) * T, 777);
+  const int NT = 256, NB = (T + NT - 1) / NT;
+  blockDim = {static_cast<unsigned>(NT), 1, 1};
+  gridDim = {static_cast<unsigned>(NB), 1, 1};
+  for (int b = 0; b < NB; ++b) {
+    std::vector<std::thread> th;
+    for (int t = 0; t < NT; ++t)
+      th.emplace_back([&, t, b] {
+        threadIdx = {static_cast<unsigned>(t), 0, 0};
+        blockIdx = {static_cast<unsigned>(b), 0, 0};
+        lsi::lsa_tree_levels_visible_kernel(pos.data(), T, block_keys, bpb, node_block, fanout, lv, vis.data());
+      });
+    for (auto& x : th) x.join();
+  }
+  save(dir, "lvis.bin", vis);
+  return 0;
+}
+
 int main(int argc, char** argv) {
   if (argc < 7) return 2;
   const char* dir = argv[1];
+  if (std::string(argv[2]) == "vis") return run_visible(dir, argc, argv);
   const int T = std::atoi(argv[2]), R = std::atoi(argv[3]), beam_w = std::atoi(argv[4]);
   const int fanout = std::atoi(argv[5]), cap = std::atoi(argv[6]);
   auto q = load<uint16_t>(dir, "q.bin", static_cast<size_t>(T) * 64);

@@ -1,4 +1,5 @@
-"""The LSA tree search's candidate-scoring kernel, compiled for the host (no GPU).
+"""The LSA tree search's candidate-scoring and level-visibility kernels, compiled
+for the host (no GPU).
 
 `lsa_tree_candidates_kernel` (`csrc/score_tree.cuh`) lists a query's
 candidates at one level -- the children of its beam (nodes of the level
@@ -10,7 +11,13 @@ emulator runs one CTA at a time) and built with g++ under AddressSanitizer.
 Inputs: the three-level reduced index's level-1 centroids with level-2 beams
 (full, partial and empty), and the bucket level with level-1 beams.
 Expected: the candidate labels in that order, exactly, and scores within
-fp32 rounding of the oracle's fp64 dot products.  Test infrastructure only.
+fp32 rounding of the oracle's fp64 dot products.
+
+`lsa_tree_levels_visible_kernel` gives each query its visible entry count at
+every level: complete key blocks at the bucket level, complete node blocks
+above, each capped by the level's size.  Expected: the oracle's
+`lsa_visible` and `lsa_tree_levels`, exactly, for positions at and around
+every block edge.  Test infrastructure only.
 """
 
 import os
@@ -33,7 +40,9 @@ def _host_source() -> str:
     with open(os.path.join(CSRC, "score_tree.cuh")) as f:
         src = f.read()
     parts = []
-    for pat in (r"__device__ __forceinline__ float dot64_bf16\(.*?\n\}\n",
+    for pat in (r"struct TreeLevels \{.*?\n\};\n",
+                r"__global__ void lsa_tree_levels_visible_kernel\(.*?\n\}\n",
+                r"__device__ __forceinline__ float dot64_bf16\(.*?\n\}\n",
                 r"__global__ void __launch_bounds__\(256\)\n    lsa_tree_candidates_kernel\(.*?\n\}\n"):
         m = re.search(pat, src, flags=re.S)
         assert m, pat
@@ -43,7 +52,7 @@ def _host_source() -> str:
     assert fma in body
     body = body.replace(fma, "acc[e] = host_fma2(acc[e], cw, q2[4 * v + e]);")
     assert "asm(" not in body
-    return ('#pragma once\n#include "cuda_shim.h"\nnamespace lsi {\nconstexpr int kLsaDim = 64;\n' + body + "}\n")
+    return ('#pragma once\n#include "cuda_shim.h"\nnamespace lsi {\nconstexpr int kLsaDim = 64;\nconstexpr int kMaxTreeLevels = 16;\n' + body + "}\n")
 
 
 @pytest.fixture(scope="module")
@@ -111,3 +120,27 @@ def test_candidates_and_scores(cand_host, level):
         got = cval[t, :nv[t]][ok]
         assert np.allclose(got, ref, rtol=1e-5, atol=1e-6), t
         assert np.all(np.isneginf(cval[t, :nv[t]][~ok])), t
+
+
+@pytest.mark.parametrize("shape", [(512, 64, 4096, 4, [5000, 1248, 312, 76]),
+                                   (512, 64, 4096, 4, [40960, 10240, 2560]),
+                                   (128, 16, 256, 2, [3000, 1500, 700, 300, 100, 40])])
+def test_level_visibility(cand_host, shape):
+    d, exe, env = cand_host
+    block_keys, bpb, blk, fan, sizes = shape
+    n_keys = sizes[0] // bpb * block_keys
+    edges = np.arange(0, n_keys + 3 * block_keys, block_keys, dtype=np.int64)
+    rng = np.random.default_rng(len(sizes))
+    pos = np.concatenate([edges - 1, edges, edges + 1, rng.integers(0, n_keys + 2 * block_keys, 700),
+                          np.asarray([0, 1, (blk // bpb) * block_keys - 1, (blk // bpb) * block_keys])]).astype(np.int64)
+    pos = pos[pos >= 0]
+    T = pos.shape[0]
+    pos.tofile(d / "pos.bin")
+    args = [str(exe), str(d), "vis", str(T), str(block_keys), str(bpb), str(blk), str(fan), str(len(sizes) - 1)]
+    r = subprocess.run(args + [str(x) for x in sizes], capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    got = np.fromfile(d / "lvis.bin", dtype=np.int32).reshape(len(sizes), T)
+    vis0 = lsa_visible(pos, block_keys, bpb, sizes[0])
+    for t in range(T):
+        want = lsa_tree_levels(int(vis0[t]), sizes[1:], blk, fan)
+        assert list(got[:, t]) == list(want), (t, int(pos[t]))
