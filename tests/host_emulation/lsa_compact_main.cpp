@@ -87,6 +87,22 @@ int main(int argc, char** argv) {
   run_grid(1, 1024, [&] {
     lsi::lsa_flag_list_kernel(over.data(), T, rows, n_chunks, list.data(), count.data(), run.data());
   });
+  // the missed rows' queries and visible counts, gathered once for all
+  // chunks; a second gather with its run flag clear must write nothing
+  auto q = load<uint16_t>(dir, "q.bin", static_cast<size_t>(T) * 64);
+  std::vector<uint16_t> qbuf(static_cast<size_t>(T) * 64, 0x7777), qidle(static_cast<size_t>(T) * 64, 0x7777);
+  std::vector<int32_t> vbuf(T, 777), vidle(T, 777);
+  const int zero = 0;
+  run_grid((T * 8 + 255) / 256, 256, [&] {
+    lsi::lsa_gather_rows_kernel(list.data(), count.data(), T, q.data(), vis.data(), &any, qbuf.data(), vbuf.data());
+  });
+  run_grid((T * 8 + 255) / 256, 256, [&] {
+    lsi::lsa_gather_rows_kernel(list.data(), count.data(), T, q.data(), vis.data(), &zero, qidle.data(), vidle.data());
+  });
+  save(dir, "qbuf.bin", qbuf);
+  save(dir, "vbuf.bin", vbuf);
+  save(dir, "qidle.bin", qidle);
+  save(dir, "vidle.bin", vidle);
   over.push_back(any);
   save(dir, "cval.bin", cval);
   save(dir, "clab.bin", clab);

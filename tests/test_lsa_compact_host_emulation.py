@@ -4,7 +4,10 @@
 that scored the row, each in four quarters with their own counts) into one
 list, and flags the rows whose list ran over or came up short;
 `lsa_flag_list_kernel` lists the flagged rows in ascending order and marks
-the fallback chunks that hold any.  Their source in `csrc/score_dot.cuh` and
+the fallback chunks that hold any; `lsa_gather_rows_kernel` copies the listed
+rows' index queries and visible counts, in list order, into the fallback's
+buffers (zeros past the count), and writes nothing while its run flag is
+clear.  Their source in `csrc/score_dot.cuh` and
 the segment arithmetic in `csrc/kernels.h` are preprocessed (static shared
 arrays become function statics: the emulator runs one CTA at a time) and
 built with g++ under AddressSanitizer, each CUDA thread an OS thread with real
@@ -12,7 +15,7 @@ barriers.  Inputs: segment contents and counts laid out as the scan writes
 them, for one query group with every CTA and for many groups with a few
 CTAs each, counts past a quarter's length (the scan's overflow), empty
 quarters, short and long lists.  Expected: the segments' entries in quarter
-order, the flags, the list and the chunk marks, exactly.  Test
+order, the flags, the list, the chunk marks and the gathered rows, exactly.  Test
 infrastructure only.
 """
 
@@ -40,11 +43,13 @@ def _host_source() -> str:
         assert m, pat
         parts.append(m.group(0))
     for pat in (r"__global__ void __launch_bounds__\(256\)\n    lsa_compact_kernel\(.*?\n\}\n",
-                r"__global__ void __launch_bounds__\(1024\)\n    lsa_flag_list_kernel\(.*?\n\}\n"):
+                r"__global__ void __launch_bounds__\(1024\)\n    lsa_flag_list_kernel\(.*?\n\}\n",
+                r"__global__ void lsa_gather_rows_kernel\(.*?\n\}\n"):
         m = re.search(pat, dot, flags=re.S)
         assert m, pat
         parts.append(m.group(0).replace("__shared__ ", "static "))
     return ('#pragma once\n#include "cuda_shim.h"\nnamespace lsi {\nstruct DotCfg { static constexpr int QB = 256; };\n'
+            'constexpr int kLsaDim = 64;\n'
             + "".join(parts) + "}\n")
 
 
@@ -130,9 +135,11 @@ def test_compaction_and_missed_rows(compact_host, T, P, top_p):
         want_over[t] = int(total > cap or total < min(top_p, vis[t]))
         want_val.append(slist[t, entries, 0] if total <= cap else None)
         want_lab.append(slist[t, entries, 1] if total <= cap else None)
+    q = rng.integers(0, 2 ** 16, size=(T, 64), dtype=np.uint16)
     slist.tofile(d / "slist.bin")
     cnt.tofile(d / "cnt.bin")
     vis.tofile(d / "vis.bin")
+    q.tofile(d / "q.bin")
     rows = 50
     n_chunks = (T + rows - 1) // rows
     r = subprocess.run([str(exe), str(d), str(T), str(P), str(cap2), str(slack), str(nseg), str(grid), str(top_p),
@@ -156,3 +163,9 @@ def test_compaction_and_missed_rows(compact_host, T, P, top_p):
     assert count == flagged.size
     assert np.array_equal(lst[:count], flagged) and np.all(lst[count:] == -1)
     assert np.array_equal(run, (np.arange(n_chunks) * rows < count).astype(np.int32))
+    qbuf = np.fromfile(d / "qbuf.bin", dtype=np.uint16).reshape(T, 64)
+    vbuf = np.fromfile(d / "vbuf.bin", dtype=np.int32)
+    assert np.array_equal(qbuf[:count], q[flagged]) and np.all(qbuf[count:] == 0)
+    assert np.array_equal(vbuf[:count], vis[flagged]) and np.all(vbuf[count:] == 0)
+    assert np.all(np.fromfile(d / "qidle.bin", dtype=np.uint16) == 0x7777)
+    assert np.all(np.fromfile(d / "vidle.bin", dtype=np.int32) == 777)
