@@ -9,6 +9,10 @@
 //   outputs: cval.bin [T][cap] f32, clab.bin [T][cap] i32, nv.bin [T] i32
 //   DIR vis T block_keys bpb node_block fanout n size_0 .. size_n
 //   inputs: pos.bin [T] i64; output: lvis.bin [n + 1][T] i32
+// and the one-level tree's and the flat search's visibility kernels
+// (lsa_tree_visible_kernel, lsa_visible_kernel):
+//   DIR vis1 T block_keys bpb P node_block fanout P1   pos.bin -> lvis.bin [2][T] i32
+//   DIR visflat T block_keys bpb P stride              pos.bin -> lvis.bin [2][T] i32 (vis, samples)
 #include "tree_cand_host.h"
 
 #include <cstdio>
@@ -72,10 +76,48 @@ static int run_visible(const char* dir, int argc, char** argv) {
   return 0;
 }
 
+// One thread per query over ceil(T / 256) CTAs of 256 threads.
+template <class F>
+static void run_per_query(int T, F body) {
+  const int NT = 256, NB = (T + NT - 1) / NT;
+  blockDim = {static_cast<unsigned>(NT), 1, 1};
+  gridDim = {static_cast<unsigned>(NB), 1, 1};
+  for (int b = 0; b < NB; ++b) {
+    std::vector<std::thread> th;
+    for (int t = 0; t < NT; ++t)
+      th.emplace_back([&, t, b] {
+        threadIdx = {static_cast<unsigned>(t), 0, 0};
+        blockIdx = {static_cast<unsigned>(b), 0, 0};
+        body();
+      });
+    for (auto& x : th) x.join();
+  }
+}
+
 int main(int argc, char** argv) {
   if (argc < 7) return 2;
   const char* dir = argv[1];
-  if (std::string(argv[2]) == "vis") return run_visible(dir, argc, argv);
+  const std::string mode = argv[2];
+  if (mode == "vis") return run_visible(dir, argc, argv);
+  if (mode == "vis1" || mode == "visflat") {
+    const int T = std::atoi(argv[3]), block_keys = std::atoi(argv[4]), bpb = std::atoi(argv[5]), P = std::atoi(argv[6]);
+    auto pos = load<int64_t>(dir, "pos.bin", static_cast<size_t>(T));
+    std::vector<int32_t> out(static_cast<size_t>(2) * T, 777);
+    if (mode == "vis1" && argc == 10) {
+      const int node_block = std::atoi(argv[7]), fanout = std::atoi(argv[8]), P1 = std::atoi(argv[9]);
+      run_per_query(T, [&] {
+        lsi::lsa_tree_visible_kernel(pos.data(), T, block_keys, bpb, P, node_block, fanout, P1, out.data(),
+                                     out.data() + T);
+      });
+    } else if (mode == "visflat" && argc == 8) {
+      const int stride = std::atoi(argv[7]);
+      run_per_query(T, [&] { lsi::lsa_visible_kernel(pos.data(), T, block_keys, bpb, P, stride, out.data(), out.data() + T); });
+    } else {
+      return 2;
+    }
+    save(dir, "lvis.bin", out);
+    return 0;
+  }
   const int T = std::atoi(argv[2]), R = std::atoi(argv[3]), beam_w = std::atoi(argv[4]);
   const int fanout = std::atoi(argv[5]), cap = std::atoi(argv[6]);
   auto q = load<uint16_t>(dir, "q.bin", static_cast<size_t>(T) * 64);

@@ -17,7 +17,9 @@ fp32 rounding of the oracle's fp64 dot products.
 every level: complete key blocks at the bucket level, complete node blocks
 above, each capped by the level's size.  Expected: the oracle's
 `lsa_visible` and `lsa_tree_levels`, exactly, for positions at and around
-every block edge.  Test infrastructure only.
+every block edge.  The one-level tree's visibility kernel and the flat
+search's (which also counts the sampled buckets below the visible count, every
+stride-th from bucket 0) are checked the same way.  Test infrastructure only.
 """
 
 import os
@@ -40,7 +42,12 @@ def _host_source() -> str:
     with open(os.path.join(CSRC, "score_tree.cuh")) as f:
         src = f.read()
     parts = []
-    for pat in (r"struct TreeLevels \{.*?\n\};\n",
+    with open(os.path.join(CSRC, "score_dot.cuh")) as f:
+        m = re.search(r"__global__ void lsa_visible_kernel\(.*?\n\}\n", f.read(), flags=re.S)
+    assert m, "lsa_visible_kernel"
+    parts.append(m.group(0))
+    for pat in (r"__global__ void lsa_tree_visible_kernel\(.*?\n\}\n",
+                r"struct TreeLevels \{.*?\n\};\n",
                 r"__global__ void lsa_tree_levels_visible_kernel\(.*?\n\}\n",
                 r"__device__ __forceinline__ float dot64_bf16\(.*?\n\}\n",
                 r"__global__ void __launch_bounds__\(256\)\n    lsa_tree_candidates_kernel\(.*?\n\}\n"):
@@ -144,3 +151,45 @@ def test_level_visibility(cand_host, shape):
     for t in range(T):
         want = lsa_tree_levels(int(vis0[t]), sizes[1:], blk, fan)
         assert list(got[:, t]) == list(want), (t, int(pos[t]))
+
+
+def _edge_positions(block_keys, n_keys, node_span, seed):
+    edges = np.arange(0, n_keys + 3 * block_keys, block_keys, dtype=np.int64)
+    rng = np.random.default_rng(seed)
+    pos = np.concatenate([edges - 1, edges, edges + 1, rng.integers(0, n_keys + 2 * block_keys, 700),
+                          np.asarray([-5, -block_keys - 1, -3 * block_keys, 0, 1, node_span - 1, node_span])]).astype(np.int64)   # negative positions are clamped to 0
+    return pos
+
+
+@pytest.mark.parametrize("shape", [(512, 64, 5000, 4096, 4, 1248), (512, 64, 131072, 4096, 4, 32768),
+                                   (128, 16, 3000, 256, 2, 700)])
+def test_one_level_visibility(cand_host, shape):
+    d, exe, env = cand_host
+    block_keys, bpb, P, blk, fan, P1 = shape
+    pos = _edge_positions(block_keys, P // bpb * block_keys, (blk // bpb) * block_keys, P)
+    pos.tofile(d / "pos.bin")
+    T = pos.size
+    r = subprocess.run([str(exe), str(d), "vis1", str(T), str(block_keys), str(bpb), str(P), str(blk), str(fan), str(P1)],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    got = np.fromfile(d / "lvis.bin", dtype=np.int32).reshape(2, T)
+    vis0 = lsa_visible(pos, block_keys, bpb, P)
+    assert np.array_equal(got[0], vis0.astype(np.int32))
+    want = [lsa_tree_levels(int(v), [P1], blk, fan)[1] for v in vis0]
+    assert np.array_equal(got[1], np.asarray(want, dtype=np.int32))
+
+
+@pytest.mark.parametrize("shape", [(512, 64, 131072, 64), (512, 64, 1310720, 64), (128, 16, 3000, 1), (512, 64, 5000, 7)])
+def test_flat_visibility_and_sample_counts(cand_host, shape):
+    d, exe, env = cand_host
+    block_keys, bpb, P, stride = shape
+    pos = _edge_positions(block_keys, P // bpb * block_keys, block_keys, stride)
+    pos.tofile(d / "pos.bin")
+    T = pos.size
+    r = subprocess.run([str(exe), str(d), "visflat", str(T), str(block_keys), str(bpb), str(P), str(stride)],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    got = np.fromfile(d / "lvis.bin", dtype=np.int32).reshape(2, T)
+    vis0 = lsa_visible(pos, block_keys, bpb, P)
+    assert np.array_equal(got[0], vis0.astype(np.int32))
+    assert np.array_equal(got[1], np.asarray([len(range(0, int(v), stride)) for v in vis0], dtype=np.int32))
