@@ -257,6 +257,13 @@ def time_loop(fn, steps, warmup, stream, marks=None):
     return total, seg
 
 
+def decode_config(wl, B, N, H, dd, world):
+    """The decode workload's `config` entry, the same on both arms."""
+    return {"workload": wl.name, "sequences_per_gpu": B, "compressed_positions": N, "tokens_per_sequence": 4 * N,
+            "heads": H, "d": dd, "k": wl.k, "parallelism": f"replicas x{world}",
+            "l2": f"inputs ({B * N * dd * 2 / 1e6:.0f} MB keys) larger than the 126 MB L2; no flush"}
+
+
 def bench_decode(L, args, world, rank, peaks, peak_kind):
     import torch
     from workloads import get_workload, make_workload
@@ -307,9 +314,7 @@ def bench_decode(L, args, world, rank, peaks, peak_kind):
         "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(d) keys and queries, N(0,1)/sqrt(H) head weights)",
-        "config": {"workload": wl.name, "sequences_per_gpu": B, "compressed_positions": N, "tokens_per_sequence": 4 * N,
-                   "heads": H, "d": dd, "k": wl.k, "parallelism": f"replicas x{world}",
-                   "l2": "inputs (537 MB keys) larger than the 126 MB L2; no flush"},
+        "config": decode_config(wl, B, N, H, dd, world),
         "selections_per_s": world * B / (ms_per_step * 1e-3),
         "breakdown_ms": {"scan": scan_ms, "topk": topk_ms},
         "kernels": {kname: {"total_ms": v[0], "launches": v[1]} for kname, v in prof.items()},
@@ -926,13 +931,18 @@ def run_reference(args):
         seqs += n
     value = statistics.median(rates)
     cores = blas_threads()
+    H, dd = d["q"].shape[1], d["q"].shape[2]
     line = {
         "impl": "reference", "metric": "indexer query-positions scored/sec (decode selection, top-512)",
         "value": value, "unit": "positions/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": N / value * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f64", "data": "synthetic", "config": {"workload": wl.name, "sequences": B, "compressed_positions": N},
+        # the time one step of the workload (all B sequences) takes at the measured rate
+        "ms_per_step": B * N / value * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "config": decode_config(wl, B, N, H, dd, 1),
         "cpu_baseline": {"value": value, "unit": "positions/s", "cores": cores, "kind": "oracle",
-                         "sample": f"whole sequences of {N} positions, {seqs} in total over {args.steps} steps"},
+                         "sample": f"whole sequences of {N} positions cycled through the batch for about "
+                                   f"{per_step_budget:.0f} s per timed step, {seqs} in total over {args.steps} "
+                                   f"steps; value = the median step's rate, ms_per_step = a {B}-sequence step "
+                                   f"at that rate"},
         "e2e": {"value": value, "unit": "positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))

@@ -84,3 +84,39 @@ def test_variant_children_isolate_failures(monkeypatch):
     assert "timed out" in res["bucket"]["error"]
     assert "exit 0" in res["lsa_flat"]["error"]
     assert set(bench.DEFAULT_VARIANTS) <= set(bench.VARIANTS)
+
+
+def test_reference_line(monkeypatch, capsys):
+    """The reference arm's line: the oracle's rate on rank 0 only, the decode
+    line's metric, unit and config, a cpu_baseline and an e2e equal to the
+    line's value with no copies declared, and a step time that is one step of
+    the workload (all its sequences) at that rate."""
+    import types
+
+    import numpy as np
+    import workloads
+
+    B, N, H, dd = 4, 1000, 32, 128
+    tiny = {"q": np.zeros((B, H, dd), np.uint16), "w": np.zeros((B, H), np.float32),
+            "k": np.zeros((B, N, dd), np.uint16)}
+    monkeypatch.setattr(workloads, "make_workload", lambda wl, **kw: tiny)
+    rates = iter([5.0e6, 9.0e6,                         # warm-up calls (ignored)
+                  2.0e6, 3.0e6, 1.0e6] * 4)             # timed steps: the median is 2.0e6
+    monkeypatch.setattr(bench, "oracle_decode_rate", lambda d, budget, k: (next(rates), 7, budget))
+    monkeypatch.setattr(bench, "blas_threads", lambda: 8)
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    assert bench.run_reference(types.SimpleNamespace(steps=3, warmup=2, workload="decode_batch")) == 0
+    line = bench.json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] == 2.0e6 and line["unit"] == "positions/s"
+    assert line["metric"].startswith("indexer query-positions scored/sec")
+    assert line["ms_per_step"] == pytest.approx(B * N / 2.0e6 * 1e3)
+    assert line["config"] == bench.decode_config(workloads.get_workload("decode_batch"), B, N, H, dd, 1)
+    assert line["cpu_baseline"]["value"] == line["value"] and line["cpu_baseline"]["cores"] == 8
+    assert line["cpu_baseline"]["kind"] == "oracle" and "21 in total over 3 steps" in line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": 2.0e6, "unit": "positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # under torchrun the other ranks exit without work or output
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.run_reference(types.SimpleNamespace(steps=3, warmup=2, workload="decode_batch")) == 0
+    assert capsys.readouterr().out == ""
