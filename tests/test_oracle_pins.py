@@ -14,10 +14,11 @@ import pytest
 import torch
 
 from oracle import brute, sizes
-from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64, f16_to_f64, pq_decode
+from oracle.formats import bf16_to_f64, dequant, e4m3_to_f64, f16_to_f64, int8_to_f64, pq_decode
 from oracle.indexer import eligible_blocks, eligible_count, indexer_scores
 from oracle.select import (
-    bucket_select, decode_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_levels_select,
+    bucket_select, decode_select, expand_buckets, lsa_flat_select, lsa_read_list, lsa_tree_levels,
+    lsa_tree_levels_select,
     lsa_tree_select, lsa_visible, prefill_select,
     prefill_select_fp8, recall_at_k, select_topk, topk_rows, two_stage_pq_select, two_stage_select,
 )
@@ -50,6 +51,13 @@ def test_e4m3_decode_all_codes():
     assert e4m3_to_f64(np.array([0x01]))[0] == 2.0 ** -9
     assert e4m3_to_f64(np.array([0x38]))[0] == 1.0
     assert e4m3_to_f64(np.array([0xB8]))[0] == -1.0
+
+
+def test_int8_decode_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.int8).to(torch.float64).numpy()
+    assert np.array_equal(int8_to_f64(codes), ref)
+    assert int8_to_f64(np.array([0x80], np.uint8))[0] == -128.0 and int8_to_f64(np.array([0x7F], np.uint8))[0] == 127.0
 
 
 def test_f16_decode_all_codes():
@@ -515,6 +523,26 @@ def test_lsa_tree_levels_one_level_equals_one_level_search():
                                 96, 32768, 4, 64, 512)
     for t in range(d["q_pos"].size):
         assert np.array_equal(one[t], lv[t]), t
+
+
+@pytest.mark.parametrize("node_block,fanout", [(16, 4), (8, 2), (12, 3)])
+def test_lsa_tree_levels_by_explicit_blocks(node_block, fanout):
+    """Level l's node j exists for a query when every entry of its node
+    cluster block at level l - 1 is visible: the block of node j is entries
+    (j // (node_block / fanout)) * node_block ... + node_block - 1 below.
+    Counted here entry by entry, up to each level's size."""
+    per = node_block // fanout
+    sizes = [97, 30, 9, 2]                               # level sizes 1..4 (level 0: the visible buckets)
+    for vis in range(0, 400, 3):
+        want, below = [vis], vis
+        for size in sizes:
+            n = sum(1 for j in range(size) if (j // per) * node_block + node_block <= below)
+            want.append(n)
+            below = n
+        assert lsa_tree_levels(vis, sizes, node_block, fanout) == want, vis
+    # 1M tokens: 131072 buckets in 32 complete 4096-bucket blocks -> 32768 level-1 nodes
+    assert lsa_tree_levels(131072, [32768, 8192], 4096, 4) == [131072, 32768, 8192]
+    assert lsa_tree_levels(131071, [32768, 8192], 4096, 4) == [131071, 31744, 7168]
 
 
 @pytest.mark.parametrize("start_nodes,beam", [(100, 5), (500, 7), (5000, 9)])
