@@ -180,6 +180,42 @@ def test_argument_checks_without_gpu(lib):
     assert lib.ls_profile_kernel(0, None, None, None) == 1
 
 
+def test_tree_levels_argument_checks(lib):
+    """ls_lsa_tree_levels_select and its workspace query refuse bad trees
+    before touching CUDA: the host arrays are read, nothing is launched."""
+    P = ctypes.c_void_p
+    dummy = P(16)
+    sizes = (ctypes.c_int * 3)(32768, 8192, 2048)
+    nodes = (ctypes.c_void_p * 3)(16, 32, 48)
+
+    def call(L=3, d=64, Pb=131072, beam=2048, start=32768, ws_bytes=1 << 40, level_sizes=sizes, node_ptrs=nodes,
+             T=4, node_block=4096, fanout=4):
+        return lib.ls_lsa_tree_levels_select(dummy, dummy, dummy, ctypes.cast(node_ptrs, P),
+                                             ctypes.cast(level_sizes, P), L, dummy, dummy, T, d, Pb, 512, 64,
+                                             node_block, fanout, beam, start, 4, 1024, 4096, dummy, dummy, None,
+                                             None, dummy, ws_bytes, None)
+
+    ws_size = lib.ls_lsa_tree_levels_workspace_size
+    good = ws_size(4, 131072, ctypes.cast(sizes, P), 3, 4096, 4, 2048, 32768, 1024)
+    assert good > 0
+    assert call(d=128) == 3                                      # the index space is 64-d
+    assert call(L=0) == 1 and call(L=17) == 1                    # 1 .. 16 levels
+    big = (ctypes.c_int * 3)(32768, 8193, 2048)                  # 8193 nodes of 4 exceed 32768 below
+    assert call(level_sizes=big) == 1
+    assert ws_size(4, 131072, ctypes.cast(big, P), 3, 4096, 4, 2048, 32768, 1024) == 0
+    assert call(beam=0) == 1 and call(beam=5000) == 1 and call(start=0) == 1
+    assert call(node_block=4098) == 1                            # not a multiple of fanout
+    assert call(Pb=100000) == 1                                  # level 1 needs 4 * 32768 buckets
+    assert "level 1" in lib.ls_last_error().decode()
+    null_level = (ctypes.c_void_p * 3)(16, None, 48)
+    assert call(node_ptrs=null_level) == 1 and b"level 2" in lib.ls_last_error()
+    odd_level = (ctypes.c_void_p * 3)(16, 32, 40)                # level 3's centroids 8-byte aligned only
+    assert call(node_ptrs=odd_level) == 1
+    assert call(ws_bytes=good - 1) == 2
+    assert call(T=0, ws_bytes=0) == 0                            # an empty batch is a no-op
+    assert ws_size(0, 131072, ctypes.cast(sizes, P), 3, 4096, 4, 2048, 32768, 1024) == 0
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from sparse_attention_indexer_lightning_b200 import _lib
     with pytest.raises(ImportError):
