@@ -222,22 +222,50 @@ def test_missing_library_fails_loudly(tmp_path):
         _lib.load_library(str(tmp_path / "libls_indexer.so"))
 
 
-def test_bindings_refuse_host_tensors():
-    """The Python calls only marshal device tensors into the C ABI: host
-    tensors are refused before anything runs (there is no CPU path)."""
+def _host_calls():
+    """One call of each Python entry point with host (CPU) tensors of the
+    right dtypes and shapes."""
     import torch
     import sparse_attention_indexer_lightning_b200 as L
-    q = torch.zeros((2, 8, 576), dtype=torch.bfloat16)
-    lat = torch.zeros((10, 576), dtype=torch.bfloat16)
-    idx = torch.zeros((2, 4), dtype=torch.int32)
+    bf, f32, i32, i64 = torch.bfloat16, torch.float32, torch.int32, torch.int64
+    z = torch.zeros
+    B, T, H, d, N, P = 2, 3, 32, 128, 64, 16
+    e4 = torch.float8_e4m3fn
+    return {
+        "ls_indexer_score": lambda: L.ls_indexer_score(z(B, T, H, d, dtype=bf), z(B, T, H), z(B, N, d, dtype=bf)),
+        "ls_topk_select": lambda: L.ls_topk_select(z(B, N), 8),
+        "ls_decode_select": lambda: L.ls_decode_select(z(B, H, d, dtype=bf), z(B, H), z(B, N, d, dtype=bf), k=8),
+        "ls_decode_select_noalloc": lambda: L.ls_decode_select_noalloc(z(B, H, d, dtype=bf), z(B, H),
+                                                                       z(B, N, d, dtype=bf), k=8),
+        "ls_indexer_score_fp8": lambda: L.ls_indexer_score_fp8(z(B, T, H, d, dtype=e4), z(B, T, H), z(B, T, H),
+                                                               z(B, N, d, dtype=e4), z(B, N)),
+        "ls_decode_two_stage_select": lambda: L.ls_decode_two_stage_select(
+            z(B, H, d, dtype=bf), z(B, H), z(B, N, d, dtype=torch.int8), z(B, N), z(B, N, d, dtype=e4), z(B, N),
+            shortlist=16, k=8),
+        "ls_indexer_score_pq": lambda: L.ls_indexer_score_pq(z(B, H, d, dtype=bf), z(B, H),
+                                                             z(B, N, 32, dtype=torch.uint8),
+                                                             z(32, 256, 4, dtype=torch.float16)),
+        "ls_bucket_select": lambda: L.ls_bucket_select(z(B, H, d, dtype=bf), z(B, H), z(P, d, dtype=bf),
+                                                       z(P + 1, dtype=i32), z(N, dtype=i32), z(N, d, dtype=bf),
+                                                       top_p=4, budget=16, k=8),
+        "ls_lsa_flat_select": lambda: L.ls_lsa_flat_select(z(T, 64, dtype=bf), z(T, dtype=i64), z(P, 64, dtype=bf),
+                                                           z(P + 1, dtype=i32), z(N, dtype=i32), top_p=4, budget=8),
+        "ls_lsa_tree_select": lambda: L.ls_lsa_tree_select(z(T, 64, dtype=bf), z(T, dtype=i64), z(P, 64, dtype=bf),
+                                                           z(P // 4, 64, dtype=bf), z(P + 1, dtype=i32),
+                                                           z(N, dtype=i32), node_block=8, beam=2, top_p=4, budget=8),
+        "ls_lsa_tree_levels_select": lambda: L.ls_lsa_tree_levels_select(
+            z(T, 64, dtype=bf), z(T, dtype=i64), z(P, 64, dtype=bf), [z(P // 4, 64, dtype=bf)],
+            z(P + 1, dtype=i32), z(N, dtype=i32), node_block=8, beam=2, start_nodes=4, top_p=4, budget=8),
+        "ls_merge_select": lambda: L.ls_merge_select(z(2, T, 8), z(2, T, 8, dtype=i32), z(2, dtype=i32), k=8),
+        "ls_sparse_attention": lambda: L.ls_sparse_attention(z(2, 8, 576, dtype=bf), z(10, 576, dtype=bf),
+                                                             z(2, 4, dtype=i32)),
+        "ls_attention_merge": lambda: L.ls_attention_merge(z(2, 3, 512), z(2, 3)),
+    }
+
+
+@pytest.mark.parametrize("name", sorted(_host_calls()))
+def test_every_binding_refuses_host_tensors(name):
+    """Each Python entry point checks its tensors before any CUDA call: host
+    tensors give a ValueError naming CUDA, whatever the machine has."""
     with pytest.raises(ValueError, match="CUDA"):
-        L.ls_sparse_attention(q, lat, idx)
-    with pytest.raises(ValueError, match="CUDA"):
-        L.ls_attention_merge(torch.zeros((2, 3, 512)), torch.zeros((2, 3)))
-    with pytest.raises(ValueError, match="CUDA"):
-        L.ls_merge_select(torch.zeros((2, 3, 8)), torch.zeros((2, 3, 8), dtype=torch.int32),
-                          torch.zeros(2, dtype=torch.int32))
-    w = torch.zeros((2, 32), dtype=torch.float32)
-    keys = torch.zeros((2, 64, 128), dtype=torch.bfloat16)
-    with pytest.raises(ValueError, match="CUDA"):
-        L.ls_decode_select(torch.zeros((2, 32, 128), dtype=torch.bfloat16), w, keys)
+        _host_calls()[name]()
