@@ -256,6 +256,12 @@ def _host_calls():
         "ls_lsa_tree_levels_select": lambda: L.ls_lsa_tree_levels_select(
             z(T, 64, dtype=bf), z(T, dtype=i64), z(P, 64, dtype=bf), [z(P // 4, 64, dtype=bf)],
             z(P + 1, dtype=i32), z(N, dtype=i32), node_block=8, beam=2, start_nodes=4, top_p=4, budget=8),
+        "ls_prefill_select_stream": lambda: L.ls_prefill_select_stream(
+            z(T, H, d, dtype=bf), z(T, H), z(T, dtype=i64), z(N, d, dtype=bf), z(16, d, dtype=bf),
+            z(16, d, dtype=bf), k=8),
+        "ls_prefill_select_stream_fp8": lambda: L.ls_prefill_select_stream_fp8(
+            z(T, H, d, dtype=e4), z(T, H), z(T, H), z(T, dtype=i64), z(N, d, dtype=e4), z(N), z(16, d, dtype=e4),
+            z(16, d, dtype=e4), k=8),
         "ls_merge_select": lambda: L.ls_merge_select(z(2, T, 8), z(2, T, 8, dtype=i32), z(2, dtype=i32), k=8),
         "ls_sparse_attention": lambda: L.ls_sparse_attention(z(2, 8, 576, dtype=bf), z(10, 576, dtype=bf),
                                                              z(2, 4, dtype=i32)),
