@@ -6,6 +6,7 @@
 //   DIR expand T top_p P budget   picked.bin [T][top_p] i32, off.bin [P+1] i32,
 //                                 mem.bin [off[P]] i32 -> cand.bin [T][budget] i32
 //   DIR counts T stride n_total   pos.bin [T] i64 -> cnt.bin [T] i32
+//   DIR fold n blocks             w.bin, qs.bin [n] f32 -> out.bin [n] f32 (fold_scales_kernel)
 #include "misc_host.h"
 
 #include <cstdio>
@@ -66,7 +67,7 @@ static void launch(int blocks, F body) {
 }
 
 int main(int argc, char** argv) {
-  if (argc < 6) return 2;
+  if (argc < 5) return 2;
   const char* dir = argv[1];
   const std::string mode = argv[2];
   const int T = std::atoi(argv[3]);
@@ -82,7 +83,17 @@ int main(int argc, char** argv) {
     save(dir, "cand.bin", cand);
     return 0;
   }
-  if (mode == "counts") {
+  if (mode == "fold" && argc == 5) {
+    const int64_t n = std::atoll(argv[3]);
+    const int blocks = std::atoi(argv[4]);
+    auto w = load<float>(dir, "w.bin", static_cast<size_t>(n));
+    auto qs = load<float>(dir, "qs.bin", static_cast<size_t>(n));
+    std::vector<float> out(static_cast<size_t>(n), 777.f);
+    launch(blocks, [&] { lsi::fold_scales_kernel(w.data(), qs.data(), n, out.data()); });
+    save(dir, "out.bin", out);
+    return 0;
+  }
+  if (mode == "counts" && argc == 6) {
     const int stride = std::atoi(argv[4]), n_total = std::atoi(argv[5]);
     auto pos = load<int64_t>(dir, "pos.bin", static_cast<size_t>(T));
     std::vector<int32_t> cnt(static_cast<size_t>(T), 777);

@@ -9,6 +9,9 @@ position t the number of stride-compressed keys it may see.  The source is
 preprocessed (launchers removed; the shim supplies the warp shuffles) and
 built with g++ under AddressSanitizer.  Expected values: the oracle's
 `expand_buckets` (the -1 tail past its list) and `eligible_count`, exactly.
+`fold_scales_kernel` (the fp8 path's head weight times query-head scale, a
+grid-stride loop) is checked against numpy's fp32 product, bit for bit, with
+grids smaller and larger than the array.
 Picked lists end in a -1 tail where fewer buckets were found, as the top-k
 writes them.  Test infrastructure only.
 """
@@ -32,7 +35,7 @@ def _host_source() -> str:
     with open(SRC) as f:
         src = f.read()
     parts = []
-    for name in ("causal_counts_kernel", "expand_kernel"):
+    for name in ("causal_counts_kernel", "fold_scales_kernel", "expand_kernel"):
         m = re.search(r"__global__ void " + name + r"\(.*?\n\}\n", src, flags=re.S)
         assert m, name
         parts.append(m.group(0))
@@ -121,3 +124,16 @@ def test_causal_counts(misc_host, stride, n_total):
     run(["counts", pos.size, stride, n_total])
     cnt = np.fromfile(d / "cnt.bin", dtype=np.int32)
     assert np.array_equal(cnt, eligible_count(pos, stride, n_total).astype(np.int32))
+
+
+@pytest.mark.parametrize("n,blocks", [(1, 1), (1000, 2), (70000, 3), (300, 8)])
+def test_fold_scales(misc_host, n, blocks):
+    d, run = misc_host
+    rng = np.random.default_rng(n)
+    w = rng.standard_normal(n).astype(np.float32)
+    qs = np.abs(rng.standard_normal(n)).astype(np.float32) * np.float32(0.01)
+    w.tofile(d / "w.bin")
+    qs.tofile(d / "qs.bin")
+    run(["fold", n, blocks])
+    out = np.fromfile(d / "out.bin", dtype=np.float32)
+    assert np.array_equal(out.view(np.uint32), (w * qs).view(np.uint32))
