@@ -135,7 +135,10 @@ ls_status ls_topk_select(const float* scores, int64_t ld, const int32_t* n_valid
 /*
  * ls_decode_select -- decode selection: one query per sequence over bf16 keys,
  * full scan then exact top-k (ls_indexer_score + ls_topk_select fused in one
- * call).  Shapes as ls_indexer_score with T = 1; outputs [B][k].
+ * call).  Shapes as ls_indexer_score with T = 1; outputs [B][k].  ("03 long
+ * context", "The Architectural Answer: Read Less of the Past": the new token's
+ * query scores every cached position with the weighted-ReLU indexer, and the k
+ * best positions go on to the sparse attention.)
  * Workspace: ls_decode_select_workspace_size(B, N) bytes.
  */
 size_t ls_decode_select_workspace_size(int B, int N);
@@ -240,7 +243,9 @@ ls_status ls_indexer_score_fp8(const uint8_t* q8, const float* q_scale, const fl
 
 /*
  * ls_prefill_select_stream_fp8 -- ls_prefill_select_stream with fp8 queries
- * and an fp8 history (the scores of ls_indexer_score_fp8):
+ * and an fp8 history (the scores of ls_indexer_score_fp8; "03 long context",
+ * "Sparsity Is a Systems Feature: The Blast Radius": the indexer key stored
+ * as 128 fp8 bytes plus a 4-byte scale):
  *
  *   q8 [T][H][d] e4m3, q_scale [T][H] fp32, w [T][H] fp32, q_pos [T] int64
  *   hist_k8 [N][d] e4m3 codes and hist_kscale [N] fp32, both in PINNED host
@@ -391,7 +396,10 @@ ls_status ls_lsa_tree_levels_select(const uint16_t* q_idx, const int64_t* q_pos,
  * S contiguous shards (one per GPU, say): each shard's exact top-k lists of
  * the same T queries are merged into the top-k of the whole history (the
  * top-k of the union of the shards' top-k lists is the global top-k, since
- * every shard contributes its own best).
+ * every shard contributes its own best).  ("03 long context", "Teamwork
+ * First: Ring Attention for the Giant Prefill": the sequence is sharded over
+ * GPUs and partial results are combined; this is that combine for the
+ * selection.)
  *
  *   vals [S][T][k_in] fp32, idx [S][T][k_in] int32: list s of query t, in
  *        canonical order, positions local to shard s, padded with -1 / -inf
@@ -511,7 +519,8 @@ ls_status ls_decode_two_stage_pq_select(const uint16_t* q, const float* w, const
  * ls_indexer_score_pq -- coarse scores of PQ compact keys (one query per
  * sequence): scores[b][n] = sum_h w[b,h] * max(0, q[b,h] . key(b,n)), key
  * decoded from pq_codes[b][n] with pq_books as in
- * ls_decode_two_stage_pq_select; -inf for n >= n_valid[b].
+ * ls_decode_two_stage_pq_select; -inf for n >= n_valid[b].  (LeanSparse
+ * podcast transcript, 07:12-07:34: the coarse pass over 32-byte compact keys.)
  *   q [B][H][d] bf16, w [B][H] fp32, pq_codes [B][N][32], pq_books [32][256][4]
  *   fp16, scores [B][N] fp32; all device pointers, 16-byte aligned.
  */
