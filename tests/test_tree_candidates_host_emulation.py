@@ -155,6 +155,8 @@ def test_level_visibility(cand_host, shape):
 
 def _edge_positions(block_keys, n_keys, node_span, seed):
     edges = np.arange(0, n_keys + 3 * block_keys, block_keys, dtype=np.int64)
+    if edges.size > 1500:                              # long histories: every few edges, the first and the last
+        edges = np.unique(np.concatenate([edges[:64], edges[::edges.size // 1000], edges[-64:]]))
     rng = np.random.default_rng(seed)
     pos = np.concatenate([edges - 1, edges, edges + 1, rng.integers(0, n_keys + 2 * block_keys, 700),
                           np.asarray([-5, -block_keys - 1, -3 * block_keys, 0, 1, node_span - 1, node_span])]).astype(np.int64)   # negative positions are clamped to 0
