@@ -13,7 +13,6 @@ tests do).  Test infrastructure only: the product has no host path.
 
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
@@ -42,22 +41,11 @@ def _host_source(src: str) -> str:
 
 
 @pytest.fixture(scope="module")
-def runner(tmp_path_factory):
-    cxx = shutil.which("g++")
-    if cxx is None:
-        pytest.skip("no host C++ compiler")
+def runner(tmp_path_factory, host_build):
     d = tmp_path_factory.mktemp("attn_host")
     with open(SRC) as f:
         (d / "kernel_host.h").write_text(_host_source(f.read()))
-    exe = d / "attn_host"
-    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
-            os.path.join(HERE, "host_emulation", "attn_main.cpp")]
-    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address", "-fno-omit-frame-pointer"] + base[1:],
-                       capture_output=True, text=True)
-    if r.returncode != 0:                       # no sanitizer runtime: plain build
-        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+    exe, env = host_build(d, "attn_host", "attn_main.cpp", ubsan=False)
 
     def attn(q, lat, idx, scale, off=None, foreign=False):
         T, H, _ = q.shape

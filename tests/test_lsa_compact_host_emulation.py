@@ -21,7 +21,6 @@ infrastructure only.
 
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
@@ -83,21 +82,10 @@ def _segments(T, P, cap2, slack, grid_cap=148):
 
 
 @pytest.fixture(scope="module")
-def compact_host(tmp_path_factory):
-    cxx = shutil.which("g++")
-    if cxx is None:
-        pytest.skip("no host C++ compiler")
+def compact_host(tmp_path_factory, host_build):
     d = tmp_path_factory.mktemp("lsa_compact_host")
     (d / "lsa_compact_host.h").write_text(_host_source())
-    exe = d / "lsa_compact_host"
-    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
-            os.path.join(HERE, "host_emulation", "lsa_compact_main.cpp")]
-    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
-                                   "-fno-omit-frame-pointer"] + base[1:], capture_output=True, text=True)
-    if r.returncode != 0:
-        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+    exe, env = host_build(d, "lsa_compact_host", "lsa_compact_main.cpp")
     return d, exe, env
 
 

@@ -16,7 +16,6 @@ exactly.  Test infrastructure only.
 
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
@@ -43,21 +42,11 @@ def _host_source() -> str:
 
 
 @pytest.fixture(scope="module")
-def expand_host(tmp_path_factory):
-    cxx = shutil.which("g++")
-    if cxx is None:
-        pytest.skip("no host C++ compiler")
+def expand_host(tmp_path_factory, host_build):
     d = tmp_path_factory.mktemp("lsa_expand_host")
     (d / "lsa_expand_host.h").write_text(_host_source())
-    exe = d / "lsa_expand_host"
-    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
-            os.path.join(HERE, "host_emulation", "lsa_expand_main.cpp")]
-    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
-                                   "-fno-omit-frame-pointer"] + base[1:], capture_output=True, text=True)
-    if r.returncode != 0:
-        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    return d, exe, dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+    exe, env = host_build(d, "lsa_expand_host", "lsa_expand_main.cpp")
+    return d, exe, env
 
 
 @pytest.mark.parametrize("top_p,budget", [(64, 512), (1500, 4096), (300, 37)])

@@ -10,7 +10,6 @@ added, and the row counts.  Test infrastructure only.
 
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
@@ -29,22 +28,11 @@ def _host_source(src: str) -> str:
 
 
 @pytest.fixture(scope="module")
-def pack(tmp_path_factory):
-    cxx = shutil.which("g++")
-    if cxx is None:
-        pytest.skip("no host C++ compiler")
+def pack(tmp_path_factory, host_build):
     d = tmp_path_factory.mktemp("merge_host")
     with open(SRC) as f:
         (d / "merge_host.h").write_text(_host_source(f.read()))
-    exe = d / "merge_host"
-    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
-            os.path.join(HERE, "host_emulation", "merge_main.cpp")]
-    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address", "-fno-omit-frame-pointer"] + base[1:],
-                       capture_output=True, text=True)
-    if r.returncode != 0:
-        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+    exe, env = host_build(d, "merge_host", "merge_main.cpp", ubsan=False)
 
     def run(vals, idx, offs):
         S, T, k_in = vals.shape

@@ -18,7 +18,6 @@ writes them.  Test infrastructure only.
 
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
@@ -43,21 +42,10 @@ def _host_source() -> str:
 
 
 @pytest.fixture(scope="module")
-def misc_host(tmp_path_factory):
-    cxx = shutil.which("g++")
-    if cxx is None:
-        pytest.skip("no host C++ compiler")
+def misc_host(tmp_path_factory, host_build):
     d = tmp_path_factory.mktemp("misc_host")
     (d / "misc_host.h").write_text(_host_source())
-    exe = d / "misc_host"
-    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
-            os.path.join(HERE, "host_emulation", "misc_main.cpp")]
-    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
-                                   "-fno-omit-frame-pointer"] + base[1:], capture_output=True, text=True)
-    if r.returncode != 0:
-        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+    exe, env = host_build(d, "misc_host", "misc_main.cpp")
 
     def run(args):
         r = subprocess.run([str(exe), str(d)] + [str(a) for a in args], capture_output=True, text=True, env=env,

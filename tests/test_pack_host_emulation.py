@@ -14,7 +14,6 @@ infrastructure only.
 
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
@@ -32,22 +31,11 @@ def _host_source(src: str) -> str:
 
 
 @pytest.fixture(scope="module")
-def pack(tmp_path_factory):
-    cxx = shutil.which("g++")
-    if cxx is None:
-        pytest.skip("no host C++ compiler")
+def pack(tmp_path_factory, host_build):
     d = tmp_path_factory.mktemp("pack_host")
     with open(SRC) as f:
         (d / "pack_host.h").write_text(_host_source(f.read()))
-    exe = d / "pack_host"
-    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
-            os.path.join(HERE, "host_emulation", "pack_main.cpp")]
-    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
-                                   "-fno-omit-frame-pointer"] + base[1:], capture_output=True, text=True)
-    if r.returncode != 0:
-        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+    exe, env = host_build(d, "pack_host", "pack_main.cpp")
 
     def run(val, lab, cnt, over, k, cap):
         T, ld = val.shape

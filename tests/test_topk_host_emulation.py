@@ -20,7 +20,6 @@ for bit.  Test infrastructure only: the product has no host path.
 
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
@@ -62,21 +61,10 @@ def _host_source() -> str:
 
 
 @pytest.fixture(scope="module")
-def topk_host(tmp_path_factory):
-    cxx = shutil.which("g++")
-    if cxx is None:
-        pytest.skip("no host C++ compiler")
+def topk_host(tmp_path_factory, host_build):
     d = tmp_path_factory.mktemp("topk_host")
     (d / "topk_host.h").write_text(_host_source())
-    exe = d / "topk_host"
-    base = [cxx, "-std=c++20", "-pthread", "-I", str(d), "-I", os.path.join(HERE, "host_emulation"), "-o", str(exe),
-            os.path.join(HERE, "host_emulation", "topk_main.cpp")]
-    r = subprocess.run(base[:1] + ["-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
-                                   "-fno-omit-frame-pointer"] + base[1:], capture_output=True, text=True)
-    if r.returncode != 0:                       # no sanitizer runtime: plain build
-        r = subprocess.run(base[:1] + ["-O2"] + base[1:], capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-3000:]
-    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0:abort_on_error=1")
+    exe, env = host_build(d, "topk_host", "topk_main.cpp")
 
     def run(form, scores, labels, n_valid, k, flags=None, grid=0, out_row=None):
         R, ld = scores.shape
